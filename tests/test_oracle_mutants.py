@@ -1,0 +1,69 @@
+"""Plants plausible mistakes in copies of the C oracle and checks that the
+pins catch every one (no GPU; nothing here touches the product path).
+
+Each mutant is the oracle source with one small edit: a wrong index, a
+dropped term, a flipped sign, a transposed layout, a wrong head mapping.  The
+pins of test_oracle_pins must fail on each, or the pins are too weak.
+"""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from oracle import build as obuild
+from tests import test_oracle_pins as pins
+
+MUTANTS = {
+    "offset-index": ("int off = t % bs;", "int off = (t / bs) % bs;"),
+    "dropped-scale": ("s[t] = scale * dot;", "s[t] = dot;"),
+    "flipped-exponent": ("double p = exp(s[t] - m);", "double p = exp(m - s[t]);"),
+    "head-mapping": ("int g = h / G;\n  int n = lens[b];", "int g = h % Hkv;\n  int n = lens[b];"),
+    "dropped-normalisation": ("for (int d = 0; d < D; ++d) out_row[d] /= denom;", ""),
+    "transposed-layout": ("return ((blk * Hkv + g) * bs + off) * (int64_t)D;",
+                          "return ((blk * bs + off) * Hkv + g) * (int64_t)D;"),
+    "merge-missing-rescale": ("L += l[i * max_parts + p] * w;", "L += l[i * max_parts + p];"),
+    "partial-max-skipped": ("if (s[t - t0] > m) m = s[t - t0];", "m = 0.0;"),
+    "bf16-wrong-half": ("uint32_t u = ((uint32_t)((const uint16_t *)base)[i]) << 16;",
+                        "uint32_t u = ((uint32_t)((const uint16_t *)base)[i]);"),
+}
+
+PIN_TESTS = [
+    pins.test_block_table_example_matches_dense,
+    lambda: [pins.test_paged_equals_dense_gqa(s) for s in (0, 1)],
+    pins.test_bruteforce_with_allocator_slots,
+    pins.test_zero_scale_gives_mean_of_values,
+    pins.test_dominant_key_selects_its_value,
+    lambda: [pins.test_partitioned_merge_equals_single_pass(p) for p in (4, 16)],
+    pins.test_bf16_inputs_match_widened_f64,
+]
+
+
+def _build_mutant(tmp_path, name, old, new):
+    src = open(obuild.SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not unique"
+    path = tmp_path / f"m_{name}.c"
+    path.write_text(src.replace(old, new))
+    so = tmp_path / f"m_{name}.so"
+    subprocess.run(["gcc", "-O1", "-fPIC", "-shared", "-std=c11", str(path), "-o", str(so), "-lm"], check=True)
+    return str(so)
+
+
+def test_original_passes_all_pins():
+    for t in PIN_TESTS:
+        t()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(tmp_path, name, monkeypatch):
+    old, new = MUTANTS[name]
+    so = _build_mutant(tmp_path, name, old, new)
+    monkeypatch.setattr(oracle, "_lib", oracle.load(so))
+    caught = 0
+    for t in PIN_TESTS:
+        try:
+            t()
+        except (AssertionError, ValueError):
+            caught += 1
+    assert caught > 0, f"no pin fails on mutant {name}"
