@@ -1,0 +1,241 @@
+/*
+ * pagedattn.h -- C ABI of the paged KV-cache decode path (sm_100a).
+ *
+ * The method ("PagedAttention Internals", wondering.app, sections "Fixed-Size
+ * KV Blocks" and "The Block Table Map"; "pagedattention" glossary entry,
+ * chipfoundryservices.com, paragraph "Paging maps logical tokens to physical
+ * blocks through a block table"): every sequence's key/value cache is stored
+ * in fixed-size physical blocks that may sit anywhere in a shared pool, and a
+ * per-sequence block table maps logical block n to its physical block.
+ * Attention follows the table; new tokens fill the sequence's current block
+ * and a new block is taken only when it is full; sequences that share a
+ * prefix (or the samples of a beam search) point at the same physical blocks,
+ * which are copied only when a sharer writes into them (glossary entry,
+ * comparison table and paragraph "It is the core of vLLM ...").
+ *
+ * Conventions for every entry point:
+ *  - Pointers named "device" are CUDA device pointers owned by the caller;
+ *    pointers named "host" are host memory owned by the caller.  The library
+ *    never allocates, frees or keeps device memory of the caller's.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Kernel launches are asynchronous on it; no call synchronises
+ *    except pa_read_device_error.
+ *  - Every call returns a pa_status.  Argument errors are found on the host
+ *    before any launch and leave every buffer untouched.
+ *  - Data errors that only the device can see (a slot or a table entry
+ *    outside the pool) never trap: the offending element is skipped and a
+ *    bit is set in a per-device error word read by pa_read_device_error.
+ *
+ * Cache layout (both pools):
+ *   k_cache, v_cache : [num_blocks][num_kv_heads][block_size][head_dim]
+ *   element (blk, h, off, d) at ((blk*num_kv_heads + h)*block_size + off)*head_dim + d,
+ *   so one (block, kv head) tile of block_size x head_dim is contiguous.
+ * A token at logical position t of a sequence with block table T lives at
+ *   slot = T[t / block_size] * block_size + t % block_size.
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,   /* a null pointer, a bad size or shape */
+  PA_ERR_UNSUPPORTED = 2,   /* dtype / head_dim / block_size / group size not built */
+  PA_ERR_OUT_OF_BLOCKS = 3, /* allocator: not enough free blocks; state unchanged */
+  PA_ERR_CUDA = 4,          /* a CUDA runtime call failed */
+  PA_ERR_NOT_FOUND = 5,     /* allocator: no such live sequence */
+  PA_ERR_TOO_SMALL = 6      /* a caller buffer (workspace, table row, output) is too small */
+} pa_status;
+
+typedef enum { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
+
+/* Bits of the device error word (pa_read_device_error). */
+#define PA_DEVERR_SLOT 0x1       /* pa_append_kv: slot >= num_blocks*block_size (row skipped) */
+#define PA_DEVERR_TABLE 0x2      /* pa_decode: a used table entry outside [0, num_blocks) (block skipped) */
+#define PA_DEVERR_PAIR 0x4       /* pa_copy_blocks: a pair entry outside [0, num_blocks) (pair skipped) */
+#define PA_DEVERR_TIMEOUT 0x8    /* a kernel gave up waiting on its own copy (work unit dropped) */
+#define PA_DEVERR_LEN 0x10       /* pa_decode: a context length < 0 or > max_context_len (row zeroed) */
+
+/* Tokens per split-context partition of pa_decode. */
+#define PA_PARTITION_TOKENS 512
+
+/* The paged pool.  k and v are device pointers of the layout above. */
+typedef struct {
+  void *k;
+  void *v;
+  int32_t dtype;        /* pa_dtype of every element of k, v, q, out and the new rows */
+  int32_t num_blocks;
+  int32_t block_size;   /* tokens per block: 8, 16 or 32 */
+  int32_t num_kv_heads;
+  int32_t head_dim;     /* 64 or 128 */
+} pa_cache_t;
+
+/* ---------------------------------------------------------------- kernels */
+
+/*
+ * KV append ("Fixed-Size KV Blocks": tokens fill the current block; the
+ * glossary's "Paging maps logical tokens ..." paragraph: the table maps
+ * logical positions to physical blocks).
+ *   k, v          device [num_tokens][num_kv_heads][head_dim], cache dtype
+ *   slot_mapping  device [num_tokens] int64: token i is written to
+ *                 k_cache/v_cache[slot/bs][h][slot%bs][:] for every head h.
+ *                 A negative slot is padding and is skipped; a slot past the
+ *                 pool sets PA_DEVERR_SLOT and is skipped.
+ * Two tokens with the same slot: which one lands is undefined.
+ */
+PA_API pa_status pa_append_kv(const void *k, const void *v, const int64_t *slot_mapping,
+                              int32_t num_tokens, const pa_cache_t *cache, void *stream);
+
+/*
+ * Paged decode attention ("The Block Table Map": attention follows the table;
+ * the glossary's "the attention kernel follows the table to gather the right
+ * keys and values").  The pages give no formula; this is the textbook
+ * scaled dot-product step.  For sequence b, query head h and its KV head
+ * g = h / (num_q_heads / num_kv_heads):
+ *   s_t = scale * <q[b,h,:], K(b,t,g)>  for t < context_lens[b]
+ *   out[b,h,:] = sum_t exp(s_t - max s) V(b,t,g) / sum_t exp(s_t - max s)
+ * with K(b,t,g) = k_cache[block_tables[b*max_blocks_per_seq + t/bs]][g][t%bs].
+ * Contexts are cut into PA_PARTITION_TOKENS-token partitions; each partition
+ * keeps (max, sum, unnormalised accumulator) in the workspace and a second
+ * kernel merges them with a log-sum-exp combine.  Arithmetic is fp32 with an
+ * online softmax; out is rounded once to the cache dtype.
+ *   q             device [num_seqs][num_q_heads][head_dim], cache dtype
+ *   block_tables  device [num_seqs][max_blocks_per_seq] int32; entries past
+ *                 ceil(len/bs) are never read
+ *   context_lens  device [num_seqs] int32 (the appended token included);
+ *                 0 gives a zero output row
+ *   max_context_len  host: an upper bound of every context_lens[b]; a larger
+ *                 length sets PA_DEVERR_LEN and zeroes that row
+ *   out           device [num_seqs][num_q_heads][head_dim], cache dtype
+ *   workspace     device scratch of at least pa_decode_workspace_size(...)
+ *                 bytes, 16-byte aligned (NULL allowed when that size is 0)
+ * num_q_heads / num_kv_heads (the group size) must be 1, 2, 4 or 8.
+ */
+PA_API pa_status pa_decode(const void *q, const pa_cache_t *cache, const int32_t *block_tables,
+                           int32_t max_blocks_per_seq, const int32_t *context_lens,
+                           int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len,
+                           float scale, void *out, void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+/* Bytes of workspace pa_decode needs for these sizes (0 when no context is
+ * longer than one partition). */
+PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                       int32_t max_context_len, int32_t head_dim);
+
+/*
+ * Copy-on-write block copy (glossary entry, comparison table "share blocks
+ * copy-on-write" and paragraph "It is the core of vLLM ...": sharers fork
+ * only when they diverge).  For every pair i, physical block
+ * src_dst_pairs[2i+1] of both pools becomes a bit copy of block
+ * src_dst_pairs[2i] (all kv heads, all slots).
+ *   src_dst_pairs device [num_pairs][2] int32
+ * Destinations must be distinct and no destination may also be a source
+ * (pa_check_copy_pairs tests this on a host copy); otherwise the result is
+ * undefined.  An entry outside the pool sets PA_DEVERR_PAIR; that pair is
+ * skipped.
+ */
+PA_API pa_status pa_copy_blocks(const int32_t *src_dst_pairs, int32_t num_pairs,
+                                const pa_cache_t *cache, void *stream);
+
+/* Host-side check of copy pairs (host memory): PA_OK, or PA_ERR_INVALID_ARG
+ * for an entry outside [0, num_blocks), a repeated destination, or a
+ * destination that is also a source. */
+PA_API pa_status pa_check_copy_pairs(const int32_t *src_dst_pairs_host, int32_t num_pairs,
+                                     int32_t num_blocks);
+
+/* Synchronises `stream`, then returns the current device's error word in
+ * *bits (PA_DEVERR_*) and clears it. */
+PA_API pa_status pa_read_device_error(void *stream, int32_t *bits);
+
+/* Static text for a status code. */
+PA_API const char *pa_status_string(pa_status s);
+
+/* Library version, "major.minor.patch". */
+PA_API const char *pa_version(void);
+
+/* ------------------------------------------------------ block allocator */
+/*
+ * Host-side reference-counted block allocator ("Fixed-Size KV Blocks",
+ * "Sharing And Dynamic Growth"; glossary "Paging maps ..." and "It is the
+ * core of vLLM ...").  Blocks are handed out one at a time as sequences
+ * grow; forks share every block (reference count + 1); a write into a shared,
+ * partially filled last block first moves the writer to a fresh block and
+ * reports a (src, dst) copy pair for pa_copy_blocks; freed blocks return to
+ * the pool.  The free list deals never-used blocks in a caller-given order
+ * and hands released blocks out again last-in first-out.  Sequence ids are
+ * never reused.  Not thread-safe: one allocator per host thread.
+ */
+typedef struct pa_allocator pa_allocator;
+
+/* free_order_host: a permutation of [0, num_blocks) (the order fresh blocks
+ * are dealt), or NULL for 0, 1, 2, ... */
+PA_API pa_status pa_alloc_create(int32_t num_blocks, int32_t block_size,
+                                 const int32_t *free_order_host, pa_allocator **out);
+PA_API void pa_alloc_destroy(pa_allocator *a);
+
+/* A new, empty sequence; its id in *seq. */
+PA_API pa_status pa_seq_new(pa_allocator *a, int32_t *seq);
+
+/* A new sequence sharing every block of `parent` (reference counts + 1). */
+PA_API pa_status pa_seq_fork(pa_allocator *a, int32_t parent, int32_t *child);
+
+/* Releases a sequence: reference counts - 1, blocks reaching 0 are freed. */
+PA_API pa_status pa_seq_free(pa_allocator *a, int32_t seq);
+
+/*
+ * Appends n tokens to one sequence.  out_slots_host[n] receives each token's
+ * slot.  A copy-on-write move, if any, is written to out_cow_pair_host[2]
+ * (src, dst) and *n_cow is 1, else 0.  PA_ERR_OUT_OF_BLOCKS leaves every
+ * state unchanged.
+ */
+PA_API pa_status pa_seq_append(pa_allocator *a, int32_t seq, int32_t n, int64_t *out_slots_host,
+                               int32_t *out_cow_pair_host, int32_t *n_cow);
+
+/*
+ * Appends n_tokens[i] tokens to seqs[i] for every i, in order, all or nothing
+ * (a sequence may appear once).  Slots go to out_slots_host, sequence by
+ * sequence (sum of n_tokens entries); copy pairs to out_cow_pairs_host
+ * (room for n_seqs pairs), *n_cow of them, in the order they were made.
+ */
+PA_API pa_status pa_batch_append(pa_allocator *a, const int32_t *seqs, const int32_t *n_tokens,
+                                 int32_t n_seqs, int64_t *out_slots_host,
+                                 int32_t *out_cow_pairs_host, int32_t *n_cow);
+
+/* Length in tokens and number of blocks of a live sequence. */
+PA_API pa_status pa_seq_len(pa_allocator *a, int32_t seq, int32_t *len, int32_t *num_blocks);
+
+/* Copies a sequence's table into out_host (room for cap entries). */
+PA_API pa_status pa_seq_block_table(pa_allocator *a, int32_t seq, int32_t *out_host, int32_t cap,
+                                    int32_t *count);
+
+/* Writes the tables of n_seqs sequences as rows of a [n_seqs][max_blocks]
+ * int32 host array padded with `pad`, and their lengths to lens_host. */
+PA_API pa_status pa_build_block_tables(pa_allocator *a, const int32_t *seqs, int32_t n_seqs,
+                                       int32_t max_blocks, int32_t pad, int32_t *tables_host,
+                                       int32_t *lens_host);
+
+/* Usage: slots holding a token (each physical slot once), slots allocated
+ * (blocks in use x block_size), free and used block counts.  Fragmentation
+ * = (allocated - used) / allocated. */
+PA_API pa_status pa_alloc_stats(pa_allocator *a, int64_t *used_slots, int64_t *allocated_slots,
+                                int32_t *free_blocks, int32_t *used_blocks);
+
+/* Reference count of a physical block. */
+PA_API pa_status pa_block_refcount(pa_allocator *a, int32_t block, int32_t *refcount);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PAGEDATTN_H */

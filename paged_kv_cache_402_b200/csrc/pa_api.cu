@@ -1,0 +1,242 @@
+// C ABI of the paged KV-cache path: argument checks, launch configuration and
+// the device error word.  Every kernel of the library is compiled in this one
+// translation unit (the error word is one __device__ symbol).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+#include "pa_copy_kernels.cuh"
+#include "pa_decode_simt.cuh"
+#include "pagedattn.h"
+
+namespace {
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int elem_bytes(int32_t dtype) { return dtype == PA_DTYPE_F32 ? 4 : 2; }
+
+pa_status check_cache(const pa_cache_t *c) {
+  if (!c || !c->k || !c->v) return PA_ERR_INVALID_ARG;
+  if (c->dtype != PA_DTYPE_F32 && c->dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
+  if (c->num_blocks <= 0 || c->num_kv_heads <= 0) return PA_ERR_INVALID_ARG;
+  if (c->block_size != 8 && c->block_size != 16 && c->block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 && c->head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (!aligned16(c->k) || !aligned16(c->v)) return PA_ERR_INVALID_ARG;
+  return PA_OK;
+}
+
+inline pa_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+inline int32_t max_parts_for(int32_t max_context_len) {
+  return (max_context_len + pa::kPart - 1) / pa::kPart;
+}
+
+inline size_t round16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+// workspace layout: m [B*Hq*P] f32 | l [B*Hq*P] f32 | acc [B*Hq*P*D] f32
+size_t workspace_bytes_for(int64_t B, int64_t Hq, int32_t max_ctx, int64_t D) {
+  if (max_ctx <= pa::kPart) return 0;
+  const int64_t rows = B * Hq * (int64_t)max_parts_for(max_ctx);
+  return round16(rows * 4) * 2 + round16(rows * D * 4);
+}
+
+// Shared-memory ring of the partition kernel: per warp `nstages` slots of a
+// K tile and a V tile, then the mbarriers.  Aimed at two CTAs per SM (about
+// 24 KiB per warp), at least one slot, never past 192 KiB per CTA.
+int choose_stages(int tile_bytes) {
+  const int per_warp_budget = 24 * 1024;
+  int n = per_warp_budget / (2 * tile_bytes);
+  if (n < 2) n = 2;
+  if (n > 8) n = 8;
+  while (n > 1 && (size_t)pa::kWarps * n * 2 * tile_bytes > 192 * 1024) --n;
+  return n;
+}
+
+template <typename T, int D, int G>
+pa_status launch_decode_t(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
+  const int tile_bytes = p.bs * D * (int)sizeof(T);
+  const int nstages = choose_stages(tile_bytes);
+  size_t smem = (size_t)pa::kWarps * nstages * 2 * tile_bytes + (size_t)pa::kWarps * nstages * 8;
+  const size_t merge = (size_t)pa::kWarps * G * (D + 2) * sizeof(float);
+  if (smem < merge) smem = merge;
+  auto kern = pa::decode_partition_simt<T, D, G>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return PA_ERR_CUDA;
+  dim3 grid(max_parts, p.Hkv, p.B);
+  kern<<<grid, pa::kWarps * 32, smem, st>>>(p, nstages);
+  pa_status s = launch_status();
+  if (s != PA_OK || max_parts <= 1) return s;
+  pa::decode_reduce<T, D><<<p.B * p.Hq, 128, (size_t)max_parts * sizeof(float), st>>>(p);
+  return launch_status();
+}
+
+template <typename T, int D>
+pa_status launch_decode_d(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
+  switch (p.G) {
+    case 1: return launch_decode_t<T, D, 1>(p, max_parts, st);
+    case 2: return launch_decode_t<T, D, 2>(p, max_parts, st);
+    case 4: return launch_decode_t<T, D, 4>(p, max_parts, st);
+    case 8: return launch_decode_t<T, D, 8>(p, max_parts, st);
+    default: return PA_ERR_UNSUPPORTED;
+  }
+}
+
+template <typename T>
+pa_status launch_decode_dtype(const pa::DecodeParams &p, int D, int32_t max_parts,
+                              cudaStream_t st) {
+  if (D == 64) return launch_decode_d<T, 64>(p, max_parts, st);
+  if (D == 128) return launch_decode_d<T, 128>(p, max_parts, st);
+  return PA_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+extern "C" {
+
+PA_API const char *pa_version(void) { return "0.1.0"; }
+
+PA_API const char *pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported dtype, head_dim, block_size or group size";
+    case PA_ERR_OUT_OF_BLOCKS: return "out of free blocks";
+    case PA_ERR_CUDA: return "CUDA runtime error";
+    case PA_ERR_NOT_FOUND: return "no such sequence";
+    case PA_ERR_TOO_SMALL: return "buffer too small";
+  }
+  return "unknown status";
+}
+
+PA_API pa_status pa_append_kv(const void *k, const void *v, const int64_t *slot_mapping,
+                              int32_t num_tokens, const pa_cache_t *cache, void *stream) {
+  pa_status s = check_cache(cache);
+  if (s != PA_OK) return s;
+  if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !slot_mapping || !aligned16(k) || !aligned16(v)) return PA_ERR_INVALID_ARG;
+  const int row_bytes = cache->head_dim * elem_bytes(cache->dtype);
+  const int row_vecs = row_bytes / 16;
+  const int64_t warps = (int64_t)num_tokens * cache->num_kv_heads;
+  const int64_t blocks = (warps * 32 + 255) / 256;
+  if (blocks > INT32_MAX) return PA_ERR_INVALID_ARG;
+  pa::append_kv_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(
+      (const uint4 *)k, (const uint4 *)v, slot_mapping, num_tokens, cache->num_kv_heads,
+      cache->block_size, row_vecs, (int64_t)cache->num_blocks * cache->block_size, (uint4 *)cache->k,
+      (uint4 *)cache->v);
+  return launch_status();
+}
+
+PA_API pa_status pa_copy_blocks(const int32_t *src_dst_pairs, int32_t num_pairs,
+                                const pa_cache_t *cache, void *stream) {
+  pa_status s = check_cache(cache);
+  if (s != PA_OK) return s;
+  if (num_pairs < 0 || num_pairs > 65535) return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (!src_dst_pairs) return PA_ERR_INVALID_ARG;
+  const int64_t block_bytes = (int64_t)cache->block_size * cache->num_kv_heads * cache->head_dim *
+                              elem_bytes(cache->dtype);
+  const int64_t block_vecs = block_bytes / 16;
+  const int64_t per_cta = 256 * pa::kCopyUnroll;
+  dim3 grid((unsigned)((block_vecs + per_cta - 1) / per_cta), (unsigned)num_pairs);
+  pa::copy_blocks_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(
+      src_dst_pairs, cache->num_blocks, block_vecs, (uint4 *)cache->k, (uint4 *)cache->v);
+  return launch_status();
+}
+
+PA_API pa_status pa_check_copy_pairs(const int32_t *pairs, int32_t num_pairs, int32_t num_blocks) {
+  if (num_pairs < 0 || num_blocks <= 0 || (num_pairs > 0 && !pairs)) return PA_ERR_INVALID_ARG;
+  std::vector<uint8_t> role(num_blocks, 0);  // bit 0: a source, bit 1: a destination
+  for (int32_t i = 0; i < num_pairs; ++i) {
+    const int32_t src = pairs[2 * i], dst = pairs[2 * i + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) return PA_ERR_INVALID_ARG;
+    if (role[dst] & 2) return PA_ERR_INVALID_ARG;  // repeated destination
+    role[src] |= 1;
+    role[dst] |= 2;
+  }
+  for (int32_t b = 0; b < num_blocks; ++b)
+    if (role[b] == 3) return PA_ERR_INVALID_ARG;  // a destination that is also a source
+  return PA_OK;
+}
+
+PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                       int32_t max_context_len, int32_t head_dim) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || max_context_len <= 0 || head_dim <= 0) return 0;
+  return workspace_bytes_for(num_seqs, num_q_heads, max_context_len, head_dim);
+}
+
+PA_API pa_status pa_decode(const void *q, const pa_cache_t *cache, const int32_t *block_tables,
+                           int32_t max_blocks_per_seq, const int32_t *context_lens,
+                           int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len,
+                           float scale, void *out, void *workspace, size_t workspace_bytes,
+                           void *stream) {
+  pa_status s = check_cache(cache);
+  if (s != PA_OK) return s;
+  if (num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0 || max_blocks_per_seq < 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  if (!q || !out || !block_tables || !context_lens || !aligned16(q) || !aligned16(out))
+    return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (num_q_heads % cache->num_kv_heads) return PA_ERR_INVALID_ARG;
+  const int32_t G = num_q_heads / cache->num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > 65535 || cache->num_kv_heads > 65535) return PA_ERR_INVALID_ARG;
+  const int32_t bs = cache->block_size;
+  if ((int64_t)max_context_len > (int64_t)max_blocks_per_seq * bs) return PA_ERR_INVALID_ARG;
+  if (max_context_len > INT32_MAX - pa::kPart) return PA_ERR_INVALID_ARG;
+  const size_t need = workspace_bytes_for(num_seqs, num_q_heads, max_context_len, cache->head_dim);
+  if (need > 0) {
+    if (!workspace || !aligned16(workspace)) return PA_ERR_INVALID_ARG;
+    if (workspace_bytes < need) return PA_ERR_TOO_SMALL;
+  }
+  const int32_t max_parts = max_context_len > 0 ? max_parts_for(max_context_len) : 1;
+
+  pa::DecodeParams p{};
+  p.q = q;
+  p.k = cache->k;
+  p.v = cache->v;
+  p.out = out;
+  p.tables = block_tables;
+  p.lens = context_lens;
+  if (need > 0) {
+    const int64_t rows = (int64_t)num_seqs * num_q_heads * max_parts;
+    char *w = static_cast<char *>(workspace);
+    p.ws_m = reinterpret_cast<float *>(w);
+    p.ws_l = reinterpret_cast<float *>(w + round16(rows * 4));
+    p.ws_acc = reinterpret_cast<float *>(w + 2 * round16(rows * 4));
+  }
+  p.num_blocks = cache->num_blocks;
+  p.Hkv = cache->num_kv_heads;
+  p.bs = bs;
+  p.Hq = num_q_heads;
+  p.G = G;
+  p.max_blocks = max_blocks_per_seq;
+  p.B = num_seqs;
+  p.max_ctx = max_context_len;
+  p.max_parts = max_parts;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cache->dtype == PA_DTYPE_F32) return launch_decode_dtype<float>(p, cache->head_dim, max_parts, st);
+  return launch_decode_dtype<__nv_bfloat16>(p, cache->head_dim, max_parts, st);
+}
+
+PA_API pa_status pa_read_device_error(void *stream, int32_t *bits) {
+  if (!bits) return PA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return PA_ERR_CUDA;
+  int32_t v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, pa::g_error, sizeof v) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(pa::g_error, &zero, sizeof zero) != cudaSuccess) return PA_ERR_CUDA;
+  *bits = v;
+  return PA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,325 @@
+// Paged decode attention, split-context partition kernel on CUDA cores, and
+// the log-sum-exp reduce that merges partitions.
+//
+// The method follows the block table ("PagedAttention Internals", "The Block
+// Table Map"; "pagedattention" glossary entry, paragraph "Paging maps logical
+// tokens to physical blocks through a block table"): for sequence b, logical
+// token t is read from physical block table[b][t / bs], offset t % bs.  The
+// attention arithmetic is the textbook decode step with an online softmax;
+// scores are kept in base-2 units (the host folds log2(e) into the scale).
+//
+// Work unit = (partition of PA_PARTITION_TOKENS tokens, kv head g, sequence b),
+// one CTA of 4 warps.  Warp w takes the unit's blocks w, w+4, w+8, ...; each
+// warp runs its own ring of `nstages` shared-memory slots filled by 1-D bulk
+// copies (TMA engine) of whole (block, kv head) tiles, K and V, which are
+// contiguous bs x D runs in the pool layout.  Lane 0 of the warp is the
+// producer.  All G query heads of the group are processed together, so each
+// key/value byte is read from HBM once per step.
+//
+// Inside a warp a row of D elements is split into 16-byte slices: lane
+// (rg, dl) owns slice dl of rows rg, rg + RPP, ...  A row's score is reduced
+// over its LPR lanes with xor shuffles; the value accumulation needs no
+// reduction until the end, where row groups and then warps are merged.
+#pragma once
+
+#include "pa_device.cuh"
+
+namespace pa {
+
+struct DecodeParams {
+  const void *q;
+  const void *k;
+  const void *v;
+  void *out;
+  const int32_t *tables;
+  const int32_t *lens;
+  float *ws_m;    // [B][Hq][max_parts] running max (base-2 units)
+  float *ws_l;    // [B][Hq][max_parts] sum of weights
+  float *ws_acc;  // [B][Hq][max_parts][D] unnormalised accumulator
+  int32_t num_blocks, Hkv, bs, Hq, G, max_blocks, B, max_ctx, max_parts;
+  float scale_log2;  // scale * log2(e)
+};
+
+constexpr int kPart = PA_PARTITION_TOKENS;
+constexpr int kWarps = 4;
+
+__device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kWarps * 32)
+    decode_partition_simt(DecodeParams p, int nstages) {
+  constexpr int VEC = Vec16<T>::N;
+  constexpr int LPR = D / VEC;  // lanes per row
+  constexpr int RPP = 32 / LPR; // rows per warp pass
+  constexpr int SUB = (G >= 8) ? 8 : 16;  // rows per softmax sub-tile
+  static_assert(LPR >= 1 && LPR <= 32 && 32 % LPR == 0, "head_dim / vector width");
+  static_assert(SUB % RPP == 0, "sub-tile");
+  constexpr int RPL = SUB / RPP;  // rows per lane per sub-tile
+
+  const int part = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rg = lane / LPR, dl = lane % LPR;
+  const int bs = p.bs;
+  T *out = reinterpret_cast<T *>(p.out);
+
+  const int ctx = p.lens[b];
+  if (ctx < 0 || ctx > p.max_ctx) {
+    if (part == 0) {
+      if (threadIdx.x == 0) raise_error(PA_DEVERR_LEN);
+      for (int i = threadIdx.x; i < G * D; i += blockDim.x)
+        store_out(out + ((size_t)b * p.Hq + g * G) * D + i, 0.f);
+    }
+    return;
+  }
+  if (ctx == 0) {
+    if (part == 0)
+      for (int i = threadIdx.x; i < G * D; i += blockDim.x)
+        store_out(out + ((size_t)b * p.Hq + g * G) * D + i, 0.f);
+    return;
+  }
+  const int t0 = part * kPart;
+  if (t0 >= ctx) return;
+  const int t1 = min(t0 + kPart, ctx);
+  const int nparts = (ctx + kPart - 1) / kPart;
+  const int j0 = t0 / bs;
+  const int nblk = (t1 - t0 + bs - 1) / bs;
+  const uint32_t tile_elems = (uint32_t)bs * D;
+  const uint32_t tile_bytes = tile_elems * sizeof(T);
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  // [kWarps][nstages] slots of (K tile, V tile), then [kWarps][nstages] mbarriers
+  T *ring = reinterpret_cast<T *>(smem) + (size_t)warp * nstages * 2 * tile_elems;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)kWarps * nstages * 2 * tile_bytes) +
+                   warp * nstages;
+
+  const T *kpool = reinterpret_cast<const T *>(p.k);
+  const T *vpool = reinterpret_cast<const T *>(p.v);
+  const int32_t *trow = p.tables + (size_t)b * p.max_blocks;
+  const int nmy = (warp < nblk) ? (nblk - warp + kWarps - 1) / kWarps : 0;
+
+  __shared__ int aborted;
+  if (threadIdx.x == 0) aborted = 0;
+  if (lane == 0) {
+    for (int s = 0; s < nstages; ++s) mbar_init(&bars[s], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const uint64_t pol = policy_evict_first();
+  auto issue = [&](int i) {  // lane 0: bring my i-th block into slot i % nstages
+    const int s = i % nstages;
+    const int32_t blk = trow[j0 + warp + kWarps * i];
+    if (blk >= 0 && blk < p.num_blocks) {
+      const size_t off = ((size_t)blk * p.Hkv + g) * tile_elems;
+      mbar_arrive_expect_tx(&bars[s], 2 * tile_bytes);
+      bulk_copy_g2s(ring + (size_t)s * 2 * tile_elems, kpool + off, tile_bytes, &bars[s], pol);
+      bulk_copy_g2s(ring + (size_t)s * 2 * tile_elems + tile_elems, vpool + off, tile_bytes,
+                    &bars[s], pol);
+    } else {
+      raise_error(PA_DEVERR_TABLE);
+      mbar_arrive(&bars[s]);  // completes the phase with nothing loaded
+    }
+  };
+  if (lane == 0)
+    for (int i = 0; i < nmy && i < nstages; ++i) issue(i);
+
+  // this lane's slice of the G query rows, pre-scaled into base-2 units
+  float qv[G][VEC];
+  {
+    const T *qb = reinterpret_cast<const T *>(p.q) + ((size_t)b * p.Hq + g * G) * D + dl * VEC;
+#pragma unroll
+    for (int gi = 0; gi < G; ++gi) {
+      Vec16<T>::load(qb + (size_t)gi * D, qv[gi]);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) qv[gi][e] *= p.scale_log2;
+    }
+  }
+
+  float m[G], l[G], acc[G][VEC];
+#pragma unroll
+  for (int gi = 0; gi < G; ++gi) {
+    m[gi] = -INFINITY;
+    l[gi] = 0.f;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[gi][e] = 0.f;
+  }
+
+  bool ok = true;
+  for (int i = 0; i < nmy; ++i) {
+    const int s = i % nstages;
+    // the vote keeps the warp converged even if one lane alone gave up
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[s], (uint32_t)((i / nstages) & 1)))) {
+      if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+      ok = false;
+      break;
+    }
+    const int j = j0 + warp + kWarps * i;
+    const int32_t blk = trow[j];
+    const int rows = min(bs, t1 - j * bs);  // valid rows of this block
+    const T *Kt = ring + (size_t)s * 2 * tile_elems;
+    const T *Vt = Kt + tile_elems;
+    if (blk >= 0 && blk < p.num_blocks) {
+      for (int r0 = 0; r0 < rows; r0 += SUB) {
+        float sc[G][RPL];
+        // scores of rows r0 + rg + RPP*k
+#pragma unroll
+        for (int k = 0; k < RPL; ++k) {
+          const int r = r0 + rg + RPP * k;
+          float x[VEC];
+          Vec16<T>::load(Kt + (size_t)(r < bs ? r : 0) * D + dl * VEC, x);
+#pragma unroll
+          for (int gi = 0; gi < G; ++gi) {
+            float d0 = 0.f;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) d0 = fmaf(qv[gi][e], x[e], d0);
+#pragma unroll
+            for (int o = 1; o < LPR; o <<= 1) d0 += __shfl_xor_sync(0xffffffffu, d0, o);
+            sc[gi][k] = (r < rows) ? d0 : -INFINITY;
+          }
+        }
+        // online softmax update (every lane ends with the same m)
+#pragma unroll
+        for (int gi = 0; gi < G; ++gi) {
+          float mx = sc[gi][0];
+#pragma unroll
+          for (int k = 1; k < RPL; ++k) mx = fmaxf(mx, sc[gi][k]);
+#pragma unroll
+          for (int o = LPR; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          const float mnew = fmaxf(m[gi], mx);
+          const float alpha = (m[gi] == mnew) ? 1.f : fast_exp2(m[gi] - mnew);
+          m[gi] = mnew;
+          l[gi] *= alpha;
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) acc[gi][e] *= alpha;
+#pragma unroll
+          for (int k = 0; k < RPL; ++k) {
+            const float w = (sc[gi][k] == -INFINITY) ? 0.f : fast_exp2(sc[gi][k] - mnew);
+            sc[gi][k] = w;
+            l[gi] += w;
+          }
+        }
+        // weighted values
+#pragma unroll
+        for (int k = 0; k < RPL; ++k) {
+          const int r = r0 + rg + RPP * k;
+          if (r < rows) {
+            float x[VEC];
+            Vec16<T>::load(Vt + (size_t)r * D + dl * VEC, x);
+#pragma unroll
+            for (int gi = 0; gi < G; ++gi)
+#pragma unroll
+              for (int e = 0; e < VEC; ++e) acc[gi][e] = fmaf(sc[gi][k], x[e], acc[gi][e]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0 && i + nstages < nmy) {
+      fence_proxy_async_smem();
+      issue(i + nstages);
+    }
+  }
+  // a warp that gave up drops the whole unit; every thread still meets the
+  // barriers below so none waits on an exited warp
+  if (!ok && lane == 0) atomicOr(&aborted, 1);
+
+  // merge row groups of this warp (they share m)
+#pragma unroll
+  for (int gi = 0; gi < G; ++gi) {
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1) {
+      l[gi] += __shfl_xor_sync(0xffffffffu, l[gi], o);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[gi][e] += __shfl_xor_sync(0xffffffffu, acc[gi][e], o);
+    }
+  }
+  __syncthreads();  // every warp is done with its ring: reuse it for the merge
+  if (aborted) return;
+  float *wm = reinterpret_cast<float *>(smem);   // [kWarps][G]
+  float *wl = wm + kWarps * G;                   // [kWarps][G]
+  float *wacc = wl + kWarps * G;                 // [kWarps][G][D]
+  if (rg == 0) {
+#pragma unroll
+    for (int gi = 0; gi < G; ++gi) {
+      if (dl == 0) {
+        wm[warp * G + gi] = m[gi];
+        wl[warp * G + gi] = l[gi];
+      }
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) wacc[(warp * G + gi) * D + dl * VEC + e] = acc[gi][e];
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+    const int gi = idx / D, d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wm[w * G + gi]);
+    float L = 0.f, A = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float mw = wm[w * G + gi];
+      const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+      L += wl[w * G + gi] * f;
+      A += wacc[(w * G + gi) * D + d] * f;
+    }
+    const int h = g * G + gi;
+    if (nparts == 1) {
+      store_out(out + ((size_t)b * p.Hq + h) * D + d, L > 0.f ? A / L : 0.f);
+    } else {
+      const size_t row = ((size_t)b * p.Hq + h) * p.max_parts + part;
+      p.ws_acc[row * D + d] = A;
+      if (d == 0) {
+        p.ws_m[row] = M;
+        p.ws_l[row] = L;
+      }
+    }
+  }
+}
+
+// Merges the partitions of one (sequence, query head):
+//   M = max_p m_p,  L = sum_p l_p 2^(m_p - M),  out = sum_p acc_p 2^(m_p - M) / L
+template <typename T, int D>
+__global__ void __launch_bounds__(128) decode_reduce(DecodeParams p) {
+  extern __shared__ float wsh[];  // [max_parts] weights
+  __shared__ float red[32];
+  const int bh = blockIdx.x;
+  const int b = bh / p.Hq;
+  const int ctx = p.lens[b];
+  if (ctx <= kPart || ctx > p.max_ctx) return;  // written directly by the partition kernel
+  const int np = (ctx + kPart - 1) / kPart;
+  const float *m = p.ws_m + (size_t)bh * p.max_parts;
+  const float *l = p.ws_l + (size_t)bh * p.max_parts;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+
+  float mx = -INFINITY;
+  for (int i = threadIdx.x; i < np; i += blockDim.x) mx = fmaxf(mx, m[i]);
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  float M = red[0];
+  for (int w = 1; w < nw; ++w) M = fmaxf(M, red[w]);
+  __syncthreads();
+
+  float ls = 0.f;
+  for (int i = threadIdx.x; i < np; i += blockDim.x) {
+    const float f = (m[i] == -INFINITY) ? 0.f : fast_exp2(m[i] - M);
+    wsh[i] = f;
+    ls += l[i] * f;
+  }
+  for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+  if (lane == 0) red[warp] = ls;
+  __syncthreads();
+  float L = 0.f;
+  for (int w = 0; w < nw; ++w) L += red[w];
+
+  const float *acc = p.ws_acc + (size_t)bh * p.max_parts * D;
+  T *out = reinterpret_cast<T *>(p.out) + (size_t)bh * D;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float a = 0.f;
+    for (int i = 0; i < np; ++i) a = fmaf(acc[(size_t)i * D + d], wsh[i], a);
+    store_out(out + d, L > 0.f ? a / L : 0.f);
+  }
+}
+
+}  // namespace pa

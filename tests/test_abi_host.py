@@ -1,0 +1,227 @@
+"""The C ABI on the host (no GPU): exported symbols, argument checks that
+return before any launch, the copy-pair check, and the C++ allocator against
+the oracle's allocator model."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import paged_kv_cache_402_b200 as pa
+from paged_kv_cache_402_b200 import synth
+
+HEADER_DIR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(HEADER_DIR):
+        if f.endswith(".h"):
+            text = open(os.path.join(HEADER_DIR, f)).read()
+            names |= set(re.findall(r"PA_API\s+[\w\s\*]*?\b(pa_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for required in ("pa_append_kv", "pa_decode", "pa_copy_blocks", "pa_decode_workspace_size",
+                     "pa_read_device_error", "pa_alloc_create", "pa_seq_append", "pa_seq_fork"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(pa.LIB_PATH)
+    missing = [n for n in _declared() if not hasattr(L, n)]
+    assert not missing, f"not exported: {missing}"
+
+
+def test_no_internal_symbols_exported():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", pa.LIB_PATH], capture_output=True, text=True).stdout
+    ours = {l.split()[-1] for l in out.splitlines() if l.split() and l.split()[-1].startswith("pa_")}
+    assert ours == set(_declared())
+
+
+def test_status_strings_and_version():
+    assert pa.lib().pa_status_string(pa.PA_OK) == b"ok"
+    assert pa.lib().pa_status_string(pa.PA_ERR_OUT_OF_BLOCKS) == b"out of free blocks"
+    assert pa.lib().pa_version().count(b".") == 2
+
+
+def _cache_struct(**kw):
+    d = dict(k=16, v=32, dtype=pa.PA_DTYPE_BF16, num_blocks=8, block_size=16, num_kv_heads=2, head_dim=128)
+    d.update(kw)
+    return pa.pa_cache_t(**d)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dtype=7), pa.PA_ERR_UNSUPPORTED),
+    (dict(block_size=12), pa.PA_ERR_UNSUPPORTED),
+    (dict(head_dim=96), pa.PA_ERR_UNSUPPORTED),
+    (dict(num_blocks=0), pa.PA_ERR_INVALID_ARG),
+    (dict(k=0), pa.PA_ERR_INVALID_ARG),
+    (dict(k=17), pa.PA_ERR_INVALID_ARG),  # misaligned pool
+])
+def test_bad_cache_rejected_before_launch(kw, expect):
+    c = _cache_struct(**kw)
+    L = pa.lib()
+    assert L.pa_append_kv(16, 16, 16, 1, ctypes.byref(c), None) == expect
+    assert L.pa_copy_blocks(16, 1, ctypes.byref(c), None) == expect
+    assert L.pa_decode(16, ctypes.byref(c), 16, 4, 16, 1, 2, 64, 1.0, 16, None, 0, None) == expect
+
+
+def test_decode_argument_checks():
+    c = _cache_struct()
+    L = pa.lib()
+    args = lambda **o: [o.get("q", 16), ctypes.byref(c), 16, o.get("mb", 4), 16, o.get("B", 1), o.get("Hq", 2),
+                        o.get("ml", 64), o.get("scale", 1.0), o.get("out", 16), o.get("ws", None),
+                        o.get("wsb", 0), None]
+    assert L.pa_decode(*args(Hq=3)) == pa.PA_ERR_INVALID_ARG          # not a multiple of Hkv
+    assert L.pa_decode(*args(Hq=6)) == pa.PA_ERR_UNSUPPORTED           # group size 3
+    assert L.pa_decode(*args(Hq=32)) == pa.PA_ERR_UNSUPPORTED          # group size 16
+    assert L.pa_decode(*args(ml=65)) == pa.PA_ERR_INVALID_ARG          # 65 tokens > 4 blocks x 16
+    assert L.pa_decode(*args(scale=float("nan"))) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_decode(*args(q=0)) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_decode(*args(out=8)) == pa.PA_ERR_INVALID_ARG          # misaligned
+    # a context past one partition needs a workspace
+    assert L.pa_decode(*args(mb=64, ml=1000)) == pa.PA_ERR_INVALID_ARG
+    need = L.pa_decode_workspace_size(1, 2, 1000, 128)
+    assert L.pa_decode(*args(mb=64, ml=1000, ws=16, wsb=need - 16)) == pa.PA_ERR_TOO_SMALL
+    assert L.pa_decode(*args(B=0)) == pa.PA_OK                         # nothing to do, no launch
+
+
+def test_workspace_size():
+    ws = pa.pa_decode_workspace_size
+    assert ws(4, 8, 512, 128) == 0
+    rows = 4 * 8 * 2
+    assert ws(4, 8, 513, 128) == 2 * ((rows * 4 + 15) // 16 * 16) + rows * 128 * 4
+    assert ws(8, 32, 131072, 128) == 2 * 8 * 32 * 256 * 4 + 8 * 32 * 256 * 128 * 4
+
+
+def test_check_copy_pairs():
+    assert pa.pa_check_copy_pairs([[1, 2], [3, 4]], 8)
+    assert not pa.pa_check_copy_pairs([[1, 2], [3, 2]], 8)   # repeated destination
+    assert not pa.pa_check_copy_pairs([[1, 2], [2, 4]], 8)   # destination is a source
+    assert not pa.pa_check_copy_pairs([[1, 8]], 8)           # outside the pool
+    assert pa.pa_check_copy_pairs(np.zeros((0, 2)), 8)
+
+
+# ------------------------------------------------------------- allocator
+
+
+def test_allocator_basics_match_model():
+    order = [8, 3, 11] + [b for b in range(12) if b not in (8, 3, 11)]
+    A = pa.Allocator(12, 16, order)
+    M = oracle.AllocatorModel(12, 16, order)
+    s, m = A.new_seq(), M.new_seq()
+    slots, cow = A.append(s, 48)
+    mslots, mcow = M.append(m, 48)
+    assert slots.tolist() == mslots and cow is None and mcow is None
+    assert A.block_table(s) == [8, 3, 11]
+    with pytest.raises(pa.OutOfBlocks):
+        A.append(s, 16 * 10)
+    assert A.seq_len(s) == (48, 3)
+
+
+def test_allocator_rejects_bad_input():
+    with pytest.raises(pa.PagedAttnError):
+        pa.Allocator(4, 16, [0, 1, 1, 2])
+    A = pa.Allocator(4, 4)
+    with pytest.raises(pa.PagedAttnError):
+        A.append(99, 1)
+    s = A.new_seq()
+    with pytest.raises(pa.PagedAttnError):
+        A.batch_append([s, s], [1, 1])
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_allocator_random_trace_matches_model(seed):
+    """Random new / fork / free / (batch) append traces: the C++ allocator and
+    the oracle's model agree on every slot, copy pair, table, refcount and
+    usage figure, and on every out-of-blocks refusal."""
+    r = synth.rng(100 + seed)
+    NB, bs = 96, int(r.choice([1, 2, 4, 8, 16]))
+    order = r.permutation(NB)
+    A, M = pa.Allocator(NB, bs, order), oracle.AllocatorModel(NB, bs, order)
+    live = []
+    for step in range(500):
+        op = int(r.integers(0, 6))
+        if op == 0 or not live:
+            a, m = A.new_seq(), M.new_seq()
+            assert a == m
+            live.append(a)
+        elif op == 1:
+            p = live[int(r.integers(len(live)))]
+            a, m = A.fork(p), M.fork(p)
+            assert a == m
+            live.append(a)
+        elif op == 2 and len(live) > 1:
+            s = live.pop(int(r.integers(len(live))))
+            A.free_seq(s)
+            M.free_seq(s)
+        elif op == 3:
+            s = live[int(r.integers(len(live)))]
+            n = int(r.integers(0, 3 * bs))
+            try:
+                got = A.append(s, n)
+                ok = True
+            except pa.OutOfBlocks:
+                ok = False
+            try:
+                want = M.append(s, n)
+                assert ok
+                assert got[0].tolist() == want[0] and got[1] == want[1]
+            except oracle.OutOfBlocks:
+                assert not ok
+        else:
+            k = int(r.integers(1, len(live) + 1))
+            sel = [int(x) for x in r.choice(live, size=k, replace=False)]
+            ns = [int(x) for x in r.integers(0, 2 * bs, size=k)]
+            try:
+                gs, gp = A.batch_append(sel, ns)
+                ok = True
+            except pa.OutOfBlocks:
+                ok = False
+            try:
+                ws, wp = M.batch_append(sel, ns)
+                assert ok
+                assert gs.tolist() == ws
+                assert [tuple(x) for x in gp.tolist()] == wp
+            except oracle.OutOfBlocks:
+                assert not ok
+        for s in live:
+            assert A.block_table(s) == M.block_table(s)
+            assert A.seq_len(s)[0] == M.lens[s]
+        st = A.stats()
+        u = M.usage()
+        assert st["used_slots"] == u.used and st["allocated_slots"] == u.allocated
+        assert st["free_blocks"] == len(M.free)
+        for b in range(NB):
+            assert A.refcount(b) == M.ref[b]
+
+
+def test_build_block_tables():
+    A = pa.Allocator(32, 4)
+    s = [A.new_seq() for _ in range(3)]
+    for i, n in zip(s, (1, 9, 4)):
+        A.append(i, n)
+    tables, lens = A.build_block_tables(s, 4, pad=-1)
+    assert lens.tolist() == [1, 9, 4]
+    for row, i in zip(tables, s):
+        t = A.block_table(i)
+        assert row[:len(t)].tolist() == t and (row[len(t):] == -1).all()
+    with pytest.raises(pa.PagedAttnError):
+        A.build_block_tables(s, 2)
+
+
+def test_fragmentation_example_through_the_allocator():
+    """The worked example's paged layout (lengths 1, 4, 2; page size 2) in the
+    C++ allocator: 8 slots allocated, 1 wasted."""
+    A = pa.Allocator(16, 2)
+    for n in (1, 4, 2):
+        A.append(A.new_seq(), n)
+    st = A.stats()
+    assert st["allocated_slots"] == 8 and st["used_slots"] == 7
+    assert st["fragmentation"] == pytest.approx(0.125)
