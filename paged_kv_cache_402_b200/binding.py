@@ -1,0 +1,325 @@
+"""Python binding of libpagedattn (the paged KV-cache decode path, sm_100a).
+
+Thin ctypes marshalling over the C ABI of ``include/pagedattn.h``: every step
+runs in the library's CUDA kernels (append, block copy, decode partition and
+reduce) or its C++ allocator.  PyTorch supplies device memory and streams
+only.  There is no fallback: if the library is missing, importing this
+module raises.
+
+Names follow the C ABI: ``pa_append_kv``, ``pa_decode``, ``pa_copy_blocks``,
+``pa_decode_workspace_size``, ``pa_read_device_error``,
+``pa_check_copy_pairs``; ``Allocator`` wraps the ``pa_alloc_*`` / ``pa_seq_*``
+calls and ``KVCache`` holds the two pools.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_OUT_OF_BLOCKS = 0, 1, 2, 3
+PA_ERR_CUDA, PA_ERR_NOT_FOUND, PA_ERR_TOO_SMALL = 4, 5, 6
+PA_DTYPE_F32, PA_DTYPE_BF16 = 0, 1
+PA_DEVERR_SLOT, PA_DEVERR_TABLE, PA_DEVERR_PAIR, PA_DEVERR_TIMEOUT, PA_DEVERR_LEN = 1, 2, 4, 8, 16
+PA_PARTITION_TOKENS = 512
+
+_DTYPES = {torch.float32: PA_DTYPE_F32, torch.bfloat16: PA_DTYPE_BF16}
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_lib.pa_status_string(status).decode()} (status {status})")
+
+
+class OutOfBlocks(PagedAttnError):
+    pass
+
+
+class pa_cache_t(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("dtype", ctypes.c_int32),
+                ("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_402_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    i32p, i64p = ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64)
+    cp = ctypes.POINTER(pa_cache_t)
+    st = ctypes.c_int
+    sigs = {
+        "pa_append_kv": (st, [vp, vp, vp, i32, cp, vp]),
+        "pa_decode": (st, [vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp, sz, vp]),
+        "pa_decode_workspace_size": (sz, [i32, i32, i32, i32]),
+        "pa_copy_blocks": (st, [vp, i32, cp, vp]),
+        "pa_check_copy_pairs": (st, [i32p, i32, i32]),
+        "pa_read_device_error": (st, [vp, i32p]),
+        "pa_status_string": (ctypes.c_char_p, [st]),
+        "pa_version": (ctypes.c_char_p, []),
+        "pa_alloc_create": (st, [i32, i32, i32p, ctypes.POINTER(vp)]),
+        "pa_alloc_destroy": (None, [vp]),
+        "pa_seq_new": (st, [vp, i32p]),
+        "pa_seq_fork": (st, [vp, i32, i32p]),
+        "pa_seq_free": (st, [vp, i32]),
+        "pa_seq_append": (st, [vp, i32, i32, i64p, i32p, i32p]),
+        "pa_batch_append": (st, [vp, i32p, i32p, i32, i64p, i32p, i32p]),
+        "pa_seq_len": (st, [vp, i32, i32p, i32p]),
+        "pa_seq_block_table": (st, [vp, i32, i32p, i32, i32p]),
+        "pa_build_block_tables": (st, [vp, i32p, i32, i32, i32, i32p, i32p]),
+        "pa_alloc_stats": (st, [vp, i64p, i64p, i32p, i32p]),
+        "pa_block_refcount": (st, [vp, i32, i32p]),
+    }
+    for name, (res, args) in sigs.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+_lib = _load()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != PA_OK:
+        if status == PA_ERR_OUT_OF_BLOCKS:
+            raise OutOfBlocks(status, what)
+        raise PagedAttnError(status, what)
+
+
+def _stream_ptr(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _dev(t: torch.Tensor, what: str, dtype=None) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{what} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _i32p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def _i64p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+
+
+# --------------------------------------------------------------------------
+# the pools
+
+
+class KVCache:
+    """The paged pools: k and v of shape [num_blocks, num_kv_heads, block_size, head_dim]."""
+
+    def __init__(self, k: torch.Tensor, v: torch.Tensor):
+        if k.shape != v.shape or k.dtype != v.dtype or k.dim() != 4:
+            raise ValueError("k and v must be [num_blocks, Hkv, block_size, head_dim] of one dtype")
+        if k.dtype not in _DTYPES:
+            raise TypeError(f"unsupported cache dtype {k.dtype}")
+        _dev(k, "k_cache")
+        _dev(v, "v_cache")
+        self.k, self.v = k, v
+        self.struct = pa_cache_t(k.data_ptr(), v.data_ptr(), _DTYPES[k.dtype], k.shape[0], k.shape[2],
+                                 k.shape[1], k.shape[3])
+
+    @classmethod
+    def empty(cls, num_blocks, num_kv_heads, block_size, head_dim, dtype=torch.bfloat16, device="cuda"):
+        shape = (num_blocks, num_kv_heads, block_size, head_dim)
+        return cls(torch.empty(shape, dtype=dtype, device=device), torch.empty(shape, dtype=dtype, device=device))
+
+    @property
+    def num_blocks(self):
+        return self.k.shape[0]
+
+    @property
+    def num_kv_heads(self):
+        return self.k.shape[1]
+
+    @property
+    def block_size(self):
+        return self.k.shape[2]
+
+    @property
+    def head_dim(self):
+        return self.k.shape[3]
+
+    @property
+    def dtype(self):
+        return self.k.dtype
+
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+
+# --------------------------------------------------------------------------
+# kernels
+
+
+def pa_append_kv(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor, cache: KVCache, stream=None) -> None:
+    """Scatters new key/value rows [N, Hkv, D] into the pools at slot_mapping [N] (int64)."""
+    n = slot_mapping.numel()
+    if k.shape != (n, cache.num_kv_heads, cache.head_dim) or v.shape != k.shape:
+        raise ValueError("k, v must be [num_tokens, num_kv_heads, head_dim]")
+    _check(_lib.pa_append_kv(_dev(k, "k", cache.dtype), _dev(v, "v", cache.dtype),
+                             _dev(slot_mapping, "slot_mapping", torch.int64), n, cache.ref(),
+                             _stream_ptr(stream)), "pa_append_kv")
+
+
+def pa_decode_workspace_size(num_seqs: int, num_q_heads: int, max_context_len: int, head_dim: int) -> int:
+    return int(_lib.pa_decode_workspace_size(num_seqs, num_q_heads, max_context_len, head_dim))
+
+
+def pa_decode(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor, context_lens: torch.Tensor,
+              max_context_len: int, scale: float, out: torch.Tensor | None = None,
+              workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Paged decode attention; returns out [B, Hq, D] in the cache dtype."""
+    B, Hq, D = q.shape
+    if D != cache.head_dim:
+        raise ValueError("head_dim mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("block_tables must be [B, max_blocks] and context_lens [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    need = pa_decode_workspace_size(B, Hq, int(max_context_len), D)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.pa_decode(_dev(q, "q", cache.dtype), cache.ref(), _dev(block_tables, "block_tables", torch.int32),
+                          block_tables.shape[1], _dev(context_lens, "context_lens", torch.int32), B, Hq,
+                          int(max_context_len), float(scale), _dev(out, "out", cache.dtype), ws_ptr, ws_bytes,
+                          _stream_ptr(stream)), "pa_decode")
+    return out
+
+
+def pa_copy_blocks(src_dst_pairs: torch.Tensor, cache: KVCache, stream=None) -> None:
+    """Copies whole blocks of both pools: pairs [n, 2] int32 (src, dst) on the device."""
+    n = src_dst_pairs.shape[0] if src_dst_pairs.numel() else 0
+    if n and (src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2):
+        raise ValueError("pairs must be [n, 2]")
+    _check(_lib.pa_copy_blocks(_dev(src_dst_pairs, "pairs", torch.int32) if n else None, n, cache.ref(),
+                               _stream_ptr(stream)), "pa_copy_blocks")
+
+
+def pa_check_copy_pairs(pairs, num_blocks: int) -> bool:
+    a = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+    return _lib.pa_check_copy_pairs(_i32p(a), a.shape[0], int(num_blocks)) == PA_OK
+
+
+def pa_read_device_error(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device error bits."""
+    bits = ctypes.c_int32(0)
+    _check(_lib.pa_read_device_error(_stream_ptr(stream), ctypes.byref(bits)), "pa_read_device_error")
+    return bits.value
+
+
+# --------------------------------------------------------------------------
+# the host allocator
+
+
+class Allocator:
+    """Reference-counted block allocator (C++), copy on write of shared partial blocks."""
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        self.num_blocks, self.block_size = int(num_blocks), int(block_size)
+        h = ctypes.c_void_p()
+        order = None
+        if free_order is not None:
+            self._order = np.ascontiguousarray(np.asarray(free_order, dtype=np.int32))
+            if self._order.shape != (self.num_blocks,):
+                raise ValueError("free_order must list every block once")
+            order = _i32p(self._order)
+        _check(_lib.pa_alloc_create(self.num_blocks, self.block_size, order, ctypes.byref(h)), "pa_alloc_create")
+        self._h = h
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            _lib.pa_alloc_destroy(h)
+            self._h = None
+
+    def new_seq(self) -> int:
+        s = ctypes.c_int32()
+        _check(_lib.pa_seq_new(self._h, ctypes.byref(s)), "pa_seq_new")
+        return s.value
+
+    def fork(self, parent: int) -> int:
+        s = ctypes.c_int32()
+        _check(_lib.pa_seq_fork(self._h, int(parent), ctypes.byref(s)), "pa_seq_fork")
+        return s.value
+
+    def free_seq(self, seq: int) -> None:
+        _check(_lib.pa_seq_free(self._h, int(seq)), "pa_seq_free")
+
+    def append(self, seq: int, n: int):
+        """Returns (slots int64 [n], cow pair (src, dst) or None)."""
+        slots = np.empty(max(n, 1), dtype=np.int64)
+        pair = np.empty(2, dtype=np.int32)
+        ncow = ctypes.c_int32()
+        _check(_lib.pa_seq_append(self._h, int(seq), int(n), _i64p(slots), _i32p(pair), ctypes.byref(ncow)),
+               "pa_seq_append")
+        return slots[:n], ((int(pair[0]), int(pair[1])) if ncow.value else None)
+
+    def batch_append(self, seqs, n_tokens, out_slots: np.ndarray | None = None, out_pairs: np.ndarray | None = None):
+        """Returns (slots int64 [sum n], cow pairs int32 [k, 2])."""
+        seqs = np.ascontiguousarray(np.asarray(seqs, dtype=np.int32))
+        n_tokens = np.ascontiguousarray(np.asarray(n_tokens, dtype=np.int32))
+        total = int(n_tokens.sum())
+        slots = out_slots if out_slots is not None else np.empty(max(total, 1), dtype=np.int64)
+        pairs = out_pairs if out_pairs is not None else np.empty((max(len(seqs), 1), 2), dtype=np.int32)
+        ncow = ctypes.c_int32()
+        _check(_lib.pa_batch_append(self._h, _i32p(seqs), _i32p(n_tokens), len(seqs), _i64p(slots),
+                                    _i32p(pairs), ctypes.byref(ncow)), "pa_batch_append")
+        return slots[:total], pairs[:ncow.value]
+
+    def seq_len(self, seq: int):
+        n, nb = ctypes.c_int32(), ctypes.c_int32()
+        _check(_lib.pa_seq_len(self._h, int(seq), ctypes.byref(n), ctypes.byref(nb)), "pa_seq_len")
+        return n.value, nb.value
+
+    def block_table(self, seq: int) -> list:
+        _, nb = self.seq_len(seq)
+        out = np.empty(max(nb, 1), dtype=np.int32)
+        cnt = ctypes.c_int32()
+        _check(_lib.pa_seq_block_table(self._h, int(seq), _i32p(out), nb, ctypes.byref(cnt)), "pa_seq_block_table")
+        return out[:cnt.value].tolist()
+
+    def build_block_tables(self, seqs, max_blocks: int, pad: int = -1, out_tables=None, out_lens=None):
+        seqs = np.ascontiguousarray(np.asarray(seqs, dtype=np.int32))
+        tables = out_tables if out_tables is not None else np.empty((len(seqs), max_blocks), dtype=np.int32)
+        lens = out_lens if out_lens is not None else np.empty(len(seqs), dtype=np.int32)
+        _check(_lib.pa_build_block_tables(self._h, _i32p(seqs), len(seqs), int(max_blocks), int(pad),
+                                          _i32p(tables), _i32p(lens)), "pa_build_block_tables")
+        return tables, lens
+
+    def stats(self) -> dict:
+        used, alloc = ctypes.c_int64(), ctypes.c_int64()
+        free, usedb = ctypes.c_int32(), ctypes.c_int32()
+        _check(_lib.pa_alloc_stats(self._h, ctypes.byref(used), ctypes.byref(alloc), ctypes.byref(free),
+                                   ctypes.byref(usedb)), "pa_alloc_stats")
+        frag = (alloc.value - used.value) / alloc.value if alloc.value else 0.0
+        return dict(used_slots=used.value, allocated_slots=alloc.value, free_blocks=free.value,
+                    used_blocks=usedb.value, fragmentation=frag)
+
+    def refcount(self, block: int) -> int:
+        r = ctypes.c_int32()
+        _check(_lib.pa_block_refcount(self._h, int(block), ctypes.byref(r)), "pa_block_refcount")
+        return r.value
