@@ -135,6 +135,38 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
                                        int32_t max_context_len, int32_t head_dim);
 
 /*
+ * pa_decode without a caller-provided workspace.  The pages have no
+ * counterpart: this is a convenience of this library for callers that cannot
+ * allocate device memory at decode time -- for example a serving process that
+ * has handed nearly all of HBM to the paged KV pool (the pool is normally
+ * sized to fill whatever memory is left, so a workspace allocation can fail),
+ * or code running behind a plugin or runtime interface that offers no device
+ * allocator.  It allocates nothing: the split-context scratch lives in one
+ * fixed array of PA_STATIC_WORKSPACE_BYTES inside the library, which every
+ * GPU that loads the library holds until the process exits.
+ *  - Arguments and results are those of pa_decode (minus the workspace).
+ *  - Sizes whose scratch, pa_decode_workspace_size(num_seqs, num_q_heads,
+ *    max_context_len, head_dim), exceeds PA_STATIC_WORKSPACE_BYTES are
+ *    rejected with PA_ERR_TOO_SMALL before any launch.
+ *  - The first call on a device looks up that device's copy of the array
+ *    (with the device current); make that first call before any stream
+ *    capture.  Later calls on the device reuse the address.
+ *  - Every call on a device shares the one array and it keeps the last call's
+ *    contents.  Nothing in it needs to start at zero: each entry the merge
+ *    step reads is written earlier in the same call.  Calls whose kernels
+ *    overlap on the GPU (different streams, no ordering between them) race
+ *    on the array and may return wrong results; order them on one stream.
+ */
+#define PA_STATIC_WORKSPACE_BYTES (8u << 20)
+
+PA_API pa_status pa_decode_static_workspace(const void *q, const pa_cache_t *cache,
+                                            const int32_t *block_tables,
+                                            int32_t max_blocks_per_seq,
+                                            const int32_t *context_lens, int32_t num_seqs,
+                                            int32_t num_q_heads, int32_t max_context_len,
+                                            float scale, void *out, void *stream);
+
+/*
  * Copy-on-write block copy (glossary entry, comparison table "share blocks
  * copy-on-write" and paragraph "It is the core of vLLM ...": sharers fork
  * only when they diverge).  For every pair i, physical block

@@ -59,6 +59,7 @@ def _load() -> ctypes.CDLL:
         "pa_append_kv": (st, [vp, vp, vp, i32, cp, vp]),
         "pa_decode": (st, [vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp, sz, vp]),
         "pa_decode_workspace_size": (sz, [i32, i32, i32, i32]),
+        "pa_decode_static_workspace": (st, [vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp]),
         "pa_copy_blocks": (st, [vp, i32, cp, vp]),
         "pa_check_copy_pairs": (st, [i32p, i32, i32]),
         "pa_read_device_error": (st, [vp, i32p]),
@@ -207,6 +208,27 @@ def pa_decode(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor, conte
                           block_tables.shape[1], _dev(context_lens, "context_lens", torch.int32), B, Hq,
                           int(max_context_len), float(scale), _dev(out, "out", cache.dtype), ws_ptr, ws_bytes,
                           _stream_ptr(stream)), "pa_decode")
+    return out
+
+
+PA_STATIC_WORKSPACE_BYTES = 8 << 20
+
+
+def pa_decode_static_workspace(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor,
+                               context_lens: torch.Tensor, max_context_len: int, scale: float,
+                               out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """pa_decode with the library's fixed scratch array instead of a
+    workspace (for callers that cannot allocate device memory); raises
+    PagedAttnError (buffer too small) past PA_STATIC_WORKSPACE_BYTES."""
+    B, Hq, D = q.shape
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("block_tables must be [B, max_blocks] and context_lens [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    _check(_lib.pa_decode_static_workspace(
+        _dev(q, "q", cache.dtype), cache.ref(), _dev(block_tables, "block_tables", torch.int32),
+        block_tables.shape[1], _dev(context_lens, "context_lens", torch.int32), B, Hq, int(max_context_len),
+        float(scale), _dev(out, "out", cache.dtype), _stream_ptr(stream)), "pa_decode_static_workspace")
     return out
 
 

@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "pa_copy_kernels.cuh"
@@ -227,6 +228,64 @@ PA_API pa_status pa_decode(const void *q, const pa_cache_t *cache, const int32_t
   cudaStream_t st = (cudaStream_t)stream;
   if (cache->dtype == PA_DTYPE_F32) return launch_decode_dtype<float>(p, cache->head_dim, max_parts, st);
   return launch_decode_dtype<__nv_bfloat16>(p, cache->head_dim, max_parts, st);
+}
+
+// ---------------------------------------------------------------------------
+// pa_decode_static_workspace: pa_decode whose split-context scratch is this
+// file-scope array instead of caller memory, for callers that cannot
+// allocate device memory.  Host code must not use the array's name as a
+// device address (it is a host-side stand-in); the device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current
+// and kept below.
+
+}  // extern "C"
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_static_workspace[PA_STATIC_WORKSPACE_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_ws_mutex;
+void *g_static_ws_ptr[kMaxDevices] = {};
+
+// Device address of this device's copy of g_static_workspace, or nullptr.
+void *static_workspace_for_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+  if (!g_static_ws_ptr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_workspace) != cudaSuccess || !ptr) return nullptr;
+    g_static_ws_ptr[dev] = ptr;
+  }
+  return g_static_ws_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+PA_API pa_status pa_decode_static_workspace(const void *q, const pa_cache_t *cache,
+                                            const int32_t *block_tables,
+                                            int32_t max_blocks_per_seq,
+                                            const int32_t *context_lens, int32_t num_seqs,
+                                            int32_t num_q_heads, int32_t max_context_len,
+                                            float scale, void *out, void *stream) {
+  pa_status s = check_cache(cache);
+  if (s != PA_OK) return s;
+  if (num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0 || cache->head_dim <= 0)
+    return PA_ERR_INVALID_ARG;
+  const size_t need =
+      num_seqs > 0 ? workspace_bytes_for(num_seqs, num_q_heads, max_context_len, cache->head_dim) : 0;
+  if (need > (size_t)PA_STATIC_WORKSPACE_BYTES) return PA_ERR_TOO_SMALL;
+  void *ws = nullptr;
+  if (need > 0) {
+    ws = static_workspace_for_current_device();
+    if (!ws) return PA_ERR_CUDA;
+  }
+  return pa_decode(q, cache, block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads,
+                   max_context_len, scale, out, ws, need > 0 ? (size_t)PA_STATIC_WORKSPACE_BYTES : 0,
+                   stream);
 }
 
 PA_API pa_status pa_read_device_error(void *stream, int32_t *bits) {
