@@ -3,15 +3,15 @@
  *
  * The method ("PagedAttention Internals", wondering.app, sections "Fixed-Size
  * KV Blocks" and "The Block Table Map"; "pagedattention" glossary entry,
- * chipfoundryservices.com, paragraph "Paging maps logical tokens to physical
- * blocks through a block table"): every sequence's key/value cache is stored
- * in fixed-size physical blocks that may sit anywhere in a shared pool, and a
- * per-sequence block table maps logical block n to its physical block.
- * Attention follows the table; new tokens fill the sequence's current block
- * and a new block is taken only when it is full; sequences that share a
- * prefix (or the samples of a beam search) point at the same physical blocks,
- * which are copied only when a sharer writes into them (glossary entry,
- * comparison table and paragraph "It is the core of vLLM ...").
+ * chipfoundryservices.com, paragraph 3 on block tables): every sequence's
+ * key/value cache is stored in fixed-size physical blocks that may sit
+ * anywhere in a shared pool, and a per-sequence block table maps logical block
+ * n to its physical block.  The attention step reads through the table; new
+ * tokens fill the sequence's current block and a new block is taken only when
+ * it is full; sequences that share a prefix (or the samples of a beam search)
+ * point at the same physical blocks, which are copied only when a sharer
+ * writes into them (glossary entry, comparison table and paragraph 5 on
+ * sharing).
  *
  * Conventions for every entry point:
  *  - Pointers named "device" are CUDA device pointers owned by the caller;
@@ -86,8 +86,8 @@ typedef struct {
 
 /*
  * KV append ("Fixed-Size KV Blocks": tokens fill the current block; the
- * glossary's "Paging maps logical tokens ..." paragraph: the table maps
- * logical positions to physical blocks).
+ * glossary's paragraph 3: the table maps logical positions to physical
+ * blocks).
  *   k, v          device [num_tokens][num_kv_heads][head_dim], cache dtype
  *   slot_mapping  device [num_tokens] int64: token i is written to
  *                 k_cache/v_cache[slot/bs][h][slot%bs][:] for every head h.
@@ -99,10 +99,10 @@ PA_API pa_status pa_append_kv(const void *k, const void *v, const int64_t *slot_
                               int32_t num_tokens, const pa_cache_t *cache, void *stream);
 
 /*
- * Paged decode attention ("The Block Table Map": attention follows the table;
- * the glossary's "the attention kernel follows the table to gather the right
- * keys and values").  The pages give no formula; this is the textbook
- * scaled dot-product step.  For sequence b, query head h and its KV head
+ * Paged decode attention ("The Block Table Map" and the glossary's paragraph
+ * 3: the attention step gathers each sequence's keys and values through its
+ * block table).  The pages give no formula; this is the textbook scaled
+ * dot-product step.  For sequence b, query head h and its KV head
  * g = h / (num_q_heads / num_kv_heads):
  *   s_t = scale * <q[b,h,:], K(b,t,g)>  for t < context_lens[b]
  *   out[b,h,:] = sum_t exp(s_t - max s) V(b,t,g) / sum_t exp(s_t - max s)
@@ -167,9 +167,9 @@ PA_API pa_status pa_decode_static_workspace(const void *q, const pa_cache_t *cac
                                             float scale, void *out, void *stream);
 
 /*
- * Copy-on-write block copy (glossary entry, comparison table "share blocks
- * copy-on-write" and paragraph "It is the core of vLLM ...": sharers fork
- * only when they diverge).  For every pair i, physical block
+ * Copy-on-write block copy (glossary entry, comparison table row on sharing
+ * and paragraph 5: sharers get their own copy of a block only when they
+ * diverge).  For every pair i, physical block
  * src_dst_pairs[2i+1] of both pools becomes a bit copy of block
  * src_dst_pairs[2i] (all kv heads, all slots).
  *   src_dst_pairs device [num_pairs][2] int32

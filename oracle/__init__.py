@@ -13,15 +13,15 @@ Sources, by page and section:
     unused capacity is confined to the incomplete last block.
   - "The Block Table Map": a per-sequence table maps logical block n to a
     physical block (the example maps logical 0, 1, 2 to physical 8, 3, 11);
-    attention follows the table; the logical order is kept.
+    the attention step reads through the table; the logical order is kept.
   - "Sharing And Dynamic Growth": sequences obtain blocks as they need them
     and release them when they finish.
 * "pagedattention" glossary entry (chipfoundryservices.com):
-  - paragraph "Paging maps logical tokens to physical blocks through a block
-    table": blocks of, say, 16 tokens, handed out one at a time.
-  - the comparison table and paragraph "It is the core of vLLM ...": a common
-    prompt prefix or the samples of a beam search point at the same physical
-    blocks and are copied on write only when they diverge.
+  - paragraph 3 (block tables): blocks of 16 tokens as the example, given to
+    a request one at a time as it grows.
+  - the comparison table and paragraph 5 (sharing): a common prompt prefix or
+    the samples of a beam search point at the same physical blocks and are
+    copied on write only when they diverge.
 * learn-ml-visualized chapter "inference-acceleration-pagedattention-vllm", the
   fragmentation worked example:
   waste = allocated - used, fragmentation = total waste / total allocated;

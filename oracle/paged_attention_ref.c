@@ -7,12 +7,11 @@
  * What it follows:
  *  - "PagedAttention Internals" (wondering.app), section "The Block Table Map":
  *    a sequence's logical block n lives in whatever physical block the
- *    sequence's block table names; attention follows the table to find the
- *    keys and values, and the logical order of tokens is kept.
- *  - "pagedattention" glossary entry (chipfoundryservices.com), paragraph
- *    "Paging maps logical tokens to physical blocks through a block table":
- *    fixed-size blocks (16 tokens as the example), one table per request, the
- *    attention kernel gathers keys and values through it.
+ *    sequence's block table names; the attention step reads keys and values
+ *    through that table, and the logical order of tokens is kept.
+ *  - "pagedattention" glossary entry (chipfoundryservices.com), paragraph 3
+ *    (block tables): fixed-size blocks (16 tokens as the example), one table
+ *    per request, and the attention kernel gathers keys and values through it.
  *  - The attention itself is the textbook scaled dot-product decode step
  *    (the pages state no formula): for one query vector q and the keys and
  *    values of tokens 0..n-1,

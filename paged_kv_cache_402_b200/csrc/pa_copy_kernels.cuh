@@ -10,7 +10,7 @@
 // (head_dim * elem bytes = 256 B at D=128 bf16 = 16 lanes x 16 B).
 //
 // Block copy ("pagedattention" glossary entry, comparison table and paragraph
-// "It is the core of vLLM ...": sharers fork copy-on-write): every (src, dst)
+// 5, sharing: sharers copy a block only when they diverge): every (src, dst)
 // pair copies a whole block of both pools, all kv heads.
 #pragma once
 

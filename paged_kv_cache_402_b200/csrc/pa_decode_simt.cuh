@@ -1,10 +1,10 @@
 // Paged decode attention, split-context partition kernel on CUDA cores, and
 // the log-sum-exp reduce that merges partitions.
 //
-// The method follows the block table ("PagedAttention Internals", "The Block
-// Table Map"; "pagedattention" glossary entry, paragraph "Paging maps logical
-// tokens to physical blocks through a block table"): for sequence b, logical
-// token t is read from physical block table[b][t / bs], offset t % bs.  The
+// The method reads keys and values through the block table ("PagedAttention
+// Internals", section "The Block Table Map"; "pagedattention" glossary entry,
+// paragraph 3, block tables): for sequence b, logical token t is read from
+// physical block table[b][t / bs], offset t % bs.  The
 // attention arithmetic is the textbook decode step with an online softmax;
 // scores are kept in base-2 units (the host folds log2(e) into the scale).
 //

@@ -2,7 +2,7 @@
 
 Facts used ("PagedAttention Internals", "Fixed-Size KV Blocks" and "The
 Block Table Map"; the "pagedattention" glossary entry, comparison table and
-paragraph "It is the core of vLLM ..."): a sequence holds ceil(n / bs) blocks
+paragraph 5, sharing): a sequence holds ceil(n / bs) blocks
 after n tokens; any free block can take the next portion; waste is confined to
 the last block; shared blocks are copied only when a sharer writes them.
 """
