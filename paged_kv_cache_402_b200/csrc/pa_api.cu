@@ -13,6 +13,7 @@
 
 #include "pa_copy_kernels.cuh"
 #include "pa_decode_simt.cuh"
+#include "pa_decode_tc.cuh"
 #include "pagedattn.h"
 
 namespace {
@@ -86,6 +87,90 @@ pa_status launch_decode_d(const pa::DecodeParams &p, int32_t max_parts, cudaStre
     case 2: return launch_decode_t<T, D, 2>(p, max_parts, st);
     case 4: return launch_decode_t<T, D, 4>(p, max_parts, st);
     case 8: return launch_decode_t<T, D, 8>(p, max_parts, st);
+    default: return PA_ERR_UNSUPPORTED;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// tensor-core decode (bf16, head_dim 128, group size <= 8)
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (EncodeTiledFn) nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// A [rows][128] bf16 matrix read in boxes of 64 columns x box_rows rows with
+// 128-byte swizzle (the layout the MMA descriptors expect).
+bool make_map_bf16_d128(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {128, rows};
+  const cuuint64_t strides[1] = {128 * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+bool tc_eligible(const pa::DecodeParams &p, int dtype, int D) {
+  if (dtype != PA_DTYPE_BF16 || D != 128) return false;
+  if (p.G < 1 || p.G > pa::TcLayout::kN || (p.G & (p.G - 1))) return false;
+  if (p.B > pa::TcLayout::kMaxSeqs) return false;
+  if ((int64_t)p.num_blocks * p.Hkv * p.bs >= (int64_t)INT32_MAX) return false;
+  if ((int64_t)p.B * p.Hq >= (int64_t)INT32_MAX) return false;
+  return true;  // a missing tensor-map encoder then fails the launch loudly (PA_ERR_CUDA)
+}
+
+template <int G>
+pa_status launch_decode_tc_g(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
+  CUtensorMap mk, mv, mq;
+  const uint64_t rows = (uint64_t)p.num_blocks * p.Hkv * p.bs;
+  if (!make_map_bf16_d128(&mk, p.k, rows, (uint32_t)p.bs) ||
+      !make_map_bf16_d128(&mv, p.v, rows, (uint32_t)p.bs) ||
+      !make_map_bf16_d128(&mq, p.q, (uint64_t)p.B * p.Hq, (uint32_t)G))
+    return PA_ERR_CUDA;
+  auto kern = pa::decode_partition_tc<G>;
+  const int smem = pa::TcLayout::kBytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return PA_ERR_CUDA;
+  const int64_t units_bound = (int64_t)p.Hkv * p.B * max_parts;
+  int grid = sm_count();
+  if (grid <= 0) return PA_ERR_CUDA;
+  if (units_bound < grid) grid = (int)units_bound;
+  kern<<<grid, pa::TcLayout::kThreads, smem, st>>>(mk, mv, mq, p);
+  pa_status s = launch_status();
+  if (s != PA_OK || max_parts <= 1) return s;
+  pa::decode_reduce<__nv_bfloat16, 128>
+      <<<p.B * p.Hq, 128, (size_t)max_parts * sizeof(float), st>>>(p);
+  return launch_status();
+}
+
+pa_status launch_decode_tc(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
+  switch (p.G) {
+    case 1: return launch_decode_tc_g<1>(p, max_parts, st);
+    case 2: return launch_decode_tc_g<2>(p, max_parts, st);
+    case 4: return launch_decode_tc_g<4>(p, max_parts, st);
+    case 8: return launch_decode_tc_g<8>(p, max_parts, st);
     default: return PA_ERR_UNSUPPORTED;
   }
 }
@@ -226,6 +311,7 @@ PA_API pa_status pa_decode(const void *q, const pa_cache_t *cache, const int32_t
   p.max_parts = max_parts;
   p.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t st = (cudaStream_t)stream;
+  if (tc_eligible(p, cache->dtype, cache->head_dim)) return launch_decode_tc(p, max_parts, st);
   if (cache->dtype == PA_DTYPE_F32) return launch_decode_dtype<float>(p, cache->head_dim, max_parts, st);
   return launch_decode_dtype<__nv_bfloat16>(p, cache->head_dim, max_parts, st);
 }

@@ -1,0 +1,499 @@
+// Paged decode attention on the 5th-generation tensor cores (bf16, head_dim
+// 128, group size 1..8): the split-context partition kernel.
+//
+// What it computes is what decode_partition_simt computes (see there for the
+// pages it follows): for every (sequence b, kv head g, 512-token partition p)
+// it reads keys and values through the block table, scores all G query heads
+// of the group at once, runs an online softmax in base-2 units and writes
+// either the final output (single-partition sequences) or the partition's
+// (max, sum, unnormalised accumulator) for the log-sum-exp reduce.
+//
+// How, on sm_100a:
+//  * Persistent grid, one CTA per SM; the CTA walks the dense list of real
+//    work units (prefix sums of the partition counts in shared memory) in
+//    round-robin order.
+//  * Warp 0 (one lane) is the TMA producer.  A unit is cut into chunks of 128
+//    tokens; for every block of a chunk it loads the (block, kv head) K tile
+//    and V tile as two 64-column boxes with 128-byte swizzle into a 3-slot K
+//    ring and a 3-slot V ring (32 KiB per slot).  Missing blocks (past the
+//    partition, or a table entry outside the pool) are loaded from rows past
+//    the end of the tensor, which the TMA fills with zeros.
+//  * Warp 1 (one lane) issues tcgen05 MMAs: per chunk c,
+//        S^T[128 tok x 16] = K_c[128 tok x 128 d] . Q^T[128 d x 16]   (K-major A and B)
+//        O^T[128 d x 16]   = V_c^T[128 d x 128 tok] . P^T[128 tok x 16] (MN-major A)
+//    with accumulators in tensor memory (S and O double-buffered); the query
+//    rows past G are zero (N = 16 is the smallest N an M = 128 MMA takes).  QK of chunk c is issued before PV of chunk c-1.
+//  * Warps 2..5 (128 threads) run the softmax on S (thread = token row) and
+//    write P^T in bf16 to shared memory, then merge O of the previous chunk
+//    into fp32 registers (thread = head-dim row), one chunk behind, so the PV
+//    MMA overlaps the next softmax.
+//  * Every mbarrier wait has an iteration limit; a thread that gives up sets
+//    PA_DEVERR_TIMEOUT and its role stops, the softmax warps leave together
+//    through a reducing barrier, the MMA lane drains its MMAs, and the CTA
+//    frees its tensor memory before returning.
+#pragma once
+
+#include "pa_decode_simt.cuh"
+#include "pa_tc.cuh"
+
+namespace pa {
+
+struct TcLayout {
+  static constexpr int kN = 16;             // MMA N: query heads of a group, zero-padded
+                                            // (M = 128 takes N in multiples of 16)
+  static constexpr int kChunk = 128;        // tokens per MMA chunk (= M)
+  static constexpr int kStages = 3;
+  static constexpr int kHalf = kChunk * 128;  // one 64-dim half of a chunk: 128 rows x 128 B
+  static constexpr int kTile = 2 * kHalf;     // 32 KiB
+  static constexpr int kQ = 2 * kN * 128;     // two halves of kN rows x 128 B
+  static constexpr int kP = 2 * kN * 128;     // two 64-token halves of kN rows x 128 B
+  static constexpr int kMaxSeqs = 2048;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kStages * kTile;
+  static constexpr int kOffQ = kOffV + kStages * kTile;
+  static constexpr int kOffP = kOffQ + 2 * kQ;
+  static constexpr int kOffBar = kOffP + 2 * kP;
+  static constexpr int kNumBars = 25;
+  static constexpr int kOffRed = kOffBar + kNumBars * 8;
+  static constexpr int kRedFloats = 2 * 4 * kN;  // [parity][warp][head]
+  static constexpr int kOffRedSum = kOffRed + kRedFloats * 4;
+  static constexpr int kOffTmem = kOffRedSum + kRedFloats * 4;
+  static constexpr int kOffScan = kOffTmem + 16;  // 8 ints
+  static constexpr int kOffPrefix = kOffScan + 32;
+  static constexpr int kBytes = kOffPrefix + (kMaxSeqs + 1) * 4 + 1024;  // + base alignment slack
+  static constexpr int kThreads = 192;
+  static constexpr uint32_t kTmemCols = 64;  // S0 S1 O0 O1, kN columns each
+};
+
+struct TcUnit {
+  int b, g, part, t0, t1, nchunks;
+  bool single;
+};
+
+__device__ __forceinline__ TcUnit tc_unit_at(const DecodeParams &p, const int32_t *prefix, int u) {
+  TcUnit un;
+  const int w = u / p.Hkv;
+  un.g = u - w * p.Hkv;
+  int lo = 0, hi = p.B - 1;  // largest b with prefix[b] <= w
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= w) lo = mid; else hi = mid - 1;
+  }
+  un.b = lo;
+  un.part = w - prefix[lo];
+  const int ctx = p.lens[lo];
+  un.t0 = un.part * kPart;
+  un.t1 = min(un.t0 + kPart, ctx);
+  un.nchunks = (un.t1 - un.t0 + TcLayout::kChunk - 1) / TcLayout::kChunk;
+  un.single = ctx <= kPart;
+  return un;
+}
+
+// OR of `pred` over the 128 softmax threads (named barrier 1).
+__device__ __forceinline__ bool wg_sync_or(int pred) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred)
+      : "memory");
+  return r != 0;
+}
+
+template <int G>
+__global__ void __launch_bounds__(TcLayout::kThreads, 1)
+    decode_partition_tc(const __grid_constant__ CUtensorMap tmap_k,
+                        const __grid_constant__ CUtensorMap tmap_v,
+                        const __grid_constant__ CUtensorMap tmap_q, DecodeParams p) {
+  using L = TcLayout;
+  constexpr int N = L::kN;
+  static_assert(G >= 1 && G <= N, "group size");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
+  uint64_t *kfull = bars, *kempty = bars + 3, *vfull = bars + 6, *vempty = bars + 9;
+  uint64_t *qfull = bars + 12, *qempty = bars + 14, *sfull = bars + 16, *pfull = bars + 18;
+  uint64_t *ofull = bars + 20, *ofree = bars + 22, *drain = bars + 24;
+  int32_t *prefix = reinterpret_cast<int32_t *>(smem + L::kOffPrefix);
+  int32_t *scan = reinterpret_cast<int32_t *>(smem + L::kOffScan);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffTmem);
+  float *red_max = reinterpret_cast<float *>(smem + L::kOffRed);
+  float *red_sum = reinterpret_cast<float *>(smem + L::kOffRedSum);
+  __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(p.out);
+
+  // ---------------------------------------------------------------- set-up
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&kfull[i], 1);
+      mbar_init(&kempty[i], 1);
+      mbar_init(&vfull[i], 1);
+      mbar_init(&vempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&qfull[i], 1);
+      mbar_init(&qempty[i], 1);
+      mbar_init(&sfull[i], 1);
+      mbar_init(&pfull[i], 128);
+      mbar_init(&ofull[i], 1);
+      mbar_init(&ofree[i], 128);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  // Q rows past G and unused P rows stay zero for the whole kernel
+  for (int i = threadIdx.x; i < (2 * L::kQ + 2 * L::kP) / 16; i += blockDim.x)
+    reinterpret_cast<uint4 *>(smem + L::kOffQ)[i] = make_uint4(0, 0, 0, 0);
+
+  // partition counts of every sequence and their exclusive prefix sums
+  const int B = p.B;
+  constexpr int kMaxSeg = (L::kMaxSeqs + L::kThreads - 1) / L::kThreads;
+  const int seg = (B + blockDim.x - 1) / blockDim.x;
+  const int b_first = threadIdx.x * seg;
+  int cnt[kMaxSeg];
+  int mine = 0;
+#pragma unroll
+  for (int i = 0; i < kMaxSeg; ++i) {
+    cnt[i] = 0;
+    const int b = b_first + i;
+    if (i < seg && b < B) {
+      const int ctx = p.lens[b];
+      const bool ok = ctx >= 0 && ctx <= p.max_ctx;
+      cnt[i] = (ok && ctx > 0) ? (ctx + kPart - 1) / kPart : 0;
+      mine += cnt[i];
+      if (blockIdx.x == 0 && (!ok || ctx == 0)) {  // rows no unit writes: zero them
+        if (!ok) raise_error(PA_DEVERR_LEN);
+        uint4 *o = reinterpret_cast<uint4 *>(out + (size_t)b * p.Hq * 128);
+        for (int e = 0; e < p.Hq * 128 / 8; ++e) o[e] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
+  int incl = mine;  // inclusive scan within the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) scan[warp] = incl;
+  if (warp == 1) tc::tmem_alloc(tmem_slot, L::kTmemCols);
+  __syncthreads();
+  int run = incl - mine;
+  for (int w = 0; w < warp; ++w) run += scan[w];
+#pragma unroll
+  for (int i = 0; i < kMaxSeg; ++i) {
+    const int b = b_first + i;
+    if (i < seg && b < B) {
+      prefix[b] = run;
+      run += cnt[i];
+      if (b == B - 1) prefix[B] = run;
+    }
+  }
+  if (warp == 1) tc::tmem_relinquish();
+  fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int num_units = p.Hkv * prefix[B];
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tc::prefetch_tensormap(&tmap_k);
+      tc::prefetch_tensormap(&tmap_v);
+      tc::prefetch_tensormap(&tmap_q);
+      const uint64_t pol_kv = policy_evict_first();
+      const uint64_t pol_q = tc::policy_evict_last();
+      const int bs = p.bs;
+      const int blocks_per_chunk = L::kChunk / bs;
+      const int oob_row = p.num_blocks * p.Hkv * bs;  // first row past the pool
+      int c = 0, qi = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        const TcUnit un = tc_unit_at(p, prefix, u);
+        const int32_t *trow = p.tables + (size_t)un.b * p.max_blocks;
+        const int qs = qi & 1;
+        if (!mbar_wait(&qempty[qs], ((qi >> 1) & 1) ^ 1)) { ok = false; break; }
+        mbar_arrive_expect_tx(&qfull[qs], 2 * G * 128);
+        uint8_t *qdst = smem + L::kOffQ + qs * L::kQ;
+        const int qy = un.b * p.Hq + un.g * G;
+        tc::tma_load_2d(qdst, &tmap_q, 0, qy, &qfull[qs], pol_q);
+        tc::tma_load_2d(qdst + N * 128, &tmap_q, 64, qy, &qfull[qs], pol_q);
+        ++qi;
+        for (int ci = 0; ci < un.nchunks; ++ci, ++c) {
+          const int slot = c % 3, use = c / 3;
+          const int jb0 = (un.t0 + ci * L::kChunk) / bs;
+          for (int which = 0; which < 2; ++which) {  // 0: K ring, 1: V ring
+            uint64_t *empty = which ? &vempty[slot] : &kempty[slot];
+            uint64_t *full = which ? &vfull[slot] : &kfull[slot];
+            const CUtensorMap *map = which ? &tmap_v : &tmap_k;
+            if (!mbar_wait(empty, (use & 1) ^ 1)) { ok = false; break; }
+            mbar_arrive_expect_tx(full, L::kTile);
+            uint8_t *dst = smem + (which ? L::kOffV : L::kOffK) + slot * L::kTile;
+            for (int jl = 0; jl < blocks_per_chunk; ++jl) {
+              const int jb = jb0 + jl;
+              int y = oob_row;
+              if (jb * bs < un.t1) {
+                const int32_t blk = trow[jb];
+                if (blk >= 0 && blk < p.num_blocks) y = (blk * p.Hkv + un.g) * bs;
+                else if (which == 0) raise_error(PA_DEVERR_TABLE);
+              }
+              tc::tma_load_2d(dst + jl * bs * 128, map, 0, y, full, pol_kv);
+              tc::tma_load_2d(dst + L::kHalf + jl * bs * 128, map, 64, y, full, pol_kv);
+            }
+          }
+          if (!ok) break;
+        }
+      }
+      if (!ok) {
+        raise_error(PA_DEVERR_TIMEOUT);
+        // wait (bounded) for the copies that may still be in flight
+        for (int k = (c > 3 ? c - 3 : 0); k <= c; ++k) {
+          mbar_wait(&kfull[k % 3], (k / 3) & 1, 100000000ull);
+          mbar_wait(&vfull[k % 3], (k / 3) & 1, 100000000ull);
+        }
+        for (int k = (qi > 2 ? qi - 2 : 0); k < qi; ++k) mbar_wait(&qfull[k & 1], (k >> 1) & 1, 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(128, N, false, false);
+      constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(128, N, true, false);
+      const uint32_t kbase0 = smem_u32(smem + L::kOffK), vbase0 = smem_u32(smem + L::kOffV);
+      const uint32_t qbase0 = smem_u32(smem + L::kOffQ), pbase0 = smem_u32(smem + L::kOffP);
+      bool ok = true;
+      auto issue_pv = [&](int c) -> bool {
+        if (!mbar_wait(&pfull[c & 1], (c >> 1) & 1)) return false;
+        if (!mbar_wait(&vfull[c % 3], (c / 3) & 1)) return false;
+        if (!mbar_wait(&ofree[c & 1], ((c >> 1) & 1) ^ 1)) return false;
+        tc::fence_after_sync();
+        const uint32_t vb = vbase0 + (c % 3) * L::kTile;
+        const uint32_t pb = pbase0 + (c & 1) * L::kP;
+        const uint32_t d = tmem + 2 * N + (c & 1) * N;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          // V^T: M = head dim (two 64-wide halves L::kHalf apart), K = 16 tokens
+          const uint64_t a = tc::smem_desc_sw128(vb + kk * 2048, L::kHalf, 1024);
+          const uint64_t bdesc = tc::smem_desc_sw128(pb + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
+          tc::mma_bf16(d, a, bdesc, idesc_pv, kk > 0);
+        }
+        tc::mma_commit(&ofull[c & 1]);
+        tc::mma_commit(&vempty[c % 3]);
+        return true;
+      };
+      int c = 0, qi = 0, pending = -1;
+      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        const TcUnit un = tc_unit_at(p, prefix, u);
+        const int qs = qi & 1;
+        if (!mbar_wait(&qfull[qs], (qi >> 1) & 1)) { ok = false; break; }
+        const uint32_t qb = qbase0 + qs * L::kQ;
+        for (int ci = 0; ci < un.nchunks; ++ci, ++c) {
+          const int slot = c % 3;
+          if (!mbar_wait(&kfull[slot], (c / 3) & 1)) { ok = false; break; }
+          tc::fence_after_sync();
+          const uint32_t kb = kbase0 + slot * L::kTile;
+          const uint32_t d = tmem + (c & 1) * N;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t koff = (kk >> 2) * L::kHalf + (kk & 3) * 32;
+            const uint64_t a = tc::smem_desc_sw128(kb + koff, 16, 1024);
+            const uint64_t bdesc = tc::smem_desc_sw128(qb + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
+            tc::mma_bf16(d, a, bdesc, idesc_qk, kk > 0);
+          }
+          tc::mma_commit(&sfull[c & 1]);
+          tc::mma_commit(&kempty[slot]);
+          if (ci == un.nchunks - 1) tc::mma_commit(&qempty[qs]);
+          if (pending >= 0 && !issue_pv(pending)) { ok = false; break; }
+          pending = c;
+        }
+        ++qi;
+      }
+      if (ok && pending >= 0 && !issue_pv(pending)) ok = false;
+      if (!ok) raise_error(PA_DEVERR_TIMEOUT);
+      // no MMA may still be running when the CTA frees its tensor memory
+      tc::mma_commit(drain);
+      mbar_wait(drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + merge
+    const int wq = warp & 3;              // this warp's quarter of the TMEM lanes
+    const int r = wq * 32 + lane;         // token row (softmax) / head-dim row (merge)
+    const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
+    const int bs = p.bs;
+    float m[G], l[G], acc[G], m_done[G], l_done[G], alpha_p[G];
+#pragma unroll
+    for (int n = 0; n < G; ++n) {
+      m[n] = -INFINITY;
+      l[n] = 0.f;
+      acc[n] = 0.f;
+      m_done[n] = -INFINITY;
+      l_done[n] = 0.f;
+      alpha_p[n] = 1.f;
+    }
+    TcUnit pun{};
+    bool pend = false, p_first = false, p_last = false;
+    int pc = 0, nunit = 0;
+    bool bad = false;   // this thread gave up on a wait
+    bool stop = false;  // some thread of the warpgroup did (uniform: from wg_sync_or)
+
+    auto epilogue = [&](const TcUnit &un, int parity) {
+      // L[n]: sum of the per-row partial sums over the 128 threads
+      float Ls[G];
+#pragma unroll
+      for (int n = 0; n < G; ++n) {
+        float v = l_done[n];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) red_sum[(parity * 4 + wq) * N + n] = v;
+      }
+      stop = wg_sync_or(bad);
+      if (stop) return;
+#pragma unroll
+      for (int n = 0; n < G; ++n) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) sum += red_sum[(parity * 4 + w) * N + n];
+        Ls[n] = sum;
+      }
+#pragma unroll
+      for (int n = 0; n < G; ++n) {
+        const int h = un.g * G + n;
+        if (un.single) {
+          out[((size_t)un.b * p.Hq + h) * 128 + r] = __float2bfloat16_rn(Ls[n] > 0.f ? acc[n] / Ls[n] : 0.f);
+        } else {
+          const size_t row = ((size_t)un.b * p.Hq + h) * p.max_parts + un.part;
+          p.ws_acc[row * 128 + r] = acc[n];
+          if (r == 0) {
+            p.ws_m[row] = m_done[n];
+            p.ws_l[row] = Ls[n];
+          }
+        }
+      }
+    };
+
+    // O of chunk pc into acc (one chunk behind the softmax), then the
+    // epilogue when pc ended its unit.  A failed wait only marks `bad`; the
+    // next warpgroup barrier turns it into a uniform stop.
+    auto merge = [&]() {
+      float o[8];
+      if (!bad && !mbar_wait(&ofull[pc & 1], (pc >> 1) & 1)) bad = true;
+      if (!bad) {
+        tc::fence_after_sync();
+        tc::tmem_ld8(trow + 2 * N + (pc & 1) * N, o);
+#pragma unroll
+        for (int n = 0; n < G; ++n) acc[n] = p_first ? o[n] : fmaf(acc[n], alpha_p[n], o[n]);
+      }
+      tc::fence_before_sync();
+      mbar_arrive(&ofree[pc & 1]);
+      if (p_last) epilogue(pun, nunit & 1);
+    };
+
+    int c = 0;
+    for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x) {
+      const TcUnit un = tc_unit_at(p, prefix, u);
+      const int32_t *tabrow = p.tables + (size_t)un.b * p.max_blocks;
+      const int tail_end = min(((un.t1 + bs - 1) / bs) * bs, un.t0 + kPart);
+#pragma unroll
+      for (int n = 0; n < G; ++n) {
+        m_done[n] = m[n];
+        l_done[n] = l[n];
+        m[n] = -INFINITY;
+        l[n] = 0.f;
+      }
+      for (int ci = 0; ci < un.nchunks; ++ci, ++c) {
+        // ---- softmax of chunk c
+        float s[8];
+        if (!bad && !mbar_wait(&sfull[c & 1], (c >> 1) & 1)) bad = true;
+        if (!bad) {
+          tc::fence_after_sync();
+          tc::tmem_ld8(trow + (c & 1) * N, s);
+        }
+        const int tok = un.t0 + ci * L::kChunk + r;
+        bool valid = tok < un.t1;
+        if (valid) {
+          const int32_t blk = tabrow[tok / bs];
+          valid = blk >= 0 && blk < p.num_blocks;
+        }
+        float x[G];
+#pragma unroll
+        for (int n = 0; n < G; ++n) {
+          x[n] = (valid && !bad) ? s[n] * p.scale_log2 : -INFINITY;
+          float v = x[n];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+          if (lane == 0) red_max[((c & 1) * 4 + wq) * N + n] = v;
+        }
+        // a masked row inside the partition's last, partly filled block holds
+        // whatever the pool has there: zero its V row before PV reads it
+        if (!bad && tok >= un.t1 && tok < tail_end) {
+          if (!mbar_wait(&vfull[c % 3], (c / 3) & 1)) {
+            bad = true;
+          } else {
+            uint4 *vr = reinterpret_cast<uint4 *>(smem + L::kOffV + (c % 3) * L::kTile + r * 128);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              vr[e] = make_uint4(0, 0, 0, 0);
+              vr[L::kHalf / 16 + e] = make_uint4(0, 0, 0, 0);
+            }
+          }
+        }
+        stop = wg_sync_or(bad);
+        if (stop) break;
+        float alpha[G];
+        __nv_bfloat16 *pb = reinterpret_cast<__nv_bfloat16 *>(smem + L::kOffP + (c & 1) * L::kP);
+        const int kh = r >> 6, rr = r & 63;
+#pragma unroll
+        for (int n = 0; n < G; ++n) {
+          float cm = red_max[((c & 1) * 4 + 0) * N + n];
+#pragma unroll
+          for (int w = 1; w < 4; ++w) cm = fmaxf(cm, red_max[((c & 1) * 4 + w) * N + n]);
+          const float mnew = fmaxf(m[n], cm);
+          alpha[n] = (mnew == -INFINITY) ? 1.f : exp2f(m[n] - mnew);
+          const float pv = valid ? exp2f(x[n] - mnew) : 0.f;
+          l[n] = fmaf(l[n], alpha[n], pv);
+          m[n] = mnew;
+          // P^T row n (K-major, 128-byte swizzle): token r in half kh
+          const int off = kh * (N * 64) + (n >> 3) * 512 + (n & 7) * 64 + (((rr >> 3) ^ (n & 7)) << 3) + (rr & 7);
+          pb[off] = __float2bfloat16_rn(pv);
+        }
+        fence_proxy_async_smem();
+        tc::fence_before_sync();
+        mbar_arrive(&pfull[c & 1]);
+        // ---- merge of chunk c-1
+        if (pend) {
+          merge();
+          if (stop) break;
+        }
+        pend = true;
+        p_first = ci == 0;
+        p_last = ci == un.nchunks - 1;
+        pun = un;
+        pc = c;
+        if (p_last) ++nunit;
+#pragma unroll
+        for (int n = 0; n < G; ++n) alpha_p[n] = alpha[n];
+      }
+    }
+    if (pend && !stop) {
+#pragma unroll
+      for (int n = 0; n < G; ++n) {
+        m_done[n] = m[n];
+        l_done[n] = l[n];
+      }
+      merge();
+    }
+    if (stop) raise_error(PA_DEVERR_TIMEOUT);
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 1) tc::tmem_dealloc(tmem, L::kTmemCols);
+}
+
+}  // namespace pa

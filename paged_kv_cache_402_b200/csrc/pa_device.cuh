@@ -41,13 +41,26 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Default limit of one mbarrier wait: a copy or MMA this library issued from
+// valid memory completes in microseconds, so a wait this long means something
+// is broken and the kernel should give up rather than hang.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
 // Waits for the phase of parity `parity` to complete.  Gives up after
-// `max_tries` polls and returns false (the caller records PA_DEVERR_TIMEOUT
-// and drops its work); a copy from valid memory always completes long before.
+// `limit_ns` nanoseconds of %globaltimer time and returns false (the caller
+// records PA_DEVERR_TIMEOUT and drops its work).  try_wait may itself suspend
+// the thread for a while, so the bound is on time, not on polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
-                                          uint32_t max_tries = (1u << 24)) {
+                                          uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t addr = smem_u32(bar);
-  for (uint32_t i = 0; i < max_tries; ++i) {
+  uint64_t start = 0;
+  for (uint32_t i = 0;; ++i) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -57,8 +70,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
         : "r"(addr), "r"(parity)
         : "memory");
     if (done) return true;
+    if (i == 0) {
+      start = global_ns();
+    } else if ((i & 63) == 0 && global_ns() - start > limit_ns) {
+      return false;
+    }
   }
-  return false;
 }
 
 // Makes this thread's earlier generic-proxy shared-memory accesses ordered

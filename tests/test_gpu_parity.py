@@ -340,3 +340,52 @@ def test_full_step_shared_prefix_cow(cuda_device):
     for b, (sk, sv) in snap.items():
         assert same_bits(gk[b], sk) and same_bits(gv[b], sv)
     assert_attn_close(out, ref, dt)
+
+
+# ------------------------------------------------------------- bf16 / head_dim 128 specifics
+
+
+def test_bf16_context_one_is_exact(cuda_device):
+    """ctx = 1: the single weight is exactly 1, so the output is the value
+    row itself, bit for bit (bf16, head_dim 128)."""
+    case = synth.random_case(46, B=3, Hq=8, Hkv=2, D=128, bs=16, lens=[1, 0, 1], dtype=torch.bfloat16)
+    out = decode_case(case, cuda_device).cpu()
+    assert torch.equal(out[1], torch.zeros_like(out[1]))
+    for b in (0, 2):
+        blk = int(case.block_tables[b, 0])
+        for h in range(8):
+            assert torch.equal(out[b, h], case.v_cache[blk, h // 4, 0])
+
+
+@pytest.mark.parametrize("B", [300, 2100])
+def test_many_sequences(cuda_device, B):
+    """More sequences than one thread's share of the in-kernel prefix sums
+    (300), and more than the tensor-core kernel keeps in shared memory
+    (2100); lengths include zeros and several partitions."""
+    lens = synth.rng(47 + B).integers(0, 1300 if B < 1000 else 80, size=B).astype(np.int32)
+    case = synth.random_case(47, B=B, Hq=8, Hkv=2, D=128, bs=16, lens=lens, dtype=torch.bfloat16)
+    out = decode_case(case, cuda_device)
+    ref = oracle.decode(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens, case.scale)
+    assert_attn_close(out, ref, torch.bfloat16)
+
+
+def test_bf16_device_errors(cuda_device):
+    """A table entry outside the pool and a length past max_context_len on
+    the bf16 head_dim-128 path: reported in the error word, no trap; the
+    other sequences are still right."""
+    lens = [700, 40, 1300]
+    case = synth.random_case(48, B=3, Hq=8, Hkv=2, D=128, bs=16, lens=lens, dtype=torch.bfloat16)
+    cache, q, tables, lens_d = to_dev(case, cuda_device)
+    bad = tables.clone()
+    bad[0, 3] = case.num_blocks + 5
+    out = pa.pa_decode(q, cache, bad, lens_d, 1300, case.scale)
+    assert pa.pa_read_device_error() & pa.PA_DEVERR_TABLE
+    ref = oracle.decode(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens, case.scale)
+    assert_attn_close(out[1:], ref[1:], torch.bfloat16)
+    lens_bad = lens_d.clone()
+    lens_bad[1] = 5000
+    out = pa.pa_decode(q, cache, tables, lens_bad, 1300, case.scale)
+    assert pa.pa_read_device_error() == pa.PA_DEVERR_LEN
+    assert torch.equal(out[1].float().cpu(), torch.zeros(8, 128))
+    assert_attn_close(out[[0, 2]], ref[[0, 2]], torch.bfloat16)
+    assert pa.pa_read_device_error() == 0
