@@ -150,62 +150,183 @@ class ClockSampler:
 # ----------------------------------------------------------------- workload
 
 
-class Instance:
-    """One independent batch: pool, allocator, sequences, and per-step inputs
-    (slots, copy pairs, tables, lengths, q and new rows) for `uses` steps."""
+def _fill_blocks_normal(cache, blocks, seed, dev, chunk=65536):
+    """N(0,1) bf16 values in the listed pool blocks only (a pool much larger
+    than what the batch uses is never read anywhere else)."""
+    from paged_kv_cache_402_b200 import synth
+    idx = torch.as_tensor(np.asarray(blocks, dtype=np.int64), device=dev)
+    shape = tuple(cache.k.shape[1:])
+    for i in range(0, len(idx), chunk):
+        part = idx[i:i + chunk]
+        cache.k.index_copy_(0, part, synth.normal((len(part),) + shape, torch.bfloat16, seed * 7919 + i, device=dev))
+        cache.v.index_copy_(0, part, synth.normal((len(part),) + shape, torch.bfloat16, seed * 7919 + i + 1, device=dev))
 
-    def __init__(self, seed: int, wl: dict, uses: int, dev, pin: bool = True):
+
+def setup_independent(seed, wl, uses, dev):
+    """Sequences of the workload's lengths; the pool is dealt from a seeded
+    shuffle of all its blocks (pool_factor x the needed blocks, or a fixed
+    pool size)."""
+    import paged_kv_cache_402_b200 as pa
+    from paged_kv_cache_402_b200 import synth
+    B, Hkv, D, bs = wl["B"], wl["Hkv"], wl["D"], wl["bs"]
+    lens = wl["lengths"](seed)
+    need = int(sum(-(-(int(L) + uses) // bs) for L in lens))
+    NB = wl.get("num_blocks") or int(math.ceil(need * wl.get("pool_factor", 2.0))) + 1
+    order = synth.rng(seed + 1).permutation(NB)
+    alloc = pa.Allocator(NB, bs, order)
+    if wl.get("fill_used_only"):
+        cache = pa.KVCache.empty(NB, Hkv, bs, D, torch.bfloat16, dev)
+        _fill_blocks_normal(cache, order[:need], seed, dev)
+    else:
+        cache = pa.KVCache(synth.normal((NB, Hkv, bs, D), torch.bfloat16, seed + 2, device=dev),
+                           synth.normal((NB, Hkv, bs, D), torch.bfloat16, seed + 3, device=dev))
+    seqs = [alloc.new_seq() for _ in range(B)]
+    alloc.batch_append(seqs, lens)  # prompt blocks; the pool's contents stand in for the prompt rows
+    return alloc, cache, [seqs]
+
+
+def setup_shared_prefix(seed, wl, uses, dev):
+    """Groups of 8 that share the blocks of a 512 + r token prefix (r in
+    [1, 15], so the prefix ends inside a shared block); each member then
+    appends its own lognormal suffix, which makes 7 members per group copy
+    that block (the copies are made on the device here, in set-up)."""
+    import paged_kv_cache_402_b200 as pa
+    from paged_kv_cache_402_b200 import synth
+    Hkv, D, bs, gsz = wl["Hkv"], wl["D"], wl["bs"], wl["group_size"]
+    groups = wl["B"] // gsz
+    pl, suffix, order, NB = synth.shared_prefix_layout(seed, groups=groups, group_size=gsz, prefix=512,
+                                                       median=800, clip=8192, bs=bs, pool_factor=1.25,
+                                                       prefix_tail=True)
+    NB += wl["B"] * (-(-uses // bs) + 1)
+    order = np.concatenate([order, np.arange(len(order), NB)]).astype(np.int32)
+    alloc = pa.Allocator(NB, bs, order)
+    cache = pa.KVCache(synth.normal((NB, Hkv, bs, D), torch.bfloat16, seed + 2, device=dev),
+                       synth.normal((NB, Hkv, bs, D), torch.bfloat16, seed + 3, device=dev))
+    roots = [alloc.new_seq() for _ in range(groups)]
+    alloc.batch_append(roots, pl)
+    seqs = []
+    for r in roots:
+        seqs += [r] + [alloc.fork(r) for _ in range(gsz - 1)]
+    _, pairs = alloc.batch_append(seqs, suffix)
+    if len(pairs):
+        pa.pa_copy_blocks(torch.from_numpy(np.ascontiguousarray(pairs)).to(dev), cache)
+    return alloc, cache, [seqs]
+
+
+def setup_cow_steps(seed, wl, uses, dev):
+    """One fresh set of groups per step: each group's 8 members share a
+    512 + r token prefix that ends inside a block, so the step's append of
+    one token to every member copies that block for 7 of them."""
+    import paged_kv_cache_402_b200 as pa
+    from paged_kv_cache_402_b200 import synth
+    Hkv, D, bs, gsz = wl["Hkv"], wl["D"], wl["bs"], wl["group_size"]
+    groups = wl["B"] // gsz
+    per_set = groups * (-(-(512 + bs) // bs) + gsz)
+    NB = uses * per_set + 1
+    order = synth.rng(seed + 1).permutation(NB)
+    alloc = pa.Allocator(NB, bs, order)
+    cache = pa.KVCache(synth.normal((NB, Hkv, bs, D), torch.bfloat16, seed + 2, device=dev),
+                       synth.normal((NB, Hkv, bs, D), torch.bfloat16, seed + 3, device=dev))
+    r = synth.rng(seed + 5)
+    sets = []
+    for _ in range(uses):
+        roots = [alloc.new_seq() for _ in range(groups)]
+        alloc.batch_append(roots, 512 + r.integers(1, bs, size=groups))
+        seqs = []
+        for root in roots:
+            seqs += [root] + [alloc.fork(root) for _ in range(gsz - 1)]
+        sets.append(seqs)
+    return alloc, cache, sets
+
+
+class Instance:
+    """One independent workload instance: pool, allocator, sequences, and the
+    inputs of `uses` steps (slots, copy pairs, tables, lengths, q and new
+    rows), all made before any timing."""
+
+    def __init__(self, seed: int, wl: dict, uses: int, dev, extra: int = 0):
         import paged_kv_cache_402_b200 as pa
         from paged_kv_cache_402_b200 import synth
 
         self.wl = wl
         B, Hq, Hkv, D, bs = wl["B"], wl["Hq"], wl["Hkv"], wl["D"], wl["bs"]
         dt = torch.bfloat16
-        self.lens0 = wl["lengths"](seed)
-        need = int(sum(-(-(int(L) + uses) // bs) for L in self.lens0))
-        NB = int(math.ceil(need * wl.get("pool_factor", 2.0))) + 1
-        order = synth.rng(seed + 1).permutation(NB)
-        self.alloc = pa.Allocator(NB, bs, order)
-        self.cache = pa.KVCache(synth.normal((NB, Hkv, bs, D), dt, seed + 2, device=dev),
-                                synth.normal((NB, Hkv, bs, D), dt, seed + 3, device=dev))
         t0 = time.perf_counter()
-        self.seqs = [self.alloc.new_seq() for _ in range(B)]
-        self.alloc.batch_append(self.seqs, self.lens0)  # prompt blocks; the pool's contents stand in for them
-        self.max_blocks = int(-(-(int(self.lens0.max()) + uses) // bs))
+        self.alloc, self.cache, self.sets = wl["setup"](seed, wl, uses + extra, dev)
+        self.uses = uses
+        torch.cuda.synchronize()
+        self.setup_s = time.perf_counter() - t0
+        lens_now = [self.alloc.seq_len(q)[0] for q in self.sets[0]]
+        self.lens0 = np.array(lens_now, dtype=np.int32)
+        self.max_blocks = int(-(-(int(max(max(self.alloc.seq_len(q)[0] for q in st) for st in self.sets))
+                                  + uses + extra + 1) // bs))
         self.steps = []
         self.host_alloc_s = 0.0
+        row_bytes = 2 * Hkv * D * 2
         for u in range(uses):
+            seqs = self.sets[u % len(self.sets)]
             t1 = time.perf_counter()
-            slots, pairs = self.alloc.batch_append(self.seqs, np.ones(B, np.int32))
-            tables, lens = self.alloc.build_block_tables(self.seqs, self.max_blocks)
+            slots, pairs = self.alloc.batch_append(seqs, np.ones(B, np.int32))
+            tables, lens = self.alloc.build_block_tables(seqs, self.max_blocks)
             self.host_alloc_s += time.perf_counter() - t1
+            nblk = (lens.astype(np.int64) + bs - 1) // bs
+            # unique bytes: every physical block once, with its fill
+            fill = {}
+            for i in range(B):
+                for j in range(int(nblk[i])):
+                    fill.setdefault(int(tables[i, j]), min(bs, int(lens[i]) - j * bs))
             st = {
+                "seqs": seqs,
                 "slots": torch.from_numpy(slots.copy()).to(dev),
                 "pairs": torch.from_numpy(np.ascontiguousarray(pairs)).to(dev) if len(pairs) else None,
+                "n_pairs": len(pairs),
                 "tables": torch.from_numpy(tables).to(dev),
                 "lens": torch.from_numpy(lens).to(dev),
                 "max_ctx": int(lens.max()),
-                "kv_bytes": int(lens.astype(np.int64).sum()) * 2 * Hkv * D * 2,
+                "kv_bytes": int(lens.astype(np.int64).sum()) * row_bytes,
+                "kv_unique_bytes": int(sum(fill.values())) * row_bytes,
                 "q": synth.normal((B, Hq, D), dt, seed * 1000 + 10 + 3 * u, device=dev),
                 "k": synth.normal((B, Hkv, D), dt, seed * 1000 + 11 + 3 * u, device=dev),
                 "v": synth.normal((B, Hkv, D), dt, seed * 1000 + 12 + 3 * u, device=dev),
             }
-            st["ws"] = torch.empty(max(16, pa.pa_decode_workspace_size(B, Hq, st["max_ctx"], D)),
-                                   dtype=torch.uint8, device=dev)
-            st["out"] = torch.empty(B, Hq, D, dtype=dt, device=dev)
-            st["algo_bytes"] = (st["kv_bytes"] + 2 * B * Hq * D * 2 + B * 4
-                                + int(((lens.astype(np.int64) + bs - 1) // bs).sum()) * 4)
+            st["algo_bytes"] = st["kv_unique_bytes"] + 2 * B * Hq * D * 2 + B * 4 + int(nblk.sum()) * 4
             self.steps.append(st)
-        self.setup_s = time.perf_counter() - t0
+        top = max(st["max_ctx"] for st in self.steps)
+        ws = torch.empty(max(16, pa.pa_decode_workspace_size(B, Hq, top + 64, D)), dtype=torch.uint8, device=dev)
+        out = torch.empty(B, Hq, D, dtype=dt, device=dev)
+        for st in self.steps:
+            st["ws"], st["out"] = ws, out
+
+
+def _lengths(fn_name):
+    def f(seed):
+        from paged_kv_cache_402_b200 import synth
+        return getattr(synth, fn_name)(seed)
+    return f
 
 
 WORKLOADS = {
     "gqa": dict(
         name="bf16 GQA decode: 32 seqs, 32 q / 8 kv heads, head_dim 128, 16-token blocks, "
              "context ~U[128,4096] +1 appended token per step, pool 2x needed (seeded shuffle)",
-        B=32, Hq=32, Hkv=8, D=128, bs=16,
-        lengths=lambda seed: __import__("paged_kv_cache_402_b200.synth", fromlist=["x"]).gqa_lengths(seed),
-        rotate=3),
+        B=32, Hq=32, Hkv=8, D=128, bs=16, lengths=_lengths("gqa_lengths"), setup=setup_independent,
+        rotate=3, max_uses=32),
+    "shared-prefix": dict(
+        name="bf16 shared-prefix decode: 256 seqs in groups of 8 sharing a 512+r token prefix (refcounted "
+             "blocks, copied on write), lognormal suffix median 800 clipped to 8192, 64 q / 8 kv heads, "
+             "head_dim 128, 16-token blocks, +1 token per step",
+        B=256, Hq=64, Hkv=8, D=128, bs=16, group_size=8, setup=setup_shared_prefix, rotate=2, max_uses=32),
+    "long-context": dict(
+        name="bf16 long-context decode: 8 seqs, context ~U[32768,131072], 32 q / 8 kv heads, head_dim 128, "
+             "16-token blocks scattered over an 80 GiB K+V pool, 512-token partitions + LSE reduce, +1 token per step",
+        B=8, Hq=32, Hkv=8, D=128, bs=16, lengths=_lengths("long_context_lengths"), setup=setup_independent,
+        num_blocks=80 * 2**30 // (2 * 8 * 16 * 128 * 2), fill_used_only=True, rotate=1, max_uses=100000),
+    "cow-step": dict(
+        name="bf16 copy-on-write step: 256 seqs in groups of 8 sharing a 512+r token prefix; each step's "
+             "append copies the shared partial block for 7 of 8 members (224 pairs), then decodes; "
+             "64 q / 8 kv heads, head_dim 128, 16-token blocks",
+        B=256, Hq=64, Hkv=8, D=128, bs=16, group_size=8, setup=setup_cow_steps, rotate=1, max_uses=100000,
+        fresh_sets=True),
 }
 
 
@@ -213,10 +334,15 @@ def run_ours(args, rank: int, world: int, dev):
     import paged_kv_cache_402_b200 as pa
 
     wl = WORKLOADS[args.workload]
-    R = args.rotate or wl["rotate"]
     total = args.warmup + args.steps
+    # enough instances that none is used more than max_uses times (each use
+    # grows every sequence by one token)
+    R = args.rotate or max(wl["rotate"], -(-total // wl["max_uses"]))
     uses = -(-total // R)
-    insts = [Instance(1000 * rank + 17 * i + 1, wl, uses, dev) for i in range(R)]
+    # instance 0 keeps room (and, for fresh-set workloads, sets) for the
+    # end-to-end leg's steps
+    insts = [Instance(1000 * rank + 17 * i + 1, wl, uses, dev, extra=args.steps if i == 0 else 0)
+             for i in range(R)]
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
@@ -247,7 +373,9 @@ def run_ours(args, rank: int, world: int, dev):
                   for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches = 0
-    kv_bytes = 0
+    kv_bytes = 0       # distinct physical K/V bytes (what HBM must serve)
+    kv_logical = 0     # per-sequence K/V bytes (shared blocks counted per sharer)
+    pairs = 0
     algo_bytes = []
     if world > 1:
         torch.distributed.barrier()
@@ -257,7 +385,9 @@ def run_ours(args, rank: int, world: int, dev):
         for i in range(args.steps):
             n, st = step(args.warmup + i, dec_events[i])
             launches += n
-            kv_bytes += st["kv_bytes"]
+            kv_bytes += st["kv_unique_bytes"]
+            kv_logical += st["kv_bytes"]
+            pairs += st["n_pairs"]
             algo_bytes.append(st["algo_bytes"])
         t_end.record(stream)
         torch.cuda.synchronize()
@@ -312,6 +442,8 @@ def run_ours(args, rank: int, world: int, dev):
                          f"working set ~{R * kv_bytes / args.steps / 1e6:.0f} MB > 126 MB L2)",
                    "parallelism": f"replicas x{world}"},
         "tokens_per_s": round(tok_all / (ms_all / 1e3), 1),
+        "kv_logical_gbs": round(kv_logical * world / 1e9 / (ms_all / 1e3), 2),
+        "copy_pairs_per_step": round(pairs / args.steps, 2),
         "kv_frac_of_hbm_peak": round(gb_all / (ms_all / 1e3) / peak, 4),
         "kv_frac_of_8tbs_nominal": round(gb_all / (ms_all / 1e3) / NOMINAL_HBM_GBS, 4),
         "host_alloc_us_per_step": round(host_alloc_us, 2),
@@ -330,14 +462,26 @@ def run_ours(args, rank: int, world: int, dev):
     return line
 
 
+def unique_kv_bytes(tables: np.ndarray, lens: np.ndarray, bs: int, row_bytes: int) -> int:
+    """K/V bytes of the distinct physical blocks a batch reads (each block
+    once, with its fill)."""
+    fill = {}
+    for i in range(len(lens)):
+        for j in range(-(-int(lens[i]) // bs)):
+            fill.setdefault(int(tables[i, j]), min(bs, int(lens[i]) - j * bs))
+    return int(sum(fill.values())) * row_bytes
+
+
 def run_e2e(args, insts, wl, dev, stream):
-    """Each step from host memory: allocator call, pinned host -> device copies
-    of the step's inputs, copy / append / decode, device -> host of the output."""
+    """Each step from host memory, through the public API: the allocator
+    call, pinned host -> device copies of the step's inputs (q, new rows,
+    slots, tables, lengths, copy pairs), copy / append / decode, and the
+    device -> host read of the output.  Wall clock, one synchronize per step."""
     import paged_kv_cache_402_b200 as pa
 
-    B, Hq, Hkv, D = wl["B"], wl["Hq"], wl["Hkv"], wl["D"]
+    B, Hq, Hkv, D, bs = wl["B"], wl["Hq"], wl["Hkv"], wl["D"], wl["bs"]
     inst = insts[0]
-    mb = inst.max_blocks + args.steps + args.warmup
+    mb = inst.max_blocks
     h = {
         "q": torch.empty(B, Hq, D, dtype=torch.bfloat16).pin_memory(),
         "k": torch.empty(B, Hkv, D, dtype=torch.bfloat16).pin_memory(),
@@ -354,20 +498,19 @@ def run_e2e(args, insts, wl, dev, stream):
     h["v"].copy_(torch.randn(B, Hkv, D, generator=g).to(torch.bfloat16))
     d = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in h.items() if k != "out"}
     out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
-    # grow capacity: a second, larger pool would be needed for long runs; the
-    # instance pool was sized for warmup + steps uses per instance
-    n_steps = max(1, min(args.steps, len(inst.steps)))
-    ws = torch.empty(max(16, pa.pa_decode_workspace_size(B, Hq, int(inst.lens0.max()) + 2 * mb, D)),
-                     dtype=torch.uint8, device=dev)
+    n_steps = max(1, args.steps)
+    ws = torch.empty(max(16, pa.pa_decode_workspace_size(B, Hq, mb * bs, D)), dtype=torch.uint8, device=dev)
     slots_np, pairs_np = h["slots"].numpy(), h["pairs"].numpy()
     tables_np, lens_np = h["tables"].numpy(), h["lens"].numpy()
-    kv_gb = 0.0
+    ones = np.ones(B, np.int32)
+    seen = []
     h2d = d2h = 0
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     for i in range(n_steps):
-        _, pairs = inst.alloc.batch_append(inst.seqs, np.ones(B, np.int32), out_slots=slots_np, out_pairs=pairs_np)
-        inst.alloc.build_block_tables(inst.seqs, mb, out_tables=tables_np, out_lens=lens_np)
+        seqs = inst.sets[inst.uses + i] if wl.get("fresh_sets") else inst.sets[0]
+        _, pairs = inst.alloc.batch_append(seqs, ones, out_slots=slots_np, out_pairs=pairs_np)
+        inst.alloc.build_block_tables(seqs, mb, out_tables=tables_np, out_lens=lens_np)
         npairs = len(pairs)
         for k in ("q", "k", "v", "slots", "tables", "lens"):
             d[k].copy_(h[k], non_blocking=True)
@@ -375,18 +518,18 @@ def run_e2e(args, insts, wl, dev, stream):
             d["pairs"][:npairs].copy_(h["pairs"][:npairs], non_blocking=True)
             pa.pa_copy_blocks(d["pairs"][:npairs], inst.cache, stream)
         pa.pa_append_kv(d["k"], d["v"], d["slots"], inst.cache, stream)
-        max_ctx = int(lens_np.max())
-        pa.pa_decode(d["q"], inst.cache, d["tables"], d["lens"], max_ctx, 1.0 / math.sqrt(D), out=out,
+        pa.pa_decode(d["q"], inst.cache, d["tables"], d["lens"], int(lens_np.max()), 1.0 / math.sqrt(D), out=out,
                      workspace=ws, stream=stream)
         h["out"].copy_(out, non_blocking=True)
         torch.cuda.synchronize()
-        kv_gb += float(lens_np.astype(np.int64).sum()) * 2 * Hkv * D * 2 / 1e9
         if i == 0:
             h2d = sum(h[k].numel() * h[k].element_size() for k in ("q", "k", "v", "slots", "tables", "lens"))
             h2d += npairs * 8
             d2h = h["out"].numel() * h["out"].element_size()
+        seen.append((tables_np.copy(), lens_np.copy()))
     seconds = time.perf_counter() - t0
-    return {"seconds": seconds, "kv_gb": kv_gb, "steps": n_steps, "h2d": h2d, "d2h": d2h}
+    kv = sum(unique_kv_bytes(t, l, bs, 2 * Hkv * D * 2) for t, l in seen)
+    return {"seconds": seconds, "kv_gb": kv / 1e9, "steps": n_steps, "h2d": h2d, "d2h": d2h}
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -483,8 +626,8 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gqa")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
@@ -511,7 +654,7 @@ def main():
                                              device_id=dev)
     try:
         line = run_ours(args, rank, world, dev)
-        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if rank == 0 and world == 1 and not args.no_cpu_baseline and "lengths" in WORKLOADS[args.workload]:
             wl = WORKLOADS[args.workload]
             gbs, secs, threads, desc = oracle_sample(wl, seed=1, budget_s=args.cpu_budget, min_s=min(5.0, args.cpu_budget))
             line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",

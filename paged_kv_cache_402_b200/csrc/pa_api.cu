@@ -125,6 +125,22 @@ bool make_map_bf16_d128(CUtensorMap *m, const void *base, uint64_t rows, uint32_
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The paged pool [rows][128] bf16 seen as 4-D (64 columns, 8 rows, 2 column
+// halves, 8-row groups) so that one box of (64, 8, 2, bs/8) is a whole
+// (block, kv head) tile and lands as [group][half][8 rows x 128 B] with
+// 128-byte swizzle.
+bool make_map_pool_4d(CUtensorMap *m, const void *base, uint64_t rows, uint32_t bs) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn || rows % 8 || bs % 8) return false;
+  const cuuint64_t dims[4] = {64, 8, 2, rows / 8};
+  const cuuint64_t strides[3] = {256, 128, 2048};
+  const cuuint32_t box[4] = {64, 8, 2, bs / 8};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -134,19 +150,18 @@ int sm_count() {
 
 bool tc_eligible(const pa::DecodeParams &p, int dtype, int D) {
   if (dtype != PA_DTYPE_BF16 || D != 128) return false;
-  if (p.G < 1 || p.G > pa::TcLayout::kN || (p.G & (p.G - 1))) return false;
-  if (p.B > pa::TcLayout::kMaxSeqs) return false;
+  if (p.G < 1 || p.G > 8 || (p.G & (p.G - 1))) return false;
   if ((int64_t)p.num_blocks * p.Hkv * p.bs >= (int64_t)INT32_MAX) return false;
   if ((int64_t)p.B * p.Hq >= (int64_t)INT32_MAX) return false;
   return true;  // a missing tensor-map encoder then fails the launch loudly (PA_ERR_CUDA)
 }
 
 template <int G>
-pa_status launch_decode_tc_g(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
+pa_status launch_decode_tc_slice(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
   CUtensorMap mk, mv, mq;
   const uint64_t rows = (uint64_t)p.num_blocks * p.Hkv * p.bs;
-  if (!make_map_bf16_d128(&mk, p.k, rows, (uint32_t)p.bs) ||
-      !make_map_bf16_d128(&mv, p.v, rows, (uint32_t)p.bs) ||
+  if (!make_map_pool_4d(&mk, p.k, rows, (uint32_t)p.bs) ||
+      !make_map_pool_4d(&mv, p.v, rows, (uint32_t)p.bs) ||
       !make_map_bf16_d128(&mq, p.q, (uint64_t)p.B * p.Hq, (uint32_t)G))
     return PA_ERR_CUDA;
   auto kern = pa::decode_partition_tc<G>;
@@ -163,6 +178,30 @@ pa_status launch_decode_tc_g(const pa::DecodeParams &p, int32_t max_parts, cudaS
   pa::decode_reduce<__nv_bfloat16, 128>
       <<<p.B * p.Hq, 128, (size_t)max_parts * sizeof(float), st>>>(p);
   return launch_status();
+}
+
+// Sequences are independent: a batch larger than the kernel's per-CTA
+// sequence tables runs as consecutive launches over slices of it.
+template <int G>
+pa_status launch_decode_tc_g(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
+  const int slice = pa::TcLayout::kMaxSeqs;
+  for (int b0 = 0; b0 < p.B; b0 += slice) {
+    pa::DecodeParams ps = p;
+    ps.B = p.B - b0 < slice ? p.B - b0 : slice;
+    const size_t rows = (size_t)b0 * p.Hq;  // (sequence, query head) rows before the slice
+    ps.q = static_cast<const __nv_bfloat16 *>(p.q) + rows * 128;
+    ps.out = static_cast<__nv_bfloat16 *>(p.out) + rows * 128;
+    ps.tables = p.tables + (size_t)b0 * p.max_blocks;
+    ps.lens = p.lens + b0;
+    if (p.ws_m) {
+      ps.ws_m = p.ws_m + rows * max_parts;
+      ps.ws_l = p.ws_l + rows * max_parts;
+      ps.ws_acc = p.ws_acc + rows * max_parts * 128;
+    }
+    const pa_status s = launch_decode_tc_slice<G>(ps, max_parts, st);
+    if (s != PA_OK) return s;
+  }
+  return PA_OK;
 }
 
 pa_status launch_decode_tc(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {

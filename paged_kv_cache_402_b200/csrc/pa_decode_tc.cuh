@@ -12,12 +12,17 @@
 //  * Persistent grid, one CTA per SM; the CTA walks the dense list of real
 //    work units (prefix sums of the partition counts in shared memory) in
 //    round-robin order.
-//  * Warp 0 (one lane) is the TMA producer.  A unit is cut into chunks of 128
-//    tokens; for every block of a chunk it loads the (block, kv head) K tile
-//    and V tile as two 64-column boxes with 128-byte swizzle into a 3-slot K
-//    ring and a 3-slot V ring (32 KiB per slot).  Missing blocks (past the
-//    partition, or a table entry outside the pool) are loaded from rows past
-//    the end of the tensor, which the TMA fills with zeros.
+//  * Warp 0 is the TMA producer.  A unit is cut into chunks of 128 tokens;
+//    each lane loads one block of a chunk: the whole (block, kv head) K tile,
+//    and then the V tile, with ONE 4-D box each (a TMA issue costs about
+//    90 ns per instruction per thread whatever its size, so the box is as big
+//    as a tile and the lanes issue in parallel).  The 4-D view (64 columns,
+//    8 rows, 2 column halves, 8-row groups) lands every tile in shared memory
+//    as [8-row group][column half][8 rows x 128 B] with 128-byte swizzle:
+//    each (group, half) is one swizzle atom, so the MMA sees uniform strides.
+//    K and V go to 3-slot rings of 32 KiB slots.  Missing blocks (past the
+//    partition, or a table entry outside the pool) are loaded from groups
+//    past the end of the tensor, which the TMA fills with zeros.
 //  * Warp 1 (one lane) issues tcgen05 MMAs: per chunk c,
 //        S^T[128 tok x 16] = K_c[128 tok x 128 d] . Q^T[128 d x 16]   (K-major A and B)
 //        O^T[128 d x 16]   = V_c^T[128 d x 128 tok] . P^T[128 tok x 16] (MN-major A)
@@ -43,8 +48,8 @@ struct TcLayout {
                                             // (M = 128 takes N in multiples of 16)
   static constexpr int kChunk = 128;        // tokens per MMA chunk (= M)
   static constexpr int kStages = 3;
-  static constexpr int kHalf = kChunk * 128;  // one 64-dim half of a chunk: 128 rows x 128 B
-  static constexpr int kTile = 2 * kHalf;     // 32 KiB
+  static constexpr int kTile = kChunk * 256;  // 128 tokens x 256 B = 32 KiB
+  static constexpr int kGroup = 2048;         // one 8-row group: two 1 KiB swizzle atoms (column halves)
   static constexpr int kQ = 2 * kN * 128;     // two halves of kN rows x 128 B
   static constexpr int kP = 2 * kN * 128;     // two 64-token halves of kN rows x 128 B
   static constexpr int kMaxSeqs = 2048;
@@ -60,7 +65,8 @@ struct TcLayout {
   static constexpr int kOffTmem = kOffRedSum + kRedFloats * 4;
   static constexpr int kOffScan = kOffTmem + 16;  // 8 ints
   static constexpr int kOffPrefix = kOffScan + 32;
-  static constexpr int kBytes = kOffPrefix + (kMaxSeqs + 1) * 4 + 1024;  // + base alignment slack
+  static constexpr int kOffCtx = kOffPrefix + (kMaxSeqs + 1) * 4;
+  static constexpr int kBytes = kOffCtx + kMaxSeqs * 4 + 1024;  // + base alignment slack
   static constexpr int kThreads = 192;
   static constexpr uint32_t kTmemCols = 64;  // S0 S1 O0 O1, kN columns each
 };
@@ -70,7 +76,8 @@ struct TcUnit {
   bool single;
 };
 
-__device__ __forceinline__ TcUnit tc_unit_at(const DecodeParams &p, const int32_t *prefix, int u) {
+__device__ __forceinline__ TcUnit tc_unit_at(const DecodeParams &p, const int32_t *prefix,
+                                             const int32_t *ctx_s, int u) {
   TcUnit un;
   const int w = u / p.Hkv;
   un.g = u - w * p.Hkv;
@@ -81,7 +88,7 @@ __device__ __forceinline__ TcUnit tc_unit_at(const DecodeParams &p, const int32_
   }
   un.b = lo;
   un.part = w - prefix[lo];
-  const int ctx = p.lens[lo];
+  const int ctx = ctx_s[lo];
   un.t0 = un.part * kPart;
   un.t1 = min(un.t0 + kPart, ctx);
   un.nchunks = (un.t1 - un.t0 + TcLayout::kChunk - 1) / TcLayout::kChunk;
@@ -120,6 +127,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   uint64_t *qfull = bars + 12, *qempty = bars + 14, *sfull = bars + 16, *pfull = bars + 18;
   uint64_t *ofull = bars + 20, *ofree = bars + 22, *drain = bars + 24;
   int32_t *prefix = reinterpret_cast<int32_t *>(smem + L::kOffPrefix);
+  int32_t *ctx_s = reinterpret_cast<int32_t *>(smem + L::kOffCtx);
   int32_t *scan = reinterpret_cast<int32_t *>(smem + L::kOffScan);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffTmem);
   float *red_max = reinterpret_cast<float *>(smem + L::kOffRed);
@@ -163,6 +171,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     if (i < seg && b < B) {
       const int ctx = p.lens[b];
       const bool ok = ctx >= 0 && ctx <= p.max_ctx;
+      ctx_s[b] = ctx;
       cnt[i] = (ok && ctx > 0) ? (ctx + kPart - 1) / kPart : 0;
       mine += cnt[i];
       if (blockIdx.x == 0 && (!ok || ctx == 0)) {  // rows no unit writes: zero them
@@ -202,62 +211,72 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // The whole warp walks the units: its lanes load a unit's table entries
+    // (at most 512 / 8 = 64) in one go, lane 0 takes them by shuffle and
+    // issues the copies.  Waits are polled by every lane and voted.
     if (lane == 0) {
       tc::prefetch_tensormap(&tmap_k);
       tc::prefetch_tensormap(&tmap_v);
       tc::prefetch_tensormap(&tmap_q);
-      const uint64_t pol_kv = policy_evict_first();
-      const uint64_t pol_q = tc::policy_evict_last();
-      const int bs = p.bs;
-      const int blocks_per_chunk = L::kChunk / bs;
-      const int oob_row = p.num_blocks * p.Hkv * bs;  // first row past the pool
-      int c = 0, qi = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-        const TcUnit un = tc_unit_at(p, prefix, u);
-        const int32_t *trow = p.tables + (size_t)un.b * p.max_blocks;
-        const int qs = qi & 1;
-        if (!mbar_wait(&qempty[qs], ((qi >> 1) & 1) ^ 1)) { ok = false; break; }
+    }
+    const uint64_t pol_kv = policy_evict_first();
+    const uint64_t pol_q = tc::policy_evict_last();
+    const int bs = p.bs;
+    const int blocks_per_chunk = L::kChunk / bs;
+    const int oob_group = p.num_blocks * p.Hkv * (bs / 8);  // first 8-row group past the pool
+    int c = 0, qi = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+      const TcUnit un = tc_unit_at(p, prefix, ctx_s, u);
+      const int32_t *trow = p.tables + (size_t)un.b * p.max_blocks + un.t0 / bs;
+      const int nb_unit = (un.t1 - un.t0 + bs - 1) / bs;
+      const int32_t e0 = lane < nb_unit ? trow[lane] : -1;
+      const int32_t e1 = lane + 32 < nb_unit ? trow[lane + 32] : -1;
+      const int qs = qi & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((qi >> 1) & 1) ^ 1))) { ok = false; break; }
+      if (lane == 0) {
         mbar_arrive_expect_tx(&qfull[qs], 2 * G * 128);
         uint8_t *qdst = smem + L::kOffQ + qs * L::kQ;
         const int qy = un.b * p.Hq + un.g * G;
         tc::tma_load_2d(qdst, &tmap_q, 0, qy, &qfull[qs], pol_q);
         tc::tma_load_2d(qdst + N * 128, &tmap_q, 64, qy, &qfull[qs], pol_q);
-        ++qi;
-        for (int ci = 0; ci < un.nchunks; ++ci, ++c) {
-          const int slot = c % 3, use = c / 3;
-          const int jb0 = (un.t0 + ci * L::kChunk) / bs;
-          for (int which = 0; which < 2; ++which) {  // 0: K ring, 1: V ring
-            uint64_t *empty = which ? &vempty[slot] : &kempty[slot];
-            uint64_t *full = which ? &vfull[slot] : &kfull[slot];
-            const CUtensorMap *map = which ? &tmap_v : &tmap_k;
-            if (!mbar_wait(empty, (use & 1) ^ 1)) { ok = false; break; }
-            mbar_arrive_expect_tx(full, L::kTile);
-            uint8_t *dst = smem + (which ? L::kOffV : L::kOffK) + slot * L::kTile;
-            for (int jl = 0; jl < blocks_per_chunk; ++jl) {
-              const int jb = jb0 + jl;
-              int y = oob_row;
-              if (jb * bs < un.t1) {
-                const int32_t blk = trow[jb];
-                if (blk >= 0 && blk < p.num_blocks) y = (blk * p.Hkv + un.g) * bs;
-                else if (which == 0) raise_error(PA_DEVERR_TABLE);
-              }
-              tc::tma_load_2d(dst + jl * bs * 128, map, 0, y, full, pol_kv);
-              tc::tma_load_2d(dst + L::kHalf + jl * bs * 128, map, 64, y, full, pol_kv);
+      }
+      ++qi;
+      for (int ci = 0; ci < un.nchunks; ++ci, ++c) {
+        const int slot = c % 3, use = c / 3;
+        for (int which = 0; which < 2; ++which) {  // 0: K ring, 1: V ring
+          uint64_t *empty = which ? &vempty[slot] : &kempty[slot];
+          uint64_t *full = which ? &vfull[slot] : &kfull[slot];
+          const CUtensorMap *map = which ? &tmap_v : &tmap_k;
+          if (!__all_sync(0xffffffffu, mbar_wait(empty, (use & 1) ^ 1))) { ok = false; break; }
+          uint8_t *dst = smem + (which ? L::kOffV : L::kOffK) + slot * L::kTile;
+          if (lane == 0) mbar_arrive_expect_tx(full, L::kTile);
+          __syncwarp();
+          // lane j loads block j of the chunk
+          const int jloc = ci * blocks_per_chunk + (lane % blocks_per_chunk);
+          const int32_t a0 = __shfl_sync(0xffffffffu, e0, jloc & 31);
+          const int32_t a1 = __shfl_sync(0xffffffffu, e1, jloc & 31);
+          if (lane < blocks_per_chunk) {
+            const int32_t blk = jloc < 32 ? a0 : a1;
+            int w = oob_group;
+            if (jloc < nb_unit) {
+              if (blk >= 0 && blk < p.num_blocks) w = (blk * p.Hkv + un.g) * (bs / 8);
+              else if (which == 0) raise_error(PA_DEVERR_TABLE);
             }
+            tc::tma_load_4d(dst + lane * (bs / 8) * L::kGroup, map, 0, 0, 0, w, full, pol_kv);
           }
-          if (!ok) break;
         }
+        if (!ok) break;
       }
-      if (!ok) {
-        raise_error(PA_DEVERR_TIMEOUT);
-        // wait (bounded) for the copies that may still be in flight
-        for (int k = (c > 3 ? c - 3 : 0); k <= c; ++k) {
-          mbar_wait(&kfull[k % 3], (k / 3) & 1, 100000000ull);
-          mbar_wait(&vfull[k % 3], (k / 3) & 1, 100000000ull);
-        }
-        for (int k = (qi > 2 ? qi - 2 : 0); k < qi; ++k) mbar_wait(&qfull[k & 1], (k >> 1) & 1, 100000000ull);
+    }
+    if (!ok && lane == 0) {
+      raise_error(PA_DEVERR_TIMEOUT);
+      // wait (bounded) for the copies that may still be in flight
+      for (int k = (c > 3 ? c - 3 : 0); k <= c; ++k) {
+        mbar_wait(&kfull[k % 3], (k / 3) & 1, 100000000ull);
+        mbar_wait(&vfull[k % 3], (k / 3) & 1, 100000000ull);
       }
+      for (int k = (qi > 2 ? qi - 2 : 0); k < qi; ++k) mbar_wait(&qfull[k & 1], (k >> 1) & 1, 100000000ull);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -277,8 +296,9 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         const uint32_t d = tmem + 2 * N + (c & 1) * N;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          // V^T: M = head dim (two 64-wide halves L::kHalf apart), K = 16 tokens
-          const uint64_t a = tc::smem_desc_sw128(vb + kk * 2048, L::kHalf, 1024);
+          // V^T, MN-major: M = head dim (two 64-wide atoms 1 KiB apart), K = 16
+          // tokens = two 8-row groups L::kGroup apart
+          const uint64_t a = tc::smem_desc_sw128(vb + kk * 2 * L::kGroup, 1024, L::kGroup);
           const uint64_t bdesc = tc::smem_desc_sw128(pb + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
           tc::mma_bf16(d, a, bdesc, idesc_pv, kk > 0);
         }
@@ -288,7 +308,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       };
       int c = 0, qi = 0, pending = -1;
       for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-        const TcUnit un = tc_unit_at(p, prefix, u);
+        const TcUnit un = tc_unit_at(p, prefix, ctx_s, u);
         const int qs = qi & 1;
         if (!mbar_wait(&qfull[qs], (qi >> 1) & 1)) { ok = false; break; }
         const uint32_t qb = qbase0 + qs * L::kQ;
@@ -300,8 +320,9 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
           const uint32_t d = tmem + (c & 1) * N;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t koff = (kk >> 2) * L::kHalf + (kk & 3) * 32;
-            const uint64_t a = tc::smem_desc_sw128(kb + koff, 16, 1024);
+            // K, K-major: 8-row groups L::kGroup apart, column half kk/4 at +1 KiB
+            const uint32_t koff = (kk >> 2) * 1024 + (kk & 3) * 32;
+            const uint64_t a = tc::smem_desc_sw128(kb + koff, 16, L::kGroup);
             const uint64_t bdesc = tc::smem_desc_sw128(qb + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
             tc::mma_bf16(d, a, bdesc, idesc_qk, kk > 0);
           }
@@ -395,9 +416,18 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
 
     int c = 0;
     for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x) {
-      const TcUnit un = tc_unit_at(p, prefix, u);
+      const TcUnit un = tc_unit_at(p, prefix, ctx_s, u);
       const int32_t *tabrow = p.tables + (size_t)un.b * p.max_blocks;
       const int tail_end = min(((un.t1 + bs - 1) / bs) * bs, un.t0 + kPart);
+      // table entries of this thread's row in every chunk of the unit, loaded
+      // together (one memory round trip per unit, not per chunk)
+      constexpr int kMaxChunks = kPart / L::kChunk;
+      int32_t ent[kMaxChunks];
+#pragma unroll
+      for (int ci = 0; ci < kMaxChunks; ++ci) {
+        const int tok = un.t0 + ci * L::kChunk + r;
+        ent[ci] = tok < un.t1 ? tabrow[tok / bs] : -1;
+      }
 #pragma unroll
       for (int n = 0; n < G; ++n) {
         m_done[n] = m[n];
@@ -414,11 +444,11 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
           tc::tmem_ld8(trow + (c & 1) * N, s);
         }
         const int tok = un.t0 + ci * L::kChunk + r;
-        bool valid = tok < un.t1;
-        if (valid) {
-          const int32_t blk = tabrow[tok / bs];
-          valid = blk >= 0 && blk < p.num_blocks;
-        }
+        int32_t blk = ent[0];
+#pragma unroll
+        for (int k = 1; k < kMaxChunks; ++k)
+          if (ci == k) blk = ent[k];
+        const bool valid = tok < un.t1 && blk >= 0 && blk < p.num_blocks;
         float x[G];
 #pragma unroll
         for (int n = 0; n < G; ++n) {
@@ -434,11 +464,12 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
           if (!mbar_wait(&vfull[c % 3], (c / 3) & 1)) {
             bad = true;
           } else {
-            uint4 *vr = reinterpret_cast<uint4 *>(smem + L::kOffV + (c % 3) * L::kTile + r * 128);
+            uint4 *vr = reinterpret_cast<uint4 *>(smem + L::kOffV + (c % 3) * L::kTile +
+                                                  (r >> 3) * L::kGroup + (r & 7) * 128);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               vr[e] = make_uint4(0, 0, 0, 0);
-              vr[L::kHalf / 16 + e] = make_uint4(0, 0, 0, 0);
+              vr[1024 / 16 + e] = make_uint4(0, 0, 0, 0);
             }
           }
         }
