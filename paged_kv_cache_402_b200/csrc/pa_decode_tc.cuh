@@ -63,7 +63,11 @@ struct TcLayout {
   static constexpr int kRedFloats = 2 * 4 * kN;  // [parity][warp][head]
   static constexpr int kOffRedSum = kOffRed + kRedFloats * 4;
   static constexpr int kOffTmem = kOffRedSum + kRedFloats * 4;
-  static constexpr int kOffScan = kOffTmem + 16;  // 8 ints
+  // per-unit description written by the producer next to the unit's Q slot:
+  // [b, g, part, t0, t1, nchunks, single, pad] + the unit's table entries
+  static constexpr int kUnitInts = 8 + kPart / 8;
+  static constexpr int kOffUnit = kOffTmem + 16;
+  static constexpr int kOffScan = kOffUnit + 2 * kUnitInts * 4;  // 8 ints
   static constexpr int kOffPrefix = kOffScan + 32;
   static constexpr int kOffCtx = kOffPrefix + (kMaxSeqs + 1) * 4;
   static constexpr int kBytes = kOffCtx + kMaxSeqs * 4 + 1024;  // + base alignment slack
@@ -129,6 +133,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   int32_t *prefix = reinterpret_cast<int32_t *>(smem + L::kOffPrefix);
   int32_t *ctx_s = reinterpret_cast<int32_t *>(smem + L::kOffCtx);
   int32_t *scan = reinterpret_cast<int32_t *>(smem + L::kOffScan);
+  int32_t *unit_slots = reinterpret_cast<int32_t *>(smem + L::kOffUnit);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffTmem);
   float *red_max = reinterpret_cast<float *>(smem + L::kOffRed);
   float *red_sum = reinterpret_cast<float *>(smem + L::kOffRedSum);
@@ -144,7 +149,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&qfull[i], 1);
-      mbar_init(&qempty[i], 1);
+      mbar_init(&qempty[i], 2);  // the MMA lane's commit + the softmax warpgroup
       mbar_init(&sfull[i], 1);
       mbar_init(&pfull[i], 128);
       mbar_init(&ofull[i], 1);
@@ -226,14 +231,43 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     const int oob_group = p.num_blocks * p.Hkv * (bs / 8);  // first 8-row group past the pool
     int c = 0, qi = 0;
     bool ok = true;
+    // a unit's table entries (at most 512 / 8 = 64) are loaded one unit ahead
+    // so their memory latency hides behind the previous unit's copies
+    auto load_entries = [&](int u, TcUnit &nu, int32_t &x0, int32_t &x1) {
+      x0 = x1 = -1;
+      if (u < num_units) {
+        nu = tc_unit_at(p, prefix, ctx_s, u);
+        const int32_t *tr = p.tables + (size_t)nu.b * p.max_blocks + nu.t0 / bs;
+        const int nb = (nu.t1 - nu.t0 + bs - 1) / bs;
+        if (lane < nb) x0 = tr[lane];
+        if (lane + 32 < nb) x1 = tr[lane + 32];
+      }
+    };
+    TcUnit un{};
+    int32_t e0, e1;
+    load_entries(blockIdx.x, un, e0, e1);
     for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-      const TcUnit un = tc_unit_at(p, prefix, ctx_s, u);
-      const int32_t *trow = p.tables + (size_t)un.b * p.max_blocks + un.t0 / bs;
       const int nb_unit = (un.t1 - un.t0 + bs - 1) / bs;
-      const int32_t e0 = lane < nb_unit ? trow[lane] : -1;
-      const int32_t e1 = lane + 32 < nb_unit ? trow[lane + 32] : -1;
+      TcUnit next{};
+      int32_t n0, n1;
+      load_entries(u + gridDim.x, next, n0, n1);
       const int qs = qi & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((qi >> 1) & 1) ^ 1))) { ok = false; break; }
+      {  // publish the unit to the MMA lane and the softmax warpgroup
+        int32_t *us = unit_slots + qs * L::kUnitInts;
+        if (lane == 0) {
+          us[0] = un.b;
+          us[1] = un.g;
+          us[2] = un.part;
+          us[3] = un.t0;
+          us[4] = un.t1;
+          us[5] = un.nchunks;
+          us[6] = un.single;
+        }
+        us[8 + lane] = e0;
+        if (L::kUnitInts > 8 + 32 + lane) us[8 + 32 + lane] = e1;
+        __syncwarp();
+      }
       if (lane == 0) {
         mbar_arrive_expect_tx(&qfull[qs], 2 * G * 128);
         uint8_t *qdst = smem + L::kOffQ + qs * L::kQ;
@@ -268,6 +302,9 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         }
         if (!ok) break;
       }
+      e0 = n0;
+      e1 = n1;
+      un = next;
     }
     if (!ok && lane == 0) {
       raise_error(PA_DEVERR_TIMEOUT);
@@ -308,11 +345,11 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       };
       int c = 0, qi = 0, pending = -1;
       for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-        const TcUnit un = tc_unit_at(p, prefix, ctx_s, u);
         const int qs = qi & 1;
         if (!mbar_wait(&qfull[qs], (qi >> 1) & 1)) { ok = false; break; }
+        const int nchunks = unit_slots[qs * L::kUnitInts + 5];
         const uint32_t qb = qbase0 + qs * L::kQ;
-        for (int ci = 0; ci < un.nchunks; ++ci, ++c) {
+        for (int ci = 0; ci < nchunks; ++ci, ++c) {
           const int slot = c % 3;
           if (!mbar_wait(&kfull[slot], (c / 3) & 1)) { ok = false; break; }
           tc::fence_after_sync();
@@ -328,7 +365,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
           }
           tc::mma_commit(&sfull[c & 1]);
           tc::mma_commit(&kempty[slot]);
-          if (ci == un.nchunks - 1) tc::mma_commit(&qempty[qs]);
+          if (ci == nchunks - 1) tc::mma_commit(&qempty[qs]);
           if (pending >= 0 && !issue_pv(pending)) { ok = false; break; }
           pending = c;
         }
@@ -414,20 +451,25 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       if (p_last) epilogue(pun, nunit & 1);
     };
 
-    int c = 0;
-    for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x) {
-      const TcUnit un = tc_unit_at(p, prefix, ctx_s, u);
-      const int32_t *tabrow = p.tables + (size_t)un.b * p.max_blocks;
-      const int tail_end = min(((un.t1 + bs - 1) / bs) * bs, un.t0 + kPart);
-      // table entries of this thread's row in every chunk of the unit, loaded
-      // together (one memory round trip per unit, not per chunk)
-      constexpr int kMaxChunks = kPart / L::kChunk;
-      int32_t ent[kMaxChunks];
-#pragma unroll
-      for (int ci = 0; ci < kMaxChunks; ++ci) {
-        const int tok = un.t0 + ci * L::kChunk + r;
-        ent[ci] = tok < un.t1 ? tabrow[tok / bs] : -1;
-      }
+    const int log2_bs = bs == 8 ? 3 : (bs == 16 ? 4 : 5);
+    int c = 0, qi = 0;
+    for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x, ++qi) {
+      // the unit, as the producer published it with its Q tile
+      const int qs = qi & 1;
+      if (!bad && !mbar_wait(&qfull[qs], (qi >> 1) & 1)) bad = true;
+      stop = wg_sync_or(bad);  // every thread reads the slot, or none does
+      if (stop) break;
+      const int32_t *us = unit_slots + qs * L::kUnitInts;
+      TcUnit un;
+      un.b = us[0];
+      un.g = us[1];
+      un.part = us[2];
+      un.t0 = us[3];
+      un.t1 = us[4];
+      un.nchunks = us[5];
+      un.single = us[6] != 0;
+      const int32_t *ents = us + 8;
+      const int tail_end = min(((un.t1 + bs - 1) >> log2_bs) << log2_bs, un.t0 + kPart);
 #pragma unroll
       for (int n = 0; n < G; ++n) {
         m_done[n] = m[n];
@@ -444,11 +486,8 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
           tc::tmem_ld8(trow + (c & 1) * N, s);
         }
         const int tok = un.t0 + ci * L::kChunk + r;
-        int32_t blk = ent[0];
-#pragma unroll
-        for (int k = 1; k < kMaxChunks; ++k)
-          if (ci == k) blk = ent[k];
-        const bool valid = tok < un.t1 && blk >= 0 && blk < p.num_blocks;
+        const int32_t blk = tok < un.t1 ? ents[(tok - un.t0) >> log2_bs] : -1;
+        const bool valid = blk >= 0 && blk < p.num_blocks;
         float x[G];
 #pragma unroll
         for (int n = 0; n < G; ++n) {
@@ -495,6 +534,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         fence_proxy_async_smem();
         tc::fence_before_sync();
         mbar_arrive(&pfull[c & 1]);
+        if (ci == un.nchunks - 1 && threadIdx.x == 64) mbar_arrive(&qempty[qs]);  // done with the unit slot
         // ---- merge of chunk c-1
         if (pend) {
           merge();
