@@ -346,51 +346,75 @@ def run_ours(args, rank: int, world: int, dev):
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
-    def step(s, ev=None):
+    def step(s, strm, ev=None):
         inst = insts[s % R]
         st = inst.steps[s // R]
         n = 0
         if st["pairs"] is not None:
-            pa.pa_copy_blocks(st["pairs"], inst.cache, stream)
+            pa.pa_copy_blocks(st["pairs"], inst.cache, strm)
             n += 1
-        pa.pa_append_kv(st["k"], st["v"], st["slots"], inst.cache, stream)
+        pa.pa_append_kv(st["k"], st["v"], st["slots"], inst.cache, strm)
         n += 1
         if ev is not None:
-            ev[0].record(stream)
+            ev[0].record(strm)
         pa.pa_decode(st["q"], inst.cache, st["tables"], st["lens"], st["max_ctx"], 1.0 / math.sqrt(wl["D"]),
-                     out=st["out"], workspace=st["ws"], stream=stream)
+                     out=st["out"], workspace=st["ws"], stream=strm)
         if ev is not None:
-            ev[1].record(stream)
+            ev[1].record(strm)
         n += 2 if st["max_ctx"] > pa.PA_PARTITION_TOKENS else 1
         return n, st
 
     for s in range(args.warmup):
-        step(s)
+        step(s, stream)
     if pa.pa_read_device_error() != 0:
         raise RuntimeError("device error during warm-up")
 
-    dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(args.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # The K timed steps (inputs precomputed, resident) are captured once into
+    # a CUDA graph and replayed, so the host's launch rate does not bound the
+    # device-side measurement.  Each step's decode launch is bracketed by
+    # events captured inside the graph.
+    # external: inside a captured graph the records become event-record nodes
+    dec_events = [(torch.cuda.Event(enable_timing=True, external=True),
+                   torch.cuda.Event(enable_timing=True, external=True)) for _ in range(args.steps)]
     launches = 0
     kv_bytes = 0       # distinct physical K/V bytes (what HBM must serve)
     kv_logical = 0     # per-sequence K/V bytes (shared blocks counted per sharer)
     pairs = 0
     algo_bytes = []
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            cap = torch.cuda.current_stream()
+            for i in range(args.steps):
+                n, st = step(args.warmup + i, cap, dec_events[i])
+                launches += n
+                kv_bytes += st["kv_unique_bytes"]
+                kv_logical += st["kv_bytes"]
+                pairs += st["n_pairs"]
+                algo_bytes.append(st["algo_bytes"])
+        graph.replay()  # one untimed replay: the graph's own warm-up
+        torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     with ClockSampler(dev) as clk:
         t_start.record(stream)
-        for i in range(args.steps):
-            n, st = step(args.warmup + i, dec_events[i])
-            launches += n
-            kv_bytes += st["kv_unique_bytes"]
-            kv_logical += st["kv_bytes"]
-            pairs += st["n_pairs"]
-            algo_bytes.append(st["algo_bytes"])
+        if graph is not None:
+            graph.replay()
+        else:
+            for i in range(args.steps):
+                n, st = step(args.warmup + i, stream, dec_events[i])
+                launches += n
+                kv_bytes += st["kv_unique_bytes"]
+                kv_logical += st["kv_bytes"]
+                pairs += st["n_pairs"]
+                algo_bytes.append(st["algo_bytes"])
         t_end.record(stream)
         torch.cuda.synchronize()
+    if graph is not None:
+        del graph
     if world > 1:
         torch.distributed.barrier()
     ms = t_start.elapsed_time(t_end)
@@ -440,7 +464,8 @@ def run_ours(args, rank: int, world: int, dev):
                    "partition_tokens": pa.PA_PARTITION_TOKENS,
                    "l2": f"{R} rotating batch instances per rank (KV per step ~{kv_bytes / args.steps / 1e6:.0f} MB, "
                          f"working set ~{R * kv_bytes / args.steps / 1e6:.0f} MB > 126 MB L2)",
-                   "parallelism": f"replicas x{world}"},
+                   "parallelism": f"replicas x{world}",
+                   "timing": "eager launches" if args.no_graph else "CUDA graph replay of the K steps"},
         "tokens_per_s": round(tok_all / (ms_all / 1e3), 1),
         "kv_logical_gbs": round(kv_logical * world / 1e9 / (ms_all / 1e3), 2),
         "copy_pairs_per_step": round(pairs / args.steps, 2),
@@ -530,6 +555,125 @@ def run_e2e(args, insts, wl, dev, stream):
     seconds = time.perf_counter() - t0
     kv = sum(unique_kv_bytes(t, l, bs, 2 * Hkv * D * 2) for t, l in seen)
     return {"seconds": seconds, "kv_gb": kv / 1e9, "steps": n_steps, "h2d": h2d, "d2h": d2h}
+
+
+def run_trace(args, dev):
+    """Continuous batching of beam-search requests over a 16 GiB K+V pool, one
+    JSON line per block size: per step the host trace driver (allocator
+    calls), host -> device copies of the step's tables / lengths / slots /
+    copy pairs, copy-on-write copies, prompt and decode appends, the decode of
+    every running beam, and the device -> host read of the output."""
+    import paged_kv_cache_402_b200 as pa
+    from paged_kv_cache_402_b200 import synth
+    from paged_kv_cache_402_b200.trace import BeamTrace
+
+    Hq, Hkv, D = 32, 8, 128
+    dt = torch.bfloat16
+    row = 2 * Hkv * D * 2
+    stream = torch.cuda.current_stream()
+    lines = []
+    sizes = [args.block_size] if args.block_size else [8, 16, 32]
+    draws = synth.trace(args.seed, steps=args.trace_steps)
+    # random rows to draw prompt / decode K, V and q from (values do not
+    # change the work; the pool of rows is reused cyclically)
+    src = synth.normal((1 << 16, Hkv, D), dt, 901, device=dev)
+    qsrc = synth.normal((8192, Hq, D), dt, 902, device=dev)
+    for bs in sizes:
+        NB = 16 * 2**30 // (2 * Hkv * bs * D * 2)
+        order = synth.rng(args.seed + bs).permutation(NB)
+        A = pa.Allocator(NB, bs, order)
+        cache = pa.KVCache.empty(NB, Hkv, bs, D, dt, dev)
+        drv = BeamTrace(A, lambda: A.stats()["free_blocks"], bs, draws)
+        out = torch.empty(8192, Hq, D, dtype=dt, device=dev)
+        ws = torch.empty(64 << 20, dtype=torch.uint8, device=dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.trace_steps)]
+        host_s = dec_ms = 0.0
+        wall = 0.0
+        uniq = logical = 0
+        beams = 0
+        frag = []
+        h2d = d2h = 0
+        launches = 0
+        torch.cuda.synchronize()
+        for s_ in range(args.trace_steps):
+            t0 = time.perf_counter()
+            plan = drv.step()
+            n = len(plan.decode_seqs)
+            if n:
+                max_ctx, mb = A.max_len(plan.decode_seqs)
+                tables, lens = A.build_block_tables(plan.decode_seqs, mb)
+            host_s += time.perf_counter() - t0
+            if n == 0:
+                wall += time.perf_counter() - t0
+                continue
+            npr = len(plan.prompt_slots)
+            h = [torch.from_numpy(plan.prompt_slots).pin_memory() if npr else None,
+                 torch.from_numpy(plan.decode_slots).pin_memory(),
+                 torch.from_numpy(np.ascontiguousarray(plan.cow_pairs)).pin_memory() if len(plan.cow_pairs) else None,
+                 torch.from_numpy(tables).pin_memory(), torch.from_numpy(lens).pin_memory()]
+            d_ = [x.to(dev, non_blocking=True) if x is not None else None for x in h]
+            ev[s_][0].record(stream)
+            if npr:
+                i0 = (s_ * 977) % ((1 << 16) - npr) if npr < (1 << 16) else 0
+                kk = src[i0:i0 + npr]
+                pa.pa_append_kv(kk, kk, d_[0], cache, stream)
+                launches += 1
+            if d_[2] is not None:
+                pa.pa_copy_blocks(d_[2], cache, stream)
+                launches += 1
+            kd = src[(s_ * 131) % ((1 << 16) - n):][:n]
+            pa.pa_append_kv(kd, kd, d_[1], cache, stream)
+            need = pa.pa_decode_workspace_size(n, Hq, max_ctx, D)
+            if need > ws.numel():
+                ws = torch.empty(need * 5 // 4, dtype=torch.uint8, device=dev)
+            q = qsrc[:n] if n <= 8192 else synth.normal((n, Hq, D), dt, s_, device=dev)
+            o = out[:n] if n <= 8192 else torch.empty(n, Hq, D, dtype=dt, device=dev)
+            pa.pa_decode(q, cache, d_[3], d_[4], max_ctx, 1 / math.sqrt(D), out=o, workspace=ws, stream=stream)
+            launches += 2 + (1 if max_ctx > pa.PA_PARTITION_TOKENS else 0)
+            ev[s_][1].record(stream)
+            res = o[:1].to("cpu", non_blocking=True)
+            torch.cuda.synchronize()
+            wall += time.perf_counter() - t0
+            dec_ms += ev[s_][0].elapsed_time(ev[s_][1])
+            st = A.stats()
+            uniq += st["used_slots"] * row
+            logical += int(lens.astype(np.int64).sum()) * row
+            beams += n
+            frag.append(st["fragmentation"])
+            h2d += sum(x.numel() * x.element_size() for x in h if x is not None)
+            d2h += res.numel() * res.element_size()
+        if pa.pa_read_device_error() != 0:
+            raise RuntimeError("device error in the trace")
+        peak, peak_kind = measured_peaks()
+        steps = args.trace_steps
+        line = {
+            "metric": METRIC, "workload": "trace",
+            "value": round(uniq / 1e9 / (dec_ms / 1e3), 2), "unit": "GB/s",
+            "n_gpus": 1, "steps": steps, "warmup": 0, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic trace (seeded)",
+            "config": {"workload": "bf16 continuous-batching trace: Poisson(4) arrivals per step, prompts "
+                                   "lognormal (median 512, max 4096), outputs geometric (mean 256), beam "
+                                   "groups of 4 re-forked copy-on-write, 32 q / 8 kv heads, head_dim 128, "
+                                   "16 GiB K+V pool",
+                       "block_size": bs, "trace_steps": steps,
+                       "timing": "device: CUDA events around each step's kernels; wall: whole step incl. host"},
+            "kv_logical_gbs": round(logical / 1e9 / (dec_ms / 1e3), 2),
+            "kv_frac_of_hbm_peak": round(uniq / 1e9 / (dec_ms / 1e3) / peak, 4),
+            "tokens_per_s": round(beams / wall, 1),
+            "device_ms_per_step": round(dec_ms / steps, 4), "wall_ms_per_step": round(1e3 * wall / steps, 4),
+            "host_driver_ms_per_step": round(1e3 * host_s / steps, 4),
+            "mean_running_beams": round(beams / steps, 1),
+            "fragmentation_mean": round(float(np.mean(frag)), 5) if frag else None,
+            "fragmentation_last": round(frag[-1], 5) if frag else None,
+            "e2e": {"value": round(uniq / 1e9 / wall, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d // steps,
+                    "d2h_bytes_per_step": d2h // steps},
+            "gpu_launches": launches,
+        }
+        lines.append(line)
+        del cache, A, drv
+        torch.cuda.empty_cache()
+    return lines
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -629,10 +773,14 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gqa")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["trace"], default="gqa")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rotate", type=int, default=0, help="batch instances to rotate (0: the workload's default)")
+    ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly instead of from a CUDA graph")
+    ap.add_argument("--block-size", type=int, default=0, help="trace workload: one block size (0: 8, 16 and 32)")
+    ap.add_argument("--trace-steps", type=int, default=1000)
+    ap.add_argument("--seed", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -652,6 +800,11 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
+    if args.workload == "trace":
+        if rank == 0:
+            for line in run_trace(args, dev):
+                print(json.dumps(line), flush=True)
+        return
     try:
         line = run_ours(args, rank, world, dev)
         if rank == 0 and world == 1 and not args.no_cpu_baseline and "lengths" in WORKLOADS[args.workload]:

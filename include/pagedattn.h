@@ -252,6 +252,11 @@ PA_API pa_status pa_seq_len(pa_allocator *a, int32_t seq, int32_t *len, int32_t 
 PA_API pa_status pa_seq_block_table(pa_allocator *a, int32_t seq, int32_t *out_host, int32_t cap,
                                     int32_t *count);
 
+/* The longest of n_seqs sequences: its length in tokens (the max_context_len
+ * pa_decode takes) and its number of blocks (the narrowest table width). */
+PA_API pa_status pa_seqs_max_len(pa_allocator *a, const int32_t *seqs, int32_t n_seqs,
+                                 int32_t *max_len, int32_t *max_blocks);
+
 /* Writes the tables of n_seqs sequences as rows of a [n_seqs][max_blocks]
  * int32 host array padded with `pad`, and their lengths to lens_host. */
 PA_API pa_status pa_build_block_tables(pa_allocator *a, const int32_t *seqs, int32_t n_seqs,

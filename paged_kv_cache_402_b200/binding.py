@@ -75,6 +75,7 @@ def _load() -> ctypes.CDLL:
         "pa_seq_len": (st, [vp, i32, i32p, i32p]),
         "pa_seq_block_table": (st, [vp, i32, i32p, i32, i32p]),
         "pa_build_block_tables": (st, [vp, i32p, i32, i32, i32, i32p, i32p]),
+        "pa_seqs_max_len": (st, [vp, i32p, i32, i32p, i32p]),
         "pa_alloc_stats": (st, [vp, i64p, i64p, i32p, i32p]),
         "pa_block_refcount": (st, [vp, i32, i32p]),
     }
@@ -323,6 +324,14 @@ class Allocator:
         cnt = ctypes.c_int32()
         _check(_lib.pa_seq_block_table(self._h, int(seq), _i32p(out), nb, ctypes.byref(cnt)), "pa_seq_block_table")
         return out[:cnt.value].tolist()
+
+    def max_len(self, seqs):
+        """(longest length in tokens, most blocks) over the sequences."""
+        seqs = np.ascontiguousarray(np.asarray(seqs, dtype=np.int32))
+        ml, mb = ctypes.c_int32(), ctypes.c_int32()
+        _check(_lib.pa_seqs_max_len(self._h, _i32p(seqs), len(seqs), ctypes.byref(ml), ctypes.byref(mb)),
+               "pa_seqs_max_len")
+        return ml.value, mb.value
 
     def build_block_tables(self, seqs, max_blocks: int, pad: int = -1, out_tables=None, out_lens=None):
         seqs = np.ascontiguousarray(np.asarray(seqs, dtype=np.int32))

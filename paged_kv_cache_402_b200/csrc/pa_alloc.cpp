@@ -236,6 +236,21 @@ PA_API pa_status pa_seq_block_table(pa_allocator *a, int32_t seq, int32_t *out_h
   return PA_OK;
 }
 
+PA_API pa_status pa_seqs_max_len(pa_allocator *a, const int32_t *seqs, int32_t n_seqs,
+                                 int32_t *max_len, int32_t *max_blocks) {
+  if (!a || n_seqs < 0 || (n_seqs > 0 && !seqs) || !max_len || !max_blocks) return PA_ERR_INVALID_ARG;
+  int32_t ml = 0, mb = 0;
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    const Seq *s = a->find(seqs[i]);
+    if (!s) return PA_ERR_NOT_FOUND;
+    if (s->len > ml) ml = s->len;
+    if ((int32_t)s->table.size() > mb) mb = (int32_t)s->table.size();
+  }
+  *max_len = ml;
+  *max_blocks = mb;
+  return PA_OK;
+}
+
 PA_API pa_status pa_build_block_tables(pa_allocator *a, const int32_t *seqs, int32_t n_seqs,
                                        int32_t max_blocks, int32_t pad, int32_t *tables_host,
                                        int32_t *lens_host) {

@@ -4,6 +4,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+#include <utility>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -36,11 +38,69 @@ inline pa_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+// Launches with programmatic stream serialization: the kernel may be
+// scheduled while the previous kernel in the stream is finishing; each of
+// the library's kernels waits (griddepcontrol.wait) before reading memory.
+template <typename... KArgs, typename... Args>
+pa_status launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                 Args &&...args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
+  return launch_status();
+}
+
 inline int32_t max_parts_for(int32_t max_context_len) {
   return (max_context_len + pa::kPart - 1) / pa::kPart;
 }
 
 inline size_t round16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+constexpr int kMaxDev = 64;
+
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return -1;
+  return dev;
+}
+
+// SM count of the current device, looked up once per device.
+int sm_count() {
+  static std::atomic<int> cache[kMaxDev] = {};
+  const int dev = current_device();
+  if (dev < 0) return 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device (and again
+// only if a larger size is asked for).  `done` belongs to that one kernel.
+template <typename Kernel>
+bool ensure_smem(Kernel kern, int bytes, std::atomic<int> (&done)[kMaxDev]) {
+  const int dev = current_device();
+  if (dev < 0) return false;
+  if (done[dev].load(std::memory_order_relaxed) >= bytes) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  done[dev].store(bytes, std::memory_order_relaxed);
+  return true;
+}
+
 
 // workspace layout: m [B*Hq*P] f32 | l [B*Hq*P] f32 | acc [B*Hq*P*D] f32
 size_t workspace_bytes_for(int64_t B, int64_t Hq, int32_t max_ctx, int64_t D) {
@@ -69,15 +129,12 @@ pa_status launch_decode_t(const pa::DecodeParams &p, int32_t max_parts, cudaStre
   const size_t merge = (size_t)pa::kWarps * G * (D + 2) * sizeof(float);
   if (smem < merge) smem = merge;
   auto kern = pa::decode_partition_simt<T, D, G>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return PA_ERR_CUDA;
+  static std::atomic<int> smem_set[kMaxDev] = {};
+  if (!ensure_smem(kern, (int)smem, smem_set)) return PA_ERR_CUDA;
   dim3 grid(max_parts, p.Hkv, p.B);
-  kern<<<grid, pa::kWarps * 32, smem, st>>>(p, nstages);
-  pa_status s = launch_status();
+  pa_status s = launch(kern, grid, dim3(pa::kWarps * 32), smem, st, p, nstages);
   if (s != PA_OK || max_parts <= 1) return s;
-  pa::decode_reduce<T, D><<<p.B * p.Hq, 128, (size_t)max_parts * sizeof(float), st>>>(p);
-  return launch_status();
+  return launch(pa::decode_reduce<T, D>, dim3(p.B * p.Hq), dim3(128), (size_t)max_parts * sizeof(float), st, p);
 }
 
 template <typename T, int D>
@@ -141,13 +198,6 @@ bool make_map_pool_4d(CUtensorMap *m, const void *base, uint64_t rows, uint32_t 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return n;
-}
-
 bool tc_eligible(const pa::DecodeParams &p, int dtype, int D) {
   if (dtype != PA_DTYPE_BF16 || D != 128) return false;
   if (p.G < 1 || p.G > 8 || (p.G & (p.G - 1))) return false;
@@ -166,25 +216,29 @@ pa_status launch_decode_tc_slice(const pa::DecodeParams &p, int32_t max_parts, c
     return PA_ERR_CUDA;
   auto kern = pa::decode_partition_tc<G>;
   const int smem = pa::TcLayout::kBytes;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return PA_ERR_CUDA;
+  static std::atomic<int> smem_set[kMaxDev] = {};
+  if (!ensure_smem(kern, smem, smem_set)) return PA_ERR_CUDA;
   const int64_t units_bound = (int64_t)p.Hkv * p.B * max_parts;
   int grid = sm_count();
   if (grid <= 0) return PA_ERR_CUDA;
   if (units_bound < grid) grid = (int)units_bound;
-  kern<<<grid, pa::TcLayout::kThreads, smem, st>>>(mk, mv, mq, p);
-  pa_status s = launch_status();
+  pa_status s = launch(kern, dim3(grid), dim3(pa::TcLayout::kThreads), (size_t)smem, st, mk, mv, mq, p);
   if (s != PA_OK || max_parts <= 1) return s;
-  pa::decode_reduce<__nv_bfloat16, 128>
-      <<<p.B * p.Hq, 128, (size_t)max_parts * sizeof(float), st>>>(p);
-  return launch_status();
+  return launch(pa::decode_reduce<__nv_bfloat16, 128>, dim3(p.B * p.Hq), dim3(128),
+                (size_t)max_parts * sizeof(float), st, p);
 }
 
 // Sequences are independent: a batch larger than the kernel's per-CTA
 // sequence tables runs as consecutive launches over slices of it.
+std::atomic<uint32_t> g_sched_ticket{0};
+
 template <int G>
 pa_status launch_decode_tc_g(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
-  const int slice = pa::TcLayout::kMaxSeqs;
+  // a slice is at most kMaxSeqs sequences, and its full partitions must fit
+  // the 20-bit counts of the kernel's packed prefix sums
+  int slice = pa::TcLayout::kMaxSeqs;
+  const int by_parts = ((1 << pa::kFullBits) - 1) / (max_parts > 0 ? max_parts : 1);
+  if (by_parts < slice) slice = by_parts > 0 ? by_parts : 1;
   for (int b0 = 0; b0 < p.B; b0 += slice) {
     pa::DecodeParams ps = p;
     ps.B = p.B - b0 < slice ? p.B - b0 : slice;
@@ -198,6 +252,7 @@ pa_status launch_decode_tc_g(const pa::DecodeParams &p, int32_t max_parts, cudaS
       ps.ws_l = p.ws_l + rows * max_parts;
       ps.ws_acc = p.ws_acc + rows * max_parts * 128;
     }
+    ps.sched_slot = (int32_t)(g_sched_ticket.fetch_add(1) % pa::kSchedSlots);
     const pa_status s = launch_decode_tc_slice<G>(ps, max_parts, st);
     if (s != PA_OK) return s;
   }
@@ -253,11 +308,10 @@ PA_API pa_status pa_append_kv(const void *k, const void *v, const int64_t *slot_
   const int64_t warps = (int64_t)num_tokens * cache->num_kv_heads;
   const int64_t blocks = (warps * 32 + 255) / 256;
   if (blocks > INT32_MAX) return PA_ERR_INVALID_ARG;
-  pa::append_kv_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(
-      (const uint4 *)k, (const uint4 *)v, slot_mapping, num_tokens, cache->num_kv_heads,
-      cache->block_size, row_vecs, (int64_t)cache->num_blocks * cache->block_size, (uint4 *)cache->k,
-      (uint4 *)cache->v);
-  return launch_status();
+  return launch(pa::append_kv_kernel, dim3((unsigned)blocks), dim3(256), 0, (cudaStream_t)stream,
+                (const uint4 *)k, (const uint4 *)v, slot_mapping, num_tokens, cache->num_kv_heads,
+                cache->block_size, row_vecs, (int64_t)cache->num_blocks * cache->block_size,
+                (uint4 *)cache->k, (uint4 *)cache->v);
 }
 
 PA_API pa_status pa_copy_blocks(const int32_t *src_dst_pairs, int32_t num_pairs,
@@ -272,9 +326,8 @@ PA_API pa_status pa_copy_blocks(const int32_t *src_dst_pairs, int32_t num_pairs,
   const int64_t block_vecs = block_bytes / 16;
   const int64_t per_cta = 256 * pa::kCopyUnroll;
   dim3 grid((unsigned)((block_vecs + per_cta - 1) / per_cta), (unsigned)num_pairs);
-  pa::copy_blocks_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(
-      src_dst_pairs, cache->num_blocks, block_vecs, (uint4 *)cache->k, (uint4 *)cache->v);
-  return launch_status();
+  return launch(pa::copy_blocks_kernel, grid, dim3(256), 0, (cudaStream_t)stream, src_dst_pairs,
+                cache->num_blocks, block_vecs, (uint4 *)cache->k, (uint4 *)cache->v);
 }
 
 PA_API pa_status pa_check_copy_pairs(const int32_t *pairs, int32_t num_pairs, int32_t num_blocks) {

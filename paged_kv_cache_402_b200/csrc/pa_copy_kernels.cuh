@@ -23,6 +23,8 @@ __global__ void __launch_bounds__(256)
                      const int64_t *__restrict__ slots, int32_t num_tokens, int32_t Hkv,
                      int32_t bs, int32_t row_vecs, int64_t pool_slots, uint4 *__restrict__ kc,
                      uint4 *__restrict__ vc) {
+  wait_prior_grid();
+  allow_next_grid();
   const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (wid >= (int64_t)num_tokens * Hkv) return;
@@ -52,6 +54,8 @@ constexpr int kCopyUnroll = 4;
 __global__ void __launch_bounds__(256)
     copy_blocks_kernel(const int32_t *__restrict__ pairs, int32_t num_blocks, int64_t block_vecs,
                        uint4 *kc, uint4 *vc) {
+  wait_prior_grid();
+  allow_next_grid();
   const int pair = blockIdx.y;
   const int32_t src = pairs[2 * pair], dst = pairs[2 * pair + 1];
   if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {

@@ -37,6 +37,7 @@ struct DecodeParams {
   float *ws_l;    // [B][Hq][max_parts] sum of weights
   float *ws_acc;  // [B][Hq][max_parts][D] unnormalised accumulator
   int32_t num_blocks, Hkv, bs, Hq, G, max_blocks, B, max_ctx, max_parts;
+  int32_t sched_slot;  // tensor-core kernel: which run-time work counter this call uses
   float scale_log2;  // scale * log2(e)
 };
 
@@ -56,6 +57,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   static_assert(SUB % RPP == 0, "sub-tile");
   constexpr int RPL = SUB / RPP;  // rows per lane per sub-tile
 
+  wait_prior_grid();  // no early trigger: this grid has many waves of CTAs
   const int part = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rg = lane / LPR, dl = lane % LPR;
@@ -283,6 +285,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(128) decode_reduce(DecodeParams p) {
   extern __shared__ float wsh[];  // [max_parts] weights
   __shared__ float red[32];
+  wait_prior_grid();
+  allow_next_grid();
   const int bh = blockIdx.x;
   const int b = bh / p.Hq;
   const int ctx = p.lens[b];

@@ -9,9 +9,12 @@
 // (max, sum, unnormalised accumulator) for the log-sum-exp reduce.
 //
 // How, on sm_100a:
-//  * Persistent grid, one CTA per SM; the CTA walks the dense list of real
-//    work units (prefix sums of the partition counts in shared memory) in
-//    round-robin order.
+//  * Persistent grid, one CTA per SM.  Work units are handed out at run time
+//    from a counter (largest first: every full 512-token partition, then the
+//    partial last partition of each sequence), so CTAs that drew short units
+//    take more of them and all finish together.  The counter lives in one of
+//    kSchedSlots library-owned slots, chosen per call, and the last CTA out
+//    resets it.
 //  * Warp 0 is the TMA producer.  A unit is cut into chunks of 128 tokens;
 //    each lane loads one block of a chunk: the whole (block, kv head) K tile,
 //    and then the V tile, with ONE 4-D box each (a TMA issue costs about
@@ -75,24 +78,46 @@ struct TcLayout {
   static constexpr uint32_t kTmemCols = 64;  // S0 S1 O0 O1, kN columns each
 };
 
+// Largest excess (base-2 units) of a score over the running reference before
+// the reference is moved: weights then stay below 2^8, far inside the range
+// of the bf16 P operand and the fp32 sums.
+constexpr float kLazyRescale = 8.0f;
+
 struct TcUnit {
   int b, g, part, t0, t1, nchunks;
   bool single;
 };
 
+// Run-time work counters: [next unit, CTAs finished] per slot.  A call takes
+// slot (ticket % kSchedSlots); the last CTA of the call puts both back to 0,
+// so the slot is ready for the call that takes it next.
+constexpr int kSchedSlots = 64;
+__device__ uint32_t g_sched[2 * kSchedSlots];
+
+// prefix[b] packs, for sequences before b, the number of full 512-token
+// partitions (bits 0..19) and of partial last partitions (bits 20..31).
+constexpr int kFullBits = 20;
+__device__ __forceinline__ int pf_of(int32_t v) { return v & ((1 << kFullBits) - 1); }
+__device__ __forceinline__ int pp_of(int32_t v) { return (int)((uint32_t)v >> kFullBits); }
+
+// Unit u of the largest-first order: units [0, F) are the full partitions
+// (sequence-major, kv head fastest), units [F, F + P) the partial ones.
 __device__ __forceinline__ TcUnit tc_unit_at(const DecodeParams &p, const int32_t *prefix,
-                                             const int32_t *ctx_s, int u) {
+                                             const int32_t *ctx_s, int u, int num_full) {
   TcUnit un;
-  const int w = u / p.Hkv;
-  un.g = u - w * p.Hkv;
-  int lo = 0, hi = p.B - 1;  // largest b with prefix[b] <= w
+  const bool full = u < num_full;
+  const int v = full ? u : u - num_full;
+  const int w = v / p.Hkv;
+  un.g = v - w * p.Hkv;
+  int lo = 0, hi = p.B - 1;  // largest b whose count before it is <= w
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (prefix[mid] <= w) lo = mid; else hi = mid - 1;
+    const int cnt = full ? pf_of(prefix[mid]) : pp_of(prefix[mid]);
+    if (cnt <= w) lo = mid; else hi = mid - 1;
   }
   un.b = lo;
-  un.part = w - prefix[lo];
   const int ctx = ctx_s[lo];
+  un.part = full ? w - pf_of(prefix[lo]) : ctx / kPart;
   un.t0 = un.part * kPart;
   un.t1 = min(un.t0 + kPart, ctx);
   un.nchunks = (un.t1 - un.t0 + TcLayout::kChunk - 1) / TcLayout::kChunk;
@@ -125,6 +150,8 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
 
+  wait_prior_grid();
+  allow_next_grid();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
   uint64_t *kfull = bars, *kempty = bars + 3, *vfull = bars + 6, *vempty = bars + 9;
@@ -177,7 +204,8 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       const int ctx = p.lens[b];
       const bool ok = ctx >= 0 && ctx <= p.max_ctx;
       ctx_s[b] = ctx;
-      cnt[i] = (ok && ctx > 0) ? (ctx + kPart - 1) / kPart : 0;
+      // full partitions in the low bits, a partial last partition in the high ones
+      cnt[i] = (ok && ctx > 0) ? (ctx / kPart) | ((ctx % kPart != 0 ? 1 : 0) << kFullBits) : 0;
       mine += cnt[i];
       if (blockIdx.x == 0 && (!ok || ctx == 0)) {  // rows no unit writes: zero them
         if (!ok) raise_error(PA_DEVERR_LEN);
@@ -212,7 +240,9 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int num_units = p.Hkv * prefix[B];
+  const int num_full = p.Hkv * pf_of(prefix[B]);
+  const int num_units = num_full + p.Hkv * pp_of(prefix[B]);
+  uint32_t *sched = g_sched + 2 * p.sched_slot;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -231,12 +261,12 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     const int oob_group = p.num_blocks * p.Hkv * (bs / 8);  // first 8-row group past the pool
     int c = 0, qi = 0;
     bool ok = true;
-    // a unit's table entries (at most 512 / 8 = 64) are loaded one unit ahead
-    // so their memory latency hides behind the previous unit's copies
+    // a unit's table entries (at most 512 / 8 = 64), loaded by the lanes
+    // right after the previous unit's copies are issued
     auto load_entries = [&](int u, TcUnit &nu, int32_t &x0, int32_t &x1) {
       x0 = x1 = -1;
       if (u < num_units) {
-        nu = tc_unit_at(p, prefix, ctx_s, u);
+        nu = tc_unit_at(p, prefix, ctx_s, u, num_full);
         const int32_t *tr = p.tables + (size_t)nu.b * p.max_blocks + nu.t0 / bs;
         const int nb = (nu.t1 - nu.t0 + bs - 1) / bs;
         if (lane < nb) x0 = tr[lane];
@@ -245,12 +275,16 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     };
     TcUnit un{};
     int32_t e0, e1;
-    load_entries(blockIdx.x, un, e0, e1);
-    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+    int u = 0;
+    if (lane == 0) u = (int)atomicAdd(sched, 1u);  // this CTA's first unit
+    u = __shfl_sync(0xffffffffu, u, 0);
+    load_entries(u, un, e0, e1);
+    while (ok && u < num_units) {
       const int nb_unit = (un.t1 - un.t0 + bs - 1) / bs;
-      TcUnit next{};
-      int32_t n0, n1;
-      load_entries(u + gridDim.x, next, n0, n1);
+      // the next unit is drawn now; its value is first needed after this
+      // unit's copies are issued, which hides the atomic's latency
+      int raw_next = 0;
+      if (lane == 0) raw_next = (int)atomicAdd(sched, 1u);
       const int qs = qi & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((qi >> 1) & 1) ^ 1))) { ok = false; break; }
       {  // publish the unit to the MMA lane and the softmax warpgroup
@@ -302,9 +336,18 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         }
         if (!ok) break;
       }
-      e0 = n0;
-      e1 = n1;
-      un = next;
+      u = __shfl_sync(0xffffffffu, raw_next, 0);
+      load_entries(u, un, e0, e1);
+    }
+    if (ok) {  // no work left: publish an empty unit so the consumers stop
+      const int qs = qi & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((qi >> 1) & 1) ^ 1))) {
+        ok = false;
+      } else {
+        if (lane == 0) unit_slots[qs * L::kUnitInts + 5] = 0;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qfull[qs]);
+      }
     }
     if (!ok && lane == 0) {
       raise_error(PA_DEVERR_TIMEOUT);
@@ -344,10 +387,11 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         return true;
       };
       int c = 0, qi = 0, pending = -1;
-      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+      while (ok) {
         const int qs = qi & 1;
         if (!mbar_wait(&qfull[qs], (qi >> 1) & 1)) { ok = false; break; }
         const int nchunks = unit_slots[qs * L::kUnitInts + 5];
+        if (nchunks == 0) break;  // the producer ran out of work
         const uint32_t qb = qbase0 + qs * L::kQ;
         for (int ci = 0; ci < nchunks; ++ci, ++c) {
           const int slot = c % 3;
@@ -453,7 +497,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
 
     const int log2_bs = bs == 8 ? 3 : (bs == 16 ? 4 : 5);
     int c = 0, qi = 0;
-    for (int u = blockIdx.x; u < num_units && !stop; u += gridDim.x, ++qi) {
+    for (; !stop; ++qi) {
       // the unit, as the producer published it with its Q tile
       const int qs = qi & 1;
       if (!bad && !mbar_wait(&qfull[qs], (qi >> 1) & 1)) bad = true;
@@ -468,6 +512,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       un.t1 = us[4];
       un.nchunks = us[5];
       un.single = us[6] != 0;
+      if (un.nchunks == 0) break;  // the producer ran out of work
       const int32_t *ents = us + 8;
       const int tail_end = min(((un.t1 + bs - 1) >> log2_bs) << log2_bs, un.t0 + kPart);
 #pragma unroll
@@ -488,14 +533,16 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         const int tok = un.t0 + ci * L::kChunk + r;
         const int32_t blk = tok < un.t1 ? ents[(tok - un.t0) >> log2_bs] : -1;
         const bool valid = blk >= 0 && blk < p.num_blocks;
+        // Scores are weighed against the running max m as long as no score
+        // exceeds it by more than kLazyRescale (weights stay below 2^8);
+        // only then, warpgroup-wide, is the chunk's exact max taken.  The
+        // result is the same: the softmax does not depend on the reference.
         float x[G];
+        bool need = false;
 #pragma unroll
         for (int n = 0; n < G; ++n) {
           x[n] = (valid && !bad) ? s[n] * p.scale_log2 : -INFINITY;
-          float v = x[n];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-          if (lane == 0) red_max[((c & 1) * 4 + wq) * N + n] = v;
+          need |= x[n] > m[n] + kLazyRescale;
         }
         // a masked row inside the partition's last, partly filled block holds
         // whatever the pool has there: zero its V row before PV reads it
@@ -512,21 +559,37 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
             }
           }
         }
-        stop = wg_sync_or(bad);
-        if (stop) break;
+        float mnew[G];
+        if (wg_sync_or(need || bad)) {  // uniform: some row needs a new reference (or gave up)
+#pragma unroll
+          for (int n = 0; n < G; ++n) {
+            float v = x[n];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+            if (lane == 0) red_max[((c & 1) * 4 + wq) * N + n] = v;
+          }
+          stop = wg_sync_or(bad);
+          if (stop) break;
+#pragma unroll
+          for (int n = 0; n < G; ++n) {
+            float cm = red_max[((c & 1) * 4 + 0) * N + n];
+#pragma unroll
+            for (int w = 1; w < 4; ++w) cm = fmaxf(cm, red_max[((c & 1) * 4 + w) * N + n]);
+            mnew[n] = fmaxf(m[n], cm);
+          }
+        } else {
+#pragma unroll
+          for (int n = 0; n < G; ++n) mnew[n] = m[n];
+        }
         float alpha[G];
         __nv_bfloat16 *pb = reinterpret_cast<__nv_bfloat16 *>(smem + L::kOffP + (c & 1) * L::kP);
         const int kh = r >> 6, rr = r & 63;
 #pragma unroll
         for (int n = 0; n < G; ++n) {
-          float cm = red_max[((c & 1) * 4 + 0) * N + n];
-#pragma unroll
-          for (int w = 1; w < 4; ++w) cm = fmaxf(cm, red_max[((c & 1) * 4 + w) * N + n]);
-          const float mnew = fmaxf(m[n], cm);
-          alpha[n] = (mnew == -INFINITY) ? 1.f : exp2f(m[n] - mnew);
-          const float pv = valid ? exp2f(x[n] - mnew) : 0.f;
+          alpha[n] = (mnew[n] == m[n]) ? 1.f : exp2f(m[n] - mnew[n]);
+          const float pv = valid ? exp2f(x[n] - mnew[n]) : 0.f;
           l[n] = fmaf(l[n], alpha[n], pv);
-          m[n] = mnew;
+          m[n] = mnew[n];
           // P^T row n (K-major, 128-byte swizzle): token r in half kh
           const int off = kh * (N * 64) + (n >> 3) * 512 + (n & 7) * 64 + (((rr >> 3) ^ (n & 7)) << 3) + (rr & 7);
           pb[off] = __float2bfloat16_rn(pv);
@@ -564,6 +627,13 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+  if (threadIdx.x == 0) {  // this CTA draws no more units; the last one out resets the slot
+    __threadfence();
+    if (atomicAdd(&sched[1], 1u) == gridDim.x - 1) {
+      atomicExch(&sched[0], 0u);
+      atomicExch(&sched[1], 0u);
+    }
+  }
   if (warp == 1) tc::tmem_dealloc(tmem, L::kTmemCols);
 }
 

@@ -16,6 +16,21 @@ __device__ int32_t g_error;
 
 __device__ __forceinline__ void raise_error(int32_t bits) { atomicOr(&g_error, bits); }
 
+// Programmatic dependent launch: every kernel of the library is launched so
+// that it may be scheduled before the kernel ahead of it in the stream has
+// finished; it then waits here, before touching any memory, until that
+// kernel has completed and its writes are visible.  Launched without that
+// attribute, the wait returns at once.
+__device__ __forceinline__ void wait_prior_grid() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Lets the kernel that follows in the stream be scheduled now (it still
+// waits for this one to complete before it reads anything).
+__device__ __forceinline__ void allow_next_grid() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

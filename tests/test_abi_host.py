@@ -225,3 +225,13 @@ def test_fragmentation_example_through_the_allocator():
     st = A.stats()
     assert st["allocated_slots"] == 8 and st["used_slots"] == 7
     assert st["fragmentation"] == pytest.approx(0.125)
+
+
+def test_seqs_max_len():
+    A = pa.Allocator(64, 8)
+    s = [A.new_seq() for _ in range(3)]
+    for i, n in zip(s, (5, 30, 17)):
+        A.append(i, n)
+    assert A.max_len(s) == (30, 4)
+    assert A.max_len(s[:1]) == (5, 1)
+    assert A.max_len([]) == (0, 0)
