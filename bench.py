@@ -65,7 +65,7 @@ def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_402_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        if f.startswith("pa_decode") or f == "pa_device.cuh":
+        if f.startswith("pa_decode") or f in ("pa_device.cuh", "pa_tc.cuh"):
             with open(os.path.join(csrc, f), "rb") as fh:
                 h.update(fh.read())
     return h.hexdigest()[:16]

@@ -25,6 +25,14 @@
  *  - Data errors that only the device can see (a slot or a table entry
  *    outside the pool) never trap: the offending element is skipped and a
  *    bit is set in a per-device error word read by pa_read_device_error.
+ *  - A kernel of this library may start while the library kernel ahead of
+ *    it on the same stream is still running (programmatic dependent
+ *    launch); it waits for that kernel before it reads or writes anything
+ *    the kernel may touch.  The one exception: the tensor-core pa_decode
+ *    reads context_lens and block_tables before that wait.  No kernel of the
+ *    library writes int32 tables or lengths, so this only forbids placing
+ *    them in memory that the preceding library call writes (a pool, an
+ *    output or a workspace).
  *
  * Cache layout (both pools):
  *   k_cache, v_cache : [num_blocks][num_kv_heads][block_size][head_dim]

@@ -9,12 +9,12 @@
 // (max, sum, unnormalised accumulator) for the log-sum-exp reduce.
 //
 // How, on sm_100a:
-//  * Persistent grid, one CTA per SM.  Work units are handed out at run time
-//    from a counter (largest first: every full 512-token partition, then the
-//    partial last partition of each sequence), so CTAs that drew short units
-//    take more of them and all finish together.  The counter lives in one of
-//    kSchedSlots library-owned slots, chosen per call, and the last CTA out
-//    resets it.
+//  * Persistent grid, one CTA per SM.  Work units are in largest-first order
+//    (every full 512-token partition, then the partial last partition of each
+//    sequence); CTA i starts with unit i and then draws the next free unit
+//    from a counter once the copies of its current unit are issued, so CTAs
+//    that drew short units take more of them and all finish together.  The counter lives in one of kSchedSlots library-owned
+//    slots, chosen per call, and the last CTA out resets it.
 //  * Warp 0 is the TMA producer.  A unit is cut into chunks of 128 tokens;
 //    each lane loads one block of a chunk: the whole (block, kv head) K tile,
 //    and then the V tile, with ONE 4-D box each (a TMA issue costs about
@@ -29,12 +29,18 @@
 //  * Warp 1 (one lane) issues tcgen05 MMAs: per chunk c,
 //        S^T[128 tok x 16] = K_c[128 tok x 128 d] . Q^T[128 d x 16]   (K-major A and B)
 //        O^T[128 d x 16]   = V_c^T[128 d x 128 tok] . P^T[128 tok x 16] (MN-major A)
-//    with accumulators in tensor memory (S and O double-buffered); the query
-//    rows past G are zero (N = 16 is the smallest N an M = 128 MMA takes).  QK of chunk c is issued before PV of chunk c-1.
+//    with accumulators in tensor memory; the query rows past G are zero
+//    (N = 16 is the smallest N an M = 128 MMA takes).  S is double-buffered
+//    by chunk; O is one accumulator per unit that every PV of the unit adds
+//    to, double-buffered by unit so a unit's output is read while the next
+//    one runs.  QK of chunk c is issued before PV of chunk c-1.
 //  * Warps 2..5 (128 threads) run the softmax on S (thread = token row) and
-//    write P^T in bf16 to shared memory, then merge O of the previous chunk
-//    into fp32 registers (thread = head-dim row), one chunk behind, so the PV
-//    MMA overlaps the next softmax.
+//    write P^T in bf16 to shared memory.  The weights are taken against a
+//    reference max that moves only when a score passes it by 2^8; when it
+//    moves, the same threads (now thread = head-dim row) rescale the unit's O
+//    in tensor memory before the next PV adds to it.  At the end of a unit
+//    (overlapped with the first chunk of the next one) they read O and write
+//    the output or the partition's statistics.
 //  * Every mbarrier wait has an iteration limit; a thread that gives up sets
 //    PA_DEVERR_TIMEOUT and its role stops, the softmax warps leave together
 //    through a reducing barrier, the MMA lane drains its MMAs, and the CTA
@@ -150,13 +156,16 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
 
-  wait_prior_grid();
-  allow_next_grid();
+  // Up to the first unit's table entries, the kernel reads only the lengths
+  // and the block tables, which no kernel of this library writes; it waits
+  // for the kernel ahead of it in the stream (and lets the next one be
+  // scheduled) only after that, so this start-up overlaps the previous
+  // kernel.  Each thread waits before it triggers.
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
   uint64_t *kfull = bars, *kempty = bars + 3, *vfull = bars + 6, *vempty = bars + 9;
   uint64_t *qfull = bars + 12, *qempty = bars + 14, *sfull = bars + 16, *pfull = bars + 18;
-  uint64_t *ofull = bars + 20, *ofree = bars + 22, *drain = bars + 24;
+  uint64_t *pvdone = bars + 20, *ofree = bars + 22, *drain = bars + 24;
   int32_t *prefix = reinterpret_cast<int32_t *>(smem + L::kOffPrefix);
   int32_t *ctx_s = reinterpret_cast<int32_t *>(smem + L::kOffCtx);
   int32_t *scan = reinterpret_cast<int32_t *>(smem + L::kOffScan);
@@ -179,8 +188,8 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       mbar_init(&qempty[i], 2);  // the MMA lane's commit + the softmax warpgroup
       mbar_init(&sfull[i], 1);
       mbar_init(&pfull[i], 128);
-      mbar_init(&ofull[i], 1);
-      mbar_init(&ofree[i], 128);
+      mbar_init(&pvdone[i], 1);  // per chunk parity: the PV MMA of the chunk completed
+      mbar_init(&ofree[i], 128);  // per unit parity: the epilogue read the unit's O
     }
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -207,11 +216,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       // full partitions in the low bits, a partial last partition in the high ones
       cnt[i] = (ok && ctx > 0) ? (ctx / kPart) | ((ctx % kPart != 0 ? 1 : 0) << kFullBits) : 0;
       mine += cnt[i];
-      if (blockIdx.x == 0 && (!ok || ctx == 0)) {  // rows no unit writes: zero them
-        if (!ok) raise_error(PA_DEVERR_LEN);
-        uint4 *o = reinterpret_cast<uint4 *>(out + (size_t)b * p.Hq * 128);
-        for (int e = 0; e < p.Hq * 128 / 8; ++e) o[e] = make_uint4(0, 0, 0, 0);
-      }
+      if (blockIdx.x == 0 && !ok) raise_error(PA_DEVERR_LEN);
     }
   }
   int incl = mine;  // inclusive scan within the warp
@@ -275,16 +280,12 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     };
     TcUnit un{};
     int32_t e0, e1;
-    int u = 0;
-    if (lane == 0) u = (int)atomicAdd(sched, 1u);  // this CTA's first unit
-    u = __shfl_sync(0xffffffffu, u, 0);
+    int u = blockIdx.x;  // the first unit of every CTA is fixed; later ones are drawn
     load_entries(u, un, e0, e1);
+    wait_prior_grid();  // the copies read the pool and Q, which may be written just before
+    allow_next_grid();
     while (ok && u < num_units) {
       const int nb_unit = (un.t1 - un.t0 + bs - 1) / bs;
-      // the next unit is drawn now; its value is first needed after this
-      // unit's copies are issued, which hides the atomic's latency
-      int raw_next = 0;
-      if (lane == 0) raw_next = (int)atomicAdd(sched, 1u);
       const int qs = qi & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((qi >> 1) & 1) ^ 1))) { ok = false; break; }
       {  // publish the unit to the MMA lane and the softmax warpgroup
@@ -336,6 +337,12 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         }
         if (!ok) break;
       }
+      if (!ok) break;
+      // The next unit is drawn only now, with the ring full of this unit's
+      // chunks (which hide the draw's latency): a CTA never holds more work
+      // than that when the queue runs dry, so all CTAs finish together.
+      int raw_next = 0;
+      if (lane == 0) raw_next = (int)gridDim.x + (int)atomicAdd(sched, 1u);
       u = __shfl_sync(0xffffffffu, raw_next, 0);
       load_entries(u, un, e0, e1);
     }
@@ -360,33 +367,43 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    wait_prior_grid();
+    allow_next_grid();
     if (lane == 0) {
       constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(128, N, false, false);
       constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(128, N, true, false);
       const uint32_t kbase0 = smem_u32(smem + L::kOffK), vbase0 = smem_u32(smem + L::kOffV);
       const uint32_t qbase0 = smem_u32(smem + L::kOffQ), pbase0 = smem_u32(smem + L::kOffP);
       bool ok = true;
-      auto issue_pv = [&](int c) -> bool {
+      struct PvJob {
+        int c;       // chunk
+        int u;       // unit (its O accumulator is u & 1)
+        bool first;  // first chunk of the unit: the PV starts the accumulator
+      };
+      auto issue_pv = [&](const PvJob &j) -> bool {
+        const int c = j.c;
         if (!mbar_wait(&pfull[c & 1], (c >> 1) & 1)) return false;
         if (!mbar_wait(&vfull[c % 3], (c / 3) & 1)) return false;
-        if (!mbar_wait(&ofree[c & 1], ((c >> 1) & 1) ^ 1)) return false;
+        // the accumulator is free once the epilogue of the unit two back read it
+        if (j.first && !mbar_wait(&ofree[j.u & 1], ((j.u >> 1) & 1) ^ 1)) return false;
         tc::fence_after_sync();
         const uint32_t vb = vbase0 + (c % 3) * L::kTile;
         const uint32_t pb = pbase0 + (c & 1) * L::kP;
-        const uint32_t d = tmem + 2 * N + (c & 1) * N;
+        const uint32_t d = tmem + 2 * N + (j.u & 1) * N;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           // V^T, MN-major: M = head dim (two 64-wide atoms 1 KiB apart), K = 16
           // tokens = two 8-row groups L::kGroup apart
           const uint64_t a = tc::smem_desc_sw128(vb + kk * 2 * L::kGroup, 1024, L::kGroup);
           const uint64_t bdesc = tc::smem_desc_sw128(pb + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
-          tc::mma_bf16(d, a, bdesc, idesc_pv, kk > 0);
+          tc::mma_bf16(d, a, bdesc, idesc_pv, (kk > 0 || !j.first) ? 1u : 0u);
         }
-        tc::mma_commit(&ofull[c & 1]);
+        tc::mma_commit(&pvdone[c & 1]);
         tc::mma_commit(&vempty[c % 3]);
         return true;
       };
-      int c = 0, qi = 0, pending = -1;
+      int c = 0, qi = 0;
+      PvJob pending{-1, 0, false};
       while (ok) {
         const int qs = qi & 1;
         if (!mbar_wait(&qfull[qs], (qi >> 1) & 1)) { ok = false; break; }
@@ -410,89 +427,93 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
           tc::mma_commit(&sfull[c & 1]);
           tc::mma_commit(&kempty[slot]);
           if (ci == nchunks - 1) tc::mma_commit(&qempty[qs]);
-          if (pending >= 0 && !issue_pv(pending)) { ok = false; break; }
-          pending = c;
+          if (pending.c >= 0 && !issue_pv(pending)) { ok = false; break; }
+          pending = PvJob{c, qi, ci == 0};
         }
         ++qi;
       }
-      if (ok && pending >= 0 && !issue_pv(pending)) ok = false;
+      if (ok && pending.c >= 0 && !issue_pv(pending)) ok = false;
       if (!ok) raise_error(PA_DEVERR_TIMEOUT);
       // no MMA may still be running when the CTA frees its tensor memory
       tc::mma_commit(drain);
       mbar_wait(drain, 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax + merge
+    // ------------------------------------------------------------ softmax + epilogue
+    wait_prior_grid();  // before the first write of out / the workspace
+    allow_next_grid();
     const int wq = warp & 3;              // this warp's quarter of the TMEM lanes
-    const int r = wq * 32 + lane;         // token row (softmax) / head-dim row (merge)
+    const int r = wq * 32 + lane;         // token row (softmax) / head-dim row (O)
+    if (blockIdx.x == 0) {  // rows no unit writes (empty or invalid length): zeros
+      for (int b = r; b < p.B; b += 128) {
+        const int ctx = ctx_s[b];
+        if (ctx <= 0 || ctx > p.max_ctx) {
+          uint4 *o = reinterpret_cast<uint4 *>(out + (size_t)b * p.Hq * 128);
+          for (int e = 0; e < p.Hq * 128 / 8; ++e) o[e] = make_uint4(0, 0, 0, 0);
+        }
+      }
+    }
     const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
     const int bs = p.bs;
-    float m[G], l[G], acc[G], m_done[G], l_done[G], alpha_p[G];
+    float m[G], l[G], m_done[G], l_done[G];
 #pragma unroll
     for (int n = 0; n < G; ++n) {
       m[n] = -INFINITY;
       l[n] = 0.f;
-      acc[n] = 0.f;
       m_done[n] = -INFINITY;
       l_done[n] = 0.f;
-      alpha_p[n] = 1.f;
     }
-    TcUnit pun{};
-    bool pend = false, p_first = false, p_last = false;
-    int pc = 0, nunit = 0;
-    bool bad = false;   // this thread gave up on a wait
-    bool stop = false;  // some thread of the warpgroup did (uniform: from wg_sync_or)
+    TcUnit pun{};        // the unit whose epilogue is pending
+    bool pend = false;
+    int p_clast = 0;     // its last chunk
+    int p_u = 0;         // its index (O accumulator p_u & 1)
+    bool bad = false;    // this warp gave up on a wait (warp-uniform)
+    bool stop = false;   // some warp of the warpgroup did (uniform: from wg_sync_or)
 
-    auto epilogue = [&](const TcUnit &un, int parity) {
-      // L[n]: sum of the per-row partial sums over the 128 threads
-      float Ls[G];
+    // Waits are voted across the warp so that `bad` stays warp-uniform: the
+    // tensor-memory loads and stores after them are warp-collective.
+    auto warp_wait = [&](uint64_t *bar, uint32_t parity) {
+      if (!bad && !__all_sync(0xffffffffu, mbar_wait(bar, parity))) bad = true;
+    };
+
+    // O of unit pun (complete once the PV of its last chunk is) and the
+    // warpgroup-wide sums l -> the output row, or the partition's statistics.
+    auto epilogue = [&]() {
+      float o[8];
+      warp_wait(&pvdone[p_clast & 1], (p_clast >> 1) & 1);
+      if (!bad) {
+        tc::fence_after_sync();
+        tc::tmem_ld8(trow + 2 * N + (p_u & 1) * N, o);
+      }
+      tc::fence_before_sync();
+      mbar_arrive(&ofree[p_u & 1]);
+      const int parity = p_u & 1;
 #pragma unroll
       for (int n = 0; n < G; ++n) {
         float v = l_done[n];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        for (int k = 16; k > 0; k >>= 1) v += __shfl_xor_sync(0xffffffffu, v, k);
         if (lane == 0) red_sum[(parity * 4 + wq) * N + n] = v;
       }
       stop = wg_sync_or(bad);
       if (stop) return;
 #pragma unroll
       for (int n = 0; n < G; ++n) {
-        float sum = 0.f;
+        float Ls = 0.f;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) sum += red_sum[(parity * 4 + w) * N + n];
-        Ls[n] = sum;
-      }
-#pragma unroll
-      for (int n = 0; n < G; ++n) {
-        const int h = un.g * G + n;
-        if (un.single) {
-          out[((size_t)un.b * p.Hq + h) * 128 + r] = __float2bfloat16_rn(Ls[n] > 0.f ? acc[n] / Ls[n] : 0.f);
+        for (int w = 0; w < 4; ++w) Ls += red_sum[(parity * 4 + w) * N + n];
+        const int h = pun.g * G + n;
+        if (pun.single) {
+          out[((size_t)pun.b * p.Hq + h) * 128 + r] = __float2bfloat16_rn(Ls > 0.f ? o[n] / Ls : 0.f);
         } else {
-          const size_t row = ((size_t)un.b * p.Hq + h) * p.max_parts + un.part;
-          p.ws_acc[row * 128 + r] = acc[n];
+          const size_t row = ((size_t)pun.b * p.Hq + h) * p.max_parts + pun.part;
+          p.ws_acc[row * 128 + r] = o[n];
           if (r == 0) {
             p.ws_m[row] = m_done[n];
-            p.ws_l[row] = Ls[n];
+            p.ws_l[row] = Ls;
           }
         }
       }
-    };
-
-    // O of chunk pc into acc (one chunk behind the softmax), then the
-    // epilogue when pc ended its unit.  A failed wait only marks `bad`; the
-    // next warpgroup barrier turns it into a uniform stop.
-    auto merge = [&]() {
-      float o[8];
-      if (!bad && !mbar_wait(&ofull[pc & 1], (pc >> 1) & 1)) bad = true;
-      if (!bad) {
-        tc::fence_after_sync();
-        tc::tmem_ld8(trow + 2 * N + (pc & 1) * N, o);
-#pragma unroll
-        for (int n = 0; n < G; ++n) acc[n] = p_first ? o[n] : fmaf(acc[n], alpha_p[n], o[n]);
-      }
-      tc::fence_before_sync();
-      mbar_arrive(&ofree[pc & 1]);
-      if (p_last) epilogue(pun, nunit & 1);
     };
 
     const int log2_bs = bs == 8 ? 3 : (bs == 16 ? 4 : 5);
@@ -500,7 +521,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     for (; !stop; ++qi) {
       // the unit, as the producer published it with its Q tile
       const int qs = qi & 1;
-      if (!bad && !mbar_wait(&qfull[qs], (qi >> 1) & 1)) bad = true;
+      warp_wait(&qfull[qs], (qi >> 1) & 1);
       stop = wg_sync_or(bad);  // every thread reads the slot, or none does
       if (stop) break;
       const int32_t *us = unit_slots + qs * L::kUnitInts;
@@ -515,6 +536,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       if (un.nchunks == 0) break;  // the producer ran out of work
       const int32_t *ents = us + 8;
       const int tail_end = min(((un.t1 + bs - 1) >> log2_bs) << log2_bs, un.t0 + kPart);
+      const uint32_t obuf = trow + 2 * N + (qi & 1) * N;
 #pragma unroll
       for (int n = 0; n < G; ++n) {
         m_done[n] = m[n];
@@ -523,9 +545,8 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         l[n] = 0.f;
       }
       for (int ci = 0; ci < un.nchunks; ++ci, ++c) {
-        // ---- softmax of chunk c
         float s[8];
-        if (!bad && !mbar_wait(&sfull[c & 1], (c >> 1) & 1)) bad = true;
+        warp_wait(&sfull[c & 1], (c >> 1) & 1);
         if (!bad) {
           tc::fence_after_sync();
           tc::tmem_ld8(trow + (c & 1) * N, s);
@@ -533,10 +554,11 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         const int tok = un.t0 + ci * L::kChunk + r;
         const int32_t blk = tok < un.t1 ? ents[(tok - un.t0) >> log2_bs] : -1;
         const bool valid = blk >= 0 && blk < p.num_blocks;
-        // Scores are weighed against the running max m as long as no score
-        // exceeds it by more than kLazyRescale (weights stay below 2^8);
-        // only then, warpgroup-wide, is the chunk's exact max taken.  The
-        // result is the same: the softmax does not depend on the reference.
+        // Scores are weighed against the running reference m as long as no
+        // score exceeds it by more than kLazyRescale (weights stay below
+        // 2^8); only then, warpgroup-wide, is the chunk's exact max taken.
+        // The result is the same: the softmax does not depend on the
+        // reference.
         float x[G];
         bool need = false;
 #pragma unroll
@@ -546,10 +568,10 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         }
         // a masked row inside the partition's last, partly filled block holds
         // whatever the pool has there: zero its V row before PV reads it
-        if (!bad && tok >= un.t1 && tok < tail_end) {
-          if (!mbar_wait(&vfull[c % 3], (c / 3) & 1)) {
-            bad = true;
-          } else {
+        const bool tail_row = tok >= un.t1 && tok < tail_end;
+        if (__any_sync(0xffffffffu, tail_row)) {
+          warp_wait(&vfull[c % 3], (c / 3) & 1);
+          if (!bad && tail_row) {
             uint4 *vr = reinterpret_cast<uint4 *>(smem + L::kOffV + (c % 3) * L::kTile +
                                                   (r >> 3) * L::kGroup + (r & 7) * 128);
 #pragma unroll
@@ -565,7 +587,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
           for (int n = 0; n < G; ++n) {
             float v = x[n];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+            for (int k = 16; k > 0; k >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, k));
             if (lane == 0) red_max[((c & 1) * 4 + wq) * N + n] = v;
           }
           stop = wg_sync_or(bad);
@@ -582,11 +604,29 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
           for (int n = 0; n < G; ++n) mnew[n] = m[n];
         }
         float alpha[G];
+        bool moved = false;  // uniform: m and mnew are the same in every thread
+#pragma unroll
+        for (int n = 0; n < G; ++n) {
+          moved |= mnew[n] != m[n];
+          alpha[n] = (mnew[n] == m[n]) ? 1.f : exp2f(m[n] - mnew[n]);
+        }
+        if (moved && ci > 0) {
+          // O of this unit holds the chunks before c weighed against the old
+          // reference: rescale it once PV(c-1) has landed, before PV(c) adds
+          warp_wait(&pvdone[(c - 1) & 1], ((c - 1) >> 1) & 1);
+          if (!bad) {
+            float o[8];
+            tc::fence_after_sync();
+            tc::tmem_ld8(obuf, o);
+#pragma unroll
+            for (int n = 0; n < G; ++n) o[n] *= alpha[n];
+            tc::tmem_st8(obuf, o);
+          }
+        }
         __nv_bfloat16 *pb = reinterpret_cast<__nv_bfloat16 *>(smem + L::kOffP + (c & 1) * L::kP);
         const int kh = r >> 6, rr = r & 63;
 #pragma unroll
         for (int n = 0; n < G; ++n) {
-          alpha[n] = (mnew[n] == m[n]) ? 1.f : exp2f(m[n] - mnew[n]);
           const float pv = valid ? exp2f(x[n] - mnew[n]) : 0.f;
           l[n] = fmaf(l[n], alpha[n], pv);
           m[n] = mnew[n];
@@ -598,20 +638,18 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         tc::fence_before_sync();
         mbar_arrive(&pfull[c & 1]);
         if (ci == un.nchunks - 1 && threadIdx.x == 64) mbar_arrive(&qempty[qs]);  // done with the unit slot
-        // ---- merge of chunk c-1
-        if (pend) {
-          merge();
+        // the previous unit's output, while this chunk's PV runs
+        if (ci == 0 && pend) {
+          epilogue();
+          pend = false;
           if (stop) break;
         }
-        pend = true;
-        p_first = ci == 0;
-        p_last = ci == un.nchunks - 1;
-        pun = un;
-        pc = c;
-        if (p_last) ++nunit;
-#pragma unroll
-        for (int n = 0; n < G; ++n) alpha_p[n] = alpha[n];
       }
+      if (stop) break;
+      pend = true;
+      pun = un;
+      p_clast = c - 1;
+      p_u = qi;
     }
     if (pend && !stop) {
 #pragma unroll
@@ -619,7 +657,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         m_done[n] = m[n];
         l_done[n] = l[n];
       }
-      merge();
+      epilogue();
     }
     if (stop) raise_error(PA_DEVERR_TIMEOUT);
   }
