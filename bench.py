@@ -268,6 +268,7 @@ class Instance:
             t1 = time.perf_counter()
             slots, pairs = self.alloc.batch_append(seqs, np.ones(B, np.int32))
             tables, lens = self.alloc.build_block_tables(seqs, self.max_blocks)
+            cow = pa.cow_sources(pairs, tables, lens, bs)
             self.host_alloc_s += time.perf_counter() - t1
             nblk = (lens.astype(np.int64) + bs - 1) // bs
             # unique bytes: every physical block once, with its fill
@@ -279,6 +280,7 @@ class Instance:
                 "seqs": seqs,
                 "slots": torch.from_numpy(slots.copy()).to(dev),
                 "pairs": torch.from_numpy(np.ascontiguousarray(pairs)).to(dev) if len(pairs) else None,
+                "cow": torch.from_numpy(cow).to(dev) if len(pairs) else None,
                 "n_pairs": len(pairs),
                 "tables": torch.from_numpy(tables).to(dev),
                 "lens": torch.from_numpy(lens).to(dev),
@@ -289,7 +291,12 @@ class Instance:
                 "k": synth.normal((B, Hkv, D), dt, seed * 1000 + 11 + 3 * u, device=dev),
                 "v": synth.normal((B, Hkv, D), dt, seed * 1000 + 12 + 3 * u, device=dev),
             }
+            # the decode's bytes: unique K/V, q and out, lengths and table entries
             st["algo_bytes"] = st["kv_unique_bytes"] + 2 * B * Hq * D * 2 + B * 4 + int(nblk.sum()) * 4
+            # the fused step also reads and writes each new row, and reads and
+            # writes each copied block
+            st["algo_bytes_fused"] = (st["algo_bytes"] + 2 * B * Hkv * D * 2 * 2
+                                      + len(pairs) * 2 * bs * Hkv * D * 2 * 2 + (B * 4 if len(pairs) else 0))
             self.steps.append(st)
         top = max(st["max_ctx"] for st in self.steps)
         ws = torch.empty(max(16, pa.pa_decode_workspace_size(B, Hq, top + 64, D)), dtype=torch.uint8, device=dev)
@@ -350,15 +357,21 @@ def run_ours(args, rank: int, world: int, dev):
         inst = insts[s % R]
         st = inst.steps[s // R]
         n = 0
-        if st["pairs"] is not None:
-            pa.pa_copy_blocks(st["pairs"], inst.cache, strm)
+        scale = 1.0 / math.sqrt(wl["D"])
+        if args.unfused:
+            if st["pairs"] is not None:
+                pa.pa_copy_blocks(st["pairs"], inst.cache, strm)
+                n += 1
+            pa.pa_append_kv(st["k"], st["v"], st["slots"], inst.cache, strm)
             n += 1
-        pa.pa_append_kv(st["k"], st["v"], st["slots"], inst.cache, strm)
-        n += 1
         if ev is not None:
             ev[0].record(strm)
-        pa.pa_decode(st["q"], inst.cache, st["tables"], st["lens"], st["max_ctx"], 1.0 / math.sqrt(wl["D"]),
-                     out=st["out"], workspace=st["ws"], stream=strm)
+        if args.unfused:
+            pa.pa_decode(st["q"], inst.cache, st["tables"], st["lens"], st["max_ctx"], scale,
+                         out=st["out"], workspace=st["ws"], stream=strm)
+        else:
+            pa.pa_append_decode(st["k"], st["v"], st["q"], inst.cache, st["tables"], st["lens"], st["max_ctx"],
+                                scale, cow_src=st["cow"], out=st["out"], workspace=st["ws"], stream=strm)
         if ev is not None:
             ev[1].record(strm)
         n += 2 if st["max_ctx"] > pa.PA_PARTITION_TOKENS else 1
@@ -371,8 +384,11 @@ def run_ours(args, rank: int, world: int, dev):
 
     # The K timed steps (inputs precomputed, resident) are captured once into
     # a CUDA graph and replayed, so the host's launch rate does not bound the
-    # device-side measurement.  Each step's decode launch is bracketed by
-    # events captured inside the graph.
+    # device-side measurement.  With the separate calls, each step's decode
+    # call is bracketed by events captured inside the graph; with the fused
+    # call the step is that one call, so its duration is the timed region / K
+    # (events between the steps would only serialise them).
+    per_step_events = args.unfused
     # external: inside a captured graph the records become event-record nodes
     dec_events = [(torch.cuda.Event(enable_timing=True, external=True),
                    torch.cuda.Event(enable_timing=True, external=True)) for _ in range(args.steps)]
@@ -387,12 +403,12 @@ def run_ours(args, rank: int, world: int, dev):
         with torch.cuda.graph(graph):
             cap = torch.cuda.current_stream()
             for i in range(args.steps):
-                n, st = step(args.warmup + i, cap, dec_events[i])
+                n, st = step(args.warmup + i, cap, dec_events[i] if per_step_events else None)
                 launches += n
                 kv_bytes += st["kv_unique_bytes"]
                 kv_logical += st["kv_bytes"]
                 pairs += st["n_pairs"]
-                algo_bytes.append(st["algo_bytes"])
+                algo_bytes.append(st["algo_bytes"] if args.unfused else st["algo_bytes_fused"])
         graph.replay()  # one untimed replay: the graph's own warm-up
         torch.cuda.synchronize()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -405,12 +421,12 @@ def run_ours(args, rank: int, world: int, dev):
             graph.replay()
         else:
             for i in range(args.steps):
-                n, st = step(args.warmup + i, stream, dec_events[i])
+                n, st = step(args.warmup + i, stream, dec_events[i] if per_step_events else None)
                 launches += n
                 kv_bytes += st["kv_unique_bytes"]
                 kv_logical += st["kv_bytes"]
                 pairs += st["n_pairs"]
-                algo_bytes.append(st["algo_bytes"])
+                algo_bytes.append(st["algo_bytes"] if args.unfused else st["algo_bytes_fused"])
         t_end.record(stream)
         torch.cuda.synchronize()
     if graph is not None:
@@ -418,7 +434,7 @@ def run_ours(args, rank: int, world: int, dev):
     if world > 1:
         torch.distributed.barrier()
     ms = t_start.elapsed_time(t_end)
-    dec_ms = [a.elapsed_time(b) for a, b in dec_events]
+    dec_ms = [a.elapsed_time(b) for a, b in dec_events] if per_step_events else [ms / args.steps]
     if pa.pa_read_device_error() != 0:
         raise RuntimeError("device error during the timed steps")
     clocks = clk.summary()
@@ -465,18 +481,24 @@ def run_ours(args, rank: int, world: int, dev):
                    "l2": f"{R} rotating batch instances per rank (KV per step ~{kv_bytes / args.steps / 1e6:.0f} MB, "
                          f"working set ~{R * kv_bytes / args.steps / 1e6:.0f} MB > 126 MB L2)",
                    "parallelism": f"replicas x{world}",
-                   "timing": "eager launches" if args.no_graph else "CUDA graph replay of the K steps"},
+                   "timing": "eager launches" if args.no_graph else "CUDA graph replay of the K steps",
+                   "step": ("pa_copy_blocks + pa_append_kv + pa_decode" if args.unfused else
+                            "pa_append_decode (copy on write + append + decode in one call)")},
         "tokens_per_s": round(tok_all / (ms_all / 1e3), 1),
         "kv_logical_gbs": round(kv_logical * world / 1e9 / (ms_all / 1e3), 2),
         "copy_pairs_per_step": round(pairs / args.steps, 2),
         "kv_frac_of_hbm_peak": round(gb_all / (ms_all / 1e3) / peak, 4),
         "kv_frac_of_8tbs_nominal": round(gb_all / (ms_all / 1e3) / NOMINAL_HBM_GBS, 4),
         "host_alloc_us_per_step": round(host_alloc_us, 2),
-        "roofline": {"bound": "hbm", "kernel": "pa_decode (partition + LSE reduce)",
+        "roofline": {"bound": "hbm",
+                     "kernel": ("pa_decode (partition + LSE reduce)" if args.unfused else
+                                "pa_append_decode (copy + append + partition in one kernel, + LSE reduce)"),
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
                      "traffic": profiled_traffic(args.workload),
                      "decode_us": round(dec_avg_s * 1e6, 2),
+                     "duration_from": ("CUDA events around each decode call in the timed graph" if per_step_events
+                                       else "CUDA events around the K-step timed region / K (one call per step)"),
                      "algo_bytes_per_launch": int(statistics.mean(algo_bytes))},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
@@ -513,6 +535,7 @@ def run_e2e(args, insts, wl, dev, stream):
         "v": torch.empty(B, Hkv, D, dtype=torch.bfloat16).pin_memory(),
         "slots": torch.empty(B, dtype=torch.int64).pin_memory(),
         "pairs": torch.empty(B, 2, dtype=torch.int32).pin_memory(),
+        "cow": torch.empty(B, dtype=torch.int32).pin_memory(),
         "tables": torch.empty(B, mb, dtype=torch.int32).pin_memory(),
         "lens": torch.empty(B, dtype=torch.int32).pin_memory(),
         "out": torch.empty(B, Hq, D, dtype=torch.bfloat16).pin_memory(),
@@ -537,19 +560,28 @@ def run_e2e(args, insts, wl, dev, stream):
         _, pairs = inst.alloc.batch_append(seqs, ones, out_slots=slots_np, out_pairs=pairs_np)
         inst.alloc.build_block_tables(seqs, mb, out_tables=tables_np, out_lens=lens_np)
         npairs = len(pairs)
-        for k in ("q", "k", "v", "slots", "tables", "lens"):
+        names = ("q", "k", "v", "slots", "tables", "lens") if args.unfused else ("q", "k", "v", "tables", "lens")
+        for k in names:
             d[k].copy_(h[k], non_blocking=True)
-        if npairs:
-            d["pairs"][:npairs].copy_(h["pairs"][:npairs], non_blocking=True)
-            pa.pa_copy_blocks(d["pairs"][:npairs], inst.cache, stream)
-        pa.pa_append_kv(d["k"], d["v"], d["slots"], inst.cache, stream)
-        pa.pa_decode(d["q"], inst.cache, d["tables"], d["lens"], int(lens_np.max()), 1.0 / math.sqrt(D), out=out,
-                     workspace=ws, stream=stream)
+        if args.unfused:
+            if npairs:
+                d["pairs"][:npairs].copy_(h["pairs"][:npairs], non_blocking=True)
+                pa.pa_copy_blocks(d["pairs"][:npairs], inst.cache, stream)
+            pa.pa_append_kv(d["k"], d["v"], d["slots"], inst.cache, stream)
+            pa.pa_decode(d["q"], inst.cache, d["tables"], d["lens"], int(lens_np.max()), 1.0 / math.sqrt(D),
+                         out=out, workspace=ws, stream=stream)
+        else:
+            if npairs:
+                pa.cow_sources(pairs, tables_np, lens_np, bs, out=h["cow"].numpy())
+                d["cow"].copy_(h["cow"], non_blocking=True)
+            pa.pa_append_decode(d["k"], d["v"], d["q"], inst.cache, d["tables"], d["lens"], int(lens_np.max()),
+                                1.0 / math.sqrt(D), cow_src=d["cow"] if npairs else None, out=out, workspace=ws,
+                                stream=stream)
         h["out"].copy_(out, non_blocking=True)
         torch.cuda.synchronize()
         if i == 0:
-            h2d = sum(h[k].numel() * h[k].element_size() for k in ("q", "k", "v", "slots", "tables", "lens"))
-            h2d += npairs * 8
+            h2d = sum(h[k].numel() * h[k].element_size() for k in names)
+            h2d += (npairs * 8) if args.unfused else (B * 4 if npairs else 0)
             d2h = h["out"].numel() * h["out"].element_size()
         seen.append((tables_np.copy(), lens_np.copy()))
     seconds = time.perf_counter() - t0
@@ -609,9 +641,12 @@ def run_trace(args, dev):
                 continue
             npr = len(plan.prompt_slots)
             h = [torch.from_numpy(plan.prompt_slots).pin_memory() if npr else None,
-                 torch.from_numpy(plan.decode_slots).pin_memory(),
-                 torch.from_numpy(np.ascontiguousarray(plan.cow_pairs)).pin_memory() if len(plan.cow_pairs) else None,
-                 torch.from_numpy(tables).pin_memory(), torch.from_numpy(lens).pin_memory()]
+                 torch.from_numpy(plan.decode_slots).pin_memory() if args.unfused else None,
+                 (torch.from_numpy(np.ascontiguousarray(plan.cow_pairs)).pin_memory()
+                  if len(plan.cow_pairs) and args.unfused else None),
+                 torch.from_numpy(tables).pin_memory(), torch.from_numpy(lens).pin_memory(),
+                 (torch.from_numpy(pa.cow_sources(plan.cow_pairs, tables, lens, bs)).pin_memory()
+                  if len(plan.cow_pairs) and not args.unfused else None)]
             d_ = [x.to(dev, non_blocking=True) if x is not None else None for x in h]
             ev[s_][0].record(stream)
             if npr:
@@ -619,18 +654,23 @@ def run_trace(args, dev):
                 kk = src[i0:i0 + npr]
                 pa.pa_append_kv(kk, kk, d_[0], cache, stream)
                 launches += 1
-            if d_[2] is not None:
-                pa.pa_copy_blocks(d_[2], cache, stream)
-                launches += 1
             kd = src[(s_ * 131) % ((1 << 16) - n):][:n]
-            pa.pa_append_kv(kd, kd, d_[1], cache, stream)
             need = pa.pa_decode_workspace_size(n, Hq, max_ctx, D)
             if need > ws.numel():
                 ws = torch.empty(need * 5 // 4, dtype=torch.uint8, device=dev)
             q = qsrc[:n] if n <= 8192 else synth.normal((n, Hq, D), dt, s_, device=dev)
             o = out[:n] if n <= 8192 else torch.empty(n, Hq, D, dtype=dt, device=dev)
-            pa.pa_decode(q, cache, d_[3], d_[4], max_ctx, 1 / math.sqrt(D), out=o, workspace=ws, stream=stream)
-            launches += 2 + (1 if max_ctx > pa.PA_PARTITION_TOKENS else 0)
+            if args.unfused:
+                if d_[2] is not None:
+                    pa.pa_copy_blocks(d_[2], cache, stream)
+                    launches += 1
+                pa.pa_append_kv(kd, kd, d_[1], cache, stream)
+                pa.pa_decode(q, cache, d_[3], d_[4], max_ctx, 1 / math.sqrt(D), out=o, workspace=ws, stream=stream)
+                launches += 2 + (1 if max_ctx > pa.PA_PARTITION_TOKENS else 0)
+            else:
+                pa.pa_append_decode(kd, kd, q, cache, d_[3], d_[4], max_ctx, 1 / math.sqrt(D), cow_src=d_[5],
+                                    out=o, workspace=ws, stream=stream)
+                launches += 1 + (1 if max_ctx > pa.PA_PARTITION_TOKENS else 0)
             ev[s_][1].record(stream)
             res = o[:1].to("cpu", non_blocking=True)
             torch.cuda.synchronize()
@@ -778,6 +818,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rotate", type=int, default=0, help="batch instances to rotate (0: the workload's default)")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly instead of from a CUDA graph")
+    ap.add_argument("--unfused", action="store_true",
+                    help="run each step as pa_copy_blocks + pa_append_kv + pa_decode instead of pa_append_decode")
     ap.add_argument("--block-size", type=int, default=0, help="trace workload: one block size (0: 8, 16 and 32)")
     ap.add_argument("--trace-steps", type=int, default=1000)
     ap.add_argument("--seed", type=int, default=5)

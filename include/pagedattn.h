@@ -137,6 +137,40 @@ PA_API pa_status pa_decode(const void *q, const pa_cache_t *cache, const int32_t
                            float scale, void *out, void *workspace, size_t workspace_bytes,
                            void *stream);
 
+/*
+ * One decode step in one call: for every sequence b, the copy-on-write copy
+ * of its last block (when cow_src asks for one), the append of its newest
+ * token, and pa_decode over the updated pool.  The pages describe the three
+ * as the steps a sequence takes when it grows ("Fixed-Size KV Blocks": a
+ * token goes into the current block; glossary paragraph 5: a shared block is
+ * copied when a sharer writes into it).  The result (pool and out) is
+ * bit-for-bit that of
+ *   pa_copy_blocks({cow_src[b], T_b[(len_b-1)/bs]} for every b with cow_src[b] >= 0)
+ *   pa_append_kv(k_new, v_new, {T_b[(len_b-1)/bs]*bs + (len_b-1)%bs})
+ *   pa_decode(q, ..., out)
+ * with T_b the block table of b and len_b = context_lens[b]; on the
+ * tensor-core path it is one launch (plus the log-sum-exp reduce), the
+ * append and copy done by the CTA that reads the block afterwards.
+ *   k_new, v_new  device [num_seqs][num_kv_heads][head_dim], cache dtype:
+ *                 the key/value rows of token len_b - 1 of sequence b
+ *   cow_src       device [num_seqs] int32, or NULL for no copies: a block
+ *                 whose tiles (every kv head) are first copied over b's last
+ *                 block, -1 for none.  A source outside the pool sets
+ *                 PA_DEVERR_PAIR and is skipped.
+ *   the rest      as pa_decode.
+ * A sequence with len_b = 0 (or an invalid length) appends nothing.  Two
+ * sequences must not have the same last block (a block that several
+ * sequences share is copied for all writers but one), and a copy's source
+ * must not be another sequence's copy destination.
+ */
+PA_API pa_status pa_append_decode(const void *k_new, const void *v_new, const int32_t *cow_src,
+                                  const void *q, const pa_cache_t *cache,
+                                  const int32_t *block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t *context_lens, int32_t num_seqs,
+                                  int32_t num_q_heads, int32_t max_context_len, float scale,
+                                  void *out, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
 /* Bytes of workspace pa_decode needs for these sizes (0 when no context is
  * longer than one partition). */
 PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
@@ -279,6 +313,18 @@ PA_API pa_status pa_alloc_stats(pa_allocator *a, int64_t *used_slots, int64_t *a
 
 /* Reference count of a physical block. */
 PA_API pa_status pa_block_refcount(pa_allocator *a, int32_t block, int32_t *refcount);
+
+/*
+ * The per-sequence form of a decode step's copy pairs, as pa_append_decode
+ * takes it: cow_src_host[i] = the source of the pair whose destination is
+ * last_blocks_host[i] (sequence i's last block after its append; -1 when it
+ * has none), else -1.  PA_ERR_INVALID_ARG when a destination repeats or a
+ * pair's destination is no sequence's last block (a pair the one-token step
+ * cannot make).
+ */
+PA_API pa_status pa_cow_sources(const int32_t *pairs_host, int32_t n_pairs,
+                                const int32_t *last_blocks_host, int32_t n_seqs,
+                                int32_t *cow_src_host);
 
 #ifdef __cplusplus
 }

@@ -60,6 +60,8 @@ def _load() -> ctypes.CDLL:
         "pa_decode": (st, [vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp, sz, vp]),
         "pa_decode_workspace_size": (sz, [i32, i32, i32, i32]),
         "pa_decode_static_workspace": (st, [vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp]),
+        "pa_append_decode": (st, [vp, vp, vp, vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp, sz, vp]),
+        "pa_cow_sources": (st, [i32p, i32, i32p, i32, i32p]),
         "pa_copy_blocks": (st, [vp, i32, cp, vp]),
         "pa_check_copy_pairs": (st, [i32p, i32, i32]),
         "pa_read_device_error": (st, [vp, i32p]),
@@ -210,6 +212,56 @@ def pa_decode(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor, conte
                           int(max_context_len), float(scale), _dev(out, "out", cache.dtype), ws_ptr, ws_bytes,
                           _stream_ptr(stream)), "pa_decode")
     return out
+
+
+def pa_append_decode(k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor, cache: KVCache,
+                     block_tables: torch.Tensor, context_lens: torch.Tensor, max_context_len: int, scale: float,
+                     cow_src: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """One decode step in one call: per sequence b, the copy of block
+    cow_src[b] over b's last block (cow_src int32 [B], -1 for none; None for
+    no copies), the append of b's newest token (k_new, v_new [B, Hkv, D],
+    written at position context_lens[b] - 1 through b's block table) and the
+    decode.  Returns out [B, Hq, D]."""
+    B, Hq, D = q.shape
+    if D != cache.head_dim:
+        raise ValueError("head_dim mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("block_tables must be [B, max_blocks] and context_lens [B]")
+    row_shape = (B, cache.num_kv_heads, D)
+    if tuple(k_new.shape) != row_shape or tuple(v_new.shape) != row_shape:
+        raise ValueError(f"k_new and v_new must be {list(row_shape)}")
+    if cow_src is not None and cow_src.shape != (B,):
+        raise ValueError("cow_src must be [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    need = pa_decode_workspace_size(B, Hq, int(max_context_len), D)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.pa_append_decode(
+        _dev(k_new, "k_new", cache.dtype), _dev(v_new, "v_new", cache.dtype),
+        _dev(cow_src, "cow_src", torch.int32) if cow_src is not None else None,
+        _dev(q, "q", cache.dtype), cache.ref(), _dev(block_tables, "block_tables", torch.int32),
+        block_tables.shape[1], _dev(context_lens, "context_lens", torch.int32), B, Hq, int(max_context_len),
+        float(scale), _dev(out, "out", cache.dtype), ws_ptr, ws_bytes, _stream_ptr(stream)), "pa_append_decode")
+    return out
+
+
+def cow_sources(pairs, tables: np.ndarray, lens: np.ndarray, block_size: int,
+                out: np.ndarray | None = None) -> np.ndarray:
+    """Host: the per-sequence copy sources pa_append_decode takes, from a
+    step's copy pairs [k, 2] and the host tables / lengths after the append."""
+    pairs = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+    tables = np.asarray(tables, dtype=np.int32)
+    lens = np.asarray(lens, dtype=np.int32)
+    n = len(lens)
+    col = np.maximum(lens - 1, 0) // int(block_size)
+    last = np.ascontiguousarray(np.where(lens > 0, tables[np.arange(n), col], -1).astype(np.int32))
+    res = out if out is not None else np.empty(n, dtype=np.int32)
+    _check(_lib.pa_cow_sources(_i32p(pairs), pairs.shape[0], _i32p(last), n, _i32p(res)), "pa_cow_sources")
+    return res
 
 
 PA_STATIC_WORKSPACE_BYTES = 8 << 20

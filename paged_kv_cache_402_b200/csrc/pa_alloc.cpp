@@ -19,6 +19,7 @@
 #include <cstdint>
 #include <cstring>
 #include <new>
+#include <unordered_map>
 #include <vector>
 
 #include "pagedattn.h"
@@ -306,6 +307,29 @@ PA_API pa_status pa_block_refcount(pa_allocator *a, int32_t block, int32_t *refc
   if (!a || !refcount || block < 0 || block >= a->num_blocks) return PA_ERR_INVALID_ARG;
   *refcount = a->ref[block];
   return PA_OK;
+}
+
+PA_API pa_status pa_cow_sources(const int32_t *pairs_host, int32_t n_pairs,
+                                const int32_t *last_blocks_host, int32_t n_seqs,
+                                int32_t *cow_src_host) {
+  if (n_pairs < 0 || n_seqs < 0 || (n_pairs > 0 && !pairs_host) ||
+      (n_seqs > 0 && (!last_blocks_host || !cow_src_host)))
+    return PA_ERR_INVALID_ARG;
+  std::unordered_map<int32_t, int32_t> src_of;  // destination -> source
+  src_of.reserve((size_t)n_pairs * 2);
+  for (int32_t i = 0; i < n_pairs; ++i)
+    if (!src_of.emplace(pairs_host[2 * i + 1], pairs_host[2 * i]).second) return PA_ERR_INVALID_ARG;
+  int32_t matched = 0;
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    cow_src_host[i] = -1;
+    if (last_blocks_host[i] < 0) continue;
+    auto it = src_of.find(last_blocks_host[i]);
+    if (it == src_of.end()) continue;
+    cow_src_host[i] = it->second;
+    src_of.erase(it);  // one writer per destination
+    ++matched;
+  }
+  return matched == n_pairs ? PA_OK : PA_ERR_INVALID_ARG;
 }
 
 }  // extern "C"

@@ -247,6 +247,11 @@ pa_status launch_decode_tc_g(const pa::DecodeParams &p, int32_t max_parts, cudaS
     ps.out = static_cast<__nv_bfloat16 *>(p.out) + rows * 128;
     ps.tables = p.tables + (size_t)b0 * p.max_blocks;
     ps.lens = p.lens + b0;
+    if (p.k_new) {  // fused step: the slice's new rows and copy sources
+      ps.k_new = static_cast<const __nv_bfloat16 *>(p.k_new) + (size_t)b0 * p.Hkv * 128;
+      ps.v_new = static_cast<const __nv_bfloat16 *>(p.v_new) + (size_t)b0 * p.Hkv * 128;
+      if (p.cow_src) ps.cow_src = p.cow_src + b0;
+    }
     if (p.ws_m) {
       ps.ws_m = p.ws_m + rows * max_parts;
       ps.ws_l = p.ws_l + rows * max_parts;
@@ -351,16 +356,26 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
   return workspace_bytes_for(num_seqs, num_q_heads, max_context_len, head_dim);
 }
 
-PA_API pa_status pa_decode(const void *q, const pa_cache_t *cache, const int32_t *block_tables,
-                           int32_t max_blocks_per_seq, const int32_t *context_lens,
-                           int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len,
-                           float scale, void *out, void *workspace, size_t workspace_bytes,
-                           void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Checks pa_decode's arguments and fills the kernel parameters.  *skip is
+// set when there is nothing to launch (no sequences).
+pa_status prepare_decode(const void *q, const pa_cache_t *cache, const int32_t *block_tables,
+                         int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
+                         int32_t num_q_heads, int32_t max_context_len, float scale, void *out,
+                         void *workspace, size_t workspace_bytes, pa::DecodeParams *pp,
+                         bool *skip) {
+  *skip = false;
   pa_status s = check_cache(cache);
   if (s != PA_OK) return s;
   if (num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0 || max_blocks_per_seq < 0)
     return PA_ERR_INVALID_ARG;
-  if (num_seqs == 0) return PA_OK;
+  if (num_seqs == 0) {
+    *skip = true;
+    return PA_OK;
+  }
   if (!q || !out || !block_tables || !context_lens || !aligned16(q) || !aligned16(out))
     return PA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
@@ -402,10 +417,64 @@ PA_API pa_status pa_decode(const void *q, const pa_cache_t *cache, const int32_t
   p.max_ctx = max_context_len;
   p.max_parts = max_parts;
   p.scale_log2 = scale * 1.4426950408889634f;
+  *pp = p;
+  return PA_OK;
+}
+
+pa_status launch_decode_any(const pa::DecodeParams &p, const pa_cache_t *cache, cudaStream_t st) {
+  if (tc_eligible(p, cache->dtype, cache->head_dim)) return launch_decode_tc(p, p.max_parts, st);
+  if (cache->dtype == PA_DTYPE_F32) return launch_decode_dtype<float>(p, cache->head_dim, p.max_parts, st);
+  return launch_decode_dtype<__nv_bfloat16>(p, cache->head_dim, p.max_parts, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+PA_API pa_status pa_decode(const void *q, const pa_cache_t *cache, const int32_t *block_tables,
+                           int32_t max_blocks_per_seq, const int32_t *context_lens,
+                           int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len,
+                           float scale, void *out, void *workspace, size_t workspace_bytes,
+                           void *stream) {
+  pa::DecodeParams p{};
+  bool skip = false;
+  const pa_status s = prepare_decode(q, cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                                     num_q_heads, max_context_len, scale, out, workspace,
+                                     workspace_bytes, &p, &skip);
+  if (s != PA_OK || skip) return s;
+  return launch_decode_any(p, cache, (cudaStream_t)stream);
+}
+
+PA_API pa_status pa_append_decode(const void *k_new, const void *v_new, const int32_t *cow_src,
+                                  const void *q, const pa_cache_t *cache,
+                                  const int32_t *block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t *context_lens, int32_t num_seqs,
+                                  int32_t num_q_heads, int32_t max_context_len, float scale,
+                                  void *out, void *workspace, size_t workspace_bytes,
+                                  void *stream) {
+  pa::DecodeParams p{};
+  bool skip = false;
+  pa_status s = prepare_decode(q, cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                               num_q_heads, max_context_len, scale, out, workspace, workspace_bytes,
+                               &p, &skip);
+  if (s != PA_OK || skip) return s;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return PA_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
-  if (tc_eligible(p, cache->dtype, cache->head_dim)) return launch_decode_tc(p, max_parts, st);
-  if (cache->dtype == PA_DTYPE_F32) return launch_decode_dtype<float>(p, cache->head_dim, max_parts, st);
-  return launch_decode_dtype<__nv_bfloat16>(p, cache->head_dim, max_parts, st);
+  if (tc_eligible(p, cache->dtype, cache->head_dim)) {
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.cow_src = cow_src;
+    return launch_decode_tc(p, p.max_parts, st);
+  }
+  // the CUDA-core decode does not append: a small kernel does it first
+  const int row_vecs = cache->head_dim * elem_bytes(cache->dtype) / 16;
+  const int64_t warps = (int64_t)num_seqs * cache->num_kv_heads;
+  s = launch(pa::append_newest_kernel, dim3((unsigned)((warps * 32 + 255) / 256)), dim3(256), 0, st,
+             (const uint4 *)k_new, (const uint4 *)v_new, cow_src, block_tables, context_lens,
+             max_blocks_per_seq, num_seqs, cache->num_kv_heads, cache->block_size, row_vecs,
+             cache->num_blocks, max_context_len, (uint4 *)cache->k, (uint4 *)cache->v);
+  if (s != PA_OK) return s;
+  return launch_decode_any(p, cache, st);
 }
 
 // ---------------------------------------------------------------------------

@@ -47,6 +47,56 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// The per-sequence half of a fused decode step, for the decode kernels that
+// do not do it themselves: one warp per (sequence b, kv head g) first copies
+// the (block, g) tile of the copy-on-write source cow_src[b] (if >= 0) over
+// the same tile of b's last block, then writes the rows of b's newest token
+// (position lens[b] - 1) there.  A sequence with an empty or invalid length
+// appends nothing; a last-block entry outside the pool is left to the decode
+// (which flags it); a source outside the pool sets PA_DEVERR_PAIR.
+__global__ void __launch_bounds__(256)
+    append_newest_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
+                         const int32_t *__restrict__ cow_src, const int32_t *__restrict__ tables,
+                         const int32_t *__restrict__ lens, int32_t max_blocks, int32_t B,
+                         int32_t Hkv, int32_t bs, int32_t row_vecs, int32_t num_blocks,
+                         int32_t max_ctx, uint4 *kc, uint4 *vc) {
+  wait_prior_grid();
+  allow_next_grid();
+  const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= (int64_t)B * Hkv) return;
+  const int b = (int)(wid / Hkv), g = (int)(wid % Hkv);
+  const int ctx = lens[b];
+  if (ctx <= 0 || ctx > max_ctx) return;
+  const int pos = ctx - 1;
+  const int32_t blk = tables[(int64_t)b * max_blocks + pos / bs];
+  if (blk < 0 || blk >= num_blocks) return;
+  const int64_t tile_vecs = (int64_t)bs * row_vecs;
+  const int64_t dst = ((int64_t)blk * Hkv + g) * tile_vecs;
+  if (cow_src) {
+    const int32_t src = cow_src[b];
+    if (src >= num_blocks) {
+      if (lane == 0) raise_error(PA_DEVERR_PAIR);
+    } else if (src >= 0) {
+      const int64_t s0 = ((int64_t)src * Hkv + g) * tile_vecs;
+      for (int64_t e = lane; e < tile_vecs; e += 32) {
+        const uint4 a = kc[s0 + e], c = vc[s0 + e];
+        kc[dst + e] = a;
+        vc[dst + e] = c;
+      }
+    }
+    __syncwarp();
+  }
+  const int64_t row = dst + (int64_t)(pos % bs) * row_vecs;
+  const int64_t src_row = ((int64_t)b * Hkv + g) * row_vecs;
+  for (int e = lane; e < 2 * row_vecs; e += 32) {
+    if (e < row_vecs)
+      kc[row + e] = k_new[src_row + e];
+    else
+      vc[row + e - row_vecs] = v_new[src_row + e - row_vecs];
+  }
+}
+
 // grid.x covers one block's vectors, grid.y = pairs.  Each thread moves
 // kUnroll vectors of each pool, all loads issued before the stores.
 constexpr int kCopyUnroll = 4;

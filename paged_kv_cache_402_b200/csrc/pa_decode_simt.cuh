@@ -39,6 +39,11 @@ struct DecodeParams {
   int32_t num_blocks, Hkv, bs, Hq, G, max_blocks, B, max_ctx, max_parts;
   int32_t sched_slot;  // tensor-core kernel: which run-time work counter this call uses
   float scale_log2;  // scale * log2(e)
+  // fused step (tensor-core kernel): the newest token's rows [B][Hkv][D] and
+  // the per-sequence copy-on-write source block (-1: none); null otherwise
+  const void *k_new;
+  const void *v_new;
+  const int32_t *cow_src;
 };
 
 constexpr int kPart = PA_PARTITION_TOKENS;

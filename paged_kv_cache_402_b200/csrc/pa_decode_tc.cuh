@@ -41,6 +41,14 @@
 //    in tensor memory before the next PV adds to it.  At the end of a unit
 //    (overlapped with the first chunk of the next one) they read O and write
 //    the output or the partition's statistics.
+//  * Fused step (k_new set): the unit that holds a sequence's newest token
+//    (its last partition, once per kv head) loads the sequence's last block
+//    from the copy-on-write source when there is one (the rows before the
+//    new one are the same); the MMA warp writes the new key/value row into
+//    the landed K and V tiles before the MMAs read them, and stores it to
+//    the pool; the producer copies the source tile over the destination
+//    after issuing the unit's loads.  No copy of this call reads what those
+//    stores write, so nothing waits for them.
 //  * Every mbarrier wait has an iteration limit; a thread that gives up sets
 //    PA_DEVERR_TIMEOUT and its role stops, the softmax warps leave together
 //    through a reducing barrier, the MMA lane drains its MMAs, and the CTA
@@ -73,7 +81,8 @@ struct TcLayout {
   static constexpr int kOffRedSum = kOffRed + kRedFloats * 4;
   static constexpr int kOffTmem = kOffRedSum + kRedFloats * 4;
   // per-unit description written by the producer next to the unit's Q slot:
-  // [b, g, part, t0, t1, nchunks, single, pad] + the unit's table entries
+  // [b, g, part, t0, t1, nchunks, single, newest-token block or -1] + the
+  // unit's table entries (as the copies read them)
   static constexpr int kUnitInts = 8 + kPart / 8;
   static constexpr int kOffUnit = kOffTmem + 16;
   static constexpr int kOffScan = kOffUnit + 2 * kUnitInts * 4;  // 8 ints
@@ -266,22 +275,74 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     const int oob_group = p.num_blocks * p.Hkv * (bs / 8);  // first 8-row group past the pool
     int c = 0, qi = 0;
     bool ok = true;
-    // a unit's table entries (at most 512 / 8 = 64), loaded by the lanes
-    // right after the previous unit's copies are issued
-    auto load_entries = [&](int u, TcUnit &nu, int32_t &x0, int32_t &x1) {
+    // A unit's table entries (at most 512 / 8 = 64), loaded by the lanes
+    // right after the previous unit's copies are issued.  In a fused step a
+    // unit that holds its sequence's newest token (position t1 - 1) also gets
+    // that token's block nd and the block ns to copy over it (-1: none); its
+    // loads then read the last block from ns.
+    auto load_entries = [&](int u, TcUnit &nu, int32_t &x0, int32_t &x1, int32_t &nd, int32_t &ns) {
       x0 = x1 = -1;
+      nd = ns = -1;
       if (u < num_units) {
         nu = tc_unit_at(p, prefix, ctx_s, u, num_full);
         const int32_t *tr = p.tables + (size_t)nu.b * p.max_blocks + nu.t0 / bs;
         const int nb = (nu.t1 - nu.t0 + bs - 1) / bs;
+        const bool newest = p.k_new != nullptr && nu.t1 == ctx_s[nu.b];
+        const int32_t src = (newest && p.cow_src != nullptr) ? p.cow_src[nu.b] : -1;
         if (lane < nb) x0 = tr[lane];
         if (lane + 32 < nb) x1 = tr[lane + 32];
+        if (newest) {
+          const int jl = (nu.t1 - 1 - nu.t0) / bs;
+          const int32_t blk = __shfl_sync(0xffffffffu, jl < 32 ? x0 : x1, jl & 31);
+          if (blk >= 0 && blk < p.num_blocks) {  // else its copy flags PA_DEVERR_TABLE
+            nd = blk;
+            if (src >= p.num_blocks) {
+              if (lane == 0) raise_error(PA_DEVERR_PAIR);
+            } else if (src >= 0) {
+              ns = src;
+              if (lane == (jl & 31)) {
+                if (jl < 32) x0 = src; else x1 = src;
+              }
+            }
+          }
+        }
+      }
+    };
+    // Copy on write of the newest token's block: the source tile over the
+    // destination's, every row but the new one (the MMA warp stores that).
+    // Nothing in this call reads the destination, so nothing waits for it.
+    auto cow_copy = [&](const TcUnit &un, int32_t dst, int32_t src) {
+      constexpr int kRowVecs = 16;  // one bf16 row of 128 in 16-byte vectors
+      const int tile_vecs = bs * kRowVecs;
+      const int off = (un.t1 - 1) % bs;
+      const uint4 *ks = static_cast<const uint4 *>(p.k) + ((size_t)src * p.Hkv + un.g) * tile_vecs;
+      const uint4 *vs = static_cast<const uint4 *>(p.v) + ((size_t)src * p.Hkv + un.g) * tile_vecs;
+      uint4 *kd = static_cast<uint4 *>(const_cast<void *>(p.k)) + ((size_t)dst * p.Hkv + un.g) * tile_vecs;
+      uint4 *vd = static_cast<uint4 *>(const_cast<void *>(p.v)) + ((size_t)dst * p.Hkv + un.g) * tile_vecs;
+      for (int base = 0; base < tile_vecs; base += 32 * 8) {
+        uint4 a[8], b8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int i = base + k * 32 + lane;
+          if (i < tile_vecs) {
+            a[k] = ks[i];
+            b8[k] = vs[i];
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int i = base + k * 32 + lane;
+          if (i < tile_vecs && (i >> 4) != off) {
+            kd[i] = a[k];
+            vd[i] = b8[k];
+          }
+        }
       }
     };
     TcUnit un{};
-    int32_t e0, e1;
+    int32_t e0, e1, nd, ns;
     int u = blockIdx.x;  // the first unit of every CTA is fixed; later ones are drawn
-    load_entries(u, un, e0, e1);
+    load_entries(u, un, e0, e1, nd, ns);
     wait_prior_grid();  // the copies read the pool and Q, which may be written just before
     allow_next_grid();
     while (ok && u < num_units) {
@@ -298,6 +359,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
           us[4] = un.t1;
           us[5] = un.nchunks;
           us[6] = un.single;
+          us[7] = nd;
         }
         us[8 + lane] = e0;
         if (L::kUnitInts > 8 + 32 + lane) us[8 + 32 + lane] = e1;
@@ -338,13 +400,14 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         if (!ok) break;
       }
       if (!ok) break;
+      if (ns >= 0) cow_copy(un, nd, ns);
       // The next unit is drawn only now, with the ring full of this unit's
       // chunks (which hide the draw's latency): a CTA never holds more work
       // than that when the queue runs dry, so all CTAs finish together.
       int raw_next = 0;
       if (lane == 0) raw_next = (int)gridDim.x + (int)atomicAdd(sched, 1u);
       u = __shfl_sync(0xffffffffu, raw_next, 0);
-      load_entries(u, un, e0, e1);
+      load_entries(u, un, e0, e1, nd, ns);
     }
     if (ok) {  // no work left: publish an empty unit so the consumers stop
       const int qs = qi & 1;
@@ -367,25 +430,52 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Lane 0 issues the MMAs and their commits; the whole warp polls the
+    // waits (voted).  In a fused step the lanes also write the newest token's
+    // key row (lanes 0-15, 16 bytes each, once the K tile has landed, before
+    // the QK MMA) and value row (lanes 16-31, once the V tile has landed,
+    // before the PV MMA) into the tiles of its chunk, and store them to the
+    // pool.
     wait_prior_grid();
     allow_next_grid();
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(128, N, false, false);
-      constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(128, N, true, false);
-      const uint32_t kbase0 = smem_u32(smem + L::kOffK), vbase0 = smem_u32(smem + L::kOffV);
-      const uint32_t qbase0 = smem_u32(smem + L::kOffQ), pbase0 = smem_u32(smem + L::kOffP);
-      bool ok = true;
-      struct PvJob {
-        int c;       // chunk
-        int u;       // unit (its O accumulator is u & 1)
-        bool first;  // first chunk of the unit: the PV starts the accumulator
-      };
-      auto issue_pv = [&](const PvJob &j) -> bool {
-        const int c = j.c;
-        if (!mbar_wait(&pfull[c & 1], (c >> 1) & 1)) return false;
-        if (!mbar_wait(&vfull[c % 3], (c / 3) & 1)) return false;
-        // the accumulator is free once the epilogue of the unit two back read it
-        if (j.first && !mbar_wait(&ofree[j.u & 1], ((j.u >> 1) & 1) ^ 1)) return false;
+    constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(128, N, false, false);
+    constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(128, N, true, false);
+    const uint32_t kbase0 = smem_u32(smem + L::kOffK), vbase0 = smem_u32(smem + L::kOffV);
+    const uint32_t qbase0 = smem_u32(smem + L::kOffQ), pbase0 = smem_u32(smem + L::kOffP);
+    bool ok = true;
+    auto warp_wait = [&](uint64_t *bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+    };
+    // smem offset of the 16-byte piece `piece` of column half `half` of row
+    // r in a K or V tile: 8-row group r / 8, half at +1 KiB, row r % 8 of
+    // the 1 KiB swizzle atom, piece j at position j ^ (r % 8)
+    auto tile_piece = [](int r, int half, int piece) {
+      return (r >> 3) * L::kGroup + half * 1024 + (r & 7) * 128 + ((piece ^ (r & 7)) << 4);
+    };
+    struct PvJob {
+      int c;       // chunk
+      int u;       // unit (its O accumulator is u & 1)
+      bool first;  // first chunk of the unit: the PV starts the accumulator
+      int patch;   // row of the newest token in this chunk, or -1
+      uint4 vrow;  // lanes 16-31: their 16 bytes of its value row
+      uint4 *pool; // lanes 16-31: where those go in the pool
+    };
+    auto issue_pv = [&](const PvJob &j) -> bool {
+      const int c = j.c;
+      if (!warp_wait(&pfull[c & 1], (c >> 1) & 1)) return false;
+      if (!warp_wait(&vfull[c % 3], (c / 3) & 1)) return false;
+      // the accumulator is free once the epilogue of the unit two back read it
+      if (j.first && !warp_wait(&ofree[j.u & 1], ((j.u >> 1) & 1) ^ 1)) return false;
+      if (j.patch >= 0) {
+        if (lane >= 16) {
+          const int off = tile_piece(j.patch, (lane >> 3) & 1, lane & 7);
+          *reinterpret_cast<uint4 *>(smem + L::kOffV + (c % 3) * L::kTile + off) = j.vrow;
+          fence_proxy_async_smem();  // before the PV MMA reads the tile
+          *j.pool = j.vrow;
+        }
+        __syncwarp();
+      }
+      if (lane == 0) {
         tc::fence_after_sync();
         const uint32_t vb = vbase0 + (c % 3) * L::kTile;
         const uint32_t pb = pbase0 + (c & 1) * L::kP;
@@ -400,19 +490,48 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         }
         tc::mma_commit(&pvdone[c & 1]);
         tc::mma_commit(&vempty[c % 3]);
-        return true;
-      };
-      int c = 0, qi = 0;
-      PvJob pending{-1, 0, false};
-      while (ok) {
-        const int qs = qi & 1;
-        if (!mbar_wait(&qfull[qs], (qi >> 1) & 1)) { ok = false; break; }
-        const int nchunks = unit_slots[qs * L::kUnitInts + 5];
-        if (nchunks == 0) break;  // the producer ran out of work
-        const uint32_t qb = qbase0 + qs * L::kQ;
-        for (int ci = 0; ci < nchunks; ++ci, ++c) {
-          const int slot = c % 3;
-          if (!mbar_wait(&kfull[slot], (c / 3) & 1)) { ok = false; break; }
+      }
+      __syncwarp();
+      return true;
+    };
+    int c = 0, qi = 0;
+    PvJob pending{-1, 0, false, -1, make_uint4(0, 0, 0, 0), nullptr};
+    while (ok) {
+      const int qs = qi & 1;
+      if (!warp_wait(&qfull[qs], (qi >> 1) & 1)) { ok = false; break; }
+      const int32_t *us = unit_slots + qs * L::kUnitInts;
+      const int nchunks = us[5];
+      if (nchunks == 0) break;  // the producer ran out of work
+      // fused step: this unit's newest token, its chunk and row there, and
+      // the lane's 16 bytes of its key (lanes 0-15) or value (16-31) row
+      const int32_t nd = us[7];
+      int patch_chunk = -1, patch_row = 0;
+      uint4 nrow = make_uint4(0, 0, 0, 0);
+      uint4 *pool_row = nullptr;
+      if (nd >= 0) {
+        const int b = us[0], g = us[1], t0 = us[3], t1 = us[4];
+        patch_chunk = (t1 - 1 - t0) / L::kChunk;
+        patch_row = (t1 - 1 - t0) % L::kChunk;
+        const uint4 *src = static_cast<const uint4 *>(lane < 16 ? p.k_new : p.v_new) +
+                           ((size_t)b * p.Hkv + g) * 16 + (lane & 15);
+        nrow = *src;
+        pool_row = static_cast<uint4 *>(const_cast<void *>(lane < 16 ? p.k : p.v)) +
+                   (((size_t)nd * p.Hkv + g) * p.bs + (t1 - 1) % p.bs) * 16 + (lane & 15);
+      }
+      const uint32_t qb = qbase0 + qs * L::kQ;
+      for (int ci = 0; ci < nchunks; ++ci, ++c) {
+        const int slot = c % 3;
+        if (!warp_wait(&kfull[slot], (c / 3) & 1)) { ok = false; break; }
+        if (ci == patch_chunk) {
+          if (lane < 16) {
+            const int off = tile_piece(patch_row, (lane >> 3) & 1, lane & 7);
+            *reinterpret_cast<uint4 *>(smem + L::kOffK + slot * L::kTile + off) = nrow;
+            fence_proxy_async_smem();  // before the QK MMA reads the tile
+            *pool_row = nrow;
+          }
+          __syncwarp();
+        }
+        if (lane == 0) {
           tc::fence_after_sync();
           const uint32_t kb = kbase0 + slot * L::kTile;
           const uint32_t d = tmem + (c & 1) * N;
@@ -427,17 +546,19 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
           tc::mma_commit(&sfull[c & 1]);
           tc::mma_commit(&kempty[slot]);
           if (ci == nchunks - 1) tc::mma_commit(&qempty[qs]);
-          if (pending.c >= 0 && !issue_pv(pending)) { ok = false; break; }
-          pending = PvJob{c, qi, ci == 0};
         }
-        ++qi;
+        __syncwarp();
+        if (pending.c >= 0 && !issue_pv(pending)) { ok = false; break; }
+        pending = PvJob{c, qi, ci == 0, ci == patch_chunk ? patch_row : -1, nrow, pool_row};
       }
-      if (ok && pending.c >= 0 && !issue_pv(pending)) ok = false;
-      if (!ok) raise_error(PA_DEVERR_TIMEOUT);
-      // no MMA may still be running when the CTA frees its tensor memory
-      tc::mma_commit(drain);
-      mbar_wait(drain, 0);
+      ++qi;
     }
+    if (ok && pending.c >= 0 && !issue_pv(pending)) ok = false;
+    if (!ok && lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+    // no MMA may still be running when the CTA frees its tensor memory
+    if (lane == 0) tc::mma_commit(drain);
+    __syncwarp();
+    mbar_wait(drain, 0);
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     wait_prior_grid();  // before the first write of out / the workspace

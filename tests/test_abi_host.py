@@ -92,6 +92,46 @@ def test_decode_argument_checks():
     assert L.pa_decode(*args(B=0)) == pa.PA_OK                         # nothing to do, no launch
 
 
+def test_append_decode_argument_checks():
+    c = _cache_struct()
+    L = pa.lib()
+    args = lambda **o: [o.get("k", 16), o.get("v", 16), o.get("cow", None), o.get("q", 16), ctypes.byref(c), 16,
+                        o.get("mb", 4), 16, o.get("B", 1), o.get("Hq", 2), o.get("ml", 64), 1.0, o.get("out", 16),
+                        None, 0, None]
+    assert L.pa_append_decode(*args(k=0)) == pa.PA_ERR_INVALID_ARG      # no new key rows
+    assert L.pa_append_decode(*args(v=8)) == pa.PA_ERR_INVALID_ARG      # misaligned
+    assert L.pa_append_decode(*args(Hq=6)) == pa.PA_ERR_UNSUPPORTED     # group size 3, as pa_decode
+    assert L.pa_append_decode(*args(ml=65)) == pa.PA_ERR_INVALID_ARG    # 65 tokens > 4 blocks x 16
+    assert L.pa_append_decode(*args(out=0)) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_append_decode(*args(B=0)) == pa.PA_OK                   # nothing to do, no launch
+
+
+def test_cow_sources():
+    tables = np.array([[4, 9, -1], [4, 7, -1], [5, 6, 2]], np.int32)
+    lens = np.array([20, 17, 33], np.int32)  # last blocks 9, 7, 2 at block size 16
+    assert pa.cow_sources([[3, 7]], tables, lens, 16).tolist() == [-1, 3, -1]
+    assert pa.cow_sources(np.zeros((0, 2)), tables, lens, 16).tolist() == [-1, -1, -1]
+    with pytest.raises(pa.PagedAttnError):
+        pa.cow_sources([[3, 8]], tables, lens, 16)           # 8 is no sequence's last block
+    with pytest.raises(pa.PagedAttnError):
+        pa.cow_sources([[3, 7], [1, 7]], tables, lens, 16)   # a repeated destination
+
+
+def test_cow_sources_of_an_allocator_step():
+    """Four sharers of a partly filled block each append one token: the first
+    three copy it (in batch order), the last writes in place."""
+    A = pa.Allocator(64, 16, list(range(64)))
+    r = A.new_seq()
+    A.batch_append([r], [20])
+    shared = A.block_table(r)[-1]
+    seqs = [r] + [A.fork(r) for _ in range(3)]
+    _, pairs = A.batch_append(seqs, [1] * 4)
+    tables, lens = A.build_block_tables(seqs, 4)
+    cow = pa.cow_sources(pairs, tables, lens, 16)
+    assert cow.tolist() == [shared, shared, shared, -1]
+    assert [int(tables[i, 1]) for i in range(3)] == [int(p[1]) for p in pairs]
+
+
 def test_workspace_size():
     ws = pa.pa_decode_workspace_size
     assert ws(4, 8, 512, 128) == 0
