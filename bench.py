@@ -753,7 +753,7 @@ def oracle_sample(wl, seed: int, budget_s: float, min_s: float):
 def run_reference(args):
     """The oracle as it stands on the host cores: W untimed and K timed steps,
     each step a bounded sample of the workload (whole (sequence, kv head)
-    groups of one batch, two per oracle thread, taken round-robin)."""
+    groups of one batch, eight per oracle thread, taken round-robin)."""
     import oracle
     from paged_kv_cache_402_b200 import synth
 
@@ -764,7 +764,7 @@ def run_reference(args):
     case = synth.random_case(1, B=B, Hq=Hq, Hkv=Hkv, D=D, bs=bs, lens=lens, dtype=torch.bfloat16, sentinel=False)
     order = synth.rng(10).permutation(B * Hkv)
     threads = oracle.max_threads()
-    per_step = 2 * threads
+    per_step = min(8 * threads, B * Hkv)
     pos = 0
     total_bytes, total_s, groups = 0, 0.0, 0
     for s in range(args.warmup + args.steps):
@@ -851,7 +851,7 @@ def main():
         line = run_ours(args, rank, world, dev)
         if rank == 0 and world == 1 and not args.no_cpu_baseline and "lengths" in WORKLOADS[args.workload]:
             wl = WORKLOADS[args.workload]
-            gbs, secs, threads, desc = oracle_sample(wl, seed=1, budget_s=args.cpu_budget, min_s=min(5.0, args.cpu_budget))
+            gbs, secs, threads, desc = oracle_sample(wl, seed=1, budget_s=args.cpu_budget, min_s=args.cpu_budget)
             line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                                     "sample": desc}
         if rank == 0:
