@@ -269,6 +269,7 @@ class Instance:
             slots, pairs = self.alloc.batch_append(seqs, np.ones(B, np.int32))
             tables, lens = self.alloc.build_block_tables(seqs, self.max_blocks)
             cow = pa.cow_sources(pairs, tables, lens, bs)
+            plan = pa.share_plan(tables, lens, bs)
             self.host_alloc_s += time.perf_counter() - t1
             nblk = (lens.astype(np.int64) + bs - 1) // bs
             # unique bytes: every physical block once, with its fill
@@ -281,6 +282,7 @@ class Instance:
                 "slots": torch.from_numpy(slots.copy()).to(dev),
                 "pairs": torch.from_numpy(np.ascontiguousarray(pairs)).to(dev) if len(pairs) else None,
                 "cow": torch.from_numpy(cow).to(dev) if len(pairs) else None,
+                "plan": plan.to(dev),
                 "n_pairs": len(pairs),
                 "tables": torch.from_numpy(tables).to(dev),
                 "lens": torch.from_numpy(lens).to(dev),
@@ -369,6 +371,10 @@ def run_ours(args, rank: int, world: int, dev):
         if args.unfused:
             pa.pa_decode(st["q"], inst.cache, st["tables"], st["lens"], st["max_ctx"], scale,
                          out=st["out"], workspace=st["ws"], stream=strm)
+        elif not args.no_share_plan:
+            pa.pa_decode_shared(st["q"], inst.cache, st["tables"], st["lens"], st["max_ctx"], scale,
+                                plan=st["plan"], k_new=st["k"], v_new=st["v"], cow_src=st["cow"],
+                                out=st["out"], workspace=st["ws"], stream=strm)
         else:
             pa.pa_append_decode(st["k"], st["v"], st["q"], inst.cache, st["tables"], st["lens"], st["max_ctx"],
                                 scale, cow_src=st["cow"], out=st["out"], workspace=st["ws"], stream=strm)
@@ -483,7 +489,12 @@ def run_ours(args, rank: int, world: int, dev):
                    "parallelism": f"replicas x{world}",
                    "timing": "eager launches" if args.no_graph else "CUDA graph replay of the K steps",
                    "step": ("pa_copy_blocks + pa_append_kv + pa_decode" if args.unfused else
-                            "pa_append_decode (copy on write + append + decode in one call)")},
+                            "pa_append_decode (copy on write + append + decode in one call)" if args.no_share_plan
+                            else "pa_decode_shared (copy on write + append + decode in one call; partitions "
+                                 "that a group of sequences holds in the same blocks read once per group of "
+                                 "up to 4)"),
+                   "share_groups_per_step": round(statistics.mean(
+                       insts[0].steps[i]["plan"].n_groups for i in range(len(insts[0].steps))), 2)},
         "tokens_per_s": round(tok_all / (ms_all / 1e3), 1),
         "kv_logical_gbs": round(kv_logical * world / 1e9 / (ms_all / 1e3), 2),
         "copy_pairs_per_step": round(pairs / args.steps, 2),
@@ -492,7 +503,10 @@ def run_ours(args, rank: int, world: int, dev):
         "host_alloc_us_per_step": round(host_alloc_us, 2),
         "roofline": {"bound": "hbm",
                      "kernel": ("pa_decode (partition + LSE reduce)" if args.unfused else
-                                "pa_append_decode (copy + append + partition in one kernel, + LSE reduce)"),
+                                "pa_append_decode (copy + append + partition in one kernel, + LSE reduce)"
+                                if args.no_share_plan else
+                                "pa_decode_shared (cascade over shared partitions + fused copy/append/partition"
+                                " + LSE reduce)"),
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
                      "traffic": profiled_traffic(args.workload),
@@ -553,6 +567,7 @@ def run_e2e(args, insts, wl, dev, stream):
     ones = np.ones(B, np.int32)
     seen = []
     h2d = d2h = 0
+    plan_bytes = 0
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     for i in range(n_steps):
@@ -574,9 +589,16 @@ def run_e2e(args, insts, wl, dev, stream):
             if npairs:
                 pa.cow_sources(pairs, tables_np, lens_np, bs, out=h["cow"].numpy())
                 d["cow"].copy_(h["cow"], non_blocking=True)
-            pa.pa_append_decode(d["k"], d["v"], d["q"], inst.cache, d["tables"], d["lens"], int(lens_np.max()),
-                                1.0 / math.sqrt(D), cow_src=d["cow"] if npairs else None, out=out, workspace=ws,
-                                stream=stream)
+            if args.no_share_plan:
+                pa.pa_append_decode(d["k"], d["v"], d["q"], inst.cache, d["tables"], d["lens"], int(lens_np.max()),
+                                    1.0 / math.sqrt(D), cow_src=d["cow"] if npairs else None, out=out,
+                                    workspace=ws, stream=stream)
+            else:
+                plan = pa.share_plan(tables_np, lens_np, bs).to(dev)
+                plan_bytes += plan.members.nbytes + plan.parts.nbytes + plan.first_part.nbytes
+                pa.pa_decode_shared(d["q"], inst.cache, d["tables"], d["lens"], int(lens_np.max()),
+                                    1.0 / math.sqrt(D), plan=plan, k_new=d["k"], v_new=d["v"],
+                                    cow_src=d["cow"] if npairs else None, out=out, workspace=ws, stream=stream)
         h["out"].copy_(out, non_blocking=True)
         torch.cuda.synchronize()
         if i == 0:
@@ -586,6 +608,7 @@ def run_e2e(args, insts, wl, dev, stream):
         seen.append((tables_np.copy(), lens_np.copy()))
     seconds = time.perf_counter() - t0
     kv = sum(unique_kv_bytes(t, l, bs, 2 * Hkv * D * 2) for t, l in seen)
+    h2d += plan_bytes // n_steps
     return {"seconds": seconds, "kv_gb": kv / 1e9, "steps": n_steps, "h2d": h2d, "d2h": d2h}
 
 
@@ -635,6 +658,7 @@ def run_trace(args, dev):
             if n:
                 max_ctx, mb = A.max_len(plan.decode_seqs)
                 tables, lens = A.build_block_tables(plan.decode_seqs, mb)
+                splan = pa.share_plan(tables, lens, bs) if not (args.unfused or args.no_share_plan) else None
             host_s += time.perf_counter() - t0
             if n == 0:
                 wall += time.perf_counter() - t0
@@ -667,10 +691,15 @@ def run_trace(args, dev):
                 pa.pa_append_kv(kd, kd, d_[1], cache, stream)
                 pa.pa_decode(q, cache, d_[3], d_[4], max_ctx, 1 / math.sqrt(D), out=o, workspace=ws, stream=stream)
                 launches += 2 + (1 if max_ctx > pa.PA_PARTITION_TOKENS else 0)
-            else:
+            elif args.no_share_plan:
                 pa.pa_append_decode(kd, kd, q, cache, d_[3], d_[4], max_ctx, 1 / math.sqrt(D), cow_src=d_[5],
                                     out=o, workspace=ws, stream=stream)
                 launches += 1 + (1 if max_ctx > pa.PA_PARTITION_TOKENS else 0)
+            else:
+                pa.pa_decode_shared(q, cache, d_[3], d_[4], max_ctx, 1 / math.sqrt(D), plan=splan.to(dev),
+                                    k_new=kd, v_new=kd, cow_src=d_[5], out=o, workspace=ws, stream=stream)
+                launches += 1 + (1 if max_ctx > pa.PA_PARTITION_TOKENS else 0) + (1 if splan.n_groups else 0)
+                h2d += splan.members.nbytes + splan.parts.nbytes + splan.first_part.nbytes
             ev[s_][1].record(stream)
             res = o[:1].to("cpu", non_blocking=True)
             torch.cuda.synchronize()
@@ -818,6 +847,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rotate", type=int, default=0, help="batch instances to rotate (0: the workload's default)")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly instead of from a CUDA graph")
+    ap.add_argument("--no-share-plan", action="store_true",
+                    help="fused step without the cascade over shared partitions (pa_append_decode)")
     ap.add_argument("--unfused", action="store_true",
                     help="run each step as pa_copy_blocks + pa_append_kv + pa_decode instead of pa_append_decode")
     ap.add_argument("--block-size", type=int, default=0, help="trace workload: one block size (0: 8, 16 and 32)")

@@ -75,6 +75,7 @@ typedef enum { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
 #define PA_DEVERR_PAIR 0x4       /* pa_copy_blocks: a pair entry outside [0, num_blocks) (pair skipped) */
 #define PA_DEVERR_TIMEOUT 0x8    /* a kernel gave up waiting on its own copy (work unit dropped) */
 #define PA_DEVERR_LEN 0x10       /* pa_decode: a context length < 0 or > max_context_len (row zeroed) */
+#define PA_DEVERR_PLAN 0x20      /* pa_decode_shared: a sharing plan entry that does not fit its sequence (ignored) */
 
 /* Tokens per split-context partition of pa_decode. */
 #define PA_PARTITION_TOKENS 512
@@ -170,6 +171,53 @@ PA_API pa_status pa_append_decode(const void *k_new, const void *v_new, const in
                                   int32_t num_q_heads, int32_t max_context_len, float scale,
                                   void *out, void *workspace, size_t workspace_bytes,
                                   void *stream);
+
+/*
+ * A sharing plan for pa_decode_shared: groups of sequences of one batch whose
+ * block tables hold the same physical blocks for their first parts[j] whole
+ * partitions (PA_PARTITION_TOKENS tokens each), every one of them before the
+ * member's last partition.  pa_share_plan builds one from host tables.
+ *   members     device [n_groups][max_members] int32: sequence indices of the
+ *               batch, a group's members first, -1 after its last
+ *   parts       device [n_groups] int32 (>= 1)
+ *   first_part  device [num_seqs] int32: parts[j] for a member of group j,
+ *               0 for a sequence in no group
+ *   max_members 1..4 (the cascade kernel's query tile holds 4 sequences)
+ * A sequence belongs to at most one group.  If the tables of a group do not
+ * agree on those partitions the results are undefined; a first_part that
+ * does not fit its sequence sets PA_DEVERR_PLAN and that sequence is
+ * computed whole (the group's statistics for it are overwritten).
+ */
+typedef struct {
+  const int32_t *members;
+  const int32_t *parts;
+  const int32_t *first_part;
+  int32_t n_groups;
+  int32_t max_members;
+} pa_share_plan_t;
+
+/*
+ * pa_decode (or pa_append_decode, when k_new and v_new are given) with a
+ * cascade over shared blocks: the partitions a plan's group shares are read
+ * once for all its members ("pagedattention" glossary entry, paragraph 5:
+ * sequences that share a prefix point at the same physical blocks;
+ * "PagedAttention Internals", "Sharing And Dynamic Growth").  The result is
+ * that of pa_decode / pa_append_decode up to the rounding of the fp32 sums
+ * (the same sums in the same order: each member's partition statistics are
+ * computed over the same tiles).  plan may be NULL or have no groups; on the
+ * CUDA-core path (not bf16 with head_dim 128) the plan is not used and every
+ * sequence computes all of its partitions.
+ *   k_new, v_new, cow_src  as pa_append_decode, or all NULL for no append
+ *   plan                   host pointer to the plan (its arrays on the device)
+ *   the rest               as pa_decode
+ */
+PA_API pa_status pa_decode_shared(const void *k_new, const void *v_new, const int32_t *cow_src,
+                                  const void *q, const pa_cache_t *cache,
+                                  const int32_t *block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t *context_lens, int32_t num_seqs,
+                                  int32_t num_q_heads, int32_t max_context_len, float scale,
+                                  const pa_share_plan_t *plan, void *out, void *workspace,
+                                  size_t workspace_bytes, void *stream);
 
 /* Bytes of workspace pa_decode needs for these sizes (0 when no context is
  * longer than one partition). */
@@ -313,6 +361,23 @@ PA_API pa_status pa_alloc_stats(pa_allocator *a, int64_t *used_slots, int64_t *a
 
 /* Reference count of a physical block. */
 PA_API pa_status pa_block_refcount(pa_allocator *a, int32_t block, int32_t *refcount);
+
+/*
+ * Builds a sharing plan from host tables (after the step's appends):
+ * sequences longer than one partition whose first partition's table entries
+ * are identical form buckets; each bucket is cut into groups of at most
+ * max_members (2..4) in sequence order, a lone leftover joins no group; a
+ * group shares every leading partition whose entries agree across it and
+ * that is whole and before the last partition of each member.
+ *   tables_host  [n_seqs][max_blocks] int32, lens_host [n_seqs] int32
+ *   members_host room for n_seqs / 2 groups x max_members, -1 padded
+ *   parts_host   room for n_seqs / 2
+ *   first_part_host [n_seqs]
+ */
+PA_API pa_status pa_share_plan(const int32_t *tables_host, int32_t max_blocks,
+                               const int32_t *lens_host, int32_t n_seqs, int32_t block_size,
+                               int32_t max_members, int32_t *members_host, int32_t *parts_host,
+                               int32_t *first_part_host, int32_t *n_groups);
 
 /*
  * The per-sequence form of a decode step's copy pairs, as pa_append_decode

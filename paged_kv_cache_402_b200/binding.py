@@ -25,7 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_OUT_OF_BLOCKS = 0, 1, 2, 3
 PA_ERR_CUDA, PA_ERR_NOT_FOUND, PA_ERR_TOO_SMALL = 4, 5, 6
 PA_DTYPE_F32, PA_DTYPE_BF16 = 0, 1
-PA_DEVERR_SLOT, PA_DEVERR_TABLE, PA_DEVERR_PAIR, PA_DEVERR_TIMEOUT, PA_DEVERR_LEN = 1, 2, 4, 8, 16
+PA_DEVERR_SLOT, PA_DEVERR_TABLE, PA_DEVERR_PAIR, PA_DEVERR_TIMEOUT, PA_DEVERR_LEN, PA_DEVERR_PLAN = 1, 2, 4, 8, 16, 32
 PA_PARTITION_TOKENS = 512
 
 _DTYPES = {torch.float32: PA_DTYPE_F32, torch.bfloat16: PA_DTYPE_BF16}
@@ -47,6 +47,11 @@ class pa_cache_t(ctypes.Structure):
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
 
 
+class pa_share_plan_t(ctypes.Structure):
+    _fields_ = [("members", ctypes.c_void_p), ("parts", ctypes.c_void_p), ("first_part", ctypes.c_void_p),
+                ("n_groups", ctypes.c_int32), ("max_members", ctypes.c_int32)]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_402_b200.build`")
@@ -62,6 +67,9 @@ def _load() -> ctypes.CDLL:
         "pa_decode_static_workspace": (st, [vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp]),
         "pa_append_decode": (st, [vp, vp, vp, vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp, sz, vp]),
         "pa_cow_sources": (st, [i32p, i32, i32p, i32, i32p]),
+        "pa_decode_shared": (st, [vp, vp, vp, vp, cp, vp, i32, vp, i32, i32, i32, f32,
+                                  ctypes.POINTER(pa_share_plan_t), vp, vp, sz, vp]),
+        "pa_share_plan": (st, [i32p, i32, i32p, i32, i32, i32, i32p, i32p, i32p, i32p]),
         "pa_copy_blocks": (st, [vp, i32, cp, vp]),
         "pa_check_copy_pairs": (st, [i32p, i32, i32]),
         "pa_read_device_error": (st, [vp, i32p]),
@@ -262,6 +270,86 @@ def cow_sources(pairs, tables: np.ndarray, lens: np.ndarray, block_size: int,
     res = out if out is not None else np.empty(n, dtype=np.int32)
     _check(_lib.pa_cow_sources(_i32p(pairs), pairs.shape[0], _i32p(last), n, _i32p(res)), "pa_cow_sources")
     return res
+
+
+class SharePlan:
+    """A sharing plan (groups of sequences that hold the same blocks for their
+    leading whole partitions) as host arrays, plus its device copy."""
+
+    def __init__(self, members: np.ndarray, parts: np.ndarray, first_part: np.ndarray):
+        self.members, self.parts, self.first_part = members, parts, first_part
+        self.n_groups, self.max_members = int(members.shape[0]), int(members.shape[1])
+        self._dev = None
+
+    def to(self, device, stream=None) -> "SharePlan":
+        """Copies the arrays to the device (kept until the plan is dropped)."""
+        nb = self.n_groups > 0
+        self._dev = tuple(torch.from_numpy(np.ascontiguousarray(a)).to(device, non_blocking=True)
+                          for a in ((self.members if nb else np.full((1, 1), -1, np.int32)),
+                                    (self.parts if nb else np.zeros(1, np.int32)), self.first_part))
+        return self
+
+    def ref(self):
+        if self.n_groups == 0:
+            return None
+        if self._dev is None:
+            raise ValueError("SharePlan.to(device) first")
+        m, pt, fp = self._dev
+        self._struct = pa_share_plan_t(m.data_ptr(), pt.data_ptr(), fp.data_ptr(), self.n_groups, self.max_members)
+        return ctypes.byref(self._struct)
+
+
+def share_plan(tables, lens, block_size: int, max_members: int = 4) -> SharePlan:
+    """Host: groups the sequences of a batch whose tables agree on their
+    leading whole partitions (pa_share_plan)."""
+    tables = np.ascontiguousarray(np.asarray(tables, dtype=np.int32))
+    lens = np.ascontiguousarray(np.asarray(lens, dtype=np.int32))
+    n = len(lens)
+    cap = max(1, n // 2)
+    members = np.empty((cap, max_members), dtype=np.int32)
+    parts = np.empty(cap, dtype=np.int32)
+    first = np.empty(n, dtype=np.int32)
+    ng = ctypes.c_int32(0)
+    _check(_lib.pa_share_plan(_i32p(tables), tables.shape[1] if tables.ndim == 2 else 0, _i32p(lens), n,
+                              int(block_size), int(max_members), _i32p(members), _i32p(parts), _i32p(first),
+                              ctypes.byref(ng)), "pa_share_plan")
+    g = ng.value
+    return SharePlan(members[:g].copy(), parts[:g].copy(), first)
+
+
+def pa_decode_shared(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor, context_lens: torch.Tensor,
+                     max_context_len: int, scale: float, plan: SharePlan | None = None,
+                     k_new: torch.Tensor | None = None, v_new: torch.Tensor | None = None,
+                     cow_src: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """pa_decode, or pa_append_decode when k_new / v_new are given, with the
+    partitions a plan's groups share read once for all their members."""
+    B, Hq, D = q.shape
+    if D != cache.head_dim:
+        raise ValueError("head_dim mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("block_tables must be [B, max_blocks] and context_lens [B]")
+    if (k_new is None) != (v_new is None):
+        raise ValueError("give both k_new and v_new, or neither")
+    row_shape = (B, cache.num_kv_heads, D)
+    if k_new is not None and (tuple(k_new.shape) != row_shape or tuple(v_new.shape) != row_shape):
+        raise ValueError(f"k_new and v_new must be {list(row_shape)}")
+    if out is None:
+        out = torch.empty_like(q)
+    need = pa_decode_workspace_size(B, Hq, int(max_context_len), D)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.pa_decode_shared(
+        _dev(k_new, "k_new", cache.dtype) if k_new is not None else None,
+        _dev(v_new, "v_new", cache.dtype) if v_new is not None else None,
+        _dev(cow_src, "cow_src", torch.int32) if cow_src is not None else None,
+        _dev(q, "q", cache.dtype), cache.ref(), _dev(block_tables, "block_tables", torch.int32),
+        block_tables.shape[1], _dev(context_lens, "context_lens", torch.int32), B, Hq, int(max_context_len),
+        float(scale), plan.ref() if plan is not None else None, _dev(out, "out", cache.dtype), ws_ptr, ws_bytes,
+        _stream_ptr(stream)), "pa_decode_shared")
+    return out
 
 
 PA_STATIC_WORKSPACE_BYTES = 8 << 20

@@ -309,6 +309,60 @@ PA_API pa_status pa_block_refcount(pa_allocator *a, int32_t block, int32_t *refc
   return PA_OK;
 }
 
+PA_API pa_status pa_share_plan(const int32_t *tables_host, int32_t max_blocks,
+                               const int32_t *lens_host, int32_t n_seqs, int32_t block_size,
+                               int32_t max_members, int32_t *members_host, int32_t *parts_host,
+                               int32_t *first_part_host, int32_t *n_groups) {
+  if (n_seqs < 0 || max_blocks < 0 || !n_groups || max_members < 2 || max_members > 4 ||
+      (block_size != 8 && block_size != 16 && block_size != 32))
+    return PA_ERR_INVALID_ARG;
+  if (n_seqs > 0 && (!tables_host || !lens_host || !members_host || !parts_host || !first_part_host))
+    return PA_ERR_INVALID_ARG;
+  *n_groups = 0;
+  const int32_t bpp = PA_PARTITION_TOKENS / block_size;  // table entries per partition
+  for (int32_t b = 0; b < n_seqs; ++b) first_part_host[b] = 0;
+  // sequences with at least two partitions (the first one whole, not the last)
+  std::vector<int32_t> cand;
+  for (int32_t b = 0; b < n_seqs; ++b)
+    if (lens_host[b] > PA_PARTITION_TOKENS && max_blocks >= bpp) cand.push_back(b);
+  auto row = [&](int32_t b) { return tables_host + (size_t)b * max_blocks; };
+  // buckets: equal first-partition entries, sequence order inside a bucket
+  std::stable_sort(cand.begin(), cand.end(), [&](int32_t x, int32_t y) {
+    return std::lexicographical_compare(row(x), row(x) + bpp, row(y), row(y) + bpp);
+  });
+  size_t i = 0;
+  while (i < cand.size()) {
+    size_t e = i + 1;
+    while (e < cand.size() && std::equal(row(cand[i]), row(cand[i]) + bpp, row(cand[e]))) ++e;
+    for (size_t g0 = i; g0 + 1 < e; g0 += (size_t)max_members) {
+      const size_t g1 = std::min(e, g0 + (size_t)max_members);
+      if (g1 - g0 < 2) break;  // a lone leftover shares with nobody
+      // leading partitions that agree, are whole and come before every member's last
+      int32_t parts = 0;
+      for (;; ++parts) {
+        const int64_t end_tok = (int64_t)(parts + 1) * PA_PARTITION_TOKENS;
+        if ((int64_t)(parts + 1) * bpp > max_blocks) break;
+        bool ok = true;
+        for (size_t k = g0; k < g1 && ok; ++k) {
+          const int32_t b = cand[k];
+          ok = lens_host[b] > end_tok &&
+               std::equal(row(cand[g0]) + (size_t)parts * bpp, row(cand[g0]) + (size_t)(parts + 1) * bpp,
+                          row(b) + (size_t)parts * bpp);
+        }
+        if (!ok) break;
+      }
+      if (parts < 1) continue;
+      int32_t *mem = members_host + (size_t)(*n_groups) * max_members;
+      for (int32_t k = 0; k < max_members; ++k) mem[k] = g0 + k < g1 ? cand[g0 + k] : -1;
+      parts_host[*n_groups] = parts;
+      for (size_t k = g0; k < g1; ++k) first_part_host[cand[k]] = parts;
+      ++*n_groups;
+    }
+    i = e;
+  }
+  return PA_OK;
+}
+
 PA_API pa_status pa_cow_sources(const int32_t *pairs_host, int32_t n_pairs,
                                 const int32_t *last_blocks_host, int32_t n_seqs,
                                 int32_t *cow_src_host) {

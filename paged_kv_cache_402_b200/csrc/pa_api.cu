@@ -15,6 +15,7 @@
 
 #include "pa_copy_kernels.cuh"
 #include "pa_decode_simt.cuh"
+#include "pa_decode_shared.cuh"
 #include "pa_decode_tc.cuh"
 #include "pagedattn.h"
 
@@ -252,6 +253,7 @@ pa_status launch_decode_tc_g(const pa::DecodeParams &p, int32_t max_parts, cudaS
       ps.v_new = static_cast<const __nv_bfloat16 *>(p.v_new) + (size_t)b0 * p.Hkv * 128;
       if (p.cow_src) ps.cow_src = p.cow_src + b0;
     }
+    if (p.first_part) ps.first_part = p.first_part + b0;
     if (p.ws_m) {
       ps.ws_m = p.ws_m + rows * max_parts;
       ps.ws_l = p.ws_l + rows * max_parts;
@@ -262,6 +264,46 @@ pa_status launch_decode_tc_g(const pa::DecodeParams &p, int32_t max_parts, cudaS
     if (s != PA_OK) return s;
   }
   return PA_OK;
+}
+
+// The cascade kernel over the shared partitions of a sharing plan, in
+// slices of at most kMaxGroups groups.
+template <int G>
+pa_status launch_decode_shared_g(const pa::DecodeParams &p, const pa_share_plan_t &plan, cudaStream_t st) {
+  CUtensorMap mk, mv, mq;
+  const uint64_t rows = (uint64_t)p.num_blocks * p.Hkv * p.bs;
+  if (!make_map_pool_4d(&mk, p.k, rows, (uint32_t)p.bs) ||
+      !make_map_pool_4d(&mv, p.v, rows, (uint32_t)p.bs) ||
+      !make_map_bf16_d128(&mq, p.q, (uint64_t)p.B * p.Hq, (uint32_t)G))
+    return PA_ERR_CUDA;
+  auto kern = pa::decode_shared_tc<G>;
+  const int smem = pa::ShLayout::kBytes;
+  static std::atomic<int> smem_set[kMaxDev] = {};
+  if (!ensure_smem(kern, smem, smem_set)) return PA_ERR_CUDA;
+  const int sms = sm_count();
+  if (sms <= 0) return PA_ERR_CUDA;
+  for (int j0 = 0; j0 < plan.n_groups; j0 += pa::ShLayout::kMaxGroups) {
+    pa::SharedParams sp{};
+    sp.n_groups = plan.n_groups - j0 < pa::ShLayout::kMaxGroups ? plan.n_groups - j0 : pa::ShLayout::kMaxGroups;
+    sp.max_members = plan.max_members;
+    sp.members = plan.members + (size_t)j0 * plan.max_members;
+    sp.parts = plan.parts + j0;
+    const int64_t units_bound = (int64_t)sp.n_groups * p.Hkv * (p.max_parts > 1 ? p.max_parts - 1 : 1);
+    const int grid = units_bound < sms ? (int)units_bound : sms;
+    const pa_status s = launch(kern, dim3(grid), dim3(pa::ShLayout::kThreads), (size_t)smem, st, mk, mv, mq, p, sp);
+    if (s != PA_OK) return s;
+  }
+  return PA_OK;
+}
+
+pa_status launch_decode_shared(const pa::DecodeParams &p, const pa_share_plan_t &plan, cudaStream_t st) {
+  switch (p.G) {
+    case 1: return launch_decode_shared_g<1>(p, plan, st);
+    case 2: return launch_decode_shared_g<2>(p, plan, st);
+    case 4: return launch_decode_shared_g<4>(p, plan, st);
+    case 8: return launch_decode_shared_g<8>(p, plan, st);
+    default: return PA_ERR_UNSUPPORTED;
+  }
 }
 
 pa_status launch_decode_tc(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
@@ -475,6 +517,54 @@ PA_API pa_status pa_append_decode(const void *k_new, const void *v_new, const in
              cache->num_blocks, max_context_len, (uint4 *)cache->k, (uint4 *)cache->v);
   if (s != PA_OK) return s;
   return launch_decode_any(p, cache, st);
+}
+
+PA_API pa_status pa_decode_shared(const void *k_new, const void *v_new, const int32_t *cow_src,
+                                  const void *q, const pa_cache_t *cache,
+                                  const int32_t *block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t *context_lens, int32_t num_seqs,
+                                  int32_t num_q_heads, int32_t max_context_len, float scale,
+                                  const pa_share_plan_t *plan, void *out, void *workspace,
+                                  size_t workspace_bytes, void *stream) {
+  pa::DecodeParams p{};
+  bool skip = false;
+  pa_status s = prepare_decode(q, cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                               num_q_heads, max_context_len, scale, out, workspace, workspace_bytes,
+                               &p, &skip);
+  if (s != PA_OK || skip) return s;
+  if ((k_new == nullptr) != (v_new == nullptr)) return PA_ERR_INVALID_ARG;
+  if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return PA_ERR_INVALID_ARG;
+  const bool grouped = plan && plan->n_groups > 0;
+  if (grouped) {
+    if (!plan->members || !plan->parts || !plan->first_part || plan->n_groups < 0 ||
+        plan->max_members < 1 || plan->max_members > pa::ShLayout::kSlots)
+      return PA_ERR_INVALID_ARG;
+    if (p.max_parts < 2) return PA_ERR_INVALID_ARG;  // a shared partition is never a sequence's last
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!tc_eligible(p, cache->dtype, cache->head_dim)) {
+    // no cascade kernel on the CUDA-core path: every sequence computes all
+    // of its partitions (the same result)
+    if (k_new) {
+      const int row_vecs = cache->head_dim * elem_bytes(cache->dtype) / 16;
+      const int64_t warps = (int64_t)num_seqs * cache->num_kv_heads;
+      s = launch(pa::append_newest_kernel, dim3((unsigned)((warps * 32 + 255) / 256)), dim3(256), 0, st,
+                 (const uint4 *)k_new, (const uint4 *)v_new, cow_src, block_tables, context_lens,
+                 max_blocks_per_seq, num_seqs, cache->num_kv_heads, cache->block_size, row_vecs,
+                 cache->num_blocks, max_context_len, (uint4 *)cache->k, (uint4 *)cache->v);
+      if (s != PA_OK) return s;
+    }
+    return launch_decode_any(p, cache, st);
+  }
+  if (grouped) {
+    s = launch_decode_shared(p, *plan, st);
+    if (s != PA_OK) return s;
+    p.first_part = plan->first_part;
+  }
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.cow_src = k_new ? cow_src : nullptr;
+  return launch_decode_tc(p, p.max_parts, st);
 }
 
 // ---------------------------------------------------------------------------

@@ -1,0 +1,545 @@
+// Cascade decode over shared prefix blocks (bf16, head_dim 128, group size
+// 1..8, tensor cores): the partitions that several sequences of a batch hold
+// in the same physical blocks are read once for all of them.
+//
+// The pages make sharing the point of the paged layout: sequences with a
+// common prefix, or the samples of one request, point at the same physical
+// blocks ("pagedattention" glossary entry, comparison table and paragraph 5;
+// "PagedAttention Internals", "Sharing And Dynamic Growth").  The attention
+// of each sequence over such a block is still its own: this kernel computes,
+// for a group of up to kSlots sequences whose block tables agree on their
+// first `parts` whole partitions, each member's split-context statistics
+// (max, sum, unnormalised accumulator) of those partitions, exactly what
+// decode_partition_tc would write for them, into the same workspace rows.
+// decode_partition_tc then does every sequence from its first private
+// partition on, and the log-sum-exp reduce merges both.
+//
+// Same machinery as decode_partition_tc (see there): persistent CTAs, a TMA
+// producer warp loading whole (block, kv head) tiles as 4-D boxes into
+// 128-byte-swizzled K and V rings, one MMA warp, a 128-thread softmax
+// warpgroup.  What differs:
+//  * a work unit is (group, kv head, shared partition): 512 tokens, always
+//    full, handed out round-robin (all units are the same size);
+//  * the Q tile holds the group's members in 8-row slots (member m: rows
+//    8m .. 8m + G - 1, one 2-D TMA box per column half per member), so the
+//    MMAs are M = 128 tokens x N = 32 query rows;
+//  * the epilogue writes workspace rows for every (member, query head), read
+//    from O at the start of the next unit;
+//  * two ring stages (the larger Q and P tiles take the third one's room).
+#pragma once
+
+#include "pa_decode_tc.cuh"
+
+namespace pa {
+
+struct ShLayout {
+  static constexpr int kSlots = 4;          // sequences per unit
+  static constexpr int kN = 8 * kSlots;     // MMA N: 8 query rows per member slot
+  static constexpr int kChunk = 128;
+  static constexpr int kStages = 2;
+  static constexpr int kTile = kChunk * 256;
+  static constexpr int kGroup = 2048;
+  static constexpr int kQ = 2 * kN * 128;   // two column halves of kN rows x 128 B
+  static constexpr int kP = 2 * kN * 128;   // two 64-token halves of kN rows x 128 B
+  static constexpr int kMaxGroups = 1024;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kStages * kTile;
+  static constexpr int kOffQ = kOffV + kStages * kTile;
+  static constexpr int kOffP = kOffQ + 2 * kQ;
+  static constexpr int kOffBar = kOffP + 2 * kP;
+  static constexpr int kNumBars = 21;
+  static constexpr int kOffRed = kOffBar + kNumBars * 8;
+  static constexpr int kRedFloats = 2 * 4 * kN;  // [parity][warp][column]
+  static constexpr int kOffRedSum = kOffRed + kRedFloats * 4;
+  static constexpr int kOffTmem = kOffRedSum + kRedFloats * 4;
+  // unit slot: [group, kv head, partition, members, b_0 .. b_3] + the table
+  // entries of the partition (from the first member's table)
+  static constexpr int kUnitInts = 8 + kPart / 8;
+  static constexpr int kOffUnit = kOffTmem + 16;
+  static constexpr int kOffScan = kOffUnit + 2 * kUnitInts * 4;
+  static constexpr int kOffPrefix = kOffScan + 32;  // shared partitions before each group
+  static constexpr int kBytes = kOffPrefix + (kMaxGroups + 1) * 4 + 1024;
+  static constexpr int kThreads = 192;
+  static constexpr uint32_t kTmemCols = 128;  // S0 S1 O0 O1, kN columns each
+};
+
+// The sharing plan of one launch: group j has members[j * max_members + m]
+// (m < max_members, -1 past its last member) sharing parts[j] partitions.
+struct SharedParams {
+  const int32_t *members;
+  const int32_t *parts;
+  int32_t n_groups;
+  int32_t max_members;
+};
+
+template <int G>
+__global__ void __launch_bounds__(ShLayout::kThreads, 1)
+    decode_shared_tc(const __grid_constant__ CUtensorMap tmap_k,
+                     const __grid_constant__ CUtensorMap tmap_v,
+                     const __grid_constant__ CUtensorMap tmap_q, DecodeParams p, SharedParams sp) {
+  using L = ShLayout;
+  constexpr int N = L::kN;
+  static_assert(G >= 1 && G <= 8, "group size");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
+  uint64_t *kfull = bars, *kempty = bars + 2, *vfull = bars + 4, *vempty = bars + 6;
+  uint64_t *qfull = bars + 8, *qempty = bars + 10, *sfull = bars + 12, *pfull = bars + 14;
+  uint64_t *pvdone = bars + 16, *ofree = bars + 18, *drain = bars + 20;
+  int32_t *gprefix = reinterpret_cast<int32_t *>(smem + L::kOffPrefix);
+  int32_t *scan = reinterpret_cast<int32_t *>(smem + L::kOffScan);
+  int32_t *unit_slots = reinterpret_cast<int32_t *>(smem + L::kOffUnit);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffTmem);
+  float *red_max = reinterpret_cast<float *>(smem + L::kOffRed);
+  float *red_sum = reinterpret_cast<float *>(smem + L::kOffRedSum);
+
+  // ---------------------------------------------------------------- set-up
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::kStages; ++i) {
+      mbar_init(&kfull[i], 1);
+      mbar_init(&kempty[i], 1);
+      mbar_init(&vfull[i], 1);
+      mbar_init(&vempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&qfull[i], 1);
+      mbar_init(&qempty[i], 2);  // the MMA lane's commit + the softmax warpgroup
+      mbar_init(&sfull[i], 1);
+      mbar_init(&pfull[i], 128);
+      mbar_init(&pvdone[i], 1);
+      mbar_init(&ofree[i], 128);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  // Q rows a member slot does not use (G..7) and unused P rows stay zero
+  for (int i = threadIdx.x; i < (2 * L::kQ + 2 * L::kP) / 16; i += blockDim.x)
+    reinterpret_cast<uint4 *>(smem + L::kOffQ)[i] = make_uint4(0, 0, 0, 0);
+
+  // shared partitions per group and their exclusive prefix sums (the plan is
+  // caller data that no kernel of the library writes: read before the wait)
+  const int NG = sp.n_groups;
+  constexpr int kMaxSeg = (L::kMaxGroups + L::kThreads - 1) / L::kThreads;
+  const int seg = (NG + blockDim.x - 1) / blockDim.x;
+  const int j_first = threadIdx.x * seg;
+  int cnt[kMaxSeg];
+  int mine = 0;
+#pragma unroll
+  for (int i = 0; i < kMaxSeg; ++i) {
+    cnt[i] = 0;
+    const int j = j_first + i;
+    if (i < seg && j < NG) {
+      cnt[i] = max(sp.parts[j], 0);
+      mine += cnt[i];
+    }
+  }
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) scan[warp] = incl;
+  if (warp == 1) tc::tmem_alloc(tmem_slot, L::kTmemCols);
+  __syncthreads();
+  int run = incl - mine;
+  for (int w = 0; w < warp; ++w) run += scan[w];
+#pragma unroll
+  for (int i = 0; i < kMaxSeg; ++i) {
+    const int j = j_first + i;
+    if (i < seg && j < NG) {
+      gprefix[j] = run;
+      run += cnt[i];
+      if (j == NG - 1) gprefix[NG] = run;
+    }
+  }
+  if (warp == 1) tc::tmem_relinquish();
+  fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int num_units = p.Hkv * gprefix[NG];
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tc::prefetch_tensormap(&tmap_k);
+      tc::prefetch_tensormap(&tmap_v);
+      tc::prefetch_tensormap(&tmap_q);
+    }
+    const uint64_t pol_kv = policy_evict_first();
+    const uint64_t pol_q = tc::policy_evict_last();
+    const int bs = p.bs;
+    const int blocks_per_chunk = L::kChunk / bs;
+    const int nb_unit = kPart / bs;  // blocks of a (whole) partition
+    const int oob_group = p.num_blocks * p.Hkv * (bs / 8);
+    int c = 0, qi = 0;
+    bool ok = true;
+    // unit u: kv head u % Hkv of shared partition u / Hkv in the groups' order
+    struct ShUnit {
+      int j, g, part, nmem;
+      int32_t b[L::kSlots];
+    };
+    auto load_unit = [&](int u, ShUnit &un, int32_t &x0, int32_t &x1) {
+      x0 = x1 = -1;
+      un.nmem = 0;
+      if (u >= num_units) return;
+      const int w = u / p.Hkv;
+      un.g = u - w * p.Hkv;
+      int lo = 0, hi = NG - 1;  // largest group whose count before it is <= w
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (gprefix[mid] <= w) lo = mid; else hi = mid - 1;
+      }
+      un.j = lo;
+      un.part = w - gprefix[lo];
+      const int32_t mb = lane < L::kSlots && lane < sp.max_members ? sp.members[(size_t)lo * sp.max_members + lane] : -1;
+      int nmem = 0;
+#pragma unroll
+      for (int m = 0; m < L::kSlots; ++m) {
+        un.b[m] = __shfl_sync(0xffffffffu, mb, m);
+        if (un.b[m] >= 0 && un.b[m] < p.B && nmem == m) nmem = m + 1;
+      }
+      un.nmem = nmem;
+      if (nmem == 0) return;
+      const int32_t *tr = p.tables + (size_t)un.b[0] * p.max_blocks + (size_t)un.part * nb_unit;
+      if (lane < nb_unit) x0 = tr[lane];
+      if (lane + 32 < nb_unit) x1 = tr[lane + 32];
+    };
+    ShUnit un{};
+    int32_t e0, e1;
+    int u = blockIdx.x;
+    load_unit(u, un, e0, e1);
+    wait_prior_grid();  // the copies read the pool and Q, which may be written just before
+    allow_next_grid();
+    while (ok && u < num_units) {
+      if (un.nmem > 0) {
+        const int qs = qi & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((qi >> 1) & 1) ^ 1))) { ok = false; break; }
+        {
+          int32_t *us = unit_slots + qs * L::kUnitInts;
+          if (lane == 0) {
+            us[0] = un.j;
+            us[1] = un.g;
+            us[2] = un.part;
+            us[3] = un.nmem;
+#pragma unroll
+            for (int m = 0; m < L::kSlots; ++m) us[4 + m] = un.b[m];
+          }
+          us[8 + lane] = e0;
+          if (L::kUnitInts > 8 + 32 + lane) us[8 + 32 + lane] = e1;
+          __syncwarp();
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&qfull[qs], un.nmem * 2 * G * 128);
+          uint8_t *qdst = smem + L::kOffQ + qs * L::kQ;
+          for (int m = 0; m < un.nmem; ++m) {
+            const int qy = un.b[m] * p.Hq + un.g * G;
+            tc::tma_load_2d(qdst + m * 8 * 128, &tmap_q, 0, qy, &qfull[qs], pol_q);
+            tc::tma_load_2d(qdst + N * 128 + m * 8 * 128, &tmap_q, 64, qy, &qfull[qs], pol_q);
+          }
+        }
+        ++qi;
+        for (int ci = 0; ci < kPart / L::kChunk; ++ci, ++c) {
+          const int slot = c % L::kStages, use = c / L::kStages;
+          for (int which = 0; which < 2; ++which) {  // 0: K ring, 1: V ring
+            uint64_t *empty = which ? &vempty[slot] : &kempty[slot];
+            uint64_t *full = which ? &vfull[slot] : &kfull[slot];
+            const CUtensorMap *map = which ? &tmap_v : &tmap_k;
+            if (!__all_sync(0xffffffffu, mbar_wait(empty, (use & 1) ^ 1))) { ok = false; break; }
+            uint8_t *dst = smem + (which ? L::kOffV : L::kOffK) + slot * L::kTile;
+            if (lane == 0) mbar_arrive_expect_tx(full, L::kTile);
+            __syncwarp();
+            const int jloc = ci * blocks_per_chunk + (lane % blocks_per_chunk);
+            const int32_t a0 = __shfl_sync(0xffffffffu, e0, jloc & 31);
+            const int32_t a1 = __shfl_sync(0xffffffffu, e1, jloc & 31);
+            if (lane < blocks_per_chunk) {
+              const int32_t blk = jloc < 32 ? a0 : a1;
+              int w = oob_group;
+              if (blk >= 0 && blk < p.num_blocks) w = (blk * p.Hkv + un.g) * (bs / 8);
+              else if (which == 0) raise_error(PA_DEVERR_TABLE);
+              tc::tma_load_4d(dst + lane * (bs / 8) * L::kGroup, map, 0, 0, 0, w, full, pol_kv);
+            }
+          }
+          if (!ok) break;
+        }
+        if (!ok) break;
+      }
+      u += gridDim.x;
+      load_unit(u, un, e0, e1);
+    }
+    if (ok) {  // no work left: an empty unit stops the consumers
+      const int qs = qi & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((qi >> 1) & 1) ^ 1))) {
+        ok = false;
+      } else {
+        if (lane == 0) unit_slots[qs * L::kUnitInts + 3] = 0;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qfull[qs]);
+      }
+    }
+    if (!ok && lane == 0) {
+      raise_error(PA_DEVERR_TIMEOUT);
+      for (int k = (c > L::kStages ? c - L::kStages : 0); k <= c; ++k) {
+        mbar_wait(&kfull[k % L::kStages], (k / L::kStages) & 1, 100000000ull);
+        mbar_wait(&vfull[k % L::kStages], (k / L::kStages) & 1, 100000000ull);
+      }
+      for (int k = (qi > 2 ? qi - 2 : 0); k < qi; ++k) mbar_wait(&qfull[k & 1], (k >> 1) & 1, 100000000ull);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    wait_prior_grid();
+    allow_next_grid();
+    constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(128, N, false, false);
+    constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(128, N, true, false);
+    const uint32_t kbase0 = smem_u32(smem + L::kOffK), vbase0 = smem_u32(smem + L::kOffV);
+    const uint32_t qbase0 = smem_u32(smem + L::kOffQ), pbase0 = smem_u32(smem + L::kOffP);
+    bool ok = true;
+    auto warp_wait = [&](uint64_t *bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+    };
+    struct PvJob {
+      int c, u;
+      bool first;
+    };
+    auto issue_pv = [&](const PvJob &j) -> bool {
+      const int c = j.c;
+      if (!warp_wait(&pfull[c & 1], (c >> 1) & 1)) return false;
+      if (!warp_wait(&vfull[c % L::kStages], (c / L::kStages) & 1)) return false;
+      if (j.first && !warp_wait(&ofree[j.u & 1], ((j.u >> 1) & 1) ^ 1)) return false;
+      if (lane == 0) {
+        tc::fence_after_sync();
+        const uint32_t vb = vbase0 + (c % L::kStages) * L::kTile;
+        const uint32_t pb = pbase0 + (c & 1) * L::kP;
+        const uint32_t d = tmem + 2 * N + (j.u & 1) * N;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = tc::smem_desc_sw128(vb + kk * 2 * L::kGroup, 1024, L::kGroup);
+          const uint64_t bdesc = tc::smem_desc_sw128(pb + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
+          tc::mma_bf16(d, a, bdesc, idesc_pv, (kk > 0 || !j.first) ? 1u : 0u);
+        }
+        tc::mma_commit(&pvdone[c & 1]);
+        tc::mma_commit(&vempty[c % L::kStages]);
+      }
+      __syncwarp();
+      return true;
+    };
+    int c = 0, qi = 0;
+    PvJob pending{-1, 0, false};
+    while (ok) {
+      const int qs = qi & 1;
+      if (!warp_wait(&qfull[qs], (qi >> 1) & 1)) { ok = false; break; }
+      if (unit_slots[qs * L::kUnitInts + 3] == 0) break;  // the producer ran out of work
+      const uint32_t qb = qbase0 + qs * L::kQ;
+      constexpr int nchunks = kPart / L::kChunk;
+      for (int ci = 0; ci < nchunks; ++ci, ++c) {
+        const int slot = c % L::kStages;
+        if (!warp_wait(&kfull[slot], (c / L::kStages) & 1)) { ok = false; break; }
+        if (lane == 0) {
+          tc::fence_after_sync();
+          const uint32_t kb = kbase0 + slot * L::kTile;
+          const uint32_t d = tmem + (c & 1) * N;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t koff = (kk >> 2) * 1024 + (kk & 3) * 32;
+            const uint64_t a = tc::smem_desc_sw128(kb + koff, 16, L::kGroup);
+            const uint64_t bdesc = tc::smem_desc_sw128(qb + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
+            tc::mma_bf16(d, a, bdesc, idesc_qk, kk > 0);
+          }
+          tc::mma_commit(&sfull[c & 1]);
+          tc::mma_commit(&kempty[slot]);
+          if (ci == nchunks - 1) tc::mma_commit(&qempty[qs]);
+        }
+        __syncwarp();
+        if (pending.c >= 0 && !issue_pv(pending)) { ok = false; break; }
+        pending = PvJob{c, qi, ci == 0};
+      }
+      ++qi;
+    }
+    if (ok && pending.c >= 0 && !issue_pv(pending)) ok = false;
+    if (!ok && lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+    if (lane == 0) tc::mma_commit(drain);
+    __syncwarp();
+    mbar_wait(drain, 0);
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    wait_prior_grid();  // before the first write of the workspace
+    allow_next_grid();
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // token row (softmax) / head-dim row (O)
+    const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
+    const int bs = p.bs;
+    const int log2_bs = bs == 8 ? 3 : (bs == 16 ? 4 : 5);
+    float m[N], l[N];
+    int pun_j = 0, pun_g = 0, pun_part = 0, pun_nmem = 0, pun_b[L::kSlots] = {0, 0, 0, 0};
+    bool pend = false;
+    int p_clast = 0, p_u = 0;
+    bool bad = false, stop = false;
+    auto warp_wait = [&](uint64_t *bar, uint32_t parity) {
+      if (!bad && !__all_sync(0xffffffffu, mbar_wait(bar, parity))) bad = true;
+    };
+    // column n of S / O: member slot n / 8, query head n % 8 of the group
+    auto col_valid = [&](int n, int nmem) { return (n >> 3) < nmem && (n & 7) < G; };
+
+    // the previous unit's O and sums -> its members' workspace rows
+    auto epilogue = [&]() {
+      float o[N];
+      warp_wait(&pvdone[p_clast & 1], (p_clast >> 1) & 1);
+      if (!bad) {
+        tc::fence_after_sync();
+        tc::tmem_ld32(trow + 2 * N + (p_u & 1) * N, o);
+      }
+      tc::fence_before_sync();
+      mbar_arrive(&ofree[p_u & 1]);
+      const int parity = p_u & 1;
+#pragma unroll
+      for (int n = 0; n < N; ++n) {
+        float v = l[n];
+#pragma unroll
+        for (int k = 16; k > 0; k >>= 1) v += __shfl_xor_sync(0xffffffffu, v, k);
+        if (lane == 0) red_sum[(parity * 4 + wq) * N + n] = v;
+      }
+      stop = wg_sync_or(bad);
+      if (stop) return;
+#pragma unroll
+      for (int n = 0; n < N; ++n) {
+        if (!col_valid(n, pun_nmem)) continue;
+        float Ls = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) Ls += red_sum[(parity * 4 + w) * N + n];
+        const int b = pun_b[n >> 3], h = pun_g * G + (n & 7);
+        const size_t row = ((size_t)b * p.Hq + h) * p.max_parts + pun_part;
+        p.ws_acc[row * 128 + r] = o[n];
+        if (r == 0) {
+          p.ws_m[row] = m[n];
+          p.ws_l[row] = Ls;
+        }
+      }
+    };
+
+    int c = 0, qi = 0;
+    for (; !stop; ++qi) {
+      const int qs = qi & 1;
+      warp_wait(&qfull[qs], (qi >> 1) & 1);
+      stop = wg_sync_or(bad);
+      if (stop) break;
+      const int32_t *us = unit_slots + qs * L::kUnitInts;
+      const int nmem = us[3];
+      // the previous unit first, while its statistics are still in m and l
+      if (pend) {
+        epilogue();
+        pend = false;
+        if (stop) break;
+      }
+      if (nmem == 0) break;  // the producer ran out of work
+      const int ug = us[1], upart = us[2];
+      int ub[L::kSlots];
+#pragma unroll
+      for (int k = 0; k < L::kSlots; ++k) ub[k] = us[4 + k];
+      const int32_t *ents = us + 8;
+#pragma unroll
+      for (int n = 0; n < N; ++n) {
+        m[n] = -INFINITY;
+        l[n] = 0.f;
+      }
+      constexpr int nchunks = kPart / L::kChunk;
+      for (int ci = 0; ci < nchunks; ++ci, ++c) {
+        float s[N];
+        warp_wait(&sfull[c & 1], (c >> 1) & 1);
+        if (!bad) {
+          tc::fence_after_sync();
+          tc::tmem_ld32(trow + (c & 1) * N, s);
+        }
+        const int32_t blk = ents[(ci * L::kChunk + r) >> log2_bs];
+        const bool valid = blk >= 0 && blk < p.num_blocks;
+        bool need = false;
+#pragma unroll
+        for (int n = 0; n < N; ++n) {
+          s[n] = (valid && !bad && col_valid(n, nmem)) ? s[n] * p.scale_log2 : -INFINITY;
+          need |= s[n] > m[n] + kLazyRescale;
+        }
+        float mnew[N];
+        if (wg_sync_or(need || bad)) {
+#pragma unroll
+          for (int n = 0; n < N; ++n) {
+            float v = s[n];
+#pragma unroll
+            for (int k = 16; k > 0; k >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, k));
+            if (lane == 0) red_max[((c & 1) * 4 + wq) * N + n] = v;
+          }
+          stop = wg_sync_or(bad);
+          if (stop) break;
+#pragma unroll
+          for (int n = 0; n < N; ++n) {
+            float cm = red_max[((c & 1) * 4 + 0) * N + n];
+#pragma unroll
+            for (int w = 1; w < 4; ++w) cm = fmaxf(cm, red_max[((c & 1) * 4 + w) * N + n]);
+            mnew[n] = fmaxf(m[n], cm);
+          }
+        } else {
+#pragma unroll
+          for (int n = 0; n < N; ++n) mnew[n] = m[n];
+        }
+        // weights of the old reference against the new one: 1 where it stays
+        auto alpha_of = [&](int n) { return mnew[n] == m[n] ? 1.f : exp2f(m[n] - mnew[n]); };
+        bool moved = false;
+#pragma unroll
+        for (int n = 0; n < N; ++n) moved |= mnew[n] != m[n];
+        if (moved && ci > 0) {
+          // rescale the unit's O once PV(c-1) has landed, before PV(c) adds
+          warp_wait(&pvdone[(c - 1) & 1], ((c - 1) >> 1) & 1);
+          if (!bad) {
+            const uint32_t obuf = trow + 2 * N + (qi & 1) * N;
+            float o[N];
+            tc::fence_after_sync();
+            tc::tmem_ld32(obuf, o);
+#pragma unroll
+            for (int k = 0; k < N / 8; ++k) {
+              float o8[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) o8[e] = o[8 * k + e] * alpha_of(8 * k + e);
+              tc::tmem_st8(obuf + 8 * k, o8);
+            }
+          }
+        }
+        __nv_bfloat16 *pb = reinterpret_cast<__nv_bfloat16 *>(smem + L::kOffP + (c & 1) * L::kP);
+        const int kh = r >> 6, rr = r & 63;
+#pragma unroll
+        for (int n = 0; n < N; ++n) {
+          const float pv = s[n] == -INFINITY ? 0.f : exp2f(s[n] - mnew[n]);
+          l[n] = fmaf(l[n], alpha_of(n), pv);
+          m[n] = mnew[n];
+          // P^T row n (K-major, 128-byte swizzle): token r in half kh
+          const int off = kh * (N * 64) + (n >> 3) * 512 + (n & 7) * 64 + (((rr >> 3) ^ (n & 7)) << 3) + (rr & 7);
+          pb[off] = __float2bfloat16_rn(pv);
+        }
+        fence_proxy_async_smem();
+        tc::fence_before_sync();
+        mbar_arrive(&pfull[c & 1]);
+        if (ci == nchunks - 1 && threadIdx.x == 64) mbar_arrive(&qempty[qs]);
+      }
+      if (stop) break;
+      pend = true;
+      pun_j = us[0];
+      pun_g = ug;
+      pun_part = upart;
+      pun_nmem = nmem;
+#pragma unroll
+      for (int k = 0; k < L::kSlots; ++k) pun_b[k] = ub[k];
+      p_clast = c - 1;
+      p_u = qi;
+    }
+    (void)pun_j;
+    if (stop) raise_error(PA_DEVERR_TIMEOUT);
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 1) tc::tmem_dealloc(tmem, L::kTmemCols);
+}
+
+}  // namespace pa

@@ -44,6 +44,10 @@ struct DecodeParams {
   const void *k_new;
   const void *v_new;
   const int32_t *cow_src;
+  // shared-prefix plan (tensor-core kernel): sequence b computes partitions
+  // from first_part[b] on; the ones before are done by the cascade kernel.
+  // Null: every sequence from partition 0.
+  const int32_t *first_part;
 };
 
 constexpr int kPart = PA_PARTITION_TOKENS;

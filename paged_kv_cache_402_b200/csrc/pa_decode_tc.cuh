@@ -69,7 +69,7 @@ struct TcLayout {
   static constexpr int kGroup = 2048;         // one 8-row group: two 1 KiB swizzle atoms (column halves)
   static constexpr int kQ = 2 * kN * 128;     // two halves of kN rows x 128 B
   static constexpr int kP = 2 * kN * 128;     // two 64-token halves of kN rows x 128 B
-  static constexpr int kMaxSeqs = 2048;
+  static constexpr int kMaxSeqs = 1024;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kStages * kTile;
   static constexpr int kOffQ = kOffV + kStages * kTile;
@@ -88,7 +88,8 @@ struct TcLayout {
   static constexpr int kOffScan = kOffUnit + 2 * kUnitInts * 4;  // 8 ints
   static constexpr int kOffPrefix = kOffScan + 32;
   static constexpr int kOffCtx = kOffPrefix + (kMaxSeqs + 1) * 4;
-  static constexpr int kBytes = kOffCtx + kMaxSeqs * 4 + 1024;  // + base alignment slack
+  static constexpr int kOffFirst = kOffCtx + kMaxSeqs * 4;  // first partition of each sequence
+  static constexpr int kBytes = kOffFirst + kMaxSeqs * 4 + 1024;  // + base alignment slack
   static constexpr int kThreads = 192;
   static constexpr uint32_t kTmemCols = 64;  // S0 S1 O0 O1, kN columns each
 };
@@ -116,9 +117,11 @@ __device__ __forceinline__ int pf_of(int32_t v) { return v & ((1 << kFullBits) -
 __device__ __forceinline__ int pp_of(int32_t v) { return (int)((uint32_t)v >> kFullBits); }
 
 // Unit u of the largest-first order: units [0, F) are the full partitions
-// (sequence-major, kv head fastest), units [F, F + P) the partial ones.
+// (sequence-major, kv head fastest; a sequence's start at its first
+// partition), units [F, F + P) the partial ones.
 __device__ __forceinline__ TcUnit tc_unit_at(const DecodeParams &p, const int32_t *prefix,
-                                             const int32_t *ctx_s, int u, int num_full) {
+                                             const int32_t *ctx_s, const int32_t *first_s, int u,
+                                             int num_full) {
   TcUnit un;
   const bool full = u < num_full;
   const int v = full ? u : u - num_full;
@@ -132,7 +135,7 @@ __device__ __forceinline__ TcUnit tc_unit_at(const DecodeParams &p, const int32_
   }
   un.b = lo;
   const int ctx = ctx_s[lo];
-  un.part = full ? w - pf_of(prefix[lo]) : ctx / kPart;
+  un.part = full ? first_s[lo] + w - pf_of(prefix[lo]) : ctx / kPart;
   un.t0 = un.part * kPart;
   un.t1 = min(un.t0 + kPart, ctx);
   un.nchunks = (un.t1 - un.t0 + TcLayout::kChunk - 1) / TcLayout::kChunk;
@@ -177,6 +180,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   uint64_t *pvdone = bars + 20, *ofree = bars + 22, *drain = bars + 24;
   int32_t *prefix = reinterpret_cast<int32_t *>(smem + L::kOffPrefix);
   int32_t *ctx_s = reinterpret_cast<int32_t *>(smem + L::kOffCtx);
+  int32_t *first_s = reinterpret_cast<int32_t *>(smem + L::kOffFirst);
   int32_t *scan = reinterpret_cast<int32_t *>(smem + L::kOffScan);
   int32_t *unit_slots = reinterpret_cast<int32_t *>(smem + L::kOffUnit);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffTmem);
@@ -222,8 +226,15 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       const int ctx = p.lens[b];
       const bool ok = ctx >= 0 && ctx <= p.max_ctx;
       ctx_s[b] = ctx;
+      // partitions the cascade kernel did: whole ones before the last
+      int fp = p.first_part ? p.first_part[b] : 0;
+      if (fp != 0 && (!ok || fp < 0 || (int64_t)fp * kPart >= ctx)) {
+        if (blockIdx.x == 0) raise_error(PA_DEVERR_PLAN);
+        fp = 0;  // this kernel then does the whole sequence
+      }
+      first_s[b] = fp;
       // full partitions in the low bits, a partial last partition in the high ones
-      cnt[i] = (ok && ctx > 0) ? (ctx / kPart) | ((ctx % kPart != 0 ? 1 : 0) << kFullBits) : 0;
+      cnt[i] = (ok && ctx > 0) ? (ctx / kPart - fp) | ((ctx % kPart != 0 ? 1 : 0) << kFullBits) : 0;
       mine += cnt[i];
       if (blockIdx.x == 0 && !ok) raise_error(PA_DEVERR_LEN);
     }
@@ -284,7 +295,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       x0 = x1 = -1;
       nd = ns = -1;
       if (u < num_units) {
-        nu = tc_unit_at(p, prefix, ctx_s, u, num_full);
+        nu = tc_unit_at(p, prefix, ctx_s, first_s, u, num_full);
         const int32_t *tr = p.tables + (size_t)nu.b * p.max_blocks + nu.t0 / bs;
         const int nb = (nu.t1 - nu.t0 + bs - 1) / bs;
         const bool newest = p.k_new != nullptr && nu.t1 == ctx_s[nu.b];

@@ -275,3 +275,61 @@ def test_seqs_max_len():
     assert A.max_len(s) == (30, 4)
     assert A.max_len(s[:1]) == (5, 1)
     assert A.max_len([]) == (0, 0)
+
+
+def test_share_plan_groups():
+    """Buckets by the first partition's entries, groups of at most
+    max_members in sequence order, a lone leftover in no group, and the shared
+    partitions stop where the tables part or a member's last partition
+    starts."""
+    t = np.full((7, 96), -1, np.int32)
+    for i in (0, 1, 2):                       # share 40 blocks, then private
+        t[i, :40] = np.arange(40)
+        t[i, 40:50] = 100 + 10 * i + np.arange(10)
+    t[3, :60] = 200 + np.arange(60)           # alone
+    t[4, :40] = np.arange(40)                 # joins 0..2 (same first partition)
+    t[4, 40:45] = 500 + np.arange(5)
+    for i in (5, 6):                          # share two whole partitions
+        t[i, :70] = 1000 + np.arange(70)
+        t[i, 70:80] = 2000 + 10 * i + np.arange(10)
+    lens = np.array([50 * 16, 49 * 16 + 3, 45 * 16, 60 * 16, 1024, 80 * 16, 75 * 16], np.int32)
+    pl = pa.share_plan(t, lens, 16)
+    assert pl.members.tolist() == [[0, 1, 2, 4], [5, 6, -1, -1]]
+    assert pl.parts.tolist() == [1, 2]
+    assert pl.first_part.tolist() == [1, 1, 1, 0, 1, 2, 2]
+    pl3 = pa.share_plan(t, lens, 16, max_members=3)       # 0, 1, 2 | 4 alone
+    assert pl3.members.tolist() == [[0, 1, 2], [5, 6, -1]]
+    assert pl3.first_part.tolist() == [1, 1, 1, 0, 0, 2, 2]
+    short = lens.copy()
+    short[6] = 1024                           # partition 1 is now 6's last: one shared partition
+    assert pa.share_plan(t, short, 16).parts.tolist() == [1, 1]
+    short[6] = 512                            # a single partition: in no group
+    pl = pa.share_plan(t, short, 16)
+    assert pl.members.tolist() == [[0, 1, 2, 4]] and pl.first_part[5] == 0 and pl.first_part[6] == 0
+
+
+def test_share_plan_of_allocator_forks():
+    """Forks of a 1300-token prompt share its first two partitions (the third
+    holds the fork point's partial block, copied on write)."""
+    A = pa.Allocator(256, 16, list(range(256)))
+    r = A.new_seq()
+    A.batch_append([r], [1300])
+    seqs = [r] + [A.fork(r) for _ in range(5)]
+    A.batch_append(seqs, [1] * 6)
+    tables, lens = A.build_block_tables(seqs, 90)
+    pl = pa.share_plan(tables, lens, 16)
+    assert pl.members.tolist() == [seqs[:4], seqs[4:] + [-1, -1]]
+    assert pl.parts.tolist() == [2, 2] and pl.first_part.tolist() == [2] * 6
+
+
+def test_decode_shared_argument_checks():
+    c = _cache_struct()
+    L = pa.lib()
+    plan = pa.pa_share_plan_t(16, 16, 16, 1, 5)
+    args = lambda **o: [None, None, None, 16, ctypes.byref(c), 16, o.get("mb", 64), 16, 1, 2, o.get("ml", 1000),
+                        1.0, ctypes.byref(o.get("plan", plan)), 16, 16, 1 << 20, None]
+    assert L.pa_decode_shared(*args()) == pa.PA_ERR_INVALID_ARG                 # 5 members > 4
+    ok_plan = pa.pa_share_plan_t(16, 16, 16, 1, 4)
+    assert L.pa_decode_shared(*args(plan=ok_plan, ml=500, mb=32)) == pa.PA_ERR_INVALID_ARG  # one partition
+    bad = pa.pa_share_plan_t(0, 16, 16, 1, 4)
+    assert L.pa_decode_shared(*args(plan=bad)) == pa.PA_ERR_INVALID_ARG         # no member array
