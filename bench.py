@@ -595,7 +595,7 @@ def run_e2e(args, insts, wl, dev, stream):
                                     workspace=ws, stream=stream)
             else:
                 plan = pa.share_plan(tables_np, lens_np, bs).to(dev)
-                plan_bytes += plan.members.nbytes + plan.parts.nbytes + plan.first_part.nbytes
+                plan_bytes += plan.nbytes
                 pa.pa_decode_shared(d["q"], inst.cache, d["tables"], d["lens"], int(lens_np.max()),
                                     1.0 / math.sqrt(D), plan=plan, k_new=d["k"], v_new=d["v"],
                                     cow_src=d["cow"] if npairs else None, out=out, workspace=ws, stream=stream)
@@ -699,7 +699,7 @@ def run_trace(args, dev):
                 pa.pa_decode_shared(q, cache, d_[3], d_[4], max_ctx, 1 / math.sqrt(D), plan=splan.to(dev),
                                     k_new=kd, v_new=kd, cow_src=d_[5], out=o, workspace=ws, stream=stream)
                 launches += 1 + (1 if max_ctx > pa.PA_PARTITION_TOKENS else 0) + (1 if splan.n_groups else 0)
-                h2d += splan.members.nbytes + splan.parts.nbytes + splan.first_part.nbytes
+                h2d += splan.nbytes
             ev[s_][1].record(stream)
             res = o[:1].to("cpu", non_blocking=True)
             torch.cuda.synchronize()

@@ -202,9 +202,9 @@ typedef struct {
  * once for all its members ("pagedattention" glossary entry, paragraph 5:
  * sequences that share a prefix point at the same physical blocks;
  * "PagedAttention Internals", "Sharing And Dynamic Growth").  The result is
- * that of pa_decode / pa_append_decode up to the rounding of the fp32 sums
- * (the same sums in the same order: each member's partition statistics are
- * computed over the same tiles).  plan may be NULL or have no groups; on the
+ * bit for bit that of pa_decode / pa_append_decode: each member's statistics
+ * over a shared partition come from the same tiles through the same
+ * per-column arithmetic.  plan may be NULL or have no groups; on the
  * CUDA-core path (not bf16 with head_dim 128) the plan is not used and every
  * sequence computes all of its partitions.
  *   k_new, v_new, cow_src  as pa_append_decode, or all NULL for no append

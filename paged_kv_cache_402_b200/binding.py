@@ -282,12 +282,17 @@ class SharePlan:
         self._dev = None
 
     def to(self, device, stream=None) -> "SharePlan":
-        """Copies the arrays to the device (kept until the plan is dropped)."""
-        nb = self.n_groups > 0
-        self._dev = tuple(torch.from_numpy(np.ascontiguousarray(a)).to(device, non_blocking=True)
-                          for a in ((self.members if nb else np.full((1, 1), -1, np.int32)),
-                                    (self.parts if nb else np.zeros(1, np.int32)), self.first_part))
+        """Copies the arrays to the device (kept until the plan is dropped);
+        a plan without groups needs none."""
+        if self.n_groups > 0:
+            self._dev = tuple(torch.from_numpy(np.ascontiguousarray(a)).to(device, non_blocking=True)
+                              for a in (self.members, self.parts, self.first_part))
         return self
+
+    @property
+    def nbytes(self) -> int:
+        """Bytes the device copy takes (0 without groups)."""
+        return 0 if self.n_groups == 0 else self.members.nbytes + self.parts.nbytes + self.first_part.nbytes
 
     def ref(self):
         if self.n_groups == 0:

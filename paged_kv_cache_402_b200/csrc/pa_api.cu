@@ -560,6 +560,7 @@ PA_API pa_status pa_decode_shared(const void *k_new, const void *v_new, const in
     s = launch_decode_shared(p, *plan, st);
     if (s != PA_OK) return s;
     p.first_part = plan->first_part;
+    p.late_wait = 1;
   }
   p.k_new = k_new;
   p.v_new = v_new;

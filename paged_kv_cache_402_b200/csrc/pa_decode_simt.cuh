@@ -48,6 +48,12 @@ struct DecodeParams {
   // from first_part[b] on; the ones before are done by the cascade kernel.
   // Null: every sequence from partition 0.
   const int32_t *first_part;
+  // tensor-core kernel launched right after the cascade kernel: nothing it
+  // reads or writes is touched by that kernel, and everything of the calls
+  // before it had completed when the cascade kernel let it start, so it waits
+  // for the cascade kernel only before it finishes (the reduce after it
+  // reads both kernels' workspace rows)
+  int32_t late_wait;
 };
 
 constexpr int kPart = PA_PARTITION_TOKENS;

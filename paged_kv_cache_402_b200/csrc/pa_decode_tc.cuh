@@ -354,7 +354,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     int32_t e0, e1, nd, ns;
     int u = blockIdx.x;  // the first unit of every CTA is fixed; later ones are drawn
     load_entries(u, un, e0, e1, nd, ns);
-    wait_prior_grid();  // the copies read the pool and Q, which may be written just before
+    if (!p.late_wait) wait_prior_grid();  // the copies read the pool and Q, which may be written just before
     allow_next_grid();
     while (ok && u < num_units) {
       const int nb_unit = (un.t1 - un.t0 + bs - 1) / bs;
@@ -447,7 +447,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     // the QK MMA) and value row (lanes 16-31, once the V tile has landed,
     // before the PV MMA) into the tiles of its chunk, and store them to the
     // pool.
-    wait_prior_grid();
+    if (!p.late_wait) wait_prior_grid();
     allow_next_grid();
     constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(128, N, false, false);
     constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(128, N, true, false);
@@ -572,7 +572,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     mbar_wait(drain, 0);
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    wait_prior_grid();  // before the first write of out / the workspace
+    if (!p.late_wait) wait_prior_grid();  // before the first write of out / the workspace
     allow_next_grid();
     const int wq = warp & 3;              // this warp's quarter of the TMEM lanes
     const int r = wq * 32 + lane;         // token row (softmax) / head-dim row (O)
@@ -794,6 +794,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     if (stop) raise_error(PA_DEVERR_TIMEOUT);
   }
 
+  if (p.late_wait) wait_prior_grid();  // complete only after the cascade kernel
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
