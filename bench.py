@@ -339,6 +339,18 @@ WORKLOADS = {
 }
 
 
+def aggregate_ranks(world: int, ms: float, kv_gb: float, tokens: float, e2e_s: float, e2e_gb: float, device):
+    """Whole-job figures of the replicas: the slowest rank's times, the sum
+    of every rank's work.  Returns (ms, GB, tokens, end-to-end GB/s).  Every
+    rank takes the same two collectives in the same order."""
+    t = torch.tensor([ms, e2e_s], dtype=torch.float64, device=device)
+    w = torch.tensor([kv_gb, tokens, e2e_gb], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.all_reduce(w, op=torch.distributed.ReduceOp.SUM)
+    return float(t[0]), float(w[0]), float(w[1]), float(w[2]) / float(t[1])
+
+
 def run_ours(args, rank: int, world: int, dev):
     import paged_kv_cache_402_b200 as pa
 
@@ -448,21 +460,8 @@ def run_ours(args, rank: int, world: int, dev):
     # end to end through the public API with pinned host buffers
     e2e = run_e2e(args, insts, wl, dev, stream)
 
-    t = torch.tensor([ms, kv_bytes / 1e9, float(args.steps * wl["B"])], dtype=torch.float64, device=dev)
-    if world > 1:
-        tmax = t[:1].clone()
-        torch.distributed.all_reduce(tmax, op=torch.distributed.ReduceOp.MAX)
-        tsum = t[1:].clone()
-        torch.distributed.all_reduce(tsum, op=torch.distributed.ReduceOp.SUM)
-        ms_all, gb_all, tok_all = float(tmax[0]), float(tsum[0]), float(tsum[1])
-        e2e_t = torch.tensor([e2e["seconds"]], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
-        e2e_gb = torch.tensor([e2e["kv_gb"]], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(e2e_gb, op=torch.distributed.ReduceOp.SUM)
-        e2e_value = float(e2e_gb[0]) / float(e2e_t[0])
-    else:
-        ms_all, gb_all, tok_all = ms, kv_bytes / 1e9, float(args.steps * wl["B"])
-        e2e_value = e2e["kv_gb"] / e2e["seconds"]
+    ms_all, gb_all, tok_all, e2e_value = aggregate_ranks(world, ms, kv_bytes / 1e9, float(args.steps * wl["B"]),
+                                                         e2e["seconds"], e2e["kv_gb"], dev)
 
     peak, peak_kind = measured_peaks()
     dec_avg_s = statistics.mean(dec_ms) / 1e3
@@ -873,12 +872,14 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
-    if args.workload == "trace":
-        if rank == 0:
-            for line in run_trace(args, dev):
-                print(json.dumps(line), flush=True)
-        return
     try:
+        if args.workload == "trace":  # one trace, on rank 0; the other ranks only join the exit
+            if rank == 0:
+                for line in run_trace(args, dev):
+                    print(json.dumps(line), flush=True)
+            if world > 1:
+                torch.distributed.barrier()
+            return
         line = run_ours(args, rank, world, dev)
         if rank == 0 and world == 1 and not args.no_cpu_baseline and "lengths" in WORKLOADS[args.workload]:
             wl = WORKLOADS[args.workload]

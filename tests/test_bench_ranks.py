@@ -1,0 +1,66 @@
+"""The replica path of bench.py on the host: two gloo ranks aggregate their
+timings (slowest rank's time, summed work), and the reference arm prints one
+line from rank 0 only."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        # rank r: 10 + r ms, (r + 1) GB, 100 tokens, e2e 2 + r s for (r + 1) GB
+        res = bench.aggregate_ranks(world, 10.0 + rank, rank + 1.0, 100.0, 2.0 + rank, rank + 1.0,
+                                    torch.device("cpu"))
+        with open(os.path.join(out_dir, f"r{rank}.json"), "w") as f:
+            json.dump(res, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_aggregation(tmp_path):
+    port = _free_port()
+    mp.start_processes(_rank_main, args=(2, port, str(tmp_path)), nprocs=2, start_method="spawn", join=True)
+    for r in range(2):
+        ms, gb, tok, e2e = json.load(open(tmp_path / f"r{r}.json"))
+        assert ms == 11.0 and gb == 3.0 and tok == 200.0
+        assert e2e == pytest.approx(3.0 / 3.0)
+
+
+def test_single_rank_aggregation_needs_no_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.aggregate_ranks(1, 5.0, 2.0, 7.0, 4.0, 2.0, torch.device("cpu")) == (5.0, 2.0, 7.0, 0.5)
+
+
+@pytest.mark.parametrize("rank", [0, 1])
+def test_reference_arm_prints_on_rank_zero_only(rank):
+    env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank), MASTER_ADDR="127.0.0.1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    if rank == 0:
+        assert len(lines) == 1
+        d = json.loads(lines[0])
+        assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+        assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+    else:
+        assert lines == []
