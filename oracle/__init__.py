@@ -73,6 +73,10 @@ def load(path: str) -> ctypes.CDLL:
     L.oracle_merge_partials.argtypes = [f64p, f64p, f64p, i32p, ctypes.c_int64,
                                         ctypes.c_int, ctypes.c_int, f64p]
     L.oracle_merge_partials.restype = None
+    L.oracle_prefill.argtypes = [vp, vp, vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                                 ctypes.c_int, ctypes.c_int, i32p, ctypes.c_int, i32p, i32p,
+                                 ctypes.c_int, ctypes.c_int, ctypes.c_double, i32p, ctypes.c_int, f64p]
+    L.oracle_prefill.restype = ctypes.c_int
     L.oracle_set_threads.argtypes = [ctypes.c_int]
     L.oracle_max_threads.restype = ctypes.c_int
     return L
@@ -176,6 +180,47 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, scale, rows=None) ->
         _ptr(out, ctypes.c_double))
     if rc:
         raise ValueError(f"oracle_decode rejected its input (code {rc})")
+    return out
+
+
+def prefill(q, k_cache, v_cache, block_tables, context_lens, query_starts, scale, rows=None) -> np.ndarray:
+    """Paged chunked-prefill attention in float64 (the C oracle).
+
+    The last n_b = query_starts[b+1] - query_starts[b] tokens of sequence b
+    (context_lens[b] tokens in all) are new; their queries are rows
+    query_starts[b] .. query_starts[b+1]-1 of q [total, Hq, D], and each
+    attends causally to the sequence's tokens up to its own position.
+    Returns [total, Hq, D] float64, or [len(rows), D] for rows = [(j, h), ...].
+    """
+    qa, qc = host_array(q)
+    ka, kc = host_array(k_cache)
+    va, vc = host_array(v_cache)
+    if not (qc == kc == vc):
+        raise TypeError("q, k_cache and v_cache must share one element type")
+    T, Hq, D = qa.shape
+    NB, Hkv, bs, D2 = ka.shape
+    if D2 != D or va.shape != ka.shape:
+        raise ValueError("shape mismatch")
+    tables = np.ascontiguousarray(np.asarray(block_tables, dtype=np.int32))
+    lens = np.ascontiguousarray(np.asarray(context_lens, dtype=np.int32))
+    qs = np.ascontiguousarray(np.asarray(query_starts, dtype=np.int32))
+    B = lens.shape[0]
+    if tables.ndim != 2 or tables.shape[0] != B or qs.shape != (B + 1,) or int(qs[-1]) != T:
+        raise ValueError("table / length / query start shape mismatch")
+    if rows is None:
+        out = np.zeros((T, Hq, D), dtype=np.float64)
+        rows_a, n_rows = None, 0
+    else:
+        rows_a = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 2))
+        n_rows = rows_a.shape[0]
+        out = np.zeros((n_rows, D), dtype=np.float64)
+    rc = lib().oracle_prefill(
+        qa.ctypes.data, ka.ctypes.data, va.ctypes.data, qc, NB, Hkv, bs, D,
+        _ptr(tables, ctypes.c_int32), tables.shape[1], _ptr(lens, ctypes.c_int32), _ptr(qs, ctypes.c_int32),
+        B, Hq, float(scale), None if rows_a is None else _ptr(rows_a, ctypes.c_int32), n_rows,
+        _ptr(out, ctypes.c_double))
+    if rc:
+        raise ValueError(f"oracle_prefill rejected its input (code {rc})")
     return out
 
 

@@ -236,3 +236,74 @@ void oracle_merge_partials(const double *m, const double *l, const double *acc,
     for (int d = 0; d < D; ++d) o[d] /= L;
   }
 }
+
+/*
+ * Paged prefill (chunked-prefill) attention.  Sequence b holds lens[b]
+ * tokens in the cache; the last n_b = qstart[b+1] - qstart[b] of them are
+ * its new tokens, whose queries are rows qstart[b] .. qstart[b+1]-1 of q.
+ * New token i sits at position p = lens[b] - n_b + i and attends to the
+ * sequence's tokens 0..p only (causal), through the block table:
+ *   s_t = scale * <q[qstart[b] + i, h], k_t>,   t = 0..p
+ *   out[qstart[b] + i, h] = sum_t exp(s_t - max_s) v_t / sum_t exp(s_t - max_s)
+ * the same textbook step as the decode, here for every new token (the decode
+ * is the case n_b = 1).  Two-pass softmax in float64, no tiling.
+ *   q   : [total][Hq][D] of `dtype`, total = qstart[B]
+ *   out : [total][Hq][D] float64 when rows == NULL, else [n_rows][D] with
+ *         rows[2*i] = query row j (0 <= j < total), rows[2*i+1] = h.
+ * Returns 0, or a nonzero code for malformed input (nothing written).
+ */
+int oracle_prefill(const void *q, const void *k_cache, const void *v_cache, int dtype,
+                   int64_t num_blocks, int Hkv, int bs, int D, const int32_t *tables,
+                   int max_blocks, const int32_t *lens, const int32_t *qstart, int B, int Hq,
+                   double scale, const int32_t *rows, int n_rows, double *out) {
+  int rc = orc_check(num_blocks, Hkv, bs, D, tables, max_blocks, lens, B, Hq);
+  if (rc) return rc;
+  if (qstart[0] != 0) return 8;
+  for (int b = 0; b < B; ++b) {
+    int n = qstart[b + 1] - qstart[b];
+    if (n < 0 || n > lens[b]) return 9;
+  }
+  const int64_t total_q = qstart[B];
+  const int G = Hq / Hkv;
+  int64_t total = rows ? (int64_t)n_rows : total_q * Hq;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t i = 0; i < total; ++i) {
+    int64_t j;
+    int h;
+    if (rows) {
+      j = rows[2 * i];
+      h = rows[2 * i + 1];
+    } else {
+      j = i / Hq;
+      h = (int)(i % Hq);
+    }
+    double *o = out + i * D;
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    if (j < 0 || j >= total_q || h < 0 || h >= Hq) continue;
+    int b = 0;  /* the sequence whose query rows hold j */
+    while (qstart[b + 1] <= j) ++b;
+    const int n = qstart[b + 1] - qstart[b];
+    const int p = lens[b] - n + (int)(j - qstart[b]);
+    const int g = h / G;
+    const int64_t qoff = (j * Hq + h) * D;
+    double *s = (double *)malloc(sizeof(double) * (size_t)(p + 1));
+    double m = -INFINITY;
+    for (int t = 0; t <= p; ++t) {
+      int64_t kr = orc_row(tables, max_blocks, b, t, Hkv, bs, D, g);
+      double dot = 0.0;
+      for (int d = 0; d < D; ++d) dot += orc_load(q, dtype, qoff + d) * orc_load(k_cache, dtype, kr + d);
+      s[t] = dot * scale;
+      if (s[t] > m) m = s[t];
+    }
+    double denom = 0.0;
+    for (int t = 0; t <= p; ++t) {
+      double w = exp(s[t] - m);
+      denom += w;
+      int64_t vr = orc_row(tables, max_blocks, b, t, Hkv, bs, D, g);
+      for (int d = 0; d < D; ++d) o[d] += w * orc_load(v_cache, dtype, vr + d);
+    }
+    for (int d = 0; d < D; ++d) o[d] /= denom;
+    free(s);
+  }
+  return 0;
+}

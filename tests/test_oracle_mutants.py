@@ -25,6 +25,10 @@ MUTANTS = {
                           "return ((blk * bs + off) * Hkv + g) * (int64_t)D;"),
     "merge-missing-rescale": ("L += l[i * max_parts + p] * w;", "L += l[i * max_parts + p];"),
     "partial-max-skipped": ("if (s[t - t0] > m) m = s[t - t0];", "m = 0.0;"),
+    "prefill-causal-limit": ("for (int t = 0; t <= p; ++t) {\n      int64_t kr", "for (int t = 0; t < p; ++t) {\n      int64_t kr"),
+    "prefill-dropped-scale": ("s[t] = dot * scale;", "s[t] = dot;"),
+    "prefill-no-prefix": ("const int p = lens[b] - n + (int)(j - qstart[b]);", "const int p = (int)(j - qstart[b]);"),
+    "prefill-query-row": ("const int64_t qoff = (j * Hq + h) * D;", "const int64_t qoff = ((int64_t)b * Hq + h) * D;"),
     "bf16-wrong-half": ("uint32_t u = ((uint32_t)((const uint16_t *)base)[i]) << 16;",
                         "uint32_t u = ((uint32_t)((const uint16_t *)base)[i]);"),
 }
@@ -37,6 +41,9 @@ PIN_TESTS = [
     pins.test_dominant_key_selects_its_value,
     lambda: [pins.test_partitioned_merge_equals_single_pass(p) for p in (4, 16)],
     pins.test_bf16_inputs_match_widened_f64,
+    lambda: [pins.test_prefill_equals_dense_causal(s) for s in (0, 1)],
+    pins.test_prefill_is_causal,
+    pins.test_prefill_last_token_is_bruteforce_decode,
 ]
 
 

@@ -313,3 +313,91 @@ def test_tiny_case_reads_no_unowned_block():
     case = synth.tiny_fp32_case(0)
     out = oracle.decode(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens, case.scale)
     assert np.isfinite(out).all()
+
+
+# ------------------------------------------------------------- prefill
+
+
+def _torch_dense_causal(qrows, kd, vd, starts, lens, scale):
+    """For every sequence b, its last n_b tokens' queries against its dense
+    keys with a causal mask (query i of the chunk sees keys 0 .. L - n + i),
+    softmax and weighted values by torch in float64."""
+    outs = []
+    for b in range(len(lens)):
+        L, n = int(lens[b]), int(starts[b + 1] - starts[b])
+        if n == 0:
+            continue
+        Q = qrows[starts[b]:starts[b + 1]].double()                    # [n, Hq, D]
+        Hq, Hkv = Q.shape[1], kd[b].shape[1]
+        K = kd[b].double().repeat_interleave(Hq // Hkv, dim=1)           # [L, Hq, D]
+        V = vd[b].double().repeat_interleave(Hq // Hkv, dim=1)
+        s = torch.einsum("ihd,thd->hit", Q, K) * scale                   # [Hq, n, L]
+        pos = torch.arange(L - n, L).view(1, n, 1)
+        s = s.masked_fill(torch.arange(L).view(1, 1, L) > pos, float("-inf"))
+        outs.append(torch.einsum("hit,thd->ihd", torch.softmax(s, dim=-1), V))
+    return torch.cat(outs).numpy()
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_prefill_equals_dense_causal(seed):
+    """Chunks of new tokens (a whole prompt, a chunk after a cached prefix, a
+    single token, none) against torch's masked softmax over the dense keys."""
+    lens = [40, 17, 70, 9]
+    news = [40, 5, 33, 0]
+    q0, kc, vc, tables, lens_a, kd, vd = _dense_case(seed, lens, Hq=6, Hkv=2, D=16, bs=4)
+    starts = np.concatenate([[0], np.cumsum(news)]).astype(np.int32)
+    g = torch.Generator().manual_seed(100 + seed)
+    qrows = torch.randn(int(starts[-1]), 6, 16, generator=g, dtype=torch.float64)
+    out = oracle.prefill(qrows, kc, vc, tables, lens_a, starts, 0.4)
+    ref = _torch_dense_causal(qrows, kd, vd, starts, lens_a, 0.4)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-13)
+
+
+def test_prefill_is_causal():
+    """Changing the keys and values after a new token's position changes
+    nothing for it, and changes the tokens that see them."""
+    lens = [30]
+    q0, kc, vc, tables, lens_a, kd, vd = _dense_case(3, lens, Hq=2, Hkv=1, D=8, bs=4)
+    starts = np.array([0, 12], np.int32)  # positions 18 .. 29 are new
+    qrows = torch.randn(12, 2, 8, generator=torch.Generator().manual_seed(7), dtype=torch.float64)
+    before = oracle.prefill(qrows, kc, vc, tables, lens_a, starts, 0.5)
+    blk, off = int(tables[0, 25 // 4]), 25 % 4  # token 25
+    kc[blk, :, off] += 3.0
+    vc[blk, :, off] -= 2.0
+    after = oracle.prefill(qrows, kc, vc, tables, lens_a, starts, 0.5)
+    np.testing.assert_array_equal(before[:25 - 18], after[:25 - 18])
+    assert np.abs(before[25 - 18:] - after[25 - 18:]).min() > 0
+
+
+def test_prefill_last_token_is_bruteforce_decode():
+    """The chunk's last token sees the whole context: the pure-Python loop
+    over the allocator's slots (no table) gives the same row."""
+    bs, Hkv, Hq, D, NB = 4, 2, 4, 8, 24
+    A = oracle.AllocatorModel(NB, bs, synth.rng(31).permutation(NB))
+    lens = [9, 14]
+    slot_lists = []
+    for L in lens:
+        sid = A.new_seq()
+        slots, cow = A.append(sid, L)
+        assert cow is None
+        slot_lists.append(slots)
+    g = torch.Generator().manual_seed(32)
+    kc = torch.randn(NB, Hkv, bs, D, generator=g, dtype=torch.float64)
+    vc = torch.randn(NB, Hkv, bs, D, generator=g, dtype=torch.float64)
+    news = [3, 14]
+    starts = np.array([0, 3, 17], np.int32)
+    qrows = torch.randn(17, Hq, D, generator=g, dtype=torch.float64)
+    tables = np.full((2, 4), -1, np.int32)
+    for s in range(2):
+        t = A.block_table(s)
+        tables[s, :len(t)] = t
+    out = oracle.prefill(qrows, kc, vc, tables, lens, starts, 0.6)
+    for b in range(2):
+        last = int(starts[b + 1]) - 1
+        ref = oracle.decode_bruteforce(qrows[last:last + 1], kc, vc, [slot_lists[b]], 0.6)
+        np.testing.assert_allclose(out[last], ref[0], rtol=0, atol=1e-12)
+        # and the chunk's first token sees only the tokens up to its position
+        first = int(starts[b])
+        p = lens[b] - news[b]
+        ref = oracle.decode_bruteforce(qrows[first:first + 1], kc, vc, [slot_lists[b][:p + 1]], 0.6)
+        np.testing.assert_allclose(out[first], ref[0], rtol=0, atol=1e-12)
