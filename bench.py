@@ -44,6 +44,7 @@ import torch  # noqa: E402
 
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 METRIC = "paged decode KV-read GB/s (% of HBM peak) and decode tokens/s at 1 B200"
 
 
@@ -58,6 +59,16 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s of this machine's B200s (burst: a kernel timed alone),
+    from MEASURED_PEAKS.json, else the fallback figure."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def kernel_source_hash() -> str:
@@ -611,6 +622,106 @@ def run_e2e(args, insts, wl, dev, stream):
     return {"seconds": seconds, "kv_gb": kv / 1e9, "steps": n_steps, "h2d": h2d, "d2h": d2h}
 
 
+def run_prefill(args, rank: int, world: int, dev):
+    """Chunked-prefill attention over batches of new prompts (the trace's
+    prompt shape: lognormal lengths, median 512, clipped to [1, 4096]), 32 q
+    / 8 kv heads, head_dim 128, 16-token blocks.  A step appends every
+    prompt's K/V rows (pa_append_kv) and runs pa_prefill over them; the
+    metric is causal attention FLOP/s (QK^T and PV, 4 * D per visible key
+    per query row and head) against the measured bf16 tensor peak."""
+    import paged_kv_cache_402_b200 as pa
+    from paged_kv_cache_402_b200 import synth
+
+    B, Hq, Hkv, D, bs = 32, 32, 8, 128, 16
+    dt = torch.bfloat16
+    R = 2
+    insts = []
+    for i in range(R):
+        seed = 1000 * rank + 31 * i + args.seed
+        r = synth.rng(seed)
+        n = np.clip(np.round(np.exp(r.normal(math.log(512), 1.0, size=B))), 1, 4096).astype(np.int64)
+        NB = 2 * int(sum(-(-int(x) // bs) for x in n)) + 8
+        A = pa.Allocator(NB, bs, synth.rng(seed + 1).permutation(NB))
+        seqs = [A.new_seq() for _ in range(B)]
+        slots, _ = A.batch_append(seqs, n.tolist())
+        mb = max(len(A.block_table(s_)) for s_ in seqs)
+        tables, lens = A.build_block_tables(seqs, mb)
+        starts = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+        T = int(starts[-1])
+        insts.append({
+            "cache": pa.KVCache.empty(NB, Hkv, bs, D, dt, dev),
+            "k": synth.normal((T, Hkv, D), dt, seed + 2, device=dev),
+            "v": synth.normal((T, Hkv, D), dt, seed + 3, device=dev),
+            "q": synth.normal((T, Hq, D), dt, seed + 4, device=dev),
+            "out": torch.empty(T, Hq, D, dtype=dt, device=dev),
+            "slots": torch.from_numpy(slots).to(dev), "tables": torch.from_numpy(tables).to(dev),
+            "lens": torch.from_numpy(lens).to(dev), "starts": torch.from_numpy(starts).to(dev),
+            "max_ctx": int(lens.max()), "max_q": int(n.max()), "tokens": T,
+            # visible keys per query row: position + 1 (whole prompts)
+            "flops": 4 * D * Hq * int(sum(x * (x + 1) // 2 for x in n)),
+        })
+    stream = torch.cuda.current_stream()
+
+    def step(s_, strm):
+        it = insts[s_ % R]
+        pa.pa_append_kv(it["k"], it["v"], it["slots"], it["cache"], strm)
+        pa.pa_prefill(it["q"], it["cache"], it["tables"], it["lens"], it["starts"], it["max_ctx"],
+                      1.0 / math.sqrt(D), max_query_len=it["max_q"], out=it["out"], stream=strm)
+        return it
+
+    for s_ in range(args.warmup):
+        step(s_, stream)
+    torch.cuda.synchronize()
+    if pa.pa_read_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+    graph = torch.cuda.CUDAGraph()
+    flops = tokens = 0
+    with torch.cuda.graph(graph):
+        cap = torch.cuda.current_stream()
+        for i in range(args.steps):
+            it = step(args.warmup + i, cap)
+            flops += it["flops"]
+            tokens += it["tokens"]
+    graph.replay()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        t0.record(stream)
+        graph.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    del graph
+    if world > 1:
+        torch.distributed.barrier()
+    ms = t0.elapsed_time(t1)
+    if pa.pa_read_device_error() != 0:
+        raise RuntimeError("device error during the timed steps")
+    ms_all, fl_all, tok_all, _ = aggregate_ranks(world, ms, flops / 1e12, float(tokens), 1.0, 0.0, dev)
+    peak, kind = measured_tensor_peak()
+    tflops = fl_all / (ms_all / 1e3)
+    return {
+        "metric": "paged chunked-prefill attention TFLOP/s (causal, bf16 in, fp32 accumulate) at 1 B200",
+        "workload": "prefill", "value": round(tflops, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_all / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) q/k/v; seeded prompt lengths and block placement)",
+        "config": {"workload": "bf16 paged prefill: 32 prompts, lengths lognormal (median 512, clipped to "
+                               "[1, 4096]), 32 q / 8 kv heads, head_dim 128, 16-token blocks; step = append of "
+                               "the prompts' K/V + causal attention of every prompt token",
+                   "global_batch": B * world, "l2": f"{R} rotating batch instances",
+                   "timing": "CUDA graph replay of the K steps", "parallelism": f"replicas x{world}"},
+        "tokens_per_s": round(tok_all / (ms_all / 1e3), 1),
+        "roofline": {"bound": "tensor", "kernel": "pa_append_kv + pa_prefill", "achieved": round(tflops, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
+                     "peak_source": f"{kind} bf16_tflops (dense, burst)", "traffic": None},
+        "clocks": clk.summary(),
+        "gpu_launches": 2 * args.steps,
+    }
+
+
 def run_trace(args, dev):
     """Continuous batching of beam-search requests over a 16 GiB K+V pool, one
     JSON line per block size: per step the host trace driver (allocator
@@ -841,7 +952,7 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["trace"], default="gqa")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["trace", "prefill"], default="gqa")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rotate", type=int, default=0, help="batch instances to rotate (0: the workload's default)")
@@ -873,6 +984,11 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
     try:
+        if args.workload == "prefill":
+            line = run_prefill(args, rank, world, dev)
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+            return
         if args.workload == "trace":  # one trace, on rank 0; the other ranks only join the exit
             if rank == 0:
                 for line in run_trace(args, dev):

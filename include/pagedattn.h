@@ -219,6 +219,32 @@ PA_API pa_status pa_decode_shared(const void *k_new, const void *v_new, const in
                                   const pa_share_plan_t *plan, void *out, void *workspace,
                                   size_t workspace_bytes, void *stream);
 
+/*
+ * Paged chunked-prefill attention: the decode step of "The Block Table Map"
+ * for every new token of a chunk, with a causal limit.  Sequence b holds
+ * context_lens[b] tokens in the cache (the chunk's own rows appended with
+ * pa_append_kv first); the last n_b = query_starts[b+1] - query_starts[b] of
+ * them are new, and new token i (position context_lens[b] - n_b + i) attends
+ * to the sequence's tokens 0 .. its own position:
+ *   out[query_starts[b] + i][h] = softmax_t(scale <q[...][h], K(b,t,g)>) . V(b,t,g), t <= position
+ * with g = h / (num_q_heads / num_kv_heads).  bf16, head_dim 128 only
+ * (PA_ERR_UNSUPPORTED otherwise); fp32 accumulation, out rounded once.
+ *   q             device [total_query_tokens][num_q_heads][128] bf16
+ *   query_starts  device [num_seqs + 1] int32, query_starts[0] = 0, ascending,
+ *                 query_starts[num_seqs] = total_query_tokens
+ *   block_tables, context_lens, max_context_len  as pa_decode
+ *   max_query_len host: an upper bound of every n_b (sizes the grid)
+ *   out           device [total_query_tokens][num_q_heads][128] bf16
+ * A sequence with n_b > context_lens[b] or a length past max_context_len
+ * sets PA_DEVERR_LEN and writes nothing; a used table entry outside the pool
+ * sets PA_DEVERR_TABLE (that sequence's rows are then undefined).
+ */
+PA_API pa_status pa_prefill(const void *q, const pa_cache_t *cache, const int32_t *block_tables,
+                            int32_t max_blocks_per_seq, const int32_t *context_lens,
+                            const int32_t *query_starts, int32_t num_seqs, int32_t num_q_heads,
+                            int32_t total_query_tokens, int32_t max_query_len,
+                            int32_t max_context_len, float scale, void *out, void *stream);
+
 /* Bytes of workspace pa_decode needs for these sizes (0 when no context is
  * longer than one partition). */
 PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,

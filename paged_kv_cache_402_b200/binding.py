@@ -70,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "pa_decode_shared": (st, [vp, vp, vp, vp, cp, vp, i32, vp, i32, i32, i32, f32,
                                   ctypes.POINTER(pa_share_plan_t), vp, vp, sz, vp]),
         "pa_share_plan": (st, [i32p, i32, i32p, i32, i32, i32, i32p, i32p, i32p, i32p]),
+        "pa_prefill": (st, [vp, cp, vp, i32, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp]),
         "pa_copy_blocks": (st, [vp, i32, cp, vp]),
         "pa_check_copy_pairs": (st, [i32p, i32, i32]),
         "pa_read_device_error": (st, [vp, i32p]),
@@ -354,6 +355,28 @@ def pa_decode_shared(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor
         block_tables.shape[1], _dev(context_lens, "context_lens", torch.int32), B, Hq, int(max_context_len),
         float(scale), plan.ref() if plan is not None else None, _dev(out, "out", cache.dtype), ws_ptr, ws_bytes,
         _stream_ptr(stream)), "pa_decode_shared")
+    return out
+
+
+def pa_prefill(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor, context_lens: torch.Tensor,
+               query_starts: torch.Tensor, max_context_len: int, scale: float, max_query_len: int | None = None,
+               out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Paged chunked-prefill attention: the last query_starts[b+1] -
+    query_starts[b] tokens of sequence b (already in the cache) attend
+    causally to the sequence; q and out are [total, Hq, 128] bf16."""
+    T, Hq, D = q.shape
+    B = context_lens.shape[0]
+    if D != cache.head_dim:
+        raise ValueError("head_dim mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or query_starts.shape != (B + 1,):
+        raise ValueError("block_tables must be [B, max_blocks] and query_starts [B + 1]")
+    if out is None:
+        out = torch.empty_like(q)
+    _check(_lib.pa_prefill(_dev(q, "q", cache.dtype), cache.ref(), _dev(block_tables, "block_tables", torch.int32),
+                           block_tables.shape[1], _dev(context_lens, "context_lens", torch.int32),
+                           _dev(query_starts, "query_starts", torch.int32), B, Hq, T,
+                           int(T if max_query_len is None else max_query_len), int(max_context_len), float(scale),
+                           _dev(out, "out", cache.dtype), _stream_ptr(stream)), "pa_prefill")
     return out
 
 

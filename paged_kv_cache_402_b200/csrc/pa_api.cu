@@ -16,6 +16,7 @@
 #include "pa_copy_kernels.cuh"
 #include "pa_decode_simt.cuh"
 #include "pa_decode_shared.cuh"
+#include "pa_prefill_tc.cuh"
 #include "pa_decode_tc.cuh"
 #include "pagedattn.h"
 
@@ -199,6 +200,21 @@ bool make_map_pool_4d(CUtensorMap *m, const void *base, uint64_t rows, uint32_t 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// q [total][Hq][128] bf16 seen as 3-D (128 columns, Hq heads, total tokens):
+// a box (64, G, Mq) is Mq tokens x the G query heads of one kv head, landing
+// as 128-byte rows ordered (token, head) with 128-byte swizzle.
+bool make_map_q3d(CUtensorMap *m, const void *base, uint64_t total, uint32_t Hq, uint32_t G, uint32_t Mq) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {128, Hq, total};
+  const cuuint64_t strides[2] = {128 * 2, (cuuint64_t)Hq * 128 * 2};
+  const cuuint32_t box[3] = {64, G, Mq};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool tc_eligible(const pa::DecodeParams &p, int dtype, int D) {
   if (dtype != PA_DTYPE_BF16 || D != 128) return false;
   if (p.G < 1 || p.G > 8 || (p.G & (p.G - 1))) return false;
@@ -304,6 +320,38 @@ pa_status launch_decode_shared(const pa::DecodeParams &p, const pa_share_plan_t 
     case 8: return launch_decode_shared_g<8>(p, plan, st);
     default: return PA_ERR_UNSUPPORTED;
   }
+}
+
+// Chunked prefill, in slices of at most kMaxSeqs sequences.
+template <int G>
+pa_status launch_prefill_g(const pa::DecodeParams &p, const int32_t *qstart, int64_t total_q,
+                           int32_t max_query_len, cudaStream_t st) {
+  constexpr int Mq = pa::PfLayout::kM / G;
+  CUtensorMap mk, mv, mq;
+  const uint64_t rows = (uint64_t)p.num_blocks * p.Hkv * p.bs;
+  if (!make_map_pool_4d(&mk, p.k, rows, (uint32_t)p.bs) ||
+      !make_map_pool_4d(&mv, p.v, rows, (uint32_t)p.bs) ||
+      !make_map_q3d(&mq, p.q, (uint64_t)total_q, (uint32_t)p.Hq, (uint32_t)G, (uint32_t)Mq))
+    return PA_ERR_CUDA;
+  auto kern = pa::prefill_tc<G>;
+  const int smem = pa::PfLayout::kBytes;
+  static std::atomic<int> smem_set[kMaxDev] = {};
+  if (!ensure_smem(kern, smem, smem_set)) return PA_ERR_CUDA;
+  const int sms = sm_count();
+  if (sms <= 0) return PA_ERR_CUDA;
+  for (int b0 = 0; b0 < p.B; b0 += pa::PfLayout::kMaxSeqs) {
+    pa::DecodeParams ps = p;
+    ps.B = p.B - b0 < pa::PfLayout::kMaxSeqs ? p.B - b0 : pa::PfLayout::kMaxSeqs;
+    ps.tables = p.tables + (size_t)b0 * p.max_blocks;
+    ps.lens = p.lens + b0;
+    ps.sched_slot = (int32_t)(g_sched_ticket.fetch_add(1) % pa::kSchedSlots);
+    pa::PrefillParams pp{qstart + b0, Mq};
+    const int64_t units_bound = (int64_t)ps.B * p.Hkv * ((max_query_len + Mq - 1) / Mq);
+    const int grid = units_bound < sms ? (int)(units_bound > 0 ? units_bound : 1) : sms;
+    const pa_status s = launch(kern, dim3(grid), dim3(pa::PfLayout::kThreads), (size_t)smem, st, mk, mv, mq, ps, pp);
+    if (s != PA_OK) return s;
+  }
+  return PA_OK;
 }
 
 pa_status launch_decode_tc(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
@@ -517,6 +565,53 @@ PA_API pa_status pa_append_decode(const void *k_new, const void *v_new, const in
              cache->num_blocks, max_context_len, (uint4 *)cache->k, (uint4 *)cache->v);
   if (s != PA_OK) return s;
   return launch_decode_any(p, cache, st);
+}
+
+PA_API pa_status pa_prefill(const void *q, const pa_cache_t *cache, const int32_t *block_tables,
+                            int32_t max_blocks_per_seq, const int32_t *context_lens,
+                            const int32_t *query_starts, int32_t num_seqs, int32_t num_q_heads,
+                            int32_t total_query_tokens, int32_t max_query_len,
+                            int32_t max_context_len, float scale, void *out, void *stream) {
+  pa_status s = check_cache(cache);
+  if (s != PA_OK) return s;
+  if (num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0 || max_blocks_per_seq < 0 ||
+      total_query_tokens < 0 || max_query_len < 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0 || total_query_tokens == 0) return PA_OK;
+  if (!q || !out || !block_tables || !context_lens || !query_starts || !aligned16(q) || !aligned16(out))
+    return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (num_q_heads % cache->num_kv_heads) return PA_ERR_INVALID_ARG;
+  const int32_t G = num_q_heads / cache->num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+  if (cache->dtype != PA_DTYPE_BF16 || cache->head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if ((int64_t)max_context_len > (int64_t)max_blocks_per_seq * cache->block_size) return PA_ERR_INVALID_ARG;
+  if (max_query_len > max_context_len) return PA_ERR_INVALID_ARG;
+  if ((int64_t)cache->num_blocks * cache->num_kv_heads * cache->block_size >= (int64_t)INT32_MAX)
+    return PA_ERR_INVALID_ARG;
+  pa::DecodeParams p{};
+  p.q = q;
+  p.k = cache->k;
+  p.v = cache->v;
+  p.out = out;
+  p.tables = block_tables;
+  p.lens = context_lens;
+  p.num_blocks = cache->num_blocks;
+  p.Hkv = cache->num_kv_heads;
+  p.bs = cache->block_size;
+  p.Hq = num_q_heads;
+  p.G = G;
+  p.max_blocks = max_blocks_per_seq;
+  p.B = num_seqs;
+  p.max_ctx = max_context_len;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t st = (cudaStream_t)stream;
+  switch (G) {
+    case 1: return launch_prefill_g<1>(p, query_starts, total_query_tokens, max_query_len, st);
+    case 2: return launch_prefill_g<2>(p, query_starts, total_query_tokens, max_query_len, st);
+    case 4: return launch_prefill_g<4>(p, query_starts, total_query_tokens, max_query_len, st);
+    default: return launch_prefill_g<8>(p, query_starts, total_query_tokens, max_query_len, st);
+  }
 }
 
 PA_API pa_status pa_decode_shared(const void *k_new, const void *v_new, const int32_t *cow_src,
