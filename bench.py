@@ -408,8 +408,9 @@ def run_ours(args, rank: int, world: int, dev):
 
     for s in range(args.warmup):
         step(s, stream)
-    if pa.pa_read_device_error() != 0:
-        raise RuntimeError("device error during warm-up")
+    bits = pa.pa_read_device_error()
+    if bits != 0:
+        raise RuntimeError(f"device error during warm-up (device error bits {bits:#x})")
 
     # The K timed steps (inputs precomputed, resident) are captured once into
     # a CUDA graph and replayed, so the host's launch rate does not bound the
@@ -464,8 +465,9 @@ def run_ours(args, rank: int, world: int, dev):
         torch.distributed.barrier()
     ms = t_start.elapsed_time(t_end)
     dec_ms = [a.elapsed_time(b) for a, b in dec_events] if per_step_events else [ms / args.steps]
-    if pa.pa_read_device_error() != 0:
-        raise RuntimeError("device error during the timed steps")
+    bits = pa.pa_read_device_error()
+    if bits != 0:
+        raise RuntimeError(f"device error during the timed steps (device error bits {bits:#x})")
     clocks = clk.summary()
 
     # end to end through the public API with pinned host buffers
@@ -672,8 +674,9 @@ def run_prefill(args, rank: int, world: int, dev):
     for s_ in range(args.warmup):
         step(s_, stream)
     torch.cuda.synchronize()
-    if pa.pa_read_device_error() != 0:
-        raise RuntimeError("device error during warm-up")
+    bits = pa.pa_read_device_error()
+    if bits != 0:
+        raise RuntimeError(f"device error during warm-up (device error bits {bits:#x})")
     graph = torch.cuda.CUDAGraph()
     flops = tokens = 0
     with torch.cuda.graph(graph):
@@ -697,8 +700,9 @@ def run_prefill(args, rank: int, world: int, dev):
     if world > 1:
         torch.distributed.barrier()
     ms = t0.elapsed_time(t1)
-    if pa.pa_read_device_error() != 0:
-        raise RuntimeError("device error during the timed steps")
+    bits = pa.pa_read_device_error()
+    if bits != 0:
+        raise RuntimeError(f"device error during the timed steps (device error bits {bits:#x})")
     ms_all, fl_all, tok_all, _ = aggregate_ranks(world, ms, flops / 1e12, float(tokens), 1.0, 0.0, dev)
     peak, kind = measured_tensor_peak()
     tflops = fl_all / (ms_all / 1e3)
@@ -822,8 +826,9 @@ def run_trace(args, dev):
             frag.append(st["fragmentation"])
             h2d += sum(x.numel() * x.element_size() for x in h if x is not None)
             d2h += res.numel() * res.element_size()
-        if pa.pa_read_device_error() != 0:
-            raise RuntimeError("device error in the trace")
+        bits = pa.pa_read_device_error()
+        if bits != 0:
+            raise RuntimeError(f"device error in the trace (device error bits {bits:#x})")
         peak, peak_kind = measured_peaks()
         steps = args.trace_steps
         line = {

@@ -18,13 +18,16 @@
 //    4-D box per (block, kv head) as the decode kernel does; warp 1 issues
 //        S[128 q x 128 keys] = Q . K^T              (M = N = 128, K = 128 d)
 //        O[128 q x 128 d]   += P . V               (M = N = 128, K = 128 keys)
-//    with S double-buffered and O double-buffered by unit in tensor memory.
+//    with S double-buffered and O double-buffered by unit in tensor memory;
+//    the PV MMA takes P from tensor memory (A operand in TMEM).  Q tiles are
+//    double-buffered in shared memory so the next unit's loads overlap.
 //  * Warps 2..5: thread r owns query row r.  Per chunk it reads its S row,
-//    masks keys past its position, and keeps a per-row reference max that
-//    moves only when a score passes it by 2^8; then it rescales its own O row
-//    in tensor memory (warp-wide when any lane of the warp needs it).  It
-//    writes its row of P in bf16 into one shared-memory tile (128-byte
-//    swizzle, K-major over keys) for the PV MMA.  The sums and maxima are per
+//    masks keys past its position (per 32-key group), and keeps a per-row
+//    reference max that moves only when a score passes it by 2^8; then it
+//    rescales its own O row in tensor memory (warp-wide when any lane of the
+//    warp needs it).  It writes its row of P in bf16 over the first half of
+//    its own S columns (each 32-column group of S is read before the 16
+//    columns of P that cover it are written).  The sums and maxima are per
 //    row, so no barrier across the warpgroup is needed per chunk.  At the
 //    end of a unit (overlapped with the next unit) it reads its O row,
 //    divides by its sum and stores the row.
@@ -37,6 +40,14 @@
 
 namespace pa {
 
+// 2^x by the MUFU approximation (flushes denormal results to zero): the
+// weights only feed a bf16 operand and fp32 sums.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 struct PfLayout {
   static constexpr int kM = 128;           // query rows per tile
   static constexpr int kChunk = 128;       // keys per chunk
@@ -47,10 +58,10 @@ struct PfLayout {
   static constexpr int kMaxSeqs = 1024;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kStages * kTile;
-  static constexpr int kOffQ = kOffV + kStages * kTile;
-  static constexpr int kOffP = kOffQ + 2 * kHalf;
-  static constexpr int kOffBar = kOffP + 2 * kHalf;
-  static constexpr int kNumBars = 20;
+  static constexpr int kOffQ = kOffV + kStages * kTile;  // two Q tiles of 2 column halves
+  static constexpr int kQ = 2 * kHalf;
+  static constexpr int kOffBar = kOffQ + 2 * kQ;
+  static constexpr int kNumBars = 21;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   // unit slot: [b, g, first query row, tokens in the tile, first position, chunks, length]
   static constexpr int kUnitInts = 8;
@@ -79,8 +90,8 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
   uint64_t *kfull = bars, *kempty = bars + 2, *vfull = bars + 4, *vempty = bars + 6;
-  uint64_t *qfull = bars + 8, *qempty = bars + 9, *sfull = bars + 10, *pfull = bars + 12;
-  uint64_t *pfree = bars + 13, *pvdone = bars + 14, *ofree = bars + 16, *drain = bars + 18;
+  uint64_t *qfull = bars + 8, *qempty = bars + 10, *sfull = bars + 12, *pfull = bars + 14;
+  uint64_t *pvdone = bars + 16, *ofree = bars + 18, *drain = bars + 20;
   int32_t *prefix = reinterpret_cast<int32_t *>(smem + L::kOffPrefix);
   int32_t *scan = reinterpret_cast<int32_t *>(smem + L::kOffScan);
   int32_t *unit_slots = reinterpret_cast<int32_t *>(smem + L::kOffUnit);
@@ -94,15 +105,14 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
       mbar_init(&vfull[i], 1);
       mbar_init(&vempty[i], 1);
     }
-    mbar_init(qfull, 1);
-    mbar_init(qempty, 2);  // the MMA warp's commit after the unit's last QK + the softmax reading the unit
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&qfull[i], 1);
+      mbar_init(&qempty[i], 2);  // the MMA warp's commit after the unit's last QK + the softmax reading the unit
       mbar_init(&sfull[i], 1);
+      mbar_init(&pfull[i], 128);  // P of the chunk written over its S
       mbar_init(&pvdone[i], 1);
       mbar_init(&ofree[i], 128);
     }
-    mbar_init(pfull, 128);
-    mbar_init(pfree, 1);
     mbar_init(drain, 1);
     fence_barrier_init();
   }
@@ -199,9 +209,10 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
         return (lane < bpc && j * bs < ctx) ? tr[j] : -1;
       };
       int32_t e_next = entry(0);
-      if (!__all_sync(0xffffffffu, mbar_wait(qempty, (qi & 1) ^ 1))) { ok = false; break; }
+      const int qs = qi & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((qi >> 1) & 1) ^ 1))) { ok = false; break; }
       if (lane == 0) {
-        int32_t *us = unit_slots + (qi & 1) * L::kUnitInts;
+        int32_t *us = unit_slots + qs * L::kUnitInts;
         us[0] = b;
         us[1] = g;
         us[2] = q0 + tok0;
@@ -209,10 +220,10 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
         us[4] = pos0;
         us[5] = nchunks;
         us[6] = ctx;
-        mbar_arrive_expect_tx(qfull, 2 * L::kHalf);
-        uint8_t *qdst = smem + L::kOffQ;
-        tc::tma_load_3d(qdst, &tmap_q, 0, g * G, q0 + tok0, qfull, pol_q);
-        tc::tma_load_3d(qdst + L::kHalf, &tmap_q, 64, g * G, q0 + tok0, qfull, pol_q);
+        mbar_arrive_expect_tx(&qfull[qs], 2 * L::kHalf);
+        uint8_t *qdst = smem + L::kOffQ + qs * L::kQ;
+        tc::tma_load_3d(qdst, &tmap_q, 0, g * G, q0 + tok0, &qfull[qs], pol_q);
+        tc::tma_load_3d(qdst + L::kHalf, &tmap_q, 64, g * G, q0 + tok0, &qfull[qs], pol_q);
       }
       ++qi;
       for (int ci = 0; ci < nchunks; ++ci, ++c) {
@@ -242,12 +253,13 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
       u = __shfl_sync(0xffffffffu, raw, 0);
     }
     if (ok) {  // an empty unit stops the consumers
-      if (!__all_sync(0xffffffffu, mbar_wait(qempty, (qi & 1) ^ 1))) {
+      const int qs = qi & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((qi >> 1) & 1) ^ 1))) {
         ok = false;
       } else {
-        if (lane == 0) unit_slots[(qi & 1) * L::kUnitInts + 5] = 0;
+        if (lane == 0) unit_slots[qs * L::kUnitInts + 5] = 0;
         __syncwarp();
-        if (lane == 0) mbar_arrive(qfull);
+        if (lane == 0) mbar_arrive(&qfull[qs]);
       }
     }
     if (!ok && lane == 0) {
@@ -256,7 +268,7 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
         mbar_wait(&kfull[k % L::kStages], (k / L::kStages) & 1, 100000000ull);
         mbar_wait(&vfull[k % L::kStages], (k / L::kStages) & 1, 100000000ull);
       }
-      if (qi > 0) mbar_wait(qfull, (qi - 1) & 1, 100000000ull);
+      for (int k = (qi > 2 ? qi - 2 : 0); k < qi; ++k) mbar_wait(&qfull[k & 1], (k >> 1) & 1, 100000000ull);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -265,7 +277,7 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
     constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(128, 128, false, false);
     constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(128, 128, false, true);
     const uint32_t kbase0 = smem_u32(smem + L::kOffK), vbase0 = smem_u32(smem + L::kOffV);
-    const uint32_t qb = smem_u32(smem + L::kOffQ), pb = smem_u32(smem + L::kOffP);
+    const uint32_t qbase0 = smem_u32(smem + L::kOffQ);
     bool ok = true;
     auto warp_wait = [&](uint64_t *bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity));
@@ -276,23 +288,22 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
     };
     auto issue_pv = [&](const PvJob &j) -> bool {
       const int c = j.c;
-      if (!warp_wait(pfull, c & 1)) return false;
+      if (!warp_wait(&pfull[c & 1], (c >> 1) & 1)) return false;
       if (!warp_wait(&vfull[c % L::kStages], (c / L::kStages) & 1)) return false;
       if (j.first && !warp_wait(&ofree[j.u & 1], ((j.u >> 1) & 1) ^ 1)) return false;
       if (lane == 0) {
         tc::fence_after_sync();
         const uint32_t vb = vbase0 + (c % L::kStages) * L::kTile;
         const uint32_t d = tmem + 256 + (j.u & 1) * 128;
+        const uint32_t pa = tmem + (c & 1) * 128;  // P over the chunk's S columns, 2 keys per column
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          // P: K-major over keys (key half kk/4 at +kHalf, 16 keys = 32 B);
-          // V: N = head dim contiguous (MN-major), 16 keys = two 8-key groups
-          const uint64_t a = tc::smem_desc_sw128(pb + (kk >> 2) * L::kHalf + (kk & 3) * 32, 16, 1024);
+          // P: 16 keys = 8 columns of tensor memory; V: N = head dim
+          // contiguous (MN-major), 16 keys = two 8-key groups
           const uint64_t bdesc = tc::smem_desc_sw128(vb + kk * 2 * L::kGroup, 1024, L::kGroup);
-          tc::mma_bf16(d, a, bdesc, idesc_pv, (kk > 0 || !j.first) ? 1u : 0u);
+          tc::mma_bf16_ts(d, pa + kk * 8, bdesc, idesc_pv, (kk > 0 || !j.first) ? 1u : 0u);
         }
         tc::mma_commit(&pvdone[c & 1]);
-        tc::mma_commit(pfree);
         tc::mma_commit(&vempty[c % L::kStages]);
       }
       __syncwarp();
@@ -301,9 +312,11 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
     int c = 0, qi = 0;
     PvJob pending{-1, 0, false};
     while (ok) {
-      if (!warp_wait(qfull, qi & 1)) { ok = false; break; }
-      const int nchunks = unit_slots[(qi & 1) * L::kUnitInts + 5];
+      const int qs = qi & 1;
+      if (!warp_wait(&qfull[qs], (qi >> 1) & 1)) { ok = false; break; }
+      const int nchunks = unit_slots[qs * L::kUnitInts + 5];
       if (nchunks == 0) break;
+      const uint32_t qb = qbase0 + qs * L::kQ;
       for (int ci = 0; ci < nchunks; ++ci, ++c) {
         const int slot = c % L::kStages;
         if (!warp_wait(&kfull[slot], (c / L::kStages) & 1)) { ok = false; break; }
@@ -321,7 +334,7 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
           }
           tc::mma_commit(&sfull[c & 1]);
           tc::mma_commit(&kempty[slot]);
-          if (ci == nchunks - 1) tc::mma_commit(qempty);
+          if (ci == nchunks - 1) tc::mma_commit(&qempty[qs]);
         }
         __syncwarp();
         if (pending.c >= 0 && !issue_pv(pending)) { ok = false; break; }
@@ -380,16 +393,17 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
 
     int c = 0, qi = 0;
     for (;; ++qi) {
-      warp_wait(qfull, qi & 1);
+      const int qs = qi & 1;
+      warp_wait(&qfull[qs], (qi >> 1) & 1);
       if (bad) break;
-      const int32_t *us = unit_slots + (qi & 1) * L::kUnitInts;
+      const int32_t *us = unit_slots + qs * L::kUnitInts;
       const int nchunks = us[5];
       const int ub = us[0], ug = us[1], urow0 = us[2], untok = us[3], upos0 = us[4], uctx = us[6];
       // keys of the sequence's last, partly filled block past its end
       const int tail_end = ((uctx + p.bs - 1) / p.bs) * p.bs;
       // the producer may reuse the Q tile once the QKs are done and this
       // unit's slot has been read: it never runs two units ahead of here
-      if (r == 0 && nchunks > 0) mbar_arrive(qempty);
+      if (r == 0 && nchunks > 0) mbar_arrive(&qempty[qs]);
       const int pos = upos0 + r / G;  // this row's position (rows past the tile's tokens: masked out)
       const bool row_live = r / G < untok;
       m = -INFINITY;
@@ -399,15 +413,22 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
         if (!bad) tc::fence_after_sync();
         const uint32_t srow = trow + (c & 1) * 128;
         const int key0 = ci * L::kChunk;
-        // pass 1: the chunk's row max over the keys this row sees
+        // keys of this chunk the row sees: the first nvis
+        const int nvis = row_live ? max(0, min(L::kChunk, pos - key0 + 1)) : 0;
+        // pass 1: the chunk's row max over those keys (base-2 units)
         float cmax = -INFINITY;
         float s[32];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           if (!bad) tc::tmem_ld32(srow + 32 * k, s);
+          if (32 * k + 32 <= nvis) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (row_live && key0 + 32 * k + e <= pos) cmax = fmaxf(cmax, s[e] * p.scale_log2);
+            for (int e = 0; e < 32; ++e) cmax = fmaxf(cmax, s[e] * p.scale_log2);
+          } else if (32 * k < nvis) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (32 * k + e < nvis) cmax = fmaxf(cmax, s[e] * p.scale_log2);
+          }
         }
         // the reference moves only when a score passes it by 2^8
         const bool need = cmax > m + kLazyRescale;
@@ -435,33 +456,32 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
         }
         l *= alpha;
         m = mnew;
-        // pass 2: P = 2^(s - m) in bf16 into the P tile, once PV(c-1) has read it
-        warp_wait(pfree, (c & 1) ^ 1);
-        uint8_t *prow = smem + L::kOffP + r * 128;
+        // pass 2: P = 2^(s - m) in bf16, two keys per column, written over
+        // columns 16k .. 16k+15 once group k of S (columns 32k ..) is read
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           if (!bad) tc::tmem_ld32(srow + 32 * k, s);
+          float pv[32];
+          if (32 * k + 32 <= nvis) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) pv[e] = ex2_approx(fmaf(s[e], p.scale_log2, -m));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              pv[e] = 32 * k + e < nvis ? ex2_approx(fmaf(s[e], p.scale_log2, -m)) : 0.f;
+          }
           uint32_t w[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const int t0 = key0 + 32 * k + 2 * e;
-            const float p0 = (row_live && t0 <= pos) ? exp2f(s[2 * e] * p.scale_log2 - m) : 0.f;
-            const float p1 = (row_live && t0 + 1 <= pos) ? exp2f(s[2 * e + 1] * p.scale_log2 - m) : 0.f;
-            l += p0 + p1;
-            const __nv_bfloat162 two = __floats2bfloat162_rn(p0, p1);
+            l += pv[2 * e] + pv[2 * e + 1];
+            const __nv_bfloat162 two = __floats2bfloat162_rn(pv[2 * e], pv[2 * e + 1]);
             w[e] = *reinterpret_cast<const uint32_t *>(&two);
           }
-          // keys 32k .. 32k+31 = 16-byte pieces 4k .. 4k+3 of the row; pieces
-          // 0..7 in key half 0, 8..15 in key half 1, piece j at j ^ (r % 8)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int piece = 4 * k + j, half = piece >> 3, pos16 = (piece & 7) ^ (r & 7);
-            *reinterpret_cast<uint4 *>(prow + half * L::kHalf + (pos16 << 4)) =
-                make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-          }
+          if (!bad) tc::tmem_st16_nowait(srow + 16 * k, w);
         }
-        // those hold whatever the pool has there: zero their V rows (thread r
-        // takes row r of the chunk) before the PV MMA reads them
+        if (!bad) tc::tmem_wait_st();
+        // V rows past the sequence's end in its last block hold whatever the
+        // pool has there: zero them (thread r takes row r of the chunk)
         const bool tail_row = key0 + r >= uctx && key0 + r < tail_end;
         if (__any_sync(0xffffffffu, tail_row)) {
           warp_wait(&vfull[c % L::kStages], (c / L::kStages) & 1);
@@ -474,10 +494,10 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
               vr[1024 / 16 + e] = make_uint4(0, 0, 0, 0);
             }
           }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
         tc::fence_before_sync();
-        mbar_arrive(pfull);
+        mbar_arrive(&pfull[c & 1]);
         // the previous unit's rows, while this chunk's PV runs
         if (ci == 0 && pend) {
           epilogue();
