@@ -676,24 +676,30 @@ def run_prefill(args, rank: int, world: int, dev):
     torch.cuda.synchronize()
     bits = pa.pa_read_device_error()
     if bits != 0:
-        raise RuntimeError(f"device error during warm-up (device error bits {bits:#x})")
-    graph = torch.cuda.CUDAGraph()
-    flops = tokens = 0
-    with torch.cuda.graph(graph):
-        cap = torch.cuda.current_stream()
-        for i in range(args.steps):
-            it = step(args.warmup + i, cap)
-            flops += it["flops"]
-            tokens += it["tokens"]
-    graph.replay()
-    torch.cuda.synchronize()
+        raise RuntimeError(f"device error during warm-up (device error bits {bits:#x}, "
+                           f"first wait given up: {pa.pa_read_wait_timeout()})")
+    flops = sum(insts[(args.warmup + i) % R]["flops"] for i in range(args.steps))
+    tokens = sum(insts[(args.warmup + i) % R]["tokens"] for i in range(args.steps))
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            cap = torch.cuda.current_stream()
+            for i in range(args.steps):
+                step(args.warmup + i, cap)
+        graph.replay()
+        torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     with ClockSampler(dev) as clk:
         t0.record(stream)
-        graph.replay()
+        if graph is not None:
+            graph.replay()
+        else:
+            for i in range(args.steps):
+                step(args.warmup + i, stream)
         t1.record(stream)
         torch.cuda.synchronize()
     del graph
@@ -702,7 +708,8 @@ def run_prefill(args, rank: int, world: int, dev):
     ms = t0.elapsed_time(t1)
     bits = pa.pa_read_device_error()
     if bits != 0:
-        raise RuntimeError(f"device error during the timed steps (device error bits {bits:#x})")
+        raise RuntimeError(f"device error during the timed steps (device error bits {bits:#x}, "
+                           f"first wait given up: {pa.pa_read_wait_timeout()})")
     ms_all, fl_all, tok_all, _ = aggregate_ranks(world, ms, flops / 1e12, float(tokens), 1.0, 0.0, dev)
     peak, kind = measured_tensor_peak()
     tflops = fl_all / (ms_all / 1e3)
@@ -716,7 +723,8 @@ def run_prefill(args, rank: int, world: int, dev):
                                "[1, 4096]), 32 q / 8 kv heads, head_dim 128, 16-token blocks; step = append of "
                                "the prompts' K/V + causal attention of every prompt token",
                    "global_batch": B * world, "l2": f"{R} rotating batch instances",
-                   "timing": "CUDA graph replay of the K steps", "parallelism": f"replicas x{world}"},
+                   "timing": "eager launches" if args.no_graph else "CUDA graph replay of the K steps",
+                   "parallelism": f"replicas x{world}"},
         "tokens_per_s": round(tok_all / (ms_all / 1e3), 1),
         "roofline": {"bound": "tensor", "kernel": "pa_append_kv + pa_prefill", "achieved": round(tflops, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),

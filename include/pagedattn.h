@@ -307,6 +307,12 @@ PA_API pa_status pa_check_copy_pairs(const int32_t *src_dst_pairs_host, int32_t 
  * *bits (PA_DEVERR_*) and clears it. */
 PA_API pa_status pa_read_device_error(void *stream, int32_t *bits);
 
+/* Synchronises `stream` and returns (and clears) where the first wait that
+ * gave up since the last call was (the cause of PA_DEVERR_TIMEOUT):
+ * info[0] = 1 if any, info[1] = the shared-memory address of its mbarrier,
+ * info[2] = its phase parity | block index << 1, info[3] = thread index. */
+PA_API pa_status pa_read_wait_timeout(void *stream, uint32_t info[4]);
+
 /* Static text for a status code. */
 PA_API const char *pa_status_string(pa_status s);
 

@@ -74,6 +74,7 @@ def _load() -> ctypes.CDLL:
         "pa_copy_blocks": (st, [vp, i32, cp, vp]),
         "pa_check_copy_pairs": (st, [i32p, i32, i32]),
         "pa_read_device_error": (st, [vp, i32p]),
+        "pa_read_wait_timeout": (st, [vp, ctypes.POINTER(ctypes.c_uint32)]),
         "pa_status_string": (ctypes.c_char_p, [st]),
         "pa_version": (ctypes.c_char_p, []),
         "pa_alloc_create": (st, [i32, i32, i32p, ctypes.POINTER(vp)]),
@@ -413,6 +414,14 @@ def pa_copy_blocks(src_dst_pairs: torch.Tensor, cache: KVCache, stream=None) -> 
 def pa_check_copy_pairs(pairs, num_blocks: int) -> bool:
     a = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
     return _lib.pa_check_copy_pairs(_i32p(a), a.shape[0], int(num_blocks)) == PA_OK
+
+
+def pa_read_wait_timeout(stream=None) -> list:
+    """Synchronises the stream; returns (and clears) [taken, mbarrier shared
+    address, parity | block << 1, thread] of the first wait that gave up."""
+    info = (ctypes.c_uint32 * 4)()
+    _check(_lib.pa_read_wait_timeout(_stream_ptr(stream), info), "pa_read_wait_timeout")
+    return list(info)
 
 
 def pa_read_device_error(stream=None) -> int:

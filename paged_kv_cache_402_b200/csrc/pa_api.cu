@@ -721,6 +721,15 @@ PA_API pa_status pa_decode_static_workspace(const void *q, const pa_cache_t *cac
                    stream);
 }
 
+PA_API pa_status pa_read_wait_timeout(void *stream, uint32_t info[4]) {
+  if (!info) return PA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return PA_ERR_CUDA;
+  uint32_t zero[4] = {0, 0, 0, 0};
+  if (cudaMemcpyFromSymbol(info, pa::g_wait_timeout, sizeof zero) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(pa::g_wait_timeout, zero, sizeof zero) != cudaSuccess) return PA_ERR_CUDA;
+  return PA_OK;
+}
+
 PA_API pa_status pa_read_device_error(void *stream, int32_t *bits) {
   if (!bits) return PA_ERR_INVALID_ARG;
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return PA_ERR_CUDA;

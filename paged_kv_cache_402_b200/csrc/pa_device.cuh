@@ -16,6 +16,11 @@ __device__ int32_t g_error;
 
 __device__ __forceinline__ void raise_error(int32_t bits) { atomicOr(&g_error, bits); }
 
+// Where the first wait that gave up was: [taken, shared-memory address of
+// its mbarrier, parity | block index << 1, thread index]; read and cleared
+// by pa_read_wait_timeout.
+__device__ uint32_t g_wait_timeout[4];
+
 // Programmatic dependent launch: every kernel of the library is launched so
 // that it may be scheduled before the kernel ahead of it in the stream has
 // finished; it then waits here, before touching any memory, until that
@@ -88,6 +93,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     if (i == 0) {
       start = global_ns();
     } else if ((i & 63) == 0 && global_ns() - start > limit_ns) {
+      if (atomicCAS(&g_wait_timeout[0], 0u, 1u) == 0u) {
+        g_wait_timeout[1] = addr;
+        g_wait_timeout[2] = parity | (blockIdx.x << 1);
+        g_wait_timeout[3] = threadIdx.x;
+      }
       return false;
     }
   }

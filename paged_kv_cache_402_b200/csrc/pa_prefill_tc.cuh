@@ -107,7 +107,11 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&qfull[i], 1);
-      mbar_init(&qempty[i], 2);  // the MMA warp's commit after the unit's last QK + the softmax reading the unit
+      // the MMA warp's commit after the unit's last QK + each of the four
+      // softmax warps once it has read the unit (they run without a common
+      // barrier, so every one must have passed its wait on qfull before the
+      // slot and its barrier phase can be reused)
+      mbar_init(&qempty[i], 1 + 4);
       mbar_init(&sfull[i], 1);
       mbar_init(&pfull[i], 128);  // P of the chunk written over its S
       mbar_init(&pvdone[i], 1);
@@ -401,9 +405,10 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
       const int ub = us[0], ug = us[1], urow0 = us[2], untok = us[3], upos0 = us[4], uctx = us[6];
       // keys of the sequence's last, partly filled block past its end
       const int tail_end = ((uctx + p.bs - 1) / p.bs) * p.bs;
-      // the producer may reuse the Q tile once the QKs are done and this
-      // unit's slot has been read: it never runs two units ahead of here
-      if (r == 0 && nchunks > 0) mbar_arrive(&qempty[qs]);
+      // the producer may reuse the Q tile once the QKs are done and every
+      // softmax warp has read this unit's slot: it never runs two units
+      // ahead of the slowest warp
+      if (lane == 0 && nchunks > 0) mbar_arrive(&qempty[qs]);
       const int pos = upos0 + r / G;  // this row's position (rows past the tile's tokens: masked out)
       const bool row_live = r / G < untok;
       m = -INFINITY;
@@ -415,71 +420,108 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
         const int key0 = ci * L::kChunk;
         // keys of this chunk the row sees: the first nvis
         const int nvis = row_live ? max(0, min(L::kChunk, pos - key0 + 1)) : 0;
-        // pass 1: the chunk's row max over those keys (base-2 units)
-        float cmax = -INFINITY;
+        // One pass against the current reference: the weights stay in
+        // registers until every row of the warp is known to stay within 2^8
+        // of its reference; otherwise (a row's first chunk, or a score past
+        // the bound) the chunk takes two passes: the row max, a rescale of
+        // the rows' O, then the weights.  Either way each row's weights are
+        // 2^(s - m) against its reference m when they are written.
         float s[32];
+        uint32_t w[64];
+        float lsum = 0.f;
+        bool over = m == -INFINITY && nvis > 0;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           if (!bad) tc::tmem_ld32(srow + 32 * k, s);
-          if (32 * k + 32 <= nvis) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) cmax = fmaxf(cmax, s[e] * p.scale_log2);
-          } else if (32 * k < nvis) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (32 * k + e < nvis) cmax = fmaxf(cmax, s[e] * p.scale_log2);
+          for (int e = 0; e < 16; ++e) {
+            const float x0 = fmaf(s[2 * e], p.scale_log2, -m), x1 = fmaf(s[2 * e + 1], p.scale_log2, -m);
+            const bool v0 = 32 * k + 2 * e < nvis, v1 = 32 * k + 2 * e + 1 < nvis;
+            over |= (v0 && x0 > kLazyRescale) || (v1 && x1 > kLazyRescale);
+            const float p0 = v0 ? ex2_approx(x0) : 0.f, p1 = v1 ? ex2_approx(x1) : 0.f;
+            lsum += p0 + p1;
+            const __nv_bfloat162 two = __floats2bfloat162_rn(p0, p1);
+            w[16 * k + e] = *reinterpret_cast<const uint32_t *>(&two);
           }
         }
-        // the reference moves only when a score passes it by 2^8
-        const bool need = cmax > m + kLazyRescale;
-        const float mnew = need ? cmax : m;
-        const float alpha = need ? exp2f(m - mnew) : 1.f;  // 0 when m was -inf
-        if (__any_sync(0xffffffffu, need) && ci > 0) {
-          // rescale this warp's O rows once PV(c-1) has landed, before PV(c) adds
-          warp_wait(&pvdone[(c - 1) & 1], ((c - 1) >> 1) & 1);
+        if (!__any_sync(0xffffffffu, over)) {
           if (!bad) {
-            const uint32_t orow = trow + 256 + (qi & 1) * 128;
-            tc::fence_after_sync();
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              float o[32];
-              tc::tmem_ld32(orow + 32 * k, o);
+              uint32_t w16[16];
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                float o8[8];
+              for (int e = 0; e < 16; ++e) w16[e] = w[16 * k + e];
+              tc::tmem_st16_nowait(srow + 16 * k, w16);
+            }
+            tc::tmem_wait_st();
+          }
+          l += lsum;
+        } else {
+          // pass 1: the chunk's row max over those keys (base-2 units)
+          float cmax = -INFINITY;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) o8[e] = o[8 * j + e] * alpha;
-                tc::tmem_st8(orow + 32 * k + 8 * j, o8);
+          for (int k = 0; k < 4; ++k) {
+            if (!bad) tc::tmem_ld32(srow + 32 * k, s);
+            if (32 * k + 32 <= nvis) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) cmax = fmaxf(cmax, s[e] * p.scale_log2);
+            } else if (32 * k < nvis) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (32 * k + e < nvis) cmax = fmaxf(cmax, s[e] * p.scale_log2);
+            }
+          }
+          // the reference moves only when a score passes it by 2^8
+          const bool need = cmax > m + kLazyRescale;
+          const float mnew = need ? cmax : m;
+          const float alpha = need ? exp2f(m - mnew) : 1.f;  // 0 when m was -inf
+          if (__any_sync(0xffffffffu, need) && ci > 0) {
+            // rescale this warp's O rows once PV(c-1) has landed, before PV(c) adds
+            warp_wait(&pvdone[(c - 1) & 1], ((c - 1) >> 1) & 1);
+            if (!bad) {
+              const uint32_t orow = trow + 256 + (qi & 1) * 128;
+              tc::fence_after_sync();
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                float o[32];
+                tc::tmem_ld32(orow + 32 * k, o);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  float o8[8];
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) o8[e] = o[8 * j + e] * alpha;
+                  tc::tmem_st8(orow + 32 * k + 8 * j, o8);
+                }
               }
             }
           }
-        }
-        l *= alpha;
-        m = mnew;
-        // pass 2: P = 2^(s - m) in bf16, two keys per column, written over
-        // columns 16k .. 16k+15 once group k of S (columns 32k ..) is read
+          l *= alpha;
+          m = mnew;
+          // pass 2: P = 2^(s - m) in bf16, two keys per column, written over
+          // columns 16k .. 16k+15 once group k of S (columns 32k ..) is read
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if (!bad) tc::tmem_ld32(srow + 32 * k, s);
-          float pv[32];
-          if (32 * k + 32 <= nvis) {
+          for (int k = 0; k < 4; ++k) {
+            if (!bad) tc::tmem_ld32(srow + 32 * k, s);
+            float pv[32];
+            if (32 * k + 32 <= nvis) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) pv[e] = ex2_approx(fmaf(s[e], p.scale_log2, -m));
-          } else {
+              for (int e = 0; e < 32; ++e) pv[e] = ex2_approx(fmaf(s[e], p.scale_log2, -m));
+            } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              pv[e] = 32 * k + e < nvis ? ex2_approx(fmaf(s[e], p.scale_log2, -m)) : 0.f;
+              for (int e = 0; e < 32; ++e)
+                pv[e] = 32 * k + e < nvis ? ex2_approx(fmaf(s[e], p.scale_log2, -m)) : 0.f;
+            }
+            uint32_t w16[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              l += pv[2 * e] + pv[2 * e + 1];
+              const __nv_bfloat162 two = __floats2bfloat162_rn(pv[2 * e], pv[2 * e + 1]);
+              w16[e] = *reinterpret_cast<const uint32_t *>(&two);
+            }
+            if (!bad) tc::tmem_st16_nowait(srow + 16 * k, w16);
           }
-          uint32_t w[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            l += pv[2 * e] + pv[2 * e + 1];
-            const __nv_bfloat162 two = __floats2bfloat162_rn(pv[2 * e], pv[2 * e + 1]);
-            w[e] = *reinterpret_cast<const uint32_t *>(&two);
-          }
-          if (!bad) tc::tmem_st16_nowait(srow + 16 * k, w);
+          if (!bad) tc::tmem_wait_st();
         }
-        if (!bad) tc::tmem_wait_st();
         // V rows past the sequence's end in its last block hold whatever the
         // pool has there: zero them (thread r takes row r of the chunk)
         const bool tail_row = key0 + r >= uctx && key0 + r < tail_end;

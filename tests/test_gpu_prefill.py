@@ -121,3 +121,27 @@ def test_prefill_bad_chunk_length_is_reported(cuda_device):
     hv, _ = oracle.host_array(cache.v.cpu())
     ref = oracle.prefill(q[:20], hk, hv, tables[:1], lens[:1], starts[:2], 0.1)
     assert_attn_close(out[:20], ref, torch.bfloat16)
+
+
+def test_prefill_many_short_units_no_timeout(cuda_device):
+    """Hundreds of one-chunk units per CTA, repeated: every softmax warp must
+    have read a unit before its Q slot is reused (a lagging warp once saw the
+    slot's barrier two phases ahead and gave up waiting).  No error bit, and
+    the output still matches the oracle."""
+    Hq, Hkv, bs = 32, 8, 16
+    r = synth.rng(97)
+    new = r.integers(1, 64, size=400)
+    cached = r.integers(0, 40, size=400)
+    cache, q, tables, lens, starts = _chunk_case(98, cached, new, Hq, Hkv, bs, cuda_device)
+    scale = 1 / math.sqrt(128)
+    args = (q.to(cuda_device), cache, torch.from_numpy(tables).to(cuda_device), torch.from_numpy(lens).to(cuda_device),
+            torch.from_numpy(starts).to(cuda_device), int(lens.max()), scale)
+    out = None
+    for _ in range(30):
+        out = pa.pa_prefill(*args, max_query_len=int(new.max()))
+    assert pa.pa_read_device_error() == 0
+    rows = [(int(j), h) for j in r.integers(0, int(starts[-1]), size=40) for h in (0, 17)]
+    hk, _ = oracle.host_array(cache.k.cpu())
+    hv, _ = oracle.host_array(cache.v.cpu())
+    ref = oracle.prefill(q, hk, hv, tables, lens, starts, scale, rows=rows)
+    assert_attn_close(torch.stack([out[j, h] for j, h in rows]), ref, torch.bfloat16)
