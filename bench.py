@@ -734,6 +734,28 @@ def run_prefill(args, rank: int, world: int, dev):
     }
 
 
+def choose_block_size(lines, frag_budget: float):
+    """The block-size choice from a trace sweep: the pages' trade-off is that
+    smaller blocks waste less of the last block of every sequence, larger
+    ones cost less bookkeeping and fewer, larger copies per key range
+    ("pagedattention" glossary entry, paragraph 6).  Rule: the fastest block
+    size (decode tokens per second of wall time) among those whose mean
+    fragmentation stays within the budget; the smallest block size if none
+    does."""
+    ok = [d for d in lines if d["fragmentation_mean"] is not None and d["fragmentation_mean"] <= frag_budget]
+    pick = (max(ok, key=lambda d: d["tokens_per_s"]) if ok
+            else min(lines, key=lambda d: d["config"]["block_size"]))
+    return {
+        "workload": "trace-sweep",
+        "block_size_choice": pick["config"]["block_size"],
+        "rule": f"fastest wall-clock decode tokens/s with mean fragmentation <= {frag_budget:.0%}",
+        "per_block_size": {str(d["config"]["block_size"]): {
+            "tokens_per_s": d["tokens_per_s"], "device_gbs_unique": d["value"],
+            "fragmentation_mean": d["fragmentation_mean"], "device_ms_per_step": d["device_ms_per_step"]}
+            for d in lines},
+    }
+
+
 def run_trace(args, dev):
     """Continuous batching of beam-search requests over a 16 GiB K+V pool, one
     JSON line per block size: per step the host trace driver (allocator
@@ -976,6 +998,8 @@ def main():
                     help="run each step as pa_copy_blocks + pa_append_kv + pa_decode instead of pa_append_decode")
     ap.add_argument("--block-size", type=int, default=0, help="trace workload: one block size (0: 8, 16 and 32)")
     ap.add_argument("--trace-steps", type=int, default=1000)
+    ap.add_argument("--frag-budget", type=float, default=0.05,
+                    help="trace sweep: largest mean fragmentation a block-size choice may have")
     ap.add_argument("--seed", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -1004,8 +1028,11 @@ def main():
             return
         if args.workload == "trace":  # one trace, on rank 0; the other ranks only join the exit
             if rank == 0:
-                for line in run_trace(args, dev):
+                lines = run_trace(args, dev)
+                for line in lines:
                     print(json.dumps(line), flush=True)
+                if len(lines) > 1:
+                    print(json.dumps(choose_block_size(lines, args.frag_budget)), flush=True)
             if world > 1:
                 torch.distributed.barrier()
             return

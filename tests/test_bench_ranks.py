@@ -64,3 +64,17 @@ def test_reference_arm_prints_on_rank_zero_only(rank):
         assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
     else:
         assert lines == []
+
+
+def test_block_size_choice_rule():
+    """The fastest block size within the fragmentation budget; the smallest
+    when none fits."""
+    sys.path.insert(0, ROOT)
+    import bench
+    mk = lambda bs, tps, fr: {"config": {"block_size": bs}, "tokens_per_s": tps, "fragmentation_mean": fr,
+                              "value": 1.0, "device_ms_per_step": 1.0}
+    lines = [mk(8, 350e3, 0.014), mk(16, 530e3, 0.028), mk(32, 650e3, 0.056)]
+    assert bench.choose_block_size(lines, 0.05)["block_size_choice"] == 16
+    assert bench.choose_block_size(lines, 0.06)["block_size_choice"] == 32
+    assert bench.choose_block_size(lines, 0.01)["block_size_choice"] == 8
+    assert set(bench.choose_block_size(lines, 0.05)["per_block_size"]) == {"8", "16", "32"}
