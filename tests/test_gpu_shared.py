@@ -135,3 +135,46 @@ def test_shared_plan_that_does_not_fit(cuda_device):
     assert pa.pa_read_device_error() == pa.PA_DEVERR_PLAN
     ref = oracle.decode(q, host_pool(case_k), host_pool(case_v), tables, lens, scale)
     assert_attn_close(out, ref, dt)
+
+
+def test_shared_plan_across_batch_slices(cuda_device):
+    """1101 sequences (two slices of the main decode kernel, 1024 + 77) in
+    groups of 3 forks, one group straddling the slice boundary; with the
+    fused append.  The cascade kernel sees the whole batch, the main kernel
+    each slice with its own first partitions."""
+    dt, Hkv, D, bs, Hq = torch.bfloat16, 2, 128, 16, 8
+    roots_n, fan = 367, 3
+    prompts = (600 + synth.rng(101).integers(0, 400, size=roots_n)).tolist()
+    NB = sum(-(-p // bs) for p in prompts) + roots_n * fan * 3 + 16
+    order = synth.rng(102).permutation(NB)
+    A, M = pa.Allocator(NB, bs, order), oracle.AllocatorModel(NB, bs, order)
+    cache, hk, hv = _pool(NB, Hkv, bs, D, dt, cuda_device)
+    roots = _prefill(A, M, prompts, cuda_device, cache, hk, hv, dt, 103)
+    seqs = _fork_groups(A, M, roots, fan)
+    n = len(seqs)
+    assert n == 1101
+    slots, pairs = A.batch_append(seqs, [1] * n)
+    mslots, mpairs = M.batch_append(seqs, [1] * n)
+    assert slots.tolist() == mslots
+    mb = max(len(M.block_table(s)) for s in seqs)
+    tables, lens = A.build_block_tables(seqs, mb)
+    cow = pa.cow_sources(pairs, tables, lens, bs)
+    plan = pa.share_plan(tables, lens, bs)
+    assert plan.n_groups == roots_n
+    assert any(min(g) < 1024 <= max(g) for g in plan.members.tolist())
+    plan.to(cuda_device)
+    kn = synth.normal((n, Hkv, D), dt, 104)
+    vn = synth.normal((n, Hkv, D), dt, 105)
+    q = synth.normal((n, Hq, D), dt, 106)
+    scale = 1 / math.sqrt(D)
+    out = pa.pa_decode_shared(q.to(cuda_device), cache, torch.from_numpy(tables).to(cuda_device),
+                              torch.from_numpy(lens).to(cuda_device), int(lens.max()), scale, plan=plan,
+                              k_new=kn.to(cuda_device), v_new=vn.to(cuda_device),
+                              cow_src=torch.from_numpy(cow).to(cuda_device) if len(pairs) else None)
+    assert pa.pa_read_device_error() == 0
+    oracle.copy_blocks(hk, hv, mpairs)
+    oracle.append_kv(hk, hv, kn, vn, mslots)
+    assert same_bits(host_pool(cache.k), hk) and same_bits(host_pool(cache.v), hv)
+    rows = [(b, h) for b in list(range(1016, 1032)) + list(range(0, 1101, 37)) for h in (0, 7)]
+    ref = oracle.decode(q, hk, hv, tables, lens, scale, rows=rows)
+    assert_attn_close(torch.stack([out[b, h] for b, h in rows]), ref, dt)
