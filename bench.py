@@ -546,82 +546,119 @@ def unique_kv_bytes(tables: np.ndarray, lens: np.ndarray, bs: int, row_bytes: in
 
 
 def run_e2e(args, insts, wl, dev, stream):
-    """Each step from host memory, through the public API: the allocator
-    call, pinned host -> device copies of the step's inputs (q, new rows,
-    slots, tables, lengths, copy pairs), copy / append / decode, and the
-    device -> host read of the output.  Wall clock, one synchronize per step."""
+    """Each step from host memory, through the public API: the step's host
+    work (one allocator call that appends the tokens and writes the tables,
+    lengths, copy-on-write sources and sharing plan; with --unfused the
+    allocator append and table build), one pinned host -> device copy of
+    every input of the step (q, new rows, tables, lengths, copy sources,
+    plan; slots and pairs for --unfused), the step's call, and the device ->
+    host copy of its output, which the host then reads.  Wall clock over all
+    steps.  Pipelined two deep: the host prepares step i + 1 while the device
+    runs step i; copies run on their own stream, ordered by events against
+    the compute stream, and every buffer has two copies."""
     import paged_kv_cache_402_b200 as pa
 
     B, Hq, Hkv, D, bs = wl["B"], wl["Hq"], wl["Hkv"], wl["D"], wl["bs"]
     inst = insts[0]
     mb = inst.max_blocks
-    h = {
-        "q": torch.empty(B, Hq, D, dtype=torch.bfloat16).pin_memory(),
-        "k": torch.empty(B, Hkv, D, dtype=torch.bfloat16).pin_memory(),
-        "v": torch.empty(B, Hkv, D, dtype=torch.bfloat16).pin_memory(),
-        "slots": torch.empty(B, dtype=torch.int64).pin_memory(),
-        "pairs": torch.empty(B, 2, dtype=torch.int32).pin_memory(),
-        "cow": torch.empty(B, dtype=torch.int32).pin_memory(),
-        "tables": torch.empty(B, mb, dtype=torch.int32).pin_memory(),
-        "lens": torch.empty(B, dtype=torch.int32).pin_memory(),
-        "out": torch.empty(B, Hq, D, dtype=torch.bfloat16).pin_memory(),
-    }
-    g = torch.Generator().manual_seed(5)
-    h["q"].copy_(torch.randn(B, Hq, D, generator=g).to(torch.bfloat16))
-    h["k"].copy_(torch.randn(B, Hkv, D, generator=g).to(torch.bfloat16))
-    h["v"].copy_(torch.randn(B, Hkv, D, generator=g).to(torch.bfloat16))
-    d = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in h.items() if k != "out"}
-    out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
     n_steps = max(1, args.steps)
+    G2 = max(1, B // 2)
+    share = 0 if (args.unfused or args.no_share_plan) else 4
+    # one packed buffer per step: (name, shape, dtype), each part 16-byte aligned
+    parts = [("q", (B, Hq, D), torch.bfloat16), ("k", (B, Hkv, D), torch.bfloat16),
+             ("v", (B, Hkv, D), torch.bfloat16), ("tables", (B, mb), torch.int32), ("lens", (B,), torch.int32),
+             ("cow_src", (B,), torch.int32), ("first_part", (B,), torch.int32), ("members", (G2, 4), torch.int32),
+             ("parts", (G2,), torch.int32), ("slots", (B,), torch.int64), ("pairs", (B, 2), torch.int32)]
+    offs, total = {}, 0
+    for name, shape, dt in parts:
+        nbytes = int(np.prod(shape)) * torch.tensor([], dtype=dt).element_size()
+        offs[name] = (total, nbytes)
+        total += (nbytes + 15) // 16 * 16
+    g = torch.Generator().manual_seed(5)
+    rows = {"q": torch.randn(B, Hq, D, generator=g).to(torch.bfloat16),
+            "k": torch.randn(B, Hkv, D, generator=g).to(torch.bfloat16),
+            "v": torch.randn(B, Hkv, D, generator=g).to(torch.bfloat16)}
+
+    def views(buf):
+        return {name: buf[offs[name][0]:offs[name][0] + offs[name][1]].view(dt).view(shape)
+                for name, shape, dt in parts}
+
+    def make_set():
+        h_buf = torch.zeros(total, dtype=torch.uint8).pin_memory()
+        d_buf = torch.empty(total, dtype=torch.uint8, device=dev)
+        hv = views(h_buf)
+        for k in ("q", "k", "v"):
+            hv[k].copy_(rows[k])
+        np_out = {k: hv[k].numpy() for k in ("tables", "lens", "cow_src", "first_part", "members", "parts")}
+        return {"h_buf": h_buf, "d_buf": d_buf, "h": hv, "d": views(d_buf), "np": np_out,
+                "out": torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev),
+                "h_out": torch.empty(B, Hq, D, dtype=torch.bfloat16).pin_memory(),
+                "ev_in": torch.cuda.Event(), "ev_kernel": torch.cuda.Event(), "ev_out": torch.cuda.Event(),
+                "used": False}
+
+    sets = [make_set(), make_set()]
+    copy_stream = torch.cuda.Stream(device=dev)
     ws = torch.empty(max(16, pa.pa_decode_workspace_size(B, Hq, mb * bs, D)), dtype=torch.uint8, device=dev)
-    slots_np, pairs_np = h["slots"].numpy(), h["pairs"].numpy()
-    tables_np, lens_np = h["tables"].numpy(), h["lens"].numpy()
     ones = np.ones(B, np.int32)
+    scale = 1.0 / math.sqrt(D)
     seen = []
-    h2d = d2h = 0
-    plan_bytes = 0
+    checksum = 0.0
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     for i in range(n_steps):
+        S = sets[i % 2]
+        h, d = S["h"], S["d"]
+        if S["used"]:
+            S["ev_in"].synchronize()        # its pinned inputs are free again
+            S["ev_out"].synchronize()       # the output of step i - 2 is on the host
+            checksum += float(S["h_out"][0, 0, 0])
         seqs = inst.sets[inst.uses + i] if wl.get("fresh_sets") else inst.sets[0]
-        _, pairs = inst.alloc.batch_append(seqs, ones, out_slots=slots_np, out_pairs=pairs_np)
-        inst.alloc.build_block_tables(seqs, mb, out_tables=tables_np, out_lens=lens_np)
-        npairs = len(pairs)
-        names = ("q", "k", "v", "slots", "tables", "lens") if args.unfused else ("q", "k", "v", "tables", "lens")
-        for k in names:
-            d[k].copy_(h[k], non_blocking=True)
+        if args.unfused:
+            _, pairs = inst.alloc.batch_append(seqs, ones, out_slots=h["slots"].numpy(),
+                                               out_pairs=h["pairs"].numpy())
+            inst.alloc.build_block_tables(seqs, mb, out_tables=S["np"]["tables"], out_lens=S["np"]["lens"])
+            npairs, max_len, plan = len(pairs), int(S["np"]["lens"].max()), None
+        else:
+            st = inst.alloc.decode_step(seqs, mb, share_max_members=share, out=S["np"])
+            npairs, max_len = st["n_copies"], st["max_len"]
+            plan = pa.SharePlan(st["members"], st["parts"], st["first_part"])
+            if plan.n_groups:
+                plan.bind(d["members"][:plan.n_groups], d["parts"][:plan.n_groups], d["first_part"])
+        with torch.cuda.stream(copy_stream):
+            if S["used"]:
+                copy_stream.wait_event(S["ev_kernel"])   # step i - 2 no longer reads these device inputs
+            S["d_buf"].copy_(S["h_buf"], non_blocking=True)
+            S["ev_in"].record(copy_stream)
+        stream.wait_event(S["ev_in"])
+        if S["used"]:
+            stream.wait_event(S["ev_out"])               # the output buffer of step i - 2 was copied out
         if args.unfused:
             if npairs:
-                d["pairs"][:npairs].copy_(h["pairs"][:npairs], non_blocking=True)
                 pa.pa_copy_blocks(d["pairs"][:npairs], inst.cache, stream)
             pa.pa_append_kv(d["k"], d["v"], d["slots"], inst.cache, stream)
-            pa.pa_decode(d["q"], inst.cache, d["tables"], d["lens"], int(lens_np.max()), 1.0 / math.sqrt(D),
-                         out=out, workspace=ws, stream=stream)
+            pa.pa_decode(d["q"], inst.cache, d["tables"], d["lens"], max_len, scale, out=S["out"],
+                         workspace=ws, stream=stream)
         else:
-            if npairs:
-                pa.cow_sources(pairs, tables_np, lens_np, bs, out=h["cow"].numpy())
-                d["cow"].copy_(h["cow"], non_blocking=True)
-            if args.no_share_plan:
-                pa.pa_append_decode(d["k"], d["v"], d["q"], inst.cache, d["tables"], d["lens"], int(lens_np.max()),
-                                    1.0 / math.sqrt(D), cow_src=d["cow"] if npairs else None, out=out,
-                                    workspace=ws, stream=stream)
-            else:
-                plan = pa.share_plan(tables_np, lens_np, bs).to(dev)
-                plan_bytes += plan.nbytes
-                pa.pa_decode_shared(d["q"], inst.cache, d["tables"], d["lens"], int(lens_np.max()),
-                                    1.0 / math.sqrt(D), plan=plan, k_new=d["k"], v_new=d["v"],
-                                    cow_src=d["cow"] if npairs else None, out=out, workspace=ws, stream=stream)
-        h["out"].copy_(out, non_blocking=True)
-        torch.cuda.synchronize()
-        if i == 0:
-            h2d = sum(h[k].numel() * h[k].element_size() for k in names)
-            h2d += (npairs * 8) if args.unfused else (B * 4 if npairs else 0)
-            d2h = h["out"].numel() * h["out"].element_size()
-        seen.append((tables_np.copy(), lens_np.copy()))
+            pa.pa_decode_shared(d["q"], inst.cache, d["tables"], d["lens"], max_len, scale, plan=plan,
+                                k_new=d["k"], v_new=d["v"], cow_src=d["cow_src"] if npairs else None,
+                                out=S["out"], workspace=ws, stream=stream)
+        S["ev_kernel"].record(stream)
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(S["ev_kernel"])
+            S["h_out"].copy_(S["out"], non_blocking=True)
+            S["ev_out"].record(copy_stream)
+        S["used"] = True
+        seen.append((S["np"]["tables"].copy(), S["np"]["lens"].copy()))
+    for S in sets:
+        if S["used"]:
+            S["ev_out"].synchronize()
+            checksum += float(S["h_out"][0, 0, 0])
     seconds = time.perf_counter() - t0
+    torch.cuda.synchronize()
+    if not math.isfinite(checksum):
+        raise RuntimeError("non-finite output in the end-to-end steps")
     kv = sum(unique_kv_bytes(t, l, bs, 2 * Hkv * D * 2) for t, l in seen)
-    h2d += plan_bytes // n_steps
-    return {"seconds": seconds, "kv_gb": kv / 1e9, "steps": n_steps, "h2d": h2d, "d2h": d2h}
+    return {"seconds": seconds, "kv_gb": kv / 1e9, "steps": n_steps, "h2d": total, "d2h": B * Hq * D * 2}
 
 
 def run_prefill(args, rank: int, world: int, dev):

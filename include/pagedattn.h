@@ -412,6 +412,29 @@ PA_API pa_status pa_share_plan(const int32_t *tables_host, int32_t max_blocks,
                                int32_t *first_part_host, int32_t *n_groups);
 
 /*
+ * One decode step's host work in one call: appends one token to each of the
+ * n_seqs sequences (all or nothing, as pa_batch_append; PA_ERR_OUT_OF_BLOCKS
+ * leaves every state unchanged), then writes what pa_decode_shared takes:
+ *   tables_host [n_seqs][max_blocks] and lens_host [n_seqs] after the
+ *     append; a row's entries past the sequence's blocks are not written (no
+ *     kernel reads them); PA_ERR_TOO_SMALL before any change when a table
+ *     would not fit max_blocks;
+ *   cow_src_host [n_seqs]: the block a sequence's copy-on-write move copies
+ *     into its new last block, -1 for none (*n_copies of them);
+ *   with share_max_members in 2..4, the sharing plan of pa_share_plan
+ *     (members_host room for n_seqs / 2 groups x share_max_members,
+ *     parts_host room for n_seqs / 2, *n_groups); with 0, no plan and
+ *     first_part_host all zeros;
+ *   *max_len: the longest length (max_context_len of the call).
+ */
+PA_API pa_status pa_decode_step_prepare(pa_allocator *a, const int32_t *seqs, int32_t n_seqs,
+                                        int32_t max_blocks, int32_t share_max_members,
+                                        int32_t *tables_host, int32_t *lens_host,
+                                        int32_t *cow_src_host, int32_t *members_host,
+                                        int32_t *parts_host, int32_t *first_part_host,
+                                        int32_t *n_groups, int32_t *n_copies, int32_t *max_len);
+
+/*
  * The per-sequence form of a decode step's copy pairs, as pa_append_decode
  * takes it: cow_src_host[i] = the source of the pair whose destination is
  * last_blocks_host[i] (sequence i's last block after its append; -1 when it

@@ -71,6 +71,8 @@ def _load() -> ctypes.CDLL:
                                   ctypes.POINTER(pa_share_plan_t), vp, vp, sz, vp]),
         "pa_share_plan": (st, [i32p, i32, i32p, i32, i32, i32, i32p, i32p, i32p, i32p]),
         "pa_prefill": (st, [vp, cp, vp, i32, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp]),
+        "pa_decode_step_prepare": (st, [vp, i32p, i32, i32, i32, i32p, i32p, i32p, i32p, i32p, i32p,
+                                        i32p, i32p, i32p]),
         "pa_copy_blocks": (st, [vp, i32, cp, vp]),
         "pa_check_copy_pairs": (st, [i32p, i32, i32]),
         "pa_read_device_error": (st, [vp, i32p]),
@@ -291,6 +293,14 @@ class SharePlan:
                               for a in (self.members, self.parts, self.first_part))
         return self
 
+    def bind(self, members: torch.Tensor, parts: torch.Tensor, first_part: torch.Tensor) -> "SharePlan":
+        """Uses caller-owned device tensors that already hold (or, in stream
+        order before the call that reads them, will hold) this plan's arrays,
+        e.g. filled by asynchronous copies from pinned host buffers."""
+        if self.n_groups > 0:
+            self._dev = (members, parts, first_part)
+        return self
+
     @property
     def nbytes(self) -> int:
         """Bytes the device copy takes (0 without groups)."""
@@ -452,9 +462,34 @@ class Allocator:
 
     def __del__(self):
         h = getattr(self, "_h", None)
-        if h is not None and h.value:
+        if h is not None and h.value and _lib is not None:
             _lib.pa_alloc_destroy(h)
             self._h = None
+
+    def decode_step(self, seqs, max_blocks: int, share_max_members: int = 4, out: dict | None = None) -> dict:
+        """One decode step's host work in one call (pa_decode_step_prepare):
+        one token appended to every sequence, then the tables, lengths,
+        copy-on-write sources and sharing plan that pa_decode_shared takes.
+        `out` may hold preallocated int32 arrays ("tables" [n, max_blocks],
+        "lens", "cow_src", "first_part" [n], "members" [n // 2, m], "parts"
+        [n // 2]); returns them (members / parts trimmed to the groups) with
+        "n_groups", "n_copies" and "max_len"."""
+        seqs = np.ascontiguousarray(np.asarray(seqs, dtype=np.int32))
+        n = len(seqs)
+        m = max(int(share_max_members), 1)
+        o = out if out is not None else {
+            "tables": np.empty((n, max_blocks), np.int32), "lens": np.empty(n, np.int32),
+            "cow_src": np.empty(n, np.int32), "first_part": np.empty(n, np.int32),
+            "members": np.empty((max(1, n // 2), m), np.int32), "parts": np.empty(max(1, n // 2), np.int32)}
+        ng, nc, ml = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int32(0)
+        _check(_lib.pa_decode_step_prepare(self._h, _i32p(seqs), n, int(max_blocks), int(share_max_members),
+                                           _i32p(o["tables"]), _i32p(o["lens"]), _i32p(o["cow_src"]),
+                                           _i32p(o["members"]), _i32p(o["parts"]), _i32p(o["first_part"]),
+                                           ctypes.byref(ng), ctypes.byref(nc), ctypes.byref(ml)), "pa_decode_step_prepare")
+        res = dict(o)
+        res["members"], res["parts"] = o["members"][:ng.value], o["parts"][:ng.value]
+        res.update(n_groups=ng.value, n_copies=nc.value, max_len=ml.value)
+        return res
 
     def new_seq(self) -> int:
         s = ctypes.c_int32()

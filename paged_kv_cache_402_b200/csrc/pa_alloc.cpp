@@ -326,14 +326,41 @@ PA_API pa_status pa_share_plan(const int32_t *tables_host, int32_t max_blocks,
   for (int32_t b = 0; b < n_seqs; ++b)
     if (lens_host[b] > PA_PARTITION_TOKENS && max_blocks >= bpp) cand.push_back(b);
   auto row = [&](int32_t b) { return tables_host + (size_t)b * max_blocks; };
-  // buckets: equal first-partition entries, sequence order inside a bucket
-  std::stable_sort(cand.begin(), cand.end(), [&](int32_t x, int32_t y) {
-    return std::lexicographical_compare(row(x), row(x) + bpp, row(y), row(y) + bpp);
+  // buckets: equal first-partition entries, sequence order inside a bucket.
+  // Sequences are ordered by a hash of those entries (FNV-1a), then inside
+  // each run of equal hashes by their entries, then by index.
+  std::vector<std::pair<uint64_t, int32_t>> keyed;
+  keyed.reserve(cand.size());
+  for (int32_t b : cand) {
+    uint64_t h = 1469598103934665603ull;
+    const int32_t *r = row(b);
+    for (int32_t j = 0; j < bpp; ++j) {
+      h ^= (uint32_t)r[j];
+      h *= 1099511628211ull;
+    }
+    keyed.emplace_back(h, b);
+  }
+  std::sort(keyed.begin(), keyed.end(), [&](const std::pair<uint64_t, int32_t> &x,
+                                            const std::pair<uint64_t, int32_t> &y) {
+    if (x.first != y.first) return x.first < y.first;
+    const int32_t *rx = row(x.second), *ry = row(y.second);
+    if (!std::equal(rx, rx + bpp, ry)) return std::lexicographical_compare(rx, rx + bpp, ry, ry + bpp);
+    return x.second < y.second;
   });
-  size_t i = 0;
-  while (i < cand.size()) {
+  for (size_t k = 0; k < keyed.size(); ++k) cand[k] = keyed[k].second;
+  // the buckets, in the order of their first (lowest) sequence index
+  std::vector<std::pair<size_t, size_t>> runs;
+  for (size_t i = 0; i < cand.size();) {
     size_t e = i + 1;
     while (e < cand.size() && std::equal(row(cand[i]), row(cand[i]) + bpp, row(cand[e]))) ++e;
+    runs.emplace_back(i, e);
+    i = e;
+  }
+  std::sort(runs.begin(), runs.end(), [&](const std::pair<size_t, size_t> &x, const std::pair<size_t, size_t> &y) {
+    return cand[x.first] < cand[y.first];
+  });
+  for (const auto &run : runs) {
+    const size_t i = run.first, e = run.second;
     for (size_t g0 = i; g0 + 1 < e; g0 += (size_t)max_members) {
       const size_t g1 = std::min(e, g0 + (size_t)max_members);
       if (g1 - g0 < 2) break;  // a lone leftover shares with nobody
@@ -358,9 +385,65 @@ PA_API pa_status pa_share_plan(const int32_t *tables_host, int32_t max_blocks,
       for (size_t k = g0; k < g1; ++k) first_part_host[cand[k]] = parts;
       ++*n_groups;
     }
-    i = e;
   }
   return PA_OK;
+}
+
+PA_API pa_status pa_decode_step_prepare(pa_allocator *a, const int32_t *seqs, int32_t n_seqs,
+                                        int32_t max_blocks, int32_t share_max_members,
+                                        int32_t *tables_host, int32_t *lens_host,
+                                        int32_t *cow_src_host, int32_t *members_host,
+                                        int32_t *parts_host, int32_t *first_part_host,
+                                        int32_t *n_groups, int32_t *n_copies, int32_t *max_len) {
+  if (!a || n_seqs < 0 || max_blocks < 0 || !n_groups || !n_copies || !max_len) return PA_ERR_INVALID_ARG;
+  if (n_seqs > 0 && (!seqs || !tables_host || !lens_host || !cow_src_host || !first_part_host))
+    return PA_ERR_INVALID_ARG;
+  if (share_max_members != 0 &&
+      (share_max_members < 2 || share_max_members > 4 || (n_seqs > 1 && (!members_host || !parts_host))))
+    return PA_ERR_INVALID_ARG;
+  *n_groups = 0;
+  *n_copies = 0;
+  *max_len = 0;
+  const int32_t bs = a->block_size;
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    const Seq *s = a->find(seqs[i]);
+    if (!s) return PA_ERR_NOT_FOUND;
+    if (s->len == INT32_MAX) return PA_ERR_INVALID_ARG;
+    if (pa_allocator::ceil_div((int64_t)s->len + 1, bs) > max_blocks) return PA_ERR_TOO_SMALL;
+  }
+  if (n_seqs > 1) {  // a sequence may appear once
+    std::vector<int32_t> ids(seqs, seqs + n_seqs);
+    std::sort(ids.begin(), ids.end());
+    if (std::adjacent_find(ids.begin(), ids.end()) != ids.end()) return PA_ERR_INVALID_ARG;
+  }
+  // one token per sequence, all or nothing
+  int64_t need = 0;
+  for (int32_t i = 0; i < n_seqs; ++i) need += a->blocks_needed(a->seqs[seqs[i]], 1);
+  a->clear_taken();
+  if (need > (int64_t)a->free_stack.size()) return PA_ERR_OUT_OF_BLOCKS;
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    int64_t slot;
+    int32_t pair[2] = {-1, -1};
+    int32_t made = 0;
+    a->do_append(a->seqs[seqs[i]], 1, &slot, pair, &made);
+    cow_src_host[i] = made ? pair[0] : -1;  // the copy lands in the sequence's (new) last block
+    *n_copies += made;
+  }
+  // the tables (entries past a sequence's blocks are not written: no kernel
+  // reads them) and lengths
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    const Seq &s = a->seqs[seqs[i]];
+    const size_t nb = s.table.size();
+    if (nb) std::memcpy(tables_host + (int64_t)i * max_blocks, s.table.data(), sizeof(int32_t) * nb);
+    lens_host[i] = s.len;
+    *max_len = std::max(*max_len, s.len);
+  }
+  if (share_max_members == 0) {
+    for (int32_t i = 0; i < n_seqs; ++i) first_part_host[i] = 0;
+    return PA_OK;
+  }
+  return pa_share_plan(tables_host, max_blocks, lens_host, n_seqs, bs, share_max_members, members_host,
+                       parts_host, first_part_host, n_groups);
 }
 
 PA_API pa_status pa_cow_sources(const int32_t *pairs_host, int32_t n_pairs,

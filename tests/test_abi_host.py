@@ -333,3 +333,43 @@ def test_decode_shared_argument_checks():
     assert L.pa_decode_shared(*args(plan=ok_plan, ml=500, mb=32)) == pa.PA_ERR_INVALID_ARG  # one partition
     bad = pa.pa_share_plan_t(0, 16, 16, 1, 4)
     assert L.pa_decode_shared(*args(plan=bad)) == pa.PA_ERR_INVALID_ARG         # no member array
+
+
+def test_decode_step_prepare_equals_the_separate_calls():
+    """One call gives what batch_append + build_block_tables + cow_sources +
+    share_plan give on an identical allocator: forks with copies on write,
+    sharing groups, fresh blocks, and all-or-nothing on a full pool."""
+    def state(seed):
+        A = pa.Allocator(600, 16, synth.rng(seed).permutation(600))
+        roots = [A.new_seq() for _ in range(5)]
+        A.batch_append(roots, [600, 700, 37, 512, 1030])
+        seqs = roots + [A.fork(roots[0]) for _ in range(3)] + [A.fork(roots[4]) for _ in range(2)]
+        return A, seqs
+    A1, seqs = state(3)
+    A2, _ = state(3)
+    for _ in range(3):
+        got = A1.decode_step(seqs, 80)
+        slots, pairs = A2.batch_append(seqs, [1] * len(seqs))
+        tables, lens = A2.build_block_tables(seqs, 80)
+        cow = pa.cow_sources(pairs, tables, lens, 16)
+        plan = pa.share_plan(tables, lens, 16)
+        assert np.array_equal(got["lens"], lens)
+        for i, L in enumerate(lens):  # entries past a sequence's blocks are not written
+            nb = -(-int(L) // 16)
+            assert np.array_equal(got["tables"][i, :nb], tables[i, :nb])
+        assert np.array_equal(got["cow_src"], cow) and got["n_copies"] == len(pairs)
+        assert np.array_equal(got["members"], plan.members) and np.array_equal(got["parts"], plan.parts)
+        assert np.array_equal(got["first_part"], plan.first_part) and got["n_groups"] == plan.n_groups
+        assert got["max_len"] == int(lens.max())
+    assert A1.stats() == A2.stats()
+    nogroups = A1.decode_step(seqs, 80, share_max_members=0)
+    assert nogroups["n_groups"] == 0 and not nogroups["first_part"].any()
+    with pytest.raises(pa.PagedAttnError):
+        A1.decode_step(seqs, 40)  # 1030 tokens do not fit 40 blocks: nothing changes
+    before = A1.stats()
+    small = pa.Allocator(70, 16, list(range(70)))
+    r = small.new_seq()
+    small.batch_append([r], [16 * 70])
+    with pytest.raises(pa.OutOfBlocks):
+        small.decode_step([r], 80)
+    assert small.seq_len(r)[0] == 16 * 70 and A1.stats() == before
