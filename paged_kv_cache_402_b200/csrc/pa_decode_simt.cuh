@@ -294,6 +294,10 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
+// Rows with at most this many partitions take the one-round path of
+// decode_reduce.
+constexpr int kReduceFast = 16;
+
 // Merges the partitions of one (sequence, query head):
 //   M = max_p m_p,  L = sum_p l_p 2^(m_p - M),  out = sum_p acc_p 2^(m_p - M) / L
 template <typename T, int D>
@@ -310,6 +314,34 @@ __global__ void __launch_bounds__(128) decode_reduce(DecodeParams p) {
   const float *m = p.ws_m + (size_t)bh * p.max_parts;
   const float *l = p.ws_l + (size_t)bh * p.max_parts;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+
+  if (np <= kReduceFast && D <= 128) {
+    // Up to kReduceFast partitions: every thread loads all the maxima and
+    // sums (the same addresses in every thread) and its own accumulator
+    // elements in one round, then merges on its own, with no barrier.
+    const int d = threadIdx.x;
+    const float *acc = p.ws_acc + (size_t)bh * p.max_parts * D;
+    float mv[kReduceFast], lv[kReduceFast], av[kReduceFast];
+#pragma unroll
+    for (int i = 0; i < kReduceFast; ++i) {
+      const bool in = i < np;
+      mv[i] = in ? __ldcg(m + i) : -INFINITY;
+      lv[i] = in ? __ldcg(l + i) : 0.f;
+      av[i] = (in && d < D) ? __ldcg(acc + (size_t)i * D + d) : 0.f;
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kReduceFast; ++i) M = fmaxf(M, mv[i]);
+    float L = 0.f, a = 0.f;
+#pragma unroll
+    for (int i = 0; i < kReduceFast; ++i) {
+      const float f = (mv[i] == -INFINITY) ? 0.f : fast_exp2(mv[i] - M);
+      L = fmaf(lv[i], f, L);
+      a = fmaf(av[i], f, a);
+    }
+    if (d < D) store_out(reinterpret_cast<T *>(p.out) + (size_t)bh * D + d, L > 0.f ? a / L : 0.f);
+    return;
+  }
 
   float mx = -INFINITY;
   for (int i = threadIdx.x; i < np; i += blockDim.x) mx = fmaxf(mx, m[i]);
