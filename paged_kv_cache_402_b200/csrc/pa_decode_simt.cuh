@@ -298,8 +298,37 @@ __global__ void __launch_bounds__(kWarps * 32)
 // decode_reduce.
 constexpr int kReduceFast = 16;
 
-// Merges the partitions of one (sequence, query head):
-//   M = max_p m_p,  L = sum_p l_p 2^(m_p - M),  out = sum_p acc_p 2^(m_p - M) / L
+// The merge of one (sequence, query head) row over its np <= NP partitions,
+// in one fixed order:
+//   M = max_i m_i,  f_i = 2^(m_i - M) (0 for an empty partition),
+//   L = sum_i l_i f_i  (i increasing, fused multiply-adds).
+// Returns L; an output element is merge_element(acc_i, f, np, L).
+template <int NP>
+__device__ __forceinline__ float merge_weights(const float (&mv)[NP], const float (&lv)[NP], int np,
+                                               float (&f)[NP]) {
+  float M = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < NP; ++i)
+    if (i < np) M = fmaxf(M, mv[i]);
+  float L = 0.f;
+#pragma unroll
+  for (int i = 0; i < NP; ++i) {
+    f[i] = (i < np && mv[i] != -INFINITY) ? fast_exp2(mv[i] - M) : 0.f;
+    if (i < np) L = fmaf(lv[i], f[i], L);
+  }
+  return L;
+}
+
+// sum_i acc_i f_i (i increasing, fused multiply-adds) / L; 0 for an empty row.
+template <int NP>
+__device__ __forceinline__ float merge_element(const float (&av)[NP], const float (&f)[NP], int np, float L) {
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < NP; ++i)
+    if (i < np) a = fmaf(av[i], f[i], a);
+  return L > 0.f ? a / L : 0.f;
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(128) decode_reduce(DecodeParams p) {
   extern __shared__ float wsh[];  // [max_parts] weights
@@ -329,17 +358,9 @@ __global__ void __launch_bounds__(128) decode_reduce(DecodeParams p) {
       lv[i] = in ? __ldcg(l + i) : 0.f;
       av[i] = (in && d < D) ? __ldcg(acc + (size_t)i * D + d) : 0.f;
     }
-    float M = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < kReduceFast; ++i) M = fmaxf(M, mv[i]);
-    float L = 0.f, a = 0.f;
-#pragma unroll
-    for (int i = 0; i < kReduceFast; ++i) {
-      const float f = (mv[i] == -INFINITY) ? 0.f : fast_exp2(mv[i] - M);
-      L = fmaf(lv[i], f, L);
-      a = fmaf(av[i], f, a);
-    }
-    if (d < D) store_out(reinterpret_cast<T *>(p.out) + (size_t)bh * D + d, L > 0.f ? a / L : 0.f);
+    float f[kReduceFast];
+    const float L = merge_weights(mv, lv, np, f);
+    if (d < D) store_out(reinterpret_cast<T *>(p.out) + (size_t)bh * D + d, merge_element(av, f, np, L));
     return;
   }
 
