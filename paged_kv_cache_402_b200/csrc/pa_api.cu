@@ -123,6 +123,25 @@ int choose_stages(int tile_bytes) {
   return n;
 }
 
+// The partition merge after a decode launch: with at most kReduceFast
+// partitions per row, the warp-per-row kernel sized to the row's partition
+// bound (NP 4, 8 or 16), over a grid of at most 4 CTAs per SM; else one
+// CTA per row.
+template <typename T, int D>
+pa_status launch_reduce(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
+  if (max_parts > pa::kReduceFast)
+    return launch(pa::decode_reduce<T, D>, dim3(p.B * p.Hq), dim3(128), (size_t)max_parts * sizeof(float), st, p);
+  const int64_t rows = (int64_t)p.B * p.Hq;
+  int64_t grid = (rows + pa::kReduceRowWarps - 1) / pa::kReduceRowWarps;
+  const int sms = sm_count();
+  if (sms <= 0) return PA_ERR_CUDA;
+  if (grid > 4 * (int64_t)sms) grid = 4 * (int64_t)sms;
+  const dim3 block(pa::kReduceRowWarps * 32);
+  if (max_parts <= 4) return launch(pa::decode_reduce_rows<T, D, 4>, dim3((unsigned)grid), block, 0, st, p);
+  if (max_parts <= 8) return launch(pa::decode_reduce_rows<T, D, 8>, dim3((unsigned)grid), block, 0, st, p);
+  return launch(pa::decode_reduce_rows<T, D, 16>, dim3((unsigned)grid), block, 0, st, p);
+}
+
 template <typename T, int D, int G>
 pa_status launch_decode_t(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
   const int tile_bytes = p.bs * D * (int)sizeof(T);
@@ -136,7 +155,7 @@ pa_status launch_decode_t(const pa::DecodeParams &p, int32_t max_parts, cudaStre
   dim3 grid(max_parts, p.Hkv, p.B);
   pa_status s = launch(kern, grid, dim3(pa::kWarps * 32), smem, st, p, nstages);
   if (s != PA_OK || max_parts <= 1) return s;
-  return launch(pa::decode_reduce<T, D>, dim3(p.B * p.Hq), dim3(128), (size_t)max_parts * sizeof(float), st, p);
+  return launch_reduce<T, D>(p, max_parts, st);
 }
 
 template <typename T, int D>
@@ -241,8 +260,7 @@ pa_status launch_decode_tc_slice(const pa::DecodeParams &p, int32_t max_parts, c
   if (units_bound < grid) grid = (int)units_bound;
   pa_status s = launch(kern, dim3(grid), dim3(pa::TcLayout::kThreads), (size_t)smem, st, mk, mv, mq, p);
   if (s != PA_OK || max_parts <= 1) return s;
-  return launch(pa::decode_reduce<__nv_bfloat16, 128>, dim3(p.B * p.Hq), dim3(128),
-                (size_t)max_parts * sizeof(float), st, p);
+  return launch_reduce<__nv_bfloat16, 128>(p, max_parts, st);
 }
 
 // Sequences are independent: a batch larger than the kernel's per-CTA

@@ -394,4 +394,61 @@ __global__ void __launch_bounds__(128) decode_reduce(DecodeParams p) {
   }
 }
 
+// decode_reduce for calls whose rows have at most NP <= kReduceFast
+// partitions: one warp per (sequence, query head) row, lane j holding the
+// head-dim elements [j * D / 32, (j + 1) * D / 32); lane i < np loads
+// partition i's max and sum and the warp shares them by shuffle.  Rows are
+// taken in a grid-stride loop, so a few resident CTAs cover any batch and
+// the register footprint follows NP.  Same merge arithmetic as decode_reduce.
+constexpr int kReduceRowWarps = 8;
+
+template <typename T, int D, int NP>
+__global__ void __launch_bounds__(kReduceRowWarps * 32, 2) decode_reduce_rows(DecodeParams p) {
+  constexpr int E = D / 32;
+  static_assert(D % 32 == 0 && (E == 1 || E == 2 || E == 4), "head_dim");
+  static_assert(NP <= kReduceFast && NP <= 32, "partitions per row");
+  wait_prior_grid();
+  allow_next_grid();
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = (int64_t)p.B * p.Hq;
+  const int64_t stride = (int64_t)gridDim.x * kReduceRowWarps;
+  T *out = reinterpret_cast<T *>(p.out);
+  for (int64_t bh = (int64_t)blockIdx.x * kReduceRowWarps + (threadIdx.x >> 5); bh < rows; bh += stride) {
+    const int ctx = p.lens[bh / p.Hq];
+    if (ctx <= kPart || ctx > p.max_ctx) continue;  // written directly by the partition kernel
+    const int np = min((ctx + kPart - 1) / kPart, NP);
+    const float mi = lane < np ? __ldcg(p.ws_m + bh * p.max_parts + lane) : -INFINITY;
+    const float li = lane < np ? __ldcg(p.ws_l + bh * p.max_parts + lane) : 0.f;
+    const float *acc = p.ws_acc + bh * p.max_parts * D + lane * E;
+    float av[E][NP];
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      if (i < np) {
+        const float *src = acc + (size_t)i * D;
+        if constexpr (E == 4) {
+          const float4 v = __ldcg(reinterpret_cast<const float4 *>(src));
+          av[0][i] = v.x; av[1][i] = v.y; av[2][i] = v.z; av[3][i] = v.w;
+        } else if constexpr (E == 2) {
+          const float2 v = __ldcg(reinterpret_cast<const float2 *>(src));
+          av[0][i] = v.x; av[1][i] = v.y;
+        } else {
+          av[0][i] = __ldcg(src);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < E; ++k) av[k][i] = 0.f;
+      }
+    }
+    float mv[NP], lv[NP], f[NP];
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      mv[i] = __shfl_sync(0xffffffffu, mi, i);
+      lv[i] = __shfl_sync(0xffffffffu, li, i);
+    }
+    const float L = merge_weights(mv, lv, np, f);
+#pragma unroll
+    for (int k = 0; k < E; ++k) store_out(out + bh * D + lane * E + k, merge_element(av[k], f, np, L));
+  }
+}
+
 }  // namespace pa
