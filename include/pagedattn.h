@@ -316,6 +316,12 @@ PA_API pa_status pa_read_wait_timeout(void *stream, uint32_t info[4]);
 /* Static text for a status code. */
 PA_API const char *pa_status_string(pa_status s);
 
+/* The cudaError_t of the CUDA call behind the calling thread's most recent
+ * PA_ERR_CUDA from this library (0 if there was none), and CUDA's static
+ * text for such a code. */
+PA_API int32_t pa_last_cuda_error(void);
+PA_API const char *pa_cuda_error_string(int32_t code);
+
 /* Library version, "major.minor.patch". */
 PA_API const char *pa_version(void);
 

@@ -34,7 +34,11 @@ _DTYPES = {torch.float32: PA_DTYPE_F32, torch.bfloat16: PA_DTYPE_BF16}
 class PagedAttnError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {_lib.pa_status_string(status).decode()} (status {status})")
+        msg = f"{what}: {_lib.pa_status_string(status).decode()} (status {status})"
+        if status == PA_ERR_CUDA:
+            code = _lib.pa_last_cuda_error()
+            msg += f": CUDA error {code} ({_lib.pa_cuda_error_string(code).decode()})"
+        super().__init__(msg)
 
 
 class OutOfBlocks(PagedAttnError):
@@ -78,6 +82,8 @@ def _load() -> ctypes.CDLL:
         "pa_read_device_error": (st, [vp, i32p]),
         "pa_read_wait_timeout": (st, [vp, ctypes.POINTER(ctypes.c_uint32)]),
         "pa_status_string": (ctypes.c_char_p, [st]),
+        "pa_last_cuda_error": (ctypes.c_int32, []),
+        "pa_cuda_error_string": (ctypes.c_char_p, [ctypes.c_int32]),
         "pa_version": (ctypes.c_char_p, []),
         "pa_alloc_create": (st, [i32, i32, i32p, ctypes.POINTER(vp)]),
         "pa_alloc_destroy": (None, [vp]),

@@ -36,8 +36,17 @@ pa_status check_cache(const pa_cache_t *c) {
   return PA_OK;
 }
 
+// The CUDA error behind this thread's most recent PA_ERR_CUDA (0: none).
+thread_local int32_t g_last_cuda_error = 0;
+
+inline pa_status cuda_failed(cudaError_t e) {
+  g_last_cuda_error = (int32_t)e;
+  return PA_ERR_CUDA;
+}
+
 inline pa_status launch_status() {
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : cuda_failed(e);
 }
 
 // Launches with programmatic stream serialization: the kernel may be
@@ -56,9 +65,10 @@ pa_status launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) {
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  if (e != cudaSuccess) {
     (void)cudaGetLastError();
-    return PA_ERR_CUDA;
+    return cuda_failed(e);
   }
   return launch_status();
 }
@@ -97,8 +107,11 @@ bool ensure_smem(Kernel kern, int bytes, std::atomic<int> (&done)[kMaxDev]) {
   const int dev = current_device();
   if (dev < 0) return false;
   if (done[dev].load(std::memory_order_relaxed) >= bytes) return true;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) {
+    g_last_cuda_error = (int32_t)e;
     return false;
+  }
   done[dev].store(bytes, std::memory_order_relaxed);
   return true;
 }
@@ -395,6 +408,12 @@ pa_status launch_decode_dtype(const pa::DecodeParams &p, int D, int32_t max_part
 extern "C" {
 
 PA_API const char *pa_version(void) { return "0.1.0"; }
+
+PA_API int32_t pa_last_cuda_error(void) { return g_last_cuda_error; }
+
+PA_API const char *pa_cuda_error_string(int32_t code) {
+  return cudaGetErrorString(static_cast<cudaError_t>(code));
+}
 
 PA_API const char *pa_status_string(pa_status s) {
   switch (s) {

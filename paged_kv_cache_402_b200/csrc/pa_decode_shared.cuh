@@ -48,7 +48,7 @@ struct ShLayout {
   static constexpr int kOffP = kOffQ + 2 * kQ;
   static constexpr int kOffBar = kOffP + 2 * kP;
   static constexpr int kNumBars = 21;
-  static constexpr int kOffRed = kOffBar + kNumBars * 8;
+  static constexpr int kOffRed = kOffBar + (kNumBars * 8 + 15) / 16 * 16;  // 16-byte aligned
   static constexpr int kRedFloats = 2 * 4 * kN;  // [parity][warp][column]
   static constexpr int kOffRedSum = kOffRed + kRedFloats * 4;
   static constexpr int kOffTmem = kOffRedSum + kRedFloats * 4;
@@ -57,11 +57,54 @@ struct ShLayout {
   static constexpr int kUnitInts = 8 + kPart / 8;
   static constexpr int kOffUnit = kOffTmem + 16;
   static constexpr int kOffScan = kOffUnit + 2 * kUnitInts * 4;
-  static constexpr int kOffPrefix = kOffScan + 32;  // shared partitions before each group
+  static constexpr int kOffPrefix = kOffScan + 64;  // shared partitions before each group
   static constexpr int kBytes = kOffPrefix + (kMaxGroups + 1) * 4 + 1024;
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 320;
   static constexpr uint32_t kTmemCols = 128;  // S0 S1 O0 O1, kN columns each
 };
+
+// Reduces 16 columns held by every lane of a warp (v[j]: this lane's value
+// of column j) and returns column (lane % 16)'s result.  Lanes differing in
+// bit 4 are combined first (all 16 columns); then each step hands half of
+// the remaining columns to the partner lane (lane ^ 8, then ^ 4, ^ 2, ^ 1)
+// and combines the other half with the partner's: 31 shuffles instead of 16
+// separate butterflies of 5.  A sum is taken over the same pairs in the same
+// order as those butterflies, so it is bit for bit the same.  v is consumed.
+template <bool kMax>
+__device__ __forceinline__ float warp_transpose_reduce16(float (&v)[16], int lane) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float recv = __shfl_xor_sync(0xffffffffu, v[i], 16);
+    v[i] = kMax ? fmaxf(v[i], recv) : v[i] + recv;
+  }
+#pragma unroll
+  for (int off = 8; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = upper ? v[i] : v[i + off];
+      const float keep = upper ? v[i + off] : v[i];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, off);
+      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
+  return v[0];
+}
+
+// OR of `pred` over the 128 threads of softmax warpgroup `grp` (named
+// barrier 1 + grp).
+__device__ __forceinline__ bool grp_sync_or(int pred, int grp) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, 128, p;\n\t"
+      "selp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred), "r"(1 + grp)
+      : "memory");
+  return r != 0;
+}
 
 // The sharing plan of one launch: group j has members[j * max_members + m]
 // (m < max_members, -1 past its last member) sharing parts[j] partitions.
@@ -72,6 +115,9 @@ struct SharedParams {
   int32_t max_members;
 };
 
+// One CTA of 320 threads per SM.  Each of the SM's four sub-partitions
+// holds 16 K registers and three of the ten warps land on two of them, so a
+// thread gets at most 168.
 template <int G>
 __global__ void __launch_bounds__(ShLayout::kThreads, 1)
     decode_shared_tc(const __grid_constant__ CUtensorMap tmap_k,
@@ -105,11 +151,11 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&qfull[i], 1);
-      mbar_init(&qempty[i], 2);  // the MMA lane's commit + the softmax warpgroup
+      mbar_init(&qempty[i], 3);  // the MMA lane's commit + each softmax warpgroup
       mbar_init(&sfull[i], 1);
-      mbar_init(&pfull[i], 128);
+      mbar_init(&pfull[i], 256);
       mbar_init(&pvdone[i], 1);
-      mbar_init(&ofree[i], 128);
+      mbar_init(&ofree[i], 256);
     }
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -209,13 +255,17 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
       if (lane < nb_unit) x0 = tr[lane];
       if (lane + 32 < nb_unit) x1 = tr[lane + 32];
     };
-    ShUnit un{};
-    int32_t e0, e1;
+    ShUnit un{}, nx{};
+    int32_t e0, e1, f0, f1;
     int u = blockIdx.x;
     load_unit(u, un, e0, e1);
     wait_prior_grid();  // the copies read the pool and Q, which may be written just before
     allow_next_grid();
     while (ok && u < num_units) {
+      // The next unit's description (members, table entries) is loaded while
+      // this unit's copies are in flight: after its second chunk's loads,
+      // where the two-stage ring makes the producer wait anyway.
+      bool have_next = false;
       if (un.nmem > 0) {
         const int qs = qi & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((qi >> 1) & 1) ^ 1))) { ok = false; break; }
@@ -265,11 +315,18 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
             }
           }
           if (!ok) break;
+          if (ci == 1) {
+            load_unit(u + gridDim.x, nx, f0, f1);
+            have_next = true;
+          }
         }
         if (!ok) break;
       }
+      if (!have_next) load_unit(u + gridDim.x, nx, f0, f1);
       u += gridDim.x;
-      load_unit(u, un, e0, e1);
+      un = nx;
+      e0 = f0;
+      e1 = f1;
     }
     if (ok) {  // no work left: an empty unit stops the consumers
       const int qs = qi & 1;
@@ -356,6 +413,12 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
         __syncwarp();
         if (pending.c >= 0 && !issue_pv(pending)) { ok = false; break; }
         pending = PvJob{c, qi, ci == 0};
+        if (ci == nchunks - 1) {
+          // the unit's last PV goes out at once: the epilogue waits for it,
+          // and the next unit's first K tile may still be on its way
+          if (!issue_pv(pending)) { ok = false; break; }
+          pending.c = -1;
+        }
       }
       ++qi;
     }
@@ -366,15 +429,22 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
     mbar_wait(drain, 0);
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    // Two warpgroups split the columns: warps 2-5 take columns 0-15 of S and
+    // O (member slots 0 and 1), warps 6-9 columns 16-31 (slots 2 and 3).
+    // Columns are independent, so each group keeps its own running maxima
+    // and sums, lazy reference and reductions (named barrier 1 + group).
     wait_prior_grid();  // before the first write of the workspace
     allow_next_grid();
-    const int wq = warp & 3;
-    const int r = wq * 32 + lane;  // token row (softmax) / head-dim row (O)
+    constexpr int NC = N / 2;         // columns of one warpgroup
+    const int grp = (warp - 2) >> 2;  // 0: warps 2-5, 1: warps 6-9
+    const int c0 = grp * NC;          // the group's first column
+    const int wq = warp & 3;          // the warp's quarter of the TMEM lanes
+    const int r = wq * 32 + lane;     // token row (softmax) / head-dim row (O)
     const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
     const int bs = p.bs;
     const int log2_bs = bs == 8 ? 3 : (bs == 16 ? 4 : 5);
-    float m[N], l[N];
-    int pun_j = 0, pun_g = 0, pun_part = 0, pun_nmem = 0, pun_b[L::kSlots] = {0, 0, 0, 0};
+    float m[NC], l[NC];
+    int pun_g = 0, pun_part = 0, pun_nmem = 0, pun_b[L::kSlots] = {0, 0, 0, 0};
     bool pend = false;
     int p_clast = 0, p_u = 0;
     bool bad = false, stop = false;
@@ -383,40 +453,48 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
     };
     // column n of S / O: member slot n / 8, query head n % 8 of the group
     auto col_valid = [&](int n, int nmem) { return (n >> 3) < nmem && (n & 7) < G; };
+    // [group][parity][warp][column] partial maxima and sums
+    auto red_at = [&](float *base, int parity) { return base + (grp * 2 + parity) * 4 * NC; };
 
     // the previous unit's O and sums -> its members' workspace rows
     auto epilogue = [&]() {
-      float o[N];
+      float o[NC];
       warp_wait(&pvdone[p_clast & 1], (p_clast >> 1) & 1);
       if (!bad) {
         tc::fence_after_sync();
-        tc::tmem_ld32(trow + 2 * N + (p_u & 1) * N, o);
+        tc::tmem_ld16(trow + 2 * N + (p_u & 1) * N + c0, o);
       }
       tc::fence_before_sync();
       mbar_arrive(&ofree[p_u & 1]);
-      const int parity = p_u & 1;
+      float *rs = red_at(red_sum, p_u & 1);
+      {  // this warp's part of every column's sum; lane j (and j + 16) holds column j
+        float v[NC];
 #pragma unroll
-      for (int n = 0; n < N; ++n) {
-        float v = l[n];
-#pragma unroll
-        for (int k = 16; k > 0; k >>= 1) v += __shfl_xor_sync(0xffffffffu, v, k);
-        if (lane == 0) red_sum[(parity * 4 + wq) * N + n] = v;
+        for (int j = 0; j < NC; ++j) v[j] = l[j];
+        const float t = warp_transpose_reduce16<false>(v, lane);
+        if (lane < NC) rs[wq * NC + lane] = t;
       }
-      stop = wg_sync_or(bad);
+      stop = grp_sync_or(bad, grp);
       if (stop) return;
+      // workspace rows of the group's two member slots at query head 0;
+      // column j is row rb[j / 8] + (j % 8) * max_parts
+      const size_t hb = (size_t)pun_g * G;
+      const size_t rb0 = ((size_t)(grp ? pun_b[2] : pun_b[0]) * p.Hq + hb) * p.max_parts + pun_part;
+      const size_t rb1 = ((size_t)(grp ? pun_b[3] : pun_b[1]) * p.Hq + hb) * p.max_parts + pun_part;
+      auto ws_row = [&](int j) { return (j < 8 ? rb0 : rb1) + (size_t)(j & 7) * p.max_parts; };
 #pragma unroll
-      for (int n = 0; n < N; ++n) {
-        if (!col_valid(n, pun_nmem)) continue;
+      for (int j = 0; j < NC; ++j)
+        if (col_valid(c0 + j, pun_nmem)) p.ws_acc[ws_row(j) * 128 + r] = o[j];
+      if (wq == 0 && lane < NC && col_valid(c0 + lane, pun_nmem)) {  // lane j: column j's max and sum
         float Ls = 0.f;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) Ls += red_sum[(parity * 4 + w) * N + n];
-        const int b = pun_b[n >> 3], h = pun_g * G + (n & 7);
-        const size_t row = ((size_t)b * p.Hq + h) * p.max_parts + pun_part;
-        p.ws_acc[row * 128 + r] = o[n];
-        if (r == 0) {
-          p.ws_m[row] = m[n];
-          p.ws_l[row] = Ls;
-        }
+        for (int w = 0; w < 4; ++w) Ls += rs[w * NC + lane];
+        float mj = 0.f;
+#pragma unroll
+        for (int j = 0; j < NC; ++j)
+          if (j == lane) mj = m[j];
+        p.ws_m[ws_row(lane)] = mj;
+        p.ws_l[ws_row(lane)] = Ls;
       }
     };
 
@@ -424,7 +502,7 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
     for (; !stop; ++qi) {
       const int qs = qi & 1;
       warp_wait(&qfull[qs], (qi >> 1) & 1);
-      stop = wg_sync_or(bad);
+      stop = grp_sync_or(bad, grp);
       if (stop) break;
       const int32_t *us = unit_slots + qs * L::kUnitInts;
       const int nmem = us[3];
@@ -441,66 +519,81 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
       for (int k = 0; k < L::kSlots; ++k) ub[k] = us[4 + k];
       const int32_t *ents = us + 8;
 #pragma unroll
-      for (int n = 0; n < N; ++n) {
-        m[n] = -INFINITY;
-        l[n] = 0.f;
+      for (int j = 0; j < NC; ++j) {
+        m[j] = -INFINITY;
+        l[j] = 0.f;
       }
       constexpr int nchunks = kPart / L::kChunk;
       for (int ci = 0; ci < nchunks; ++ci, ++c) {
-        float s[N];
+        float s[NC];
         warp_wait(&sfull[c & 1], (c >> 1) & 1);
         if (!bad) {
           tc::fence_after_sync();
-          tc::tmem_ld32(trow + (c & 1) * N, s);
+          tc::tmem_ld16(trow + (c & 1) * N + c0, s);
         }
         const int32_t blk = ents[(ci * L::kChunk + r) >> log2_bs];
         const bool valid = blk >= 0 && blk < p.num_blocks;
         bool need = false;
 #pragma unroll
-        for (int n = 0; n < N; ++n) {
-          s[n] = (valid && !bad && col_valid(n, nmem)) ? s[n] * p.scale_log2 : -INFINITY;
-          need |= s[n] > m[n] + kLazyRescale;
+        for (int j = 0; j < NC; ++j) {
+          s[j] = (valid && !bad && col_valid(c0 + j, nmem)) ? s[j] * p.scale_log2 : -INFINITY;
+          need |= s[j] > m[j] + kLazyRescale;
         }
-        float mnew[N];
-        if (wg_sync_or(need || bad)) {
+        float mnew[NC];
+        if (grp_sync_or(need || bad, grp)) {
+          float *rm = red_at(red_max, c & 1);
+          {  // this warp's max of every column; lane j (and j + 16) holds column j
+            float v[NC];
 #pragma unroll
-          for (int n = 0; n < N; ++n) {
-            float v = s[n];
-#pragma unroll
-            for (int k = 16; k > 0; k >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, k));
-            if (lane == 0) red_max[((c & 1) * 4 + wq) * N + n] = v;
+            for (int j = 0; j < NC; ++j) v[j] = s[j];
+            const float t = warp_transpose_reduce16<true>(v, lane);
+            if (lane < NC) rm[wq * NC + lane] = t;
           }
-          stop = wg_sync_or(bad);
+          stop = grp_sync_or(bad, grp);
           if (stop) break;
+          const float4 *rm4 = reinterpret_cast<const float4 *>(rm);
 #pragma unroll
-          for (int n = 0; n < N; ++n) {
-            float cm = red_max[((c & 1) * 4 + 0) * N + n];
+          for (int j4 = 0; j4 < NC / 4; ++j4) {
+            float4 cm = rm4[j4];
 #pragma unroll
-            for (int w = 1; w < 4; ++w) cm = fmaxf(cm, red_max[((c & 1) * 4 + w) * N + n]);
-            mnew[n] = fmaxf(m[n], cm);
+            for (int w = 1; w < 4; ++w) {
+              const float4 x = rm4[w * (NC / 4) + j4];
+              cm.x = fmaxf(cm.x, x.x);
+              cm.y = fmaxf(cm.y, x.y);
+              cm.z = fmaxf(cm.z, x.z);
+              cm.w = fmaxf(cm.w, x.w);
+            }
+            mnew[4 * j4 + 0] = fmaxf(m[4 * j4 + 0], cm.x);
+            mnew[4 * j4 + 1] = fmaxf(m[4 * j4 + 1], cm.y);
+            mnew[4 * j4 + 2] = fmaxf(m[4 * j4 + 2], cm.z);
+            mnew[4 * j4 + 3] = fmaxf(m[4 * j4 + 3], cm.w);
           }
         } else {
 #pragma unroll
-          for (int n = 0; n < N; ++n) mnew[n] = m[n];
+          for (int j = 0; j < NC; ++j) mnew[j] = m[j];
         }
         // weights of the old reference against the new one: 1 where it stays
-        auto alpha_of = [&](int n) { return mnew[n] == m[n] ? 1.f : exp2f(m[n] - mnew[n]); };
+        float alpha[NC];
         bool moved = false;
 #pragma unroll
-        for (int n = 0; n < N; ++n) moved |= mnew[n] != m[n];
+        for (int j = 0; j < NC; ++j) {
+          moved |= mnew[j] != m[j];
+          alpha[j] = (mnew[j] == m[j]) ? 1.f : ex2_approx(m[j] - mnew[j]);
+        }
         if (moved && ci > 0) {
-          // rescale the unit's O once PV(c-1) has landed, before PV(c) adds
+          // rescale the group's columns of the unit's O once PV(c-1) has
+          // landed, before PV(c) adds
           warp_wait(&pvdone[(c - 1) & 1], ((c - 1) >> 1) & 1);
           if (!bad) {
-            const uint32_t obuf = trow + 2 * N + (qi & 1) * N;
-            float o[N];
+            const uint32_t obuf = trow + 2 * N + (qi & 1) * N + c0;
+            float o[NC];
             tc::fence_after_sync();
-            tc::tmem_ld32(obuf, o);
+            tc::tmem_ld16(obuf, o);
 #pragma unroll
-            for (int k = 0; k < N / 8; ++k) {
+            for (int k = 0; k < NC / 8; ++k) {
               float o8[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) o8[e] = o[8 * k + e] * alpha_of(8 * k + e);
+              for (int e = 0; e < 8; ++e) o8[e] = o[8 * k + e] * alpha[8 * k + e];
               tc::tmem_st8(obuf + 8 * k, o8);
             }
           }
@@ -508,10 +601,11 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
         __nv_bfloat16 *pb = reinterpret_cast<__nv_bfloat16 *>(smem + L::kOffP + (c & 1) * L::kP);
         const int kh = r >> 6, rr = r & 63;
 #pragma unroll
-        for (int n = 0; n < N; ++n) {
-          const float pv = s[n] == -INFINITY ? 0.f : exp2f(s[n] - mnew[n]);
-          l[n] = fmaf(l[n], alpha_of(n), pv);
-          m[n] = mnew[n];
+        for (int j = 0; j < NC; ++j) {
+          const int n = c0 + j;
+          const float pv = s[j] == -INFINITY ? 0.f : ex2_approx(s[j] - mnew[j]);
+          l[j] = fmaf(l[j], alpha[j], pv);
+          m[j] = mnew[j];
           // P^T row n (K-major, 128-byte swizzle): token r in half kh
           const int off = kh * (N * 64) + (n >> 3) * 512 + (n & 7) * 64 + (((rr >> 3) ^ (n & 7)) << 3) + (rr & 7);
           pb[off] = __float2bfloat16_rn(pv);
@@ -519,11 +613,10 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
         fence_proxy_async_smem();
         tc::fence_before_sync();
         mbar_arrive(&pfull[c & 1]);
-        if (ci == nchunks - 1 && threadIdx.x == 64) mbar_arrive(&qempty[qs]);
+        if (ci == nchunks - 1 && r == 0) mbar_arrive(&qempty[qs]);  // one arrive per group
       }
       if (stop) break;
       pend = true;
-      pun_j = us[0];
       pun_g = ug;
       pun_part = upart;
       pun_nmem = nmem;
@@ -532,7 +625,6 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
       p_clast = c - 1;
       p_u = qi;
     }
-    (void)pun_j;
     if (stop) raise_error(PA_DEVERR_TIMEOUT);
   }
 

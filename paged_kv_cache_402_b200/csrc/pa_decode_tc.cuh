@@ -94,6 +94,16 @@ struct TcLayout {
   static constexpr uint32_t kTmemCols = 64;  // S0 S1 O0 O1, kN columns each
 };
 
+// 2^x by the MUFU approximation (flushes denormal results to zero): the
+// weights only feed a bf16 operand and fp32 sums.  Every tensor-core kernel
+// takes its softmax weights with it, so that the cascade and the partition
+// kernel give the same statistics for the same tiles.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Largest excess (base-2 units) of a score over the running reference before
 // the reference is moved: weights then stay below 2^8, far inside the range
 // of the bf16 P operand and the fp32 sums.
@@ -740,7 +750,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
 #pragma unroll
         for (int n = 0; n < G; ++n) {
           moved |= mnew[n] != m[n];
-          alpha[n] = (mnew[n] == m[n]) ? 1.f : exp2f(m[n] - mnew[n]);
+          alpha[n] = (mnew[n] == m[n]) ? 1.f : ex2_approx(m[n] - mnew[n]);
         }
         if (moved && ci > 0) {
           // O of this unit holds the chunks before c weighed against the old
@@ -759,7 +769,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         const int kh = r >> 6, rr = r & 63;
 #pragma unroll
         for (int n = 0; n < G; ++n) {
-          const float pv = valid ? exp2f(x[n] - mnew[n]) : 0.f;
+          const float pv = valid ? ex2_approx(x[n] - mnew[n]) : 0.f;
           l[n] = fmaf(l[n], alpha[n], pv);
           m[n] = mnew[n];
           // P^T row n (K-major, 128-byte swizzle): token r in half kh

@@ -40,14 +40,6 @@
 
 namespace pa {
 
-// 2^x by the MUFU approximation (flushes denormal results to zero): the
-// weights only feed a bf16 operand and fp32 sums.
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 struct PfLayout {
   static constexpr int kM = 128;           // query rows per tile
   static constexpr int kChunk = 128;       // keys per chunk

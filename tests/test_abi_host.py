@@ -48,6 +48,10 @@ def test_status_strings_and_version():
     assert pa.lib().pa_status_string(pa.PA_OK) == b"ok"
     assert pa.lib().pa_status_string(pa.PA_ERR_OUT_OF_BLOCKS) == b"out of free blocks"
     assert pa.lib().pa_version().count(b".") == 2
+    # no CUDA call of the library has failed on this thread
+    assert pa.lib().pa_last_cuda_error() == 0
+    assert pa.lib().pa_cuda_error_string(0) == b"no error"
+    assert pa.lib().pa_cuda_error_string(2) == b"out of memory"
 
 
 def _cache_struct(**kw):
