@@ -63,34 +63,6 @@ struct ShLayout {
   static constexpr uint32_t kTmemCols = 128;  // S0 S1 O0 O1, kN columns each
 };
 
-// Reduces 16 columns held by every lane of a warp (v[j]: this lane's value
-// of column j) and returns column (lane % 16)'s result.  Lanes differing in
-// bit 4 are combined first (all 16 columns); then each step hands half of
-// the remaining columns to the partner lane (lane ^ 8, then ^ 4, ^ 2, ^ 1)
-// and combines the other half with the partner's: 31 shuffles instead of 16
-// separate butterflies of 5.  A sum is taken over the same pairs in the same
-// order as those butterflies, so it is bit for bit the same.  v is consumed.
-template <bool kMax>
-__device__ __forceinline__ float warp_transpose_reduce16(float (&v)[16], int lane) {
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float recv = __shfl_xor_sync(0xffffffffu, v[i], 16);
-    v[i] = kMax ? fmaxf(v[i], recv) : v[i] + recv;
-  }
-#pragma unroll
-  for (int off = 8; off >= 1; off >>= 1) {
-    const bool upper = (lane & off) != 0;
-#pragma unroll
-    for (int i = 0; i < off; ++i) {
-      const float send = upper ? v[i] : v[i + off];
-      const float keep = upper ? v[i + off] : v[i];
-      const float recv = __shfl_xor_sync(0xffffffffu, send, off);
-      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
-    }
-  }
-  return v[0];
-}
-
 // OR of `pred` over the 128 threads of softmax warpgroup `grp` (named
 // barrier 1 + grp).
 __device__ __forceinline__ bool grp_sync_or(int pred, int grp) {
@@ -471,7 +443,7 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
         float v[NC];
 #pragma unroll
         for (int j = 0; j < NC; ++j) v[j] = l[j];
-        const float t = warp_transpose_reduce16<false>(v, lane);
+        const float t = warp_reduce_columns<NC, false>(v, lane);
         if (lane < NC) rs[wq * NC + lane] = t;
       }
       stop = grp_sync_or(bad, grp);
@@ -546,7 +518,7 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
             float v[NC];
 #pragma unroll
             for (int j = 0; j < NC; ++j) v[j] = s[j];
-            const float t = warp_transpose_reduce16<true>(v, lane);
+            const float t = warp_reduce_columns<NC, true>(v, lane);
             if (lane < NC) rm[wq * NC + lane] = t;
           }
           stop = grp_sync_or(bad, grp);

@@ -76,7 +76,7 @@ struct TcLayout {
   static constexpr int kOffP = kOffQ + 2 * kQ;
   static constexpr int kOffBar = kOffP + 2 * kP;
   static constexpr int kNumBars = 25;
-  static constexpr int kOffRed = kOffBar + kNumBars * 8;
+  static constexpr int kOffRed = kOffBar + (kNumBars * 8 + 15) / 16 * 16;  // 16-byte aligned
   static constexpr int kRedFloats = 2 * 4 * kN;  // [parity][warp][head]
   static constexpr int kOffRedSum = kOffRed + kRedFloats * 4;
   static constexpr int kOffTmem = kOffRedSum + kRedFloats * 4;
@@ -102,6 +102,63 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Reduces NC columns held by every lane of a warp (v[n]: this lane's value
+// of column n) and returns column (lane % NC)'s result.  Lanes differing in
+// bit 4, then 3, ... down to bit log2(NC) are combined over all columns; then
+// each further step hands half of the remaining columns to the partner lane
+// (lane ^ NC/2, ..., lane ^ 1) and combines the other half with the
+// partner's.  NC log2(32 / NC) + NC - 1 shuffles instead of 5 NC.  A sum is
+// taken over the same pairs in the same order as a butterfly per column
+// (bit 4 first, ..., bit 0), so it has the same bits.  v is consumed.
+template <int NC, bool kMax>
+__device__ __forceinline__ float warp_reduce_columns(float (&v)[NC], int lane) {
+  static_assert(NC >= 1 && NC <= 32 && (NC & (NC - 1)) == 0, "columns");
+#pragma unroll
+  for (int off = 16; off >= NC; off >>= 1) {
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+      const float recv = __shfl_xor_sync(0xffffffffu, v[i], off);
+      v[i] = kMax ? fmaxf(v[i], recv) : v[i] + recv;
+    }
+  }
+#pragma unroll
+  for (int off = NC / 2; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = upper ? v[i] : v[i + off];
+      const float keep = upper ? v[i + off] : v[i];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, off);
+      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
+  return v[0];
+}
+
+// Combines the four warps' partial results of columns 0..NC-1 (red[w * ld + n],
+// 16-byte aligned rows) in warp order: out[n] = op(...op(op(init, red[n]),
+// red[ld + n])..., red[3 ld + n]).
+template <int NC, bool kMax>
+__device__ __forceinline__ void combine_warps(const float *red, int ld, float init, float (&out)[NC]) {
+#pragma unroll
+  for (int n = 0; n < NC; ++n) out[n] = init;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    if constexpr (NC % 4 == 0) {
+#pragma unroll
+      for (int n4 = 0; n4 < NC / 4; ++n4) {
+        const float4 x = reinterpret_cast<const float4 *>(red + w * ld)[n4];
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) out[4 * n4 + k] = kMax ? fmaxf(out[4 * n4 + k], xs[k]) : out[4 * n4 + k] + xs[k];
+      }
+    } else {
+#pragma unroll
+      for (int n = 0; n < NC; ++n) out[n] = kMax ? fmaxf(out[n], red[w * ld + n]) : out[n] + red[w * ld + n];
+    }
+  }
 }
 
 // Largest excess (base-2 units) of a score over the running reference before
@@ -421,12 +478,13 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         if (!ok) break;
       }
       if (!ok) break;
-      if (ns >= 0) cow_copy(un, nd, ns);
       // The next unit is drawn only now, with the ring full of this unit's
       // chunks (which hide the draw's latency): a CTA never holds more work
-      // than that when the queue runs dry, so all CTAs finish together.
+      // than that when the queue runs dry, so all CTAs finish together.  The
+      // copy on write goes out while the draw is in flight.
       int raw_next = 0;
       if (lane == 0) raw_next = (int)gridDim.x + (int)atomicAdd(sched, 1u);
+      if (ns >= 0) cow_copy(un, nd, ns);
       u = __shfl_sync(0xffffffffu, raw_next, 0);
       load_entries(u, un, e0, e1, nd, ns);
     }
@@ -630,29 +688,28 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       tc::fence_before_sync();
       mbar_arrive(&ofree[p_u & 1]);
       const int parity = p_u & 1;
+      {  // this warp's part of every head's sum; lane n holds head n % G
+        float v[G];
 #pragma unroll
-      for (int n = 0; n < G; ++n) {
-        float v = l_done[n];
-#pragma unroll
-        for (int k = 16; k > 0; k >>= 1) v += __shfl_xor_sync(0xffffffffu, v, k);
-        if (lane == 0) red_sum[(parity * 4 + wq) * N + n] = v;
+        for (int n = 0; n < G; ++n) v[n] = l_done[n];
+        const float t = warp_reduce_columns<G, false>(v, lane);
+        if (lane < G) red_sum[(parity * 4 + wq) * N + lane] = t;
       }
       stop = wg_sync_or(bad);
       if (stop) return;
+      float Ls[G];
+      combine_warps<G, false>(red_sum + parity * 4 * N, N, 0.f, Ls);
+      const size_t hrow = (size_t)pun.b * p.Hq + pun.g * G;  // query row of head 0 of the group
 #pragma unroll
       for (int n = 0; n < G; ++n) {
-        float Ls = 0.f;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) Ls += red_sum[(parity * 4 + w) * N + n];
-        const int h = pun.g * G + n;
         if (pun.single) {
-          out[((size_t)pun.b * p.Hq + h) * 128 + r] = __float2bfloat16_rn(Ls > 0.f ? o[n] / Ls : 0.f);
+          out[(hrow + n) * 128 + r] = __float2bfloat16_rn(Ls[n] > 0.f ? o[n] / Ls[n] : 0.f);
         } else {
-          const size_t row = ((size_t)pun.b * p.Hq + h) * p.max_parts + pun.part;
+          const size_t row = (hrow + n) * p.max_parts + pun.part;
           p.ws_acc[row * 128 + r] = o[n];
           if (r == 0) {
             p.ws_m[row] = m_done[n];
-            p.ws_l[row] = Ls;
+            p.ws_l[row] = Ls[n];
           }
         }
       }
@@ -725,22 +782,19 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         }
         float mnew[G];
         if (wg_sync_or(need || bad)) {  // uniform: some row needs a new reference (or gave up)
+          {  // this warp's max of every head; lane n holds head n % G
+            float v[G];
 #pragma unroll
-          for (int n = 0; n < G; ++n) {
-            float v = x[n];
-#pragma unroll
-            for (int k = 16; k > 0; k >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, k));
-            if (lane == 0) red_max[((c & 1) * 4 + wq) * N + n] = v;
+            for (int n = 0; n < G; ++n) v[n] = x[n];
+            const float t = warp_reduce_columns<G, true>(v, lane);
+            if (lane < G) red_max[((c & 1) * 4 + wq) * N + lane] = t;
           }
           stop = wg_sync_or(bad);
           if (stop) break;
+          float cm[G];
+          combine_warps<G, true>(red_max + (c & 1) * 4 * N, N, -INFINITY, cm);
 #pragma unroll
-          for (int n = 0; n < G; ++n) {
-            float cm = red_max[((c & 1) * 4 + 0) * N + n];
-#pragma unroll
-            for (int w = 1; w < 4; ++w) cm = fmaxf(cm, red_max[((c & 1) * 4 + w) * N + n]);
-            mnew[n] = fmaxf(m[n], cm);
-          }
+          for (int n = 0; n < G; ++n) mnew[n] = fmaxf(m[n], cm[n]);
         } else {
 #pragma unroll
           for (int n = 0; n < G; ++n) mnew[n] = m[n];
