@@ -72,13 +72,14 @@ def measured_tensor_peak():
 
 
 def kernel_source_hash() -> str:
-    """Hash of the decode kernel sources; ties an ncu traffic figure to them."""
+    """Hash of the sources the partition kernel and its reduce are built from
+    (not the cascade's, which they do not include); ties an ncu traffic
+    figure to them."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_402_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.startswith("pa_decode") or f in ("pa_device.cuh", "pa_tc.cuh"):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(fh.read())
+    for f in ("pa_decode_tc.cuh", "pa_decode_simt.cuh", "pa_device.cuh", "pa_tc.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()[:16]
 
 

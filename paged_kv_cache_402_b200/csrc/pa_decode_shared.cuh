@@ -16,15 +16,20 @@
 //
 // Same machinery as decode_partition_tc (see there): persistent CTAs, a TMA
 // producer warp loading whole (block, kv head) tiles as 4-D boxes into
-// 128-byte-swizzled K and V rings, one MMA warp, a 128-thread softmax
-// warpgroup.  What differs:
+// 128-byte-swizzled K and V rings, one MMA warp, softmax warps with the lazy
+// reference and the transposed column reductions.  What differs:
 //  * a work unit is (group, kv head, shared partition): 512 tokens, always
-//    full, handed out round-robin (all units are the same size);
+//    full, handed out round-robin (all units are the same size); the
+//    producer loads the next unit's description while the current unit's
+//    copies are in flight;
 //  * the Q tile holds the group's members in 8-row slots (member m: rows
 //    8m .. 8m + G - 1, one 2-D TMA box per column half per member), so the
 //    MMAs are M = 128 tokens x N = 32 query rows;
+//  * two softmax warpgroups (warps 2-5 and 6-9) take columns 0-15 and 16-31
+//    of S and O, each with its own running statistics and named barrier;
 //  * the epilogue writes workspace rows for every (member, query head), read
-//    from O at the start of the next unit;
+//    from O at the start of the next unit (the MMA warp issues a unit's last
+//    PV at once, so it does not wait for the next unit's first K tile);
 //  * two ring stages (the larger Q and P tiles take the third one's room).
 #pragma once
 
