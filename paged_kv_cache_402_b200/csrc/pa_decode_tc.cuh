@@ -46,9 +46,10 @@
 //    from the copy-on-write source when there is one (the rows before the
 //    new one are the same); the MMA warp writes the new key/value row into
 //    the landed K and V tiles before the MMAs read them, and stores it to
-//    the pool; the producer copies the source tile over the destination
-//    after issuing the unit's loads.  No copy of this call reads what those
-//    stores write, so nothing waits for them.
+//    the pool; the softmax threads copy the source tile over the
+//    destination (loads at the unit's start, stores once its first chunk's
+//    weights are out).  No copy of this call reads what those stores write,
+//    so nothing waits for them.
 //  * Every mbarrier wait has an iteration limit; a thread that gives up sets
 //    PA_DEVERR_TIMEOUT and its role stops, the softmax warps leave together
 //    through a reducing barrier, the MMA lane drains its MMAs, and the CTA
@@ -81,9 +82,11 @@ struct TcLayout {
   static constexpr int kOffRedSum = kOffRed + kRedFloats * 4;
   static constexpr int kOffTmem = kOffRedSum + kRedFloats * 4;
   // per-unit description written by the producer next to the unit's Q slot:
-  // [b, g, part, t0, t1, nchunks, single, newest-token block or -1] + the
-  // unit's table entries (as the copies read them)
-  static constexpr int kUnitInts = 8 + kPart / 8;
+  // [b, g, part, t0, t1, nchunks, single, newest-token block or -1,
+  //  copy-on-write source of that block or -1, 0] + the unit's table entries
+  // (as the copies read them)
+  static constexpr int kUnitHead = 10;
+  static constexpr int kUnitInts = kUnitHead + kPart / 8;
   static constexpr int kOffUnit = kOffTmem + 16;
   static constexpr int kOffScan = kOffUnit + 2 * kUnitInts * 4;  // 8 ints
   static constexpr int kOffPrefix = kOffScan + 32;
@@ -386,37 +389,6 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         }
       }
     };
-    // Copy on write of the newest token's block: the source tile over the
-    // destination's, every row but the new one (the MMA warp stores that).
-    // Nothing in this call reads the destination, so nothing waits for it.
-    auto cow_copy = [&](const TcUnit &un, int32_t dst, int32_t src) {
-      constexpr int kRowVecs = 16;  // one bf16 row of 128 in 16-byte vectors
-      const int tile_vecs = bs * kRowVecs;
-      const int off = (un.t1 - 1) % bs;
-      const uint4 *ks = static_cast<const uint4 *>(p.k) + ((size_t)src * p.Hkv + un.g) * tile_vecs;
-      const uint4 *vs = static_cast<const uint4 *>(p.v) + ((size_t)src * p.Hkv + un.g) * tile_vecs;
-      uint4 *kd = static_cast<uint4 *>(const_cast<void *>(p.k)) + ((size_t)dst * p.Hkv + un.g) * tile_vecs;
-      uint4 *vd = static_cast<uint4 *>(const_cast<void *>(p.v)) + ((size_t)dst * p.Hkv + un.g) * tile_vecs;
-      for (int base = 0; base < tile_vecs; base += 32 * 8) {
-        uint4 a[8], b8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int i = base + k * 32 + lane;
-          if (i < tile_vecs) {
-            a[k] = ks[i];
-            b8[k] = vs[i];
-          }
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int i = base + k * 32 + lane;
-          if (i < tile_vecs && (i >> 4) != off) {
-            kd[i] = a[k];
-            vd[i] = b8[k];
-          }
-        }
-      }
-    };
     TcUnit un{};
     int32_t e0, e1, nd, ns;
     int u = blockIdx.x;  // the first unit of every CTA is fixed; later ones are drawn
@@ -438,9 +410,11 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
           us[5] = un.nchunks;
           us[6] = un.single;
           us[7] = nd;
+          us[8] = ns;
+          us[9] = 0;
         }
-        us[8 + lane] = e0;
-        if (L::kUnitInts > 8 + 32 + lane) us[8 + 32 + lane] = e1;
+        us[L::kUnitHead + lane] = e0;
+        if (L::kUnitInts > L::kUnitHead + 32 + lane) us[L::kUnitHead + 32 + lane] = e1;
         __syncwarp();
       }
       if (lane == 0) {
@@ -484,7 +458,6 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       // copy on write goes out while the draw is in flight.
       int raw_next = 0;
       if (lane == 0) raw_next = (int)gridDim.x + (int)atomicAdd(sched, 1u);
-      if (ns >= 0) cow_copy(un, nd, ns);
       u = __shfl_sync(0xffffffffu, raw_next, 0);
       load_entries(u, un, e0, e1, nd, ns);
     }
@@ -733,9 +706,48 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       un.nchunks = us[5];
       un.single = us[6] != 0;
       if (un.nchunks == 0) break;  // the producer ran out of work
-      const int32_t *ents = us + 8;
+      const int32_t *ents = us + L::kUnitHead;
       const int tail_end = min(((un.t1 + bs - 1) >> log2_bs) << log2_bs, un.t0 + kPart);
       const uint32_t obuf = trow + 2 * N + (qi & 1) * N;
+      // Copy on write of the unit's newest block (fused step): the source
+      // tile over the destination's, every row but the new one (the MMA warp
+      // stores that).  Nothing in this call reads the destination.  Thread r
+      // takes vectors r, r + 128, ... of the K and V tiles; the first two are
+      // loaded now and stored once the first chunk's weights are out.
+      const int32_t cw_src = us[8], cw_dst = us[7];
+      const int cw_vecs = bs * 16, cw_skip = (un.t1 - 1) & (bs - 1);
+      uint4 cwk[2], cwv[2];
+      if (cw_src >= 0) {
+        const size_t s0 = ((size_t)cw_src * p.Hkv + un.g) * cw_vecs;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int i = r + 128 * j;
+          if (i < cw_vecs) {
+            cwk[j] = static_cast<const uint4 *>(p.k)[s0 + i];
+            cwv[j] = static_cast<const uint4 *>(p.v)[s0 + i];
+          }
+        }
+      }
+      auto cw_store = [&]() {
+        const size_t s0 = ((size_t)cw_src * p.Hkv + un.g) * cw_vecs;
+        const size_t d0 = ((size_t)cw_dst * p.Hkv + un.g) * cw_vecs;
+        uint4 *kd = static_cast<uint4 *>(const_cast<void *>(p.k)) + d0;
+        uint4 *vd = static_cast<uint4 *>(const_cast<void *>(p.v)) + d0;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int i = r + 128 * j;
+          if (i < cw_vecs && (i >> 4) != cw_skip) {
+            kd[i] = cwk[j];
+            vd[i] = cwv[j];
+          }
+        }
+        for (int i = r + 256; i < cw_vecs; i += 128) {  // 32-token blocks: the rest
+          if ((i >> 4) != cw_skip) {
+            kd[i] = static_cast<const uint4 *>(p.k)[s0 + i];
+            vd[i] = static_cast<const uint4 *>(p.v)[s0 + i];
+          }
+        }
+      };
 #pragma unroll
       for (int n = 0; n < G; ++n) {
         m_done[n] = m[n];
@@ -840,6 +852,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
           pend = false;
           if (stop) break;
         }
+        if (ci == 0 && cw_src >= 0) cw_store();
       }
       if (stop) break;
       pend = true;
