@@ -78,3 +78,32 @@ def test_block_size_choice_rule():
     assert bench.choose_block_size(lines, 0.06)["block_size_choice"] == 32
     assert bench.choose_block_size(lines, 0.01)["block_size_choice"] == 8
     assert set(bench.choose_block_size(lines, 0.05)["per_block_size"]) == {"8", "16", "32"}
+
+
+def test_traffic_record_follows_the_kernel_sources(tmp_path, monkeypatch):
+    """The roofline's ncu traffic is reported only while the partition
+    kernel's sources hash to the ones the record was captured on: a record of
+    other sources gives None, and the hash moves when one of those sources
+    does."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.profiled_traffic("no-such-workload") is None
+    # a copy of the kernel sources with records of its own
+    root = tmp_path / "tree"
+    csrc = root / "paged_kv_cache_402_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (root / "profiles").mkdir()
+    for f in ("pa_decode_tc.cuh", "pa_decode_simt.cuh", "pa_device.cuh", "pa_tc.cuh"):
+        (csrc / f).write_bytes(open(os.path.join(ROOT, "paged_kv_cache_402_b200", "csrc", f), "rb").read())
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    h0 = bench.kernel_source_hash()
+    rec = {"kernel_hash": h0, "bytes_per_launch": 123}
+    (root / "profiles" / "traffic.json").write_text(json.dumps({"gqa": rec}))
+    assert bench.profiled_traffic("gqa") == 123
+    (root / "profiles" / "traffic.json").write_text(json.dumps({"gqa": dict(rec, kernel_hash="0" * 16)}))
+    assert bench.profiled_traffic("gqa") is None
+    (root / "profiles" / "traffic.json").write_text(json.dumps({"gqa": rec}))
+    with open(csrc / "pa_decode_tc.cuh", "a") as f:
+        f.write("\n")
+    assert bench.kernel_source_hash() != h0
+    assert bench.profiled_traffic("gqa") is None
