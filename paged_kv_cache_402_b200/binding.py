@@ -61,7 +61,10 @@ def _load() -> ctypes.CDLL:
         raise ImportError(f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_402_b200.build`")
     L = ctypes.CDLL(LIB_PATH)
     vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
-    i32p, i64p = ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64)
+    # host int32 / int64 arrays go in as plain addresses (_i32p / _i64p check
+    # their dtype and layout), which ctypes converts far faster than typed
+    # pointers; ctypes.byref() results are accepted there too
+    i32p, i64p = vp, vp
     cp = ctypes.POINTER(pa_cache_t)
     st = ctypes.c_int
     sigs = {
@@ -136,12 +139,18 @@ def _dev(t: torch.Tensor, what: str, dtype=None) -> int:
     return t.data_ptr()
 
 
-def _i32p(a: np.ndarray):
-    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+def _i32p(a: np.ndarray) -> int:
+    """Address of a C-contiguous int32 host array."""
+    if a.dtype != np.int32 or not a.flags.c_contiguous:
+        raise TypeError("expected a C-contiguous int32 array")
+    return a.ctypes.data
 
 
-def _i64p(a: np.ndarray):
-    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+def _i64p(a: np.ndarray) -> int:
+    """Address of a C-contiguous int64 host array."""
+    if a.dtype != np.int64 or not a.flags.c_contiguous:
+        raise TypeError("expected a C-contiguous int64 array")
+    return a.ctypes.data
 
 
 # --------------------------------------------------------------------------
