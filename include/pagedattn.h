@@ -442,15 +442,32 @@ PA_API pa_status pa_decode_step_prepare(pa_allocator *a, const int32_t *seqs, in
 
 /*
  * The per-sequence form of a decode step's copy pairs, as pa_append_decode
- * takes it: cow_src_host[i] = the source of the pair whose destination is
- * last_blocks_host[i] (sequence i's last block after its append; -1 when it
- * has none), else -1.  PA_ERR_INVALID_ARG when a destination repeats or a
- * pair's destination is no sequence's last block (a pair the one-token step
- * cannot make).
+ * takes it.  Sequence i's last block is the table entry of its newest token,
+ * tables_host[i][(lens_host[i] - 1) / block_size] ("The Block Table Map":
+ * logical block n of a sequence is entry n of its table); cow_src_host[i] is
+ * the source of the pair whose destination is that block, else -1 (also
+ * for lens_host[i] <= 0, a sequence with no block).
+ *   pairs_host   [n_pairs][2] int32 (src, dst), as the allocator made them
+ *   tables_host  [n_seqs][max_blocks] int32, lens_host [n_seqs] int32: the
+ *                step's tables and lengths after its appends
+ * PA_ERR_INVALID_ARG when a destination repeats, when a pair's destination
+ * is no sequence's last block (a pair the one-token step cannot make), or
+ * when a newest token's entry lies past max_blocks.
  */
 PA_API pa_status pa_cow_sources(const int32_t *pairs_host, int32_t n_pairs,
-                                const int32_t *last_blocks_host, int32_t n_seqs,
+                                const int32_t *tables_host, int32_t max_blocks,
+                                const int32_t *lens_host, int32_t n_seqs, int32_t block_size,
                                 int32_t *cow_src_host);
+
+/*
+ * Internal fragmentation of the pool as it stands: the share of allocated
+ * slots (blocks in use x block_size) that hold no token, (allocated - used) /
+ * allocated with the counts of pa_alloc_stats (each physical slot once), 0
+ * when no block is in use.  This is the measure of the learn-ml-visualized
+ * chapter "inference-acceleration-pagedattention-vllm", fragmentation worked
+ * example: waste = allocated - used, taken as a fraction of what is allocated.
+ */
+PA_API pa_status pa_alloc_fragmentation(pa_allocator *a, double *fragmentation);
 
 #ifdef __cplusplus
 }

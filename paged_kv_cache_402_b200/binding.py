@@ -73,7 +73,7 @@ def _load() -> ctypes.CDLL:
         "pa_decode_workspace_size": (sz, [i32, i32, i32, i32]),
         "pa_decode_static_workspace": (st, [vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp]),
         "pa_append_decode": (st, [vp, vp, vp, vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp, sz, vp]),
-        "pa_cow_sources": (st, [i32p, i32, i32p, i32, i32p]),
+        "pa_cow_sources": (st, [i32p, i32, i32p, i32, i32p, i32, i32, i32p]),
         "pa_decode_shared": (st, [vp, vp, vp, vp, cp, vp, i32, vp, i32, i32, i32, f32,
                                   ctypes.POINTER(pa_share_plan_t), vp, vp, sz, vp]),
         "pa_share_plan": (st, [i32p, i32, i32p, i32, i32, i32, i32p, i32p, i32p, i32p]),
@@ -100,6 +100,7 @@ def _load() -> ctypes.CDLL:
         "pa_build_block_tables": (st, [vp, i32p, i32, i32, i32, i32p, i32p]),
         "pa_seqs_max_len": (st, [vp, i32p, i32, i32p, i32p]),
         "pa_alloc_stats": (st, [vp, i64p, i64p, i32p, i32p]),
+        "pa_alloc_fragmentation": (st, [vp, ctypes.POINTER(ctypes.c_double)]),
         "pa_block_refcount": (st, [vp, i32, i32p]),
     }
     for name, (res, args) in sigs.items():
@@ -279,15 +280,17 @@ def pa_append_decode(k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor, 
 def cow_sources(pairs, tables: np.ndarray, lens: np.ndarray, block_size: int,
                 out: np.ndarray | None = None) -> np.ndarray:
     """Host: the per-sequence copy sources pa_append_decode takes, from a
-    step's copy pairs [k, 2] and the host tables / lengths after the append."""
+    step's copy pairs [k, 2] and the host tables / lengths after the append
+    (pa_cow_sources)."""
     pairs = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
-    tables = np.asarray(tables, dtype=np.int32)
-    lens = np.asarray(lens, dtype=np.int32)
+    tables = np.ascontiguousarray(np.asarray(tables, dtype=np.int32))
+    lens = np.ascontiguousarray(np.asarray(lens, dtype=np.int32))
     n = len(lens)
-    col = np.maximum(lens - 1, 0) // int(block_size)
-    last = np.ascontiguousarray(np.where(lens > 0, tables[np.arange(n), col], -1).astype(np.int32))
+    if tables.ndim != 2 or tables.shape[0] != n:
+        raise ValueError("tables must be [n_seqs, max_blocks]")
     res = out if out is not None else np.empty(n, dtype=np.int32)
-    _check(_lib.pa_cow_sources(_i32p(pairs), pairs.shape[0], _i32p(last), n, _i32p(res)), "pa_cow_sources")
+    _check(_lib.pa_cow_sources(_i32p(pairs), pairs.shape[0], _i32p(tables), tables.shape[1], _i32p(lens), n,
+                               int(block_size), _i32p(res)), "pa_cow_sources")
     return res
 
 
@@ -571,11 +574,12 @@ class Allocator:
     def stats(self) -> dict:
         used, alloc = ctypes.c_int64(), ctypes.c_int64()
         free, usedb = ctypes.c_int32(), ctypes.c_int32()
+        frag = ctypes.c_double()
         _check(_lib.pa_alloc_stats(self._h, ctypes.byref(used), ctypes.byref(alloc), ctypes.byref(free),
                                    ctypes.byref(usedb)), "pa_alloc_stats")
-        frag = (alloc.value - used.value) / alloc.value if alloc.value else 0.0
+        _check(_lib.pa_alloc_fragmentation(self._h, ctypes.byref(frag)), "pa_alloc_fragmentation")
         return dict(used_slots=used.value, allocated_slots=alloc.value, free_blocks=free.value,
-                    used_blocks=usedb.value, fragmentation=frag)
+                    used_blocks=usedb.value, fragmentation=frag.value)
 
     def refcount(self, block: int) -> int:
         r = ctypes.c_int32()

@@ -447,10 +447,11 @@ PA_API pa_status pa_decode_step_prepare(pa_allocator *a, const int32_t *seqs, in
 }
 
 PA_API pa_status pa_cow_sources(const int32_t *pairs_host, int32_t n_pairs,
-                                const int32_t *last_blocks_host, int32_t n_seqs,
+                                const int32_t *tables_host, int32_t max_blocks,
+                                const int32_t *lens_host, int32_t n_seqs, int32_t block_size,
                                 int32_t *cow_src_host) {
-  if (n_pairs < 0 || n_seqs < 0 || (n_pairs > 0 && !pairs_host) ||
-      (n_seqs > 0 && (!last_blocks_host || !cow_src_host)))
+  if (n_pairs < 0 || n_seqs < 0 || max_blocks < 0 || block_size <= 0 || (n_pairs > 0 && !pairs_host) ||
+      (n_seqs > 0 && (!tables_host || !lens_host || !cow_src_host)))
     return PA_ERR_INVALID_ARG;
   std::unordered_map<int32_t, int32_t> src_of;  // destination -> source
   src_of.reserve((size_t)n_pairs * 2);
@@ -459,14 +460,27 @@ PA_API pa_status pa_cow_sources(const int32_t *pairs_host, int32_t n_pairs,
   int32_t matched = 0;
   for (int32_t i = 0; i < n_seqs; ++i) {
     cow_src_host[i] = -1;
-    if (last_blocks_host[i] < 0) continue;
-    auto it = src_of.find(last_blocks_host[i]);
+    const int32_t len = lens_host[i];
+    if (len <= 0) continue;  // no last block
+    const int64_t col = (int64_t)(len - 1) / block_size;  // the table entry of the newest token
+    if (col >= max_blocks) return PA_ERR_INVALID_ARG;
+    auto it = src_of.find(tables_host[(int64_t)i * max_blocks + col]);
     if (it == src_of.end()) continue;
     cow_src_host[i] = it->second;
     src_of.erase(it);  // one writer per destination
     ++matched;
   }
   return matched == n_pairs ? PA_OK : PA_ERR_INVALID_ARG;
+}
+
+PA_API pa_status pa_alloc_fragmentation(pa_allocator *a, double *fragmentation) {
+  if (!a || !fragmentation) return PA_ERR_INVALID_ARG;
+  int64_t used = 0, allocated = 0;
+  const pa_status s = pa_alloc_stats(a, &used, &allocated, nullptr, nullptr);
+  if (s != PA_OK) return s;
+  // waste over what is held: (allocated - used) / allocated
+  *fragmentation = allocated > 0 ? (double)(allocated - used) / (double)allocated : 0.0;
+  return PA_OK;
 }
 
 }  // extern "C"

@@ -136,6 +136,48 @@ def test_cow_sources_of_an_allocator_step():
     assert [int(tables[i, 1]) for i in range(3)] == [int(p[1]) for p in pairs]
 
 
+def test_cow_sources_walks_the_table_in_c():
+    """The library finds each sequence's last block itself: the newest
+    token's table entry, (len - 1) / bs; a length of 0 has none, and a
+    newest token past the table's width is an argument error."""
+    L = pa.lib()
+    tables = np.array([[4, 9, -1], [4, 7, -1], [5, 6, 2], [8, -1, -1]], np.int32)
+    lens = np.array([20, 17, 33, 0], np.int32)
+    pairs = np.array([[3, 7], [1, 2]], np.int32)
+    out = np.full(4, 99, np.int32)
+    assert L.pa_cow_sources(pairs.ctypes.data, 2, tables.ctypes.data, 3, lens.ctypes.data, 4, 16,
+                            out.ctypes.data) == pa.PA_OK
+    assert out.tolist() == [-1, 3, 1, -1]
+    assert L.pa_cow_sources(pairs.ctypes.data, 2, tables.ctypes.data, 3, lens.ctypes.data, 4, 8,
+                            out.ctypes.data) == pa.PA_ERR_INVALID_ARG   # 33 tokens need entry 4 at bs 8
+    assert L.pa_cow_sources(pairs.ctypes.data, 1, tables.ctypes.data, 3, lens.ctypes.data, 4, 0,
+                            out.ctypes.data) == pa.PA_ERR_INVALID_ARG
+
+
+def test_fragmentation_of_a_shared_step_by_hand():
+    """The C++ allocator's fragmentation on the hand-counted case of the
+    oracle's pins (learn-ml-visualized worked example's measure, waste over
+    allocated): a root of 6 tokens at block size 4 forked twice holds 8
+    slots with 6 used (0.25); after one token each (two copies on write) 16
+    slots with 13 used (3/16)."""
+    A = pa.Allocator(32, 4, [10, 11, 12, 13] + [b for b in range(32) if b not in (10, 11, 12, 13)])
+    root = A.new_seq()
+    A.append(root, 6)
+    kids = [A.fork(root), A.fork(root)]
+    st = A.stats()
+    assert (st["allocated_slots"], st["used_slots"], st["fragmentation"]) == (8, 6, 0.25)
+    _, pairs = A.batch_append([root] + kids, [1, 1, 1])
+    assert pairs.tolist() == [[11, 12], [11, 13]]
+    st = A.stats()
+    assert (st["allocated_slots"], st["used_slots"], st["fragmentation"]) == (16, 13, 3 / 16)
+    frag = ctypes.c_double(-1.0)
+    assert pa.lib().pa_alloc_fragmentation(A._h, ctypes.byref(frag)) == pa.PA_OK
+    assert frag.value == 3 / 16
+    empty = pa.Allocator(8, 4)
+    assert empty.stats()["fragmentation"] == 0.0
+    assert pa.lib().pa_alloc_fragmentation(None, ctypes.byref(frag)) == pa.PA_ERR_INVALID_ARG
+
+
 def test_workspace_size():
     ws = pa.pa_decode_workspace_size
     assert ws(4, 8, 512, 128) == 0

@@ -178,3 +178,72 @@ def test_append_and_copy_bit_exact_and_padding_skipped():
     oracle.copy_blocks(k, v, [(1, 4)])
     assert np.array_equal(k[4], k[1]) and np.array_equal(v[4], v[1])
     assert np.array_equal(k[0], k0[0])
+
+
+# ------------------------------------------------------------------ usage under sharing
+#
+# The fragmentation measure is the one of the learn-ml-visualized chapter
+# "inference-acceleration-pagedattention-vllm" (fragmentation worked example):
+# waste = allocated - used, fragmentation = waste / allocated.  With shared
+# blocks the allocation is physical: a block in use counts once however many
+# tables hold it, and its tokens once.  The counts below are worked out by
+# hand, not by the model.
+
+
+def test_usage_reproduces_the_paged_worked_example():
+    """Lengths 1, 4, 2 grown through the allocator in pages of 2: 8 slots held,
+    7 used, the single wasted slot in the length-1 sequence's half-empty page."""
+    A = oracle.AllocatorModel(16, 2)
+    for L in (1, 4, 2):
+        A.append(A.new_seq(), L)
+    u = A.usage()
+    assert (u.allocated, u.used, u.wasted) == (8, 7, 1)
+    assert u.fragmentation == 1 / 8
+
+
+def test_usage_of_a_shared_partial_block_by_hand():
+    """Block size 4.  A root of 6 tokens holds block 10 (4 tokens) and block
+    11 (2 tokens); two forks share both (reference count 3).  Physically:
+    8 slots held, 6 used.  One token is then appended to the root, the first
+    fork and the second fork, in that order: the root copies 11 into 12, the
+    first fork copies 11 into 13, and the second fork, by then the only
+    holder of 11, writes into it in place.  Physically: 10 (4 tokens, shared
+    by three), 11, 12 and 13 (3 tokens each): 16 slots held, 13 used, 3
+    wasted."""
+    A = oracle.AllocatorModel(32, 4, [10, 11, 12, 13] + [b for b in range(32) if b not in (10, 11, 12, 13)])
+    root = A.new_seq()
+    A.append(root, 6)
+    kids = [A.fork(root), A.fork(root)]
+    u = A.usage()
+    assert (u.allocated, u.used) == (8, 6)
+    assert u.fragmentation == 2 / 8
+    slots, cows = A.batch_append([root] + kids, [1, 1, 1])
+    assert cows == [(11, 12), (11, 13)]
+    assert slots == [12 * 4 + 2, 13 * 4 + 2, 11 * 4 + 2]
+    u = A.usage()
+    assert (u.allocated, u.used, u.wasted) == (16, 13, 3)
+    assert u.fragmentation == 3 / 16
+
+
+def test_usage_of_full_shared_blocks_by_hand():
+    """Block size 4.  A root of 8 tokens fills blocks 10 and 11; two forks
+    share them.  One token appended to each of the three takes a fresh
+    block each (12, 13, 14; full blocks are never copied).  Physically: 10
+    and 11 (4 tokens each, counted once), 12, 13, 14 (1 token each): 20
+    slots held, 11 used.  Freeing the root then releases only its own block
+    12: 16 held, 10 used."""
+    A = oracle.AllocatorModel(32, 4, list(range(10, 32)) + list(range(10)))
+    root = A.new_seq()
+    A.append(root, 8)
+    kids = [A.fork(root), A.fork(root)]
+    u = A.usage()
+    assert (u.allocated, u.used) == (8, 8)
+    _, cows = A.batch_append([root] + kids, [1, 1, 1])
+    assert cows == []
+    assert [A.block_table(s) for s in [root] + kids] == [[10, 11, 12], [10, 11, 13], [10, 11, 14]]
+    u = A.usage()
+    assert (u.allocated, u.used, u.wasted) == (20, 11, 9)
+    A.free_seq(root)
+    u = A.usage()
+    assert (u.allocated, u.used) == (16, 10)
+    assert A.ref[10] == 2 and A.ref[12] == 0

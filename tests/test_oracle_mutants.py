@@ -47,6 +47,45 @@ PIN_TESTS = [
 ]
 
 
+def _usage_per_sharer(self):
+    """A plausible mistake: every table's blocks counted, so a block shared
+    by k sequences is held k times and its tokens used k times."""
+    bs = self.block_size
+    return oracle.Usage(allocated=bs * sum(len(t) for t in self.tables.values()), used=sum(self.lens.values()))
+
+
+def _usage_tokens_per_sharer(self):
+    """A plausible mistake: physical blocks counted once, but every
+    sequence's tokens counted, so shared tokens are used several times."""
+    bs = self.block_size
+    blocks = {b for t in self.tables.values() for b in t}
+    return oracle.Usage(allocated=bs * len(blocks), used=sum(self.lens.values()))
+
+
+USAGE_MUTANTS = {"usage-per-sharer": _usage_per_sharer, "usage-tokens-per-sharer": _usage_tokens_per_sharer}
+
+
+def _usage_pins():
+    from tests import test_oracle_allocator as alloc_pins
+    return [alloc_pins.test_usage_reproduces_the_paged_worked_example,
+            alloc_pins.test_usage_of_a_shared_partial_block_by_hand,
+            alloc_pins.test_usage_of_full_shared_blocks_by_hand]
+
+
+@pytest.mark.parametrize("name", sorted(USAGE_MUTANTS))
+def test_usage_mutant_is_caught(name, monkeypatch):
+    for t in _usage_pins():
+        t()  # the model as it stands passes every pin
+    monkeypatch.setattr(oracle.AllocatorModel, "usage", USAGE_MUTANTS[name])
+    caught = 0
+    for t in _usage_pins():
+        try:
+            t()
+        except AssertionError:
+            caught += 1
+    assert caught > 0, f"no pin fails on mutant {name}"
+
+
 def _build_mutant(tmp_path, name, old, new):
     src = open(obuild.SRC).read()
     assert src.count(old) == 1, f"mutation site for {name} not unique"
