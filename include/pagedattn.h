@@ -264,9 +264,13 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
  *  - Sizes whose scratch, pa_decode_workspace_size(num_seqs, num_q_heads,
  *    max_context_len, head_dim), exceeds PA_STATIC_WORKSPACE_BYTES are
  *    rejected with PA_ERR_TOO_SMALL before any launch.
- *  - The first call on a device looks up that device's copy of the array
- *    (with the device current); make that first call before any stream
- *    capture.  Later calls on the device reuse the address.
+ *  - The first call in a CUDA context looks up that context's copy of the
+ *    array (with the context current, the runtime's current device's
+ *    primary context unless the caller bound another); make that first call
+ *    before any stream capture.  Later calls in the same context reuse the
+ *    address.  The address is tied to the context it was looked up in: a
+ *    context created later (another context of the device, or the primary
+ *    context again after cudaDeviceReset) gets a lookup of its own.
  *  - Every call on a device shares the one array and it keeps the last call's
  *    contents.  Nothing in it needs to start at zero: each entry the merge
  *    step reads is written earlier in the same call.  Calls whose kernels

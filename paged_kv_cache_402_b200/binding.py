@@ -154,6 +154,15 @@ def _i64p(a: np.ndarray) -> int:
     return a.ctypes.data
 
 
+def _check_q_out(q: torch.Tensor, out, cache) -> None:
+    """q must be [B, Hq, head_dim] of the cache; a given out must have q's
+    shape (the library writes B x Hq x head_dim elements there)."""
+    if q.dim() != 3 or q.shape[2] != cache.head_dim:
+        raise ValueError(f"q must be [B, Hq, {cache.head_dim}] (the cache's head_dim), got {list(q.shape)}")
+    if out is not None and tuple(out.shape) != tuple(q.shape):
+        raise ValueError(f"out must have q's shape {list(q.shape)}, got {list(out.shape)}")
+
+
 # --------------------------------------------------------------------------
 # the pools
 
@@ -223,9 +232,8 @@ def pa_decode(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor, conte
               max_context_len: int, scale: float, out: torch.Tensor | None = None,
               workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Paged decode attention; returns out [B, Hq, D] in the cache dtype."""
+    _check_q_out(q, out, cache)
     B, Hq, D = q.shape
-    if D != cache.head_dim:
-        raise ValueError("head_dim mismatch")
     if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
         raise ValueError("block_tables must be [B, max_blocks] and context_lens [B]")
     if out is None:
@@ -251,9 +259,8 @@ def pa_append_decode(k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor, 
     no copies), the append of b's newest token (k_new, v_new [B, Hkv, D],
     written at position context_lens[b] - 1 through b's block table) and the
     decode.  Returns out [B, Hq, D]."""
+    _check_q_out(q, out, cache)
     B, Hq, D = q.shape
-    if D != cache.head_dim:
-        raise ValueError("head_dim mismatch")
     if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
         raise ValueError("block_tables must be [B, max_blocks] and context_lens [B]")
     row_shape = (B, cache.num_kv_heads, D)
@@ -359,9 +366,8 @@ def pa_decode_shared(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor
                      workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """pa_decode, or pa_append_decode when k_new / v_new are given, with the
     partitions a plan's groups share read once for all their members."""
+    _check_q_out(q, out, cache)
     B, Hq, D = q.shape
-    if D != cache.head_dim:
-        raise ValueError("head_dim mismatch")
     if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
         raise ValueError("block_tables must be [B, max_blocks] and context_lens [B]")
     if (k_new is None) != (v_new is None):
@@ -393,10 +399,9 @@ def pa_prefill(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor, cont
     """Paged chunked-prefill attention: the last query_starts[b+1] -
     query_starts[b] tokens of sequence b (already in the cache) attend
     causally to the sequence; q and out are [total, Hq, 128] bf16."""
+    _check_q_out(q, out, cache)
     T, Hq, D = q.shape
     B = context_lens.shape[0]
-    if D != cache.head_dim:
-        raise ValueError("head_dim mismatch")
     if block_tables.dim() != 2 or block_tables.shape[0] != B or query_starts.shape != (B + 1,):
         raise ValueError("block_tables must be [B, max_blocks] and query_starts [B + 1]")
     if out is None:
@@ -418,6 +423,7 @@ def pa_decode_static_workspace(q: torch.Tensor, cache: KVCache, block_tables: to
     """pa_decode with the library's fixed scratch array instead of a
     workspace (for callers that cannot allocate device memory); raises
     PagedAttnError (buffer too small) past PA_STATIC_WORKSPACE_BYTES."""
+    _check_q_out(q, out, cache)
     B, Hq, D = q.shape
     if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
         raise ValueError("block_tables must be [B, max_blocks] and context_lens [B]")

@@ -74,7 +74,8 @@ pa_status launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
 }
 
 inline int32_t max_parts_for(int32_t max_context_len) {
-  return (max_context_len + pa::kPart - 1) / pa::kPart;
+  // in 64 bits: a length near INT32_MAX must not wrap before the division
+  return (int32_t)(((int64_t)max_context_len + pa::kPart - 1) / pa::kPart);
 }
 
 inline size_t round16(size_t x) { return (x + 15) & ~(size_t)15; }
@@ -705,8 +706,8 @@ PA_API pa_status pa_decode_shared(const void *k_new, const void *v_new, const in
 // file-scope array instead of caller memory, for callers that cannot
 // allocate device memory.  Host code must not use the array's name as a
 // device address (it is a host-side stand-in); the device address comes from
-// cudaGetSymbolAddress, looked up once per device with that device current
-// and kept below.
+// cudaGetSymbolAddress, looked up once per CUDA context with that context
+// current and kept below.
 
 }  // extern "C"
 
@@ -714,21 +715,58 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_static_workspace[PA_STATIC_WORKSPACE_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_static_ws_mutex;
-void *g_static_ws_ptr[kMaxDevices] = {};
+// The array's device address differs between CUDA contexts (each context
+// loads the module on its own), so the address looked up is kept per
+// context, keyed by the context's unique id (cuCtxGetId: ids are never
+// reused within a process, unlike context handles or device ordinals).  A
+// context that is destroyed and re-created, e.g. after cudaDeviceReset,
+// gets a new id and so a fresh lookup.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
 
-// Device address of this device's copy of g_static_workspace, or nullptr.
-void *static_workspace_for_current_device() {
+template <typename Fn>
+Fn driver_entry(const char *name) {
+  void *f = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &f, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(f);
+}
+
+constexpr int kStaticWsEntries = 64;
+struct StaticWsEntry {
+  unsigned long long ctx_id;
+  void *ptr;
+};
+std::mutex g_static_ws_mutex;
+StaticWsEntry g_static_ws[kStaticWsEntries] = {};
+int g_static_ws_next = 0;  // the slot a new context takes (round-robin once all are used)
+
+// Device address of the current context's copy of g_static_workspace, or
+// nullptr (no context could be made current, or a lookup failed).
+void *static_workspace_for_current_context() {
+  static const CtxGetCurrentFn get_current = driver_entry<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_entry<CtxGetIdFn>("cuCtxGetId");
+  if (!get_current || !get_id) return nullptr;
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
-  if (!g_static_ws_ptr[dev]) {
-    void *ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_static_workspace) != cudaSuccess || !ptr) return nullptr;
-    g_static_ws_ptr[dev] = ptr;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) {
+    // no context bound to this thread yet: the runtime makes the current
+    // device's primary context current (cudaSetDevice initialises it), then
+    // ask again
+    if (cudaSetDevice(dev) != cudaSuccess || get_current(&ctx) != CUDA_SUCCESS || !ctx) return nullptr;
   }
-  return g_static_ws_ptr[dev];
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return nullptr;
+  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+  for (const StaticWsEntry &e : g_static_ws)
+    if (e.ptr && e.ctx_id == id) return e.ptr;
+  void *ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_static_workspace) != cudaSuccess || !ptr) return nullptr;
+  g_static_ws[g_static_ws_next] = StaticWsEntry{id, ptr};
+  g_static_ws_next = (g_static_ws_next + 1) % kStaticWsEntries;
+  return ptr;
 }
 
 }  // namespace
@@ -743,14 +781,16 @@ PA_API pa_status pa_decode_static_workspace(const void *q, const pa_cache_t *cac
                                             float scale, void *out, void *stream) {
   pa_status s = check_cache(cache);
   if (s != PA_OK) return s;
+  // the range checks pa_decode makes, before the scratch size is computed
   if (num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0 || cache->head_dim <= 0)
     return PA_ERR_INVALID_ARG;
+  if (num_seqs > 65535 || max_context_len > INT32_MAX - pa::kPart) return PA_ERR_INVALID_ARG;
   const size_t need =
       num_seqs > 0 ? workspace_bytes_for(num_seqs, num_q_heads, max_context_len, cache->head_dim) : 0;
   if (need > (size_t)PA_STATIC_WORKSPACE_BYTES) return PA_ERR_TOO_SMALL;
   void *ws = nullptr;
   if (need > 0) {
-    ws = static_workspace_for_current_device();
+    ws = static_workspace_for_current_context();
     if (!ws) return PA_ERR_CUDA;
   }
   return pa_decode(q, cache, block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads,

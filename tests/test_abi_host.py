@@ -178,6 +178,33 @@ def test_fragmentation_of_a_shared_step_by_hand():
     assert pa.lib().pa_alloc_fragmentation(None, ctypes.byref(frag)) == pa.PA_ERR_INVALID_ARG
 
 
+def test_wrappers_check_q_and_out_before_any_launch():
+    """The Python wrappers refuse a q whose head_dim is not the cache's, or an
+    out of another shape, before the library is called (the C side writes
+    B x Hq x head_dim elements of out)."""
+    import types
+    import torch
+    cache = types.SimpleNamespace(head_dim=128, num_kv_heads=2, dtype=torch.bfloat16)
+    q64 = torch.zeros(2, 4, 64, dtype=torch.bfloat16)
+    q = torch.zeros(2, 4, 128, dtype=torch.bfloat16)
+    t = torch.zeros(2, 4, dtype=torch.int32)
+    n = torch.zeros(2, dtype=torch.int32)
+    for fn in (pa.pa_decode, pa.pa_decode_static_workspace, pa.pa_decode_shared):
+        with pytest.raises(ValueError, match="head_dim"):
+            fn(q64, cache, t, n, 16, 0.1)
+        with pytest.raises(ValueError, match="out must"):
+            fn(q, cache, t, n, 16, 0.1, out=torch.zeros(1, 4, 128, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="head_dim"):
+        pa.pa_append_decode(q, q, q64, cache, t, n, 16, 0.1)
+
+
+def test_workspace_size_of_huge_lengths():
+    """A length near INT32_MAX sizes its partitions without wrapping."""
+    ws = pa.pa_decode_workspace_size(1, 1, 2**31 - 1, 128)
+    parts = -(-(2**31 - 1) // 512)
+    assert ws == 2 * ((parts * 4 + 15) // 16 * 16) + parts * 128 * 4
+
+
 def test_workspace_size():
     ws = pa.pa_decode_workspace_size
     assert ws(4, 8, 512, 128) == 0
