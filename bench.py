@@ -83,10 +83,12 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """Per-launch DRAM traffic (bytes) recorded by an ncu capture of the
-    current decode kernel, scaled to the workload, or None when no capture
-    matches the current sources."""
+def profiled_traffic(workload: str, algo_bytes_per_launch: float):
+    """Per-launch DRAM traffic (read + write bytes) of the step's kernels as an
+    ncu capture of the current decode sources measured it, applied to this
+    run's launches: the captured traffic / algorithmic-bytes ratio times this
+    run's mean algorithmic bytes per launch (traffic grows in proportion to
+    the K/V read).  None when no capture matches the current sources."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -96,12 +98,16 @@ def profiled_traffic(workload: str):
     rec = d.get(workload)
     if not rec or rec.get("kernel_hash") != kernel_source_hash():
         return None
-    return rec.get("bytes_per_launch")
+    cap = rec["captured_launch"]
+    ratio = (cap["dram_read_bytes"] + cap["dram_write_bytes"]) / cap["algorithmic_bytes"]
+    return int(round(ratio * algo_bytes_per_launch))
 
 
 class ClockSampler:
-    """SM clock and throttle reasons sampled through NVML by a thread about
-    every millisecond while the timed region runs (the region is short)."""
+    """SM clock and throttle reasons sampled through NVML by a thread as fast
+    as NVML answers (every ~0.1 ms) while the timed region runs: the region
+    is K steps of a few hundred microseconds each, so a slower rate would
+    leave only a handful of samples."""
 
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4}
@@ -139,7 +145,7 @@ class ClockSampler:
                 except Exception as e:
                     self.error = str(e)
                     return
-                time.sleep(0.001)
+                time.sleep(0.0001)
 
         self._thread = threading.Thread(target=run, daemon=True)
         self._thread.start()
@@ -157,6 +163,39 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [self.error]}
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+
+
+def bandwidth_probes(dev, nbytes: int = 4 << 30, reps: int = 6):
+    """HBM bandwidth measured in this job, outside the timed region, on a
+    4 GiB buffer (32x the L2): a read-only stream (torch's sum of float32
+    values: every byte read once, nothing written but the scalar) and a copy
+    (read + write bytes of copy_ into a second buffer).  Best of three runs
+    of `reps` launches each, CUDA events on the current stream.  Returns
+    (read GB/s, copy GB/s)."""
+    x = torch.ones(nbytes // 4, dtype=torch.float32, device=dev)
+    y = torch.empty_like(x)
+    acc = torch.empty((), dtype=torch.float32, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def best(fn, bytes_per_rep):
+        for _ in range(2):
+            fn()
+        out = 0.0
+        for _ in range(3):
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(reps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            out = max(out, reps * bytes_per_rep / (e0.elapsed_time(e1) / 1e3) / 1e9)
+        return out
+
+    read = best(lambda: torch.sum(x, dtype=torch.float32, out=acc), nbytes)
+    copy = best(lambda: y.copy_(x), 2 * nbytes)
+    del x, y
+    torch.cuda.empty_cache()
+    return read, copy
 
 
 # ----------------------------------------------------------------- workload
@@ -473,6 +512,7 @@ def run_ours(args, rank: int, world: int, dev):
 
     # end to end through the public API with pinned host buffers
     e2e = run_e2e(args, insts, wl, dev, stream)
+    read_gbs, copy_gbs = bandwidth_probes(dev)
 
     ms_all, gb_all, tok_all, e2e_value = aggregate_ranks(world, ms, kv_bytes / 1e9, float(args.steps * wl["B"]),
                                                          e2e["seconds"], e2e["kv_gb"], dev)
@@ -513,6 +553,10 @@ def run_ours(args, rank: int, world: int, dev):
         "copy_pairs_per_step": round(pairs / args.steps, 2),
         "kv_frac_of_hbm_peak": round(gb_all / (ms_all / 1e3) / peak, 4),
         "kv_frac_of_8tbs_nominal": round(gb_all / (ms_all / 1e3) / NOMINAL_HBM_GBS, 4),
+        "kv_frac_of_read_peak": round(gb_all / (ms_all / 1e3) / (read_gbs * world), 4),
+        "probes": {"read_gbs": round(read_gbs, 1), "copy_gbs": round(copy_gbs, 1),
+                   "how": "this job, after the timed region: torch sum (read-only) and copy_ over 4 GiB, "
+                          "best of 3 x 6 launches"},
         "host_alloc_us_per_step": round(host_alloc_us, 2),
         "roofline": {"bound": "hbm",
                      "kernel": ("pa_decode (partition + LSE reduce)" if args.unfused else
@@ -522,7 +566,7 @@ def run_ours(args, rank: int, world: int, dev):
                                 " + LSE reduce)"),
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
-                     "traffic": profiled_traffic(args.workload),
+                     "traffic": profiled_traffic(args.workload, statistics.mean(algo_bytes)),
                      "decode_us": round(dec_avg_s * 1e6, 2),
                      "duration_from": ("CUDA events around each decode call in the timed graph" if per_step_events
                                        else "CUDA events around the K-step timed region / K (one call per step)"),
@@ -935,35 +979,72 @@ def run_trace(args, dev):
 # ----------------------------------------------------------------- CPU oracle
 
 
-def oracle_sample(wl, seed: int, budget_s: float, min_s: float):
-    """Times the float64 oracle on the host over whole (sequence, kv head)
-    groups of one batch of the workload until about budget_s of work.
-    Returns (GB/s of KV processed, seconds, threads, description)."""
-    import oracle
+ORACLE_CASE_BYTES = 768 << 20  # K/V the host-side case of the oracle holds at most
+
+
+def oracle_case(wl, seed: int):
+    """The oracle's host-side case: the workload's batch (its lengths, +1 for
+    the step's appended token), cut to its first sequences when the whole
+    batch would hold more than ORACLE_CASE_BYTES of K/V (the long-context
+    batch holds 2.7 GB).  Returns (case, lengths, description of the cut)."""
     from paged_kv_cache_402_b200 import synth
 
     B, Hq, Hkv, D, bs = wl["B"], wl["Hq"], wl["Hkv"], wl["D"], wl["bs"]
     lens = wl["lengths"](seed) + 1
-    case = synth.random_case(seed, B=B, Hq=Hq, Hkv=Hkv, D=D, bs=bs, lens=lens, dtype=torch.bfloat16, sentinel=False)
+    row = 2 * Hkv * D * 2
+    n = 1
+    while n < B and int(lens[:n + 1].astype(np.int64).sum()) * row <= ORACLE_CASE_BYTES:
+        n += 1
+    lens = lens[:n]
+    case = synth.random_case(seed, B=n, Hq=Hq, Hkv=Hkv, D=D, bs=bs, lens=lens, dtype=torch.bfloat16,
+                             sentinel=False, pool_factor=1.0 if n < B else 2.0)
+    cut = "the whole batch" if n == B else f"its first {n} of {B} sequences"
+    return case, lens, cut
+
+
+def _oracle_rows(order, start, count, Hkv, G):
+    chunk = [int(order[(start + i) % len(order)]) for i in range(count)]
+    return chunk, [(u // Hkv, (u % Hkv) * G + gi) for u in chunk for gi in range(G)]
+
+
+def oracle_sample(wl, seed: int, budget_s: float, min_s: float, threads: int | None = None):
+    """Times the float64 oracle on the host over whole (sequence, kv head)
+    groups of one batch of the workload until about budget_s of work, on
+    `threads` OpenMP threads (all of them by default).  Returns (GB/s of KV
+    processed, seconds, threads, description)."""
+    import oracle
+
+    Hq, Hkv, D = wl["Hq"], wl["Hkv"], wl["D"]
+    case, lens, cut = oracle_case(wl, seed)
     G = Hq // Hkv
-    order = synth.rng(seed + 9).permutation(B * Hkv)
-    threads = oracle.max_threads()
-    done_bytes, t_total, groups = 0, 0.0, 0
-    i = 0
-    while t_total < budget_s:
-        chunk = order[i % len(order): i % len(order) + max(1, 2 * threads)]
-        i += len(chunk)
-        rows = [(int(u) // Hkv, (int(u) % Hkv) * G + gi) for u in chunk for gi in range(G)]
-        t0 = time.perf_counter()
-        oracle.decode(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens, case.scale, rows=rows)
-        t_total += time.perf_counter() - t0
-        done_bytes += sum(int(lens[int(u) // Hkv]) * 2 * D * 2 for u in chunk)
-        groups += len(chunk)
-        if t_total >= min_s and groups >= len(order):
-            break
-    desc = (f"{groups} (sequence, kv head) groups ({groups * G} query rows) of one batch of the workload, "
-            f"{t_total:.1f} s of oracle time")
-    return done_bytes / 1e9 / t_total, t_total, threads, desc
+    order = synth_rng(seed + 9).permutation(len(lens) * Hkv)
+    prev = oracle.max_threads()
+    if threads is not None:
+        oracle.set_threads(threads)
+    used = oracle.max_threads()
+    try:
+        done_bytes, t_total, groups, pos = 0, 0.0, 0, 0
+        while t_total < budget_s:
+            chunk, rows = _oracle_rows(order, pos, min(len(order), max(1, 2 * used)), Hkv, G)
+            pos += len(chunk)
+            t0 = time.perf_counter()
+            oracle.decode(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens, case.scale,
+                          rows=rows)
+            t_total += time.perf_counter() - t0
+            done_bytes += sum(int(lens[u // Hkv]) * 2 * D * 2 for u in chunk)
+            groups += len(chunk)
+            if t_total >= min_s and groups >= len(order):
+                break
+    finally:
+        oracle.set_threads(prev)
+    desc = (f"{groups} (sequence, kv head) groups ({groups * G} query rows) of {cut} of one batch of the "
+            f"workload, {t_total:.1f} s of oracle time on {used} thread(s)")
+    return done_bytes / 1e9 / t_total, t_total, used, desc
+
+
+def synth_rng(seed):
+    from paged_kv_cache_402_b200 import synth
+    return synth.rng(seed)
 
 
 def run_reference(args):
@@ -971,22 +1052,21 @@ def run_reference(args):
     each step a bounded sample of the workload (whole (sequence, kv head)
     groups of one batch, eight per oracle thread, taken round-robin)."""
     import oracle
-    from paged_kv_cache_402_b200 import synth
 
-    wl = WORKLOADS[args.workload]
-    B, Hq, Hkv, D, bs = wl["B"], wl["Hq"], wl["Hkv"], wl["D"], wl["bs"]
+    wl = WORKLOADS[args.workload] if args.workload in WORKLOADS else WORKLOADS["long-context"]
+    if "lengths" not in wl:
+        wl = WORKLOADS["long-context"]
+    Hq, Hkv, D = wl["Hq"], wl["Hkv"], wl["D"]
     G = Hq // Hkv
-    lens = wl["lengths"](1) + 1
-    case = synth.random_case(1, B=B, Hq=Hq, Hkv=Hkv, D=D, bs=bs, lens=lens, dtype=torch.bfloat16, sentinel=False)
-    order = synth.rng(10).permutation(B * Hkv)
+    case, lens, cut = oracle_case(wl, 1)
+    order = synth_rng(10).permutation(len(lens) * Hkv)
     threads = oracle.max_threads()
-    per_step = min(8 * threads, B * Hkv)
+    per_step = min(8 * threads, len(order))
     pos = 0
     total_bytes, total_s, groups = 0, 0.0, 0
     for s in range(args.warmup + args.steps):
-        chunk = [int(order[(pos + i) % len(order)]) for i in range(per_step)]
+        chunk, rows = _oracle_rows(order, pos, per_step, Hkv, G)
         pos += per_step
-        rows = [(u // Hkv, (u % Hkv) * G + gi) for u in chunk for gi in range(G)]
         t0 = time.perf_counter()
         oracle.decode(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens, case.scale, rows=rows)
         dt = time.perf_counter() - t0
@@ -997,7 +1077,7 @@ def run_reference(args):
     gbs = total_bytes / 1e9 / total_s
     seq_bytes = float(np.mean(lens)) * 2 * Hkv * D * 2
     desc = (f"{args.steps} steps of {per_step} (sequence, kv head) groups ({per_step * G} query rows) each, "
-            f"round-robin over one batch of the workload; {total_s:.1f} s timed")
+            f"round-robin over {cut} of one batch of the workload; {total_s:.1f} s timed")
     return {
         "impl": "reference",
         "metric": METRIC,
@@ -1029,7 +1109,7 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["trace", "prefill"], default="gqa")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["trace", "prefill"], default="long-context")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rotate", type=int, default=0, help="batch instances to rotate (0: the workload's default)")
@@ -1084,6 +1164,10 @@ def main():
             gbs, secs, threads, desc = oracle_sample(wl, seed=1, budget_s=args.cpu_budget, min_s=args.cpu_budget)
             line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                                     "sample": desc}
+            # the same oracle on one host core, beside the all-core figure
+            gbs1, _, _, desc1 = oracle_sample(wl, seed=1, budget_s=args.cpu_budget / 4, min_s=0.0, threads=1)
+            line["cpu_baseline"]["single_core"] = {"value": round(gbs1, 4), "unit": "GB/s", "cores": 1,
+                                                   "sample": desc1}
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

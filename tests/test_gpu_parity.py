@@ -389,105 +389,3 @@ def test_bf16_device_errors(cuda_device):
     assert torch.equal(out[1].float().cpu(), torch.zeros(8, 128))
     assert_attn_close(out[[0, 2]], ref[[0, 2]], torch.bfloat16)
     assert pa.pa_read_device_error() == 0
-
-
-# ------------------------------------------------------------- full-size sampled checks
-
-
-def _sampled_check(case_dev, q_host, tables_np, lens_np, out, rows, scale, kv_heads):
-    """Oracle on sampled (b, h) rows: the blocks those sequences use are
-    copied from the device pool (their contents were drawn by torch, not
-    written by this library's kernels) into a compact host pool with a
-    renumbered table."""
-    k_cache, v_cache = case_dev
-    Hq = out.shape[1]
-    G = Hq // kv_heads
-    bs = k_cache.shape[2]
-    seqs = sorted({b for b, _ in rows})
-    got = out.float().cpu().double().numpy()
-    for b in seqs:
-        nb = -(-int(lens_np[b]) // bs)
-        blocks = torch.as_tensor(tables_np[b, :nb].astype(np.int64), device=k_cache.device)
-        kc = k_cache.index_select(0, blocks).cpu()
-        vc = v_cache.index_select(0, blocks).cpu()
-        hs = [h for bb, h in rows if bb == b]
-        q1 = q_host[b:b + 1]
-        ref = oracle.decode(q1, kc, vc, np.arange(nb, dtype=np.int32)[None, :], np.array([lens_np[b]], np.int32),
-                            scale, rows=[(0, h) for h in hs])
-        for i, h in enumerate(hs):
-            g = got[b, h]
-            bound = BF16_ATOL + BF16_RTOL * np.abs(ref[i])
-            assert (np.abs(g - ref[i]) <= bound).all(), f"row ({b}, {h})"
-
-
-
-def test_long_context_full_size_sampled(cuda_device):
-    """8 sequences of 32768..131072 tokens, 32 query / 8 kv heads, blocks
-    scattered over an 80 GiB K+V pool (the launch the long-context benchmark
-    times): sampled rows against the oracle, every output finite."""
-    B, Hq, Hkv, D, bs = 8, 32, 8, 128, 16
-    NB = 80 * 2**30 // (2 * Hkv * bs * D * 2)
-    lens = synth.long_context_lengths(4)
-    tables = synth.scattered_blocks(5, lens, bs, NB)
-    used = np.unique(tables[tables >= 0])
-    k = torch.empty(NB, Hkv, bs, D, dtype=torch.bfloat16, device=cuda_device)
-    v = torch.empty_like(k)
-    idx = torch.as_tensor(used.astype(np.int64), device=cuda_device)
-    for i in range(0, len(idx), 65536):
-        part = idx[i:i + 65536]
-        k.index_copy_(0, part, synth.normal((len(part), Hkv, bs, D), torch.bfloat16, 100 + i, device=cuda_device))
-        v.index_copy_(0, part, synth.normal((len(part), Hkv, bs, D), torch.bfloat16, 200 + i, device=cuda_device))
-    q_host = synth.normal((B, Hq, D), torch.bfloat16, 6)
-    cache = pa.KVCache(k, v)
-    scale = 1 / math.sqrt(D)
-    out = pa.pa_decode(q_host.to(cuda_device), cache, torch.from_numpy(tables).to(cuda_device),
-                       torch.from_numpy(lens).to(cuda_device), int(lens.max()), scale)
-    assert pa.pa_read_device_error() == 0
-    assert torch.isfinite(out.float()).all()
-    r = synth.rng(7)
-    rows = [(int(b), int(h)) for b, h in zip(r.integers(0, B, 6), r.integers(0, Hq, 6))]
-    rows += [(int(np.argmax(lens)), 0), (int(np.argmax(lens)), Hq - 1)]
-    _sampled_check((k, v), q_host, tables, lens, out, rows, scale, Hkv)
-    del k, v, cache
-    torch.cuda.empty_cache()
-
-
-def test_shared_prefix_full_size_sampled(cuda_device):
-    """256 sequences in 32 groups of 8 sharing a 512+r token prefix through
-    refcounted blocks (copied on write when the suffixes were appended),
-    lognormal suffixes (median 800, up to 8192), 64 query / 8 kv heads:
-    sampled rows against the oracle, the shared blocks read by every member."""
-    B, Hq, Hkv, D, bs, gsz = 256, 64, 8, 128, 16, 8
-    pl, suffix, order, NB = synth.shared_prefix_layout(11, groups=32, group_size=gsz, prefix=512,
-                                                       median=800, clip=8192, bs=bs, prefix_tail=True)
-    A = pa.Allocator(NB, bs, order)
-    k = synth.normal((NB, Hkv, bs, D), torch.bfloat16, 12, device=cuda_device)
-    v = synth.normal((NB, Hkv, bs, D), torch.bfloat16, 13, device=cuda_device)
-    roots = [A.new_seq() for _ in range(32)]
-    A.batch_append(roots, pl)
-    seqs = []
-    for rt in roots:
-        seqs += [rt] + [A.fork(rt) for _ in range(gsz - 1)]
-    _, pairs = A.batch_append(seqs, suffix)
-    assert len(pairs) == 32 * (gsz - 1)
-    # the copies, done with torch (an independent route), so the pool the
-    # oracle sees does not depend on this library's copy kernel
-    src = torch.as_tensor(pairs[:, 0].astype(np.int64), device=cuda_device)
-    dst = torch.as_tensor(pairs[:, 1].astype(np.int64), device=cuda_device)
-    k.index_copy_(0, dst, k.index_select(0, src))
-    v.index_copy_(0, dst, v.index_select(0, src))
-    mb = max(A.seq_len(s_)[1] for s_ in seqs)
-    tables, lens = A.build_block_tables(seqs, mb)
-    # the first 32 blocks of every member of a group are the same physical blocks
-    assert all((tables[g * gsz:(g + 1) * gsz, :32] == tables[g * gsz, :32]).all() for g in range(32))
-    q_host = synth.normal((B, Hq, D), torch.bfloat16, 14)
-    cache = pa.KVCache(k, v)
-    scale = 1 / math.sqrt(D)
-    out = pa.pa_decode(q_host.to(cuda_device), cache, torch.from_numpy(tables).to(cuda_device),
-                       torch.from_numpy(lens).to(cuda_device), int(lens.max()), scale)
-    assert pa.pa_read_device_error() == 0
-    assert torch.isfinite(out.float()).all()
-    r = synth.rng(15)
-    rows = [(int(b), int(h)) for b, h in zip(r.integers(0, B, 24), r.integers(0, Hq, 24))]
-    rows += [(int(np.argmax(lens)), 7)]
-    _sampled_check((k, v), q_host, tables, lens, out, rows, scale, Hkv)
