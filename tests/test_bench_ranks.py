@@ -84,10 +84,11 @@ def test_traffic_record_follows_the_kernel_sources(tmp_path, monkeypatch):
     """The roofline's ncu traffic is reported only while the partition
     kernel's sources hash to the ones the record was captured on: a record of
     other sources gives None, and the hash moves when one of those sources
-    does."""
+    does.  It is the captured traffic / algorithmic ratio applied to this
+    run's algorithmic bytes per launch."""
     sys.path.insert(0, ROOT)
     import bench
-    assert bench.profiled_traffic("no-such-workload") is None
+    assert bench.profiled_traffic("no-such-workload", 1e9) is None
     # a copy of the kernel sources with records of its own
     root = tmp_path / "tree"
     csrc = root / "paged_kv_cache_402_b200" / "csrc"
@@ -97,13 +98,14 @@ def test_traffic_record_follows_the_kernel_sources(tmp_path, monkeypatch):
         (csrc / f).write_bytes(open(os.path.join(ROOT, "paged_kv_cache_402_b200", "csrc", f), "rb").read())
     monkeypatch.setattr(bench, "ROOT", str(root))
     h0 = bench.kernel_source_hash()
-    rec = {"kernel_hash": h0, "bytes_per_launch": 123}
+    rec = {"kernel_hash": h0,
+           "captured_launch": {"dram_read_bytes": 1010, "dram_write_bytes": 10, "algorithmic_bytes": 1000}}
     (root / "profiles" / "traffic.json").write_text(json.dumps({"gqa": rec}))
-    assert bench.profiled_traffic("gqa") == 123
+    assert bench.profiled_traffic("gqa", 5000) == 5100
     (root / "profiles" / "traffic.json").write_text(json.dumps({"gqa": dict(rec, kernel_hash="0" * 16)}))
-    assert bench.profiled_traffic("gqa") is None
+    assert bench.profiled_traffic("gqa", 5000) is None
     (root / "profiles" / "traffic.json").write_text(json.dumps({"gqa": rec}))
     with open(csrc / "pa_decode_tc.cuh", "a") as f:
         f.write("\n")
     assert bench.kernel_source_hash() != h0
-    assert bench.profiled_traffic("gqa") is None
+    assert bench.profiled_traffic("gqa", 5000) is None
