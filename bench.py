@@ -603,6 +603,8 @@ def run_e2e(args, insts, wl, dev, stream):
     the compute stream, and every buffer has two copies."""
     import paged_kv_cache_402_b200 as pa
 
+    if not args.unfused:
+        return run_e2e_native(args, insts, wl, dev, stream)
     B, Hq, Hkv, D, bs = wl["B"], wl["Hq"], wl["Hkv"], wl["D"], wl["bs"]
     inst = insts[0]
     mb = inst.max_blocks
@@ -704,6 +706,81 @@ def run_e2e(args, insts, wl, dev, stream):
         raise RuntimeError("non-finite output in the end-to-end steps")
     kv = sum(unique_kv_bytes(t, l, bs, 2 * Hkv * D * 2) for t, l in seen)
     return {"seconds": seconds, "kv_gb": kv / 1e9, "steps": n_steps, "h2d": total, "d2h": B * Hq * D * 2}
+
+
+def run_e2e_native(args, insts, wl, dev, stream):
+    """The end-to-end leg through the library's one-call step
+    (pa.DecodeStepper over pa_decode_step): per step one native call does the
+    allocator's step (one token per sequence, tables, lengths, copy-on-write
+    sources, sharing plan) into a pinned staging area, one host -> device copy
+    of it (q, new rows and the host-built arrays), the fused decode, and the
+    device -> host copy of the output; the host reads each output once its
+    slot comes round again.  Two slots alternate, so the host prepares step
+    i + 1 while the device runs step i.  Wall clock over all steps.
+
+    The K/V bytes of each step: its lengths are read from the slot's staging
+    area (B ints); the bytes the batch's sharers hold in common are taken
+    from the batch's tables after the loop, which stay valid for every step
+    because no step of these workloads changes what is shared (asserted: no
+    step copies on write, except in fresh-set workloads, whose every set is
+    stepped once and is read after the loop as the step left it)."""
+    import paged_kv_cache_402_b200 as pa
+
+    B, Hq, Hkv, D, bs = wl["B"], wl["Hq"], wl["Hkv"], wl["D"], wl["bs"]
+    inst = insts[0]
+    mb = inst.max_blocks
+    n_steps = max(1, args.steps)
+    share = 0 if args.no_share_plan else 4
+    row = 2 * Hkv * D * 2
+    stepper = pa.DecodeStepper(inst.alloc, inst.cache, B, Hq, mb, 1.0 / math.sqrt(D), share_max_members=share,
+                               stream=stream)
+    g = torch.Generator().manual_seed(5)
+    rows = (torch.randn(B, Hq, D, generator=g).to(torch.bfloat16),
+            torch.randn(B, Hkv, D, generator=g).to(torch.bfloat16),
+            torch.randn(B, Hkv, D, generator=g).to(torch.bfloat16))
+    for _ in range(2):  # the rows of both slots (the values do not change the work)
+        for dst, src in zip(stepper.inputs(), rows):
+            dst.copy_(src)
+        stepper.i += 1
+    stepper.i = 0
+    lens_view = [stepper._slots[k]["keep"][0][stepper.layout.lens:stepper.layout.lens + 4 * B].view(torch.int32).numpy()
+                 for k in range(2)]
+    fresh = bool(wl.get("fresh_sets"))
+    logical = np.zeros(n_steps, np.int64)
+    copies = 0
+    checksum = 0.0
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(n_steps):
+        k = stepper.next_slot
+        if i >= 2:
+            stepper.wait(k)
+            checksum += float(stepper.output(k)[0, 0, 0])
+        seqs = inst.sets[inst.uses + i] if fresh else inst.sets[0]
+        info = stepper.step(seqs)
+        copies += info["n_copies"]
+        logical[i] = int(lens_view[k].sum(dtype=np.int64))
+    for k in range(min(2, n_steps)):
+        stepper.wait((n_steps - 1 - k) % 2)
+        checksum += float(stepper.output((n_steps - 1 - k) % 2)[0, 0, 0])
+    seconds = time.perf_counter() - t0
+    torch.cuda.synchronize()
+    stepper.close()
+    if not math.isfinite(checksum):
+        raise RuntimeError("non-finite output in the end-to-end steps")
+    if fresh:
+        kv = 0
+        for i in range(n_steps):
+            tables, lens = inst.alloc.build_block_tables(inst.sets[inst.uses + i], mb)
+            kv += unique_kv_bytes(tables, lens, bs, row)
+    else:
+        if copies:
+            raise RuntimeError("a step copied on write: the shared bytes changed during the end-to-end leg")
+        tables, lens = inst.alloc.build_block_tables(inst.sets[0], mb)
+        shared_excess = int(lens.astype(np.int64).sum()) * row - unique_kv_bytes(tables, lens, bs, row)
+        kv = int(logical.sum()) * row - n_steps * shared_excess
+    return {"seconds": seconds, "kv_gb": kv / 1e9, "steps": n_steps, "h2d": stepper.h2d_bytes,
+            "d2h": stepper.d2h_bytes}
 
 
 def run_prefill(args, rank: int, world: int, dev):

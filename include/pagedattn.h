@@ -444,6 +444,90 @@ PA_API pa_status pa_decode_step_prepare(pa_allocator *a, const int32_t *seqs, in
                                         int32_t *parts_host, int32_t *first_part_host,
                                         int32_t *n_groups, int32_t *n_copies, int32_t *max_len);
 
+/* ------------------------------------------------- one decode step, end to end */
+/*
+ * A whole decode step from host memory in one call, for serving loops that
+ * hold their queries and new key/value rows in pinned host buffers: the
+ * step's host work (pa_decode_step_prepare: one token per sequence through
+ * the allocator, the tables, lengths, copy-on-write sources and sharing
+ * plan), one host-to-device copy of every input, pa_decode_shared (copy on
+ * write, append, decode), and the device-to-host copy of the output.  The
+ * pages describe these as what each step of a growing sequence does
+ * ("Fixed-Size KV Blocks": the new token goes into the current block, a
+ * block is taken only when it is full; "pagedattention" glossary entry,
+ * paragraph 5: shared blocks are copied when a sharer writes).
+ *
+ * A step slot holds one step's buffers; alternating two slots lets the host
+ * prepare step i + 1 while the device runs step i.  Every buffer is the
+ * caller's:
+ *   host      pinned host staging area of pa_step_layout(...).bytes bytes:
+ *             the caller writes q, k_new and v_new at their offsets before
+ *             the call; the call writes the rest
+ *   dev       device buffer of the same size (the staging area's mirror)
+ *   out_host  pinned host [n_seqs][num_q_heads][head_dim], cache dtype
+ *   out_dev   device, same shape
+ *   workspace device scratch of pa_decode_workspace_size(n_seqs, num_q_heads,
+ *             max_blocks * block_size, head_dim) bytes (or more)
+ *   ev_in, ev_kernel, ev_out   CUDA events (cudaEvent_t) of the slot, made by
+ *             pa_step_slot_events and released by pa_step_slot_release
+ */
+typedef struct {
+  size_t q, k_new, v_new, tables, lens, cow_src, first_part, members, parts;  /* byte offsets */
+  size_t bytes;                                                              /* total */
+} pa_step_layout_t;
+
+typedef struct {
+  void *host;
+  void *dev;
+  void *out_host;
+  void *out_dev;
+  void *workspace;
+  size_t workspace_bytes;
+  void *ev_in;      /* recorded on copy_stream once the inputs are on the device */
+  void *ev_kernel;  /* recorded on stream once the decode has run */
+  void *ev_out;     /* recorded on copy_stream once out is on the host */
+} pa_step_slot_t;
+
+/* Offsets (16-byte aligned) of a step's inputs in the staging area:
+ * q [n][Hq][D], k_new and v_new [n][Hkv][D] (cache dtype), tables
+ * [n][max_blocks], lens [n], cow_src [n], first_part [n], members
+ * [n / 2][share_max_members], parts [n / 2] (int32). */
+PA_API pa_status pa_step_layout(int32_t n_seqs, int32_t num_q_heads, const pa_cache_t *cache,
+                                int32_t max_blocks, int32_t share_max_members, pa_step_layout_t *layout);
+
+/* Creates the slot's three events (timing disabled) on the current device. */
+PA_API pa_status pa_step_slot_events(pa_step_slot_t *slot);
+/* Destroys the slot's events (after the slot's last step is done). */
+PA_API pa_status pa_step_slot_release(pa_step_slot_t *slot);
+/* Blocks the host until the slot's last step has copied its inputs to the
+ * device (its staging area may be rewritten) and its output to the host
+ * (out_host holds that step's result).  A slot never used returns at once. */
+PA_API pa_status pa_step_slot_wait(const pa_step_slot_t *slot);
+
+/*
+ * One decode step of n_seqs sequences (host ids seqs_host) through `slot`:
+ *  1. pa_decode_step_prepare into the staging area (all or nothing: an
+ *     error here, e.g. PA_ERR_OUT_OF_BLOCKS, leaves the allocator and the
+ *     device untouched);
+ *  2. on copy_stream, after the slot's previous decode: one cudaMemcpyAsync
+ *     of the staging area to dev, then ev_in;
+ *  3. on stream, after ev_in and the slot's previous output copy:
+ *     pa_decode_shared with the plan (share_max_members 2..4, or 0 for none),
+ *     the copy sources and the new rows, then ev_kernel;
+ *  4. on copy_stream, after ev_kernel: cudaMemcpyAsync of out_dev to
+ *     out_host, then ev_out.
+ * Nothing is synchronised: call pa_step_slot_wait(slot) before rewriting
+ * the slot's staging area or reading its out_host.  stream and copy_stream
+ * may be the same stream.  *n_copies, *n_groups and *max_len report the
+ * step's copies on write, plan groups and longest context.  A CUDA error
+ * after step 1 returns PA_ERR_CUDA with the allocator already advanced.
+ */
+PA_API pa_status pa_decode_step(pa_allocator *a, const int32_t *seqs_host, int32_t n_seqs,
+                                int32_t max_blocks, int32_t share_max_members,
+                                const pa_cache_t *cache, int32_t num_q_heads, float scale,
+                                const pa_step_slot_t *slot, void *stream, void *copy_stream,
+                                int32_t *n_copies, int32_t *n_groups, int32_t *max_len);
+
 /*
  * The per-sequence form of a decode step's copy pairs, as pa_append_decode
  * takes it.  Sequence i's last block is the table entry of its newest token,

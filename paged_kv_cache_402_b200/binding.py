@@ -51,6 +51,17 @@ class pa_cache_t(ctypes.Structure):
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
 
 
+class pa_step_layout_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in ("q", "k_new", "v_new", "tables", "lens", "cow_src", "first_part",
+                                             "members", "parts", "bytes")]
+
+
+class pa_step_slot_t(ctypes.Structure):
+    _fields_ = [("host", ctypes.c_void_p), ("dev", ctypes.c_void_p), ("out_host", ctypes.c_void_p),
+                ("out_dev", ctypes.c_void_p), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("ev_in", ctypes.c_void_p), ("ev_kernel", ctypes.c_void_p), ("ev_out", ctypes.c_void_p)]
+
+
 class pa_share_plan_t(ctypes.Structure):
     _fields_ = [("members", ctypes.c_void_p), ("parts", ctypes.c_void_p), ("first_part", ctypes.c_void_p),
                 ("n_groups", ctypes.c_int32), ("max_members", ctypes.c_int32)]
@@ -80,6 +91,12 @@ def _load() -> ctypes.CDLL:
         "pa_prefill": (st, [vp, cp, vp, i32, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp]),
         "pa_decode_step_prepare": (st, [vp, i32p, i32, i32, i32, i32p, i32p, i32p, i32p, i32p, i32p,
                                         i32p, i32p, i32p]),
+        "pa_step_layout": (st, [i32, i32, cp, i32, i32, ctypes.POINTER(pa_step_layout_t)]),
+        "pa_step_slot_events": (st, [ctypes.POINTER(pa_step_slot_t)]),
+        "pa_step_slot_release": (st, [ctypes.POINTER(pa_step_slot_t)]),
+        "pa_step_slot_wait": (st, [ctypes.POINTER(pa_step_slot_t)]),
+        "pa_decode_step": (st, [vp, i32p, i32, i32, i32, cp, i32, f32, ctypes.POINTER(pa_step_slot_t), vp, vp,
+                                i32p, i32p, i32p]),
         "pa_copy_blocks": (st, [vp, i32, cp, vp]),
         "pa_check_copy_pairs": (st, [i32p, i32, i32]),
         "pa_read_device_error": (st, [vp, i32p]),
@@ -463,6 +480,108 @@ def pa_read_device_error(stream=None) -> int:
     bits = ctypes.c_int32(0)
     _check(_lib.pa_read_device_error(_stream_ptr(stream), ctypes.byref(bits)), "pa_read_device_error")
     return bits.value
+
+
+# --------------------------------------------------------------------------
+# one decode step from pinned host buffers
+
+
+class DecodeStepper:
+    """Decode steps of a fixed batch of sequences from pinned host buffers,
+    one native call per step (pa_decode_step): the allocator's step, one
+    copy of the inputs to the device, the fused copy-on-write + append +
+    decode, and the copy of the output back.  `slots` step slots (default 2)
+    alternate, so the host prepares step i + 1 while the device runs step i.
+
+    Per step: ``q, k_new, v_new = stepper.inputs()`` gives the next slot's
+    pinned input views (after waiting for that slot's previous step), the
+    caller fills them, ``stepper.step(seqs)`` launches, and
+    ``stepper.output(slot)`` is that slot's pinned output once
+    ``stepper.wait(slot)`` returned."""
+
+    def __init__(self, alloc: "Allocator", cache: KVCache, n_seqs: int, num_q_heads: int, max_blocks: int,
+                 scale: float, share_max_members: int = 4, slots: int = 2, stream=None, copy_stream=None):
+        self.alloc, self.cache = alloc, cache
+        self.n, self.Hq, self.max_blocks = int(n_seqs), int(num_q_heads), int(max_blocks)
+        self.share, self.scale = int(share_max_members), float(scale)
+        dev = cache.k.device
+        lay = pa_step_layout_t()
+        _check(_lib.pa_step_layout(self.n, self.Hq, cache.ref(), self.max_blocks, self.share, ctypes.byref(lay)),
+               "pa_step_layout")
+        self.layout = lay
+        ws_bytes = max(16, pa_decode_workspace_size(self.n, self.Hq, self.max_blocks * cache.block_size,
+                                                    cache.head_dim))
+        Hkv, D, dt = cache.num_kv_heads, cache.head_dim, cache.dtype
+        self._slots = []
+        for _ in range(int(slots)):
+            host = torch.zeros(lay.bytes, dtype=torch.uint8).pin_memory()
+            devb = torch.empty(lay.bytes, dtype=torch.uint8, device=dev)
+            out_host = torch.empty(self.n, self.Hq, D, dtype=dt).pin_memory()
+            out_dev = torch.empty(self.n, self.Hq, D, dtype=dt, device=dev)
+            ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+            st = pa_step_slot_t(host.data_ptr(), devb.data_ptr(), out_host.data_ptr(), out_dev.data_ptr(),
+                                ws.data_ptr(), ws_bytes, None, None, None)
+            _check(_lib.pa_step_slot_events(ctypes.byref(st)), "pa_step_slot_events")
+
+            def view(off, shape):
+                nb = int(np.prod(shape)) * torch.tensor([], dtype=dt).element_size()
+                return host[off:off + nb].view(dt).view(shape)
+            self._slots.append({"struct": st, "keep": (host, devb, out_host, out_dev, ws), "out_host": out_host,
+                                "q": view(lay.q, (self.n, self.Hq, D)), "k": view(lay.k_new, (self.n, Hkv, D)),
+                                "v": view(lay.v_new, (self.n, Hkv, D))})
+        self.stream = stream if stream is not None else torch.cuda.current_stream(dev)
+        self.copy_stream = copy_stream if copy_stream is not None else torch.cuda.Stream(device=dev)
+        self.i = 0
+        self.h2d_bytes = lay.bytes
+        self.d2h_bytes = self.n * self.Hq * D * torch.tensor([], dtype=dt).element_size()
+
+    @property
+    def next_slot(self) -> int:
+        return self.i % len(self._slots)
+
+    def wait(self, slot: int) -> None:
+        """Until the slot's last step has its inputs on the device and its
+        output on the host."""
+        _check(_lib.pa_step_slot_wait(ctypes.byref(self._slots[slot]["struct"])), "pa_step_slot_wait")
+
+    def inputs(self):
+        """(q, k_new, v_new) pinned views of the next slot, after waiting for
+        its previous step."""
+        S = self._slots[self.next_slot]
+        self.wait(self.next_slot)
+        return S["q"], S["k"], S["v"]
+
+    def output(self, slot: int) -> torch.Tensor:
+        return self._slots[slot]["out_host"]
+
+    def step(self, seqs) -> dict:
+        """Launches one step through the next slot; returns the slot index,
+        the step's copies on write, plan groups and longest context."""
+        seqs = np.ascontiguousarray(np.asarray(seqs, dtype=np.int32))
+        if len(seqs) != self.n:
+            raise ValueError(f"a stepper of {self.n} sequences got {len(seqs)}")
+        k = self.next_slot
+        nc, ng, ml = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int32(0)
+        _check(_lib.pa_decode_step(self.alloc._h, _i32p(seqs), self.n, self.max_blocks, self.share,
+                                   self.cache.ref(), self.Hq, self.scale, ctypes.byref(self._slots[k]["struct"]),
+                                   self.stream.cuda_stream, self.copy_stream.cuda_stream, ctypes.byref(nc),
+                                   ctypes.byref(ng), ctypes.byref(ml)), "pa_decode_step")
+        self.i += 1
+        return {"slot": k, "n_copies": nc.value, "n_groups": ng.value, "max_len": ml.value}
+
+    def close(self) -> None:
+        """Waits for every slot and releases their events."""
+        for k, S in enumerate(self._slots):
+            if S["struct"].ev_in:
+                self.wait(k)
+                _check(_lib.pa_step_slot_release(ctypes.byref(S["struct"])), "pa_step_slot_release")
+
+    def __del__(self):
+        try:
+            if _lib is not None:
+                self.close()
+        except Exception:
+            pass
 
 
 # --------------------------------------------------------------------------

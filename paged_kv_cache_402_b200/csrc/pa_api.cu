@@ -818,3 +818,143 @@ PA_API pa_status pa_read_device_error(void *stream, int32_t *bits) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// One decode step from pinned host buffers: host work, one copy in, the
+// decode, one copy out, ordered by the slot's events.
+
+namespace {
+
+inline size_t layout_take(size_t *at, size_t bytes) {
+  const size_t off = *at;
+  *at = round16(*at + bytes);
+  return off;
+}
+
+}  // namespace
+
+extern "C" {
+
+PA_API pa_status pa_step_layout(int32_t n_seqs, int32_t num_q_heads, const pa_cache_t *cache,
+                                int32_t max_blocks, int32_t share_max_members, pa_step_layout_t *layout) {
+  if (!layout || !cache || n_seqs < 0 || num_q_heads <= 0 || max_blocks < 0 || share_max_members < 0 ||
+      share_max_members > 4 || cache->num_kv_heads <= 0 || cache->head_dim <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (cache->dtype != PA_DTYPE_F32 && cache->dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
+  const size_t es = (size_t)elem_bytes(cache->dtype), n = (size_t)n_seqs, D = (size_t)cache->head_dim;
+  const size_t groups = n / 2 > 0 ? n / 2 : 1;
+  const size_t members = (size_t)(share_max_members > 0 ? share_max_members : 1);
+  size_t at = 0;
+  pa_step_layout_t L{};
+  L.q = layout_take(&at, n * num_q_heads * D * es);
+  L.k_new = layout_take(&at, n * cache->num_kv_heads * D * es);
+  L.v_new = layout_take(&at, n * cache->num_kv_heads * D * es);
+  L.tables = layout_take(&at, n * (size_t)max_blocks * 4);
+  L.lens = layout_take(&at, n * 4);
+  L.cow_src = layout_take(&at, n * 4);
+  L.first_part = layout_take(&at, n * 4);
+  L.members = layout_take(&at, groups * members * 4);
+  L.parts = layout_take(&at, groups * 4);
+  L.bytes = at;
+  *layout = L;
+  return PA_OK;
+}
+
+PA_API pa_status pa_step_slot_events(pa_step_slot_t *slot) {
+  if (!slot) return PA_ERR_INVALID_ARG;
+  cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
+  for (int i = 0; i < 3; ++i) {
+    const cudaError_t e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(ev[j]);
+      return cuda_failed(e);
+    }
+  }
+  slot->ev_in = ev[0];
+  slot->ev_kernel = ev[1];
+  slot->ev_out = ev[2];
+  return PA_OK;
+}
+
+PA_API pa_status pa_step_slot_release(pa_step_slot_t *slot) {
+  if (!slot) return PA_ERR_INVALID_ARG;
+  void **evs[3] = {&slot->ev_in, &slot->ev_kernel, &slot->ev_out};
+  pa_status s = PA_OK;
+  for (void **e : evs) {
+    if (*e) {
+      const cudaError_t r = cudaEventDestroy(static_cast<cudaEvent_t>(*e));
+      if (r != cudaSuccess) s = cuda_failed(r);
+      *e = nullptr;
+    }
+  }
+  return s;
+}
+
+PA_API pa_status pa_step_slot_wait(const pa_step_slot_t *slot) {
+  if (!slot || !slot->ev_in || !slot->ev_out) return PA_ERR_INVALID_ARG;
+  cudaError_t e = cudaEventSynchronize(static_cast<cudaEvent_t>(slot->ev_in));
+  if (e == cudaSuccess) e = cudaEventSynchronize(static_cast<cudaEvent_t>(slot->ev_out));
+  return e == cudaSuccess ? PA_OK : cuda_failed(e);
+}
+
+PA_API pa_status pa_decode_step(pa_allocator *a, const int32_t *seqs_host, int32_t n_seqs,
+                                int32_t max_blocks, int32_t share_max_members,
+                                const pa_cache_t *cache, int32_t num_q_heads, float scale,
+                                const pa_step_slot_t *slot, void *stream, void *copy_stream,
+                                int32_t *n_copies, int32_t *n_groups, int32_t *max_len) {
+  if (!a || !slot || !n_copies || !n_groups || !max_len || !slot->host || !slot->dev || !slot->out_host ||
+      !slot->out_dev || !slot->ev_in || !slot->ev_kernel || !slot->ev_out)
+    return PA_ERR_INVALID_ARG;
+  pa_step_layout_t L{};
+  pa_status s = pa_step_layout(n_seqs, num_q_heads, cache, max_blocks, share_max_members, &L);
+  if (s != PA_OK) return s;
+  s = check_cache(cache);
+  if (s != PA_OK) return s;
+  if (!aligned16(slot->host) || !aligned16(slot->dev)) return PA_ERR_INVALID_ARG;
+  // the decode's own checks, before the allocator moves (a step too long
+  // for the table width is refused by the preparation itself)
+  if (num_q_heads % cache->num_kv_heads) return PA_ERR_INVALID_ARG;
+  const int64_t ctx_cap = (int64_t)max_blocks * cache->block_size;
+  if (ctx_cap > INT32_MAX - pa::kPart) return PA_ERR_INVALID_ARG;
+  const size_t need_ws =
+      n_seqs > 0 ? workspace_bytes_for(n_seqs, num_q_heads, (int32_t)ctx_cap, cache->head_dim) : 0;
+  if (need_ws > 0 && (!slot->workspace || slot->workspace_bytes < need_ws)) return PA_ERR_TOO_SMALL;
+  char *h = static_cast<char *>(slot->host);
+  char *d = static_cast<char *>(slot->dev);
+  auto hi = [&](size_t off) { return reinterpret_cast<int32_t *>(h + off); };
+  auto di = [&](size_t off) { return reinterpret_cast<int32_t *>(d + off); };
+  s = pa_decode_step_prepare(a, seqs_host, n_seqs, max_blocks, share_max_members, hi(L.tables), hi(L.lens),
+                             hi(L.cow_src), hi(L.members), hi(L.parts), hi(L.first_part), n_groups, n_copies,
+                             max_len);
+  if (s != PA_OK || n_seqs == 0) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStream_t cst = static_cast<cudaStream_t>(copy_stream);
+  cudaEvent_t ev_in = static_cast<cudaEvent_t>(slot->ev_in);
+  cudaEvent_t ev_kernel = static_cast<cudaEvent_t>(slot->ev_kernel);
+  cudaEvent_t ev_out = static_cast<cudaEvent_t>(slot->ev_out);
+  cudaError_t e;
+  // inputs: after the slot's previous decode has read its device copy
+  if ((e = cudaStreamWaitEvent(cst, ev_kernel, 0)) != cudaSuccess) return cuda_failed(e);
+  if ((e = cudaMemcpyAsync(d, h, L.bytes, cudaMemcpyHostToDevice, cst)) != cudaSuccess) return cuda_failed(e);
+  if ((e = cudaEventRecord(ev_in, cst)) != cudaSuccess) return cuda_failed(e);
+  // the decode: after the inputs, and after the previous output left out_dev
+  if ((e = cudaStreamWaitEvent(st, ev_in, 0)) != cudaSuccess) return cuda_failed(e);
+  if ((e = cudaStreamWaitEvent(st, ev_out, 0)) != cudaSuccess) return cuda_failed(e);
+  pa_share_plan_t plan{di(L.members), di(L.parts), di(L.first_part), *n_groups,
+                       share_max_members > 0 ? share_max_members : 1};
+  s = pa_decode_shared(d + L.k_new, d + L.v_new, *n_copies > 0 ? di(L.cow_src) : nullptr, d + L.q, cache,
+                       di(L.tables), max_blocks, di(L.lens), n_seqs, num_q_heads, *max_len, scale,
+                       *n_groups > 0 ? &plan : nullptr, slot->out_dev, slot->workspace, slot->workspace_bytes,
+                       stream);
+  if (s != PA_OK) return s;
+  if ((e = cudaEventRecord(ev_kernel, st)) != cudaSuccess) return cuda_failed(e);
+  // the output, back to the host
+  if ((e = cudaStreamWaitEvent(cst, ev_kernel, 0)) != cudaSuccess) return cuda_failed(e);
+  const size_t out_bytes = (size_t)n_seqs * num_q_heads * cache->head_dim * elem_bytes(cache->dtype);
+  if ((e = cudaMemcpyAsync(slot->out_host, slot->out_dev, out_bytes, cudaMemcpyDeviceToHost, cst)) != cudaSuccess)
+    return cuda_failed(e);
+  if ((e = cudaEventRecord(ev_out, cst)) != cudaSuccess) return cuda_failed(e);
+  return PA_OK;
+}
+
+}  // extern "C"

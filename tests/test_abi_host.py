@@ -205,6 +205,38 @@ def test_workspace_size_of_huge_lengths():
     assert ws == 2 * ((parts * 4 + 15) // 16 * 16) + parts * 128 * 4
 
 
+def test_step_layout():
+    """The staging area of one decode step: q, new rows, then the int32
+    arrays the step's host work writes, each 16-byte aligned, in order."""
+    L = pa.pa_step_layout_t()
+    c = _cache_struct(num_kv_heads=8)
+    assert pa.lib().pa_step_layout(32, 32, ctypes.byref(c), 257, 4, ctypes.byref(L)) == pa.PA_OK
+    offs = [L.q, L.k_new, L.v_new, L.tables, L.lens, L.cow_src, L.first_part, L.members, L.parts, L.bytes]
+    assert offs == sorted(offs) and all(o % 16 == 0 for o in offs)
+    assert L.k_new - L.q == 32 * 32 * 128 * 2 and L.v_new - L.k_new == 32 * 8 * 128 * 2
+    assert L.lens - L.tables >= 32 * 257 * 4 and L.parts - L.members >= 16 * 4 * 4
+    assert pa.lib().pa_step_layout(32, 32, ctypes.byref(c), 257, 5, ctypes.byref(L)) == pa.PA_ERR_INVALID_ARG
+
+
+def test_decode_step_refuses_before_the_allocator_moves():
+    """Argument errors of pa_decode_step come before the allocator's step: a
+    slot without buffers, or a workspace too small, leaves every sequence as
+    it was."""
+    A = pa.Allocator(64, 16)
+    s = A.new_seq()
+    A.append(s, 600)
+    seqs = np.array([s], np.int32)
+    nc, ng, ml = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    c = _cache_struct(num_blocks=64, num_kv_heads=2)
+    slot = pa.pa_step_slot_t()
+    args = lambda sl: (A._h, seqs.ctypes.data, 1, 64, 0, ctypes.byref(c), 8, ctypes.c_float(0.1), ctypes.byref(sl),
+                       None, None, ctypes.byref(nc), ctypes.byref(ng), ctypes.byref(ml))
+    assert pa.lib().pa_decode_step(*args(slot)) == pa.PA_ERR_INVALID_ARG
+    slot = pa.pa_step_slot_t(16, 32, 48, 64, None, 0, 1, 2, 3)  # fake addresses, no workspace
+    assert pa.lib().pa_decode_step(*args(slot)) == pa.PA_ERR_TOO_SMALL  # 64 x 16 tokens of room need a workspace
+    assert A.seq_len(s) == (600, 38)
+
+
 def test_workspace_size():
     ws = pa.pa_decode_workspace_size
     assert ws(4, 8, 512, 128) == 0
