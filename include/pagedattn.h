@@ -77,7 +77,8 @@ typedef enum { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
 #define PA_DEVERR_LEN 0x10       /* pa_decode: a context length < 0 or > max_context_len (row zeroed) */
 #define PA_DEVERR_PLAN 0x20      /* pa_decode_shared: a sharing plan entry that does not fit its sequence (ignored) */
 
-/* Tokens per split-context partition of pa_decode. */
+/* Tokens per split-context partition of the decode calls unless the pool
+ * says otherwise (pa_cache_t.partition_tokens). */
 #define PA_PARTITION_TOKENS 512
 
 /* The paged pool.  k and v are device pointers of the layout above. */
@@ -89,6 +90,11 @@ typedef struct {
   int32_t block_size;   /* tokens per block: 8, 16 or 32 */
   int32_t num_kv_heads;
   int32_t head_dim;     /* 64 or 128 */
+  /* Tokens per split-context partition of the decode calls over this pool:
+   * 256, 512 or 1024, or 0 for PA_PARTITION_TOKENS.  It sets the workspace
+   * size (pa_decode_workspace_size_p) and the unit of sharing of a plan
+   * (pa_share_plan), which must be built for the same size. */
+  int32_t partition_tokens;
 } pa_cache_t;
 
 /* ---------------------------------------------------------------- kernels */
@@ -116,7 +122,7 @@ PA_API pa_status pa_append_kv(const void *k, const void *v, const int64_t *slot_
  *   s_t = scale * <q[b,h,:], K(b,t,g)>  for t < context_lens[b]
  *   out[b,h,:] = sum_t exp(s_t - max s) V(b,t,g) / sum_t exp(s_t - max s)
  * with K(b,t,g) = k_cache[block_tables[b*max_blocks_per_seq + t/bs]][g][t%bs].
- * Contexts are cut into PA_PARTITION_TOKENS-token partitions; each partition
+ * Contexts are cut into partitions of the pool's partition_tokens; each partition
  * keeps (max, sum, unnormalised accumulator) in the workspace and a second
  * kernel merges them with a log-sum-exp combine.  Arithmetic is fp32 with an
  * online softmax; out is rounded once to the cache dtype.
@@ -128,8 +134,9 @@ PA_API pa_status pa_append_kv(const void *k, const void *v, const int64_t *slot_
  *   max_context_len  host: an upper bound of every context_lens[b]; a larger
  *                 length sets PA_DEVERR_LEN and zeroes that row
  *   out           device [num_seqs][num_q_heads][head_dim], cache dtype
- *   workspace     device scratch of at least pa_decode_workspace_size(...)
- *                 bytes, 16-byte aligned (NULL allowed when that size is 0)
+ *   workspace     device scratch of at least pa_decode_workspace_size_p(...,
+ *                 cache->partition_tokens) bytes, 16-byte aligned (NULL
+ *                 allowed when that size is 0)
  * num_q_heads / num_kv_heads (the group size) must be 1, 2, 4 or 8.
  */
 PA_API pa_status pa_decode(const void *q, const pa_cache_t *cache, const int32_t *block_tables,
@@ -175,7 +182,7 @@ PA_API pa_status pa_append_decode(const void *k_new, const void *v_new, const in
 /*
  * A sharing plan for pa_decode_shared: groups of sequences of one batch whose
  * block tables hold the same physical blocks for their first parts[j] whole
- * partitions (PA_PARTITION_TOKENS tokens each), every one of them before the
+ * partitions (of the pool's partition_tokens), every one of them before the
  * member's last partition.  pa_share_plan builds one from host tables.
  *   members     device [n_groups][max_members] int32: sequence indices of the
  *               batch, a group's members first, -1 after its last
@@ -245,10 +252,17 @@ PA_API pa_status pa_prefill(const void *q, const pa_cache_t *cache, const int32_
                             int32_t total_query_tokens, int32_t max_query_len,
                             int32_t max_context_len, float scale, void *out, void *stream);
 
-/* Bytes of workspace pa_decode needs for these sizes (0 when no context is
- * longer than one partition). */
+/* Bytes of workspace pa_decode needs for these sizes with partitions of
+ * PA_PARTITION_TOKENS tokens (0 when no context is longer than one
+ * partition). */
 PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
                                        int32_t max_context_len, int32_t head_dim);
+
+/* The same for partitions of partition_tokens tokens (256, 512 or 1024; 0
+ * for PA_PARTITION_TOKENS); 0 for any other size. */
+PA_API size_t pa_decode_workspace_size_p(int32_t num_seqs, int32_t num_q_heads,
+                                         int32_t max_context_len, int32_t head_dim,
+                                         int32_t partition_tokens);
 
 /*
  * pa_decode without a caller-provided workspace.  The pages have no
@@ -261,9 +275,10 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
  * fixed array of PA_STATIC_WORKSPACE_BYTES inside the library, which every
  * GPU that loads the library holds until the process exits.
  *  - Arguments and results are those of pa_decode (minus the workspace).
- *  - Sizes whose scratch, pa_decode_workspace_size(num_seqs, num_q_heads,
- *    max_context_len, head_dim), exceeds PA_STATIC_WORKSPACE_BYTES are
- *    rejected with PA_ERR_TOO_SMALL before any launch.
+ *  - Sizes whose scratch, pa_decode_workspace_size_p(num_seqs, num_q_heads,
+ *    max_context_len, head_dim, partition), exceeds PA_STATIC_WORKSPACE_BYTES are
+ *    rejected with PA_ERR_TOO_SMALL before any launch (with the pool's
+ *    partition_tokens: pa_decode_workspace_size_p).
  *  - The first call in a CUDA context looks up that context's copy of the
  *    array (with the context current, the runtime's current device's
  *    primary context unless the caller bound another); make that first call
@@ -405,7 +420,9 @@ PA_API pa_status pa_alloc_stats(pa_allocator *a, int64_t *used_slots, int64_t *a
 PA_API pa_status pa_block_refcount(pa_allocator *a, int32_t block, int32_t *refcount);
 
 /*
- * Builds a sharing plan from host tables (after the step's appends):
+ * Builds a sharing plan from host tables (after the step's appends), for
+ * partitions of partition_tokens tokens (256, 512 or 1024; 0 for
+ * PA_PARTITION_TOKENS):
  * sequences longer than one partition whose first partition's table entries
  * are identical form buckets; each bucket is cut into groups of at most
  * max_members (2..4) in sequence order, a lone leftover joins no group; a
@@ -418,8 +435,8 @@ PA_API pa_status pa_block_refcount(pa_allocator *a, int32_t block, int32_t *refc
  */
 PA_API pa_status pa_share_plan(const int32_t *tables_host, int32_t max_blocks,
                                const int32_t *lens_host, int32_t n_seqs, int32_t block_size,
-                               int32_t max_members, int32_t *members_host, int32_t *parts_host,
-                               int32_t *first_part_host, int32_t *n_groups);
+                               int32_t partition_tokens, int32_t max_members, int32_t *members_host,
+                               int32_t *parts_host, int32_t *first_part_host, int32_t *n_groups);
 
 /*
  * One decode step's host work in one call: appends one token to each of the
@@ -431,14 +448,16 @@ PA_API pa_status pa_share_plan(const int32_t *tables_host, int32_t max_blocks,
  *     would not fit max_blocks;
  *   cow_src_host [n_seqs]: the block a sequence's copy-on-write move copies
  *     into its new last block, -1 for none (*n_copies of them);
- *   with share_max_members in 2..4, the sharing plan of pa_share_plan
+ *   with share_max_members in 2..4, the sharing plan of pa_share_plan for
+ *     partitions of partition_tokens tokens
  *     (members_host room for n_seqs / 2 groups x share_max_members,
  *     parts_host room for n_seqs / 2, *n_groups); with 0, no plan and
  *     first_part_host all zeros;
  *   *max_len: the longest length (max_context_len of the call).
  */
 PA_API pa_status pa_decode_step_prepare(pa_allocator *a, const int32_t *seqs, int32_t n_seqs,
-                                        int32_t max_blocks, int32_t share_max_members,
+                                        int32_t max_blocks, int32_t partition_tokens,
+                                        int32_t share_max_members,
                                         int32_t *tables_host, int32_t *lens_host,
                                         int32_t *cow_src_host, int32_t *members_host,
                                         int32_t *parts_host, int32_t *first_part_host,
@@ -466,8 +485,9 @@ PA_API pa_status pa_decode_step_prepare(pa_allocator *a, const int32_t *seqs, in
  *   dev       device buffer of the same size (the staging area's mirror)
  *   out_host  pinned host [n_seqs][num_q_heads][head_dim], cache dtype
  *   out_dev   device, same shape
- *   workspace device scratch of pa_decode_workspace_size(n_seqs, num_q_heads,
- *             max_blocks * block_size, head_dim) bytes (or more)
+ *   workspace device scratch of pa_decode_workspace_size_p(n_seqs, num_q_heads,
+ *             max_blocks * block_size, head_dim, cache->partition_tokens)
+ *             bytes (or more)
  *   ev_in, ev_kernel, ev_out   CUDA events (cudaEvent_t) of the slot, made by
  *             pa_step_slot_events and released by pa_step_slot_release
  */
@@ -512,7 +532,8 @@ PA_API pa_status pa_step_slot_wait(const pa_step_slot_t *slot);
  *  2. on copy_stream, after the slot's previous decode: one cudaMemcpyAsync
  *     of the staging area to dev, then ev_in;
  *  3. on stream, after ev_in and the slot's previous output copy:
- *     pa_decode_shared with the plan (share_max_members 2..4, or 0 for none),
+ *     pa_decode_shared with the plan (share_max_members 2..4, or 0 for none;
+ *     built for the pool's partition_tokens),
  *     the copy sources and the new rows, then ev_kernel;
  *  4. on copy_stream, after ev_kernel: cudaMemcpyAsync of out_dev to
  *     out_host, then ev_out.

@@ -48,7 +48,8 @@ class OutOfBlocks(PagedAttnError):
 class pa_cache_t(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("dtype", ctypes.c_int32),
                 ("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
-                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("partition_tokens", ctypes.c_int32)]
 
 
 class pa_step_layout_t(ctypes.Structure):
@@ -82,14 +83,15 @@ def _load() -> ctypes.CDLL:
         "pa_append_kv": (st, [vp, vp, vp, i32, cp, vp]),
         "pa_decode": (st, [vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp, sz, vp]),
         "pa_decode_workspace_size": (sz, [i32, i32, i32, i32]),
+        "pa_decode_workspace_size_p": (sz, [i32, i32, i32, i32, i32]),
         "pa_decode_static_workspace": (st, [vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp]),
         "pa_append_decode": (st, [vp, vp, vp, vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp, sz, vp]),
         "pa_cow_sources": (st, [i32p, i32, i32p, i32, i32p, i32, i32, i32p]),
         "pa_decode_shared": (st, [vp, vp, vp, vp, cp, vp, i32, vp, i32, i32, i32, f32,
                                   ctypes.POINTER(pa_share_plan_t), vp, vp, sz, vp]),
-        "pa_share_plan": (st, [i32p, i32, i32p, i32, i32, i32, i32p, i32p, i32p, i32p]),
+        "pa_share_plan": (st, [i32p, i32, i32p, i32, i32, i32, i32, i32p, i32p, i32p, i32p]),
         "pa_prefill": (st, [vp, cp, vp, i32, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp]),
-        "pa_decode_step_prepare": (st, [vp, i32p, i32, i32, i32, i32p, i32p, i32p, i32p, i32p, i32p,
+        "pa_decode_step_prepare": (st, [vp, i32p, i32, i32, i32, i32, i32p, i32p, i32p, i32p, i32p, i32p,
                                         i32p, i32p, i32p]),
         "pa_step_layout": (st, [i32, i32, cp, i32, i32, ctypes.POINTER(pa_step_layout_t)]),
         "pa_step_slot_events": (st, [ctypes.POINTER(pa_step_slot_t)]),
@@ -185,23 +187,30 @@ def _check_q_out(q: torch.Tensor, out, cache) -> None:
 
 
 class KVCache:
-    """The paged pools: k and v of shape [num_blocks, num_kv_heads, block_size, head_dim]."""
+    """The paged pools: k and v of shape [num_blocks, num_kv_heads, block_size, head_dim];
+    partition_tokens is the split-context partition of the decode calls over
+    them (256, 512 or 1024)."""
 
-    def __init__(self, k: torch.Tensor, v: torch.Tensor):
+    def __init__(self, k: torch.Tensor, v: torch.Tensor, partition_tokens: int = PA_PARTITION_TOKENS):
         if k.shape != v.shape or k.dtype != v.dtype or k.dim() != 4:
             raise ValueError("k and v must be [num_blocks, Hkv, block_size, head_dim] of one dtype")
         if k.dtype not in _DTYPES:
             raise TypeError(f"unsupported cache dtype {k.dtype}")
         _dev(k, "k_cache")
         _dev(v, "v_cache")
+        if partition_tokens not in (256, 512, 1024):
+            raise ValueError("partition_tokens must be 256, 512 or 1024")
         self.k, self.v = k, v
+        self.partition_tokens = int(partition_tokens)
         self.struct = pa_cache_t(k.data_ptr(), v.data_ptr(), _DTYPES[k.dtype], k.shape[0], k.shape[2],
-                                 k.shape[1], k.shape[3])
+                                 k.shape[1], k.shape[3], self.partition_tokens)
 
     @classmethod
-    def empty(cls, num_blocks, num_kv_heads, block_size, head_dim, dtype=torch.bfloat16, device="cuda"):
+    def empty(cls, num_blocks, num_kv_heads, block_size, head_dim, dtype=torch.bfloat16, device="cuda",
+              partition_tokens: int = PA_PARTITION_TOKENS):
         shape = (num_blocks, num_kv_heads, block_size, head_dim)
-        return cls(torch.empty(shape, dtype=dtype, device=device), torch.empty(shape, dtype=dtype, device=device))
+        return cls(torch.empty(shape, dtype=dtype, device=device), torch.empty(shape, dtype=dtype, device=device),
+                   partition_tokens)
 
     @property
     def num_blocks(self):
@@ -241,8 +250,10 @@ def pa_append_kv(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor, c
                              _stream_ptr(stream)), "pa_append_kv")
 
 
-def pa_decode_workspace_size(num_seqs: int, num_q_heads: int, max_context_len: int, head_dim: int) -> int:
-    return int(_lib.pa_decode_workspace_size(num_seqs, num_q_heads, max_context_len, head_dim))
+def pa_decode_workspace_size(num_seqs: int, num_q_heads: int, max_context_len: int, head_dim: int,
+                             partition_tokens: int = PA_PARTITION_TOKENS) -> int:
+    return int(_lib.pa_decode_workspace_size_p(num_seqs, num_q_heads, max_context_len, head_dim,
+                                               int(partition_tokens)))
 
 
 def pa_decode(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor, context_lens: torch.Tensor,
@@ -255,7 +266,7 @@ def pa_decode(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor, conte
         raise ValueError("block_tables must be [B, max_blocks] and context_lens [B]")
     if out is None:
         out = torch.empty_like(q)
-    need = pa_decode_workspace_size(B, Hq, int(max_context_len), D)
+    need = pa_decode_workspace_size(B, Hq, int(max_context_len), D, cache.partition_tokens)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = _dev(workspace, "workspace") if workspace is not None else None
@@ -287,7 +298,7 @@ def pa_append_decode(k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor, 
         raise ValueError("cow_src must be [B]")
     if out is None:
         out = torch.empty_like(q)
-    need = pa_decode_workspace_size(B, Hq, int(max_context_len), D)
+    need = pa_decode_workspace_size(B, Hq, int(max_context_len), D, cache.partition_tokens)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = _dev(workspace, "workspace") if workspace is not None else None
@@ -358,9 +369,11 @@ class SharePlan:
         return ctypes.byref(self._struct)
 
 
-def share_plan(tables, lens, block_size: int, max_members: int = 4) -> SharePlan:
+def share_plan(tables, lens, block_size: int, max_members: int = 4,
+               partition_tokens: int = PA_PARTITION_TOKENS) -> SharePlan:
     """Host: groups the sequences of a batch whose tables agree on their
-    leading whole partitions (pa_share_plan)."""
+    leading whole partitions of partition_tokens tokens (pa_share_plan; the
+    decode's pool must have the same partition size)."""
     tables = np.ascontiguousarray(np.asarray(tables, dtype=np.int32))
     lens = np.ascontiguousarray(np.asarray(lens, dtype=np.int32))
     n = len(lens)
@@ -370,8 +383,8 @@ def share_plan(tables, lens, block_size: int, max_members: int = 4) -> SharePlan
     first = np.empty(n, dtype=np.int32)
     ng = ctypes.c_int32(0)
     _check(_lib.pa_share_plan(_i32p(tables), tables.shape[1] if tables.ndim == 2 else 0, _i32p(lens), n,
-                              int(block_size), int(max_members), _i32p(members), _i32p(parts), _i32p(first),
-                              ctypes.byref(ng)), "pa_share_plan")
+                              int(block_size), int(partition_tokens), int(max_members), _i32p(members), _i32p(parts),
+                              _i32p(first), ctypes.byref(ng)), "pa_share_plan")
     g = ng.value
     return SharePlan(members[:g].copy(), parts[:g].copy(), first)
 
@@ -394,7 +407,7 @@ def pa_decode_shared(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor
         raise ValueError(f"k_new and v_new must be {list(row_shape)}")
     if out is None:
         out = torch.empty_like(q)
-    need = pa_decode_workspace_size(B, Hq, int(max_context_len), D)
+    need = pa_decode_workspace_size(B, Hq, int(max_context_len), D, cache.partition_tokens)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = _dev(workspace, "workspace") if workspace is not None else None
@@ -510,7 +523,7 @@ class DecodeStepper:
                "pa_step_layout")
         self.layout = lay
         ws_bytes = max(16, pa_decode_workspace_size(self.n, self.Hq, self.max_blocks * cache.block_size,
-                                                    cache.head_dim))
+                                                    cache.head_dim, cache.partition_tokens))
         Hkv, D, dt = cache.num_kv_heads, cache.head_dim, cache.dtype
         self._slots = []
         for _ in range(int(slots)):
@@ -609,7 +622,8 @@ class Allocator:
             _lib.pa_alloc_destroy(h)
             self._h = None
 
-    def decode_step(self, seqs, max_blocks: int, share_max_members: int = 4, out: dict | None = None) -> dict:
+    def decode_step(self, seqs, max_blocks: int, share_max_members: int = 4, out: dict | None = None,
+                    partition_tokens: int = PA_PARTITION_TOKENS) -> dict:
         """One decode step's host work in one call (pa_decode_step_prepare):
         one token appended to every sequence, then the tables, lengths,
         copy-on-write sources and sharing plan that pa_decode_shared takes.
@@ -625,7 +639,8 @@ class Allocator:
             "cow_src": np.empty(n, np.int32), "first_part": np.empty(n, np.int32),
             "members": np.empty((max(1, n // 2), m), np.int32), "parts": np.empty(max(1, n // 2), np.int32)}
         ng, nc, ml = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int32(0)
-        _check(_lib.pa_decode_step_prepare(self._h, _i32p(seqs), n, int(max_blocks), int(share_max_members),
+        _check(_lib.pa_decode_step_prepare(self._h, _i32p(seqs), n, int(max_blocks), int(partition_tokens),
+                                           int(share_max_members),
                                            _i32p(o["tables"]), _i32p(o["lens"]), _i32p(o["cow_src"]),
                                            _i32p(o["members"]), _i32p(o["parts"]), _i32p(o["first_part"]),
                                            ctypes.byref(ng), ctypes.byref(nc), ctypes.byref(ml)), "pa_decode_step_prepare")

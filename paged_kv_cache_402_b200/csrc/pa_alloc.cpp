@@ -311,20 +311,23 @@ PA_API pa_status pa_block_refcount(pa_allocator *a, int32_t block, int32_t *refc
 
 PA_API pa_status pa_share_plan(const int32_t *tables_host, int32_t max_blocks,
                                const int32_t *lens_host, int32_t n_seqs, int32_t block_size,
-                               int32_t max_members, int32_t *members_host, int32_t *parts_host,
-                               int32_t *first_part_host, int32_t *n_groups) {
+                               int32_t partition_tokens, int32_t max_members, int32_t *members_host,
+                               int32_t *parts_host, int32_t *first_part_host, int32_t *n_groups) {
+  if (partition_tokens == 0) partition_tokens = PA_PARTITION_TOKENS;
   if (n_seqs < 0 || max_blocks < 0 || !n_groups || max_members < 2 || max_members > 4 ||
-      (block_size != 8 && block_size != 16 && block_size != 32))
+      (block_size != 8 && block_size != 16 && block_size != 32) ||
+      (partition_tokens != 256 && partition_tokens != 512 && partition_tokens != 1024))
     return PA_ERR_INVALID_ARG;
+  const int32_t part = partition_tokens;
   if (n_seqs > 0 && (!tables_host || !lens_host || !members_host || !parts_host || !first_part_host))
     return PA_ERR_INVALID_ARG;
   *n_groups = 0;
-  const int32_t bpp = PA_PARTITION_TOKENS / block_size;  // table entries per partition
+  const int32_t bpp = part / block_size;  // table entries per partition
   for (int32_t b = 0; b < n_seqs; ++b) first_part_host[b] = 0;
   // sequences with at least two partitions (the first one whole, not the last)
   std::vector<int32_t> cand;
   for (int32_t b = 0; b < n_seqs; ++b)
-    if (lens_host[b] > PA_PARTITION_TOKENS && max_blocks >= bpp) cand.push_back(b);
+    if (lens_host[b] > part && max_blocks >= bpp) cand.push_back(b);
   auto row = [&](int32_t b) { return tables_host + (size_t)b * max_blocks; };
   // buckets: equal first-partition entries, sequence order inside a bucket.
   // Sequences are ordered by a hash of those entries (FNV-1a), then inside
@@ -367,7 +370,7 @@ PA_API pa_status pa_share_plan(const int32_t *tables_host, int32_t max_blocks,
       // leading partitions that agree, are whole and come before every member's last
       int32_t parts = 0;
       for (;; ++parts) {
-        const int64_t end_tok = (int64_t)(parts + 1) * PA_PARTITION_TOKENS;
+        const int64_t end_tok = (int64_t)(parts + 1) * part;
         if ((int64_t)(parts + 1) * bpp > max_blocks) break;
         bool ok = true;
         for (size_t k = g0; k < g1 && ok; ++k) {
@@ -390,7 +393,8 @@ PA_API pa_status pa_share_plan(const int32_t *tables_host, int32_t max_blocks,
 }
 
 PA_API pa_status pa_decode_step_prepare(pa_allocator *a, const int32_t *seqs, int32_t n_seqs,
-                                        int32_t max_blocks, int32_t share_max_members,
+                                        int32_t max_blocks, int32_t partition_tokens,
+                                        int32_t share_max_members,
                                         int32_t *tables_host, int32_t *lens_host,
                                         int32_t *cow_src_host, int32_t *members_host,
                                         int32_t *parts_host, int32_t *first_part_host,
@@ -400,6 +404,8 @@ PA_API pa_status pa_decode_step_prepare(pa_allocator *a, const int32_t *seqs, in
     return PA_ERR_INVALID_ARG;
   if (share_max_members != 0 &&
       (share_max_members < 2 || share_max_members > 4 || (n_seqs > 1 && (!members_host || !parts_host))))
+    return PA_ERR_INVALID_ARG;
+  if (partition_tokens != 0 && partition_tokens != 256 && partition_tokens != 512 && partition_tokens != 1024)
     return PA_ERR_INVALID_ARG;
   *n_groups = 0;
   *n_copies = 0;
@@ -442,8 +448,8 @@ PA_API pa_status pa_decode_step_prepare(pa_allocator *a, const int32_t *seqs, in
     for (int32_t i = 0; i < n_seqs; ++i) first_part_host[i] = 0;
     return PA_OK;
   }
-  return pa_share_plan(tables_host, max_blocks, lens_host, n_seqs, bs, share_max_members, members_host,
-                       parts_host, first_part_host, n_groups);
+  return pa_share_plan(tables_host, max_blocks, lens_host, n_seqs, bs, partition_tokens, share_max_members,
+                       members_host, parts_host, first_part_host, n_groups);
 }
 
 PA_API pa_status pa_cow_sources(const int32_t *pairs_host, int32_t n_pairs,

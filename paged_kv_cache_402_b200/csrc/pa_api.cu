@@ -33,8 +33,16 @@ pa_status check_cache(const pa_cache_t *c) {
   if (c->block_size != 8 && c->block_size != 16 && c->block_size != 32) return PA_ERR_UNSUPPORTED;
   if (c->head_dim != 64 && c->head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (!aligned16(c->k) || !aligned16(c->v)) return PA_ERR_INVALID_ARG;
+  if (c->partition_tokens != 0 && c->partition_tokens != 256 && c->partition_tokens != 512 &&
+      c->partition_tokens != 1024)
+    return PA_ERR_UNSUPPORTED;
   return PA_OK;
 }
+
+// Tokens per split-context partition of decode calls over the pool.
+inline int32_t part_of(const pa_cache_t *c) { return c->partition_tokens ? c->partition_tokens : pa::kPart; }
+
+inline bool part_ok(int32_t part) { return part == 256 || part == 512 || part == 1024; }
 
 // The CUDA error behind this thread's most recent PA_ERR_CUDA (0: none).
 thread_local int32_t g_last_cuda_error = 0;
@@ -73,9 +81,9 @@ pa_status launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
   return launch_status();
 }
 
-inline int32_t max_parts_for(int32_t max_context_len) {
+inline int32_t max_parts_for(int32_t max_context_len, int32_t part) {
   // in 64 bits: a length near INT32_MAX must not wrap before the division
-  return (int32_t)(((int64_t)max_context_len + pa::kPart - 1) / pa::kPart);
+  return (int32_t)(((int64_t)max_context_len + part - 1) / part);
 }
 
 inline size_t round16(size_t x) { return (x + 15) & ~(size_t)15; }
@@ -119,9 +127,9 @@ bool ensure_smem(Kernel kern, int bytes, std::atomic<int> (&done)[kMaxDev]) {
 
 
 // workspace layout: m [B*Hq*P] f32 | l [B*Hq*P] f32 | acc [B*Hq*P*D] f32
-size_t workspace_bytes_for(int64_t B, int64_t Hq, int32_t max_ctx, int64_t D) {
-  if (max_ctx <= pa::kPart) return 0;
-  const int64_t rows = B * Hq * (int64_t)max_parts_for(max_ctx);
+size_t workspace_bytes_for(int64_t B, int64_t Hq, int32_t max_ctx, int64_t D, int32_t part) {
+  if (max_ctx <= part) return 0;
+  const int64_t rows = B * Hq * (int64_t)max_parts_for(max_ctx, part);
   return round16(rows * 4) * 2 + round16(rows * D * 4);
 }
 
@@ -256,7 +264,7 @@ bool tc_eligible(const pa::DecodeParams &p, int dtype, int D) {
   return true;  // a missing tensor-map encoder then fails the launch loudly (PA_ERR_CUDA)
 }
 
-template <int G>
+template <int G, int PART>
 pa_status launch_decode_tc_slice(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
   CUtensorMap mk, mv, mq;
   const uint64_t rows = (uint64_t)p.num_blocks * p.Hkv * p.bs;
@@ -264,7 +272,7 @@ pa_status launch_decode_tc_slice(const pa::DecodeParams &p, int32_t max_parts, c
       !make_map_pool_4d(&mv, p.v, rows, (uint32_t)p.bs) ||
       !make_map_bf16_d128(&mq, p.q, (uint64_t)p.B * p.Hq, (uint32_t)G))
     return PA_ERR_CUDA;
-  auto kern = pa::decode_partition_tc<G>;
+  auto kern = pa::decode_partition_tc<G, PART>;
   const int smem = pa::TcLayout::kBytes;
   static std::atomic<int> smem_set[kMaxDev] = {};
   if (!ensure_smem(kern, smem, smem_set)) return PA_ERR_CUDA;
@@ -281,7 +289,7 @@ pa_status launch_decode_tc_slice(const pa::DecodeParams &p, int32_t max_parts, c
 // sequence tables runs as consecutive launches over slices of it.
 std::atomic<uint32_t> g_sched_ticket{0};
 
-template <int G>
+template <int G, int PART>
 pa_status launch_decode_tc_g(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
   // a slice is at most kMaxSeqs sequences, and its full partitions must fit
   // the 20-bit counts of the kernel's packed prefix sums
@@ -308,7 +316,7 @@ pa_status launch_decode_tc_g(const pa::DecodeParams &p, int32_t max_parts, cudaS
       ps.ws_acc = p.ws_acc + rows * max_parts * 128;
     }
     ps.sched_slot = (int32_t)(g_sched_ticket.fetch_add(1) % pa::kSchedSlots);
-    const pa_status s = launch_decode_tc_slice<G>(ps, max_parts, st);
+    const pa_status s = launch_decode_tc_slice<G, PART>(ps, max_parts, st);
     if (s != PA_OK) return s;
   }
   return PA_OK;
@@ -316,7 +324,7 @@ pa_status launch_decode_tc_g(const pa::DecodeParams &p, int32_t max_parts, cudaS
 
 // The cascade kernel over the shared partitions of a sharing plan, in
 // slices of at most kMaxGroups groups.
-template <int G>
+template <int G, int PART>
 pa_status launch_decode_shared_g(const pa::DecodeParams &p, const pa_share_plan_t &plan, cudaStream_t st) {
   CUtensorMap mk, mv, mq;
   const uint64_t rows = (uint64_t)p.num_blocks * p.Hkv * p.bs;
@@ -324,7 +332,7 @@ pa_status launch_decode_shared_g(const pa::DecodeParams &p, const pa_share_plan_
       !make_map_pool_4d(&mv, p.v, rows, (uint32_t)p.bs) ||
       !make_map_bf16_d128(&mq, p.q, (uint64_t)p.B * p.Hq, (uint32_t)G))
     return PA_ERR_CUDA;
-  auto kern = pa::decode_shared_tc<G>;
+  auto kern = pa::decode_shared_tc<G, PART>;
   const int smem = pa::ShLayout::kBytes;
   static std::atomic<int> smem_set[kMaxDev] = {};
   if (!ensure_smem(kern, smem, smem_set)) return PA_ERR_CUDA;
@@ -344,12 +352,22 @@ pa_status launch_decode_shared_g(const pa::DecodeParams &p, const pa_share_plan_
   return PA_OK;
 }
 
-pa_status launch_decode_shared(const pa::DecodeParams &p, const pa_share_plan_t &plan, cudaStream_t st) {
+template <int PART>
+pa_status launch_decode_shared_p(const pa::DecodeParams &p, const pa_share_plan_t &plan, cudaStream_t st) {
   switch (p.G) {
-    case 1: return launch_decode_shared_g<1>(p, plan, st);
-    case 2: return launch_decode_shared_g<2>(p, plan, st);
-    case 4: return launch_decode_shared_g<4>(p, plan, st);
-    case 8: return launch_decode_shared_g<8>(p, plan, st);
+    case 1: return launch_decode_shared_g<1, PART>(p, plan, st);
+    case 2: return launch_decode_shared_g<2, PART>(p, plan, st);
+    case 4: return launch_decode_shared_g<4, PART>(p, plan, st);
+    case 8: return launch_decode_shared_g<8, PART>(p, plan, st);
+    default: return PA_ERR_UNSUPPORTED;
+  }
+}
+
+pa_status launch_decode_shared(const pa::DecodeParams &p, const pa_share_plan_t &plan, cudaStream_t st) {
+  switch (p.part) {
+    case 256: return launch_decode_shared_p<256>(p, plan, st);
+    case 512: return launch_decode_shared_p<512>(p, plan, st);
+    case 1024: return launch_decode_shared_p<1024>(p, plan, st);
     default: return PA_ERR_UNSUPPORTED;
   }
 }
@@ -386,12 +404,22 @@ pa_status launch_prefill_g(const pa::DecodeParams &p, const int32_t *qstart, int
   return PA_OK;
 }
 
-pa_status launch_decode_tc(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
+template <int PART>
+pa_status launch_decode_tc_p(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
   switch (p.G) {
-    case 1: return launch_decode_tc_g<1>(p, max_parts, st);
-    case 2: return launch_decode_tc_g<2>(p, max_parts, st);
-    case 4: return launch_decode_tc_g<4>(p, max_parts, st);
-    case 8: return launch_decode_tc_g<8>(p, max_parts, st);
+    case 1: return launch_decode_tc_g<1, PART>(p, max_parts, st);
+    case 2: return launch_decode_tc_g<2, PART>(p, max_parts, st);
+    case 4: return launch_decode_tc_g<4, PART>(p, max_parts, st);
+    case 8: return launch_decode_tc_g<8, PART>(p, max_parts, st);
+    default: return PA_ERR_UNSUPPORTED;
+  }
+}
+
+pa_status launch_decode_tc(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
+  switch (p.part) {
+    case 256: return launch_decode_tc_p<256>(p, max_parts, st);
+    case 512: return launch_decode_tc_p<512>(p, max_parts, st);
+    case 1024: return launch_decode_tc_p<1024>(p, max_parts, st);
     default: return PA_ERR_UNSUPPORTED;
   }
 }
@@ -478,10 +506,17 @@ PA_API pa_status pa_check_copy_pairs(const int32_t *pairs, int32_t num_pairs, in
   return PA_OK;
 }
 
+PA_API size_t pa_decode_workspace_size_p(int32_t num_seqs, int32_t num_q_heads,
+                                         int32_t max_context_len, int32_t head_dim,
+                                         int32_t partition_tokens) {
+  const int32_t part = partition_tokens ? partition_tokens : pa::kPart;
+  if (num_seqs <= 0 || num_q_heads <= 0 || max_context_len <= 0 || head_dim <= 0 || !part_ok(part)) return 0;
+  return workspace_bytes_for(num_seqs, num_q_heads, max_context_len, head_dim, part);
+}
+
 PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
                                        int32_t max_context_len, int32_t head_dim) {
-  if (num_seqs <= 0 || num_q_heads <= 0 || max_context_len <= 0 || head_dim <= 0) return 0;
-  return workspace_bytes_for(num_seqs, num_q_heads, max_context_len, head_dim);
+  return pa_decode_workspace_size_p(num_seqs, num_q_heads, max_context_len, head_dim, pa::kPart);
 }
 
 }  // extern "C"
@@ -513,13 +548,14 @@ pa_status prepare_decode(const void *q, const pa_cache_t *cache, const int32_t *
   if (num_seqs > 65535 || cache->num_kv_heads > 65535) return PA_ERR_INVALID_ARG;
   const int32_t bs = cache->block_size;
   if ((int64_t)max_context_len > (int64_t)max_blocks_per_seq * bs) return PA_ERR_INVALID_ARG;
-  if (max_context_len > INT32_MAX - pa::kPart) return PA_ERR_INVALID_ARG;
-  const size_t need = workspace_bytes_for(num_seqs, num_q_heads, max_context_len, cache->head_dim);
+  const int32_t part = part_of(cache);
+  if (max_context_len > INT32_MAX - part) return PA_ERR_INVALID_ARG;
+  const size_t need = workspace_bytes_for(num_seqs, num_q_heads, max_context_len, cache->head_dim, part);
   if (need > 0) {
     if (!workspace || !aligned16(workspace)) return PA_ERR_INVALID_ARG;
     if (workspace_bytes < need) return PA_ERR_TOO_SMALL;
   }
-  const int32_t max_parts = max_context_len > 0 ? max_parts_for(max_context_len) : 1;
+  const int32_t max_parts = max_context_len > 0 ? max_parts_for(max_context_len, part) : 1;
 
   pa::DecodeParams p{};
   p.q = q;
@@ -544,6 +580,7 @@ pa_status prepare_decode(const void *q, const pa_cache_t *cache, const int32_t *
   p.B = num_seqs;
   p.max_ctx = max_context_len;
   p.max_parts = max_parts;
+  p.part = part;
   p.scale_log2 = scale * 1.4426950408889634f;
   *pp = p;
   return PA_OK;
@@ -784,9 +821,10 @@ PA_API pa_status pa_decode_static_workspace(const void *q, const pa_cache_t *cac
   // the range checks pa_decode makes, before the scratch size is computed
   if (num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0 || cache->head_dim <= 0)
     return PA_ERR_INVALID_ARG;
-  if (num_seqs > 65535 || max_context_len > INT32_MAX - pa::kPart) return PA_ERR_INVALID_ARG;
+  const int32_t part = part_of(cache);
+  if (num_seqs > 65535 || max_context_len > INT32_MAX - part) return PA_ERR_INVALID_ARG;
   const size_t need =
-      num_seqs > 0 ? workspace_bytes_for(num_seqs, num_q_heads, max_context_len, cache->head_dim) : 0;
+      num_seqs > 0 ? workspace_bytes_for(num_seqs, num_q_heads, max_context_len, cache->head_dim, part) : 0;
   if (need > (size_t)PA_STATIC_WORKSPACE_BYTES) return PA_ERR_TOO_SMALL;
   void *ws = nullptr;
   if (need > 0) {
@@ -915,15 +953,16 @@ PA_API pa_status pa_decode_step(pa_allocator *a, const int32_t *seqs_host, int32
   // for the table width is refused by the preparation itself)
   if (num_q_heads % cache->num_kv_heads) return PA_ERR_INVALID_ARG;
   const int64_t ctx_cap = (int64_t)max_blocks * cache->block_size;
-  if (ctx_cap > INT32_MAX - pa::kPart) return PA_ERR_INVALID_ARG;
+  const int32_t part = part_of(cache);
+  if (ctx_cap > INT32_MAX - part) return PA_ERR_INVALID_ARG;
   const size_t need_ws =
-      n_seqs > 0 ? workspace_bytes_for(n_seqs, num_q_heads, (int32_t)ctx_cap, cache->head_dim) : 0;
+      n_seqs > 0 ? workspace_bytes_for(n_seqs, num_q_heads, (int32_t)ctx_cap, cache->head_dim, part) : 0;
   if (need_ws > 0 && (!slot->workspace || slot->workspace_bytes < need_ws)) return PA_ERR_TOO_SMALL;
   char *h = static_cast<char *>(slot->host);
   char *d = static_cast<char *>(slot->dev);
   auto hi = [&](size_t off) { return reinterpret_cast<int32_t *>(h + off); };
   auto di = [&](size_t off) { return reinterpret_cast<int32_t *>(d + off); };
-  s = pa_decode_step_prepare(a, seqs_host, n_seqs, max_blocks, share_max_members, hi(L.tables), hi(L.lens),
+  s = pa_decode_step_prepare(a, seqs_host, n_seqs, max_blocks, part, share_max_members, hi(L.tables), hi(L.lens),
                              hi(L.cow_src), hi(L.members), hi(L.parts), hi(L.first_part), n_groups, n_copies,
                              max_len);
   if (s != PA_OK || n_seqs == 0) return s;

@@ -59,7 +59,7 @@ struct ShLayout {
   static constexpr int kOffTmem = kOffRedSum + kRedFloats * 4;
   // unit slot: [group, kv head, partition, members, b_0 .. b_3] + the table
   // entries of the partition (from the first member's table)
-  static constexpr int kUnitInts = 8 + kPart / 8;
+  static constexpr int kUnitInts = 8 + TcLayout::kMaxPart / 8;
   static constexpr int kOffUnit = kOffTmem + 16;
   static constexpr int kOffScan = kOffUnit + 2 * kUnitInts * 4;
   static constexpr int kOffPrefix = kOffScan + 64;  // shared partitions before each group
@@ -95,7 +95,8 @@ struct SharedParams {
 // One CTA of 320 threads per SM.  Each of the SM's four sub-partitions
 // holds 16 K registers and three of the ten warps land on two of them, so a
 // thread gets at most 168.
-template <int G>
+// PART: tokens per partition (256, 512 or 1024); the caller's p.part.
+template <int G, int PART>
 __global__ void __launch_bounds__(ShLayout::kThreads, 1)
     decode_shared_tc(const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v,
@@ -103,6 +104,8 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
   using L = ShLayout;
   constexpr int N = L::kN;
   static_assert(G >= 1 && G <= 8, "group size");
+  static_assert(PART == 256 || PART == 512 || PART == 1024, "partition size");
+  constexpr int NE = PART / 8 / 32;  // table entries per lane of a unit (bs >= 8)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
 
@@ -197,7 +200,7 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
     const uint64_t pol_q = tc::policy_evict_last();
     const int bs = p.bs;
     const int blocks_per_chunk = L::kChunk / bs;
-    const int nb_unit = kPart / bs;  // blocks of a (whole) partition
+    const int nb_unit = PART / bs;  // blocks of a (whole) partition
     const int oob_group = p.num_blocks * p.Hkv * (bs / 8);
     int c = 0, qi = 0;
     bool ok = true;
@@ -206,8 +209,15 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
       int j, g, part, nmem;
       int32_t b[L::kSlots];
     };
-    auto load_unit = [&](int u, ShUnit &un, int32_t &x0, int32_t &x1) {
-      x0 = x1 = -1;
+    auto pick = [](const int32_t (&x)[NE], int k) {  // x[k] by selects, never a local-memory index
+      int32_t v = x[0];
+#pragma unroll
+      for (int i = 1; i < NE; ++i) v = select_i32(k == i, x[i], v);
+      return v;
+    };
+    auto load_unit = [&](int u, ShUnit &un, int32_t (&x)[NE]) {
+#pragma unroll
+      for (int k = 0; k < NE; ++k) x[k] = -1;
       un.nmem = 0;
       if (u >= num_units) return;
       const int w = u / p.Hkv;
@@ -229,13 +239,14 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
       un.nmem = nmem;
       if (nmem == 0) return;
       const int32_t *tr = p.tables + (size_t)un.b[0] * p.max_blocks + (size_t)un.part * nb_unit;
-      if (lane < nb_unit) x0 = tr[lane];
-      if (lane + 32 < nb_unit) x1 = tr[lane + 32];
+#pragma unroll
+      for (int k = 0; k < NE; ++k)
+        if (lane + 32 * k < nb_unit) x[k] = tr[lane + 32 * k];
     };
     ShUnit un{}, nx{};
-    int32_t e0, e1, f0, f1;
+    int32_t e[NE], f[NE];
     int u = blockIdx.x;
-    load_unit(u, un, e0, e1);
+    load_unit(u, un, e);
     wait_prior_grid();  // the copies read the pool and Q, which may be written just before
     allow_next_grid();
     while (ok && u < num_units) {
@@ -256,8 +267,8 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
 #pragma unroll
             for (int m = 0; m < L::kSlots; ++m) us[4 + m] = un.b[m];
           }
-          us[8 + lane] = e0;
-          if (L::kUnitInts > 8 + 32 + lane) us[8 + 32 + lane] = e1;
+#pragma unroll
+          for (int k = 0; k < NE; ++k) us[8 + 32 * k + lane] = e[k];
           __syncwarp();
         }
         if (lane == 0) {
@@ -270,7 +281,7 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
           }
         }
         ++qi;
-        for (int ci = 0; ci < kPart / L::kChunk; ++ci, ++c) {
+        for (int ci = 0; ci < PART / L::kChunk; ++ci, ++c) {
           const int slot = c % L::kStages, use = c / L::kStages;
           for (int which = 0; which < 2; ++which) {  // 0: K ring, 1: V ring
             uint64_t *empty = which ? &vempty[slot] : &kempty[slot];
@@ -281,10 +292,8 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
             if (lane == 0) mbar_arrive_expect_tx(full, L::kTile);
             __syncwarp();
             const int jloc = ci * blocks_per_chunk + (lane % blocks_per_chunk);
-            const int32_t a0 = __shfl_sync(0xffffffffu, e0, jloc & 31);
-            const int32_t a1 = __shfl_sync(0xffffffffu, e1, jloc & 31);
+            const int32_t blk = __shfl_sync(0xffffffffu, pick(e, (ci * blocks_per_chunk) >> 5), jloc & 31);
             if (lane < blocks_per_chunk) {
-              const int32_t blk = jloc < 32 ? a0 : a1;
               int w = oob_group;
               if (blk >= 0 && blk < p.num_blocks) w = (blk * p.Hkv + un.g) * (bs / 8);
               else if (which == 0) raise_error(PA_DEVERR_TABLE);
@@ -293,17 +302,17 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
           }
           if (!ok) break;
           if (ci == 1) {
-            load_unit(u + gridDim.x, nx, f0, f1);
+            load_unit(u + gridDim.x, nx, f);
             have_next = true;
           }
         }
         if (!ok) break;
       }
-      if (!have_next) load_unit(u + gridDim.x, nx, f0, f1);
+      if (!have_next) load_unit(u + gridDim.x, nx, f);
       u += gridDim.x;
       un = nx;
-      e0 = f0;
-      e1 = f1;
+#pragma unroll
+      for (int k = 0; k < NE; ++k) e[k] = f[k];
     }
     if (ok) {  // no work left: an empty unit stops the consumers
       const int qs = qi & 1;
@@ -368,7 +377,7 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
       if (!warp_wait(&qfull[qs], (qi >> 1) & 1)) { ok = false; break; }
       if (unit_slots[qs * L::kUnitInts + 3] == 0) break;  // the producer ran out of work
       const uint32_t qb = qbase0 + qs * L::kQ;
-      constexpr int nchunks = kPart / L::kChunk;
+      constexpr int nchunks = PART / L::kChunk;
       for (int ci = 0; ci < nchunks; ++ci, ++c) {
         const int slot = c % L::kStages;
         if (!warp_wait(&kfull[slot], (c / L::kStages) & 1)) { ok = false; break; }
@@ -500,7 +509,7 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
         m[j] = -INFINITY;
         l[j] = 0.f;
       }
-      constexpr int nchunks = kPart / L::kChunk;
+      constexpr int nchunks = PART / L::kChunk;
       for (int ci = 0; ci < nchunks; ++ci, ++c) {
         float s[NC];
         warp_wait(&sfull[c & 1], (c >> 1) & 1);

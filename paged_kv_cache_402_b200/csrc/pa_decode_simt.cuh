@@ -8,7 +8,7 @@
 // attention arithmetic is the textbook decode step with an online softmax;
 // scores are kept in base-2 units (the host folds log2(e) into the scale).
 //
-// Work unit = (partition of PA_PARTITION_TOKENS tokens, kv head g, sequence b),
+// Work unit = (partition of p.part tokens, kv head g, sequence b),
 // one CTA of 4 warps.  Warp w takes the unit's blocks w, w+4, w+8, ...; each
 // warp runs its own ring of `nstages` shared-memory slots filled by 1-D bulk
 // copies (TMA engine) of whole (block, kv head) tiles, K and V, which are
@@ -37,6 +37,7 @@ struct DecodeParams {
   float *ws_l;    // [B][Hq][max_parts] sum of weights
   float *ws_acc;  // [B][Hq][max_parts][D] unnormalised accumulator
   int32_t num_blocks, Hkv, bs, Hq, G, max_blocks, B, max_ctx, max_parts;
+  int32_t part;  // tokens per split-context partition (256, 512 or 1024)
   int32_t sched_slot;  // tensor-core kernel: which run-time work counter this call uses
   float scale_log2;  // scale * log2(e)
   // fused step (tensor-core kernel): the newest token's rows [B][Hkv][D] and
@@ -56,7 +57,7 @@ struct DecodeParams {
   int32_t late_wait;
 };
 
-constexpr int kPart = PA_PARTITION_TOKENS;
+constexpr int kPart = PA_PARTITION_TOKENS;  // the default partition size
 constexpr int kWarps = 4;
 
 __device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
@@ -94,10 +95,10 @@ __global__ void __launch_bounds__(kWarps * 32)
         store_out(out + ((size_t)b * p.Hq + g * G) * D + i, 0.f);
     return;
   }
-  const int t0 = part * kPart;
+  const int t0 = part * p.part;
   if (t0 >= ctx) return;
-  const int t1 = min(t0 + kPart, ctx);
-  const int nparts = (ctx + kPart - 1) / kPart;
+  const int t1 = min(t0 + p.part, ctx);
+  const int nparts = (ctx + p.part - 1) / p.part;
   const int j0 = t0 / bs;
   const int nblk = (t1 - t0 + bs - 1) / bs;
   const uint32_t tile_elems = (uint32_t)bs * D;
@@ -338,8 +339,8 @@ __global__ void __launch_bounds__(128) decode_reduce(DecodeParams p) {
   const int bh = blockIdx.x;
   const int b = bh / p.Hq;
   const int ctx = p.lens[b];
-  if (ctx <= kPart || ctx > p.max_ctx) return;  // written directly by the partition kernel
-  const int np = (ctx + kPart - 1) / kPart;
+  if (ctx <= p.part || ctx > p.max_ctx) return;  // written directly by the partition kernel
+  const int np = (ctx + p.part - 1) / p.part;
   const float *m = p.ws_m + (size_t)bh * p.max_parts;
   const float *l = p.ws_l + (size_t)bh * p.max_parts;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -415,8 +416,8 @@ __global__ void __launch_bounds__(kReduceRowWarps * 32, 2) decode_reduce_rows(De
   T *out = reinterpret_cast<T *>(p.out);
   for (int64_t bh = (int64_t)blockIdx.x * kReduceRowWarps + (threadIdx.x >> 5); bh < rows; bh += stride) {
     const int ctx = p.lens[bh / p.Hq];
-    if (ctx <= kPart || ctx > p.max_ctx) continue;  // written directly by the partition kernel
-    const int np = min((ctx + kPart - 1) / kPart, NP);
+    if (ctx <= p.part || ctx > p.max_ctx) continue;  // written directly by the partition kernel
+    const int np = min((ctx + p.part - 1) / p.part, NP);
     const float mi = lane < np ? __ldcg(p.ws_m + bh * p.max_parts + lane) : -INFINITY;
     const float li = lane < np ? __ldcg(p.ws_l + bh * p.max_parts + lane) : 0.f;
     const float *acc = p.ws_acc + bh * p.max_parts * D + lane * E;

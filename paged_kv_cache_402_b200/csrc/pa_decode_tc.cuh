@@ -86,10 +86,11 @@ struct TcLayout {
   //  copy-on-write source of that block or -1, 0] + the unit's table entries
   // (as the copies read them)
   static constexpr int kUnitHead = 10;
-  static constexpr int kUnitInts = kUnitHead + kPart / 8;
+  static constexpr int kMaxPart = 1024;  // the largest partition built (256, 512 or 1024 tokens)
+  static constexpr int kUnitInts = kUnitHead + kMaxPart / 8;
   static constexpr int kOffUnit = kOffTmem + 16;
-  static constexpr int kOffScan = kOffUnit + 2 * kUnitInts * 4;  // 8 ints
-  static constexpr int kOffPrefix = kOffScan + 32;
+  static constexpr int kOffScan = kOffUnit + 2 * kUnitInts * 4;  // 3 x 8 ints
+  static constexpr int kOffPrefix = kOffScan + 96;
   static constexpr int kOffCtx = kOffPrefix + (kMaxSeqs + 1) * 4;
   static constexpr int kOffFirst = kOffCtx + kMaxSeqs * 4;  // first partition of each sequence
   static constexpr int kBytes = kOffFirst + kMaxSeqs * 4 + 1024;  // + base alignment slack
@@ -171,6 +172,7 @@ constexpr float kLazyRescale = 8.0f;
 
 struct TcUnit {
   int b, g, part, t0, t1, nchunks;
+  int hg;  // kv heads of the unit: g .. g + hg - 1 (1 for a full partition)
   bool single;
 };
 
@@ -188,15 +190,20 @@ __device__ __forceinline__ int pp_of(int32_t v) { return (int)((uint32_t)v >> kF
 
 // Unit u of the largest-first order: units [0, F) are the full partitions
 // (sequence-major, kv head fastest; a sequence's start at its first
-// partition), units [F, F + P) the partial ones.
+// partition), one kv head each; units [F, F + P) the partial last
+// partitions, each of tail_hg consecutive kv heads of one sequence
+// (Hkv / tail_hg units per sequence).
+template <int PART>
 __device__ __forceinline__ TcUnit tc_unit_at(const DecodeParams &p, const int32_t *prefix,
                                              const int32_t *ctx_s, const int32_t *first_s, int u,
-                                             int num_full) {
+                                             int num_full, int tail_hg) {
   TcUnit un;
   const bool full = u < num_full;
   const int v = full ? u : u - num_full;
-  const int w = v / p.Hkv;
-  un.g = v - w * p.Hkv;
+  const int per_seq = full ? p.Hkv : p.Hkv / tail_hg;
+  const int w = v / per_seq;
+  un.hg = full ? 1 : tail_hg;
+  un.g = (v - w * per_seq) * un.hg;
   int lo = 0, hi = p.B - 1;  // largest b whose count before it is <= w
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -205,12 +212,23 @@ __device__ __forceinline__ TcUnit tc_unit_at(const DecodeParams &p, const int32_
   }
   un.b = lo;
   const int ctx = ctx_s[lo];
-  un.part = full ? first_s[lo] + w - pf_of(prefix[lo]) : ctx / kPart;
-  un.t0 = un.part * kPart;
-  un.t1 = min(un.t0 + kPart, ctx);
+  un.part = full ? first_s[lo] + w - pf_of(prefix[lo]) : ctx / PART;
+  un.t0 = un.part * PART;
+  un.t1 = min(un.t0 + PART, ctx);
   un.nchunks = (un.t1 - un.t0 + TcLayout::kChunk - 1) / TcLayout::kChunk;
-  un.single = ctx <= kPart;
+  un.single = ctx <= PART;
   return un;
+}
+
+// c ? a : b as one selp the compiler keeps: a chain of these over a small
+// register array stays in registers (a plain ?: chain may be turned back
+// into an indexed load from local memory).
+__device__ __forceinline__ int32_t select_i32(bool c, int32_t a, int32_t b) {
+  int32_t r;
+  asm("{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %3, 0;\n\tselp.b32 %0, %1, %2, q;\n\t}"
+      : "=r"(r)
+      : "r"(a), "r"(b), "r"((int)c));
+  return r;
 }
 
 // OR of `pred` over the 128 softmax threads (named barrier 1).
@@ -227,7 +245,8 @@ __device__ __forceinline__ bool wg_sync_or(int pred) {
   return r != 0;
 }
 
-template <int G>
+// PART: tokens per partition (256, 512 or 1024); the caller's p.part.
+template <int G, int PART>
 __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     decode_partition_tc(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v,
@@ -235,6 +254,8 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   using L = TcLayout;
   constexpr int N = L::kN;
   static_assert(G >= 1 && G <= N, "group size");
+  static_assert(PART == 256 || PART == 512 || PART == 1024, "partition size");
+  constexpr int NE = PART / 8 / 32;  // table entries per lane of a unit (bs >= 8)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
 
@@ -288,6 +309,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   const int b_first = threadIdx.x * seg;
   int cnt[kMaxSeg];
   int mine = 0;
+  int tail_chunks = 0, tails = 0;  // chunks of this thread's partial last partitions, and their count
 #pragma unroll
   for (int i = 0; i < kMaxSeg; ++i) {
     cnt[i] = 0;
@@ -295,16 +317,20 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     if (i < seg && b < B) {
       const int ctx = p.lens[b];
       const bool ok = ctx >= 0 && ctx <= p.max_ctx;
+      if (ok && ctx % PART != 0) {
+        tail_chunks += (ctx % PART + TcLayout::kChunk - 1) / TcLayout::kChunk;
+        ++tails;
+      }
       ctx_s[b] = ctx;
       // partitions the cascade kernel did: whole ones before the last
       int fp = p.first_part ? p.first_part[b] : 0;
-      if (fp != 0 && (!ok || fp < 0 || (int64_t)fp * kPart >= ctx)) {
+      if (fp != 0 && (!ok || fp < 0 || (int64_t)fp * PART >= ctx)) {
         if (blockIdx.x == 0) raise_error(PA_DEVERR_PLAN);
         fp = 0;  // this kernel then does the whole sequence
       }
       first_s[b] = fp;
       // full partitions in the low bits, a partial last partition in the high ones
-      cnt[i] = (ok && ctx > 0) ? (ctx / kPart - fp) | ((ctx % kPart != 0 ? 1 : 0) << kFullBits) : 0;
+      cnt[i] = (ok && ctx > 0) ? (ctx / PART - fp) | ((ctx % PART != 0 ? 1 : 0) << kFullBits) : 0;
       mine += cnt[i];
       if (blockIdx.x == 0 && !ok) raise_error(PA_DEVERR_LEN);
     }
@@ -316,6 +342,15 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     if (lane >= o) incl += v;
   }
   if (lane == 31) scan[warp] = incl;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    tail_chunks += __shfl_xor_sync(0xffffffffu, tail_chunks, o);
+    tails += __shfl_xor_sync(0xffffffffu, tails, o);
+  }
+  if (lane == 0) {
+    scan[8 + warp] = tail_chunks;
+    scan[16 + warp] = tails;
+  }
   if (warp == 1) tc::tmem_alloc(tmem_slot, L::kTmemCols);
   __syncthreads();
   int run = incl - mine;
@@ -336,7 +371,27 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const int num_full = p.Hkv * pf_of(prefix[B]);
-  const int num_units = num_full + p.Hkv * pp_of(prefix[B]);
+  // A partial last partition of a few chunks is a short unit, and a unit's
+  // scheduling (the draw, the unit's lookup, its table entries) is a serial
+  // chain of the producer; so the partial partitions of one sequence go out
+  // tail_hg kv heads per unit, about a full partition's worth of chunks (the
+  // same table entries serve every head).  Every CTA takes the same
+  // decision from the same lengths; a launch keeps at least 4 units per CTA.
+  int tail_hg = 1;
+  {
+    int tc_sum = 0, tn = 0;
+    for (int w = 0; w < L::kThreads / 32; ++w) {
+      tc_sum += scan[8 + w];
+      tn += scan[16 + w];
+    }
+    if (tn > 0 && tc_sum > 0) {
+      // kv heads per unit: a full partition's chunks over the mean tail's, rounded
+      int h = min((2 * (PART / L::kChunk) * tn + tc_sum) / (2 * tc_sum), p.Hkv);
+      while (h > 1 && (p.Hkv % h != 0 || num_full + (p.Hkv / h) * tn < 4 * (int)gridDim.x)) --h;
+      tail_hg = max(h, 1);
+    }
+  }
+  const int num_units = num_full + (p.Hkv / tail_hg) * pp_of(prefix[B]);
   uint32_t *sched = g_sched + 2 * p.sched_slot;
 
   if (warp == 0) {
@@ -356,98 +411,108 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     const int oob_group = p.num_blocks * p.Hkv * (bs / 8);  // first 8-row group past the pool
     int c = 0, qi = 0;
     bool ok = true;
-    // A unit's table entries (at most 512 / 8 = 64), loaded by the lanes
-    // right after the previous unit's copies are issued.  In a fused step a
-    // unit that holds its sequence's newest token (position t1 - 1) also gets
-    // that token's block nd and the block ns to copy over it (-1: none); its
-    // loads then read the last block from ns.
-    auto load_entries = [&](int u, TcUnit &nu, int32_t &x0, int32_t &x1, int32_t &nd, int32_t &ns) {
-      x0 = x1 = -1;
+    // A unit's table entries (at most PART / 8), entry 32 k + lane in
+    // x[k] of the lane, loaded right after the previous unit's copies are
+    // issued.  In a fused step a unit that holds its sequence's newest token
+    // (position t1 - 1) also gets that token's block nd and the block ns to
+    // copy over it (-1: none); its loads then read the last block from ns.
+    auto pick = [](const int32_t (&x)[NE], int k) {  // x[k] by selects, never a local-memory index
+      int32_t v = x[0];
+#pragma unroll
+      for (int i = 1; i < NE; ++i) v = select_i32(k == i, x[i], v);
+      return v;
+    };
+    auto load_entries = [&](int u, TcUnit &nu, int32_t (&x)[NE], int32_t &nd, int32_t &ns) {
+#pragma unroll
+      for (int k = 0; k < NE; ++k) x[k] = -1;
       nd = ns = -1;
       if (u < num_units) {
-        nu = tc_unit_at(p, prefix, ctx_s, first_s, u, num_full);
+        nu = tc_unit_at<PART>(p, prefix, ctx_s, first_s, u, num_full, tail_hg);
         const int32_t *tr = p.tables + (size_t)nu.b * p.max_blocks + nu.t0 / bs;
         const int nb = (nu.t1 - nu.t0 + bs - 1) / bs;
         const bool newest = p.k_new != nullptr && nu.t1 == ctx_s[nu.b];
         const int32_t src = (newest && p.cow_src != nullptr) ? p.cow_src[nu.b] : -1;
-        if (lane < nb) x0 = tr[lane];
-        if (lane + 32 < nb) x1 = tr[lane + 32];
+#pragma unroll
+        for (int k = 0; k < NE; ++k)
+          if (lane + 32 * k < nb) x[k] = tr[lane + 32 * k];
         if (newest) {
           const int jl = (nu.t1 - 1 - nu.t0) / bs;
-          const int32_t blk = __shfl_sync(0xffffffffu, jl < 32 ? x0 : x1, jl & 31);
+          const int32_t blk = __shfl_sync(0xffffffffu, pick(x, jl >> 5), jl & 31);
           if (blk >= 0 && blk < p.num_blocks) {  // else its copy flags PA_DEVERR_TABLE
             nd = blk;
             if (src >= p.num_blocks) {
               if (lane == 0) raise_error(PA_DEVERR_PAIR);
             } else if (src >= 0) {
               ns = src;
-              if (lane == (jl & 31)) {
-                if (jl < 32) x0 = src; else x1 = src;
-              }
+#pragma unroll
+              for (int k = 0; k < NE; ++k) x[k] = select_i32(lane == (jl & 31) && k == (jl >> 5), src, x[k]);
             }
           }
         }
       }
     };
     TcUnit un{};
-    int32_t e0, e1, nd, ns;
+    int32_t e[NE], nd, ns;
     int u = blockIdx.x;  // the first unit of every CTA is fixed; later ones are drawn
-    load_entries(u, un, e0, e1, nd, ns);
+    load_entries(u, un, e, nd, ns);
     if (!p.late_wait) wait_prior_grid();  // the copies read the pool and Q, which may be written just before
     allow_next_grid();
     while (ok && u < num_units) {
       const int nb_unit = (un.t1 - un.t0 + bs - 1) / bs;
-      const int qs = qi & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((qi >> 1) & 1) ^ 1))) { ok = false; break; }
-      {  // publish the unit to the MMA lane and the softmax warpgroup
-        int32_t *us = unit_slots + qs * L::kUnitInts;
-        if (lane == 0) {
-          us[0] = un.b;
-          us[1] = un.g;
-          us[2] = un.part;
-          us[3] = un.t0;
-          us[4] = un.t1;
-          us[5] = un.nchunks;
-          us[6] = un.single;
-          us[7] = nd;
-          us[8] = ns;
-          us[9] = 0;
-        }
-        us[L::kUnitHead + lane] = e0;
-        if (L::kUnitInts > L::kUnitHead + 32 + lane) us[L::kUnitHead + 32 + lane] = e1;
-        __syncwarp();
-      }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&qfull[qs], 2 * G * 128);
-        uint8_t *qdst = smem + L::kOffQ + qs * L::kQ;
-        const int qy = un.b * p.Hq + un.g * G;
-        tc::tma_load_2d(qdst, &tmap_q, 0, qy, &qfull[qs], pol_q);
-        tc::tma_load_2d(qdst + N * 128, &tmap_q, 64, qy, &qfull[qs], pol_q);
-      }
-      ++qi;
-      for (int ci = 0; ci < un.nchunks; ++ci, ++c) {
-        const int slot = c % 3, use = c / 3;
-        for (int which = 0; which < 2; ++which) {  // 0: K ring, 1: V ring
-          uint64_t *empty = which ? &vempty[slot] : &kempty[slot];
-          uint64_t *full = which ? &vfull[slot] : &kfull[slot];
-          const CUtensorMap *map = which ? &tmap_v : &tmap_k;
-          if (!__all_sync(0xffffffffu, mbar_wait(empty, (use & 1) ^ 1))) { ok = false; break; }
-          uint8_t *dst = smem + (which ? L::kOffV : L::kOffK) + slot * L::kTile;
-          if (lane == 0) mbar_arrive_expect_tx(full, L::kTile);
-          __syncwarp();
-          // lane j loads block j of the chunk
-          const int jloc = ci * blocks_per_chunk + (lane % blocks_per_chunk);
-          const int32_t a0 = __shfl_sync(0xffffffffu, e0, jloc & 31);
-          const int32_t a1 = __shfl_sync(0xffffffffu, e1, jloc & 31);
-          if (lane < blocks_per_chunk) {
-            const int32_t blk = jloc < 32 ? a0 : a1;
-            int w = oob_group;
-            if (jloc < nb_unit) {
-              if (blk >= 0 && blk < p.num_blocks) w = (blk * p.Hkv + un.g) * (bs / 8);
-              else if (which == 0) raise_error(PA_DEVERR_TABLE);
-            }
-            tc::tma_load_4d(dst + lane * (bs / 8) * L::kGroup, map, 0, 0, 0, w, full, pol_kv);
+      for (int hh = 0; hh < un.hg; ++hh) {  // one (sequence, kv head, partition) at a time
+        const int g = un.g + hh;
+        const int qs = qi & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((qi >> 1) & 1) ^ 1))) { ok = false; break; }
+        {  // publish the unit to the MMA lane and the softmax warpgroup
+          int32_t *us = unit_slots + qs * L::kUnitInts;
+          if (lane == 0) {
+            us[0] = un.b;
+            us[1] = g;
+            us[2] = un.part;
+            us[3] = un.t0;
+            us[4] = un.t1;
+            us[5] = un.nchunks;
+            us[6] = un.single;
+            us[7] = nd;
+            us[8] = ns;
+            us[9] = 0;
           }
+#pragma unroll
+          for (int k = 0; k < NE; ++k) us[L::kUnitHead + 32 * k + lane] = e[k];
+          __syncwarp();
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&qfull[qs], 2 * G * 128);
+          uint8_t *qdst = smem + L::kOffQ + qs * L::kQ;
+          const int qy = un.b * p.Hq + g * G;
+          tc::tma_load_2d(qdst, &tmap_q, 0, qy, &qfull[qs], pol_q);
+          tc::tma_load_2d(qdst + N * 128, &tmap_q, 64, qy, &qfull[qs], pol_q);
+        }
+        ++qi;
+        for (int ci = 0; ci < un.nchunks; ++ci, ++c) {
+          const int slot = c % 3, use = c / 3;
+          for (int which = 0; which < 2; ++which) {  // 0: K ring, 1: V ring
+            uint64_t *empty = which ? &vempty[slot] : &kempty[slot];
+            uint64_t *full = which ? &vfull[slot] : &kfull[slot];
+            const CUtensorMap *map = which ? &tmap_v : &tmap_k;
+            if (!__all_sync(0xffffffffu, mbar_wait(empty, (use & 1) ^ 1))) { ok = false; break; }
+            uint8_t *dst = smem + (which ? L::kOffV : L::kOffK) + slot * L::kTile;
+            if (lane == 0) mbar_arrive_expect_tx(full, L::kTile);
+            __syncwarp();
+            // lane j loads block j of the chunk; a chunk's entries lie in one
+            // 32-entry group (blocks_per_chunk divides 32)
+            const int jloc = ci * blocks_per_chunk + (lane % blocks_per_chunk);
+            const int32_t blk = __shfl_sync(0xffffffffu, pick(e, (ci * blocks_per_chunk) >> 5), jloc & 31);
+            if (lane < blocks_per_chunk) {
+              int w = oob_group;
+              if (jloc < nb_unit) {
+                if (blk >= 0 && blk < p.num_blocks) w = (blk * p.Hkv + g) * (bs / 8);
+                else if (which == 0 && hh == 0) raise_error(PA_DEVERR_TABLE);
+              }
+              tc::tma_load_4d(dst + lane * (bs / 8) * L::kGroup, map, 0, 0, 0, w, full, pol_kv);
+            }
+          }
+          if (!ok) break;
         }
         if (!ok) break;
       }
@@ -459,7 +524,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       int raw_next = 0;
       if (lane == 0) raw_next = (int)gridDim.x + (int)atomicAdd(sched, 1u);
       u = __shfl_sync(0xffffffffu, raw_next, 0);
-      load_entries(u, un, e0, e1, nd, ns);
+      load_entries(u, un, e, nd, ns);
     }
     if (ok) {  // no work left: publish an empty unit so the consumers stop
       const int qs = qi & 1;
@@ -707,7 +772,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       un.single = us[6] != 0;
       if (un.nchunks == 0) break;  // the producer ran out of work
       const int32_t *ents = us + L::kUnitHead;
-      const int tail_end = min(((un.t1 + bs - 1) >> log2_bs) << log2_bs, un.t0 + kPart);
+      const int tail_end = min(((un.t1 + bs - 1) >> log2_bs) << log2_bs, un.t0 + PART);
       const uint32_t obuf = trow + 2 * N + (qi & 1) * N;
       // Copy on write of the unit's newest block (fused step): the source
       // tile over the destination's, every row but the new one (the MMA warp

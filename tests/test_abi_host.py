@@ -237,6 +237,31 @@ def test_decode_step_refuses_before_the_allocator_moves():
     assert A.seq_len(s) == (600, 38)
 
 
+def test_share_plan_partition_sizes():
+    """The plan's unit of sharing is the pool's partition: two sequences
+    whose first 600 tokens sit in the same blocks (then diverge) share two
+    256-token partitions, one of 512, none of 1024 (a shared partition is
+    whole, agrees across the group, and comes before each member's last)."""
+    bs = 16
+    common = np.arange(100, 100 + 600 // bs + 1, dtype=np.int32)  # 38 blocks, the last partly shared
+    t = np.full((2, 80), -1, np.int32)
+    t[0, :38] = common[:38]
+    t[1, :38] = common[:38]
+    t[0, 37:70] = np.arange(500, 533)
+    t[1, 37:70] = np.arange(600, 633)
+    lens = np.array([1100, 1090], np.int32)
+    for part, want in ((256, 2), (512, 1), (1024, 0)):
+        plan = pa.share_plan(t, lens, bs, partition_tokens=part)
+        assert (plan.n_groups, plan.parts.tolist()) == ((1, [want]) if want else (0, [])), part
+        assert plan.first_part.tolist() == [want, want]
+    with pytest.raises(pa.PagedAttnError):
+        pa.share_plan(t, lens, bs, partition_tokens=384)
+    ws = pa.pa_decode_workspace_size
+    assert ws(2, 8, 1000, 128, 256) == 2 * ((2 * 8 * 4 * 4 + 15) // 16 * 16) + 2 * 8 * 4 * 128 * 4
+    assert ws(2, 8, 1000, 128, 1024) == 0 and ws(2, 8, 1000, 128, 384) == 0
+    assert ws(2, 8, 1000, 128) == ws(2, 8, 1000, 128, 512)
+
+
 def test_workspace_size():
     ws = pa.pa_decode_workspace_size
     assert ws(4, 8, 512, 128) == 0
