@@ -226,11 +226,11 @@ def setup_independent(seed, wl, uses, dev):
     order = synth.rng(seed + 1).permutation(NB)
     alloc = pa.Allocator(NB, bs, order)
     if wl.get("fill_used_only"):
-        cache = pa.KVCache.empty(NB, Hkv, bs, D, torch.bfloat16, dev)
+        cache = pa.KVCache.empty(NB, Hkv, bs, D, torch.bfloat16, dev, partition_tokens=wl["part"])
         _fill_blocks_normal(cache, order[:need], seed, dev)
     else:
         cache = pa.KVCache(synth.normal((NB, Hkv, bs, D), torch.bfloat16, seed + 2, device=dev),
-                           synth.normal((NB, Hkv, bs, D), torch.bfloat16, seed + 3, device=dev))
+                           synth.normal((NB, Hkv, bs, D), torch.bfloat16, seed + 3, device=dev), wl["part"])
     seqs = [alloc.new_seq() for _ in range(B)]
     alloc.batch_append(seqs, lens)  # prompt blocks; the pool's contents stand in for the prompt rows
     return alloc, cache, [seqs]
@@ -252,7 +252,7 @@ def setup_shared_prefix(seed, wl, uses, dev):
     order = np.concatenate([order, np.arange(len(order), NB)]).astype(np.int32)
     alloc = pa.Allocator(NB, bs, order)
     cache = pa.KVCache(synth.normal((NB, Hkv, bs, D), torch.bfloat16, seed + 2, device=dev),
-                       synth.normal((NB, Hkv, bs, D), torch.bfloat16, seed + 3, device=dev))
+                       synth.normal((NB, Hkv, bs, D), torch.bfloat16, seed + 3, device=dev), wl["part"])
     roots = [alloc.new_seq() for _ in range(groups)]
     alloc.batch_append(roots, pl)
     seqs = []
@@ -277,7 +277,7 @@ def setup_cow_steps(seed, wl, uses, dev):
     order = synth.rng(seed + 1).permutation(NB)
     alloc = pa.Allocator(NB, bs, order)
     cache = pa.KVCache(synth.normal((NB, Hkv, bs, D), torch.bfloat16, seed + 2, device=dev),
-                       synth.normal((NB, Hkv, bs, D), torch.bfloat16, seed + 3, device=dev))
+                       synth.normal((NB, Hkv, bs, D), torch.bfloat16, seed + 3, device=dev), wl["part"])
     r = synth.rng(seed + 5)
     sets = []
     for _ in range(uses):
@@ -320,7 +320,7 @@ class Instance:
             slots, pairs = self.alloc.batch_append(seqs, np.ones(B, np.int32))
             tables, lens = self.alloc.build_block_tables(seqs, self.max_blocks)
             cow = pa.cow_sources(pairs, tables, lens, bs)
-            plan = pa.share_plan(tables, lens, bs)
+            plan = pa.share_plan(tables, lens, bs, partition_tokens=wl["part"])
             self.host_alloc_s += time.perf_counter() - t1
             nblk = (lens.astype(np.int64) + bs - 1) // bs
             # unique bytes: every physical block once, with its fill
@@ -352,7 +352,8 @@ class Instance:
                                       + len(pairs) * 2 * bs * Hkv * D * 2 * 2 + (B * 4 if len(pairs) else 0))
             self.steps.append(st)
         top = max(st["max_ctx"] for st in self.steps)
-        ws = torch.empty(max(16, pa.pa_decode_workspace_size(B, Hq, top + 64, D)), dtype=torch.uint8, device=dev)
+        ws = torch.empty(max(16, pa.pa_decode_workspace_size(B, Hq, top + 64, D, wl["part"])), dtype=torch.uint8,
+                         device=dev)
         out = torch.empty(B, Hq, D, dtype=dt, device=dev)
         for st in self.steps:
             st["ws"], st["out"] = ws, out
@@ -405,7 +406,7 @@ def aggregate_ranks(world: int, ms: float, kv_gb: float, tokens: float, e2e_s: f
 def run_ours(args, rank: int, world: int, dev):
     import paged_kv_cache_402_b200 as pa
 
-    wl = WORKLOADS[args.workload]
+    wl = dict(WORKLOADS[args.workload], part=args.partition)
     total = args.warmup + args.steps
     # enough instances that none is used more than max_uses times (each use
     # grows every sequence by one token)
@@ -443,7 +444,7 @@ def run_ours(args, rank: int, world: int, dev):
                                 scale, cow_src=st["cow"], out=st["out"], workspace=st["ws"], stream=strm)
         if ev is not None:
             ev[1].record(strm)
-        n += 2 if st["max_ctx"] > pa.PA_PARTITION_TOKENS else 1
+        n += 2 if st["max_ctx"] > wl["part"] else 1
         return n, st
 
     for s in range(args.warmup):
@@ -536,7 +537,7 @@ def run_ours(args, rank: int, world: int, dev):
         "data": "synthetic (seeded N(0,1) q/k/v; seeded lengths and block placement)",
         "config": {"workload": wl["name"], "global_batch": wl["B"] * world, "block_size": wl["bs"],
                    "q_heads": wl["Hq"], "kv_heads": wl["Hkv"], "head_dim": wl["D"],
-                   "partition_tokens": pa.PA_PARTITION_TOKENS,
+                   "partition_tokens": wl["part"],
                    "l2": f"{R} rotating batch instances per rank (KV per step ~{kv_bytes / args.steps / 1e6:.0f} MB, "
                          f"working set ~{R * kv_bytes / args.steps / 1e6:.0f} MB > 126 MB L2)",
                    "parallelism": f"replicas x{world}",
@@ -645,7 +646,8 @@ def run_e2e(args, insts, wl, dev, stream):
 
     sets = [make_set(), make_set()]
     copy_stream = torch.cuda.Stream(device=dev)
-    ws = torch.empty(max(16, pa.pa_decode_workspace_size(B, Hq, mb * bs, D)), dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(16, pa.pa_decode_workspace_size(B, Hq, mb * bs, D, wl["part"])), dtype=torch.uint8,
+                     device=dev)
     ones = np.ones(B, np.int32)
     scale = 1.0 / math.sqrt(D)
     seen = []
@@ -894,21 +896,27 @@ def run_prefill(args, rank: int, world: int, dev):
 
 
 def choose_block_size(lines, frag_budget: float):
-    """The block-size choice from a trace sweep: the pages' trade-off is that
-    smaller blocks waste less of the last block of every sequence, larger
-    ones cost less bookkeeping and fewer, larger copies per key range
-    ("pagedattention" glossary entry, paragraph 6).  Rule: the fastest block
-    size (decode tokens per second of wall time) among those whose mean
-    fragmentation stays within the budget; the smallest block size if none
-    does."""
+    """The block-size and partition-size choice from a trace sweep.  The
+    pages' trade-off: smaller blocks waste less of the last block of every
+    sequence, larger ones cost less bookkeeping and fewer, larger copies per
+    key range ("pagedattention" glossary entry, paragraph 6).  The partition
+    size is the grain of the split-context decode and of sharing: a smaller
+    one lets a plan share more of a common prefix, at more work units per
+    step.  Rule: the fastest layout (decode tokens per second of wall time)
+    among those whose mean fragmentation stays within the budget; the
+    smallest block size if none does."""
     ok = [d for d in lines if d["fragmentation_mean"] is not None and d["fragmentation_mean"] <= frag_budget]
     pick = (max(ok, key=lambda d: d["tokens_per_s"]) if ok
-            else min(lines, key=lambda d: d["config"]["block_size"]))
+            else min(lines, key=lambda d: (d["config"]["block_size"], d["config"].get("partition_tokens", 512))))
+
+    def key(d):
+        return f"bs{d['config']['block_size']}/p{d['config'].get('partition_tokens', 512)}"
     return {
         "workload": "trace-sweep",
         "block_size_choice": pick["config"]["block_size"],
+        "partition_choice": pick["config"].get("partition_tokens", 512),
         "rule": f"fastest wall-clock decode tokens/s with mean fragmentation <= {frag_budget:.0%}",
-        "per_block_size": {str(d["config"]["block_size"]): {
+        "per_layout": {key(d): {
             "tokens_per_s": d["tokens_per_s"], "device_gbs_unique": d["value"],
             "fragmentation_mean": d["fragmentation_mean"], "device_ms_per_step": d["device_ms_per_step"]}
             for d in lines},
@@ -930,17 +938,20 @@ def run_trace(args, dev):
     row = 2 * Hkv * D * 2
     stream = torch.cuda.current_stream()
     lines = []
-    sizes = [args.block_size] if args.block_size else [8, 16, 32]
+    if args.block_size or args.partition != 512:
+        layouts = [(args.block_size or 16, args.partition)]
+    else:  # block sizes at the default partition, then partition sizes at 16-token blocks
+        layouts = [(8, 512), (16, 512), (32, 512), (16, 256), (16, 1024)]
     draws = synth.trace(args.seed, steps=args.trace_steps)
     # random rows to draw prompt / decode K, V and q from (values do not
     # change the work; the pool of rows is reused cyclically)
     src = synth.normal((1 << 16, Hkv, D), dt, 901, device=dev)
     qsrc = synth.normal((8192, Hq, D), dt, 902, device=dev)
-    for bs in sizes:
+    for bs, part in layouts:
         NB = 16 * 2**30 // (2 * Hkv * bs * D * 2)
         order = synth.rng(args.seed + bs).permutation(NB)
         A = pa.Allocator(NB, bs, order)
-        cache = pa.KVCache.empty(NB, Hkv, bs, D, dt, dev)
+        cache = pa.KVCache.empty(NB, Hkv, bs, D, dt, dev, partition_tokens=part)
         drv = BeamTrace(A, lambda: A.stats()["free_blocks"], bs, draws)
         out = torch.empty(8192, Hq, D, dtype=dt, device=dev)
         ws = torch.empty(64 << 20, dtype=torch.uint8, device=dev)
@@ -961,7 +972,8 @@ def run_trace(args, dev):
             if n:
                 max_ctx, mb = A.max_len(plan.decode_seqs)
                 tables, lens = A.build_block_tables(plan.decode_seqs, mb)
-                splan = pa.share_plan(tables, lens, bs) if not (args.unfused or args.no_share_plan) else None
+                splan = (pa.share_plan(tables, lens, bs, partition_tokens=part)
+                         if not (args.unfused or args.no_share_plan) else None)
             host_s += time.perf_counter() - t0
             if n == 0:
                 wall += time.perf_counter() - t0
@@ -979,7 +991,7 @@ def run_trace(args, dev):
             # step's first event: inputs, plan, workspace, q and out
             dplan = splan.to(dev) if splan is not None else None
             kd = src[(s_ * 131) % ((1 << 16) - n):][:n]
-            need = pa.pa_decode_workspace_size(n, Hq, max_ctx, D)
+            need = pa.pa_decode_workspace_size(n, Hq, max_ctx, D, part)
             if need > ws.numel():
                 ws = torch.empty(need * 5 // 4, dtype=torch.uint8, device=dev)
             q = qsrc[:n] if n <= 8192 else synth.normal((n, Hq, D), dt, s_, device=dev)
@@ -997,15 +1009,15 @@ def run_trace(args, dev):
                     launches += 1
                 pa.pa_append_kv(kd, kd, d_[1], cache, stream)
                 pa.pa_decode(q, cache, d_[3], d_[4], max_ctx, 1 / math.sqrt(D), out=o, workspace=ws, stream=stream)
-                launches += 2 + (1 if max_ctx > pa.PA_PARTITION_TOKENS else 0)
+                launches += 2 + (1 if max_ctx > part else 0)
             elif args.no_share_plan:
                 pa.pa_append_decode(kd, kd, q, cache, d_[3], d_[4], max_ctx, 1 / math.sqrt(D), cow_src=d_[5],
                                     out=o, workspace=ws, stream=stream)
-                launches += 1 + (1 if max_ctx > pa.PA_PARTITION_TOKENS else 0)
+                launches += 1 + (1 if max_ctx > part else 0)
             else:
                 pa.pa_decode_shared(q, cache, d_[3], d_[4], max_ctx, 1 / math.sqrt(D), plan=dplan,
                                     k_new=kd, v_new=kd, cow_src=d_[5], out=o, workspace=ws, stream=stream)
-                launches += 1 + (1 if max_ctx > pa.PA_PARTITION_TOKENS else 0) + (1 if splan.n_groups else 0)
+                launches += 1 + (1 if max_ctx > part else 0) + (1 if splan.n_groups else 0)
                 h2d += splan.nbytes
             ev[s_][1].record(stream)
             res = o[:1].to("cpu", non_blocking=True)
@@ -1033,7 +1045,7 @@ def run_trace(args, dev):
                                    "lognormal (median 512, max 4096), outputs geometric (mean 256), beam "
                                    "groups of 4 re-forked copy-on-write, 32 q / 8 kv heads, head_dim 128, "
                                    "16 GiB K+V pool",
-                       "block_size": bs, "trace_steps": steps,
+                       "block_size": bs, "partition_tokens": part, "trace_steps": steps,
                        "timing": "device: CUDA events around each step's kernels; wall: whole step incl. host"},
             "kv_logical_gbs": round(logical / 1e9 / (dec_ms / 1e3), 2),
             "kv_frac_of_hbm_peak": round(uniq / 1e9 / (dec_ms / 1e3) / peak, 4),
@@ -1196,6 +1208,9 @@ def main():
     ap.add_argument("--unfused", action="store_true",
                     help="run each step as pa_copy_blocks + pa_append_kv + pa_decode instead of pa_append_decode")
     ap.add_argument("--block-size", type=int, default=0, help="trace workload: one block size (0: 8, 16 and 32)")
+    ap.add_argument("--partition", type=int, default=512, choices=[256, 512, 1024],
+                    help="tokens per split-context partition of the decode (trace: with the default 512 the sweep "
+                         "also runs 256 and 1024 at 16-token blocks)")
     ap.add_argument("--trace-steps", type=int, default=1000)
     ap.add_argument("--frag-budget", type=float, default=0.05,
                     help="trace sweep: largest mean fragmentation a block-size choice may have")

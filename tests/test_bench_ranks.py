@@ -67,8 +67,8 @@ def test_reference_arm_prints_on_rank_zero_only(rank):
 
 
 def test_block_size_choice_rule():
-    """The fastest block size within the fragmentation budget; the smallest
-    when none fits."""
+    """The fastest layout (block size, partition size) within the
+    fragmentation budget; the smallest block size when none fits."""
     sys.path.insert(0, ROOT)
     import bench
     mk = lambda bs, tps, fr: {"config": {"block_size": bs}, "tokens_per_s": tps, "fragmentation_mean": fr,
@@ -77,7 +77,11 @@ def test_block_size_choice_rule():
     assert bench.choose_block_size(lines, 0.05)["block_size_choice"] == 16
     assert bench.choose_block_size(lines, 0.06)["block_size_choice"] == 32
     assert bench.choose_block_size(lines, 0.01)["block_size_choice"] == 8
-    assert set(bench.choose_block_size(lines, 0.05)["per_block_size"]) == {"8", "16", "32"}
+    assert set(bench.choose_block_size(lines, 0.05)["per_layout"]) == {"bs8/p512", "bs16/p512", "bs32/p512"}
+    # a partition size of the sweep wins when it is the fastest within the budget
+    lines.append(dict(mk(16, 600e3, 0.028), config={"block_size": 16, "partition_tokens": 256}))
+    pick = bench.choose_block_size(lines, 0.05)
+    assert (pick["block_size_choice"], pick["partition_choice"]) == (16, 256)
 
 
 def test_traffic_record_follows_the_kernel_sources(tmp_path, monkeypatch):
