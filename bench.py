@@ -382,6 +382,12 @@ WORKLOADS = {
              "16-token blocks scattered over an 80 GiB K+V pool, 512-token partitions + LSE reduce, +1 token per step",
         B=8, Hq=32, Hkv=8, D=128, bs=16, lengths=_lengths("long_context_lengths"), setup=setup_independent,
         num_blocks=80 * 2**30 // (2 * 8 * 16 * 128 * 2), fill_used_only=True, rotate=1, max_uses=100000),
+    "long-context-small": dict(
+        name="bf16 long-context decode, profiler-sized: the first 2 of the long-context lengths (context "
+             "~U[32768,131072]), 32 q / 8 kv heads, head_dim 128, 16-token blocks scattered over a 4 GiB K+V pool, "
+             "512-token partitions + LSE reduce, +1 token per step",
+        B=2, Hq=32, Hkv=8, D=128, bs=16, lengths=_lengths("long_context_lengths_small"), setup=setup_independent,
+        num_blocks=4 * 2**30 // (2 * 8 * 16 * 128 * 2), fill_used_only=True, rotate=1, max_uses=100000),
     "cow-step": dict(
         name="bf16 copy-on-write step: 256 seqs in groups of 8 sharing a 512+r token prefix; each step's "
              "append copies the shared partial block for 7 of 8 members (224 pairs), then decodes; "

@@ -185,6 +185,12 @@ def long_context_lengths(seed: int, B: int = 8, lo: int = 32768, hi: int = 13107
     return rng(seed).integers(lo, hi + 1, size=B).astype(np.int32)
 
 
+def long_context_lengths_small(seed: int) -> np.ndarray:
+    """The first two lengths of long_context_lengths(seed): a batch small
+    enough for a profiler capture, drawn from the same distribution."""
+    return long_context_lengths(seed)[:2]
+
+
 def scattered_blocks(seed: int, lens, bs: int, num_blocks: int) -> np.ndarray:
     """Block tables whose entries are drawn without replacement, uniformly
     from a pool of num_blocks."""
