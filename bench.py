@@ -191,7 +191,7 @@ def bandwidth_probes(dev, nbytes: int = 4 << 30, reps: int = 6):
             out = max(out, reps * bytes_per_rep / (e0.elapsed_time(e1) / 1e3) / 1e9)
         return out
 
-    read = best(lambda: torch.sum(x, dtype=torch.float32, out=acc), nbytes)
+    read = best(lambda: torch.sum(x, dim=0, dtype=torch.float32, out=acc), nbytes)
     copy = best(lambda: y.copy_(x), 2 * nbytes)
     del x, y
     torch.cuda.empty_cache()

@@ -503,9 +503,9 @@ typedef struct {
   void *out_dev;
   void *workspace;
   size_t workspace_bytes;
-  void *ev_in;      /* recorded on copy_stream once the inputs are on the device */
+  void *ev_in;      /* recorded on h2d_stream once the inputs are on the device */
   void *ev_kernel;  /* recorded on stream once the decode has run */
-  void *ev_out;     /* recorded on copy_stream once out is on the host */
+  void *ev_out;     /* recorded on d2h_stream once out is on the host */
 } pa_step_slot_t;
 
 /* Offsets (16-byte aligned) of a step's inputs in the staging area:
@@ -529,24 +529,28 @@ PA_API pa_status pa_step_slot_wait(const pa_step_slot_t *slot);
  *  1. pa_decode_step_prepare into the staging area (all or nothing: an
  *     error here, e.g. PA_ERR_OUT_OF_BLOCKS, leaves the allocator and the
  *     device untouched);
- *  2. on copy_stream, after the slot's previous decode: one cudaMemcpyAsync
+ *  2. on h2d_stream, after the slot's previous decode: one cudaMemcpyAsync
  *     of the staging area to dev, then ev_in;
  *  3. on stream, after ev_in and the slot's previous output copy:
  *     pa_decode_shared with the plan (share_max_members 2..4, or 0 for none;
  *     built for the pool's partition_tokens),
  *     the copy sources and the new rows, then ev_kernel;
- *  4. on copy_stream, after ev_kernel: cudaMemcpyAsync of out_dev to
+ *  4. on d2h_stream, after ev_kernel: cudaMemcpyAsync of out_dev to
  *     out_host, then ev_out.
  * Nothing is synchronised: call pa_step_slot_wait(slot) before rewriting
- * the slot's staging area or reading its out_host.  stream and copy_stream
- * may be the same stream.  *n_copies, *n_groups and *max_len report the
+ * the slot's staging area or reading its out_host.  Any of the three
+ * streams may be the same stream; with three distinct streams the copies of
+ * step i + 1 in and of step i out run beside the decodes (a copy stream
+ * shared by both directions would put step i + 1's inputs behind step i's
+ * output, and so behind step i's decode).  *n_copies, *n_groups and *max_len report the
  * step's copies on write, plan groups and longest context.  A CUDA error
  * after step 1 returns PA_ERR_CUDA with the allocator already advanced.
  */
 PA_API pa_status pa_decode_step(pa_allocator *a, const int32_t *seqs_host, int32_t n_seqs,
                                 int32_t max_blocks, int32_t share_max_members,
                                 const pa_cache_t *cache, int32_t num_q_heads, float scale,
-                                const pa_step_slot_t *slot, void *stream, void *copy_stream,
+                                const pa_step_slot_t *slot, void *stream, void *h2d_stream,
+                                void *d2h_stream,
                                 int32_t *n_copies, int32_t *n_groups, int32_t *max_len);
 
 /*

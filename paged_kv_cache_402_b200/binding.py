@@ -98,7 +98,7 @@ def _load() -> ctypes.CDLL:
         "pa_step_slot_release": (st, [ctypes.POINTER(pa_step_slot_t)]),
         "pa_step_slot_wait": (st, [ctypes.POINTER(pa_step_slot_t)]),
         "pa_decode_step": (st, [vp, i32p, i32, i32, i32, cp, i32, f32, ctypes.POINTER(pa_step_slot_t), vp, vp,
-                                i32p, i32p, i32p]),
+                                vp, i32p, i32p, i32p]),
         "pa_copy_blocks": (st, [vp, i32, cp, vp]),
         "pa_check_copy_pairs": (st, [i32p, i32, i32]),
         "pa_read_device_error": (st, [vp, i32p]),
@@ -513,7 +513,8 @@ class DecodeStepper:
     ``stepper.wait(slot)`` returned."""
 
     def __init__(self, alloc: "Allocator", cache: KVCache, n_seqs: int, num_q_heads: int, max_blocks: int,
-                 scale: float, share_max_members: int = 4, slots: int = 2, stream=None, copy_stream=None):
+                 scale: float, share_max_members: int = 4, slots: int = 2, stream=None, h2d_stream=None,
+                 d2h_stream=None):
         self.alloc, self.cache = alloc, cache
         self.n, self.Hq, self.max_blocks = int(n_seqs), int(num_q_heads), int(max_blocks)
         self.share, self.scale = int(share_max_members), float(scale)
@@ -543,7 +544,10 @@ class DecodeStepper:
                                 "q": view(lay.q, (self.n, self.Hq, D)), "k": view(lay.k_new, (self.n, Hkv, D)),
                                 "v": view(lay.v_new, (self.n, Hkv, D))})
         self.stream = stream if stream is not None else torch.cuda.current_stream(dev)
-        self.copy_stream = copy_stream if copy_stream is not None else torch.cuda.Stream(device=dev)
+        # inputs and outputs on streams of their own, so that step i + 1's
+        # inputs do not queue behind step i's output copy
+        self.h2d_stream = h2d_stream if h2d_stream is not None else torch.cuda.Stream(device=dev)
+        self.d2h_stream = d2h_stream if d2h_stream is not None else torch.cuda.Stream(device=dev)
         self.i = 0
         self.h2d_bytes = lay.bytes
         self.d2h_bytes = self.n * self.Hq * D * torch.tensor([], dtype=dt).element_size()
@@ -577,7 +581,8 @@ class DecodeStepper:
         nc, ng, ml = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int32(0)
         _check(_lib.pa_decode_step(self.alloc._h, _i32p(seqs), self.n, self.max_blocks, self.share,
                                    self.cache.ref(), self.Hq, self.scale, ctypes.byref(self._slots[k]["struct"]),
-                                   self.stream.cuda_stream, self.copy_stream.cuda_stream, ctypes.byref(nc),
+                                   self.stream.cuda_stream, self.h2d_stream.cuda_stream,
+                                   self.d2h_stream.cuda_stream, ctypes.byref(nc),
                                    ctypes.byref(ng), ctypes.byref(ml)), "pa_decode_step")
         self.i += 1
         return {"slot": k, "n_copies": nc.value, "n_groups": ng.value, "max_len": ml.value}

@@ -938,7 +938,8 @@ PA_API pa_status pa_step_slot_wait(const pa_step_slot_t *slot) {
 PA_API pa_status pa_decode_step(pa_allocator *a, const int32_t *seqs_host, int32_t n_seqs,
                                 int32_t max_blocks, int32_t share_max_members,
                                 const pa_cache_t *cache, int32_t num_q_heads, float scale,
-                                const pa_step_slot_t *slot, void *stream, void *copy_stream,
+                                const pa_step_slot_t *slot, void *stream, void *h2d_stream,
+                                void *d2h_stream,
                                 int32_t *n_copies, int32_t *n_groups, int32_t *max_len) {
   if (!a || !slot || !n_copies || !n_groups || !max_len || !slot->host || !slot->dev || !slot->out_host ||
       !slot->out_dev || !slot->ev_in || !slot->ev_kernel || !slot->ev_out)
@@ -967,15 +968,16 @@ PA_API pa_status pa_decode_step(pa_allocator *a, const int32_t *seqs_host, int32
                              max_len);
   if (s != PA_OK || n_seqs == 0) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaStream_t cst = static_cast<cudaStream_t>(copy_stream);
+  cudaStream_t hst = static_cast<cudaStream_t>(h2d_stream);
+  cudaStream_t dst = static_cast<cudaStream_t>(d2h_stream);
   cudaEvent_t ev_in = static_cast<cudaEvent_t>(slot->ev_in);
   cudaEvent_t ev_kernel = static_cast<cudaEvent_t>(slot->ev_kernel);
   cudaEvent_t ev_out = static_cast<cudaEvent_t>(slot->ev_out);
   cudaError_t e;
   // inputs: after the slot's previous decode has read its device copy
-  if ((e = cudaStreamWaitEvent(cst, ev_kernel, 0)) != cudaSuccess) return cuda_failed(e);
-  if ((e = cudaMemcpyAsync(d, h, L.bytes, cudaMemcpyHostToDevice, cst)) != cudaSuccess) return cuda_failed(e);
-  if ((e = cudaEventRecord(ev_in, cst)) != cudaSuccess) return cuda_failed(e);
+  if ((e = cudaStreamWaitEvent(hst, ev_kernel, 0)) != cudaSuccess) return cuda_failed(e);
+  if ((e = cudaMemcpyAsync(d, h, L.bytes, cudaMemcpyHostToDevice, hst)) != cudaSuccess) return cuda_failed(e);
+  if ((e = cudaEventRecord(ev_in, hst)) != cudaSuccess) return cuda_failed(e);
   // the decode: after the inputs, and after the previous output left out_dev
   if ((e = cudaStreamWaitEvent(st, ev_in, 0)) != cudaSuccess) return cuda_failed(e);
   if ((e = cudaStreamWaitEvent(st, ev_out, 0)) != cudaSuccess) return cuda_failed(e);
@@ -988,11 +990,11 @@ PA_API pa_status pa_decode_step(pa_allocator *a, const int32_t *seqs_host, int32
   if (s != PA_OK) return s;
   if ((e = cudaEventRecord(ev_kernel, st)) != cudaSuccess) return cuda_failed(e);
   // the output, back to the host
-  if ((e = cudaStreamWaitEvent(cst, ev_kernel, 0)) != cudaSuccess) return cuda_failed(e);
+  if ((e = cudaStreamWaitEvent(dst, ev_kernel, 0)) != cudaSuccess) return cuda_failed(e);
   const size_t out_bytes = (size_t)n_seqs * num_q_heads * cache->head_dim * elem_bytes(cache->dtype);
-  if ((e = cudaMemcpyAsync(slot->out_host, slot->out_dev, out_bytes, cudaMemcpyDeviceToHost, cst)) != cudaSuccess)
+  if ((e = cudaMemcpyAsync(slot->out_host, slot->out_dev, out_bytes, cudaMemcpyDeviceToHost, dst)) != cudaSuccess)
     return cuda_failed(e);
-  if ((e = cudaEventRecord(ev_out, cst)) != cudaSuccess) return cuda_failed(e);
+  if ((e = cudaEventRecord(ev_out, dst)) != cudaSuccess) return cuda_failed(e);
   return PA_OK;
 }
 

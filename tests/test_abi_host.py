@@ -230,7 +230,7 @@ def test_decode_step_refuses_before_the_allocator_moves():
     c = _cache_struct(num_blocks=64, num_kv_heads=2)
     slot = pa.pa_step_slot_t()
     args = lambda sl: (A._h, seqs.ctypes.data, 1, 64, 0, ctypes.byref(c), 8, ctypes.c_float(0.1), ctypes.byref(sl),
-                       None, None, ctypes.byref(nc), ctypes.byref(ng), ctypes.byref(ml))
+                       None, None, None, ctypes.byref(nc), ctypes.byref(ng), ctypes.byref(ml))
     assert pa.lib().pa_decode_step(*args(slot)) == pa.PA_ERR_INVALID_ARG
     slot = pa.pa_step_slot_t(16, 32, 48, 64, None, 0, 1, 2, 3)  # fake addresses, no workspace
     assert pa.lib().pa_decode_step(*args(slot)) == pa.PA_ERR_TOO_SMALL  # 64 x 16 tokens of room need a workspace
