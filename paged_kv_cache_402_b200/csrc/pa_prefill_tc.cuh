@@ -21,16 +21,19 @@
 //    with S double-buffered and O double-buffered by unit in tensor memory;
 //    the PV MMA takes P from tensor memory (A operand in TMEM).  Q tiles are
 //    double-buffered in shared memory so the next unit's loads overlap.
-//  * Warps 2..5: thread r owns query row r.  Per chunk it reads its S row,
-//    masks keys past its position (per 32-key group), and keeps a per-row
-//    reference max that moves only when a score passes it by 2^8; then it
-//    rescales its own O row in tensor memory (warp-wide when any lane of the
-//    warp needs it).  It writes its row of P in bf16 over the first half of
-//    its own S columns (each 32-column group of S is read before the 16
-//    columns of P that cover it are written).  The sums and maxima are per
-//    row, so no barrier across the warpgroup is needed per chunk.  At the
-//    end of a unit (overlapped with the next unit) it reads its O row,
-//    divides by its sum and stores the row.
+//  * Warps 2..9, two halves of four warps: half h takes keys 64h .. 64h + 63
+//    of every chunk and head-dim columns 64h .. 64h + 63 of O, and thread r
+//    of a half owns query row r, so each row is shared by one warp of each
+//    half (the pair of warps on the same tensor-memory lanes).  Per chunk a
+//    thread reads its half of the row's S, masks keys past its position (per
+//    32-key group), and weighs against a per-row reference max that moves
+//    only when a score passes it by 2^8; the pair agrees on the reference
+//    (and on any rescale of its O rows, each half rescaling its columns)
+//    through one named barrier per chunk.  It writes its half of the row of
+//    P in bf16 over the first half of its own S columns.  Each half keeps its
+//    own sum of weights; at the end of a unit (overlapped with the next
+//    unit) each half reads its columns of the row of O, divides by the sum
+//    of both halves' sums and stores them.
 //  * Every wait has a time limit (PA_DEVERR_TIMEOUT; the kernel drains and
 //    frees tensor memory).  A table entry outside the pool is loaded as zeros
 //    and sets PA_DEVERR_TABLE; that sequence's rows are then undefined.
@@ -59,9 +62,13 @@ struct PfLayout {
   static constexpr int kUnitInts = 8;
   static constexpr int kOffUnit = kOffTmem + 16;
   static constexpr int kOffScan = kOffUnit + 2 * kUnitInts * 4;
-  static constexpr int kOffPrefix = kOffScan + 32;  // tiles before each sequence
+  // row statistics the two softmax halves of a row exchange: [half][row]
+  // maxima, and [unit parity][half][row] sums
+  static constexpr int kOffXMax = kOffScan + 64;
+  static constexpr int kOffXSum = kOffXMax + 2 * kM * 4;
+  static constexpr int kOffPrefix = kOffXSum + 2 * 2 * kM * 4;  // tiles before each sequence
   static constexpr int kBytes = kOffPrefix + (kMaxSeqs + 1) * 4 + 1024;
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 320;
   static constexpr uint32_t kTmemCols = 512;  // S0 S1 O0 O1, 128 columns each
 };
 
@@ -103,11 +110,11 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
       // softmax warps once it has read the unit (they run without a common
       // barrier, so every one must have passed its wait on qfull before the
       // slot and its barrier phase can be reused)
-      mbar_init(&qempty[i], 1 + 4);
+      mbar_init(&qempty[i], 1 + 8);
       mbar_init(&sfull[i], 1);
-      mbar_init(&pfull[i], 128);  // P of the chunk written over its S
+      mbar_init(&pfull[i], 256);  // P of the chunk written over its S (both halves)
       mbar_init(&pvdone[i], 1);
-      mbar_init(&ofree[i], 128);
+      mbar_init(&ofree[i], 256);
     }
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -297,7 +304,9 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
           // P: 16 keys = 8 columns of tensor memory; V: N = head dim
           // contiguous (MN-major), 16 keys = two 8-key groups
           const uint64_t bdesc = tc::smem_desc_sw128(vb + kk * 2 * L::kGroup, 1024, L::kGroup);
-          tc::mma_bf16_ts(d, pa + kk * 8, bdesc, idesc_pv, (kk > 0 || !j.first) ? 1u : 0u);
+          // keys 0..63 in columns 0..31, keys 64..127 in columns 64..95 (each
+          // softmax half writes its P over the first half of its own S columns)
+          tc::mma_bf16_ts(d, pa + (kk >> 2) * 64 + (kk & 3) * 8, bdesc, idesc_pv, (kk > 0 || !j.first) ? 1u : 0u);
         }
         tc::mma_commit(&pvdone[c & 1]);
         tc::mma_commit(&vempty[c % L::kStages]);
@@ -345,31 +354,59 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
     mbar_wait(drain, 0);
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    // Two halves of four warps: half h (warps 2-5: h = 0; warps 6-9: h = 1)
+    // takes keys 64h .. 64h + 63 of every chunk and head-dim columns
+    // 64h .. 64h + 63 of O.  Thread r of a half owns query row r (its warp's
+    // tensor-memory lane quadrant), so each row is held by one warp of each
+    // half; the two warps of a quadrant form a pair that agrees, through
+    // named barrier 1 + quadrant over their 64 threads, on the row's
+    // reference and on stopping.  Each half keeps its own sum of weights over
+    // its keys against the shared reference; the epilogue adds the two.
     wait_prior_grid();  // before the first write of out
     allow_next_grid();
+    const int half = (warp - 2) >> 2;
     const int wq = warp & 3;
     const int r = wq * 32 + lane;            // query row: token r / G, head r % G
+    const int pair_bar = 1 + wq;
     const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
+    float *xmax = reinterpret_cast<float *>(smem + L::kOffXMax);  // [half][row]
+    float *xsum = reinterpret_cast<float *>(smem + L::kOffXSum);  // [unit parity][half][row]
     bool bad = false;
     auto warp_wait = [&](uint64_t *bar, uint32_t parity) {
       if (!bad && !__all_sync(0xffffffffu, mbar_wait(bar, parity))) bad = true;
     };
+    // OR of pred over the pair's 64 threads; both warps of a pair take the
+    // same sequence of these, so the pair never waits on a warp that left
+    auto pair_or = [&](bool pred) {
+      int res;
+      asm volatile(
+          "{\n\t.reg .pred p, q;\n\t"
+          "setp.ne.b32 p, %1, 0;\n\t"
+          "bar.red.or.pred q, %2, 64, p;\n\t"
+          "selp.s32 %0, 1, 0, q;\n\t}"
+          : "=r"(res)
+          : "r"((int)pred), "r"(pair_bar)
+          : "memory");
+      return res != 0;
+    };
     float m = -INFINITY, l = 0.f;
     // the unit whose output is pending
     bool pend = false;
-    int p_b = 0, p_g = 0, p_row0 = 0, p_ntok = 0, p_clast = 0, p_u = 0;
-    float p_l = 0.f;
+    int p_g = 0, p_row0 = 0, p_ntok = 0, p_clast = 0, p_u = 0;
     auto epilogue = [&]() {
       warp_wait(&pvdone[p_clast & 1], (p_clast >> 1) & 1);
-      float o[32];
+      // the row's sum over both halves' keys (each half wrote its part at the
+      // unit's end, before the pair's next barrier); the same order in both
+      const float lrow = xsum[((p_u & 1) * 2 + 0) * L::kM + r] + xsum[((p_u & 1) * 2 + 1) * L::kM + r];
+      const float inv = lrow > 0.f ? 1.f / lrow : 0.f;
       const int tok = r / G, h = p_g * G + (r % G);
       const bool row_ok = tok < p_ntok && !bad;
-      __nv_bfloat16 *dst = out + ((size_t)(p_row0 + tok) * p.Hq + h) * 128;
-      const float inv = p_l > 0.f ? 1.f / p_l : 0.f;
+      __nv_bfloat16 *dst = out + ((size_t)(p_row0 + tok) * p.Hq + h) * 128 + 64 * half;
       if (!bad) tc::fence_after_sync();
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if (!bad) tc::tmem_ld32(trow + 256 + (p_u & 1) * 128 + 32 * k, o);
+      for (int k = 0; k < 2; ++k) {
+        float o[32];
+        if (!bad) tc::tmem_ld32(trow + 256 + (p_u & 1) * 128 + 64 * half + 32 * k, o);
         if (row_ok) {
           uint4 v[4];
           uint32_t *w = reinterpret_cast<uint32_t *>(v);
@@ -391,39 +428,52 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
     for (;; ++qi) {
       const int qs = qi & 1;
       warp_wait(&qfull[qs], (qi >> 1) & 1);
-      if (bad) break;
+      if (pair_or(bad)) {
+        bad = true;
+        break;
+      }
       const int32_t *us = unit_slots + qs * L::kUnitInts;
       const int nchunks = us[5];
-      const int ub = us[0], ug = us[1], urow0 = us[2], untok = us[3], upos0 = us[4], uctx = us[6];
+      const int ug = us[1], urow0 = us[2], untok = us[3], upos0 = us[4], uctx = us[6];
       // keys of the sequence's last, partly filled block past its end
       const int tail_end = ((uctx + p.bs - 1) / p.bs) * p.bs;
       // the producer may reuse the Q tile once the QKs are done and every
       // softmax warp has read this unit's slot: it never runs two units
       // ahead of the slowest warp
       if (lane == 0 && nchunks > 0) mbar_arrive(&qempty[qs]);
+      if (nchunks == 0) {
+        if (pend) {
+          asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");  // the partner's last sum is written
+          epilogue();
+        }
+        break;
+      }
       const int pos = upos0 + r / G;  // this row's position (rows past the tile's tokens: masked out)
       const bool row_live = r / G < untok;
       m = -INFINITY;
       l = 0.f;
+      bool stop = false;
       for (int ci = 0; ci < nchunks; ++ci, ++c) {
         warp_wait(&sfull[c & 1], (c >> 1) & 1);
         if (!bad) tc::fence_after_sync();
-        const uint32_t srow = trow + (c & 1) * 128;
+        const uint32_t srow = trow + (c & 1) * 128 + 64 * half;  // this half's 64 columns of S
         const int key0 = ci * L::kChunk;
-        // keys of this chunk the row sees: the first nvis
-        const int nvis = row_live ? max(0, min(L::kChunk, pos - key0 + 1)) : 0;
+        // keys of this chunk the row sees (the first nrow), and of this half's
+        const int nrow = row_live ? max(0, min(L::kChunk, pos - key0 + 1)) : 0;
+        const int nvis = max(0, min(64, nrow - 64 * half));
         // One pass against the current reference: the weights stay in
-        // registers until every row of the warp is known to stay within 2^8
-        // of its reference; otherwise (a row's first chunk, or a score past
-        // the bound) the chunk takes two passes: the row max, a rescale of
-        // the rows' O, then the weights.  Either way each row's weights are
-        // 2^(s - m) against its reference m when they are written.
+        // registers until the pair knows that every row of its quadrant stays
+        // within 2^8 of its reference; otherwise (a row's first chunk, or a
+        // score past the bound in either half) the chunk takes two passes:
+        // the row max over both halves, a rescale of the rows' O, then the
+        // weights.  Either way the weights are 2^(s - m) against the row's
+        // reference m, the same in both halves.
         float s[32];
-        uint32_t w[64];
+        uint32_t w[32];
         float lsum = 0.f;
-        bool over = m == -INFINITY && nvis > 0;
+        bool over = m == -INFINITY && nrow > 0;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < 2; ++k) {
           if (!bad) tc::tmem_ld32(srow + 32 * k, s);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -436,10 +486,10 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
             w[16 * k + e] = *reinterpret_cast<const uint32_t *>(&two);
           }
         }
-        if (!__any_sync(0xffffffffu, over)) {
+        if (!pair_or(over || bad)) {
           if (!bad) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < 2; ++k) {
               uint32_t w16[16];
 #pragma unroll
               for (int e = 0; e < 16; ++e) w16[e] = w[16 * k + e];
@@ -449,10 +499,11 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
           }
           l += lsum;
         } else {
-          // pass 1: the chunk's row max over those keys (base-2 units)
+          // pass 1: this half's max over its visible keys (base-2 units),
+          // then the row's over both halves
           float cmax = -INFINITY;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
+          for (int k = 0; k < 2; ++k) {
             if (!bad) tc::tmem_ld32(srow + 32 * k, s);
             if (32 * k + 32 <= nvis) {
 #pragma unroll
@@ -463,18 +514,25 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
                 if (32 * k + e < nvis) cmax = fmaxf(cmax, s[e] * p.scale_log2);
             }
           }
+          xmax[half * L::kM + r] = cmax;
+          if (pair_or(bad)) {  // also makes both halves' maxima visible to the pair
+            stop = true;
+            break;
+          }
+          cmax = fmaxf(xmax[r], xmax[L::kM + r]);
           // the reference moves only when a score passes it by 2^8
           const bool need = cmax > m + kLazyRescale;
           const float mnew = need ? cmax : m;
           const float alpha = need ? exp2f(m - mnew) : 1.f;  // 0 when m was -inf
           if (__any_sync(0xffffffffu, need) && ci > 0) {
-            // rescale this warp's O rows once PV(c-1) has landed, before PV(c) adds
+            // rescale this half's columns of the warp's O rows once PV(c-1)
+            // has landed, before PV(c) adds
             warp_wait(&pvdone[(c - 1) & 1], ((c - 1) >> 1) & 1);
             if (!bad) {
-              const uint32_t orow = trow + 256 + (qi & 1) * 128;
+              const uint32_t orow = trow + 256 + (qi & 1) * 128 + 64 * half;
               tc::fence_after_sync();
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
+              for (int k = 0; k < 2; ++k) {
                 float o[32];
                 tc::tmem_ld32(orow + 32 * k, o);
 #pragma unroll
@@ -490,9 +548,10 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
           l *= alpha;
           m = mnew;
           // pass 2: P = 2^(s - m) in bf16, two keys per column, written over
-          // columns 16k .. 16k+15 once group k of S (columns 32k ..) is read
+          // columns 16k .. 16k + 15 of this half once group k of its S
+          // (columns 32k ..) is read
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
+          for (int k = 0; k < 2; ++k) {
             if (!bad) tc::tmem_ld32(srow + 32 * k, s);
             float pv[32];
             if (32 * k + 32 <= nvis) {
@@ -515,9 +574,10 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
           if (!bad) tc::tmem_wait_st();
         }
         // V rows past the sequence's end in its last block hold whatever the
-        // pool has there: zero them (thread r takes row r of the chunk)
-        const bool tail_row = key0 + r >= uctx && key0 + r < tail_end;
-        if (__any_sync(0xffffffffu, tail_row)) {
+        // pool has there: zero them (thread r of the first half takes row r
+        // of the chunk)
+        const bool tail_row = half == 0 && key0 + r >= uctx && key0 + r < tail_end;
+        if (half == 0 && __any_sync(0xffffffffu, tail_row)) {
           warp_wait(&vfull[c % L::kStages], (c / L::kStages) & 1);
           if (!bad && tail_row) {
             uint4 *vr = reinterpret_cast<uint4 *>(smem + L::kOffV + (c % L::kStages) * L::kTile +
@@ -538,20 +598,19 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
           pend = false;
         }
       }
-      if (nchunks == 0) {
-        if (pend) epilogue();
+      if (stop) {
+        bad = true;
         break;
       }
+      // this half's sum of the unit's weights, for the epilogue
+      xsum[((qi & 1) * 2 + half) * L::kM + r] = l;
       pend = true;
-      p_b = ub;
       p_g = ug;
       p_row0 = urow0;
       p_ntok = untok;
       p_clast = c - 1;
       p_u = qi;
-      p_l = l;
     }
-    (void)p_b;
     if (bad) raise_error(PA_DEVERR_TIMEOUT);
   }
 
