@@ -145,13 +145,13 @@ int choose_stages(int tile_bytes) {
   return n;
 }
 
-// The partition merge after a decode launch: with at most kReduceFast
-// partitions per row, the warp-per-row kernel sized to the row's partition
-// bound (NP 4, 8 or 16), over a grid of at most 4 CTAs per SM; else one
-// CTA per row.
+// The partition merge after a decode launch: with at most kReduceWide
+// partitions per row, a warp-per-row kernel (sized to the row's partition
+// bound, NP 4, 8 or 16, or the one that reads up to 32 partitions in rounds),
+// over a grid of at most 4 CTAs per SM; else one CTA per row.
 template <typename T, int D>
 pa_status launch_reduce(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
-  if (max_parts > pa::kReduceFast)
+  if (max_parts > pa::kReduceWide)
     return launch(pa::decode_reduce<T, D>, dim3(p.B * p.Hq), dim3(128), (size_t)max_parts * sizeof(float), st, p);
   const int64_t rows = (int64_t)p.B * p.Hq;
   int64_t grid = (rows + pa::kReduceRowWarps - 1) / pa::kReduceRowWarps;
@@ -161,7 +161,8 @@ pa_status launch_reduce(const pa::DecodeParams &p, int32_t max_parts, cudaStream
   const dim3 block(pa::kReduceRowWarps * 32);
   if (max_parts <= 4) return launch(pa::decode_reduce_rows<T, D, 4>, dim3((unsigned)grid), block, 0, st, p);
   if (max_parts <= 8) return launch(pa::decode_reduce_rows<T, D, 8>, dim3((unsigned)grid), block, 0, st, p);
-  return launch(pa::decode_reduce_rows<T, D, 16>, dim3((unsigned)grid), block, 0, st, p);
+  if (max_parts <= 16) return launch(pa::decode_reduce_rows<T, D, 16>, dim3((unsigned)grid), block, 0, st, p);
+  return launch(pa::decode_reduce_rows_wide<T, D>, dim3((unsigned)grid), block, 0, st, p);
 }
 
 template <typename T, int D, int G>

@@ -374,17 +374,18 @@ __global__ void __launch_bounds__(128) decode_reduce(DecodeParams p) {
   for (int w = 1; w < nw; ++w) M = fmaxf(M, red[w]);
   __syncthreads();
 
-  float ls = 0.f;
-  for (int i = threadIdx.x; i < np; i += blockDim.x) {
-    const float f = (m[i] == -INFINITY) ? 0.f : fast_exp2(m[i] - M);
-    wsh[i] = f;
-    ls += l[i] * f;
-  }
-  for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-  if (lane == 0) red[warp] = ls;
+  for (int i = threadIdx.x; i < np; i += blockDim.x) wsh[i] = (m[i] == -INFINITY) ? 0.f : fast_exp2(m[i] - M);
   __syncthreads();
-  float L = 0.f;
-  for (int w = 0; w < nw; ++w) L += red[w];
+  // L = sum_i l_i f_i in partition order by fused multiply-adds, the order
+  // of merge_weights, so that every merge kernel gives the same bits
+  if (threadIdx.x == 0) {
+    float ls = 0.f;
+    for (int i = 0; i < np; ++i) ls = fmaf(l[i], wsh[i], ls);
+    red[0] = ls;
+  }
+  __syncthreads();
+  const float L = red[0];
+  (void)nw;
 
   const float *acc = p.ws_acc + (size_t)bh * p.max_parts * D;
   T *out = reinterpret_cast<T *>(p.out) + (size_t)bh * D;
@@ -449,6 +450,76 @@ __global__ void __launch_bounds__(kReduceRowWarps * 32, 2) decode_reduce_rows(De
     const float L = merge_weights(mv, lv, np, f);
 #pragma unroll
     for (int k = 0; k < E; ++k) store_out(out + bh * D + lane * E + k, merge_element(av[k], f, np, L));
+  }
+}
+
+// decode_reduce for calls whose rows have at most kReduceWide partitions:
+// one warp per row as decode_reduce_rows, lane i holding partition i's max
+// and sum; the accumulators are read in rounds of kReduceRound partitions
+// (one load per lane per partition in a round, then the round's fused
+// multiply-adds in partition order).  The merge takes the steps of
+// merge_weights and merge_element in their order, so its bits are those of
+// the other merge kernels.
+constexpr int kReduceWide = 32;
+constexpr int kReduceRound = 8;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kReduceRowWarps * 32, 2) decode_reduce_rows_wide(DecodeParams p) {
+  constexpr int E = D / 32;
+  static_assert(D % 32 == 0 && (E == 1 || E == 2 || E == 4), "head_dim");
+  wait_prior_grid();
+  allow_next_grid();
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = (int64_t)p.B * p.Hq;
+  const int64_t stride = (int64_t)gridDim.x * kReduceRowWarps;
+  T *out = reinterpret_cast<T *>(p.out);
+  for (int64_t bh = (int64_t)blockIdx.x * kReduceRowWarps + (threadIdx.x >> 5); bh < rows; bh += stride) {
+    const int ctx = p.lens[bh / p.Hq];
+    if (ctx <= p.part || ctx > p.max_ctx) continue;  // written directly by the partition kernel
+    const int np = min((ctx + p.part - 1) / p.part, kReduceWide);
+    const float mi = lane < np ? __ldcg(p.ws_m + bh * p.max_parts + lane) : -INFINITY;
+    const float li = lane < np ? __ldcg(p.ws_l + bh * p.max_parts + lane) : 0.f;
+    float M = mi;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float fi = (lane < np && mi != -INFINITY) ? fast_exp2(mi - M) : 0.f;
+    float L = 0.f;
+    for (int i = 0; i < np; ++i) L = fmaf(__shfl_sync(0xffffffffu, li, i), __shfl_sync(0xffffffffu, fi, i), L);
+    const float *acc = p.ws_acc + bh * p.max_parts * D + lane * E;
+    float a[E];
+#pragma unroll
+    for (int k = 0; k < E; ++k) a[k] = 0.f;
+    for (int i0 = 0; i0 < np; i0 += kReduceRound) {
+      float av[kReduceRound][E];
+#pragma unroll
+      for (int j = 0; j < kReduceRound; ++j) {
+        const float *src = acc + (size_t)(i0 + j) * D;
+        if (i0 + j < np) {
+          if constexpr (E == 4) {
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(src));
+            av[j][0] = v.x; av[j][1] = v.y; av[j][2] = v.z; av[j][3] = v.w;
+          } else if constexpr (E == 2) {
+            const float2 v = __ldcg(reinterpret_cast<const float2 *>(src));
+            av[j][0] = v.x; av[j][1] = v.y;
+          } else {
+            av[j][0] = __ldcg(src);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < E; ++k) av[j][k] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kReduceRound; ++j) {
+        const float f = __shfl_sync(0xffffffffu, fi, (i0 + j) & 31);
+        if (i0 + j < np) {
+#pragma unroll
+          for (int k = 0; k < E; ++k) a[k] = fmaf(av[j][k], f, a[k]);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < E; ++k) store_out(out + bh * D + lane * E + k, L > 0.f ? a[k] / L : 0.f);
   }
 }
 

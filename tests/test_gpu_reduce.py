@@ -1,11 +1,12 @@
 """The partition merge (log-sum-exp reduce) kernels against the oracle and
 against each other.
 
-A call whose rows have at most 16 partitions merges one row per warp
-(decode_reduce_rows, sized for 4, 8 or 16 partitions); a longer declared
-maximum context takes the one-CTA-per-row decode_reduce.  Both merge in the
-same order with the same arithmetic, so for the same partition statistics
-their outputs must agree bit for bit.
+A call whose rows have at most 32 partitions merges one row per warp
+(decode_reduce_rows, sized for 4, 8 or 16 partitions, and
+decode_reduce_rows_wide up to 32); a longer declared maximum context takes
+the one-CTA-per-row decode_reduce.  All merge in the same order with the
+same arithmetic, so for the same partition statistics their outputs must
+agree bit for bit.
 """
 import numpy as np
 import pytest
@@ -26,13 +27,13 @@ def _bits(t: torch.Tensor) -> torch.Tensor:
     return t.view(torch.int32 if t.dtype == torch.float32 else torch.int16).cpu()
 
 
-@pytest.mark.parametrize("parts", [2, 4, 8, 16])
+@pytest.mark.parametrize("parts", [2, 4, 8, 16, 17, 24, 32])
 @pytest.mark.parametrize("G,dtype,D", [(1, torch.bfloat16, 128), (4, torch.bfloat16, 128),
                                        (8, torch.bfloat16, 128), (2, torch.float32, 128),
                                        (4, torch.float32, 64)])
 def test_row_reduce_matches_block_reduce_bits(cuda_device, parts, G, dtype, D):
     """Lengths from 1 token to exactly `parts` partitions: the call with the
-    true maximum merges with the warp-per-row kernel, the call declaring 17
+    true maximum merges with a warp-per-row kernel, the call declaring 33
     partitions with the one-CTA-per-row kernel; same bits, and within the
     bound of the oracle."""
     Hkv = 2
@@ -42,7 +43,7 @@ def test_row_reduce_matches_block_reduce_bits(cuda_device, parts, G, dtype, D):
                              dtype=dtype)
     cache, q, tables, lens_d = to_dev(case, cuda_device)
     # wide enough a table for the longer declared maximum to be a valid call
-    long_max = 16 * PART + 1
+    long_max = 32 * PART + 1
     cols = -(-long_max // 16)
     tables = torch.cat([tables, torch.full_like(tables[:, :1], -1).expand(-1, cols - tables.shape[1])],
                        dim=1).contiguous()
