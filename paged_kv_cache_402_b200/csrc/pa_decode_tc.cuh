@@ -188,18 +188,22 @@ constexpr int kFullBits = 20;
 __device__ __forceinline__ int pf_of(int32_t v) { return v & ((1 << kFullBits) - 1); }
 __device__ __forceinline__ int pp_of(int32_t v) { return (int)((uint32_t)v >> kFullBits); }
 
-// Unit u of the largest-first order: units [0, F) are the full partitions
-// (sequence-major, kv head fastest; a sequence's start at its first
-// partition), one kv head each; units [F, F + P) the partial last
-// partitions, each of tail_hg consecutive kv heads of one sequence
-// (Hkv / tail_hg units per sequence).
+// Unit u of the largest-first order.  The full partitions (sequence-major,
+// kv head fastest; a sequence's start at its first partition) are one kv
+// head each; the partial last partitions are tail_hg consecutive kv heads of
+// one sequence each (Hkv / tail_hg units per sequence).  With one head per
+// tail unit the full partitions come first (units [0, F)), the partial ones
+// after; with several heads a tail unit is about as large as a full one or
+// larger, so the tail units come first (units [0, T)) and the full ones
+// after, and a launch ends on units of one full partition either way.
 template <int PART>
 __device__ __forceinline__ TcUnit tc_unit_at(const DecodeParams &p, const int32_t *prefix,
                                              const int32_t *ctx_s, const int32_t *first_s, int u,
-                                             int num_full, int tail_hg) {
+                                             int num_full, int num_tail, int tail_hg) {
   TcUnit un;
-  const bool full = u < num_full;
-  const int v = full ? u : u - num_full;
+  const bool tails_first = tail_hg > 1;
+  const bool full = tails_first ? u >= num_tail : u < num_full;
+  const int v = full ? (tails_first ? u - num_tail : u) : (tails_first ? u : u - num_full);
   const int per_seq = full ? p.Hkv : p.Hkv / tail_hg;
   const int w = v / per_seq;
   un.hg = full ? 1 : tail_hg;
@@ -391,7 +395,8 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       tail_hg = max(h, 1);
     }
   }
-  const int num_units = num_full + (p.Hkv / tail_hg) * pp_of(prefix[B]);
+  const int num_tail = (p.Hkv / tail_hg) * pp_of(prefix[B]);
+  const int num_units = num_full + num_tail;
   uint32_t *sched = g_sched + 2 * p.sched_slot;
 
   if (warp == 0) {
@@ -427,7 +432,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       for (int k = 0; k < NE; ++k) x[k] = -1;
       nd = ns = -1;
       if (u < num_units) {
-        nu = tc_unit_at<PART>(p, prefix, ctx_s, first_s, u, num_full, tail_hg);
+        nu = tc_unit_at<PART>(p, prefix, ctx_s, first_s, u, num_full, num_tail, tail_hg);
         const int32_t *tr = p.tables + (size_t)nu.b * p.max_blocks + nu.t0 / bs;
         const int nb = (nu.t1 - nu.t0 + bs - 1) / bs;
         const bool newest = p.k_new != nullptr && nu.t1 == ctx_s[nu.b];
