@@ -78,10 +78,16 @@ def test_block_size_choice_rule():
     assert bench.choose_block_size(lines, 0.06)["block_size_choice"] == 32
     assert bench.choose_block_size(lines, 0.01)["block_size_choice"] == 8
     assert set(bench.choose_block_size(lines, 0.05)["per_layout"]) == {"bs8/p512", "bs16/p512", "bs32/p512"}
-    # a partition size of the sweep wins when it is the fastest within the budget
-    lines.append(dict(mk(16, 600e3, 0.028), config={"block_size": 16, "partition_tokens": 256}))
+    # the partition size is the one of least device time at the chosen block
+    # size, whatever the wall clock (host noise) says
+    lines.append(dict(mk(16, 600e3, 0.028), config={"block_size": 16, "partition_tokens": 256},
+                      device_ms_per_step=0.9))
+    lines.append(dict(mk(16, 700e3, 0.028), config={"block_size": 16, "partition_tokens": 1024},
+                      device_ms_per_step=1.1))
     pick = bench.choose_block_size(lines, 0.05)
     assert (pick["block_size_choice"], pick["partition_choice"]) == (16, 256)
+    lines[-2]["device_ms_per_step"] = 1.2
+    assert bench.choose_block_size(lines, 0.05)["partition_choice"] == 512
 
 
 def test_traffic_record_follows_the_kernel_sources(tmp_path, monkeypatch):
