@@ -323,7 +323,7 @@ class Instance:
             slots, pairs = self.alloc.batch_append(seqs, np.ones(B, np.int32))
             tables, lens = self.alloc.build_block_tables(seqs, self.max_blocks)
             cow = pa.cow_sources(pairs, tables, lens, bs)
-            plan = pa.share_plan(tables, lens, bs, partition_tokens=wl["part"])
+            plan = pa.share_plan(tables, lens, bs)
             self.host_alloc_s += time.perf_counter() - t1
             nblk = (lens.astype(np.int64) + bs - 1) // bs
             # unique bytes: every physical block once, with its fill
@@ -355,8 +355,8 @@ class Instance:
                                       + len(pairs) * 2 * bs * Hkv * D * 2 * 2 + (B * 4 if len(pairs) else 0))
             self.steps.append(st)
         top = max(st["max_ctx"] for st in self.steps)
-        ws = torch.empty(max(16, pa.pa_decode_workspace_size(B, Hq, top + 64, D, wl["part"])), dtype=torch.uint8,
-                         device=dev)
+        ws = torch.empty(max(16, pa.pa_decode_shared_workspace_size(B, Hq, top + 64, D, wl["part"])),
+                         dtype=torch.uint8, device=dev)
         out = torch.empty(B, Hq, D, dtype=dt, device=dev)
         for st in self.steps:
             st["ws"], st["out"] = ws, out
@@ -624,8 +624,8 @@ def run_e2e(args, insts, wl, dev, stream):
     # one packed buffer per step: (name, shape, dtype), each part 16-byte aligned
     parts = [("q", (B, Hq, D), torch.bfloat16), ("k", (B, Hkv, D), torch.bfloat16),
              ("v", (B, Hkv, D), torch.bfloat16), ("tables", (B, mb), torch.int32), ("lens", (B,), torch.int32),
-             ("cow_src", (B,), torch.int32), ("first_part", (B,), torch.int32), ("members", (G2, 4), torch.int32),
-             ("parts", (G2,), torch.int32), ("slots", (B,), torch.int64), ("pairs", (B, 2), torch.int32)]
+             ("cow_src", (B,), torch.int32), ("first_token", (B,), torch.int32), ("members", (G2, 4), torch.int32),
+             ("shared_tokens", (G2,), torch.int32), ("slots", (B,), torch.int64), ("pairs", (B, 2), torch.int32)]
     offs, total = {}, 0
     for name, shape, dt in parts:
         nbytes = int(np.prod(shape)) * torch.tensor([], dtype=dt).element_size()
@@ -646,7 +646,7 @@ def run_e2e(args, insts, wl, dev, stream):
         hv = views(h_buf)
         for k in ("q", "k", "v"):
             hv[k].copy_(rows[k])
-        np_out = {k: hv[k].numpy() for k in ("tables", "lens", "cow_src", "first_part", "members", "parts")}
+        np_out = {k: hv[k].numpy() for k in ("tables", "lens", "cow_src", "first_token", "members", "shared_tokens")}
         return {"h_buf": h_buf, "d_buf": d_buf, "h": hv, "d": views(d_buf), "np": np_out,
                 "out": torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev),
                 "h_out": torch.empty(B, Hq, D, dtype=torch.bfloat16).pin_memory(),
@@ -679,9 +679,9 @@ def run_e2e(args, insts, wl, dev, stream):
         else:
             st = inst.alloc.decode_step(seqs, mb, share_max_members=share, out=S["np"])
             npairs, max_len = st["n_copies"], st["max_len"]
-            plan = pa.SharePlan(st["members"], st["parts"], st["first_part"])
+            plan = pa.SharePlan(st["members"], st["shared_tokens"], st["first_token"])
             if plan.n_groups:
-                plan.bind(d["members"][:plan.n_groups], d["parts"][:plan.n_groups], d["first_part"])
+                plan.bind(d["members"][:plan.n_groups], d["shared_tokens"][:plan.n_groups], d["first_token"])
         with torch.cuda.stream(copy_stream):
             if S["used"]:
                 copy_stream.wait_event(S["ev_kernel"])   # step i - 2 no longer reads these device inputs
@@ -990,7 +990,7 @@ def run_trace(args, dev):
             if n:
                 max_ctx, mb = A.max_len(plan.decode_seqs)
                 tables, lens = A.build_block_tables(plan.decode_seqs, mb)
-                splan = (pa.share_plan(tables, lens, bs, partition_tokens=part)
+                splan = (pa.share_plan(tables, lens, bs)
                          if not (args.unfused or args.no_share_plan) else None)
             host_s += time.perf_counter() - t0
             if n == 0:
@@ -1009,7 +1009,8 @@ def run_trace(args, dev):
             # step's first event: inputs, plan, workspace, q and out
             dplan = splan.to(dev) if splan is not None else None
             kd = src[(s_ * 131) % ((1 << 16) - n):][:n]
-            need = pa.pa_decode_workspace_size(n, Hq, max_ctx, D, part)
+            need = (pa.pa_decode_shared_workspace_size if splan is not None and splan.n_groups
+                    else pa.pa_decode_workspace_size)(n, Hq, max_ctx, D, part)
             if need > ws.numel():
                 ws = torch.empty(need * 5 // 4, dtype=torch.uint8, device=dev)
             q = qsrc[:n] if n <= 8192 else synth.normal((n, Hq, D), dt, s_, device=dev)

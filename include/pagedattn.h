@@ -92,8 +92,7 @@ typedef struct {
   int32_t head_dim;     /* 64 or 128 */
   /* Tokens per split-context partition of the decode calls over this pool:
    * 256, 512 or 1024, or 0 for PA_PARTITION_TOKENS.  It sets the workspace
-   * size (pa_decode_workspace_size_p) and the unit of sharing of a plan
-   * (pa_share_plan), which must be built for the same size. */
+   * size (pa_decode_workspace_size_p, pa_decode_shared_workspace_size). */
   int32_t partition_tokens;
 } pa_cache_t;
 
@@ -181,41 +180,50 @@ PA_API pa_status pa_append_decode(const void *k_new, const void *v_new, const in
 
 /*
  * A sharing plan for pa_decode_shared: groups of sequences of one batch whose
- * block tables hold the same physical blocks for their first parts[j] whole
- * partitions (of the pool's partition_tokens), every one of them before the
- * member's last partition.  pa_share_plan builds one from host tables.
- *   members     device [n_groups][max_members] int32: sequence indices of the
- *               batch, a group's members first, -1 after its last
- *   parts       device [n_groups] int32 (>= 1)
- *   first_part  device [num_seqs] int32: parts[j] for a member of group j,
- *               0 for a sequence in no group
- *   max_members 1..4 (the cascade kernel's query tile holds 4 sequences)
+ * block tables hold the same physical blocks for their first
+ * shared_tokens[j] tokens (whole blocks, every one of them before each
+ * member's last block).  pa_share_plan builds one from host tables.
+ *   members       device [n_groups][max_members] int32: sequence indices of
+ *                 the batch, a group's members first, -1 after its last
+ *   shared_tokens device [n_groups] int32 (> 0, a multiple of the block size)
+ *   first_token   device [num_seqs] int32: shared_tokens[j] for a member of
+ *                 group j, 0 for a sequence in no group
+ *   max_members   1..4 (the cascade kernel's query tile holds 4 sequences)
  * A sequence belongs to at most one group.  If the tables of a group do not
- * agree on those partitions the results are undefined; a first_part that
- * does not fit its sequence sets PA_DEVERR_PLAN and that sequence is
- * computed whole (the group's statistics for it are overwritten).
+ * agree on those blocks the results are undefined; a first_token that is
+ * not a multiple of the block size or not below its sequence's length sets
+ * PA_DEVERR_PLAN and that sequence is computed whole.
  */
+/* Shared prefixes shorter than this are not worth a cascade unit. */
+#define PA_SHARE_MIN_TOKENS 128
+
 typedef struct {
   const int32_t *members;
-  const int32_t *parts;
-  const int32_t *first_part;
+  const int32_t *shared_tokens;
+  const int32_t *first_token;
   int32_t n_groups;
   int32_t max_members;
 } pa_share_plan_t;
 
 /*
  * pa_decode (or pa_append_decode, when k_new and v_new are given) with a
- * cascade over shared blocks: the partitions a plan's group shares are read
- * once for all its members ("pagedattention" glossary entry, paragraph 5:
+ * cascade over shared blocks: the prefix a plan's group shares is read once
+ * for all its members ("pagedattention" glossary entry, paragraph 5:
  * sequences that share a prefix point at the same physical blocks;
- * "PagedAttention Internals", "Sharing And Dynamic Growth").  The result is
- * bit for bit that of pa_decode / pa_append_decode: each member's statistics
- * over a shared partition come from the same tiles through the same
- * per-column arithmetic.  plan may be NULL or have no groups; on the
- * CUDA-core path (not bf16 with head_dim 128) the plan is not used and every
- * sequence computes all of its partitions.
+ * "PagedAttention Internals", "Sharing And Dynamic Growth").  The cascade
+ * computes each member's statistics over the shared prefix in pieces of the
+ * pool's partitions; when a prefix ends inside a partition, that partition's
+ * statistics come in two parts (the shared piece, kept in an extra workspace
+ * row, and the member's own rest), which the log-sum-exp reduce merges with
+ * the others.  The result is the same attention: within the decode's
+ * tolerances of pa_decode / pa_append_decode, and bit for bit when every
+ * group's prefix ends on a partition boundary.  plan may be NULL or have no
+ * groups; on the CUDA-core path (not bf16 with head_dim 128) the plan is not
+ * used and every sequence computes all of its partitions.
  *   k_new, v_new, cow_src  as pa_append_decode, or all NULL for no append
  *   plan                   host pointer to the plan (its arrays on the device)
+ *   workspace              with a plan that has groups: at least
+ *                          pa_decode_shared_workspace_size(...) bytes
  *   the rest               as pa_decode
  */
 PA_API pa_status pa_decode_shared(const void *k_new, const void *v_new, const int32_t *cow_src,
@@ -263,6 +271,14 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
 PA_API size_t pa_decode_workspace_size_p(int32_t num_seqs, int32_t num_q_heads,
                                          int32_t max_context_len, int32_t head_dim,
                                          int32_t partition_tokens);
+
+/* Bytes of workspace pa_decode_shared needs with a sharing plan that has
+ * groups: one more row per (sequence, query head) than pa_decode (the
+ * shared piece of the partition a prefix ends in), and some even when no
+ * context is longer than one partition.  0 for an unsupported size. */
+PA_API size_t pa_decode_shared_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                              int32_t max_context_len, int32_t head_dim,
+                                              int32_t partition_tokens);
 
 /*
  * pa_decode without a caller-provided workspace.  The pages have no
@@ -420,23 +436,23 @@ PA_API pa_status pa_alloc_stats(pa_allocator *a, int64_t *used_slots, int64_t *a
 PA_API pa_status pa_block_refcount(pa_allocator *a, int32_t block, int32_t *refcount);
 
 /*
- * Builds a sharing plan from host tables (after the step's appends), for
- * partitions of partition_tokens tokens (256, 512 or 1024; 0 for
- * PA_PARTITION_TOKENS):
- * sequences longer than one partition whose first partition's table entries
- * are identical form buckets; each bucket is cut into groups of at most
- * max_members (2..4) in sequence order, a lone leftover joins no group; a
- * group shares every leading partition whose entries agree across it and
- * that is whole and before the last partition of each member.
+ * Builds a sharing plan from host tables (after the step's appends):
+ * sequences with a block before their last one whose first table entries
+ * are the same physical block form buckets (sharers point at the same blocks
+ * from the start); each bucket is cut into groups of at most max_members
+ * (2..4) in sequence order, a lone leftover joins no group; a group shares
+ * the leading blocks on which all its members' tables agree, each before
+ * every member's last block, and is kept when that is at least
+ * PA_SHARE_MIN_TOKENS tokens.
  *   tables_host  [n_seqs][max_blocks] int32, lens_host [n_seqs] int32
  *   members_host room for n_seqs / 2 groups x max_members, -1 padded
- *   parts_host   room for n_seqs / 2
- *   first_part_host [n_seqs]
+ *   shared_host  room for n_seqs / 2: each group's shared tokens
+ *   first_token_host [n_seqs]
  */
 PA_API pa_status pa_share_plan(const int32_t *tables_host, int32_t max_blocks,
                                const int32_t *lens_host, int32_t n_seqs, int32_t block_size,
-                               int32_t partition_tokens, int32_t max_members, int32_t *members_host,
-                               int32_t *parts_host, int32_t *first_part_host, int32_t *n_groups);
+                               int32_t max_members, int32_t *members_host, int32_t *shared_host,
+                               int32_t *first_token_host, int32_t *n_groups);
 
 /*
  * One decode step's host work in one call: appends one token to each of the
@@ -448,19 +464,17 @@ PA_API pa_status pa_share_plan(const int32_t *tables_host, int32_t max_blocks,
  *     would not fit max_blocks;
  *   cow_src_host [n_seqs]: the block a sequence's copy-on-write move copies
  *     into its new last block, -1 for none (*n_copies of them);
- *   with share_max_members in 2..4, the sharing plan of pa_share_plan for
- *     partitions of partition_tokens tokens
+ *   with share_max_members in 2..4, the sharing plan of pa_share_plan
  *     (members_host room for n_seqs / 2 groups x share_max_members,
- *     parts_host room for n_seqs / 2, *n_groups); with 0, no plan and
- *     first_part_host all zeros;
+ *     shared_host room for n_seqs / 2, *n_groups); with 0, no plan and
+ *     first_token_host all zeros;
  *   *max_len: the longest length (max_context_len of the call).
  */
 PA_API pa_status pa_decode_step_prepare(pa_allocator *a, const int32_t *seqs, int32_t n_seqs,
-                                        int32_t max_blocks, int32_t partition_tokens,
-                                        int32_t share_max_members,
+                                        int32_t max_blocks, int32_t share_max_members,
                                         int32_t *tables_host, int32_t *lens_host,
                                         int32_t *cow_src_host, int32_t *members_host,
-                                        int32_t *parts_host, int32_t *first_part_host,
+                                        int32_t *shared_host, int32_t *first_token_host,
                                         int32_t *n_groups, int32_t *n_copies, int32_t *max_len);
 
 /* ------------------------------------------------- one decode step, end to end */
@@ -485,14 +499,15 @@ PA_API pa_status pa_decode_step_prepare(pa_allocator *a, const int32_t *seqs, in
  *   dev       device buffer of the same size (the staging area's mirror)
  *   out_host  pinned host [n_seqs][num_q_heads][head_dim], cache dtype
  *   out_dev   device, same shape
- *   workspace device scratch of pa_decode_workspace_size_p(n_seqs, num_q_heads,
- *             max_blocks * block_size, head_dim, cache->partition_tokens)
- *             bytes (or more)
+ *   workspace device scratch of pa_decode_shared_workspace_size(n_seqs,
+ *             num_q_heads, max_blocks * block_size, head_dim,
+ *             cache->partition_tokens) bytes (or more) with a plan
+ *             (share_max_members > 0), else pa_decode_workspace_size_p(...)
  *   ev_in, ev_kernel, ev_out   CUDA events (cudaEvent_t) of the slot, made by
  *             pa_step_slot_events and released by pa_step_slot_release
  */
 typedef struct {
-  size_t q, k_new, v_new, tables, lens, cow_src, first_part, members, parts;  /* byte offsets */
+  size_t q, k_new, v_new, tables, lens, cow_src, first_token, members, shared_tokens;  /* byte offsets */
   size_t bytes;                                                              /* total */
 } pa_step_layout_t;
 
@@ -510,8 +525,8 @@ typedef struct {
 
 /* Offsets (16-byte aligned) of a step's inputs in the staging area:
  * q [n][Hq][D], k_new and v_new [n][Hkv][D] (cache dtype), tables
- * [n][max_blocks], lens [n], cow_src [n], first_part [n], members
- * [n / 2][share_max_members], parts [n / 2] (int32). */
+ * [n][max_blocks], lens [n], cow_src [n], first_token [n], members
+ * [n / 2][share_max_members], shared_tokens [n / 2] (int32). */
 PA_API pa_status pa_step_layout(int32_t n_seqs, int32_t num_q_heads, const pa_cache_t *cache,
                                 int32_t max_blocks, int32_t share_max_members, pa_step_layout_t *layout);
 
@@ -532,8 +547,7 @@ PA_API pa_status pa_step_slot_wait(const pa_step_slot_t *slot);
  *  2. on h2d_stream, after the slot's previous decode: one cudaMemcpyAsync
  *     of the staging area to dev, then ev_in;
  *  3. on stream, after ev_in and the slot's previous output copy:
- *     pa_decode_shared with the plan (share_max_members 2..4, or 0 for none;
- *     built for the pool's partition_tokens),
+ *     pa_decode_shared with the plan (share_max_members 2..4, or 0 for none),
  *     the copy sources and the new rows, then ev_kernel;
  *  4. on d2h_stream, after ev_kernel: cudaMemcpyAsync of out_dev to
  *     out_host, then ev_out.

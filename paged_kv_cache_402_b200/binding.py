@@ -27,6 +27,7 @@ PA_ERR_CUDA, PA_ERR_NOT_FOUND, PA_ERR_TOO_SMALL = 4, 5, 6
 PA_DTYPE_F32, PA_DTYPE_BF16 = 0, 1
 PA_DEVERR_SLOT, PA_DEVERR_TABLE, PA_DEVERR_PAIR, PA_DEVERR_TIMEOUT, PA_DEVERR_LEN, PA_DEVERR_PLAN = 1, 2, 4, 8, 16, 32
 PA_PARTITION_TOKENS = 512
+PA_SHARE_MIN_TOKENS = 128  # shortest shared prefix a plan group takes
 
 _DTYPES = {torch.float32: PA_DTYPE_F32, torch.bfloat16: PA_DTYPE_BF16}
 
@@ -53,8 +54,8 @@ class pa_cache_t(ctypes.Structure):
 
 
 class pa_step_layout_t(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_size_t) for n in ("q", "k_new", "v_new", "tables", "lens", "cow_src", "first_part",
-                                             "members", "parts", "bytes")]
+    _fields_ = [(n, ctypes.c_size_t) for n in ("q", "k_new", "v_new", "tables", "lens", "cow_src", "first_token",
+                                             "members", "shared_tokens", "bytes")]
 
 
 class pa_step_slot_t(ctypes.Structure):
@@ -64,7 +65,7 @@ class pa_step_slot_t(ctypes.Structure):
 
 
 class pa_share_plan_t(ctypes.Structure):
-    _fields_ = [("members", ctypes.c_void_p), ("parts", ctypes.c_void_p), ("first_part", ctypes.c_void_p),
+    _fields_ = [("members", ctypes.c_void_p), ("shared_tokens", ctypes.c_void_p), ("first_token", ctypes.c_void_p),
                 ("n_groups", ctypes.c_int32), ("max_members", ctypes.c_int32)]
 
 
@@ -84,14 +85,15 @@ def _load() -> ctypes.CDLL:
         "pa_decode": (st, [vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp, sz, vp]),
         "pa_decode_workspace_size": (sz, [i32, i32, i32, i32]),
         "pa_decode_workspace_size_p": (sz, [i32, i32, i32, i32, i32]),
+        "pa_decode_shared_workspace_size": (sz, [i32, i32, i32, i32, i32]),
         "pa_decode_static_workspace": (st, [vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp]),
         "pa_append_decode": (st, [vp, vp, vp, vp, cp, vp, i32, vp, i32, i32, i32, f32, vp, vp, sz, vp]),
         "pa_cow_sources": (st, [i32p, i32, i32p, i32, i32p, i32, i32, i32p]),
         "pa_decode_shared": (st, [vp, vp, vp, vp, cp, vp, i32, vp, i32, i32, i32, f32,
                                   ctypes.POINTER(pa_share_plan_t), vp, vp, sz, vp]),
-        "pa_share_plan": (st, [i32p, i32, i32p, i32, i32, i32, i32, i32p, i32p, i32p, i32p]),
+        "pa_share_plan": (st, [i32p, i32, i32p, i32, i32, i32, i32p, i32p, i32p, i32p]),
         "pa_prefill": (st, [vp, cp, vp, i32, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp]),
-        "pa_decode_step_prepare": (st, [vp, i32p, i32, i32, i32, i32, i32p, i32p, i32p, i32p, i32p, i32p,
+        "pa_decode_step_prepare": (st, [vp, i32p, i32, i32, i32, i32p, i32p, i32p, i32p, i32p, i32p,
                                         i32p, i32p, i32p]),
         "pa_step_layout": (st, [i32, i32, cp, i32, i32, ctypes.POINTER(pa_step_layout_t)]),
         "pa_step_slot_events": (st, [ctypes.POINTER(pa_step_slot_t)]),
@@ -256,6 +258,14 @@ def pa_decode_workspace_size(num_seqs: int, num_q_heads: int, max_context_len: i
                                                int(partition_tokens)))
 
 
+def pa_decode_shared_workspace_size(num_seqs: int, num_q_heads: int, max_context_len: int, head_dim: int,
+                                    partition_tokens: int = PA_PARTITION_TOKENS) -> int:
+    """Scratch of pa_decode_shared with a plan that has groups (one more row
+    per (sequence, query head) than pa_decode_workspace_size)."""
+    return int(_lib.pa_decode_shared_workspace_size(num_seqs, num_q_heads, max_context_len, head_dim,
+                                                    int(partition_tokens)))
+
+
 def pa_decode(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor, context_lens: torch.Tensor,
               max_context_len: int, scale: float, out: torch.Tensor | None = None,
               workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
@@ -331,10 +341,12 @@ def cow_sources(pairs, tables: np.ndarray, lens: np.ndarray, block_size: int,
 
 class SharePlan:
     """A sharing plan (groups of sequences that hold the same blocks for their
-    leading whole partitions) as host arrays, plus its device copy."""
+    leading tokens, a whole number of blocks) as host arrays, plus its device
+    copy: members [n_groups, max_members], shared_tokens [n_groups],
+    first_token [n_seqs]."""
 
-    def __init__(self, members: np.ndarray, parts: np.ndarray, first_part: np.ndarray):
-        self.members, self.parts, self.first_part = members, parts, first_part
+    def __init__(self, members: np.ndarray, shared_tokens: np.ndarray, first_token: np.ndarray):
+        self.members, self.shared_tokens, self.first_token = members, shared_tokens, first_token
         self.n_groups, self.max_members = int(members.shape[0]), int(members.shape[1])
         self._dev = None
 
@@ -343,50 +355,48 @@ class SharePlan:
         a plan without groups needs none."""
         if self.n_groups > 0:
             self._dev = tuple(torch.from_numpy(np.ascontiguousarray(a)).to(device, non_blocking=True)
-                              for a in (self.members, self.parts, self.first_part))
+                              for a in (self.members, self.shared_tokens, self.first_token))
         return self
 
-    def bind(self, members: torch.Tensor, parts: torch.Tensor, first_part: torch.Tensor) -> "SharePlan":
+    def bind(self, members: torch.Tensor, shared_tokens: torch.Tensor, first_token: torch.Tensor) -> "SharePlan":
         """Uses caller-owned device tensors that already hold (or, in stream
         order before the call that reads them, will hold) this plan's arrays,
         e.g. filled by asynchronous copies from pinned host buffers."""
         if self.n_groups > 0:
-            self._dev = (members, parts, first_part)
+            self._dev = (members, shared_tokens, first_token)
         return self
 
     @property
     def nbytes(self) -> int:
         """Bytes the device copy takes (0 without groups)."""
-        return 0 if self.n_groups == 0 else self.members.nbytes + self.parts.nbytes + self.first_part.nbytes
+        return 0 if self.n_groups == 0 else self.members.nbytes + self.shared_tokens.nbytes + self.first_token.nbytes
 
     def ref(self):
         if self.n_groups == 0:
             return None
         if self._dev is None:
             raise ValueError("SharePlan.to(device) first")
-        m, pt, fp = self._dev
-        self._struct = pa_share_plan_t(m.data_ptr(), pt.data_ptr(), fp.data_ptr(), self.n_groups, self.max_members)
+        m, sh, ft = self._dev
+        self._struct = pa_share_plan_t(m.data_ptr(), sh.data_ptr(), ft.data_ptr(), self.n_groups, self.max_members)
         return ctypes.byref(self._struct)
 
 
-def share_plan(tables, lens, block_size: int, max_members: int = 4,
-               partition_tokens: int = PA_PARTITION_TOKENS) -> SharePlan:
+def share_plan(tables, lens, block_size: int, max_members: int = 4) -> SharePlan:
     """Host: groups the sequences of a batch whose tables agree on their
-    leading whole partitions of partition_tokens tokens (pa_share_plan; the
-    decode's pool must have the same partition size)."""
+    leading blocks (pa_share_plan)."""
     tables = np.ascontiguousarray(np.asarray(tables, dtype=np.int32))
     lens = np.ascontiguousarray(np.asarray(lens, dtype=np.int32))
     n = len(lens)
     cap = max(1, n // 2)
     members = np.empty((cap, max_members), dtype=np.int32)
-    parts = np.empty(cap, dtype=np.int32)
+    shared = np.empty(cap, dtype=np.int32)
     first = np.empty(n, dtype=np.int32)
     ng = ctypes.c_int32(0)
     _check(_lib.pa_share_plan(_i32p(tables), tables.shape[1] if tables.ndim == 2 else 0, _i32p(lens), n,
-                              int(block_size), int(partition_tokens), int(max_members), _i32p(members), _i32p(parts),
+                              int(block_size), int(max_members), _i32p(members), _i32p(shared),
                               _i32p(first), ctypes.byref(ng)), "pa_share_plan")
     g = ng.value
-    return SharePlan(members[:g].copy(), parts[:g].copy(), first)
+    return SharePlan(members[:g].copy(), shared[:g].copy(), first)
 
 
 def pa_decode_shared(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor, context_lens: torch.Tensor,
@@ -395,7 +405,7 @@ def pa_decode_shared(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor
                      cow_src: torch.Tensor | None = None, out: torch.Tensor | None = None,
                      workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """pa_decode, or pa_append_decode when k_new / v_new are given, with the
-    partitions a plan's groups share read once for all their members."""
+    blocks a plan's groups share read once for all their members."""
     _check_q_out(q, out, cache)
     B, Hq, D = q.shape
     if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
@@ -407,7 +417,9 @@ def pa_decode_shared(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor
         raise ValueError(f"k_new and v_new must be {list(row_shape)}")
     if out is None:
         out = torch.empty_like(q)
-    need = pa_decode_workspace_size(B, Hq, int(max_context_len), D, cache.partition_tokens)
+    size = (pa_decode_shared_workspace_size if plan is not None and plan.n_groups > 0
+            else pa_decode_workspace_size)
+    need = size(B, Hq, int(max_context_len), D, cache.partition_tokens)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = _dev(workspace, "workspace") if workspace is not None else None
@@ -523,8 +535,9 @@ class DecodeStepper:
         _check(_lib.pa_step_layout(self.n, self.Hq, cache.ref(), self.max_blocks, self.share, ctypes.byref(lay)),
                "pa_step_layout")
         self.layout = lay
-        ws_bytes = max(16, pa_decode_workspace_size(self.n, self.Hq, self.max_blocks * cache.block_size,
-                                                    cache.head_dim, cache.partition_tokens))
+        size = pa_decode_shared_workspace_size if self.share > 0 else pa_decode_workspace_size
+        ws_bytes = max(16, size(self.n, self.Hq, self.max_blocks * cache.block_size, cache.head_dim,
+                                cache.partition_tokens))
         Hkv, D, dt = cache.num_kv_heads, cache.head_dim, cache.dtype
         self._slots = []
         for _ in range(int(slots)):
@@ -627,30 +640,29 @@ class Allocator:
             _lib.pa_alloc_destroy(h)
             self._h = None
 
-    def decode_step(self, seqs, max_blocks: int, share_max_members: int = 4, out: dict | None = None,
-                    partition_tokens: int = PA_PARTITION_TOKENS) -> dict:
+    def decode_step(self, seqs, max_blocks: int, share_max_members: int = 4, out: dict | None = None) -> dict:
         """One decode step's host work in one call (pa_decode_step_prepare):
         one token appended to every sequence, then the tables, lengths,
         copy-on-write sources and sharing plan that pa_decode_shared takes.
         `out` may hold preallocated int32 arrays ("tables" [n, max_blocks],
-        "lens", "cow_src", "first_part" [n], "members" [n // 2, m], "parts"
-        [n // 2]); returns them (members / parts trimmed to the groups) with
+        "lens", "cow_src", "first_token" [n], "members" [n // 2, m],
+        "shared_tokens" [n // 2]); returns them (members / shared_tokens
+        trimmed to the groups) with
         "n_groups", "n_copies" and "max_len"."""
         seqs = np.ascontiguousarray(np.asarray(seqs, dtype=np.int32))
         n = len(seqs)
         m = max(int(share_max_members), 1)
         o = out if out is not None else {
             "tables": np.empty((n, max_blocks), np.int32), "lens": np.empty(n, np.int32),
-            "cow_src": np.empty(n, np.int32), "first_part": np.empty(n, np.int32),
-            "members": np.empty((max(1, n // 2), m), np.int32), "parts": np.empty(max(1, n // 2), np.int32)}
+            "cow_src": np.empty(n, np.int32), "first_token": np.empty(n, np.int32),
+            "members": np.empty((max(1, n // 2), m), np.int32), "shared_tokens": np.empty(max(1, n // 2), np.int32)}
         ng, nc, ml = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int32(0)
-        _check(_lib.pa_decode_step_prepare(self._h, _i32p(seqs), n, int(max_blocks), int(partition_tokens),
-                                           int(share_max_members),
+        _check(_lib.pa_decode_step_prepare(self._h, _i32p(seqs), n, int(max_blocks), int(share_max_members),
                                            _i32p(o["tables"]), _i32p(o["lens"]), _i32p(o["cow_src"]),
-                                           _i32p(o["members"]), _i32p(o["parts"]), _i32p(o["first_part"]),
+                                           _i32p(o["members"]), _i32p(o["shared_tokens"]), _i32p(o["first_token"]),
                                            ctypes.byref(ng), ctypes.byref(nc), ctypes.byref(ml)), "pa_decode_step_prepare")
         res = dict(o)
-        res["members"], res["parts"] = o["members"][:ng.value], o["parts"][:ng.value]
+        res["members"], res["shared_tokens"] = o["members"][:ng.value], o["shared_tokens"][:ng.value]
         res.update(n_groups=ng.value, n_copies=nc.value, max_len=ml.value)
         return res
 

@@ -311,51 +311,32 @@ PA_API pa_status pa_block_refcount(pa_allocator *a, int32_t block, int32_t *refc
 
 PA_API pa_status pa_share_plan(const int32_t *tables_host, int32_t max_blocks,
                                const int32_t *lens_host, int32_t n_seqs, int32_t block_size,
-                               int32_t partition_tokens, int32_t max_members, int32_t *members_host,
-                               int32_t *parts_host, int32_t *first_part_host, int32_t *n_groups) {
-  if (partition_tokens == 0) partition_tokens = PA_PARTITION_TOKENS;
+                               int32_t max_members, int32_t *members_host, int32_t *shared_host,
+                               int32_t *first_token_host, int32_t *n_groups) {
   if (n_seqs < 0 || max_blocks < 0 || !n_groups || max_members < 2 || max_members > 4 ||
-      (block_size != 8 && block_size != 16 && block_size != 32) ||
-      (partition_tokens != 256 && partition_tokens != 512 && partition_tokens != 1024))
+      (block_size != 8 && block_size != 16 && block_size != 32))
     return PA_ERR_INVALID_ARG;
-  const int32_t part = partition_tokens;
-  if (n_seqs > 0 && (!tables_host || !lens_host || !members_host || !parts_host || !first_part_host))
+  if (n_seqs > 0 && (!tables_host || !lens_host || !members_host || !shared_host || !first_token_host))
     return PA_ERR_INVALID_ARG;
   *n_groups = 0;
-  const int32_t bpp = part / block_size;  // table entries per partition
-  for (int32_t b = 0; b < n_seqs; ++b) first_part_host[b] = 0;
-  // sequences with at least two partitions (the first one whole, not the last)
-  std::vector<int32_t> cand;
-  for (int32_t b = 0; b < n_seqs; ++b)
-    if (lens_host[b] > part && max_blocks >= bpp) cand.push_back(b);
+  for (int32_t b = 0; b < n_seqs; ++b) first_token_host[b] = 0;
   auto row = [&](int32_t b) { return tables_host + (size_t)b * max_blocks; };
-  // buckets: equal first-partition entries, sequence order inside a bucket.
-  // Sequences are ordered by a hash of those entries (FNV-1a), then inside
-  // each run of equal hashes by their entries, then by index.
-  std::vector<std::pair<uint64_t, int32_t>> keyed;
-  keyed.reserve(cand.size());
-  for (int32_t b : cand) {
-    uint64_t h = 1469598103934665603ull;
-    const int32_t *r = row(b);
-    for (int32_t j = 0; j < bpp; ++j) {
-      h ^= (uint32_t)r[j];
-      h *= 1099511628211ull;
-    }
-    keyed.emplace_back(h, b);
+  auto nblocks = [&](int32_t b) { return (int32_t)(((int64_t)lens_host[b] + block_size - 1) / block_size); };
+  // sequences with a block before their last one: only such blocks can be
+  // shared (a sequence's last block is the one it writes)
+  std::vector<int32_t> cand;
+  for (int32_t b = 0; b < n_seqs; ++b) {
+    const int32_t nb = nblocks(b);
+    if (lens_host[b] > 0 && nb >= 2 && nb <= max_blocks) cand.push_back(b);
   }
-  std::sort(keyed.begin(), keyed.end(), [&](const std::pair<uint64_t, int32_t> &x,
-                                            const std::pair<uint64_t, int32_t> &y) {
-    if (x.first != y.first) return x.first < y.first;
-    const int32_t *rx = row(x.second), *ry = row(y.second);
-    if (!std::equal(rx, rx + bpp, ry)) return std::lexicographical_compare(rx, rx + bpp, ry, ry + bpp);
-    return x.second < y.second;
-  });
-  for (size_t k = 0; k < keyed.size(); ++k) cand[k] = keyed[k].second;
-  // the buckets, in the order of their first (lowest) sequence index
+  // buckets: the same first physical block (sharers point at the same blocks
+  // from the start), sequence order inside a bucket; buckets in the order of
+  // their first (lowest) sequence index
+  std::stable_sort(cand.begin(), cand.end(), [&](int32_t x, int32_t y) { return row(x)[0] < row(y)[0]; });
   std::vector<std::pair<size_t, size_t>> runs;
   for (size_t i = 0; i < cand.size();) {
     size_t e = i + 1;
-    while (e < cand.size() && std::equal(row(cand[i]), row(cand[i]) + bpp, row(cand[e]))) ++e;
+    while (e < cand.size() && row(cand[e])[0] == row(cand[i])[0]) ++e;
     runs.emplace_back(i, e);
     i = e;
   }
@@ -363,29 +344,27 @@ PA_API pa_status pa_share_plan(const int32_t *tables_host, int32_t max_blocks,
     return cand[x.first] < cand[y.first];
   });
   for (const auto &run : runs) {
-    const size_t i = run.first, e = run.second;
-    for (size_t g0 = i; g0 + 1 < e; g0 += (size_t)max_members) {
-      const size_t g1 = std::min(e, g0 + (size_t)max_members);
+    for (size_t g0 = run.first; g0 + 1 < run.second; g0 += (size_t)max_members) {
+      const size_t g1 = std::min(run.second, g0 + (size_t)max_members);
       if (g1 - g0 < 2) break;  // a lone leftover shares with nobody
-      // leading partitions that agree, are whole and come before every member's last
-      int32_t parts = 0;
-      for (;; ++parts) {
-        const int64_t end_tok = (int64_t)(parts + 1) * part;
-        if ((int64_t)(parts + 1) * bpp > max_blocks) break;
-        bool ok = true;
-        for (size_t k = g0; k < g1 && ok; ++k) {
-          const int32_t b = cand[k];
-          ok = lens_host[b] > end_tok &&
-               std::equal(row(cand[g0]) + (size_t)parts * bpp, row(cand[g0]) + (size_t)(parts + 1) * bpp,
-                          row(b) + (size_t)parts * bpp);
-        }
-        if (!ok) break;
+      // leading blocks on which every member agrees, each before every
+      // member's last block
+      int32_t lim = INT32_MAX;
+      for (size_t k = g0; k < g1; ++k) lim = std::min(lim, nblocks(cand[k]) - 1);
+      int32_t nshared = 0;
+      const int32_t *r0 = row(cand[g0]);
+      while (nshared < lim) {
+        bool same = true;
+        for (size_t k = g0 + 1; k < g1 && same; ++k) same = row(cand[k])[nshared] == r0[nshared];
+        if (!same) break;
+        ++nshared;
       }
-      if (parts < 1) continue;
+      const int32_t tokens = nshared * block_size;
+      if (tokens < PA_SHARE_MIN_TOKENS) continue;
       int32_t *mem = members_host + (size_t)(*n_groups) * max_members;
       for (int32_t k = 0; k < max_members; ++k) mem[k] = g0 + k < g1 ? cand[g0 + k] : -1;
-      parts_host[*n_groups] = parts;
-      for (size_t k = g0; k < g1; ++k) first_part_host[cand[k]] = parts;
+      shared_host[*n_groups] = tokens;
+      for (size_t k = g0; k < g1; ++k) first_token_host[cand[k]] = tokens;
       ++*n_groups;
     }
   }
@@ -393,19 +372,16 @@ PA_API pa_status pa_share_plan(const int32_t *tables_host, int32_t max_blocks,
 }
 
 PA_API pa_status pa_decode_step_prepare(pa_allocator *a, const int32_t *seqs, int32_t n_seqs,
-                                        int32_t max_blocks, int32_t partition_tokens,
-                                        int32_t share_max_members,
+                                        int32_t max_blocks, int32_t share_max_members,
                                         int32_t *tables_host, int32_t *lens_host,
                                         int32_t *cow_src_host, int32_t *members_host,
-                                        int32_t *parts_host, int32_t *first_part_host,
+                                        int32_t *shared_host, int32_t *first_token_host,
                                         int32_t *n_groups, int32_t *n_copies, int32_t *max_len) {
   if (!a || n_seqs < 0 || max_blocks < 0 || !n_groups || !n_copies || !max_len) return PA_ERR_INVALID_ARG;
-  if (n_seqs > 0 && (!seqs || !tables_host || !lens_host || !cow_src_host || !first_part_host))
+  if (n_seqs > 0 && (!seqs || !tables_host || !lens_host || !cow_src_host || !first_token_host))
     return PA_ERR_INVALID_ARG;
   if (share_max_members != 0 &&
-      (share_max_members < 2 || share_max_members > 4 || (n_seqs > 1 && (!members_host || !parts_host))))
-    return PA_ERR_INVALID_ARG;
-  if (partition_tokens != 0 && partition_tokens != 256 && partition_tokens != 512 && partition_tokens != 1024)
+      (share_max_members < 2 || share_max_members > 4 || (n_seqs > 1 && (!members_host || !shared_host))))
     return PA_ERR_INVALID_ARG;
   *n_groups = 0;
   *n_copies = 0;
@@ -445,11 +421,11 @@ PA_API pa_status pa_decode_step_prepare(pa_allocator *a, const int32_t *seqs, in
     *max_len = std::max(*max_len, s.len);
   }
   if (share_max_members == 0) {
-    for (int32_t i = 0; i < n_seqs; ++i) first_part_host[i] = 0;
+    for (int32_t i = 0; i < n_seqs; ++i) first_token_host[i] = 0;
     return PA_OK;
   }
-  return pa_share_plan(tables_host, max_blocks, lens_host, n_seqs, bs, partition_tokens, share_max_members,
-                       members_host, parts_host, first_part_host, n_groups);
+  return pa_share_plan(tables_host, max_blocks, lens_host, n_seqs, bs, share_max_members, members_host,
+                       shared_host, first_token_host, n_groups);
 }
 
 PA_API pa_status pa_cow_sources(const int32_t *pairs_host, int32_t n_pairs,

@@ -126,10 +126,18 @@ bool ensure_smem(Kernel kern, int bytes, std::atomic<int> (&done)[kMaxDev]) {
 }
 
 
-// workspace layout: m [B*Hq*P] f32 | l [B*Hq*P] f32 | acc [B*Hq*P*D] f32
-size_t workspace_bytes_for(int64_t B, int64_t Hq, int32_t max_ctx, int64_t D, int32_t part) {
-  if (max_ctx <= part) return 0;
-  const int64_t rows = B * Hq * (int64_t)max_parts_for(max_ctx, part);
+// workspace layout: m [B*Hq*R] f32 | l [B*Hq*R] f32 | acc [B*Hq*R*D] f32,
+// R rows per (sequence, query head): one per partition, plus, with a
+// sharing plan (extra), the row of the cascade's piece of the partition a
+// shared prefix ends in.
+int64_t row_stride_for(int32_t max_ctx, int32_t part, bool extra) {
+  return (max_ctx > 0 ? (int64_t)max_parts_for(max_ctx, part) : 1) + (extra ? 1 : 0);
+}
+
+size_t workspace_bytes_for(int64_t B, int64_t Hq, int32_t max_ctx, int64_t D, int32_t part,
+                           bool extra = false) {
+  if (!extra && max_ctx <= part) return 0;
+  const int64_t rows = B * Hq * row_stride_for(max_ctx, part, extra);
   return round16(rows * 4) * 2 + round16(rows * D * 4);
 }
 
@@ -146,11 +154,12 @@ int choose_stages(int tile_bytes) {
 }
 
 // The partition merge after a decode launch: with at most kReduceWide
-// partitions per row, a warp-per-row kernel (sized to the row's partition
-// bound, NP 4, 8 or 16, or the one that reads up to 32 partitions in rounds),
+// workspace rows per (sequence, query head), a warp-per-row kernel (sized to
+// the bound, NP 4, 8 or 16, or the one that reads up to 32 rows in rounds),
 // over a grid of at most 4 CTAs per SM; else one CTA per row.
 template <typename T, int D>
-pa_status launch_reduce(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
+pa_status launch_reduce(const pa::DecodeParams &p, cudaStream_t st) {
+  const int32_t max_parts = p.row_stride;  // rows a merge may read
   if (max_parts > pa::kReduceWide)
     return launch(pa::decode_reduce<T, D>, dim3(p.B * p.Hq), dim3(128), (size_t)max_parts * sizeof(float), st, p);
   const int64_t rows = (int64_t)p.B * p.Hq;
@@ -178,7 +187,7 @@ pa_status launch_decode_t(const pa::DecodeParams &p, int32_t max_parts, cudaStre
   dim3 grid(max_parts, p.Hkv, p.B);
   pa_status s = launch(kern, grid, dim3(pa::kWarps * 32), smem, st, p, nstages);
   if (s != PA_OK || max_parts <= 1) return s;
-  return launch_reduce<T, D>(p, max_parts, st);
+  return launch_reduce<T, D>(p, st);
 }
 
 template <typename T, int D>
@@ -267,11 +276,15 @@ bool tc_eligible(const pa::DecodeParams &p, int dtype, int D) {
 
 template <int G, int PART>
 pa_status launch_decode_tc_slice(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
-  CUtensorMap mk, mv, mq;
+  CUtensorMap mk, mv, mq, mq4;
   const uint64_t rows = (uint64_t)p.num_blocks * p.Hkv * p.bs;
+  // the query rows of a head-packed pass (pa::kPackHeads kv heads), when the
+  // group size allows packing
+  const uint32_t pack_rows = G <= 4 ? (uint32_t)(pa::kPackHeads * G) : (uint32_t)G;
   if (!make_map_pool_4d(&mk, p.k, rows, (uint32_t)p.bs) ||
       !make_map_pool_4d(&mv, p.v, rows, (uint32_t)p.bs) ||
-      !make_map_bf16_d128(&mq, p.q, (uint64_t)p.B * p.Hq, (uint32_t)G))
+      !make_map_bf16_d128(&mq, p.q, (uint64_t)p.B * p.Hq, (uint32_t)G) ||
+      !make_map_bf16_d128(&mq4, p.q, (uint64_t)p.B * p.Hq, pack_rows))
     return PA_ERR_CUDA;
   auto kern = pa::decode_partition_tc<G, PART>;
   const int smem = pa::TcLayout::kBytes;
@@ -281,13 +294,13 @@ pa_status launch_decode_tc_slice(const pa::DecodeParams &p, int32_t max_parts, c
   int grid = sm_count();
   if (grid <= 0) return PA_ERR_CUDA;
   if (units_bound < grid) grid = (int)units_bound;
-  pa_status s = launch(kern, dim3(grid), dim3(pa::TcLayout::kThreads), (size_t)smem, st, mk, mv, mq, p);
-  if (s != PA_OK || max_parts <= 1) return s;
-  return launch_reduce<__nv_bfloat16, 128>(p, max_parts, st);
+  return launch(kern, dim3(grid), dim3(pa::TcLayout::kThreads), (size_t)smem, st, mk, mv, mq, mq4, p);
 }
 
 // Sequences are independent: a batch larger than the kernel's per-CTA
-// sequence tables runs as consecutive launches over slices of it.
+// sequence tables runs as consecutive launches over slices of it, and one
+// reduce over the whole batch follows the last (each launch completes only
+// after the one before it, so the reduce sees every slice's rows).
 std::atomic<uint32_t> g_sched_ticket{0};
 
 template <int G, int PART>
@@ -310,21 +323,22 @@ pa_status launch_decode_tc_g(const pa::DecodeParams &p, int32_t max_parts, cudaS
       ps.v_new = static_cast<const __nv_bfloat16 *>(p.v_new) + (size_t)b0 * p.Hkv * 128;
       if (p.cow_src) ps.cow_src = p.cow_src + b0;
     }
-    if (p.first_part) ps.first_part = p.first_part + b0;
+    if (p.first_tok) ps.first_tok = p.first_tok + b0;
     if (p.ws_m) {
-      ps.ws_m = p.ws_m + rows * max_parts;
-      ps.ws_l = p.ws_l + rows * max_parts;
-      ps.ws_acc = p.ws_acc + rows * max_parts * 128;
+      ps.ws_m = p.ws_m + rows * p.row_stride;
+      ps.ws_l = p.ws_l + rows * p.row_stride;
+      ps.ws_acc = p.ws_acc + rows * p.row_stride * 128;
     }
     ps.sched_slot = (int32_t)(g_sched_ticket.fetch_add(1) % pa::kSchedSlots);
     const pa_status s = launch_decode_tc_slice<G, PART>(ps, max_parts, st);
     if (s != PA_OK) return s;
   }
-  return PA_OK;
+  if (p.row_stride <= 1) return PA_OK;  // one partition, no plan: written directly
+  return launch_reduce<__nv_bfloat16, 128>(p, st);
 }
 
-// The cascade kernel over the shared partitions of a sharing plan, in
-// slices of at most kMaxGroups groups.
+// The cascade kernel over the shared tokens of a sharing plan, in slices of
+// at most kMaxGroups groups.
 template <int G, int PART>
 pa_status launch_decode_shared_g(const pa::DecodeParams &p, const pa_share_plan_t &plan, cudaStream_t st) {
   CUtensorMap mk, mv, mq;
@@ -344,8 +358,8 @@ pa_status launch_decode_shared_g(const pa::DecodeParams &p, const pa_share_plan_
     sp.n_groups = plan.n_groups - j0 < pa::ShLayout::kMaxGroups ? plan.n_groups - j0 : pa::ShLayout::kMaxGroups;
     sp.max_members = plan.max_members;
     sp.members = plan.members + (size_t)j0 * plan.max_members;
-    sp.parts = plan.parts + j0;
-    const int64_t units_bound = (int64_t)sp.n_groups * p.Hkv * (p.max_parts > 1 ? p.max_parts - 1 : 1);
+    sp.shared = plan.shared_tokens + j0;
+    const int64_t units_bound = (int64_t)sp.n_groups * p.Hkv * (p.max_parts > 0 ? p.max_parts : 1);
     const int grid = units_bound < sms ? (int)units_bound : sms;
     const pa_status s = launch(kern, dim3(grid), dim3(pa::ShLayout::kThreads), (size_t)smem, st, mk, mv, mq, p, sp);
     if (s != PA_OK) return s;
@@ -520,6 +534,14 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
   return pa_decode_workspace_size_p(num_seqs, num_q_heads, max_context_len, head_dim, pa::kPart);
 }
 
+PA_API size_t pa_decode_shared_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                              int32_t max_context_len, int32_t head_dim,
+                                              int32_t partition_tokens) {
+  const int32_t part = partition_tokens ? partition_tokens : pa::kPart;
+  if (num_seqs <= 0 || num_q_heads <= 0 || max_context_len <= 0 || head_dim <= 0 || !part_ok(part)) return 0;
+  return workspace_bytes_for(num_seqs, num_q_heads, max_context_len, head_dim, part, true);
+}
+
 }  // extern "C"
 
 namespace {
@@ -530,7 +552,7 @@ pa_status prepare_decode(const void *q, const pa_cache_t *cache, const int32_t *
                          int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
                          int32_t num_q_heads, int32_t max_context_len, float scale, void *out,
                          void *workspace, size_t workspace_bytes, pa::DecodeParams *pp,
-                         bool *skip) {
+                         bool *skip, bool extra_row = false) {
   *skip = false;
   pa_status s = check_cache(cache);
   if (s != PA_OK) return s;
@@ -551,12 +573,13 @@ pa_status prepare_decode(const void *q, const pa_cache_t *cache, const int32_t *
   if ((int64_t)max_context_len > (int64_t)max_blocks_per_seq * bs) return PA_ERR_INVALID_ARG;
   const int32_t part = part_of(cache);
   if (max_context_len > INT32_MAX - part) return PA_ERR_INVALID_ARG;
-  const size_t need = workspace_bytes_for(num_seqs, num_q_heads, max_context_len, cache->head_dim, part);
+  const size_t need = workspace_bytes_for(num_seqs, num_q_heads, max_context_len, cache->head_dim, part, extra_row);
   if (need > 0) {
     if (!workspace || !aligned16(workspace)) return PA_ERR_INVALID_ARG;
     if (workspace_bytes < need) return PA_ERR_TOO_SMALL;
   }
   const int32_t max_parts = max_context_len > 0 ? max_parts_for(max_context_len, part) : 1;
+  const int64_t row_stride = row_stride_for(max_context_len, part, extra_row);
 
   pa::DecodeParams p{};
   p.q = q;
@@ -566,7 +589,7 @@ pa_status prepare_decode(const void *q, const pa_cache_t *cache, const int32_t *
   p.tables = block_tables;
   p.lens = context_lens;
   if (need > 0) {
-    const int64_t rows = (int64_t)num_seqs * num_q_heads * max_parts;
+    const int64_t rows = (int64_t)num_seqs * num_q_heads * row_stride;
     char *w = static_cast<char *>(workspace);
     p.ws_m = reinterpret_cast<float *>(w);
     p.ws_l = reinterpret_cast<float *>(w + round16(rows * 4));
@@ -581,6 +604,7 @@ pa_status prepare_decode(const void *q, const pa_cache_t *cache, const int32_t *
   p.B = num_seqs;
   p.max_ctx = max_context_len;
   p.max_parts = max_parts;
+  p.row_stride = (int32_t)row_stride;
   p.part = part;
   p.scale_log2 = scale * 1.4426950408889634f;
   *pp = p;
@@ -699,19 +723,16 @@ PA_API pa_status pa_decode_shared(const void *k_new, const void *v_new, const in
                                   size_t workspace_bytes, void *stream) {
   pa::DecodeParams p{};
   bool skip = false;
+  const bool grouped = plan && plan->n_groups > 0;
+  if (grouped && (!plan->members || !plan->shared_tokens || !plan->first_token ||
+                  plan->max_members < 1 || plan->max_members > pa::ShLayout::kSlots))
+    return PA_ERR_INVALID_ARG;
   pa_status s = prepare_decode(q, cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
                                num_q_heads, max_context_len, scale, out, workspace, workspace_bytes,
-                               &p, &skip);
+                               &p, &skip, grouped);
   if (s != PA_OK || skip) return s;
   if ((k_new == nullptr) != (v_new == nullptr)) return PA_ERR_INVALID_ARG;
   if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return PA_ERR_INVALID_ARG;
-  const bool grouped = plan && plan->n_groups > 0;
-  if (grouped) {
-    if (!plan->members || !plan->parts || !plan->first_part || plan->n_groups < 0 ||
-        plan->max_members < 1 || plan->max_members > pa::ShLayout::kSlots)
-      return PA_ERR_INVALID_ARG;
-    if (p.max_parts < 2) return PA_ERR_INVALID_ARG;  // a shared partition is never a sequence's last
-  }
   cudaStream_t st = (cudaStream_t)stream;
   if (!tc_eligible(p, cache->dtype, cache->head_dim)) {
     // no cascade kernel on the CUDA-core path: every sequence computes all
@@ -730,7 +751,7 @@ PA_API pa_status pa_decode_shared(const void *k_new, const void *v_new, const in
   if (grouped) {
     s = launch_decode_shared(p, *plan, st);
     if (s != PA_OK) return s;
-    p.first_part = plan->first_part;
+    p.first_tok = plan->first_token;
     p.late_wait = 1;
   }
   p.k_new = k_new;
@@ -891,9 +912,9 @@ PA_API pa_status pa_step_layout(int32_t n_seqs, int32_t num_q_heads, const pa_ca
   L.tables = layout_take(&at, n * (size_t)max_blocks * 4);
   L.lens = layout_take(&at, n * 4);
   L.cow_src = layout_take(&at, n * 4);
-  L.first_part = layout_take(&at, n * 4);
+  L.first_token = layout_take(&at, n * 4);
   L.members = layout_take(&at, groups * members * 4);
-  L.parts = layout_take(&at, groups * 4);
+  L.shared_tokens = layout_take(&at, groups * 4);
   L.bytes = at;
   *layout = L;
   return PA_OK;
@@ -958,15 +979,17 @@ PA_API pa_status pa_decode_step(pa_allocator *a, const int32_t *seqs_host, int32
   const int32_t part = part_of(cache);
   if (ctx_cap > INT32_MAX - part) return PA_ERR_INVALID_ARG;
   const size_t need_ws =
-      n_seqs > 0 ? workspace_bytes_for(n_seqs, num_q_heads, (int32_t)ctx_cap, cache->head_dim, part) : 0;
+      n_seqs > 0 ? workspace_bytes_for(n_seqs, num_q_heads, (int32_t)ctx_cap, cache->head_dim, part,
+                                       share_max_members > 0)
+                 : 0;
   if (need_ws > 0 && (!slot->workspace || slot->workspace_bytes < need_ws)) return PA_ERR_TOO_SMALL;
   char *h = static_cast<char *>(slot->host);
   char *d = static_cast<char *>(slot->dev);
   auto hi = [&](size_t off) { return reinterpret_cast<int32_t *>(h + off); };
   auto di = [&](size_t off) { return reinterpret_cast<int32_t *>(d + off); };
-  s = pa_decode_step_prepare(a, seqs_host, n_seqs, max_blocks, part, share_max_members, hi(L.tables), hi(L.lens),
-                             hi(L.cow_src), hi(L.members), hi(L.parts), hi(L.first_part), n_groups, n_copies,
-                             max_len);
+  s = pa_decode_step_prepare(a, seqs_host, n_seqs, max_blocks, share_max_members, hi(L.tables), hi(L.lens),
+                             hi(L.cow_src), hi(L.members), hi(L.shared_tokens), hi(L.first_token), n_groups,
+                             n_copies, max_len);
   if (s != PA_OK || n_seqs == 0) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaStream_t hst = static_cast<cudaStream_t>(h2d_stream);
@@ -982,7 +1005,7 @@ PA_API pa_status pa_decode_step(pa_allocator *a, const int32_t *seqs_host, int32
   // the decode: after the inputs, and after the previous output left out_dev
   if ((e = cudaStreamWaitEvent(st, ev_in, 0)) != cudaSuccess) return cuda_failed(e);
   if ((e = cudaStreamWaitEvent(st, ev_out, 0)) != cudaSuccess) return cuda_failed(e);
-  pa_share_plan_t plan{di(L.members), di(L.parts), di(L.first_part), *n_groups,
+  pa_share_plan_t plan{di(L.members), di(L.shared_tokens), di(L.first_token), *n_groups,
                        share_max_members > 0 ? share_max_members : 1};
   s = pa_decode_shared(d + L.k_new, d + L.v_new, *n_copies > 0 ? di(L.cow_src) : nullptr, d + L.q, cache,
                        di(L.tables), max_blocks, di(L.lens), n_seqs, num_q_heads, *max_len, scale,

@@ -8,20 +8,22 @@
 // "PagedAttention Internals", "Sharing And Dynamic Growth").  The attention
 // of each sequence over such a block is still its own: this kernel computes,
 // for a group of up to kSlots sequences whose block tables agree on their
-// first `parts` whole partitions, each member's split-context statistics
-// (max, sum, unnormalised accumulator) of those partitions, exactly what
-// decode_partition_tc would write for them, into the same workspace rows.
-// decode_partition_tc then does every sequence from its first private
-// partition on, and the log-sum-exp reduce merges both.
+// first `shared` tokens (a whole number of blocks), each member's
+// split-context statistics (max, sum, unnormalised accumulator) of those
+// tokens, cut at the partition boundaries: the whole partitions among them
+// go to the rows decode_partition_tc would write for them, the piece of the
+// partition the shared tokens end in (if they end inside one) to the
+// member's extra row.  decode_partition_tc then does every sequence from its
+// first private token on, and the log-sum-exp reduce merges them all.
 //
 // Same machinery as decode_partition_tc (see there): persistent CTAs, a TMA
 // producer warp loading whole (block, kv head) tiles as 4-D boxes into
 // 128-byte-swizzled K and V rings, one MMA warp, softmax warps with the lazy
 // reference and the transposed column reductions.  What differs:
-//  * a work unit is (group, kv head, shared partition): 512 tokens, always
-//    full, handed out round-robin (all units are the same size); the
-//    producer loads the next unit's description while the current unit's
-//    copies are in flight;
+//  * a work unit is (group, kv head, piece): a whole partition or the
+//    shorter piece at the end of the shared tokens, handed out round-robin;
+//    the producer loads the next unit's description while the current
+//    unit's copies are in flight;
 //  * the Q tile holds the group's members in 8-row slots (member m: rows
 //    8m .. 8m + G - 1, one 2-D TMA box per column half per member), so the
 //    MMAs are M = 128 tokens x N = 32 query rows;
@@ -57,13 +59,15 @@ struct ShLayout {
   static constexpr int kRedFloats = 2 * 4 * kN;  // [parity][warp][column]
   static constexpr int kOffRedSum = kOffRed + kRedFloats * 4;
   static constexpr int kOffTmem = kOffRedSum + kRedFloats * 4;
-  // unit slot: [group, kv head, partition, members, b_0 .. b_3] + the table
-  // entries of the partition (from the first member's table)
-  static constexpr int kUnitInts = 8 + TcLayout::kMaxPart / 8;
+  // unit slot: [group, kv head, workspace row, members, b_0 .. b_3, chunks,
+  // -, -, -] + the table entries of the piece (from the first member's table)
+  static constexpr int kUnitHead = 12;
+  static constexpr int kUnitInts = kUnitHead + TcLayout::kMaxPart / 8;
   static constexpr int kOffUnit = kOffTmem + 16;
   static constexpr int kOffScan = kOffUnit + 2 * kUnitInts * 4;
-  static constexpr int kOffPrefix = kOffScan + 64;  // shared partitions before each group
-  static constexpr int kBytes = kOffPrefix + (kMaxGroups + 1) * 4 + 1024;
+  static constexpr int kOffPrefix = kOffScan + 64;  // pieces before each group
+  static constexpr int kOffShared = kOffPrefix + (kMaxGroups + 1) * 4;  // each group's shared tokens
+  static constexpr int kBytes = kOffShared + kMaxGroups * 4 + 1024;
   static constexpr int kThreads = 320;
   static constexpr uint32_t kTmemCols = 128;  // S0 S1 O0 O1, kN columns each
 };
@@ -84,10 +88,11 @@ __device__ __forceinline__ bool grp_sync_or(int pred, int grp) {
 }
 
 // The sharing plan of one launch: group j has members[j * max_members + m]
-// (m < max_members, -1 past its last member) sharing parts[j] partitions.
+// (m < max_members, -1 past its last member) sharing their first shared[j]
+// tokens (a whole number of blocks).
 struct SharedParams {
   const int32_t *members;
-  const int32_t *parts;
+  const int32_t *shared;
   int32_t n_groups;
   int32_t max_members;
 };
@@ -115,6 +120,7 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
   uint64_t *qfull = bars + 8, *qempty = bars + 10, *sfull = bars + 12, *pfull = bars + 14;
   uint64_t *pvdone = bars + 16, *ofree = bars + 18, *drain = bars + 20;
   int32_t *gprefix = reinterpret_cast<int32_t *>(smem + L::kOffPrefix);
+  int32_t *gshared = reinterpret_cast<int32_t *>(smem + L::kOffShared);
   int32_t *scan = reinterpret_cast<int32_t *>(smem + L::kOffScan);
   int32_t *unit_slots = reinterpret_cast<int32_t *>(smem + L::kOffUnit);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffTmem);
@@ -144,8 +150,9 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
   for (int i = threadIdx.x; i < (2 * L::kQ + 2 * L::kP) / 16; i += blockDim.x)
     reinterpret_cast<uint4 *>(smem + L::kOffQ)[i] = make_uint4(0, 0, 0, 0);
 
-  // shared partitions per group and their exclusive prefix sums (the plan is
-  // caller data that no kernel of the library writes: read before the wait)
+  // pieces per group (its shared tokens cut at the partition boundaries) and
+  // their exclusive prefix sums (the plan is caller data that no kernel of
+  // the library writes: read before the wait)
   const int NG = sp.n_groups;
   constexpr int kMaxSeg = (L::kMaxGroups + L::kThreads - 1) / L::kThreads;
   const int seg = (NG + blockDim.x - 1) / blockDim.x;
@@ -157,7 +164,13 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
     cnt[i] = 0;
     const int j = j_first + i;
     if (i < seg && j < NG) {
-      cnt[i] = max(sp.parts[j], 0);
+      const int S = sp.shared[j];
+      if (S < 0 || S % p.bs != 0 || S / p.bs > p.max_blocks) {
+        if (blockIdx.x == 0) raise_error(PA_DEVERR_PLAN);
+      } else {
+        cnt[i] = (S + PART - 1) / PART;
+      }
+      gshared[j] = S;
       mine += cnt[i];
     }
   }
@@ -200,13 +213,13 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
     const uint64_t pol_q = tc::policy_evict_last();
     const int bs = p.bs;
     const int blocks_per_chunk = L::kChunk / bs;
-    const int nb_unit = PART / bs;  // blocks of a (whole) partition
     const int oob_group = p.num_blocks * p.Hkv * (bs / 8);
+    const int lg_bs = bs == 8 ? 3 : (bs == 16 ? 4 : 5);
     int c = 0, qi = 0;
     bool ok = true;
-    // unit u: kv head u % Hkv of shared partition u / Hkv in the groups' order
+    // unit u: kv head u % Hkv of piece u / Hkv in the groups' order
     struct ShUnit {
-      int j, g, part, nmem;
+      int j, g, row, nmem, nb, nchunks;
       int32_t b[L::kSlots];
     };
     auto pick = [](const int32_t (&x)[NE], int k) {  // x[k] by selects, never a local-memory index
@@ -228,7 +241,13 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
         if (gprefix[mid] <= w) lo = mid; else hi = mid - 1;
       }
       un.j = lo;
-      un.part = w - gprefix[lo];
+      // piece k: tokens [k PART, min((k + 1) PART, S)); a whole partition
+      // goes to row k, the shorter last piece to the extra row max_parts
+      const int k = w - gprefix[lo], S = gshared[lo];
+      const int t0 = k * PART, t1 = min(t0 + PART, S);
+      un.row = t1 - t0 == PART ? k : p.max_parts;
+      un.nb = (t1 - t0) >> lg_bs;
+      un.nchunks = (t1 - t0 + L::kChunk - 1) / L::kChunk;
       const int32_t mb = lane < L::kSlots && lane < sp.max_members ? sp.members[(size_t)lo * sp.max_members + lane] : -1;
       int nmem = 0;
 #pragma unroll
@@ -238,10 +257,10 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
       }
       un.nmem = nmem;
       if (nmem == 0) return;
-      const int32_t *tr = p.tables + (size_t)un.b[0] * p.max_blocks + (size_t)un.part * nb_unit;
+      const int32_t *tr = p.tables + (size_t)un.b[0] * p.max_blocks + (t0 >> lg_bs);
 #pragma unroll
-      for (int k = 0; k < NE; ++k)
-        if (lane + 32 * k < nb_unit) x[k] = tr[lane + 32 * k];
+      for (int e = 0; e < NE; ++e)
+        if (lane + 32 * e < un.nb) x[e] = tr[lane + 32 * e];
     };
     ShUnit un{}, nx{};
     int32_t e[NE], f[NE];
@@ -262,13 +281,14 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
           if (lane == 0) {
             us[0] = un.j;
             us[1] = un.g;
-            us[2] = un.part;
+            us[2] = un.row;
             us[3] = un.nmem;
 #pragma unroll
             for (int m = 0; m < L::kSlots; ++m) us[4 + m] = un.b[m];
+            us[8] = un.nchunks;
           }
 #pragma unroll
-          for (int k = 0; k < NE; ++k) us[8 + 32 * k + lane] = e[k];
+          for (int k = 0; k < NE; ++k) us[L::kUnitHead + 32 * k + lane] = e[k];
           __syncwarp();
         }
         if (lane == 0) {
@@ -281,7 +301,7 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
           }
         }
         ++qi;
-        for (int ci = 0; ci < PART / L::kChunk; ++ci, ++c) {
+        for (int ci = 0; ci < un.nchunks; ++ci, ++c) {
           const int slot = c % L::kStages, use = c / L::kStages;
           for (int which = 0; which < 2; ++which) {  // 0: K ring, 1: V ring
             uint64_t *empty = which ? &vempty[slot] : &kempty[slot];
@@ -294,9 +314,11 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
             const int jloc = ci * blocks_per_chunk + (lane % blocks_per_chunk);
             const int32_t blk = __shfl_sync(0xffffffffu, pick(e, (ci * blocks_per_chunk) >> 5), jloc & 31);
             if (lane < blocks_per_chunk) {
-              int w = oob_group;
-              if (blk >= 0 && blk < p.num_blocks) w = (blk * p.Hkv + un.g) * (bs / 8);
-              else if (which == 0) raise_error(PA_DEVERR_TABLE);
+              int w = oob_group;  // past the piece's last block: the fill value
+              if (jloc < un.nb) {
+                if (blk >= 0 && blk < p.num_blocks) w = (blk * p.Hkv + un.g) * (bs / 8);
+                else if (which == 0) raise_error(PA_DEVERR_TABLE);
+              }
               tc::tma_load_4d(dst + lane * (bs / 8) * L::kGroup, map, 0, 0, 0, w, full, pol_kv);
             }
           }
@@ -377,7 +399,7 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
       if (!warp_wait(&qfull[qs], (qi >> 1) & 1)) { ok = false; break; }
       if (unit_slots[qs * L::kUnitInts + 3] == 0) break;  // the producer ran out of work
       const uint32_t qb = qbase0 + qs * L::kQ;
-      constexpr int nchunks = PART / L::kChunk;
+      const int nchunks = unit_slots[qs * L::kUnitInts + 8];
       for (int ci = 0; ci < nchunks; ++ci, ++c) {
         const int slot = c % L::kStages;
         if (!warp_wait(&kfull[slot], (c / L::kStages) & 1)) { ok = false; break; }
@@ -430,7 +452,7 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
     const int bs = p.bs;
     const int log2_bs = bs == 8 ? 3 : (bs == 16 ? 4 : 5);
     float m[NC], l[NC];
-    int pun_g = 0, pun_part = 0, pun_nmem = 0, pun_b[L::kSlots] = {0, 0, 0, 0};
+    int pun_g = 0, pun_row = 0, pun_nmem = 0, pun_b[L::kSlots] = {0, 0, 0, 0};
     bool pend = false;
     int p_clast = 0, p_u = 0;
     bool bad = false, stop = false;
@@ -463,11 +485,11 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
       stop = grp_sync_or(bad, grp);
       if (stop) return;
       // workspace rows of the group's two member slots at query head 0;
-      // column j is row rb[j / 8] + (j % 8) * max_parts
+      // column j is row rb[j / 8] + (j % 8) * row_stride
       const size_t hb = (size_t)pun_g * G;
-      const size_t rb0 = ((size_t)(grp ? pun_b[2] : pun_b[0]) * p.Hq + hb) * p.max_parts + pun_part;
-      const size_t rb1 = ((size_t)(grp ? pun_b[3] : pun_b[1]) * p.Hq + hb) * p.max_parts + pun_part;
-      auto ws_row = [&](int j) { return (j < 8 ? rb0 : rb1) + (size_t)(j & 7) * p.max_parts; };
+      const size_t rb0 = ((size_t)(grp ? pun_b[2] : pun_b[0]) * p.Hq + hb) * p.row_stride + pun_row;
+      const size_t rb1 = ((size_t)(grp ? pun_b[3] : pun_b[1]) * p.Hq + hb) * p.row_stride + pun_row;
+      auto ws_row = [&](int j) { return (j < 8 ? rb0 : rb1) + (size_t)(j & 7) * p.row_stride; };
 #pragma unroll
       for (int j = 0; j < NC; ++j)
         if (col_valid(c0 + j, pun_nmem)) p.ws_acc[ws_row(j) * 128 + r] = o[j];
@@ -499,17 +521,16 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
         if (stop) break;
       }
       if (nmem == 0) break;  // the producer ran out of work
-      const int ug = us[1], upart = us[2];
+      const int ug = us[1], urow = us[2], nchunks = us[8];
       int ub[L::kSlots];
 #pragma unroll
       for (int k = 0; k < L::kSlots; ++k) ub[k] = us[4 + k];
-      const int32_t *ents = us + 8;
+      const int32_t *ents = us + L::kUnitHead;  // -1 past the piece: those tokens are masked
 #pragma unroll
       for (int j = 0; j < NC; ++j) {
         m[j] = -INFINITY;
         l[j] = 0.f;
       }
-      constexpr int nchunks = PART / L::kChunk;
       for (int ci = 0; ci < nchunks; ++ci, ++c) {
         float s[NC];
         warp_wait(&sfull[c & 1], (c >> 1) & 1);
@@ -604,7 +625,7 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
       if (stop) break;
       pend = true;
       pun_g = ug;
-      pun_part = upart;
+      pun_row = urow;
       pun_nmem = nmem;
 #pragma unroll
       for (int k = 0; k < L::kSlots; ++k) pun_b[k] = ub[k];

@@ -38,6 +38,10 @@ struct DecodeParams {
   float *ws_acc;  // [B][Hq][max_parts][D] unnormalised accumulator
   int32_t num_blocks, Hkv, bs, Hq, G, max_blocks, B, max_ctx, max_parts;
   int32_t part;  // tokens per split-context partition (256, 512 or 1024)
+  // workspace rows per (sequence, query head): max_parts, or max_parts + 1
+  // with a sharing plan (row max_parts: the cascade's piece of the partition
+  // a shared prefix ends in)
+  int32_t row_stride;
   int32_t sched_slot;  // tensor-core kernel: which run-time work counter this call uses
   float scale_log2;  // scale * log2(e)
   // fused step (tensor-core kernel): the newest token's rows [B][Hkv][D] and
@@ -45,10 +49,10 @@ struct DecodeParams {
   const void *k_new;
   const void *v_new;
   const int32_t *cow_src;
-  // shared-prefix plan (tensor-core kernel): sequence b computes partitions
-  // from first_part[b] on; the ones before are done by the cascade kernel.
-  // Null: every sequence from partition 0.
-  const int32_t *first_part;
+  // shared-prefix plan (tensor-core kernel): sequence b's tokens before
+  // first_tok[b] are done by the cascade kernel, the partition kernel does
+  // the rest.  Null: every sequence from token 0.
+  const int32_t *first_tok;
   // tensor-core kernel launched right after the cascade kernel: nothing it
   // reads or writes is touched by that kernel, and everything of the calls
   // before it had completed when the cascade kernel let it start, so it waits
@@ -285,7 +289,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     if (nparts == 1) {
       store_out(out + ((size_t)b * p.Hq + h) * D + d, L > 0.f ? A / L : 0.f);
     } else {
-      const size_t row = ((size_t)b * p.Hq + h) * p.max_parts + part;
+      const size_t row = ((size_t)b * p.Hq + h) * p.row_stride + part;
       p.ws_acc[row * D + d] = A;
       if (d == 0) {
         p.ws_m[row] = M;
@@ -330,6 +334,32 @@ __device__ __forceinline__ float merge_element(const float (&av)[NP], const floa
   return L > 0.f ? a / L : 0.f;
 }
 
+// The first token of sequence b that the partition kernel does: first_tok[b]
+// when it is a whole number of blocks inside the sequence, else 0 (the
+// partition kernel then does the whole sequence).  The partition kernel and
+// the merges apply the same rule.
+__device__ __forceinline__ int first_token_of(const DecodeParams &p, int b, int ctx) {
+  if (!p.first_tok) return 0;
+  const int t = p.first_tok[b];
+  return (t > 0 && t < ctx && t % p.bs == 0) ? t : 0;
+}
+
+// The merge of row (b, h) takes np = ceil(ctx / part) partition rows, then,
+// when the sequence's shared prefix ends inside a partition, the extra row
+// (index max_parts) with the cascade's piece of that partition: the number
+// of such slots, 0 when the partition kernel wrote the output directly (one
+// partition, no shared prefix) or the length is out of range.
+__device__ __forceinline__ int merge_slots(const DecodeParams &p, int ctx, int ft) {
+  if (ctx <= 0 || ctx > p.max_ctx) return 0;
+  if (ctx <= p.part && ft == 0) return 0;
+  return (ctx + p.part - 1) / p.part + (ft % p.part != 0 ? 1 : 0);
+}
+
+// The workspace row of merge slot i of a sequence of np partitions.
+__device__ __forceinline__ int slot_row(const DecodeParams &p, int np, int i) {
+  return i < np ? i : p.max_parts;
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(128) decode_reduce(DecodeParams p) {
   extern __shared__ float wsh[];  // [max_parts] weights
@@ -339,34 +369,39 @@ __global__ void __launch_bounds__(128) decode_reduce(DecodeParams p) {
   const int bh = blockIdx.x;
   const int b = bh / p.Hq;
   const int ctx = p.lens[b];
-  if (ctx <= p.part || ctx > p.max_ctx) return;  // written directly by the partition kernel
-  const int np = (ctx + p.part - 1) / p.part;
-  const float *m = p.ws_m + (size_t)bh * p.max_parts;
-  const float *l = p.ws_l + (size_t)bh * p.max_parts;
+  const int ns = merge_slots(p, ctx, first_token_of(p, b, ctx));
+  if (ns == 0) return;  // written directly by the partition kernel
+  const int npart = (ctx + p.part - 1) / p.part;
+  const float *m = p.ws_m + (size_t)bh * p.row_stride;
+  const float *l = p.ws_l + (size_t)bh * p.row_stride;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
 
-  if (np <= kReduceFast && D <= 128) {
-    // Up to kReduceFast partitions: every thread loads all the maxima and
-    // sums (the same addresses in every thread) and its own accumulator
-    // elements in one round, then merges on its own, with no barrier.
+  if (ns <= kReduceFast && D <= 128) {
+    // Up to kReduceFast slots: every thread loads all the maxima and sums
+    // (the same addresses in every thread) and its own accumulator elements
+    // in one round, then merges on its own, with no barrier.
     const int d = threadIdx.x;
-    const float *acc = p.ws_acc + (size_t)bh * p.max_parts * D;
+    const float *acc = p.ws_acc + (size_t)bh * p.row_stride * D;
     float mv[kReduceFast], lv[kReduceFast], av[kReduceFast];
 #pragma unroll
     for (int i = 0; i < kReduceFast; ++i) {
-      const bool in = i < np;
-      mv[i] = in ? __ldcg(m + i) : -INFINITY;
-      lv[i] = in ? __ldcg(l + i) : 0.f;
-      av[i] = (in && d < D) ? __ldcg(acc + (size_t)i * D + d) : 0.f;
+      const bool in = i < ns;
+      const int rw = slot_row(p, npart, i);
+      mv[i] = in ? __ldcg(m + rw) : -INFINITY;
+      lv[i] = in ? __ldcg(l + rw) : 0.f;
+      av[i] = (in && d < D) ? __ldcg(acc + (size_t)rw * D + d) : 0.f;
     }
     float f[kReduceFast];
-    const float L = merge_weights(mv, lv, np, f);
-    if (d < D) store_out(reinterpret_cast<T *>(p.out) + (size_t)bh * D + d, merge_element(av, f, np, L));
+    const float L = merge_weights(mv, lv, ns, f);
+    if (d < D) store_out(reinterpret_cast<T *>(p.out) + (size_t)bh * D + d, merge_element(av, f, ns, L));
     return;
   }
 
-  float mx = -INFINITY;
-  for (int i = threadIdx.x; i < np; i += blockDim.x) mx = fmaxf(mx, m[i]);
+  // slots 0 .. npart - 1 are rows 0 .. npart - 1; a last slot past them
+  // (extra) is row max_parts
+  const bool extra = ns > npart;
+  float mx = extra && threadIdx.x == 0 ? m[p.max_parts] : -INFINITY;
+  for (int i = threadIdx.x; i < npart; i += blockDim.x) mx = fmaxf(mx, m[i]);
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   if (lane == 0) red[warp] = mx;
   __syncthreads();
@@ -374,90 +409,124 @@ __global__ void __launch_bounds__(128) decode_reduce(DecodeParams p) {
   for (int w = 1; w < nw; ++w) M = fmaxf(M, red[w]);
   __syncthreads();
 
-  for (int i = threadIdx.x; i < np; i += blockDim.x) wsh[i] = (m[i] == -INFINITY) ? 0.f : fast_exp2(m[i] - M);
+  for (int i = threadIdx.x; i < ns; i += blockDim.x) {
+    const float mi = m[i < npart ? i : p.max_parts];
+    wsh[i] = (mi == -INFINITY) ? 0.f : fast_exp2(mi - M);
+  }
   __syncthreads();
   // L = sum_i l_i f_i in partition order by fused multiply-adds, the order
   // of merge_weights, so that every merge kernel gives the same bits
   if (threadIdx.x == 0) {
     float ls = 0.f;
-    for (int i = 0; i < np; ++i) ls = fmaf(l[i], wsh[i], ls);
+    for (int i = 0; i < npart; ++i) ls = fmaf(l[i], wsh[i], ls);
+    if (extra) ls = fmaf(l[p.max_parts], wsh[npart], ls);
     red[0] = ls;
   }
   __syncthreads();
   const float L = red[0];
   (void)nw;
 
-  const float *acc = p.ws_acc + (size_t)bh * p.max_parts * D;
+  const float *acc = p.ws_acc + (size_t)bh * p.row_stride * D;
   T *out = reinterpret_cast<T *>(p.out) + (size_t)bh * D;
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     float a = 0.f;
-    for (int i = 0; i < np; ++i) a = fmaf(acc[(size_t)i * D + d], wsh[i], a);
+    for (int i = 0; i < npart; ++i) a = fmaf(acc[(size_t)i * D + d], wsh[i], a);
+    if (extra) a = fmaf(acc[(size_t)p.max_parts * D + d], wsh[npart], a);
     store_out(out + d, L > 0.f ? a / L : 0.f);
   }
 }
 
-// decode_reduce for calls whose rows have at most NP <= kReduceFast
-// partitions: one warp per (sequence, query head) row, lane j holding the
-// head-dim elements [j * D / 32, (j + 1) * D / 32); lane i < np loads
-// partition i's max and sum and the warp shares them by shuffle.  Rows are
-// taken in a grid-stride loop, so a few resident CTAs cover any batch and
-// the register footprint follows NP.  Same merge arithmetic as decode_reduce.
+// decode_reduce for calls whose rows have at most NP <= kReduceFast merge
+// slots: one warp per (sequence, query head) row, lane j holding the
+// head-dim elements [j * D / 32, (j + 1) * D / 32).  A row's loads do not
+// wait for its length: lane i < row_stride loads workspace row i's max and
+// sum, and every lane its elements of rows 0 .. kReducePre - 1 and of the
+// extra row, all at once with the length and first token; the row's slot
+// count then picks among them (rows past it are read but not used), and
+// the slots past the preloaded rows are loaded after it, all before the
+// first multiply-add.  Rows are taken in a grid-stride loop.  Same merge
+// arithmetic, in the same slot order, as decode_reduce.
 constexpr int kReduceRowWarps = 8;
+constexpr int kReducePre = 4;
+
+template <int E>
+__device__ __forceinline__ void load_acc_row(const float *src, float (&v)[E]) {
+  if constexpr (E == 4) {
+    const float4 x = __ldcg(reinterpret_cast<const float4 *>(src));
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else if constexpr (E == 2) {
+    const float2 x = __ldcg(reinterpret_cast<const float2 *>(src));
+    v[0] = x.x; v[1] = x.y;
+  } else {
+    v[0] = __ldcg(src);
+  }
+}
 
 template <typename T, int D, int NP>
 __global__ void __launch_bounds__(kReduceRowWarps * 32, 2) decode_reduce_rows(DecodeParams p) {
   constexpr int E = D / 32;
   static_assert(D % 32 == 0 && (E == 1 || E == 2 || E == 4), "head_dim");
   static_assert(NP <= kReduceFast && NP <= 32, "partitions per row");
+  constexpr int R = NP < kReducePre ? NP : kReducePre;
   wait_prior_grid();
   allow_next_grid();
   const int lane = threadIdx.x & 31;
   const int64_t rows = (int64_t)p.B * p.Hq;
   const int64_t stride = (int64_t)gridDim.x * kReduceRowWarps;
+  const bool has_extra = p.row_stride > p.max_parts;  // the workspace has the extra row
   T *out = reinterpret_cast<T *>(p.out);
   for (int64_t bh = (int64_t)blockIdx.x * kReduceRowWarps + (threadIdx.x >> 5); bh < rows; bh += stride) {
-    const int ctx = p.lens[bh / p.Hq];
-    if (ctx <= p.part || ctx > p.max_ctx) continue;  // written directly by the partition kernel
-    const int np = min((ctx + p.part - 1) / p.part, NP);
-    const float mi = lane < np ? __ldcg(p.ws_m + bh * p.max_parts + lane) : -INFINITY;
-    const float li = lane < np ? __ldcg(p.ws_l + bh * p.max_parts + lane) : 0.f;
-    const float *acc = p.ws_acc + bh * p.max_parts * D + lane * E;
-    float av[E][NP];
+    const int b = (int)(bh / p.Hq);
+    const int ctx = p.lens[b];
+    const int ft_raw = p.first_tok ? p.first_tok[b] : 0;
+    const float *mrow = p.ws_m + bh * p.row_stride;
+    const float *lrow = p.ws_l + bh * p.row_stride;
+    const float *acc = p.ws_acc + bh * p.row_stride * D + lane * E;
+    const float mr = lane < p.row_stride ? __ldcg(mrow + lane) : -INFINITY;
+    const float lr = lane < p.row_stride ? __ldcg(lrow + lane) : 0.f;
+    float av[NP][E], ax[E];
 #pragma unroll
-    for (int i = 0; i < NP; ++i) {
-      if (i < np) {
-        const float *src = acc + (size_t)i * D;
-        if constexpr (E == 4) {
-          const float4 v = __ldcg(reinterpret_cast<const float4 *>(src));
-          av[0][i] = v.x; av[1][i] = v.y; av[2][i] = v.z; av[3][i] = v.w;
-        } else if constexpr (E == 2) {
-          const float2 v = __ldcg(reinterpret_cast<const float2 *>(src));
-          av[0][i] = v.x; av[1][i] = v.y;
-        } else {
-          av[0][i] = __ldcg(src);
-        }
-      } else {
-#pragma unroll
-        for (int k = 0; k < E; ++k) av[k][i] = 0.f;
-      }
+    for (int i = 0; i < R; ++i) {
+      if (i < p.max_parts) load_acc_row<E>(acc + (size_t)i * D, av[i]);
     }
+    if (has_extra) load_acc_row<E>(acc + (size_t)p.max_parts * D, ax);
+    const int ft = (ft_raw > 0 && ft_raw < ctx && ft_raw % p.bs == 0) ? ft_raw : 0;  // first_token_of
+    const int np = min(merge_slots(p, ctx, ft), NP);
+    if (np == 0) continue;  // written directly by the partition kernel
+    const int npart = (ctx + p.part - 1) / p.part;
     float mv[NP], lv[NP], f[NP];
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
-      mv[i] = __shfl_sync(0xffffffffu, mi, i);
-      lv[i] = __shfl_sync(0xffffffffu, li, i);
+      const int rw = slot_row(p, npart, i);
+      mv[i] = __shfl_sync(0xffffffffu, mr, rw & 31);
+      lv[i] = __shfl_sync(0xffffffffu, lr, rw & 31);
     }
-    const float L = merge_weights(mv, lv, np, f);
 #pragma unroll
-    for (int k = 0; k < E; ++k) store_out(out + bh * D + lane * E + k, merge_element(av[k], f, np, L));
+    for (int i = R; i < NP; ++i)
+      if (i < np && i < npart) load_acc_row<E>(acc + (size_t)i * D, av[i]);
+    const float L = merge_weights(mv, lv, np, f);
+    float a[E];
+#pragma unroll
+    for (int k = 0; k < E; ++k) a[k] = 0.f;
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      if (i < np) {
+        const bool x = i >= npart;  // the extra row (the last slot)
+#pragma unroll
+        for (int k = 0; k < E; ++k) a[k] = fmaf(x ? ax[k] : av[i][k], f[i], a[k]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < E; ++k) store_out(out + bh * D + lane * E + k, L > 0.f ? a[k] / L : 0.f);
   }
 }
 
-// decode_reduce for calls whose rows have at most kReduceWide partitions:
-// one warp per row as decode_reduce_rows, lane i holding partition i's max
-// and sum; the accumulators are read in rounds of kReduceRound partitions
-// (one load per lane per partition in a round, then the round's fused
-// multiply-adds in partition order).  The merge takes the steps of
+// decode_reduce for calls whose rows have at most kReduceWide merge slots:
+// one warp per row as decode_reduce_rows, lane i holding slot i's max and
+// sum; the accumulators are read in rounds of kReduceRound slots (one load
+// per lane per slot in a round, then the round's fused multiply-adds in
+// slot order).  As in decode_reduce_rows, the maxima and sums are loaded
+// before the row's length is known.  The merge takes the steps of
 // merge_weights and merge_element in their order, so its bits are those of
 // the other merge kernels.
 constexpr int kReduceWide = 32;
@@ -474,18 +543,29 @@ __global__ void __launch_bounds__(kReduceRowWarps * 32, 2) decode_reduce_rows_wi
   const int64_t stride = (int64_t)gridDim.x * kReduceRowWarps;
   T *out = reinterpret_cast<T *>(p.out);
   for (int64_t bh = (int64_t)blockIdx.x * kReduceRowWarps + (threadIdx.x >> 5); bh < rows; bh += stride) {
-    const int ctx = p.lens[bh / p.Hq];
-    if (ctx <= p.part || ctx > p.max_ctx) continue;  // written directly by the partition kernel
-    const int np = min((ctx + p.part - 1) / p.part, kReduceWide);
-    const float mi = lane < np ? __ldcg(p.ws_m + bh * p.max_parts + lane) : -INFINITY;
-    const float li = lane < np ? __ldcg(p.ws_l + bh * p.max_parts + lane) : 0.f;
+    const int b = (int)(bh / p.Hq);
+    // issued before the length is known: every workspace row's max and sum
+    // (the accumulators, which are larger, only for the row's slots)
+    const int ctx = p.lens[b];
+    const int ft_raw = p.first_tok ? p.first_tok[b] : 0;
+    const float mr = lane < p.row_stride ? __ldcg(p.ws_m + bh * p.row_stride + lane) : -INFINITY;
+    const float lr = lane < p.row_stride ? __ldcg(p.ws_l + bh * p.row_stride + lane) : 0.f;
+    const float *acc = p.ws_acc + bh * p.row_stride * D + lane * E;
+    const int ft = (ft_raw > 0 && ft_raw < ctx && ft_raw % p.bs == 0) ? ft_raw : 0;  // first_token_of
+    const int np = min(merge_slots(p, ctx, ft), kReduceWide);
+    if (np == 0) continue;  // written directly by the partition kernel
+    const int npart = (ctx + p.part - 1) / p.part;
+    const int lrow = slot_row(p, npart, lane);
+    const float ms = __shfl_sync(0xffffffffu, mr, lrow & 31);  // every lane takes part
+    const float ls = __shfl_sync(0xffffffffu, lr, lrow & 31);
+    const float mi = lane < np ? ms : -INFINITY;
+    const float li = lane < np ? ls : 0.f;
     float M = mi;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     const float fi = (lane < np && mi != -INFINITY) ? fast_exp2(mi - M) : 0.f;
     float L = 0.f;
     for (int i = 0; i < np; ++i) L = fmaf(__shfl_sync(0xffffffffu, li, i), __shfl_sync(0xffffffffu, fi, i), L);
-    const float *acc = p.ws_acc + bh * p.max_parts * D + lane * E;
     float a[E];
 #pragma unroll
     for (int k = 0; k < E; ++k) a[k] = 0.f;
@@ -493,17 +573,9 @@ __global__ void __launch_bounds__(kReduceRowWarps * 32, 2) decode_reduce_rows_wi
       float av[kReduceRound][E];
 #pragma unroll
       for (int j = 0; j < kReduceRound; ++j) {
-        const float *src = acc + (size_t)(i0 + j) * D;
-        if (i0 + j < np) {
-          if constexpr (E == 4) {
-            const float4 v = __ldcg(reinterpret_cast<const float4 *>(src));
-            av[j][0] = v.x; av[j][1] = v.y; av[j][2] = v.z; av[j][3] = v.w;
-          } else if constexpr (E == 2) {
-            const float2 v = __ldcg(reinterpret_cast<const float2 *>(src));
-            av[j][0] = v.x; av[j][1] = v.y;
-          } else {
-            av[j][0] = __ldcg(src);
-          }
+        const int i = i0 + j;
+        if (i < np) {
+          load_acc_row<E>(acc + (size_t)slot_row(p, npart, i) * D, av[j]);
         } else {
 #pragma unroll
           for (int k = 0; k < E; ++k) av[j][k] = 0.f;

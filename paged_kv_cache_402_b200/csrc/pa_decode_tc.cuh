@@ -83,20 +83,34 @@ struct TcLayout {
   static constexpr int kOffTmem = kOffRedSum + kRedFloats * 4;
   // per-unit description written by the producer next to the unit's Q slot:
   // [b, g, part, t0, t1, nchunks, single, newest-token block or -1,
-  //  copy-on-write source of that block or -1, 0] + the unit's table entries
-  // (as the copies read them)
+  //  copy-on-write source of that block or -1, packed] + the unit's table
+  // entries (as the copies read them)
   static constexpr int kUnitHead = 10;
   static constexpr int kMaxPart = 1024;  // the largest partition built (256, 512 or 1024 tokens)
   static constexpr int kUnitInts = kUnitHead + kMaxPart / 8;
   static constexpr int kOffUnit = kOffTmem + 16;
-  static constexpr int kOffScan = kOffUnit + 2 * kUnitInts * 4;  // 3 x 8 ints
-  static constexpr int kOffPrefix = kOffScan + 96;
+  static constexpr int kOffScan = kOffUnit + 2 * kUnitInts * 4;  // 4 x 8 ints
+  // head-packed passes: each warp's column maxima (by chunk parity) and
+  // weights of the old reference, and the pending unit's maxima (by unit
+  // parity), 16 columns each
+  static constexpr int kOffPack = kOffScan + 128;
+  static constexpr int kOffPrefix = kOffPack + 3 * 2 * kN * 4;
   static constexpr int kOffCtx = kOffPrefix + (kMaxSeqs + 1) * 4;
   static constexpr int kOffFirst = kOffCtx + kMaxSeqs * 4;  // first partition of each sequence
   static constexpr int kBytes = kOffFirst + kMaxSeqs * 4 + 1024;  // + base alignment slack
   static constexpr int kThreads = 192;
   static constexpr uint32_t kTmemCols = 64;  // S0 S1 O0 O1, kN columns each
 };
+static_assert(TcLayout::kBytes <= 227 * 1024, "shared memory of the partition kernel");
+
+// Head packing of short partial partitions (group size <= 4, a multiple of 4
+// kv heads): one pass covers 4 kv heads of a sequence, with 32 rows of the
+// 128-row K and V tiles per head, so that a head's rows are one softmax
+// warp's.  Its query tile holds the 4 G query rows of the 4 heads (adjacent
+// in q), S and O are block diagonal: a score counts only where the row's
+// head is the column's.
+constexpr int kPackHeads = 4;
+constexpr int kPackRows = TcLayout::kChunk / kPackHeads;
 
 // 2^x by the MUFU approximation (flushes denormal results to zero): the
 // weights only feed a bf16 operand and fp32 sums.  Every tensor-core kernel
@@ -174,6 +188,7 @@ struct TcUnit {
   int b, g, part, t0, t1, nchunks;
   int hg;  // kv heads of the unit: g .. g + hg - 1 (1 for a full partition)
   bool single;
+  bool pack;  // passes of kPackHeads heads, kPackRows tokens per head per chunk
 };
 
 // Run-time work counters: [next unit, CTAs finished] per slot.  A call takes
@@ -189,17 +204,19 @@ __device__ __forceinline__ int pf_of(int32_t v) { return v & ((1 << kFullBits) -
 __device__ __forceinline__ int pp_of(int32_t v) { return (int)((uint32_t)v >> kFullBits); }
 
 // Unit u of the largest-first order.  The full partitions (sequence-major,
-// kv head fastest; a sequence's start at its first partition) are one kv
-// head each; the partial last partitions are tail_hg consecutive kv heads of
+// kv head fastest; a sequence's first one is the partition its first token
+// first_s[b] falls in, which then starts at that token) are one kv head each; the partial last partitions are tail_hg consecutive kv heads of
 // one sequence each (Hkv / tail_hg units per sequence).  With one head per
 // tail unit the full partitions come first (units [0, F)), the partial ones
 // after; with several heads a tail unit is about as large as a full one or
 // larger, so the tail units come first (units [0, T)) and the full ones
-// after, and a launch ends on units of one full partition either way.
+// after, and a launch ends on units of one full partition either way.  With
+// pack_ok (tail_hg then a multiple of kPackHeads), a tail unit goes in
+// head-packed passes when they take fewer chunks in all.
 template <int PART>
 __device__ __forceinline__ TcUnit tc_unit_at(const DecodeParams &p, const int32_t *prefix,
                                              const int32_t *ctx_s, const int32_t *first_s, int u,
-                                             int num_full, int num_tail, int tail_hg) {
+                                             int num_full, int num_tail, int tail_hg, bool pack_ok) {
   TcUnit un;
   const bool tails_first = tail_hg > 1;
   const bool full = tails_first ? u >= num_tail : u < num_full;
@@ -216,11 +233,16 @@ __device__ __forceinline__ TcUnit tc_unit_at(const DecodeParams &p, const int32_
   }
   un.b = lo;
   const int ctx = ctx_s[lo];
-  un.part = full ? first_s[lo] + w - pf_of(prefix[lo]) : ctx / PART;
-  un.t0 = un.part * PART;
-  un.t1 = min(un.t0 + PART, ctx);
-  un.nchunks = (un.t1 - un.t0 + TcLayout::kChunk - 1) / TcLayout::kChunk;
-  un.single = ctx <= PART;
+  const int first = first_s[lo];
+  un.part = full ? first / PART + w - pf_of(prefix[lo]) : ctx / PART;
+  un.t0 = max(un.part * PART, first);
+  un.t1 = min((un.part + 1) * PART, ctx);
+  const int len = un.t1 - un.t0;
+  const int nc_plain = (len + TcLayout::kChunk - 1) / TcLayout::kChunk;
+  const int nc_pack = (len + kPackRows - 1) / kPackRows;
+  un.pack = pack_ok && !full && nc_pack < kPackHeads * nc_plain;
+  un.nchunks = un.pack ? nc_pack : nc_plain;
+  un.single = ctx <= PART && first == 0;
   return un;
 }
 
@@ -254,7 +276,8 @@ template <int G, int PART>
 __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     decode_partition_tc(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v,
-                        const __grid_constant__ CUtensorMap tmap_q, DecodeParams p) {
+                        const __grid_constant__ CUtensorMap tmap_q,
+                        const __grid_constant__ CUtensorMap tmap_q4, DecodeParams p) {
   using L = TcLayout;
   constexpr int N = L::kN;
   static_assert(G >= 1 && G <= N, "group size");
@@ -263,6 +286,10 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
 
+  // tmap_q4: q in boxes of kPackHeads * G rows (the query rows of a
+  // head-packed pass), used when G <= 4 and Hkv is a multiple of kPackHeads.
+  constexpr bool kCanPack = G <= 4;
+  const bool pack_ok = kCanPack && p.Hkv % kPackHeads == 0;
   // Up to the first unit's table entries, the kernel reads only the lengths
   // and the block tables, which no kernel of this library writes; it waits
   // for the kernel ahead of it in the stream (and lets the next one be
@@ -281,6 +308,8 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffTmem);
   float *red_max = reinterpret_cast<float *>(smem + L::kOffRed);
   float *red_sum = reinterpret_cast<float *>(smem + L::kOffRedSum);
+  float *pk_alpha = reinterpret_cast<float *>(smem + L::kOffPack);         // [parity][16]
+  float *pk_mdone = pk_alpha + 2 * N;                                       // [parity][16]
   __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(p.out);
 
   // ---------------------------------------------------------------- set-up
@@ -302,7 +331,9 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     mbar_init(drain, 1);
     fence_barrier_init();
   }
-  // Q rows past G and unused P rows stay zero for the whole kernel
+  // Q rows past G and the P tiles start zero (a plain unit only reads
+  // columns 0 .. G - 1 of S and O, so what a head-packed pass leaves in the
+  // other rows of Q and P does not reach its output)
   for (int i = threadIdx.x; i < (2 * L::kQ + 2 * L::kP) / 16; i += blockDim.x)
     reinterpret_cast<uint4 *>(smem + L::kOffQ)[i] = make_uint4(0, 0, 0, 0);
 
@@ -313,7 +344,9 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   const int b_first = threadIdx.x * seg;
   int cnt[kMaxSeg];
   int mine = 0;
-  int tail_chunks = 0, tails = 0;  // chunks of this thread's partial last partitions, and their count
+  // chunks of this thread's partial last partitions (128-token chunks, and
+  // kPackRows-token ones of a packed pass), and their count
+  int tail_chunks = 0, tail_pchunks = 0, tails = 0;
 #pragma unroll
   for (int i = 0; i < kMaxSeg; ++i) {
     cnt[i] = 0;
@@ -321,20 +354,23 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     if (i < seg && b < B) {
       const int ctx = p.lens[b];
       const bool ok = ctx >= 0 && ctx <= p.max_ctx;
+      // tokens the cascade kernel did: a whole number of blocks before the last
+      int ft = p.first_tok ? p.first_tok[b] : 0;
+      if (ft != 0 && (!ok || ft < 0 || ft >= ctx || ft % p.bs != 0)) {
+        if (blockIdx.x == 0) raise_error(PA_DEVERR_PLAN);
+        ft = 0;  // this kernel then does the whole sequence
+      }
       if (ok && ctx % PART != 0) {
-        tail_chunks += (ctx % PART + TcLayout::kChunk - 1) / TcLayout::kChunk;
+        const int tl = ctx - max(ctx / PART * PART, ft);
+        tail_chunks += (tl + TcLayout::kChunk - 1) / TcLayout::kChunk;
+        tail_pchunks += (tl + kPackRows - 1) / kPackRows;
         ++tails;
       }
       ctx_s[b] = ctx;
-      // partitions the cascade kernel did: whole ones before the last
-      int fp = p.first_part ? p.first_part[b] : 0;
-      if (fp != 0 && (!ok || fp < 0 || (int64_t)fp * PART >= ctx)) {
-        if (blockIdx.x == 0) raise_error(PA_DEVERR_PLAN);
-        fp = 0;  // this kernel then does the whole sequence
-      }
-      first_s[b] = fp;
-      // full partitions in the low bits, a partial last partition in the high ones
-      cnt[i] = (ok && ctx > 0) ? (ctx / PART - fp) | ((ctx % PART != 0 ? 1 : 0) << kFullBits) : 0;
+      first_s[b] = ft;
+      // partitions from the one token ft falls in: the ones that end on a
+      // partition boundary in the low bits, a partial last one in the high ones
+      cnt[i] = (ok && ctx > 0) ? (ctx / PART - ft / PART) | ((ctx % PART != 0 ? 1 : 0) << kFullBits) : 0;
       mine += cnt[i];
       if (blockIdx.x == 0 && !ok) raise_error(PA_DEVERR_LEN);
     }
@@ -349,11 +385,13 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) {
     tail_chunks += __shfl_xor_sync(0xffffffffu, tail_chunks, o);
+    tail_pchunks += __shfl_xor_sync(0xffffffffu, tail_pchunks, o);
     tails += __shfl_xor_sync(0xffffffffu, tails, o);
   }
   if (lane == 0) {
     scan[8 + warp] = tail_chunks;
     scan[16 + warp] = tails;
+    scan[24 + warp] = tail_pchunks;
   }
   if (warp == 1) tc::tmem_alloc(tmem_slot, L::kTmemCols);
   __syncthreads();
@@ -383,16 +421,24 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   // decision from the same lengths; a launch keeps at least 4 units per CTA.
   int tail_hg = 1;
   {
-    int tc_sum = 0, tn = 0;
+    int tc_sum = 0, tp_sum = 0, tn = 0;
     for (int w = 0; w < L::kThreads / 32; ++w) {
       tc_sum += scan[8 + w];
       tn += scan[16 + w];
+      tp_sum += scan[24 + w];
     }
     if (tn > 0 && tc_sum > 0) {
-      // kv heads per unit: a full partition's chunks over the mean tail's, rounded
-      int h = min((2 * (PART / L::kChunk) * tn + tc_sum) / (2 * tc_sum), p.Hkv);
-      while (h > 1 && (p.Hkv % h != 0 || num_full + (p.Hkv / h) * tn < 4 * (int)gridDim.x)) --h;
-      tail_hg = max(h, 1);
+      // kv heads per unit: a full partition's chunks over the mean tail's,
+      // rounded; with packing, packed passes of kPackHeads heads over the
+      // mean packed pass's chunks
+      const int step = pack_ok ? kPackHeads : 1;
+      const int per = pack_ok ? tp_sum : tc_sum;
+      int h = step * max((2 * (PART / L::kChunk) * tn + per) / (2 * per), 1);
+      h = min(h, p.Hkv);
+      while (h > step && (p.Hkv % h != 0 || num_full + (p.Hkv / h) * tn < 4 * (int)gridDim.x)) h -= step;
+      tail_hg = h;
+    } else if (pack_ok) {
+      tail_hg = kPackHeads;
     }
   }
   const int num_tail = (p.Hkv / tail_hg) * pp_of(prefix[B]);
@@ -408,11 +454,14 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       tc::prefetch_tensormap(&tmap_k);
       tc::prefetch_tensormap(&tmap_v);
       tc::prefetch_tensormap(&tmap_q);
+      if (pack_ok) tc::prefetch_tensormap(&tmap_q4);
     }
     const uint64_t pol_kv = policy_evict_first();
     const uint64_t pol_q = tc::policy_evict_last();
     const int bs = p.bs;
     const int blocks_per_chunk = L::kChunk / bs;
+    const int blocks_per_pack = kPackRows / bs;  // blocks of one head in a packed chunk
+    const int lg_bs = bs == 8 ? 3 : (bs == 16 ? 4 : 5);
     const int oob_group = p.num_blocks * p.Hkv * (bs / 8);  // first 8-row group past the pool
     int c = 0, qi = 0;
     bool ok = true;
@@ -432,16 +481,16 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       for (int k = 0; k < NE; ++k) x[k] = -1;
       nd = ns = -1;
       if (u < num_units) {
-        nu = tc_unit_at<PART>(p, prefix, ctx_s, first_s, u, num_full, num_tail, tail_hg);
-        const int32_t *tr = p.tables + (size_t)nu.b * p.max_blocks + nu.t0 / bs;
-        const int nb = (nu.t1 - nu.t0 + bs - 1) / bs;
+        nu = tc_unit_at<PART>(p, prefix, ctx_s, first_s, u, num_full, num_tail, tail_hg, pack_ok);
+        const int32_t *tr = p.tables + (size_t)nu.b * p.max_blocks + (nu.t0 >> lg_bs);
+        const int nb = (nu.t1 - nu.t0 + bs - 1) >> lg_bs;
         const bool newest = p.k_new != nullptr && nu.t1 == ctx_s[nu.b];
         const int32_t src = (newest && p.cow_src != nullptr) ? p.cow_src[nu.b] : -1;
 #pragma unroll
         for (int k = 0; k < NE; ++k)
           if (lane + 32 * k < nb) x[k] = tr[lane + 32 * k];
         if (newest) {
-          const int jl = (nu.t1 - 1 - nu.t0) / bs;
+          const int jl = (nu.t1 - 1 - nu.t0) >> lg_bs;
           const int32_t blk = __shfl_sync(0xffffffffu, pick(x, jl >> 5), jl & 31);
           if (blk >= 0 && blk < p.num_blocks) {  // else its copy flags PA_DEVERR_TABLE
             nd = blk;
@@ -463,8 +512,10 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     if (!p.late_wait) wait_prior_grid();  // the copies read the pool and Q, which may be written just before
     allow_next_grid();
     while (ok && u < num_units) {
-      const int nb_unit = (un.t1 - un.t0 + bs - 1) / bs;
-      for (int hh = 0; hh < un.hg; ++hh) {  // one (sequence, kv head, partition) at a time
+      const int nb_unit = (un.t1 - un.t0 + bs - 1) >> lg_bs;
+      const int hstep = un.pack ? kPackHeads : 1;
+      // one (sequence, kv head, partition) at a time, or kPackHeads heads in a packed pass
+      for (int hh = 0; hh < un.hg; hh += hstep) {
         const int g = un.g + hh;
         const int qs = qi & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((qi >> 1) & 1) ^ 1))) { ok = false; break; }
@@ -480,18 +531,19 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
             us[6] = un.single;
             us[7] = nd;
             us[8] = ns;
-            us[9] = 0;
+            us[9] = un.pack;
           }
 #pragma unroll
           for (int k = 0; k < NE; ++k) us[L::kUnitHead + 32 * k + lane] = e[k];
           __syncwarp();
         }
         if (lane == 0) {
-          mbar_arrive_expect_tx(&qfull[qs], 2 * G * 128);
           uint8_t *qdst = smem + L::kOffQ + qs * L::kQ;
           const int qy = un.b * p.Hq + g * G;
-          tc::tma_load_2d(qdst, &tmap_q, 0, qy, &qfull[qs], pol_q);
-          tc::tma_load_2d(qdst + N * 128, &tmap_q, 64, qy, &qfull[qs], pol_q);
+          const CUtensorMap *qmap = un.pack ? &tmap_q4 : &tmap_q;
+          mbar_arrive_expect_tx(&qfull[qs], 2 * (un.pack ? kPackHeads * G : G) * 128);
+          tc::tma_load_2d(qdst, qmap, 0, qy, &qfull[qs], pol_q);
+          tc::tma_load_2d(qdst + N * 128, qmap, 64, qy, &qfull[qs], pol_q);
         }
         ++qi;
         for (int ci = 0; ci < un.nchunks; ++ci, ++c) {
@@ -504,14 +556,18 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
             uint8_t *dst = smem + (which ? L::kOffV : L::kOffK) + slot * L::kTile;
             if (lane == 0) mbar_arrive_expect_tx(full, L::kTile);
             __syncwarp();
-            // lane j loads block j of the chunk; a chunk's entries lie in one
-            // 32-entry group (blocks_per_chunk divides 32)
-            const int jloc = ci * blocks_per_chunk + (lane % blocks_per_chunk);
-            const int32_t blk = __shfl_sync(0xffffffffu, pick(e, (ci * blocks_per_chunk) >> 5), jloc & 31);
+            // lane j loads block j of the chunk (rows j bs ..), or in a packed
+            // pass block j % bpp of head j / bpp (bpp blocks per head); a
+            // chunk's entries lie in one 32-entry group (blocks_per_chunk and
+            // blocks_per_pack divide 32)
+            const int bpc = un.pack ? blocks_per_pack : blocks_per_chunk;
+            const int jloc = ci * bpc + (lane % bpc);
+            const int head = g + (un.pack ? (lane / bpc) % kPackHeads : 0);
+            const int32_t blk = __shfl_sync(0xffffffffu, pick(e, (ci * bpc) >> 5), jloc & 31);
             if (lane < blocks_per_chunk) {
               int w = oob_group;
               if (jloc < nb_unit) {
-                if (blk >= 0 && blk < p.num_blocks) w = (blk * p.Hkv + g) * (bs / 8);
+                if (blk >= 0 && blk < p.num_blocks) w = (blk * p.Hkv + head) * (bs / 8);
                 else if (which == 0 && hh == 0) raise_error(PA_DEVERR_TABLE);
               }
               tc::tma_load_4d(dst + lane * (bs / 8) * L::kGroup, map, 0, 0, 0, w, full, pol_kv);
@@ -574,13 +630,17 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     auto tile_piece = [](int r, int half, int piece) {
       return (r >> 3) * L::kGroup + half * 1024 + (r & 7) * 128 + ((piece ^ (r & 7)) << 4);
     };
+    // A packed pass has one newest token per head: rows patch + j kPackRows
+    // (j < npatch) of the chunk.
+    constexpr int kNP = kCanPack ? kPackHeads : 1;
     struct PvJob {
       int c;       // chunk
       int u;       // unit (its O accumulator is u & 1)
       bool first;  // first chunk of the unit: the PV starts the accumulator
       int patch;   // row of the newest token in this chunk, or -1
-      uint4 vrow;  // lanes 16-31: their 16 bytes of its value row
-      uint4 *pool; // lanes 16-31: where those go in the pool
+      int npatch;  // heads with a newest-token row in it
+      uint4 vrow[kNP];  // lanes 16-31: their 16 bytes of each value row
+      uint4 *pool[kNP]; // lanes 16-31: where those go in the pool
     };
     auto issue_pv = [&](const PvJob &j) -> bool {
       const int c = j.c;
@@ -590,10 +650,15 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       if (j.first && !warp_wait(&ofree[j.u & 1], ((j.u >> 1) & 1) ^ 1)) return false;
       if (j.patch >= 0) {
         if (lane >= 16) {
-          const int off = tile_piece(j.patch, (lane >> 3) & 1, lane & 7);
-          *reinterpret_cast<uint4 *>(smem + L::kOffV + (c % 3) * L::kTile + off) = j.vrow;
+#pragma unroll
+          for (int h = 0; h < kNP; ++h) {
+            if (h < j.npatch) {
+              const int off = tile_piece(j.patch + h * kPackRows, (lane >> 3) & 1, lane & 7);
+              *reinterpret_cast<uint4 *>(smem + L::kOffV + (c % 3) * L::kTile + off) = j.vrow[h];
+              *j.pool[h] = j.vrow[h];
+            }
+          }
           fence_proxy_async_smem();  // before the PV MMA reads the tile
-          *j.pool = j.vrow;
         }
         __syncwarp();
       }
@@ -617,7 +682,9 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       return true;
     };
     int c = 0, qi = 0;
-    PvJob pending{-1, 0, false, -1, make_uint4(0, 0, 0, 0), nullptr};
+    PvJob pending{};
+    pending.c = -1;
+    pending.patch = -1;
     while (ok) {
       const int qs = qi & 1;
       if (!warp_wait(&qfull[qs], (qi >> 1) & 1)) { ok = false; break; }
@@ -627,18 +694,31 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       // fused step: this unit's newest token, its chunk and row there, and
       // the lane's 16 bytes of its key (lanes 0-15) or value (16-31) row
       const int32_t nd = us[7];
+      const bool upack = us[9] != 0;
       int patch_chunk = -1, patch_row = 0;
-      uint4 nrow = make_uint4(0, 0, 0, 0);
-      uint4 *pool_row = nullptr;
+      const int npatch = upack ? kPackHeads : 1;
+      uint4 nrow[kNP];
+      uint4 *pool_row[kNP];
+#pragma unroll
+      for (int h = 0; h < kNP; ++h) {
+        nrow[h] = make_uint4(0, 0, 0, 0);
+        pool_row[h] = nullptr;
+      }
       if (nd >= 0) {
         const int b = us[0], g = us[1], t0 = us[3], t1 = us[4];
-        patch_chunk = (t1 - 1 - t0) / L::kChunk;
-        patch_row = (t1 - 1 - t0) % L::kChunk;
-        const uint4 *src = static_cast<const uint4 *>(lane < 16 ? p.k_new : p.v_new) +
-                           ((size_t)b * p.Hkv + g) * 16 + (lane & 15);
-        nrow = *src;
-        pool_row = static_cast<uint4 *>(const_cast<void *>(lane < 16 ? p.k : p.v)) +
-                   (((size_t)nd * p.Hkv + g) * p.bs + (t1 - 1) % p.bs) * 16 + (lane & 15);
+        const int rows = upack ? kPackRows : L::kChunk;  // tokens of one head in a chunk
+        patch_chunk = (t1 - 1 - t0) / rows;
+        patch_row = (t1 - 1 - t0) % rows;
+#pragma unroll
+        for (int h = 0; h < kNP; ++h) {
+          if (h < npatch) {
+            const uint4 *src = static_cast<const uint4 *>(lane < 16 ? p.k_new : p.v_new) +
+                               ((size_t)b * p.Hkv + g + h) * 16 + (lane & 15);
+            nrow[h] = *src;
+            pool_row[h] = static_cast<uint4 *>(const_cast<void *>(lane < 16 ? p.k : p.v)) +
+                          (((size_t)nd * p.Hkv + g + h) * p.bs + (t1 - 1) % p.bs) * 16 + (lane & 15);
+          }
+        }
       }
       const uint32_t qb = qbase0 + qs * L::kQ;
       for (int ci = 0; ci < nchunks; ++ci, ++c) {
@@ -646,10 +726,15 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         if (!warp_wait(&kfull[slot], (c / 3) & 1)) { ok = false; break; }
         if (ci == patch_chunk) {
           if (lane < 16) {
-            const int off = tile_piece(patch_row, (lane >> 3) & 1, lane & 7);
-            *reinterpret_cast<uint4 *>(smem + L::kOffK + slot * L::kTile + off) = nrow;
+#pragma unroll
+            for (int h = 0; h < kNP; ++h) {
+              if (h < npatch) {
+                const int off = tile_piece(patch_row + h * kPackRows, (lane >> 3) & 1, lane & 7);
+                *reinterpret_cast<uint4 *>(smem + L::kOffK + slot * L::kTile + off) = nrow[h];
+                *pool_row[h] = nrow[h];
+              }
+            }
             fence_proxy_async_smem();  // before the QK MMA reads the tile
-            *pool_row = nrow;
           }
           __syncwarp();
         }
@@ -671,7 +756,16 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         }
         __syncwarp();
         if (pending.c >= 0 && !issue_pv(pending)) { ok = false; break; }
-        pending = PvJob{c, qi, ci == 0, ci == patch_chunk ? patch_row : -1, nrow, pool_row};
+        pending.c = c;
+        pending.u = qi;
+        pending.first = ci == 0;
+        pending.patch = ci == patch_chunk ? patch_row : -1;
+        pending.npatch = npatch;
+#pragma unroll
+        for (int h = 0; h < kNP; ++h) {
+          pending.vrow[h] = nrow[h];
+          pending.pool[h] = pool_row[h];
+        }
       }
       ++qi;
     }
@@ -721,7 +815,62 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
 
     // O of unit pun (complete once the PV of its last chunk is) and the
     // warpgroup-wide sums l -> the output row, or the partition's statistics.
+    // A head-packed pass: each warp's sums and maxima are its own head's
+    // (columns wq G ..), all 4 G columns go out.
+    auto epilogue_packed = [&]() {
+      float o[16];
+      warp_wait(&pvdone[p_clast & 1], (p_clast >> 1) & 1);
+      if (!bad) {
+        tc::fence_after_sync();
+        tc::tmem_ld16(trow + 2 * N + (p_u & 1) * N, o);
+      }
+      tc::fence_before_sync();
+      mbar_arrive(&ofree[p_u & 1]);
+      const int parity = p_u & 1;
+      {
+        float v[G];
+        float md = 0.f;
+#pragma unroll
+        for (int n = 0; n < G; ++n) {
+          v[n] = l_done[n];
+          if (lane == n) md = m_done[n];
+        }
+        const float t = warp_reduce_columns<G, false>(v, lane);
+        if (lane < G) {
+          red_sum[(parity * 4 + wq) * N + lane] = t;
+          pk_mdone[parity * N + wq * G + lane] = md;
+        }
+      }
+      stop = wg_sync_or(bad);
+      if (stop) return;
+      constexpr int NC = kPackHeads * G < 16 ? kPackHeads * G : 16;  // the pass's columns
+      float Ls[NC];
+#pragma unroll
+      for (int n = 0; n < NC; ++n) Ls[n] = red_sum[(parity * 4 + n / G) * N + n % G];
+      const size_t hrow = (size_t)pun.b * p.Hq + pun.g * G;  // query row of head 0 of the pass
+      if (pun.single) {
+        __nv_bfloat16 *dst = out + hrow * 128 + r;
+#pragma unroll
+        for (int n = 0; n < NC; ++n) dst[(size_t)n * 128] = __float2bfloat16_rn(Ls[n] > 0.f ? o[n] / Ls[n] : 0.f);
+      } else {
+        const size_t row0 = hrow * p.row_stride + pun.part, rs = p.row_stride;
+        float *acc = p.ws_acc + row0 * 128 + r;
+#pragma unroll
+        for (int n = 0; n < NC; ++n) acc[n * rs * 128] = o[n];
+        if (r == 0) {
+#pragma unroll
+          for (int n = 0; n < NC; ++n) {
+            p.ws_m[row0 + n * rs] = pk_mdone[parity * N + n];
+            p.ws_l[row0 + n * rs] = Ls[n];
+          }
+        }
+      }
+    };
     auto epilogue = [&]() {
+      if (kCanPack && pun.pack) {
+        epilogue_packed();
+        return;
+      }
       float o[8];
       warp_wait(&pvdone[p_clast & 1], (p_clast >> 1) & 1);
       if (!bad) {
@@ -743,22 +892,27 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       float Ls[G];
       combine_warps<G, false>(red_sum + parity * 4 * N, N, 0.f, Ls);
       const size_t hrow = (size_t)pun.b * p.Hq + pun.g * G;  // query row of head 0 of the group
+      if (pun.single) {
+        __nv_bfloat16 *dst = out + hrow * 128 + r;
 #pragma unroll
-      for (int n = 0; n < G; ++n) {
-        if (pun.single) {
-          out[(hrow + n) * 128 + r] = __float2bfloat16_rn(Ls[n] > 0.f ? o[n] / Ls[n] : 0.f);
-        } else {
-          const size_t row = (hrow + n) * p.max_parts + pun.part;
-          p.ws_acc[row * 128 + r] = o[n];
-          if (r == 0) {
-            p.ws_m[row] = m_done[n];
-            p.ws_l[row] = Ls[n];
+        for (int n = 0; n < G; ++n) dst[(size_t)n * 128] = __float2bfloat16_rn(Ls[n] > 0.f ? o[n] / Ls[n] : 0.f);
+      } else {
+        const size_t row0 = hrow * p.row_stride + pun.part, rs = p.row_stride;
+        float *acc = p.ws_acc + row0 * 128 + r;
+#pragma unroll
+        for (int n = 0; n < G; ++n) acc[n * rs * 128] = o[n];
+        if (r == 0) {
+#pragma unroll
+          for (int n = 0; n < G; ++n) {
+            p.ws_m[row0 + n * rs] = m_done[n];
+            p.ws_l[row0 + n * rs] = Ls[n];
           }
         }
       }
     };
 
     const int log2_bs = bs == 8 ? 3 : (bs == 16 ? 4 : 5);
+    uint32_t p_plain = 0;  // bit i: the last chunk to write P buffer i was a plain one
     int c = 0, qi = 0;
     for (; !stop; ++qi) {
       // the unit, as the producer published it with its Q tile
@@ -775,6 +929,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       un.t1 = us[4];
       un.nchunks = us[5];
       un.single = us[6] != 0;
+      un.pack = kCanPack && us[9] != 0;
       if (un.nchunks == 0) break;  // the producer ran out of work
       const int32_t *ents = us + L::kUnitHead;
       const int tail_end = min(((un.t1 + bs - 1) >> log2_bs) << log2_bs, un.t0 + PART);
@@ -817,6 +972,17 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
             vd[i] = static_cast<const uint4 *>(p.v)[s0 + i];
           }
         }
+        if (un.pack) {  // the pass's other heads
+          for (int h = 1; h < kPackHeads; ++h) {
+            const size_t hs = s0 + (size_t)h * cw_vecs, hd = (size_t)h * cw_vecs;
+            for (int i = r; i < cw_vecs; i += 128) {
+              if ((i >> 4) != cw_skip) {
+                kd[hd + i] = static_cast<const uint4 *>(p.k)[hs + i];
+                vd[hd + i] = static_cast<const uint4 *>(p.v)[hs + i];
+              }
+            }
+          }
+        }
       };
 #pragma unroll
       for (int n = 0; n < G; ++n) {
@@ -828,11 +994,13 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       for (int ci = 0; ci < un.nchunks; ++ci, ++c) {
         float s[8];
         warp_wait(&sfull[c & 1], (c >> 1) & 1);
+        // packed: this warp's rows are head wq's, its columns wq G ..
+        const int col0 = un.pack ? wq * G : 0;
         if (!bad) {
           tc::fence_after_sync();
-          tc::tmem_ld8(trow + (c & 1) * N, s);
+          tc::tmem_ld8(trow + (c & 1) * N + col0, s);
         }
-        const int tok = un.t0 + ci * L::kChunk + r;
+        const int tok = un.pack ? un.t0 + ci * kPackRows + lane : un.t0 + ci * L::kChunk + r;
         const int32_t blk = tok < un.t1 ? ents[(tok - un.t0) >> log2_bs] : -1;
         const bool valid = blk >= 0 && blk < p.num_blocks;
         // Scores are weighed against the running reference m as long as no
@@ -863,7 +1031,8 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
           }
         }
         float mnew[G];
-        if (wg_sync_or(need || bad)) {  // uniform: some row needs a new reference (or gave up)
+        const bool red_path = wg_sync_or(need || bad);
+        if (red_path) {  // uniform: some row needs a new reference (or gave up)
           {  // this warp's max of every head; lane n holds head n % G
             float v[G];
 #pragma unroll
@@ -874,7 +1043,12 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
           stop = wg_sync_or(bad);
           if (stop) break;
           float cm[G];
-          combine_warps<G, true>(red_max + (c & 1) * 4 * N, N, -INFINITY, cm);
+          if (un.pack) {  // the warp's own head
+#pragma unroll
+            for (int n = 0; n < G; ++n) cm[n] = red_max[((c & 1) * 4 + wq) * N + n];
+          } else {
+            combine_warps<G, true>(red_max + (c & 1) * 4 * N, N, -INFINITY, cm);
+          }
 #pragma unroll
           for (int n = 0; n < G; ++n) mnew[n] = fmaxf(m[n], cm[n]);
         } else {
@@ -882,35 +1056,75 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
           for (int n = 0; n < G; ++n) mnew[n] = m[n];
         }
         float alpha[G];
-        bool moved = false;  // uniform: m and mnew are the same in every thread
+        bool moved = false;  // uniform: m and mnew are the same in every thread (packed: in the warp)
 #pragma unroll
         for (int n = 0; n < G; ++n) {
           moved |= mnew[n] != m[n];
           alpha[n] = (mnew[n] == m[n]) ? 1.f : ex2_approx(m[n] - mnew[n]);
+        }
+        if (un.pack && red_path) {
+          // every thread rescales all heads' columns of its O row: publish
+          // this warp's weights, and agree on whether any head moved
+          float a = 1.f;
+#pragma unroll
+          for (int n = 0; n < G; ++n)
+            if (lane == n) a = alpha[n];
+          if (lane < G) pk_alpha[(c & 1) * N + wq * G + lane] = a;
+          moved = wg_sync_or(moved);
         }
         if (moved && ci > 0) {
           // O of this unit holds the chunks before c weighed against the old
           // reference: rescale it once PV(c-1) has landed, before PV(c) adds
           warp_wait(&pvdone[(c - 1) & 1], ((c - 1) >> 1) & 1);
           if (!bad) {
-            float o[8];
             tc::fence_after_sync();
-            tc::tmem_ld8(obuf, o);
+            if (kCanPack && un.pack) {
+              float o[16];
+              tc::tmem_ld16(obuf, o);
 #pragma unroll
-            for (int n = 0; n < G; ++n) o[n] *= alpha[n];
-            tc::tmem_st8(obuf, o);
+              for (int n = 0; n < 16; ++n)
+                if (n < kPackHeads * G) o[n] *= pk_alpha[(c & 1) * N + n];
+              tc::tmem_st16(obuf, o);
+            } else {
+              float o[8];
+              tc::tmem_ld8(obuf, o);
+#pragma unroll
+              for (int n = 0; n < G; ++n) o[n] *= alpha[n];
+              tc::tmem_st8(obuf, o);
+            }
           }
         }
         __nv_bfloat16 *pb = reinterpret_cast<__nv_bfloat16 *>(smem + L::kOffP + (c & 1) * L::kP);
         const int kh = r >> 6, rr = r & 63;
+        // P^T row n (K-major, 128-byte swizzle): token r in half kh
+        auto p_off = [&](int n) {
+          return kh * (N * 64) + (n >> 3) * 512 + (n & 7) * 64 + (((rr >> 3) ^ (n & 7)) << 3) + (rr & 7);
+        };
 #pragma unroll
         for (int n = 0; n < G; ++n) {
           const float pv = valid ? ex2_approx(x[n] - mnew[n]) : 0.f;
           l[n] = fmaf(l[n], alpha[n], pv);
           m[n] = mnew[n];
-          // P^T row n (K-major, 128-byte swizzle): token r in half kh
-          const int off = kh * (N * 64) + (n >> 3) * 512 + (n & 7) * 64 + (((rr >> 3) ^ (n & 7)) << 3) + (rr & 7);
-          pb[off] = __float2bfloat16_rn(pv);
+          pb[p_off(col0 + n)] = __float2bfloat16_rn(pv);
+        }
+        // A packed chunk needs 0 in the other heads' columns of this row.  A
+        // thread's rows are always its warp's head in packed chunks, so those
+        // columns stay 0 from its last packed chunk in this buffer; only a
+        // plain chunk there since (which writes columns 0 .. G - 1 of every
+        // row) makes columns 0 .. G - 1 of the rows of heads 1.. stale.
+        if (kCanPack) {
+          const uint32_t bit = 1u << (c & 1);
+          if (un.pack) {
+            if (p_plain & bit) {
+              if (wq != 0) {
+#pragma unroll
+                for (int n = 0; n < G; ++n) pb[p_off(n)] = __float2bfloat16_rn(0.f);
+              }
+              p_plain &= ~bit;
+            }
+          } else {
+            p_plain |= bit;
+          }
         }
         fence_proxy_async_smem();
         tc::fence_before_sync();

@@ -44,6 +44,21 @@ def test_no_internal_symbols_exported():
     assert ours == set(_declared())
 
 
+def test_header_constants_match_the_binding():
+    """Every numeric #define of the header that the binding mirrors has the
+    same value there."""
+    hdr = open(os.path.join(os.path.dirname(__file__), "..", "include", "pagedattn.h")).read()
+    found = {}
+    for name, val in re.findall(r"^#define (PA_[A-Z_]+) \(?([0-9xu<> ]+)\)?", hdr, re.M):
+        val = val.replace("u", "").strip()
+        found[name] = eval(val, {})
+    mirrored = [n for n in found if hasattr(pa, n)]
+    assert {"PA_PARTITION_TOKENS", "PA_SHARE_MIN_TOKENS", "PA_STATIC_WORKSPACE_BYTES",
+            "PA_DEVERR_PLAN"} <= set(mirrored)
+    for n in mirrored:
+        assert getattr(pa, n) == found[n], n
+
+
 def test_status_strings_and_version():
     assert pa.lib().pa_status_string(pa.PA_OK) == b"ok"
     assert pa.lib().pa_status_string(pa.PA_ERR_OUT_OF_BLOCKS) == b"out of free blocks"
@@ -211,10 +226,11 @@ def test_step_layout():
     L = pa.pa_step_layout_t()
     c = _cache_struct(num_kv_heads=8)
     assert pa.lib().pa_step_layout(32, 32, ctypes.byref(c), 257, 4, ctypes.byref(L)) == pa.PA_OK
-    offs = [L.q, L.k_new, L.v_new, L.tables, L.lens, L.cow_src, L.first_part, L.members, L.parts, L.bytes]
+    offs = [L.q, L.k_new, L.v_new, L.tables, L.lens, L.cow_src, L.first_token, L.members, L.shared_tokens,
+            L.bytes]
     assert offs == sorted(offs) and all(o % 16 == 0 for o in offs)
     assert L.k_new - L.q == 32 * 32 * 128 * 2 and L.v_new - L.k_new == 32 * 8 * 128 * 2
-    assert L.lens - L.tables >= 32 * 257 * 4 and L.parts - L.members >= 16 * 4 * 4
+    assert L.lens - L.tables >= 32 * 257 * 4 and L.shared_tokens - L.members >= 16 * 4 * 4
     assert pa.lib().pa_step_layout(32, 32, ctypes.byref(c), 257, 5, ctypes.byref(L)) == pa.PA_ERR_INVALID_ARG
 
 
@@ -237,27 +253,37 @@ def test_decode_step_refuses_before_the_allocator_moves():
     assert A.seq_len(s) == (600, 38)
 
 
-def test_share_plan_partition_sizes():
-    """The plan's unit of sharing is the pool's partition: two sequences
-    whose first 600 tokens sit in the same blocks (then diverge) share two
-    256-token partitions, one of 512, none of 1024 (a shared partition is
-    whole, agrees across the group, and comes before each member's last)."""
+def test_share_plan_block_granular():
+    """The plan's unit of sharing is the block, whatever the partition size:
+    two sequences whose first 600 tokens sit in the same blocks, the 38th
+    only partly (copied on write when they diverged), share 37 blocks."""
     bs = 16
-    common = np.arange(100, 100 + 600 // bs + 1, dtype=np.int32)  # 38 blocks, the last partly shared
+    common = np.arange(100, 100 + 600 // bs + 1, dtype=np.int32)
     t = np.full((2, 80), -1, np.int32)
     t[0, :38] = common[:38]
     t[1, :38] = common[:38]
     t[0, 37:70] = np.arange(500, 533)
     t[1, 37:70] = np.arange(600, 633)
     lens = np.array([1100, 1090], np.int32)
-    for part, want in ((256, 2), (512, 1), (1024, 0)):
-        plan = pa.share_plan(t, lens, bs, partition_tokens=part)
-        assert (plan.n_groups, plan.parts.tolist()) == ((1, [want]) if want else (0, [])), part
-        assert plan.first_part.tolist() == [want, want]
-    with pytest.raises(pa.PagedAttnError):
-        pa.share_plan(t, lens, bs, partition_tokens=384)
-    ws = pa.pa_decode_workspace_size
-    assert ws(2, 8, 1000, 128, 256) == 2 * ((2 * 8 * 4 * 4 + 15) // 16 * 16) + 2 * 8 * 4 * 128 * 4
+    plan = pa.share_plan(t, lens, bs)
+    assert plan.n_groups == 1 and plan.shared_tokens.tolist() == [37 * bs]
+    assert plan.first_token.tolist() == [37 * bs, 37 * bs]
+    for bad_bs in (12, 64):
+        with pytest.raises(pa.PagedAttnError):
+            pa.share_plan(t, lens, bad_bs)
+
+
+def test_shared_workspace_size():
+    """With a plan, the scratch holds one more row per (sequence, query head)
+    than the plain decode's (the piece of the partition a shared prefix ends
+    in), and is needed even when every sequence fits one partition."""
+    rows = lambda r: 2 * ((r * 4 + 15) // 16 * 16) + r * 128 * 4
+    ws, wss = pa.pa_decode_workspace_size, pa.pa_decode_shared_workspace_size
+    assert ws(2, 8, 1000, 128, 256) == rows(2 * 8 * 4)
+    assert wss(2, 8, 1000, 128, 256) == rows(2 * 8 * 5)
+    assert wss(3, 4, 1000, 128, 512) == rows(3 * 4 * 3)
+    assert ws(3, 4, 500, 128, 512) == 0 and wss(3, 4, 500, 128, 512) == rows(3 * 4 * 2)
+    assert wss(3, 4, 500, 128, 384) == 0 and wss(0, 4, 500, 128, 512) == 0
     assert ws(2, 8, 1000, 128, 1024) == 0 and ws(2, 8, 1000, 128, 384) == 0
     assert ws(2, 8, 1000, 128) == ws(2, 8, 1000, 128, 512)
 
@@ -408,39 +434,43 @@ def test_seqs_max_len():
 
 
 def test_share_plan_groups():
-    """Buckets by the first partition's entries, groups of at most
-    max_members in sequence order, a lone leftover in no group, and the shared
-    partitions stop where the tables part or a member's last partition
-    starts."""
+    """Buckets by the first block, groups of at most max_members in sequence
+    order, a lone leftover in no group; the shared blocks stop where the
+    tables part or before a member's last block, and a group that would
+    share fewer than PA_SHARE_MIN_TOKENS tokens is dropped."""
     t = np.full((7, 96), -1, np.int32)
     for i in (0, 1, 2):                       # share 40 blocks, then private
         t[i, :40] = np.arange(40)
         t[i, 40:50] = 100 + 10 * i + np.arange(10)
     t[3, :60] = 200 + np.arange(60)           # alone
-    t[4, :40] = np.arange(40)                 # joins 0..2 (same first partition)
+    t[4, :40] = np.arange(40)                 # joins 0..2 (same first block)
     t[4, 40:45] = 500 + np.arange(5)
-    for i in (5, 6):                          # share two whole partitions
+    for i in (5, 6):                          # share 70 blocks
         t[i, :70] = 1000 + np.arange(70)
         t[i, 70:80] = 2000 + 10 * i + np.arange(10)
     lens = np.array([50 * 16, 49 * 16 + 3, 45 * 16, 60 * 16, 1024, 80 * 16, 75 * 16], np.int32)
     pl = pa.share_plan(t, lens, 16)
     assert pl.members.tolist() == [[0, 1, 2, 4], [5, 6, -1, -1]]
-    assert pl.parts.tolist() == [1, 2]
-    assert pl.first_part.tolist() == [1, 1, 1, 0, 1, 2, 2]
+    assert pl.shared_tokens.tolist() == [640, 1120]
+    assert pl.first_token.tolist() == [640, 640, 640, 0, 640, 1120, 1120]
     pl3 = pa.share_plan(t, lens, 16, max_members=3)       # 0, 1, 2 | 4 alone
     assert pl3.members.tolist() == [[0, 1, 2], [5, 6, -1]]
-    assert pl3.first_part.tolist() == [1, 1, 1, 0, 0, 2, 2]
+    assert pl3.first_token.tolist() == [640, 640, 640, 0, 0, 1120, 1120]
     short = lens.copy()
-    short[6] = 1024                           # partition 1 is now 6's last: one shared partition
-    assert pa.share_plan(t, short, 16).parts.tolist() == [1, 1]
-    short[6] = 512                            # a single partition: in no group
+    short[6] = 1024                           # 64 blocks: 63 before 6's last
+    assert pa.share_plan(t, short, 16).shared_tokens.tolist() == [640, 1008]
+    short[6] = 8 * 16                         # 7 blocks before the last: under the minimum
     pl = pa.share_plan(t, short, 16)
-    assert pl.members.tolist() == [[0, 1, 2, 4]] and pl.first_part[5] == 0 and pl.first_part[6] == 0
+    assert pl.members.tolist() == [[0, 1, 2, 4]] and pl.first_token[5] == 0 and pl.first_token[6] == 0
+    short[6] = 9 * 16                         # 8 blocks: exactly the minimum
+    assert pa.share_plan(t, short, 16).shared_tokens.tolist() == [640, 128]
+    short[6] = 16                             # one block: nothing before its last
+    assert pa.share_plan(t, short, 16).n_groups == 1
 
 
 def test_share_plan_of_allocator_forks():
-    """Forks of a 1300-token prompt share its first two partitions (the third
-    holds the fork point's partial block, copied on write)."""
+    """Forks of a 1300-token prompt share its 81 full blocks (the 82nd, the
+    fork point's partial block, is copied on write by all but one)."""
     A = pa.Allocator(256, 16, list(range(256)))
     r = A.new_seq()
     A.batch_append([r], [1300])
@@ -449,7 +479,7 @@ def test_share_plan_of_allocator_forks():
     tables, lens = A.build_block_tables(seqs, 90)
     pl = pa.share_plan(tables, lens, 16)
     assert pl.members.tolist() == [seqs[:4], seqs[4:] + [-1, -1]]
-    assert pl.parts.tolist() == [2, 2] and pl.first_part.tolist() == [2] * 6
+    assert pl.shared_tokens.tolist() == [1296, 1296] and pl.first_token.tolist() == [1296] * 6
 
 
 def test_decode_shared_argument_checks():
@@ -459,10 +489,18 @@ def test_decode_shared_argument_checks():
     args = lambda **o: [None, None, None, 16, ctypes.byref(c), 16, o.get("mb", 64), 16, 1, 2, o.get("ml", 1000),
                         1.0, ctypes.byref(o.get("plan", plan)), 16, 16, 1 << 20, None]
     assert L.pa_decode_shared(*args()) == pa.PA_ERR_INVALID_ARG                 # 5 members > 4
-    ok_plan = pa.pa_share_plan_t(16, 16, 16, 1, 4)
-    assert L.pa_decode_shared(*args(plan=ok_plan, ml=500, mb=32)) == pa.PA_ERR_INVALID_ARG  # one partition
     bad = pa.pa_share_plan_t(0, 16, 16, 1, 4)
     assert L.pa_decode_shared(*args(plan=bad)) == pa.PA_ERR_INVALID_ARG         # no member array
+    bad = pa.pa_share_plan_t(16, 0, 16, 1, 4)
+    assert L.pa_decode_shared(*args(plan=bad)) == pa.PA_ERR_INVALID_ARG         # no shared tokens
+    # with groups the scratch has the extra row: the plain decode's size is
+    # too small, even for one partition (500 tokens)
+    ok_plan = pa.pa_share_plan_t(16, 16, 16, 1, 4)
+    for ml, mb in ((1000, 64), (500, 32)):
+        plain = max(16, pa.pa_decode_workspace_size(1, 2, ml, 128))
+        a = args(plan=ok_plan, ml=ml, mb=mb)
+        a[15] = plain
+        assert L.pa_decode_shared(*a) == pa.PA_ERR_TOO_SMALL
 
 
 def test_decode_step_prepare_equals_the_separate_calls():
@@ -488,12 +526,13 @@ def test_decode_step_prepare_equals_the_separate_calls():
             nb = -(-int(L) // 16)
             assert np.array_equal(got["tables"][i, :nb], tables[i, :nb])
         assert np.array_equal(got["cow_src"], cow) and got["n_copies"] == len(pairs)
-        assert np.array_equal(got["members"], plan.members) and np.array_equal(got["parts"], plan.parts)
-        assert np.array_equal(got["first_part"], plan.first_part) and got["n_groups"] == plan.n_groups
+        assert np.array_equal(got["members"], plan.members)
+        assert np.array_equal(got["shared_tokens"], plan.shared_tokens)
+        assert np.array_equal(got["first_token"], plan.first_token) and got["n_groups"] == plan.n_groups
         assert got["max_len"] == int(lens.max())
     assert A1.stats() == A2.stats()
     nogroups = A1.decode_step(seqs, 80, share_max_members=0)
-    assert nogroups["n_groups"] == 0 and not nogroups["first_part"].any()
+    assert nogroups["n_groups"] == 0 and not nogroups["first_token"].any()
     with pytest.raises(pa.PagedAttnError):
         A1.decode_step(seqs, 40)  # 1030 tokens do not fit 40 blocks: nothing changes
     before = A1.stats()

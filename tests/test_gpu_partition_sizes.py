@@ -84,14 +84,17 @@ def test_partials_partition_size(cuda_device, part, dtype):
 
 
 @pytest.mark.parametrize("part", PARTS)
-def test_shared_fused_step_partition_size(cuda_device, part):
+@pytest.mark.parametrize("off", [0, 37])
+def test_shared_fused_step_partition_size(cuda_device, part, off):
     """Groups of 8 forks share a prompt of several partitions; one fused step
-    (copies on write, appends, the cascade over the plan's shared partitions
-    of this size) against the oracle, the pool bit for bit, and the output
-    bit-identical to the same step without the plan."""
+    (copies on write, appends, the cascade over the plan's shared blocks cut
+    at partitions of this size) against the oracle, the pool bit for bit.
+    With off = 0 the shared blocks end on a partition boundary and the
+    output is bit-identical to the same step without the plan; with off = 37
+    they end 32 tokens into a partition, which then comes in two pieces."""
     dt, Hkv, D, bs, G = torch.bfloat16, 2, 128, 16, 4
     Hq = G * Hkv
-    prompts = [2 * part + 5, 3 * part + 9, part + 3]
+    prompts = [2 * part + 5 + off, 3 * part + 9 + off, part + 3 + off]
     NB = 3 * 8 * (-(-(max(prompts) + 64) // bs)) + 64
     order = synth.rng(91).permutation(NB)
     outs = []
@@ -108,12 +111,13 @@ def test_shared_fused_step_partition_size(cuda_device, part):
         mb = max(len(M.block_table(s)) for s in seqs)
         tables, lens = A.build_block_tables(seqs, mb)
         cow = pa.cow_sources(pairs, tables, lens, bs)
-        plan = pa.share_plan(tables, lens, bs, partition_tokens=part).to(cuda_device) if use_plan else None
+        plan = pa.share_plan(tables, lens, bs).to(cuda_device) if use_plan else None
         if use_plan:
-            # two plan groups of 4 forks per prompt, sharing the prompt's whole
-            # partitions before its partly filled (copied) last block: 2, 3, 1
+            # two plan groups of 4 forks per prompt, sharing the prompt's full
+            # blocks before its partly filled (copied) last block
             assert plan.n_groups == 6
-            assert sorted(set(plan.parts.tolist())) == [1, 2, 3]
+            sh = 32 if off else 0
+            assert sorted(set(plan.shared_tokens.tolist())) == [part + sh, 2 * part + sh, 3 * part + sh]
         kn = synth.normal((n, Hkv, D), dt, 93)
         vn = synth.normal((n, Hkv, D), dt, 94)
         q = synth.normal((n, Hq, D), dt, 95)
@@ -128,7 +132,8 @@ def test_shared_fused_step_partition_size(cuda_device, part):
         ref = oracle.decode(q, hk, hv, tables, lens, 1 / math.sqrt(D))
         assert_attn_close(out, ref, dt)
         outs.append(out)
-    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    if off == 0:
+        assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
 
 
 @pytest.mark.parametrize("part", [256])

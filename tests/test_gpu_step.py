@@ -7,8 +7,8 @@ per sequence; the oracle copies on write, appends and decodes on its host
 pool.  The output the step copies back to pinned host memory must be within
 the bf16 bound |gpu - ref| <= 2e-2 + 1e-2 |ref| (fp32: max-abs 1e-5), the
 pool bit for bit at the end.  The batch shares prompt blocks (forks of a
-root whose prompt ends inside a block, so the first step copies on write)
-and whole 512-token partitions (so the sharing plan has groups).
+root whose prompt ends inside a block, so the first step copies on write),
+so the sharing plan has groups over the prompts' full blocks.
 """
 import math
 

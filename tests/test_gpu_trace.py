@@ -93,7 +93,7 @@ def test_trace_measured_step(cuda_device, bs):
     the running beams, their copy-on-write sources (pa_cow_sources) and
     their decode tokens' rows.  Beams of one request share the prompt's
     blocks and are copied when they write ("pagedattention" glossary entry,
-    paragraph 5); prompts long enough for whole shared partitions make the
+    paragraph 5); beams whose prompts hold enough full blocks make the
     plan's groups.  Every decode row of every step is checked against the
     oracle, the pools bit for bit every 4 steps and at the end."""
     dev = cuda_device
