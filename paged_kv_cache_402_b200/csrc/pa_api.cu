@@ -266,6 +266,21 @@ bool make_map_q3d(CUtensorMap *m, const void *base, uint64_t total, uint32_t Hq,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// q [rows][128] bf16 seen as 3-D (64 columns, rows, 2 column halves) so that
+// one box of (64, box_rows, 2) lands as [half][box_rows rows x 128 B] with
+// 128-byte swizzle: a query tile's two column halves in one copy.
+bool make_map_q_halves(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {64, rows, 2};
+  const cuuint64_t strides[2] = {128 * 2, 64 * 2};
+  const cuuint32_t box[3] = {64, box_rows, 2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool tc_eligible(const pa::DecodeParams &p, int dtype, int D) {
   if (dtype != PA_DTYPE_BF16 || D != 128) return false;
   if (p.G < 1 || p.G > 8 || (p.G & (p.G - 1))) return false;
@@ -276,15 +291,12 @@ bool tc_eligible(const pa::DecodeParams &p, int dtype, int D) {
 
 template <int G, int PART>
 pa_status launch_decode_tc_slice(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
-  CUtensorMap mk, mv, mq, mq4;
+  CUtensorMap mk, mv, mq;
   const uint64_t rows = (uint64_t)p.num_blocks * p.Hkv * p.bs;
-  // the query rows of a head-packed pass (pa::kPackHeads kv heads), when the
-  // group size allows packing
-  const uint32_t pack_rows = G <= 4 ? (uint32_t)(pa::kPackHeads * G) : (uint32_t)G;
+  // a query tile: the kN rows from a group's first query row, both halves
   if (!make_map_pool_4d(&mk, p.k, rows, (uint32_t)p.bs) ||
       !make_map_pool_4d(&mv, p.v, rows, (uint32_t)p.bs) ||
-      !make_map_bf16_d128(&mq, p.q, (uint64_t)p.B * p.Hq, (uint32_t)G) ||
-      !make_map_bf16_d128(&mq4, p.q, (uint64_t)p.B * p.Hq, pack_rows))
+      !make_map_q_halves(&mq, p.q, (uint64_t)p.B * p.Hq, (uint32_t)pa::TcLayout::kN))
     return PA_ERR_CUDA;
   auto kern = pa::decode_partition_tc<G, PART>;
   const int smem = pa::TcLayout::kBytes;
@@ -294,7 +306,7 @@ pa_status launch_decode_tc_slice(const pa::DecodeParams &p, int32_t max_parts, c
   int grid = sm_count();
   if (grid <= 0) return PA_ERR_CUDA;
   if (units_bound < grid) grid = (int)units_bound;
-  return launch(kern, dim3(grid), dim3(pa::TcLayout::kThreads), (size_t)smem, st, mk, mv, mq, mq4, p);
+  return launch(kern, dim3(grid), dim3(pa::TcLayout::kThreads), (size_t)smem, st, mk, mv, mq, p);
 }
 
 // Sequences are independent: a batch larger than the kernel's per-CTA

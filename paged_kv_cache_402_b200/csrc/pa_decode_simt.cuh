@@ -438,16 +438,17 @@ __global__ void __launch_bounds__(128) decode_reduce(DecodeParams p) {
 
 // decode_reduce for calls whose rows have at most NP <= kReduceFast merge
 // slots: one warp per (sequence, query head) row, lane j holding the
-// head-dim elements [j * D / 32, (j + 1) * D / 32).  A row's loads do not
-// wait for its length: lane i < row_stride loads workspace row i's max and
-// sum, and every lane its elements of rows 0 .. kReducePre - 1 and of the
-// extra row, all at once with the length and first token; the row's slot
-// count then picks among them (rows past it are read but not used), and
-// the slots past the preloaded rows are loaded after it, all before the
-// first multiply-add.  Rows are taken in a grid-stride loop.  Same merge
-// arithmetic, in the same slot order, as decode_reduce.
+// head-dim elements [j * D / 32, (j + 1) * D / 32), lane i slot i's max and
+// sum.  A row's loads do not wait for its length: every workspace row's max
+// and sum, and the elements of rows 0 .. kReducePre - 1 and of the extra
+// row, are loaded at once with the length and first token; the row's slot
+// count then picks among them (rows past it are read but not used), and the
+// slots past the preloaded rows are read in rounds of kReducePre.  Few
+// registers per thread, so that many rows are in flight per SM.  Rows are
+// taken in a grid-stride loop.  Same merge arithmetic, in the same slot
+// order, as decode_reduce.
 constexpr int kReduceRowWarps = 8;
-constexpr int kReducePre = 4;
+constexpr int kReducePre = 2;
 
 template <int E>
 __device__ __forceinline__ void load_acc_row(const float *src, float (&v)[E]) {
@@ -463,11 +464,11 @@ __device__ __forceinline__ void load_acc_row(const float *src, float (&v)[E]) {
 }
 
 template <typename T, int D, int NP>
-__global__ void __launch_bounds__(kReduceRowWarps * 32, 2) decode_reduce_rows(DecodeParams p) {
+__global__ void __launch_bounds__(kReduceRowWarps * 32, 3) decode_reduce_rows(DecodeParams p) {
   constexpr int E = D / 32;
+  constexpr int R = kReducePre;
   static_assert(D % 32 == 0 && (E == 1 || E == 2 || E == 4), "head_dim");
   static_assert(NP <= kReduceFast && NP <= 32, "partitions per row");
-  constexpr int R = NP < kReducePre ? NP : kReducePre;
   wait_prior_grid();
   allow_next_grid();
   const int lane = threadIdx.x & 31;
@@ -479,41 +480,50 @@ __global__ void __launch_bounds__(kReduceRowWarps * 32, 2) decode_reduce_rows(De
     const int b = (int)(bh / p.Hq);
     const int ctx = p.lens[b];
     const int ft_raw = p.first_tok ? p.first_tok[b] : 0;
-    const float *mrow = p.ws_m + bh * p.row_stride;
-    const float *lrow = p.ws_l + bh * p.row_stride;
+    const float mr = lane < p.row_stride ? __ldcg(p.ws_m + bh * p.row_stride + lane) : -INFINITY;
+    const float lr = lane < p.row_stride ? __ldcg(p.ws_l + bh * p.row_stride + lane) : 0.f;
     const float *acc = p.ws_acc + bh * p.row_stride * D + lane * E;
-    const float mr = lane < p.row_stride ? __ldcg(mrow + lane) : -INFINITY;
-    const float lr = lane < p.row_stride ? __ldcg(lrow + lane) : 0.f;
-    float av[NP][E], ax[E];
+    float a0[R][E], ax[E];
 #pragma unroll
-    for (int i = 0; i < R; ++i) {
-      if (i < p.max_parts) load_acc_row<E>(acc + (size_t)i * D, av[i]);
-    }
+    for (int i = 0; i < R; ++i)
+      if (i < p.max_parts) load_acc_row<E>(acc + (size_t)i * D, a0[i]);
     if (has_extra) load_acc_row<E>(acc + (size_t)p.max_parts * D, ax);
     const int ft = (ft_raw > 0 && ft_raw < ctx && ft_raw % p.bs == 0) ? ft_raw : 0;  // first_token_of
     const int np = min(merge_slots(p, ctx, ft), NP);
     if (np == 0) continue;  // written directly by the partition kernel
     const int npart = (ctx + p.part - 1) / p.part;
-    float mv[NP], lv[NP], f[NP];
+    // lane i: slot i's max and sum (every lane takes part in the shuffles)
+    const int lrow = slot_row(p, npart, lane);
+    const float ms = __shfl_sync(0xffffffffu, mr, lrow & 31);
+    const float ls = __shfl_sync(0xffffffffu, lr, lrow & 31);
+    const float mi = lane < np ? ms : -INFINITY;
+    float M = mi;
 #pragma unroll
-    for (int i = 0; i < NP; ++i) {
-      const int rw = slot_row(p, npart, i);
-      mv[i] = __shfl_sync(0xffffffffu, mr, rw & 31);
-      lv[i] = __shfl_sync(0xffffffffu, lr, rw & 31);
-    }
-#pragma unroll
-    for (int i = R; i < NP; ++i)
-      if (i < np && i < npart) load_acc_row<E>(acc + (size_t)i * D, av[i]);
-    const float L = merge_weights(mv, lv, np, f);
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float fi = (lane < np && mi != -INFINITY) ? fast_exp2(mi - M) : 0.f;
+    float L = 0.f;
+    for (int i = 0; i < np; ++i) L = fmaf(__shfl_sync(0xffffffffu, ls, i), __shfl_sync(0xffffffffu, fi, i), L);
     float a[E];
 #pragma unroll
     for (int k = 0; k < E; ++k) a[k] = 0.f;
+    for (int i0 = 0; i0 < np; i0 += R) {
+      float av[R][E];
 #pragma unroll
-    for (int i = 0; i < NP; ++i) {
-      if (i < np) {
-        const bool x = i >= npart;  // the extra row (the last slot)
+      for (int j = 0; j < R; ++j) {
+        const int i = i0 + j;
+        if (i < np && i < npart && i >= R) load_acc_row<E>(acc + (size_t)i * D, av[j]);
+      }
 #pragma unroll
-        for (int k = 0; k < E; ++k) a[k] = fmaf(x ? ax[k] : av[i][k], f[i], a[k]);
+      for (int j = 0; j < R; ++j) {
+        const int i = i0 + j;
+        const float f = __shfl_sync(0xffffffffu, fi, i & 31);
+        if (i < np) {
+#pragma unroll
+          for (int k = 0; k < E; ++k) {
+            const float v = i >= npart ? ax[k] : (i < R ? a0[j][k] : av[j][k]);
+            a[k] = fmaf(v, f, a[k]);
+          }
+        }
       }
     }
 #pragma unroll

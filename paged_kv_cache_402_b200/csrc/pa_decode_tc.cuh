@@ -29,8 +29,9 @@
 //  * Warp 1 (one lane) issues tcgen05 MMAs: per chunk c,
 //        S^T[128 tok x 16] = K_c[128 tok x 128 d] . Q^T[128 d x 16]   (K-major A and B)
 //        O^T[128 d x 16]   = V_c^T[128 d x 128 tok] . P^T[128 tok x 16] (MN-major A)
-//    with accumulators in tensor memory; the query rows past G are zero
-//    (N = 16 is the smallest N an M = 128 MMA takes).  S is double-buffered
+//    with accumulators in tensor memory; the Q tile is the 16 query rows
+//    from the group's first, one 3-D box (N = 16 is the smallest N an
+//    M = 128 MMA takes; columns past G are not read).  S is double-buffered
 //    by chunk; O is one accumulator per unit that every PV of the unit adds
 //    to, double-buffered by unit so a unit's output is read while the next
 //    one runs.  QK of chunk c is issued before PV of chunk c-1.
@@ -62,7 +63,7 @@
 namespace pa {
 
 struct TcLayout {
-  static constexpr int kN = 16;             // MMA N: query heads of a group, zero-padded
+  static constexpr int kN = 16;             // MMA N: the group's query heads, then the next rows
                                             // (M = 128 takes N in multiples of 16)
   static constexpr int kChunk = 128;        // tokens per MMA chunk (= M)
   static constexpr int kStages = 3;
@@ -276,8 +277,7 @@ template <int G, int PART>
 __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     decode_partition_tc(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v,
-                        const __grid_constant__ CUtensorMap tmap_q,
-                        const __grid_constant__ CUtensorMap tmap_q4, DecodeParams p) {
+                        const __grid_constant__ CUtensorMap tmap_q, DecodeParams p) {
   using L = TcLayout;
   constexpr int N = L::kN;
   static_assert(G >= 1 && G <= N, "group size");
@@ -286,8 +286,10 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
 
-  // tmap_q4: q in boxes of kPackHeads * G rows (the query rows of a
-  // head-packed pass), used when G <= 4 and Hkv is a multiple of kPackHeads.
+  // tmap_q: q in boxes of kN rows and both column halves.  A unit's tile
+  // takes the kN query rows from its group's first one: the group's G (or a
+  // head-packed pass's kPackHeads * G), then the next heads' (or the zero
+  // fill past the end), whose S and O columns nothing reads.
   constexpr bool kCanPack = G <= 4;
   const bool pack_ok = kCanPack && p.Hkv % kPackHeads == 0;
   // Up to the first unit's table entries, the kernel reads only the lengths
@@ -331,9 +333,9 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     mbar_init(drain, 1);
     fence_barrier_init();
   }
-  // Q rows past G and the P tiles start zero (a plain unit only reads
-  // columns 0 .. G - 1 of S and O, so what a head-packed pass leaves in the
-  // other rows of Q and P does not reach its output)
+  // The P tiles start zero (a plain unit only reads columns 0 .. G - 1 of S
+  // and O, so what its Q tile holds past row G, and what a head-packed pass
+  // leaves in the other rows of P, does not reach its output)
   for (int i = threadIdx.x; i < (2 * L::kQ + 2 * L::kP) / 16; i += blockDim.x)
     reinterpret_cast<uint4 *>(smem + L::kOffQ)[i] = make_uint4(0, 0, 0, 0);
 
@@ -454,7 +456,6 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       tc::prefetch_tensormap(&tmap_k);
       tc::prefetch_tensormap(&tmap_v);
       tc::prefetch_tensormap(&tmap_q);
-      if (pack_ok) tc::prefetch_tensormap(&tmap_q4);
     }
     const uint64_t pol_kv = policy_evict_first();
     const uint64_t pol_q = tc::policy_evict_last();
@@ -540,10 +541,8 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         if (lane == 0) {
           uint8_t *qdst = smem + L::kOffQ + qs * L::kQ;
           const int qy = un.b * p.Hq + g * G;
-          const CUtensorMap *qmap = un.pack ? &tmap_q4 : &tmap_q;
-          mbar_arrive_expect_tx(&qfull[qs], 2 * (un.pack ? kPackHeads * G : G) * 128);
-          tc::tma_load_2d(qdst, qmap, 0, qy, &qfull[qs], pol_q);
-          tc::tma_load_2d(qdst + N * 128, qmap, 64, qy, &qfull[qs], pol_q);
+          mbar_arrive_expect_tx(&qfull[qs], L::kQ);
+          tc::tma_load_3d(qdst, &tmap_q, 0, qy, 0, &qfull[qs], pol_q);
         }
         ++qi;
         for (int ci = 0; ci < un.nchunks; ++ci, ++c) {
