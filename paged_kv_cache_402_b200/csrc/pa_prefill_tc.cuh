@@ -229,27 +229,36 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
         tc::tma_load_3d(qdst + L::kHalf, &tmap_q, 64, g * G, q0 + tok0, &qfull[qs], pol_q);
       }
       ++qi;
+      // chunk cc's K (which 0) or V (which 1) tiles, table entry e of this lane
+      auto issue = [&](int cc, int ci_, int which, int32_t e) -> bool {
+        const int slot = cc % L::kStages, use = cc / L::kStages;
+        uint64_t *empty = which ? &vempty[slot] : &kempty[slot];
+        uint64_t *full = which ? &vfull[slot] : &kfull[slot];
+        const CUtensorMap *map = which ? &tmap_v : &tmap_k;
+        if (!__all_sync(0xffffffffu, mbar_wait(empty, (use & 1) ^ 1))) return false;
+        uint8_t *dst = smem + (which ? L::kOffV : L::kOffK) + slot * L::kTile;
+        if (lane == 0) mbar_arrive_expect_tx(full, L::kTile);
+        __syncwarp();
+        if (lane < bpc) {
+          int wq = oob_group;  // keys past the sequence: zeros (masked anyway)
+          if (e >= 0 && e < p.num_blocks) wq = (e * p.Hkv + g) * (bs / 8);
+          else if (which == 0 && (ci_ * bpc + lane) * bs < ctx) raise_error(PA_DEVERR_TABLE);
+          tc::tma_load_4d(dst + lane * (bs / 8) * L::kGroup, map, 0, 0, 0, wq, full, pol_kv);
+        }
+        return true;
+      };
+      // K runs one chunk ahead of V: a K slot frees when its QK is done, a V
+      // slot only when its PV is, after the chunk's softmax; so the next
+      // chunk's K does not wait behind a V slot.
+      int32_t e_prev = -1;
       for (int ci = 0; ci < nchunks; ++ci, ++c) {
         const int32_t e = e_next;
-        const int slot = c % L::kStages, use = c / L::kStages;
-        for (int which = 0; which < 2; ++which) {
-          uint64_t *empty = which ? &vempty[slot] : &kempty[slot];
-          uint64_t *full = which ? &vfull[slot] : &kfull[slot];
-          const CUtensorMap *map = which ? &tmap_v : &tmap_k;
-          if (!__all_sync(0xffffffffu, mbar_wait(empty, (use & 1) ^ 1))) { ok = false; break; }
-          uint8_t *dst = smem + (which ? L::kOffV : L::kOffK) + slot * L::kTile;
-          if (lane == 0) mbar_arrive_expect_tx(full, L::kTile);
-          __syncwarp();
-          if (lane < bpc) {
-            int wq = oob_group;  // keys past the sequence: zeros (masked anyway)
-            if (e >= 0 && e < p.num_blocks) wq = (e * p.Hkv + g) * (bs / 8);
-            else if (which == 0 && (ci * bpc + lane) * bs < ctx) raise_error(PA_DEVERR_TABLE);
-            tc::tma_load_4d(dst + lane * (bs / 8) * L::kGroup, map, 0, 0, 0, wq, full, pol_kv);
-          }
-        }
-        if (!ok) break;
+        if (!issue(c, ci, 0, e)) { ok = false; break; }
+        if (ci > 0 && !issue(c - 1, ci - 1, 1, e_prev)) { ok = false; break; }
+        e_prev = e;
         if (ci + 1 < nchunks) e_next = entry(ci + 1);
       }
+      if (ok && !issue(c - 1, nchunks - 1, 1, e_prev)) ok = false;
       if (!ok) break;
       int raw = 0;
       if (lane == 0) raw = (int)gridDim.x + (int)atomicAdd(sched, 1u);
@@ -463,15 +472,25 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
         const int nvis = max(0, min(64, nrow - 64 * half));
         // One pass against the current reference: the weights stay in
         // registers until the pair knows that every row of its quadrant stays
-        // within 2^8 of its reference; otherwise (a row's first chunk, or a
-        // score past the bound in either half) the chunk takes two passes:
+        // within 2^8 of its reference; otherwise (a score past the bound in
+        // either half) the chunk takes two passes:
         // the row max over both halves, a rescale of the rows' O, then the
         // weights.  Either way the weights are 2^(s - m) against the row's
         // reference m, the same in both halves.
         float s[32];
         uint32_t w[32];
         float lsum = 0.f;
-        bool over = m == -INFINITY && nrow > 0;
+        if (ci == 0 && !bad) {
+          // A unit's first chunk: the row's reference starts at its score of
+          // key 0 (visible to every row of the tile; both halves read the same
+          // column, so they start from the same reference).  Scores within 2^8
+          // of it keep the one pass; a larger one takes the two passes.  The
+          // TMEM load is warp-wide (every lane takes part, live row or not).
+          float s8[8];
+          tc::tmem_ld8(trow + (c & 1) * 128, s8);
+          if (row_live) m = s8[0] * p.scale_log2;
+        }
+        bool over = false;
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           if (!bad) tc::tmem_ld32(srow + 32 * k, s);
