@@ -491,18 +491,39 @@ __global__ void __launch_bounds__(PfLayout::kThreads, 1)
           if (row_live) m = s8[0] * p.scale_log2;
         }
         bool over = false;
+        if (__all_sync(0xffffffffu, nvis == 64)) {
+          // every row of the warp sees all of this half's keys (the chunks
+          // before the diagonal): no masks, and one max instead of a test
+          // per score
+          float xmax = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          if (!bad) tc::tmem_ld32(srow + 32 * k, s);
+          for (int k = 0; k < 2; ++k) {
+            if (!bad) tc::tmem_ld32(srow + 32 * k, s);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float x0 = fmaf(s[2 * e], p.scale_log2, -m), x1 = fmaf(s[2 * e + 1], p.scale_log2, -m);
-            const bool v0 = 32 * k + 2 * e < nvis, v1 = 32 * k + 2 * e + 1 < nvis;
-            over |= (v0 && x0 > kLazyRescale) || (v1 && x1 > kLazyRescale);
-            const float p0 = v0 ? ex2_approx(x0) : 0.f, p1 = v1 ? ex2_approx(x1) : 0.f;
-            lsum += p0 + p1;
-            const __nv_bfloat162 two = __floats2bfloat162_rn(p0, p1);
-            w[16 * k + e] = *reinterpret_cast<const uint32_t *>(&two);
+            for (int e = 0; e < 16; ++e) {
+              const float x0 = fmaf(s[2 * e], p.scale_log2, -m), x1 = fmaf(s[2 * e + 1], p.scale_log2, -m);
+              xmax = fmaxf(xmax, fmaxf(x0, x1));
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              lsum += p0 + p1;
+              const __nv_bfloat162 two = __floats2bfloat162_rn(p0, p1);
+              w[16 * k + e] = *reinterpret_cast<const uint32_t *>(&two);
+            }
+          }
+          over = xmax > kLazyRescale;
+        } else {
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            if (!bad) tc::tmem_ld32(srow + 32 * k, s);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float x0 = fmaf(s[2 * e], p.scale_log2, -m), x1 = fmaf(s[2 * e + 1], p.scale_log2, -m);
+              const bool v0 = 32 * k + 2 * e < nvis, v1 = 32 * k + 2 * e + 1 < nvis;
+              over |= (v0 && x0 > kLazyRescale) || (v1 && x1 > kLazyRescale);
+              const float p0 = v0 ? ex2_approx(x0) : 0.f, p1 = v1 ? ex2_approx(x1) : 0.f;
+              lsum += p0 + p1;
+              const __nv_bfloat162 two = __floats2bfloat162_rn(p0, p1);
+              w[16 * k + e] = *reinterpret_cast<const uint32_t *>(&two);
+            }
           }
         }
         if (!pair_or(over || bad)) {
