@@ -85,8 +85,8 @@ def test_trace_step_by_step(cuda_device, bs):
     assert checked > 0 and len(ta.running) > 0
 
 
-@pytest.mark.parametrize("bs", [8, 16, 32])
-def test_trace_measured_step(cuda_device, bs):
+@pytest.mark.parametrize("bs,part", [(8, 512), (16, 512), (32, 512), (16, 1024), (16, 256)])
+def test_trace_measured_step(cuda_device, bs, part):
     """The trace step exactly as the benchmark times it, step by step against
     the oracle: the prompts' rows through pa_append_kv, then one
     pa_decode_shared call per step with the sharing plan (pa_share_plan) of
@@ -95,7 +95,9 @@ def test_trace_measured_step(cuda_device, bs):
     blocks and are copied when they write ("pagedattention" glossary entry,
     paragraph 5); beams whose prompts hold enough full blocks make the
     plan's groups.  Every decode row of every step is checked against the
-    oracle, the pools bit for bit every 4 steps and at the end."""
+    oracle, the pools bit for bit every 4 steps and at the end.  The
+    partition sizes the trace sweep compares at 16-token blocks run too
+    (1024: the sweep's choice on the full trace)."""
     dev = cuda_device
     Hq, Hkv, D, steps = 32, 8, 128, 40
     NB = 65536 // bs
@@ -108,7 +110,7 @@ def test_trace_measured_step(cuda_device, bs):
     tm = BeamTrace(M, lambda: len(M.free), bs, draws)
     k0 = synth.sentinel_(torch.empty(NB, Hkv, bs, D, dtype=dt))
     v0 = synth.sentinel_(torch.empty(NB, Hkv, bs, D, dtype=dt))
-    cache = pa.KVCache(k0.to(dev), v0.to(dev))
+    cache = pa.KVCache(k0.to(dev), v0.to(dev), partition_tokens=part)
     hk = oracle.host_array(k0)[0].copy()
     hv = oracle.host_array(v0)[0].copy()
     scale = 1 / math.sqrt(D)
