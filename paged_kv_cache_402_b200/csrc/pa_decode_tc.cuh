@@ -15,6 +15,13 @@
 //    from a counter once the copies of its current unit are issued, so CTAs
 //    that drew short units take more of them and all finish together.  The counter lives in one of kSchedSlots library-owned
 //    slots, chosen per call, and the last CTA out resets it.
+//  * Warp 6, on batches of mostly whole partitions, is the scheduler: it
+//    draws the CTA's next unit, looks it up and loads its table entries
+//    while the producer issues the current unit's copies, and hands the
+//    description over through a one-slot queue in shared memory.  On
+//    batches of mostly short tails the producer does that itself (the
+//    scheduler's lookups would take issue slots from the softmax warp that
+//    shares its sub-partition, once per short unit).
 //  * Warp 0 is the TMA producer.  A unit is cut into chunks of 128 tokens;
 //    each lane loads one block of a chunk: the whole (block, kv head) K tile,
 //    and then the V tile, with ONE 4-D box each (a TMA issue costs about
@@ -77,7 +84,7 @@ struct TcLayout {
   static constexpr int kOffQ = kOffV + kStages * kTile;
   static constexpr int kOffP = kOffQ + 2 * kQ;
   static constexpr int kOffBar = kOffP + 2 * kP;
-  static constexpr int kNumBars = 25;
+  static constexpr int kNumBars = 27;
   static constexpr int kOffRed = kOffBar + (kNumBars * 8 + 15) / 16 * 16;  // 16-byte aligned
   static constexpr int kRedFloats = 2 * 4 * kN;  // [parity][warp][head]
   static constexpr int kOffRedSum = kOffRed + kRedFloats * 4;
@@ -98,8 +105,13 @@ struct TcLayout {
   static constexpr int kOffPrefix = kOffPack + 3 * 2 * kN * 4;
   static constexpr int kOffCtx = kOffPrefix + (kMaxSeqs + 1) * 4;
   static constexpr int kOffFirst = kOffCtx + kMaxSeqs * 4;  // first partition of each sequence
-  static constexpr int kBytes = kOffFirst + kMaxSeqs * 4 + 1024;  // + base alignment slack
-  static constexpr int kThreads = 192;
+  // the next unit's description, from the scheduler warp to the producer:
+  // [valid, b, g, part, t0, t1, nchunks, hg, single, pack, nd, ns, -, -, -, -]
+  // + the unit's table entries
+  static constexpr int kDescHead = 16;
+  static constexpr int kOffDesc = kOffFirst + kMaxSeqs * 4;
+  static constexpr int kBytes = kOffDesc + (kDescHead + kMaxPart / 8) * 4 + 1024;  // + alignment slack
+  static constexpr int kThreads = 224;
   static constexpr uint32_t kTmemCols = 64;  // S0 S1 O0 O1, kN columns each
 };
 static_assert(TcLayout::kBytes <= 227 * 1024, "shared memory of the partition kernel");
@@ -302,6 +314,8 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   uint64_t *kfull = bars, *kempty = bars + 3, *vfull = bars + 6, *vempty = bars + 9;
   uint64_t *qfull = bars + 12, *qempty = bars + 14, *sfull = bars + 16, *pfull = bars + 18;
   uint64_t *pvdone = bars + 20, *ofree = bars + 22, *drain = bars + 24;
+  uint64_t *dfull = bars + 25, *dempty = bars + 26;  // the description slot
+  int32_t *desc = reinterpret_cast<int32_t *>(smem + L::kOffDesc);
   int32_t *prefix = reinterpret_cast<int32_t *>(smem + L::kOffPrefix);
   int32_t *ctx_s = reinterpret_cast<int32_t *>(smem + L::kOffCtx);
   int32_t *first_s = reinterpret_cast<int32_t *>(smem + L::kOffFirst);
@@ -331,6 +345,8 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       mbar_init(&ofree[i], 128);  // per unit parity: the epilogue read the unit's O
     }
     mbar_init(drain, 1);
+    mbar_init(dfull, 1);
+    mbar_init(dempty, 1);
     fence_barrier_init();
   }
   // The P tiles start zero (a plain unit only reads columns 0 .. G - 1 of S
@@ -445,9 +461,102 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   }
   const int num_tail = (p.Hkv / tail_hg) * pp_of(prefix[B]);
   const int num_units = num_full + num_tail;
+  // Batches of mostly whole partitions: a scheduler warp draws and looks up
+  // the units, so the producer's chain per unit holds only its copies.  On
+  // batches of mostly short tails its lookups would take issue slots from
+  // the softmax warp beside it on every unit; there the producer does them
+  // itself.  Every CTA takes the same decision from the same counts.
+  const bool use_sched = (int64_t)num_full * (PART / L::kChunk) >= 4 * (int64_t)num_tail;
   uint32_t *sched = g_sched + 2 * p.sched_slot;
+  const int bs = p.bs;
+  const int lg_bs = bs == 8 ? 3 : (bs == 16 ? 4 : 5);
+  // A unit's table entries (at most PART / 8), entry 32 k + lane in
+  // x[k] of the lane, loaded right after the previous unit's copies are
+  // issued.  In a fused step a unit that holds its sequence's newest token
+  // (position t1 - 1) also gets that token's block nd and the block ns to
+  // copy over it (-1: none); its loads then read the last block from ns.
+  auto pick = [](const int32_t (&x)[NE], int k) {  // x[k] by selects, never a local-memory index
+    int32_t v = x[0];
+#pragma unroll
+    for (int i = 1; i < NE; ++i) v = select_i32(k == i, x[i], v);
+    return v;
+  };
+  auto load_entries = [&](int u, TcUnit &nu, int32_t (&x)[NE], int32_t &nd, int32_t &ns) {
+#pragma unroll
+    for (int k = 0; k < NE; ++k) x[k] = -1;
+    nd = ns = -1;
+    if (u < num_units) {
+      nu = tc_unit_at<PART>(p, prefix, ctx_s, first_s, u, num_full, num_tail, tail_hg, pack_ok);
+      const int32_t *tr = p.tables + (size_t)nu.b * p.max_blocks + (nu.t0 >> lg_bs);
+      const int nb = (nu.t1 - nu.t0 + bs - 1) >> lg_bs;
+      const bool newest = p.k_new != nullptr && nu.t1 == ctx_s[nu.b];
+      const int32_t src = (newest && p.cow_src != nullptr) ? p.cow_src[nu.b] : -1;
+#pragma unroll
+      for (int k = 0; k < NE; ++k)
+        if (lane + 32 * k < nb) x[k] = tr[lane + 32 * k];
+      if (newest) {
+        const int jl = (nu.t1 - 1 - nu.t0) >> lg_bs;
+        const int32_t blk = __shfl_sync(0xffffffffu, pick(x, jl >> 5), jl & 31);
+        if (blk >= 0 && blk < p.num_blocks) {  // else its copy flags PA_DEVERR_TABLE
+          nd = blk;
+          if (src >= p.num_blocks) {
+            if (lane == 0) raise_error(PA_DEVERR_PAIR);
+          } else if (src >= 0) {
+            ns = src;
+#pragma unroll
+            for (int k = 0; k < NE; ++k) x[k] = select_i32(lane == (jl & 31) && k == (jl >> 5), src, x[k]);
+          }
+        }
+      }
+    }
+  };
 
-  if (warp == 0) {
+  if (warp == 6) {
+    // ------------------------------------------------------------ scheduler
+    // Draws the CTA's units (the first is fixed, later ones come from the
+    // call's work counter), looks each up and loads its table entries, and
+    // hands the description to the producer through the one-slot queue, so
+    // the producer's chain per unit holds only its copies.  The lookups read
+    // the lengths, tables and copy sources, which no kernel of the library
+    // writes.
+    int u = blockIdx.x, di = 0;
+    bool okq = true, first = true;
+    for (; use_sched;) {
+      TcUnit nu{};
+      int32_t x[NE], nd_, ns_;
+      load_entries(u, nu, x, nd_, ns_);
+      if (!__all_sync(0xffffffffu, mbar_wait_idle(dempty, (di & 1) ^ 1))) { okq = false; break; }
+      if (lane == 0) {
+        desc[0] = u < num_units;
+        desc[1] = nu.b;
+        desc[2] = nu.g;
+        desc[3] = nu.part;
+        desc[4] = nu.t0;
+        desc[5] = nu.t1;
+        desc[6] = nu.nchunks;
+        desc[7] = nu.hg;
+        desc[8] = nu.single;
+        desc[9] = nu.pack;
+        desc[10] = nd_;
+        desc[11] = ns_;
+      }
+#pragma unroll
+      for (int k = 0; k < NE; ++k) desc[L::kDescHead + 32 * k + lane] = x[k];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dfull);
+      ++di;
+      if (first) {
+        first = false;
+        wait_prior_grid();
+        allow_next_grid();
+      }
+      if (u >= num_units) break;
+      int raw = 0;
+      if (lane == 0) raw = (int)gridDim.x + (int)atomicAdd(sched, 1u);
+      u = __shfl_sync(0xffffffffu, raw, 0);
+    }
+    if (!okq && lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+  } else if (warp == 0) {
     // ------------------------------------------------------------ producer
     // The whole warp walks the units: its lanes load a unit's table entries
     // (at most 512 / 8 = 64) in one go, lane 0 takes them by shuffle and
@@ -459,60 +568,47 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     }
     const uint64_t pol_kv = policy_evict_first();
     const uint64_t pol_q = tc::policy_evict_last();
-    const int bs = p.bs;
     const int blocks_per_chunk = L::kChunk / bs;
     const int blocks_per_pack = kPackRows / bs;  // blocks of one head in a packed chunk
-    const int lg_bs = bs == 8 ? 3 : (bs == 16 ? 4 : 5);
     const int oob_group = p.num_blocks * p.Hkv * (bs / 8);  // first 8-row group past the pool
     int c = 0, qi = 0;
     bool ok = true;
-    // A unit's table entries (at most PART / 8), entry 32 k + lane in
-    // x[k] of the lane, loaded right after the previous unit's copies are
-    // issued.  In a fused step a unit that holds its sequence's newest token
-    // (position t1 - 1) also gets that token's block nd and the block ns to
-    // copy over it (-1: none); its loads then read the last block from ns.
-    auto pick = [](const int32_t (&x)[NE], int k) {  // x[k] by selects, never a local-memory index
-      int32_t v = x[0];
+    // the next unit's description, as the scheduler warp wrote it
+    int di = 0;
+    bool valid = false;
+    auto take = [&](TcUnit &nu, int32_t (&x)[NE], int32_t &nd_, int32_t &ns_) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(dfull, di & 1))) return false;
+      valid = desc[0] != 0;
+      nu.b = desc[1];
+      nu.g = desc[2];
+      nu.part = desc[3];
+      nu.t0 = desc[4];
+      nu.t1 = desc[5];
+      nu.nchunks = desc[6];
+      nu.hg = desc[7];
+      nu.single = desc[8] != 0;
+      nu.pack = desc[9] != 0;
+      nd_ = desc[10];
+      ns_ = desc[11];
 #pragma unroll
-      for (int i = 1; i < NE; ++i) v = select_i32(k == i, x[i], v);
-      return v;
-    };
-    auto load_entries = [&](int u, TcUnit &nu, int32_t (&x)[NE], int32_t &nd, int32_t &ns) {
-#pragma unroll
-      for (int k = 0; k < NE; ++k) x[k] = -1;
-      nd = ns = -1;
-      if (u < num_units) {
-        nu = tc_unit_at<PART>(p, prefix, ctx_s, first_s, u, num_full, num_tail, tail_hg, pack_ok);
-        const int32_t *tr = p.tables + (size_t)nu.b * p.max_blocks + (nu.t0 >> lg_bs);
-        const int nb = (nu.t1 - nu.t0 + bs - 1) >> lg_bs;
-        const bool newest = p.k_new != nullptr && nu.t1 == ctx_s[nu.b];
-        const int32_t src = (newest && p.cow_src != nullptr) ? p.cow_src[nu.b] : -1;
-#pragma unroll
-        for (int k = 0; k < NE; ++k)
-          if (lane + 32 * k < nb) x[k] = tr[lane + 32 * k];
-        if (newest) {
-          const int jl = (nu.t1 - 1 - nu.t0) >> lg_bs;
-          const int32_t blk = __shfl_sync(0xffffffffu, pick(x, jl >> 5), jl & 31);
-          if (blk >= 0 && blk < p.num_blocks) {  // else its copy flags PA_DEVERR_TABLE
-            nd = blk;
-            if (src >= p.num_blocks) {
-              if (lane == 0) raise_error(PA_DEVERR_PAIR);
-            } else if (src >= 0) {
-              ns = src;
-#pragma unroll
-              for (int k = 0; k < NE; ++k) x[k] = select_i32(lane == (jl & 31) && k == (jl >> 5), src, x[k]);
-            }
-          }
-        }
-      }
+      for (int k = 0; k < NE; ++k) x[k] = desc[L::kDescHead + 32 * k + lane];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dempty);
+      ++di;
+      return true;
     };
     TcUnit un{};
     int32_t e[NE], nd, ns;
-    int u = blockIdx.x;  // the first unit of every CTA is fixed; later ones are drawn
-    load_entries(u, un, e, nd, ns);
+    int u = blockIdx.x;  // without the scheduler: the first unit of every CTA is fixed, later ones drawn
+    if (use_sched) {
+      if (!take(un, e, nd, ns)) ok = false;
+    } else {
+      load_entries(u, un, e, nd, ns);
+      valid = u < num_units;
+    }
     if (!p.late_wait) wait_prior_grid();  // the copies read the pool and Q, which may be written just before
     allow_next_grid();
-    while (ok && u < num_units) {
+    while (ok && valid) {
       const int nb_unit = (un.t1 - un.t0 + bs - 1) >> lg_bs;
       const int hstep = un.pack ? kPackHeads : 1;
       // one (sequence, kv head, partition) at a time, or kPackHeads heads in a packed pass
@@ -577,14 +673,21 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
         if (!ok) break;
       }
       if (!ok) break;
-      // The next unit is drawn only now, with the ring full of this unit's
-      // chunks (which hide the draw's latency): a CTA never holds more work
-      // than that when the queue runs dry, so all CTAs finish together.  The
-      // copy on write goes out while the draw is in flight.
-      int raw_next = 0;
-      if (lane == 0) raw_next = (int)gridDim.x + (int)atomicAdd(sched, 1u);
-      u = __shfl_sync(0xffffffffu, raw_next, 0);
-      load_entries(u, un, e, nd, ns);
+      if (use_sched) {
+        // the next unit, which the scheduler warp drew and looked up while
+        // this one's copies went out
+        if (!take(un, e, nd, ns)) { ok = false; break; }
+      } else {
+        // The next unit is drawn only now, with the ring full of this unit's
+        // chunks (which hide the draw's latency): a CTA never holds more work
+        // than that when the queue runs dry, so all CTAs finish together.
+        // The copy on write goes out while the draw is in flight.
+        int raw_next = 0;
+        if (lane == 0) raw_next = (int)gridDim.x + (int)atomicAdd(sched, 1u);
+        u = __shfl_sync(0xffffffffu, raw_next, 0);
+        load_entries(u, un, e, nd, ns);
+        valid = u < num_units;
+      }
     }
     if (ok) {  // no work left: publish an empty unit so the consumers stop
       const int qs = qi & 1;
@@ -774,7 +877,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     if (lane == 0) tc::mma_commit(drain);
     __syncwarp();
     mbar_wait(drain, 0);
-  } else {
+  } else if (warp < 6) {
     // ------------------------------------------------------------ softmax + epilogue
     if (!p.late_wait) wait_prior_grid();  // before the first write of out / the workspace
     allow_next_grid();

@@ -103,6 +103,35 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
   }
 }
 
+// mbar_wait for a warp that is not on a critical path: between polls it
+// sleeps, so that it leaves the issue slots of its sub-partition to the
+// warps beside it.
+__device__ __forceinline__ bool mbar_wait_idle(uint64_t *bar, uint32_t parity,
+                                               uint64_t limit_ns = kWaitLimitNs) {
+  const uint32_t addr = smem_u32(bar);
+  const uint64_t start = global_ns();
+  for (;;) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (global_ns() - start > limit_ns) {
+      if (atomicCAS(&g_wait_timeout[0], 0u, 1u) == 0u) {
+        g_wait_timeout[1] = addr;
+        g_wait_timeout[2] = parity | (blockIdx.x << 1);
+        g_wait_timeout[3] = threadIdx.x;
+      }
+      return false;
+    }
+    __nanosleep(100);
+  }
+}
+
 // Makes this thread's earlier generic-proxy shared-memory accesses ordered
 // before later async-proxy (bulk copy) accesses of the same memory.
 __device__ __forceinline__ void fence_proxy_async_smem() {
