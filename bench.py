@@ -400,6 +400,21 @@ WORKLOADS = {
 }
 
 
+def decode_launches(n_seqs: int, max_ctx: int, part: int, n_groups: int = 0) -> int:
+    """Kernel launches of one decode call: with a plan that has groups, the
+    cascade (one launch per 1024 groups); the partition kernel (one per slice
+    of at most 1024 sequences whose whole partitions fit its 20-bit counts);
+    the log-sum-exp reduce (more than one partition, or a plan)."""
+    max_parts = max(-(-max_ctx // part), 1)
+    per_launch = max(min(1024, ((1 << 20) - 1) // max_parts), 1)
+    n = -(-n_seqs // per_launch)
+    if n_groups:
+        n += -(-n_groups // 1024)
+    if max_parts > 1 or n_groups:
+        n += 1
+    return n
+
+
 def aggregate_ranks(world: int, ms: float, kv_gb: float, tokens: float, e2e_s: float, e2e_gb: float, device):
     """Whole-job figures of the replicas: the slowest rank's times, the sum
     of every rank's work.  Returns (ms, GB, tokens, end-to-end GB/s).  Every
@@ -453,7 +468,8 @@ def run_ours(args, rank: int, world: int, dev):
                                 scale, cow_src=st["cow"], out=st["out"], workspace=st["ws"], stream=strm)
         if ev is not None:
             ev[1].record(strm)
-        n += 2 if st["max_ctx"] > wl["part"] else 1
+        groups = st["plan"].n_groups if (st["plan"] is not None and not args.unfused and not args.no_share_plan) else 0
+        n += decode_launches(len(st["lens"]), st["max_ctx"], wl["part"], groups)
         return n, st
 
     for s in range(args.warmup):
@@ -1028,15 +1044,15 @@ def run_trace(args, dev):
                     launches += 1
                 pa.pa_append_kv(kd, kd, d_[1], cache, stream)
                 pa.pa_decode(q, cache, d_[3], d_[4], max_ctx, 1 / math.sqrt(D), out=o, workspace=ws, stream=stream)
-                launches += 2 + (1 if max_ctx > part else 0)
+                launches += 1 + decode_launches(n, max_ctx, part)
             elif args.no_share_plan:
                 pa.pa_append_decode(kd, kd, q, cache, d_[3], d_[4], max_ctx, 1 / math.sqrt(D), cow_src=d_[5],
                                     out=o, workspace=ws, stream=stream)
-                launches += 1 + (1 if max_ctx > part else 0)
+                launches += decode_launches(n, max_ctx, part)
             else:
                 pa.pa_decode_shared(q, cache, d_[3], d_[4], max_ctx, 1 / math.sqrt(D), plan=dplan,
                                     k_new=kd, v_new=kd, cow_src=d_[5], out=o, workspace=ws, stream=stream)
-                launches += 1 + (1 if max_ctx > part else 0) + (1 if splan.n_groups else 0)
+                launches += decode_launches(n, max_ctx, part, splan.n_groups)
                 h2d += splan.nbytes
             ev[s_][1].record(stream)
             res = o[:1].to("cpu", non_blocking=True)
