@@ -403,10 +403,11 @@ WORKLOADS = {
 def decode_launches(n_seqs: int, max_ctx: int, part: int, n_groups: int = 0) -> int:
     """Kernel launches of one decode call: with a plan that has groups, the
     cascade (one launch per 1024 groups); the partition kernel (one per slice
-    of at most 1024 sequences whose whole partitions fit its 20-bit counts);
-    the log-sum-exp reduce (more than one partition, or a plan)."""
+    of at most 8192 sequences, or 1024 when the batch holds no more, whose
+    whole partitions fit 20 bits); the log-sum-exp reduce (more than one
+    partition, or a plan)."""
     max_parts = max(-(-max_ctx // part), 1)
-    per_launch = max(min(1024, ((1 << 20) - 1) // max_parts), 1)
+    per_launch = max(min(1024 if n_seqs <= 1024 else 8192, ((1 << 20) - 1) // max_parts), 1)
     n = -(-n_seqs // per_launch)
     if n_groups:
         n += -(-n_groups // 1024)

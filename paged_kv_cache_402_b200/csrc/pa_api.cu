@@ -289,7 +289,7 @@ bool tc_eligible(const pa::DecodeParams &p, int dtype, int D) {
   return true;  // a missing tensor-map encoder then fails the launch loudly (PA_ERR_CUDA)
 }
 
-template <int G, int PART>
+template <int G, int PART, bool COARSE>
 pa_status launch_decode_tc_slice(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
   CUtensorMap mk, mv, mq;
   const uint64_t rows = (uint64_t)p.num_blocks * p.Hkv * p.bs;
@@ -298,7 +298,7 @@ pa_status launch_decode_tc_slice(const pa::DecodeParams &p, int32_t max_parts, c
       !make_map_pool_4d(&mv, p.v, rows, (uint32_t)p.bs) ||
       !make_map_q_halves(&mq, p.q, (uint64_t)p.B * p.Hq, (uint32_t)pa::TcLayout::kN))
     return PA_ERR_CUDA;
-  auto kern = pa::decode_partition_tc<G, PART>;
+  auto kern = pa::decode_partition_tc<G, PART, COARSE>;
   const int smem = pa::TcLayout::kBytes;
   static std::atomic<int> smem_set[kMaxDev] = {};
   if (!ensure_smem(kern, smem, smem_set)) return PA_ERR_CUDA;
@@ -310,16 +310,17 @@ pa_status launch_decode_tc_slice(const pa::DecodeParams &p, int32_t max_parts, c
 }
 
 // Sequences are independent: a batch larger than the kernel's per-CTA
-// sequence tables runs as consecutive launches over slices of it, and one
-// reduce over the whole batch follows the last (each launch completes only
-// after the one before it, so the reduce sees every slice's rows).
+// sequence tables (kMaxSeqs sequences, or kCoarse times that in its coarse
+// form) runs as consecutive launches over slices of it, and one reduce over
+// the whole batch follows the last (each launch completes only after the one
+// before it, so the reduce sees every slice's rows).
 std::atomic<uint32_t> g_sched_ticket{0};
 
 template <int G, int PART>
 pa_status launch_decode_tc_g(const pa::DecodeParams &p, int32_t max_parts, cudaStream_t st) {
-  // a slice is at most kMaxSeqs sequences, and its full partitions must fit
-  // the 20-bit counts of the kernel's packed prefix sums
-  int slice = pa::TcLayout::kMaxSeqs;
+  // a slice is at most kCoarse x kMaxSeqs sequences, and, at most kMaxSeqs
+  // of them (the packed prefix sums), its full partitions must fit 20 bits
+  int slice = p.B > pa::TcLayout::kMaxSeqs ? pa::kCoarse * pa::TcLayout::kMaxSeqs : pa::TcLayout::kMaxSeqs;
   const int by_parts = ((1 << pa::kFullBits) - 1) / (max_parts > 0 ? max_parts : 1);
   if (by_parts < slice) slice = by_parts > 0 ? by_parts : 1;
   for (int b0 = 0; b0 < p.B; b0 += slice) {
@@ -342,7 +343,8 @@ pa_status launch_decode_tc_g(const pa::DecodeParams &p, int32_t max_parts, cudaS
       ps.ws_acc = p.ws_acc + rows * p.row_stride * 128;
     }
     ps.sched_slot = (int32_t)(g_sched_ticket.fetch_add(1) % pa::kSchedSlots);
-    const pa_status s = launch_decode_tc_slice<G, PART>(ps, max_parts, st);
+    const pa_status s = ps.B > pa::TcLayout::kMaxSeqs ? launch_decode_tc_slice<G, PART, true>(ps, max_parts, st)
+                                                       : launch_decode_tc_slice<G, PART, false>(ps, max_parts, st);
     if (s != PA_OK) return s;
   }
   if (p.row_stride <= 1) return PA_OK;  // one partition, no plan: written directly

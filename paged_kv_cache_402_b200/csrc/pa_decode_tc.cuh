@@ -199,6 +199,7 @@ constexpr float kLazyRescale = 8.0f;
 
 struct TcUnit {
   int b, g, part, t0, t1, nchunks;
+  int ctx;  // the sequence's length
   int hg;  // kv heads of the unit: g .. g + hg - 1 (1 for a full partition)
   bool single;
   bool pack;  // passes of kPackHeads heads, kPackRows tokens per head per chunk
@@ -216,6 +217,30 @@ constexpr int kFullBits = 20;
 __device__ __forceinline__ int pf_of(int32_t v) { return v & ((1 << kFullBits) - 1); }
 __device__ __forceinline__ int pp_of(int32_t v) { return (int)((uint32_t)v >> kFullBits); }
 
+// Launches of more than TcLayout::kMaxSeqs sequences (up to kCoarse times
+// that) take the kernel's COARSE form: for entries of kCoarse consecutive
+// sequences, the prefix sums of their full partitions (prefix) and of their
+// partial last ones (pprefix, where ctx_s is in the other form), unpacked;
+// a lookup finds the entry, then the sequence from its members' lengths,
+// one lane each.  One launch then covers a whole batch of a few thousand
+// sequences.
+constexpr int kCoarse = 8;
+
+// Sequence b's length, first token (as validated: 0 unless a whole number
+// of blocks inside the sequence), and its full partitions (from the one its
+// first token falls in) and partial last one.
+template <int PART>
+__device__ __forceinline__ void seq_counts(const DecodeParams &p, int b, int &ctx, int &ft, int &nfull,
+                                           int &npart) {
+  ctx = p.lens[b];
+  ft = p.first_tok ? p.first_tok[b] : 0;
+  const bool ok = ctx >= 0 && ctx <= p.max_ctx;
+  if (ft != 0 && (!ok || ft < 0 || ft >= ctx || ft % p.bs != 0)) ft = 0;
+  const bool own = ok && ctx > 0;
+  nfull = own ? ctx / PART - ft / PART : 0;
+  npart = own && ctx % PART != 0 ? 1 : 0;
+}
+
 // Unit u of the largest-first order.  The full partitions (sequence-major,
 // kv head fastest; a sequence's first one is the partition its first token
 // first_s[b] falls in, which then starts at that token) are one kv head each; the partial last partitions are tail_hg consecutive kv heads of
@@ -226,10 +251,12 @@ __device__ __forceinline__ int pp_of(int32_t v) { return (int)((uint32_t)v >> kF
 // after, and a launch ends on units of one full partition either way.  With
 // pack_ok (tail_hg then a multiple of kPackHeads), a tail unit goes in
 // head-packed passes when they take fewer chunks in all.
-template <int PART>
+// Called by a whole warp with the same u (a coarse lookup shares the work).
+template <int PART, bool COARSE>
 __device__ __forceinline__ TcUnit tc_unit_at(const DecodeParams &p, const int32_t *prefix,
                                              const int32_t *ctx_s, const int32_t *first_s, int u,
-                                             int num_full, int num_tail, int tail_hg, bool pack_ok) {
+                                             int num_full, int num_tail, int tail_hg, bool pack_ok,
+                                             int n_ent) {
   TcUnit un;
   const bool tails_first = tail_hg > 1;
   const bool full = tails_first ? u >= num_tail : u < num_full;
@@ -238,16 +265,49 @@ __device__ __forceinline__ TcUnit tc_unit_at(const DecodeParams &p, const int32_
   const int w = v / per_seq;
   un.hg = full ? 1 : tail_hg;
   un.g = (v - w * per_seq) * un.hg;
-  int lo = 0, hi = p.B - 1;  // largest b whose count before it is <= w
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    const int cnt = full ? pf_of(prefix[mid]) : pp_of(prefix[mid]);
-    if (cnt <= w) lo = mid; else hi = mid - 1;
+  int ctx, first, before;  // before: the unit's kind of partitions ahead of its sequence's
+  if constexpr (!COARSE) {
+    int lo = 0, hi = p.B - 1;  // largest b whose count before it is <= w
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      const int cnt = full ? pf_of(prefix[mid]) : pp_of(prefix[mid]);
+      if (cnt <= w) lo = mid; else hi = mid - 1;
+    }
+    un.b = lo;
+    ctx = ctx_s[lo];
+    first = first_s[lo];
+    before = pf_of(prefix[lo]);
+  } else {
+    const int32_t *pre = full ? prefix : ctx_s;  // the full / partial prefix sums
+    int lo = 0, hi = n_ent - 1;  // largest entry whose count before it is <= w
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pre[mid] <= w) lo = mid; else hi = mid - 1;
+    }
+    // lane i < kCoarse: the entry's i-th sequence, its count of the unit's kind
+    const int lane = threadIdx.x & 31, i = lane & (kCoarse - 1);
+    const int b = lo * kCoarse + i;
+    int c = 0, sctx = 0, sft = 0, nf = 0, np = 0;
+    if (lane < kCoarse && b < p.B) {
+      seq_counts<PART>(p, b, sctx, sft, nf, np);
+      c = full ? nf : np;
+    }
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < kCoarse; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o, kCoarse);
+      if (i >= o) incl += t;
+    }
+    const int rel = w - pre[lo];
+    const unsigned hit = __ballot_sync(0xffffffffu, lane < kCoarse && incl - c <= rel && rel < incl);
+    const int src = hit ? __ffs(hit) - 1 : 0;
+    un.b = lo * kCoarse + src;
+    ctx = __shfl_sync(0xffffffffu, sctx, src);
+    first = __shfl_sync(0xffffffffu, sft, src);
+    before = pre[lo] + __shfl_sync(0xffffffffu, incl - c, src);
   }
-  un.b = lo;
-  const int ctx = ctx_s[lo];
-  const int first = first_s[lo];
-  un.part = full ? first / PART + w - pf_of(prefix[lo]) : ctx / PART;
+  un.ctx = ctx;
+  un.part = full ? first / PART + w - before : ctx / PART;
   un.t0 = max(un.part * PART, first);
   un.t1 = min((un.part + 1) * PART, ctx);
   const int len = un.t1 - un.t0;
@@ -285,7 +345,7 @@ __device__ __forceinline__ bool wg_sync_or(int pred) {
 }
 
 // PART: tokens per partition (256, 512 or 1024); the caller's p.part.
-template <int G, int PART>
+template <int G, int PART, bool COARSE>
 __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     decode_partition_tc(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v,
@@ -355,73 +415,160 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   for (int i = threadIdx.x; i < (2 * L::kQ + 2 * L::kP) / 16; i += blockDim.x)
     reinterpret_cast<uint4 *>(smem + L::kOffQ)[i] = make_uint4(0, 0, 0, 0);
 
-  // partition counts of every sequence and their exclusive prefix sums
+  // partition counts of every sequence (COARSE: of every entry of kCoarse
+  // sequences) and their exclusive prefix sums
   const int B = p.B;
-  constexpr int kMaxSeg = (L::kMaxSeqs + L::kThreads - 1) / L::kThreads;
-  const int seg = (B + blockDim.x - 1) / blockDim.x;
-  const int b_first = threadIdx.x * seg;
-  int cnt[kMaxSeg];
-  int mine = 0;
-  // chunks of this thread's partial last partitions (128-token chunks, and
-  // kPackRows-token ones of a packed pass), and their count
-  int tail_chunks = 0, tail_pchunks = 0, tails = 0;
+  const int n_ent = COARSE ? (B + kCoarse - 1) / kCoarse : B;
+  if constexpr (!COARSE) {
+    constexpr int kMaxSeg = (L::kMaxSeqs + L::kThreads - 1) / L::kThreads;
+    const int seg = (B + blockDim.x - 1) / blockDim.x;
+    const int b_first = threadIdx.x * seg;
+    int cnt[kMaxSeg];
+    int mine = 0;
+    // chunks of this thread's partial last partitions (128-token chunks, and
+    // kPackRows-token ones of a packed pass), and their count
+    int tail_chunks = 0, tail_pchunks = 0, tails = 0;
 #pragma unroll
-  for (int i = 0; i < kMaxSeg; ++i) {
-    cnt[i] = 0;
-    const int b = b_first + i;
-    if (i < seg && b < B) {
-      const int ctx = p.lens[b];
-      const bool ok = ctx >= 0 && ctx <= p.max_ctx;
-      // tokens the cascade kernel did: a whole number of blocks before the last
-      int ft = p.first_tok ? p.first_tok[b] : 0;
-      if (ft != 0 && (!ok || ft < 0 || ft >= ctx || ft % p.bs != 0)) {
-        if (blockIdx.x == 0) raise_error(PA_DEVERR_PLAN);
-        ft = 0;  // this kernel then does the whole sequence
+    for (int i = 0; i < kMaxSeg; ++i) {
+      cnt[i] = 0;
+      const int b = b_first + i;
+      if (i < seg && b < B) {
+        const int ctx = p.lens[b];
+        const bool ok = ctx >= 0 && ctx <= p.max_ctx;
+        // tokens the cascade kernel did: a whole number of blocks before the last
+        int ft = p.first_tok ? p.first_tok[b] : 0;
+        if (ft != 0 && (!ok || ft < 0 || ft >= ctx || ft % p.bs != 0)) {
+          if (blockIdx.x == 0) raise_error(PA_DEVERR_PLAN);
+          ft = 0;  // this kernel then does the whole sequence
+        }
+        if (ok && ctx % PART != 0) {
+          const int tl = ctx - max(ctx / PART * PART, ft);
+          tail_chunks += (tl + TcLayout::kChunk - 1) / TcLayout::kChunk;
+          tail_pchunks += (tl + kPackRows - 1) / kPackRows;
+          ++tails;
+        }
+        ctx_s[b] = ctx;
+        first_s[b] = ft;
+        // partitions from the one token ft falls in: the ones that end on a
+        // partition boundary in the low bits, a partial last one in the high ones
+        cnt[i] = (ok && ctx > 0) ? (ctx / PART - ft / PART) | ((ctx % PART != 0 ? 1 : 0) << kFullBits) : 0;
+        mine += cnt[i];
+        if (blockIdx.x == 0 && !ok) raise_error(PA_DEVERR_LEN);
       }
-      if (ok && ctx % PART != 0) {
-        const int tl = ctx - max(ctx / PART * PART, ft);
-        tail_chunks += (tl + TcLayout::kChunk - 1) / TcLayout::kChunk;
-        tail_pchunks += (tl + kPackRows - 1) / kPackRows;
-        ++tails;
-      }
-      ctx_s[b] = ctx;
-      first_s[b] = ft;
-      // partitions from the one token ft falls in: the ones that end on a
-      // partition boundary in the low bits, a partial last one in the high ones
-      cnt[i] = (ok && ctx > 0) ? (ctx / PART - ft / PART) | ((ctx % PART != 0 ? 1 : 0) << kFullBits) : 0;
-      mine += cnt[i];
-      if (blockIdx.x == 0 && !ok) raise_error(PA_DEVERR_LEN);
     }
-  }
-  int incl = mine;  // inclusive scan within the warp
+    int incl = mine;  // inclusive scan within the warp
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) scan[warp] = incl;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) scan[warp] = incl;
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    tail_chunks += __shfl_xor_sync(0xffffffffu, tail_chunks, o);
-    tail_pchunks += __shfl_xor_sync(0xffffffffu, tail_pchunks, o);
-    tails += __shfl_xor_sync(0xffffffffu, tails, o);
-  }
-  if (lane == 0) {
-    scan[8 + warp] = tail_chunks;
-    scan[16 + warp] = tails;
-    scan[24 + warp] = tail_pchunks;
-  }
-  if (warp == 1) tc::tmem_alloc(tmem_slot, L::kTmemCols);
-  __syncthreads();
-  int run = incl - mine;
-  for (int w = 0; w < warp; ++w) run += scan[w];
+    for (int o = 16; o >= 1; o >>= 1) {
+      tail_chunks += __shfl_xor_sync(0xffffffffu, tail_chunks, o);
+      tail_pchunks += __shfl_xor_sync(0xffffffffu, tail_pchunks, o);
+      tails += __shfl_xor_sync(0xffffffffu, tails, o);
+    }
+    if (lane == 0) {
+      scan[8 + warp] = tail_chunks;
+      scan[16 + warp] = tails;
+      scan[24 + warp] = tail_pchunks;
+    }
+    if (warp == 1) tc::tmem_alloc(tmem_slot, L::kTmemCols);
+    __syncthreads();
+    int run = incl - mine;
+    for (int w = 0; w < warp; ++w) run += scan[w];
 #pragma unroll
-  for (int i = 0; i < kMaxSeg; ++i) {
-    const int b = b_first + i;
-    if (i < seg && b < B) {
-      prefix[b] = run;
-      run += cnt[i];
-      if (b == B - 1) prefix[B] = run;
+    for (int i = 0; i < kMaxSeg; ++i) {
+      const int b = b_first + i;
+      if (i < seg && b < B) {
+        prefix[b] = run;
+        run += cnt[i];
+        if (b == B - 1) prefix[B] = run;
+      }
+    }
+  } else {
+    constexpr int kMaxSeg = (L::kMaxSeqs + L::kThreads - 1) / L::kThreads;
+    const int seg = (n_ent + blockDim.x - 1) / blockDim.x;
+    const int e_first = threadIdx.x * seg;
+    int cnt[kMaxSeg], cntp[kMaxSeg];
+    int mine = 0, minep = 0;
+    int tail_chunks = 0, tail_pchunks = 0, tails = 0;
+#pragma unroll
+    for (int i = 0; i < kMaxSeg; ++i) {
+      cnt[i] = cntp[i] = 0;
+      const int e = e_first + i;
+      if (i < seg && e < n_ent) {
+#pragma unroll
+        for (int k = 0; k < kCoarse; ++k) {
+          const int b = e * kCoarse + k;
+          if (b < B) {
+            int ctx, ft, nf, np;
+            seq_counts<PART>(p, b, ctx, ft, nf, np);
+            if (blockIdx.x == 0 && p.first_tok && p.first_tok[b] != ft) raise_error(PA_DEVERR_PLAN);
+            if (blockIdx.x == 0 && !(ctx >= 0 && ctx <= p.max_ctx)) raise_error(PA_DEVERR_LEN);
+            if (np) {
+              const int tl = ctx - max(ctx / PART * PART, ft);
+              tail_chunks += (tl + TcLayout::kChunk - 1) / TcLayout::kChunk;
+              tail_pchunks += (tl + kPackRows - 1) / kPackRows;
+              ++tails;
+            }
+            cnt[i] += nf;
+            cntp[i] += np;
+          }
+        }
+        mine += cnt[i];
+        minep += cntp[i];
+      }
+    }
+    int incl = mine, inclp = minep;  // inclusive scans within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      const int vp = __shfl_up_sync(0xffffffffu, inclp, o);
+      if (lane >= o) {
+        incl += v;
+        inclp += vp;
+      }
+    }
+    // the warps' partial-count totals go to first_s[8 ..] (first_s is not
+    // used in this form; the partial prefix sums reach first_s[0] at most)
+    if (lane == 31) {
+      scan[warp] = incl;
+      first_s[8 + warp] = inclp;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      tail_chunks += __shfl_xor_sync(0xffffffffu, tail_chunks, o);
+      tail_pchunks += __shfl_xor_sync(0xffffffffu, tail_pchunks, o);
+      tails += __shfl_xor_sync(0xffffffffu, tails, o);
+    }
+    if (lane == 0) {
+      scan[8 + warp] = tail_chunks;
+      scan[16 + warp] = tails;
+      scan[24 + warp] = tail_pchunks;
+    }
+    if (warp == 1) tc::tmem_alloc(tmem_slot, L::kTmemCols);
+    __syncthreads();
+    int run = incl - mine, runp = inclp - minep;
+    for (int w = 0; w < warp; ++w) {
+      run += scan[w];
+      runp += first_s[8 + w];
+    }
+    int32_t *pprefix = ctx_s;
+#pragma unroll
+    for (int i = 0; i < kMaxSeg; ++i) {
+      const int e = e_first + i;
+      if (i < seg && e < n_ent) {
+        prefix[e] = run;
+        pprefix[e] = runp;
+        run += cnt[i];
+        runp += cntp[i];
+        if (e == n_ent - 1) {
+          prefix[n_ent] = run;
+          pprefix[n_ent] = runp;
+        }
+      }
     }
   }
   if (warp == 1) tc::tmem_relinquish();
@@ -430,7 +577,9 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int num_full = p.Hkv * pf_of(prefix[B]);
+  const int full_total = COARSE ? prefix[n_ent] : pf_of(prefix[B]);
+  const int part_total = COARSE ? ctx_s[n_ent] : pp_of(prefix[B]);
+  const int num_full = p.Hkv * full_total;
   // A partial last partition of a few chunks is a short unit, and a unit's
   // scheduling (the draw, the unit's lookup, its table entries) is a serial
   // chain of the producer; so the partial partitions of one sequence go out
@@ -459,7 +608,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
       tail_hg = kPackHeads;
     }
   }
-  const int num_tail = (p.Hkv / tail_hg) * pp_of(prefix[B]);
+  const int num_tail = (p.Hkv / tail_hg) * part_total;
   const int num_units = num_full + num_tail;
   // Batches of mostly whole partitions: a scheduler warp draws and looks up
   // the units, so the producer's chain per unit holds only its copies.  On
@@ -486,10 +635,10 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     for (int k = 0; k < NE; ++k) x[k] = -1;
     nd = ns = -1;
     if (u < num_units) {
-      nu = tc_unit_at<PART>(p, prefix, ctx_s, first_s, u, num_full, num_tail, tail_hg, pack_ok);
+      nu = tc_unit_at<PART, COARSE>(p, prefix, ctx_s, first_s, u, num_full, num_tail, tail_hg, pack_ok, n_ent);
       const int32_t *tr = p.tables + (size_t)nu.b * p.max_blocks + (nu.t0 >> lg_bs);
       const int nb = (nu.t1 - nu.t0 + bs - 1) >> lg_bs;
-      const bool newest = p.k_new != nullptr && nu.t1 == ctx_s[nu.b];
+      const bool newest = p.k_new != nullptr && nu.t1 == nu.ctx;
       const int32_t src = (newest && p.cow_src != nullptr) ? p.cow_src[nu.b] : -1;
 #pragma unroll
       for (int k = 0; k < NE; ++k)
@@ -885,7 +1034,7 @@ __global__ void __launch_bounds__(TcLayout::kThreads, 1)
     const int r = wq * 32 + lane;         // token row (softmax) / head-dim row (O)
     if (blockIdx.x == 0) {  // rows no unit writes (empty or invalid length): zeros
       for (int b = r; b < p.B; b += 128) {
-        const int ctx = ctx_s[b];
+        const int ctx = COARSE ? p.lens[b] : ctx_s[b];
         if (ctx <= 0 || ctx > p.max_ctx) {
           uint4 *o = reinterpret_cast<uint4 *>(out + (size_t)b * p.Hq * 128);
           for (int e = 0; e < p.Hq * 128 / 8; ++e) o[e] = make_uint4(0, 0, 0, 0);

@@ -56,24 +56,29 @@ def test_row_reduce_matches_block_reduce_bits(cuda_device, parts, G, dtype, D):
     assert_attn_close(rows_path, ref, dtype)
 
 
-@pytest.mark.parametrize("B,G", [(1100, 4), (1500, 8)])
+@pytest.mark.parametrize("B,G", [(1100, 4), (1500, 8), (8300, 1)])
 def test_row_reduce_many_rows(cuda_device, B, G):
-    """1100 sequences (two launches of the tensor-core kernel, 1024 + 76, each
-    with its own reduce) and 1500 x 16 query heads = 24000 rows (more rows
-    than the grid-stride reduce has warps), every fifth sequence with 2 to 4
-    partitions.  Sampled rows against the oracle."""
+    """More sequences than the tensor-core kernel's per-sequence tables hold
+    (1024): 1100 and 1500 take its coarse tables (entries of 8 sequences) in
+    one launch, 8300 two launches (8192 + 108) before one reduce; 1500 x 16
+    query heads = 24000 rows is more than the grid-stride reduce has warps.
+    Every fifth sequence (every 25th of 8300) has 2 to 4 partitions.
+    Sampled rows against the oracle."""
     Hkv = 2
     r = synth.rng(95 + B)
     lens = r.integers(1, 64, size=B).astype(np.int32)
-    multi = np.arange(0, B, 5)
+    multi = np.arange(0, B, 5 if B < 4096 else 25)
     lens[multi] = r.integers(PART + 1, 4 * PART, size=len(multi))
     lens[1020:1030] = 4 * PART - 3
+    if B > 8192:
+        lens[8188:8196] = 4 * PART - 5
     case = synth.random_case(95, B=B, Hq=G * Hkv, Hkv=Hkv, D=128, bs=16, lens=lens, dtype=torch.bfloat16,
                              pool_factor=1.05)
     cache, q, tables, lens_d = to_dev(case, cuda_device)
     out = pa.pa_decode(q, cache, tables, lens_d, int(lens.max()), case.scale)
     assert pa.pa_read_device_error() == 0
-    seqs = sorted(set(list(range(0, B, 15)) + list(range(1016, 1032))))
+    seqs = sorted(set(list(range(0, B, 15)) + list(range(1016, 1032)) +
+                      (list(range(8184, 8200)) if B > 8192 else [])))
     rows = [(b, h) for b in seqs for h in (0, G * Hkv - 1)]
     ref = oracle.decode(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens, case.scale,
                         rows=rows)

@@ -147,10 +147,9 @@ def test_shared_plan_that_does_not_fit(cuda_device, bad):
 
 
 def test_shared_plan_across_batch_slices(cuda_device):
-    """1101 sequences (two slices of the main decode kernel, 1024 + 77) in
-    groups of 3 forks, one group straddling the slice boundary; with the
-    fused append.  The cascade kernel sees the whole batch, the main kernel
-    each slice with its own first tokens."""
+    """1101 sequences (more than the partition kernel's per-sequence tables:
+    its coarse form, entries of 8 sequences) in groups of 3 forks, one group
+    straddling sequence 1024; with the fused append."""
     dt, Hkv, D, bs, Hq = torch.bfloat16, 2, 128, 16, 8
     roots_n, fan = 367, 3
     prompts = (600 + synth.rng(101).integers(0, 400, size=roots_n)).tolist()
