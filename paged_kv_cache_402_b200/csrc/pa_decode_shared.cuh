@@ -18,8 +18,11 @@
 //
 // Same machinery as decode_partition_tc (see there): persistent CTAs, a TMA
 // producer warp loading whole (block, kv head) tiles as 4-D boxes into
-// 128-byte-swizzled K and V rings, one MMA warp, softmax warps with the lazy
-// reference and the transposed column reductions.  What differs:
+// 128-byte-swizzled K and V rings, softmax warps with the lazy reference and
+// the transposed column reductions.  What differs:
+//  * two MMA lanes: warp 1 issues the QKs, warp 10 the PVs (one lane issuing
+//    both streams in order set the pace: a chunk's PV waited behind the next
+//    chunk's K tile and QK issue);
 //  * a work unit is (group, kv head, piece): a whole partition or the
 //    shorter piece at the end of the shared tokens, handed out round-robin;
 //    the producer loads the next unit's description while the current
@@ -68,7 +71,7 @@ struct ShLayout {
   static constexpr int kOffPrefix = kOffScan + 64;  // pieces before each group
   static constexpr int kOffShared = kOffPrefix + (kMaxGroups + 1) * 4;  // each group's shared tokens
   static constexpr int kBytes = kOffShared + kMaxGroups * 4 + 1024;
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 352;  // producer, QK lane, 8 softmax warps, PV lane
   static constexpr uint32_t kTmemCols = 128;  // S0 S1 O0 O1, kN columns each
 };
 
@@ -137,13 +140,13 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&qfull[i], 1);
-      mbar_init(&qempty[i], 3);  // the MMA lane's commit + each softmax warpgroup
+      mbar_init(&qempty[i], 4);  // the QK lane's commit, each softmax warpgroup, the PV lane
       mbar_init(&sfull[i], 1);
       mbar_init(&pfull[i], 256);
       mbar_init(&pvdone[i], 1);
       mbar_init(&ofree[i], 256);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, 2);  // the QK and the PV lanes' last commits
     fence_barrier_init();
   }
   // Q rows a member slot does not use (G..7) and unused P rows stay zero
@@ -354,84 +357,84 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
       }
       for (int k = (qi > 2 ? qi - 2 : 0); k < qi; ++k) mbar_wait(&qfull[k & 1], (k >> 1) & 1, 100000000ull);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 10) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two lanes issue the MMAs, so that neither waits behind the other's
+    // stream: warp 1 the QKs (as each K tile lands, and once the softmax has
+    // written P(c - 2), so has read S(c - 2) whose buffer QK(c) takes), warp
+    // 10 the PVs (as each chunk's P and V are in).  Each commits its own
+    // barriers; the softmax waits for PV(c - 2) before it writes P(c) over
+    // P(c - 2)'s buffer.
     wait_prior_grid();
     allow_next_grid();
     constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(128, N, false, false);
     constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(128, N, true, false);
     const uint32_t kbase0 = smem_u32(smem + L::kOffK), vbase0 = smem_u32(smem + L::kOffV);
     const uint32_t qbase0 = smem_u32(smem + L::kOffQ), pbase0 = smem_u32(smem + L::kOffP);
+    const bool qk_lane = warp == 1;
     bool ok = true;
     auto warp_wait = [&](uint64_t *bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity));
     };
-    struct PvJob {
-      int c, u;
-      bool first;
-    };
-    auto issue_pv = [&](const PvJob &j) -> bool {
-      const int c = j.c;
-      if (!warp_wait(&pfull[c & 1], (c >> 1) & 1)) return false;
-      if (!warp_wait(&vfull[c % L::kStages], (c / L::kStages) & 1)) return false;
-      if (j.first && !warp_wait(&ofree[j.u & 1], ((j.u >> 1) & 1) ^ 1)) return false;
-      if (lane == 0) {
-        tc::fence_after_sync();
-        const uint32_t vb = vbase0 + (c % L::kStages) * L::kTile;
-        const uint32_t pb = pbase0 + (c & 1) * L::kP;
-        const uint32_t d = tmem + 2 * N + (j.u & 1) * N;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = tc::smem_desc_sw128(vb + kk * 2 * L::kGroup, 1024, L::kGroup);
-          const uint64_t bdesc = tc::smem_desc_sw128(pb + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
-          tc::mma_bf16(d, a, bdesc, idesc_pv, (kk > 0 || !j.first) ? 1u : 0u);
-        }
-        tc::mma_commit(&pvdone[c & 1]);
-        tc::mma_commit(&vempty[c % L::kStages]);
-      }
-      __syncwarp();
-      return true;
-    };
     int c = 0, qi = 0;
-    PvJob pending{-1, 0, false};
     while (ok) {
       const int qs = qi & 1;
       if (!warp_wait(&qfull[qs], (qi >> 1) & 1)) { ok = false; break; }
-      if (unit_slots[qs * L::kUnitInts + 3] == 0) break;  // the producer ran out of work
+      const int nmem = unit_slots[qs * L::kUnitInts + 3];
       const uint32_t qb = qbase0 + qs * L::kQ;
       const int nchunks = unit_slots[qs * L::kUnitInts + 8];
+      if (!qk_lane) {  // the PV lane has read the unit: the slot may be taken again
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qempty[qs]);
+      }
+      if (nmem == 0) break;  // the producer ran out of work
       for (int ci = 0; ci < nchunks; ++ci, ++c) {
         const int slot = c % L::kStages;
-        if (!warp_wait(&kfull[slot], (c / L::kStages) & 1)) { ok = false; break; }
-        if (lane == 0) {
-          tc::fence_after_sync();
-          const uint32_t kb = kbase0 + slot * L::kTile;
-          const uint32_t d = tmem + (c & 1) * N;
+        if (qk_lane) {
+          if (!warp_wait(&kfull[slot], (c / L::kStages) & 1)) { ok = false; break; }
+          if (c >= 2 && !warp_wait(&pfull[c & 1], ((c - 2) >> 1) & 1)) { ok = false; break; }
+          if (lane == 0) {
+            tc::fence_after_sync();
+            const uint32_t kb = kbase0 + slot * L::kTile;
+            const uint32_t d = tmem + (c & 1) * N;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t koff = (kk >> 2) * 1024 + (kk & 3) * 32;
-            const uint64_t a = tc::smem_desc_sw128(kb + koff, 16, L::kGroup);
-            const uint64_t bdesc = tc::smem_desc_sw128(qb + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
-            tc::mma_bf16(d, a, bdesc, idesc_qk, kk > 0);
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t koff = (kk >> 2) * 1024 + (kk & 3) * 32;
+              const uint64_t a = tc::smem_desc_sw128(kb + koff, 16, L::kGroup);
+              const uint64_t bdesc = tc::smem_desc_sw128(qb + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
+              tc::mma_bf16(d, a, bdesc, idesc_qk, kk > 0);
+            }
+            tc::mma_commit(&sfull[c & 1]);
+            tc::mma_commit(&kempty[slot]);
+            if (ci == nchunks - 1) tc::mma_commit(&qempty[qs]);
           }
-          tc::mma_commit(&sfull[c & 1]);
-          tc::mma_commit(&kempty[slot]);
-          if (ci == nchunks - 1) tc::mma_commit(&qempty[qs]);
-        }
-        __syncwarp();
-        if (pending.c >= 0 && !issue_pv(pending)) { ok = false; break; }
-        pending = PvJob{c, qi, ci == 0};
-        if (ci == nchunks - 1) {
-          // the unit's last PV goes out at once: the epilogue waits for it,
-          // and the next unit's first K tile may still be on its way
-          if (!issue_pv(pending)) { ok = false; break; }
-          pending.c = -1;
+          __syncwarp();
+        } else {
+          if (!warp_wait(&pfull[c & 1], (c >> 1) & 1)) { ok = false; break; }
+          if (!warp_wait(&vfull[slot], (c / L::kStages) & 1)) { ok = false; break; }
+          // the accumulator is free once the epilogue of the unit two back read it
+          if (ci == 0 && !warp_wait(&ofree[qi & 1], ((qi >> 1) & 1) ^ 1)) { ok = false; break; }
+          if (lane == 0) {
+            tc::fence_after_sync();
+            const uint32_t vb = vbase0 + slot * L::kTile;
+            const uint32_t pb = pbase0 + (c & 1) * L::kP;
+            const uint32_t d = tmem + 2 * N + (qi & 1) * N;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t a = tc::smem_desc_sw128(vb + kk * 2 * L::kGroup, 1024, L::kGroup);
+              const uint64_t bdesc = tc::smem_desc_sw128(pb + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
+              tc::mma_bf16(d, a, bdesc, idesc_pv, (kk > 0 || ci > 0) ? 1u : 0u);
+            }
+            tc::mma_commit(&pvdone[c & 1]);
+            tc::mma_commit(&vempty[slot]);
+          }
+          __syncwarp();
         }
       }
       ++qi;
     }
-    if (ok && pending.c >= 0 && !issue_pv(pending)) ok = false;
     if (!ok && lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+    // no MMA of this lane may still be running when the CTA frees its tensor memory
     if (lane == 0) tc::mma_commit(drain);
     __syncwarp();
     mbar_wait(drain, 0);
@@ -605,6 +608,8 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
             }
           }
         }
+        // P(c) goes over P(c - 2), which PV(c - 2) must have read
+        if (c >= 2) warp_wait(&pvdone[c & 1], ((c - 2) >> 1) & 1);
         __nv_bfloat16 *pb = reinterpret_cast<__nv_bfloat16 *>(smem + L::kOffP + (c & 1) * L::kP);
         const int kh = r >> 6, rr = r & 63;
 #pragma unroll
