@@ -100,9 +100,9 @@ struct SharedParams {
   int32_t max_members;
 };
 
-// One CTA of 320 threads per SM.  Each of the SM's four sub-partitions
-// holds 16 K registers and three of the ten warps land on two of them, so a
-// thread gets at most 168.
+// One CTA of 352 threads per SM.  Each of the SM's four sub-partitions
+// holds 16 K registers and three of the eleven warps land on three of them,
+// so a thread gets at most 168.
 // PART: tokens per partition (256, 512 or 1024); the caller's p.part.
 template <int G, int PART>
 __global__ void __launch_bounds__(ShLayout::kThreads, 1)
