@@ -119,3 +119,21 @@ def test_traffic_record_follows_the_kernel_sources(tmp_path, monkeypatch):
         f.write("\n")
     assert bench.kernel_source_hash() != h0
     assert bench.profiled_traffic("gqa", 5000) is None
+
+
+def test_decode_launch_count():
+    """gpu_launches counts every kernel of a decode call: the partition
+    kernel once per slice (1024 sequences in its fine form, 8192 in its
+    coarse form, fewer when the whole partitions would overflow 20 bits),
+    the cascade once per 1024 plan groups, and the reduce when a row can
+    have more than one partition or a plan is given."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.decode_launches(8, 131072, 512) == 2            # long context: partition + reduce
+    assert bench.decode_launches(32, 400, 512) == 1              # one partition a row: no reduce
+    assert bench.decode_launches(256, 8000, 512, n_groups=64) == 3   # cascade + partition + reduce
+    assert bench.decode_launches(1024, 500, 1024, n_groups=1) == 3   # a plan alone needs the reduce
+    assert bench.decode_launches(3000, 4000, 1024, n_groups=800) == 3  # coarse form: one partition launch
+    assert bench.decode_launches(9000, 1000, 1024, n_groups=2100) == 2 + 3 + 1  # 2 slices, 3 cascades
+    # 2^20 - 1 whole partitions at most per launch: 256 partitions a row -> 4095 sequences
+    assert bench.decode_launches(5000, 256 * 512, 512) == 2 + 1
