@@ -35,7 +35,8 @@
 //  * the epilogue writes workspace rows for every (member, query head), read
 //    from O at the start of the next unit (the MMA warp issues a unit's last
 //    PV at once, so it does not wait for the next unit's first K tile);
-//  * two ring stages (the larger Q and P tiles take the third one's room).
+//  * two K and three V ring slots (the larger Q and P tiles take the third K
+//    slot's room; a V tile is held longer, until its PV has run).
 #pragma once
 
 #include "pa_decode_tc.cuh"
@@ -46,18 +47,21 @@ struct ShLayout {
   static constexpr int kSlots = 4;          // sequences per unit
   static constexpr int kN = 8 * kSlots;     // MMA N: 8 query rows per member slot
   static constexpr int kChunk = 128;
-  static constexpr int kStages = 2;
+  // ring slots: a V tile is held until its chunk's PV has run (after the
+  // softmax), a K tile only until its QK has, so V gets the third slot
+  static constexpr int kKStages = 2;
+  static constexpr int kVStages = 3;
   static constexpr int kTile = kChunk * 256;
   static constexpr int kGroup = 2048;
   static constexpr int kQ = 2 * kN * 128;   // two column halves of kN rows x 128 B
   static constexpr int kP = 2 * kN * 128;   // two 64-token halves of kN rows x 128 B
   static constexpr int kMaxGroups = 1024;
   static constexpr int kOffK = 0;
-  static constexpr int kOffV = kOffK + kStages * kTile;
-  static constexpr int kOffQ = kOffV + kStages * kTile;
+  static constexpr int kOffV = kOffK + kKStages * kTile;
+  static constexpr int kOffQ = kOffV + kVStages * kTile;
   static constexpr int kOffP = kOffQ + 2 * kQ;
   static constexpr int kOffBar = kOffP + 2 * kP;
-  static constexpr int kNumBars = 21;
+  static constexpr int kNumBars = 23;
   static constexpr int kOffRed = kOffBar + (kNumBars * 8 + 15) / 16 * 16;  // 16-byte aligned
   static constexpr int kRedFloats = 2 * 4 * kN;  // [parity][warp][column]
   static constexpr int kOffRedSum = kOffRed + kRedFloats * 4;
@@ -74,6 +78,8 @@ struct ShLayout {
   static constexpr int kThreads = 352;  // producer, QK lane, 8 softmax warps, PV lane
   static constexpr uint32_t kTmemCols = 128;  // S0 S1 O0 O1, kN columns each
 };
+
+static_assert(ShLayout::kBytes <= 227 * 1024, "shared memory of the cascade kernel");
 
 // OR of `pred` over the 128 threads of softmax warpgroup `grp` (named
 // barrier 1 + grp).
@@ -119,9 +125,9 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
-  uint64_t *kfull = bars, *kempty = bars + 2, *vfull = bars + 4, *vempty = bars + 6;
-  uint64_t *qfull = bars + 8, *qempty = bars + 10, *sfull = bars + 12, *pfull = bars + 14;
-  uint64_t *pvdone = bars + 16, *ofree = bars + 18, *drain = bars + 20;
+  uint64_t *kfull = bars, *kempty = bars + 2, *vfull = bars + 4, *vempty = bars + 7;
+  uint64_t *qfull = bars + 10, *qempty = bars + 12, *sfull = bars + 14, *pfull = bars + 16;
+  uint64_t *pvdone = bars + 18, *ofree = bars + 20, *drain = bars + 22;
   int32_t *gprefix = reinterpret_cast<int32_t *>(smem + L::kOffPrefix);
   int32_t *gshared = reinterpret_cast<int32_t *>(smem + L::kOffShared);
   int32_t *scan = reinterpret_cast<int32_t *>(smem + L::kOffScan);
@@ -132,9 +138,11 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
-    for (int i = 0; i < L::kStages; ++i) {
+    for (int i = 0; i < L::kKStages; ++i) {
       mbar_init(&kfull[i], 1);
       mbar_init(&kempty[i], 1);
+    }
+    for (int i = 0; i < L::kVStages; ++i) {
       mbar_init(&vfull[i], 1);
       mbar_init(&vempty[i], 1);
     }
@@ -305,8 +313,9 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
         }
         ++qi;
         for (int ci = 0; ci < un.nchunks; ++ci, ++c) {
-          const int slot = c % L::kStages, use = c / L::kStages;
           for (int which = 0; which < 2; ++which) {  // 0: K ring, 1: V ring
+            const int st = which ? L::kVStages : L::kKStages;
+            const int slot = c % st, use = c / st;
             uint64_t *empty = which ? &vempty[slot] : &kempty[slot];
             uint64_t *full = which ? &vfull[slot] : &kfull[slot];
             const CUtensorMap *map = which ? &tmap_v : &tmap_k;
@@ -351,9 +360,9 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
     }
     if (!ok && lane == 0) {
       raise_error(PA_DEVERR_TIMEOUT);
-      for (int k = (c > L::kStages ? c - L::kStages : 0); k <= c; ++k) {
-        mbar_wait(&kfull[k % L::kStages], (k / L::kStages) & 1, 100000000ull);
-        mbar_wait(&vfull[k % L::kStages], (k / L::kStages) & 1, 100000000ull);
+      for (int k = (c > L::kVStages ? c - L::kVStages : 0); k <= c; ++k) {
+        mbar_wait(&kfull[k % L::kKStages], (k / L::kKStages) & 1, 100000000ull);
+        mbar_wait(&vfull[k % L::kVStages], (k / L::kVStages) & 1, 100000000ull);
       }
       for (int k = (qi > 2 ? qi - 2 : 0); k < qi; ++k) mbar_wait(&qfull[k & 1], (k >> 1) & 1, 100000000ull);
     }
@@ -389,9 +398,9 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
       }
       if (nmem == 0) break;  // the producer ran out of work
       for (int ci = 0; ci < nchunks; ++ci, ++c) {
-        const int slot = c % L::kStages;
+        const int slot = c % L::kKStages, vslot = c % L::kVStages;
         if (qk_lane) {
-          if (!warp_wait(&kfull[slot], (c / L::kStages) & 1)) { ok = false; break; }
+          if (!warp_wait(&kfull[slot], (c / L::kKStages) & 1)) { ok = false; break; }
           if (c >= 2 && !warp_wait(&pfull[c & 1], ((c - 2) >> 1) & 1)) { ok = false; break; }
           if (lane == 0) {
             tc::fence_after_sync();
@@ -411,12 +420,12 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
           __syncwarp();
         } else {
           if (!warp_wait(&pfull[c & 1], (c >> 1) & 1)) { ok = false; break; }
-          if (!warp_wait(&vfull[slot], (c / L::kStages) & 1)) { ok = false; break; }
+          if (!warp_wait(&vfull[vslot], (c / L::kVStages) & 1)) { ok = false; break; }
           // the accumulator is free once the epilogue of the unit two back read it
           if (ci == 0 && !warp_wait(&ofree[qi & 1], ((qi >> 1) & 1) ^ 1)) { ok = false; break; }
           if (lane == 0) {
             tc::fence_after_sync();
-            const uint32_t vb = vbase0 + slot * L::kTile;
+            const uint32_t vb = vbase0 + vslot * L::kTile;
             const uint32_t pb = pbase0 + (c & 1) * L::kP;
             const uint32_t d = tmem + 2 * N + (qi & 1) * N;
 #pragma unroll
@@ -426,7 +435,7 @@ __global__ void __launch_bounds__(ShLayout::kThreads, 1)
               tc::mma_bf16(d, a, bdesc, idesc_pv, (kk > 0 || ci > 0) ? 1u : 0u);
             }
             tc::mma_commit(&pvdone[c & 1]);
-            tc::mma_commit(&vempty[slot]);
+            tc::mma_commit(&vempty[vslot]);
           }
           __syncwarp();
         }
