@@ -33,8 +33,9 @@
 //  * two softmax warpgroups (warps 2-5 and 6-9) take columns 0-15 and 16-31
 //    of S and O, each with its own running statistics and named barrier;
 //  * the epilogue writes workspace rows for every (member, query head), read
-//    from O at the start of the next unit (the MMA warp issues a unit's last
-//    PV at once, so it does not wait for the next unit's first K tile);
+//    from O at the start of the next unit (the PV lane issues a unit's last
+//    PV as soon as its P is in, so it does not wait for the next unit's
+//    first K tile);
 //  * two K and three V ring slots (the larger Q and P tiles take the third K
 //    slot's room; a V tile is held longer, until its PV has run).
 #pragma once
