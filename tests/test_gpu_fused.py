@@ -216,10 +216,12 @@ def test_fused_empty_and_bad_rows(cuda_device, dtype):
     assert not out[0].any()
 
 
-def test_fused_many_sequences_two_slices(cuda_device):
-    """2100 sequences run as two launches of the tensor-core kernel; each
-    slice takes its own new rows and copy sources.  Some sequences copy a
-    block of another sequence (a full first block) over their last block."""
+def test_fused_many_sequences_coarse(cuda_device):
+    """2100 sequences run as one launch of the tensor-core kernel's coarse
+    form (its tables count whole entries of 8 sequences), which places each
+    sequence's new row and copy source from those tables.  Some sequences
+    copy a block of another sequence (a full first block) over their last
+    block."""
     B, Hq, Hkv, D, bs = 2100, 8, 2, 128, 16
     dt = torch.bfloat16
     lens = synth.rng(48).integers(1, 80, size=B).astype(np.int32)
