@@ -169,15 +169,21 @@ def test_append_and_copy_bit_exact_and_padding_skipped():
     r = synth.rng(4)
     nk = r.integers(0, 2**16, size=(3, Hkv, D), dtype=np.uint16)
     nv = r.integers(0, 2**16, size=(3, Hkv, D), dtype=np.uint16)
-    oracle.append_kv(k, v, nk, nv, [5, -1, 22])
-    assert np.array_equal(k[1, :, 1], nk[0]) and np.array_equal(v[5, :, 2], nv[2])
-    changed = np.argwhere((k != k0).any(axis=-1))
-    assert {(int(a), int(c)) for a, _, c in changed} <= {(1, 1), (5, 2)}
+    oracle.append_kv(k, v, nk, nv, [9, -1, 22])
+    # slot s is row s % bs of block s // bs, every kv head
+    for (blk, off), i in (((2, 1), 0), ((5, 2), 2)):
+        assert np.array_equal(k[blk, :, off], nk[i]) and np.array_equal(v[blk, :, off], nv[i])
+    for cache, before in ((k, k0), (v, v0)):
+        changed = np.argwhere((cache != before).any(axis=-1))
+        assert {(int(a), int(c)) for a, _, c in changed} <= {(2, 1), (5, 2)}
     with pytest.raises(IndexError):
         oracle.append_kv(k, v, nk[:1], nv[:1], [NB * bs])
+    # block 4 becomes what block 1 held; block 1 and the rest stay as they were
+    k1, v1 = k.copy(), v.copy()
     oracle.copy_blocks(k, v, [(1, 4)])
-    assert np.array_equal(k[4], k[1]) and np.array_equal(v[4], v[1])
-    assert np.array_equal(k[0], k0[0])
+    for cache, before in ((k, k1), (v, v1)):
+        assert np.array_equal(cache[4], before[1])
+        assert all(np.array_equal(cache[b], before[b]) for b in range(NB) if b != 4)
 
 
 # ------------------------------------------------------------------ usage under sharing

@@ -9,6 +9,7 @@ import ctypes
 import os
 import subprocess
 
+import numpy as np
 import pytest
 
 import oracle
@@ -70,6 +71,87 @@ def _usage_pins():
     return [alloc_pins.test_usage_reproduces_the_paged_worked_example,
             alloc_pins.test_usage_of_a_shared_partial_block_by_hand,
             alloc_pins.test_usage_of_full_shared_blocks_by_hand]
+
+
+def _append_transposed_offset(k_cache, v_cache, k, v, slot_mapping):
+    """A plausible mistake: block and row of a slot swapped."""
+    ka, _ = oracle.host_array(k)
+    va, _ = oracle.host_array(v)
+    bs = k_cache.shape[2]
+    for i, s in enumerate(np.asarray(slot_mapping, dtype=np.int64).tolist()):
+        if s >= 0:
+            off, blk = divmod(s, bs)
+            k_cache[blk, :, off, :] = ka[i]
+            v_cache[blk, :, off, :] = va[i]
+
+
+def _append_padding_written(k_cache, v_cache, k, v, slot_mapping):
+    """A plausible mistake: a negative (padding) slot is not skipped and
+    lands, by negative indexing, in the last block."""
+    ka, _ = oracle.host_array(k)
+    va, _ = oracle.host_array(v)
+    NB, bs = k_cache.shape[0], k_cache.shape[2]
+    for i, s in enumerate(np.asarray(slot_mapping, dtype=np.int64).tolist()):
+        if s >= NB * bs:
+            raise IndexError(s)
+        blk, off = divmod(s, bs)
+        k_cache[blk, :, off, :] = ka[i]
+        v_cache[blk, :, off, :] = va[i]
+
+
+def _append_key_as_value(k_cache, v_cache, k, v, slot_mapping):
+    """A plausible mistake: the key row written into both caches."""
+    ka, _ = oracle.host_array(k)
+    bs = k_cache.shape[2]
+    for i, s in enumerate(np.asarray(slot_mapping, dtype=np.int64).tolist()):
+        if s >= 0:
+            blk, off = divmod(s, bs)
+            if blk >= k_cache.shape[0]:
+                raise IndexError(s)
+            k_cache[blk, :, off, :] = ka[i]
+            v_cache[blk, :, off, :] = ka[i]
+
+
+def _copy_reversed(k_cache, v_cache, pairs):
+    """A plausible mistake: the pair read as (dst, src)."""
+    for src, dst in np.asarray(pairs, dtype=np.int64).reshape(-1, 2).tolist():
+        k_cache[src] = k_cache[dst]
+        v_cache[src] = v_cache[dst]
+
+
+def _copy_keys_only(k_cache, v_cache, pairs):
+    """A plausible mistake: the value block left behind."""
+    for src, dst in np.asarray(pairs, dtype=np.int64).reshape(-1, 2).tolist():
+        k_cache[dst] = k_cache[src]
+
+
+APPEND_COPY_MUTANTS = {
+    "append-transposed-offset": ("append_kv", _append_transposed_offset),
+    "append-padding-written": ("append_kv", _append_padding_written),
+    "append-key-as-value": ("append_kv", _append_key_as_value),
+    "copy-reversed": ("copy_blocks", _copy_reversed),
+    "copy-keys-only": ("copy_blocks", _copy_keys_only),
+}
+
+
+def _append_copy_pins():
+    from tests import test_oracle_allocator as alloc_pins
+    return [alloc_pins.test_append_and_copy_bit_exact_and_padding_skipped]
+
+
+@pytest.mark.parametrize("name", sorted(APPEND_COPY_MUTANTS))
+def test_append_copy_mutant_is_caught(name, monkeypatch):
+    for t in _append_copy_pins():
+        t()  # the oracle as it stands passes every pin
+    attr, fn = APPEND_COPY_MUTANTS[name]
+    monkeypatch.setattr(oracle, attr, fn)
+    caught = 0
+    for t in _append_copy_pins():
+        try:
+            t()
+        except (AssertionError, IndexError):
+            caught += 1
+    assert caught > 0, f"no pin fails on mutant {name}"
 
 
 @pytest.mark.parametrize("name", sorted(USAGE_MUTANTS))
