@@ -150,6 +150,30 @@ def test_k_sharers_make_k_minus_1_copies():
         assert A.ref[last] == 1
 
 
+def test_copy_on_write_counts_against_the_free_list():
+    """A write into a shared partial block takes a free block for its copy,
+    so a batch is refused, state unchanged, when the copies do not fit; k
+    sharers need k - 1 copies, not k (the last writer owns the block by its
+    turn)."""
+    for k in (2, 3, 5):
+        # root: 5 tokens in 2 blocks of 4, the second shared by all k
+        for spare in (k - 2, k - 1):
+            A = oracle.AllocatorModel(2 + spare, 4)
+            root = A.new_seq()
+            A.append(root, 5)
+            sids = [root] + [A.fork(root) for _ in range(k - 1)]
+            assert len(A.free) == spare
+            before = (list(A.free), list(A.ref), {s: list(t) for s, t in A.tables.items()}, dict(A.lens))
+            if spare < k - 1:
+                with pytest.raises(oracle.OutOfBlocks):
+                    A.batch_append(sids, [1] * k)
+                assert (list(A.free), list(A.ref), {s: list(t) for s, t in A.tables.items()},
+                        dict(A.lens)) == before
+            else:
+                _, cows = A.batch_append(sids, [1] * k)
+                assert len(cows) == k - 1 and not A.free
+
+
 def test_free_returns_blocks_lifo():
     A = oracle.AllocatorModel(8, 2, [0, 1, 2, 3, 4, 5, 6, 7])
     a = A.new_seq()

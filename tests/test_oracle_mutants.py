@@ -6,8 +6,10 @@ dropped term, a flipped sign, a transposed layout, a wrong head mapping.  The
 pins of test_oracle_pins must fail on each, or the pins are too weak.
 """
 import ctypes
+import inspect
 import os
 import subprocess
+import textwrap
 
 import numpy as np
 import pytest
@@ -150,6 +152,51 @@ def test_append_copy_mutant_is_caught(name, monkeypatch):
         try:
             t()
         except (AssertionError, IndexError):
+            caught += 1
+    assert caught > 0, f"no pin fails on mutant {name}"
+
+
+# Mistakes planted in one method of the allocator model: (method, the
+# original text, its replacement).
+ALLOCATOR_MUTANTS = {
+    "fork-takes-no-reference": ("fork", "self.ref[blk] += 1", "pass"),
+    "free-list-fifo": ("free_seq", "self.free.append(blk)", "self.free.insert(0, blk)"),
+    "copy-keeps-reference": ("batch_append", "self.ref[last] -= 1", "pass"),
+    "copy-unshared-block": ("batch_append", "if self.ref[last] > 1:", "if self.ref[last] >= 1:"),
+    "copy-pair-reversed": ("batch_append", "cows.append((last, new))", "cows.append((new, last))"),
+    "slot-drops-offset": ("batch_append", "slots.append(table[pos // bs] * bs + pos % bs)",
+                          "slots.append(table[pos // bs] * bs)"),
+    "need-ignores-copies": ("_blocks_needed", "need += 1", "pass"),
+    "need-counts-every-sharer": ("_blocks_needed", "self.ref[last] - ref_taken.get(last, 0) > 1",
+                                 "self.ref[last] > 1"),
+}
+
+
+def _mutated_method(name, old, new):
+    src = textwrap.dedent(inspect.getsource(getattr(oracle.AllocatorModel, name)))
+    assert src.count(old) == 1, f"mutation site in {name} not unique"
+    ns = {}
+    exec(src.replace(old, new), vars(oracle), ns)
+    return ns[name]
+
+
+def _allocator_pins():
+    from tests import test_oracle_allocator as alloc_pins
+    return [getattr(alloc_pins, n) for n in sorted(dir(alloc_pins))
+            if n.startswith("test_") and not inspect.signature(getattr(alloc_pins, n)).parameters]
+
+
+@pytest.mark.parametrize("name", sorted(ALLOCATOR_MUTANTS))
+def test_allocator_mutant_is_caught(name, monkeypatch):
+    for t in _allocator_pins():
+        t()  # the model as it stands passes every pin
+    method, old, new = ALLOCATOR_MUTANTS[name]
+    monkeypatch.setattr(oracle.AllocatorModel, method, _mutated_method(method, old, new))
+    caught = 0
+    for t in _allocator_pins():
+        try:
+            t()
+        except (AssertionError, IndexError, oracle.OutOfBlocks, pytest.fail.Exception):
             caught += 1
     assert caught > 0, f"no pin fails on mutant {name}"
 
