@@ -398,6 +398,35 @@ def test_allocator_random_trace_matches_model(seed):
             assert A.refcount(b) == M.ref[b]
 
 
+def test_allocator_copies_count_against_the_free_list():
+    """k sharers of a partial last block appending in one batch need k - 1
+    copy blocks: with one fewer free the library refuses the batch and its
+    tables, lengths and refcounts stay as they were, like the model's; with
+    exactly k - 1 both make the same copies."""
+    for k in (2, 3, 5):
+        for spare in (k - 2, k - 1):
+            A, M = pa.Allocator(2 + spare, 4), oracle.AllocatorModel(2 + spare, 4)
+            root = A.new_seq()
+            assert M.new_seq() == root
+            A.append(root, 5)
+            M.append(root, 5)
+            sids = [root] + [A.fork(root) for _ in range(k - 1)]
+            assert [M.fork(root) for _ in range(k - 1)] == sids[1:]
+            before = [(A.block_table(s), A.seq_len(s)[0]) for s in sids], [A.refcount(b) for b in range(2 + spare)]
+            if spare < k - 1:
+                with pytest.raises(pa.OutOfBlocks):
+                    A.batch_append(sids, [1] * k)
+                with pytest.raises(oracle.OutOfBlocks):
+                    M.batch_append(sids, [1] * k)
+                assert ([(A.block_table(s), A.seq_len(s)[0]) for s in sids],
+                        [A.refcount(b) for b in range(2 + spare)]) == before
+            else:
+                gs, gp = A.batch_append(sids, [1] * k)
+                ws, wp = M.batch_append(sids, [1] * k)
+                assert gs.tolist() == ws and [tuple(x) for x in gp.tolist()] == wp and len(wp) == k - 1
+                assert A.stats()["free_blocks"] == 0
+
+
 def test_build_block_tables():
     A = pa.Allocator(32, 4)
     s = [A.new_seq() for _ in range(3)]
