@@ -201,6 +201,49 @@ def test_allocator_mutant_is_caught(name, monkeypatch):
     assert caught > 0, f"no pin fails on mutant {name}"
 
 
+# Mistakes planted in the fragmentation measures (learn-ml-visualized,
+# fragmentation worked example): (function, original text, replacement).
+FRAGMENTATION_MUTANTS = {
+    "paged-rounds-down": ("paged_usage", "-(-L // page_size)", "L // page_size"),
+    "paged-extra-page": ("paged_usage", "-(-L // page_size)", "L // page_size + 1"),
+    "naive-one-reservation": ("naive_usage", "allocated=reserve * len(lengths)", "allocated=reserve"),
+    "naive-reserves-the-longest": ("naive_usage", "allocated=reserve * len(lengths)",
+                                   "allocated=max(lengths) * len(lengths)"),
+}
+
+
+def _mutated_function(name, old, new):
+    src = inspect.getsource(getattr(oracle, name))
+    assert src.count(old) == 1, f"mutation site in {name} not unique"
+    ns = {}
+    exec(src.replace(old, new), vars(oracle), ns)
+    return ns[name]
+
+
+def _fragmentation_pins():
+    return ([lambda c=c: pins.test_fragmentation_golden(c) for c in pins._golden("fragmentation.json")["cases"]]
+            + [pins.test_naive_rejects_overlong, pins.test_paged_waste_under_one_page_any_length])
+
+
+@pytest.mark.parametrize("name", sorted(FRAGMENTATION_MUTANTS) + ["waste-over-used"])
+def test_fragmentation_mutant_is_caught(name, monkeypatch):
+    for t in _fragmentation_pins():
+        t()  # the measures as they stand pass every pin
+    if name == "waste-over-used":
+        # the fraction taken over the slots used instead of those allocated
+        monkeypatch.setattr(oracle.Usage, "fragmentation", property(lambda u: u.wasted / u.used))
+    else:
+        fn, old, new = FRAGMENTATION_MUTANTS[name]
+        monkeypatch.setattr(oracle, fn, _mutated_function(fn, old, new))
+    caught = 0
+    for t in _fragmentation_pins():
+        try:
+            t()
+        except (AssertionError, pytest.fail.Exception):
+            caught += 1
+    assert caught > 0, f"no pin fails on mutant {name}"
+
+
 @pytest.mark.parametrize("name", sorted(USAGE_MUTANTS))
 def test_usage_mutant_is_caught(name, monkeypatch):
     for t in _usage_pins():
