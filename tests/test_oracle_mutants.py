@@ -1,9 +1,12 @@
-"""Plants plausible mistakes in copies of the C oracle and checks that the
-pins catch every one (no GPU; nothing here touches the product path).
+"""Plants plausible mistakes in the oracle and checks that the pins catch
+every one (no GPU; nothing here touches the product path).
 
-Each mutant is the oracle source with one small edit: a wrong index, a
-dropped term, a flipped sign, a transposed layout, a wrong head mapping.  The
-pins of test_oracle_pins must fail on each, or the pins are too weak.
+Each mutant is one small edit: in a copy of the C attention oracle (a wrong
+index, a dropped term, a flipped sign, a transposed layout, a wrong head
+mapping), or in one Python function or method of the oracle, swapped in for
+the test (the append and the block copy, the allocator model, the usage and
+fragmentation measures).  The pins of test_oracle_pins and
+test_oracle_allocator must fail on each, or the pins are too weak.
 """
 import ctypes
 import inspect
